@@ -1,0 +1,391 @@
+"""Decode-step benchmark for the packed few-bit KV cache on B200.
+
+One step = one decode step of a GQA layer of the workload: append the new token of every
+sequence (kvq_quantize, n_new = 1) and run decode attention over the whole packed cache
+(kvq_decode_attention). Metric: KV tokens/s = sum over steps of (batch x context length)
+divided by the device time; also the packed HBM GB/s of the decode call.
+
+    python bench.py [--gpus N --steps K --warmup W --workload llama8b --impl ours|reference]
+
+With N > 1 (torchrun), every rank runs its own full copy of the workload (independent
+sequences, no collective on the data path: weak scaling); the time is the max over ranks.
+The timed region rotates over several cache replicas whose total size exceeds the 126 MB L2,
+so every step reads its cache from HBM. Inputs of all steps are resident in HBM before timing.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kvq_inputs import WORKLOADS, generate  # noqa: E402
+from kvq_inputs.workloads import rotation_and_sketch  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama8b", choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+
+class ClockSampler:
+    """Polls NVML (read-only) for SM clock and throttle reasons while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "hw_power_brake_slowdown": 0x80, "sw_power_cap": 0x4}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                r = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                break
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() and args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle (CPU) timing
+
+def oracle_prepare(w, pairs, ctx, data=None):
+    """Codes of ctx - 1 cached tokens for `pairs` (sequence 0, kv-head) pairs, prepared by the
+    oracle itself (untimed: this is the prefill, not the decode step)."""
+    from oracle import codec, tables
+    signs, S = rotation_and_sketch(w)
+    ck, tk = tables.lloyd_max_tables_f32(w.k_bits)
+    cv, tv = tables.lloyd_max_tables_f32(w.v_bits)
+    kS = S if w.k_mode == "lm_qjl" else None
+    vS = S if w.v_mode == "lm_qjl" else None
+    data = data or generate(w, "cpu", seqs=range(1), ctx=ctx)
+    K = data["k"][0].double().numpy()
+    V = data["v"][0].double().numpy()
+    q = data["q"][0].double().numpy()
+    prepared = []
+    for hk in range(pairs):
+        h = hk % w.n_kv_heads
+        rk = [codec.quantize_vector(x, w.k_bits, signs, ck, tk, kS) for x in K[h, :ctx - 1]]
+        rv = [codec.quantize_vector(x, w.v_bits, signs, cv, tv, vS) for x in V[h, :ctx - 1]]
+        prepared.append((h, rk, rv, K[h, ctx - 1], V[h, ctx - 1], q[h * w.group:(h + 1) * w.group]))
+    return dict(w=w, signs=signs, ck=ck, tk=tk, cv=cv, tv=tv, kS=kS, vS=vS, pairs=prepared, ctx=ctx)
+
+
+def oracle_step(P):
+    """One timed oracle decode step over the prepared pairs: quantize the new token, dequantize
+    the cache, attend. Returns (seconds, KV tokens the step covers in the metric's unit)."""
+    from oracle import attention, codec
+    w, signs = P["w"], P["signs"]
+    scale = 1.0 / math.sqrt(w.head_dim)
+    t0 = time.perf_counter()
+    for h, rk, rv, knew, vnew, qh in P["pairs"]:
+        rk2 = rk + [codec.quantize_vector(knew, w.k_bits, signs, P["ck"], P["tk"], P["kS"])]
+        rv2 = rv + [codec.quantize_vector(vnew, w.v_bits, signs, P["cv"], P["tv"], P["vS"])]
+        Kh = attention.dequantize_many(np.stack([r["codes"] for r in rk2]), np.array([r["n16"] for r in rk2]),
+                                       P["ck"], signs, np.array([r.get("gamma16", 0.0) for r in rk2]),
+                                       np.stack([r["z"] for r in rk2]) if P["kS"] is not None else None, P["kS"])
+        Vh = attention.dequantize_many(np.stack([r["codes"] for r in rv2]), np.array([r["n16"] for r in rv2]),
+                                       P["cv"], signs, np.array([r.get("gamma16", 0.0) for r in rv2]),
+                                       np.stack([r["z"] for r in rv2]) if P["vS"] is not None else None, P["vS"])
+        attention.decode_attention(qh, Kh, Vh, scale)
+    dt = time.perf_counter() - t0
+    return dt, len(P["pairs"]) * P["ctx"] / w.n_kv_heads
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def run_reference(args, world, rank):
+    w = WORKLOADS[args.workload]
+    metric, unit = "quantized-KV decode attention: KV tokens/s", "KV tokens/s"
+    if rank != 0:
+        return
+    if w.k_mode == "fp4":
+        print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the LM workloads"}))
+        return
+    pairs = 1
+    P = oracle_prepare(w, pairs, w.ctx)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, toks = oracle_step(P)
+        if i >= args.warmup:
+            times.append(dt)
+    per_step = sum(times) / len(times)
+    value = toks / per_step
+    sample = f"{pairs} (sequence, kv-head) pair of {w.batch * w.n_kv_heads} per step, ctx {w.ctx}"
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import bit_kv_cache_seeded_b200 as kvq
+    kvq.load()
+    w = WORKLOADS[args.workload]
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    cfg = kvq.cfg_for_workload(w)
+    signs, S = (None, None) if w.k_mode == "fp4" else rotation_and_sketch(w)
+    per_tok = kvq.kvq_packed_bytes_per_token(cfg)
+    heads_kv = 1 if w.k_mode == "fp4" else w.n_kv_heads
+    bytes_prefix = w.batch * heads_kv * w.ctx * per_tok
+    replicas = max(2, math.ceil(2.5 * L2_BYTES / max(bytes_prefix, 1)))
+    n_steps = args.warmup + args.steps
+    capacity = w.ctx + n_steps
+
+    # Prefix of ctx - 1 tokens in every replica (identical content), built in sequence slices.
+    caches = [kvq.KvqCache(cfg, w.batch, capacity, signs, S, device=dev) for _ in range(replicas)]
+    step_b = max(1, w.batch // 8)
+    q = None
+    for b0 in range(0, w.batch, step_b):
+        seqs = list(range(b0, min(w.batch, b0 + step_b)))
+        d = generate(w, dev, seqs=seqs, ctx=w.ctx - 1)
+        a, bb = ("latent", "rope") if w.k_mode == "fp4" else ("k", "v")
+        for c in caches:
+            c.quantize(d[a], d[bb], seq_ids=seqs)
+        q = d["q"] if q is None else torch.cat([q, d["q"]])
+        del d
+    # New tokens of every step, resident in HBM.
+    news = []
+    for s in range(n_steps):
+        d = generate(w, dev, step=s)
+        news.append((d["latent"], d["rope"]) if w.k_mode == "fp4" else (d["k"], d["v"]))
+    out = torch.empty((w.batch, w.n_q_heads, caches[0].out_dim), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    lens0 = int(caches[0].lengths()[0])
+
+    def step(i, timed_idx=None):
+        c = caches[i % replicas]
+        k_new, v_new = news[i]
+        c.quantize(k_new, v_new)
+        if timed_idx is not None:
+            ev[timed_idx][0].record(stream)
+        c.decode(q, out)
+        if timed_idx is not None:
+            ev[timed_idx][1].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kv_tokens = 0
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        start.record(stream)
+        for j in range(args.steps):
+            i = args.warmup + j
+            step(i, j)
+            kv_tokens += w.batch * (int(caches[i % replicas].lengths()[0]))
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    elapsed_ms = start.elapsed_time(end)
+    dec_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    dec_ms = max_over_ranks(dec_ms, world)
+    ms_per_step = elapsed_ms / args.steps
+    value = world * kv_tokens / (elapsed_ms / 1e3)
+
+    # End to end: host (pinned) inputs copied in, result copied out, every step.
+    host_news = [(a.cpu().pin_memory(), b.cpu().pin_memory()) for a, b in news[:args.steps]]
+    host_q = q.cpu().pin_memory()
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_k = torch.empty_like(news[0][0])
+    dev_v = torch.empty_like(news[0][1])
+    dev_q = torch.empty_like(q)
+    e2e_caches = caches  # continue appending after the timed run (capacity allows warmup+steps)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    e2e_tokens = 0
+    n_e2e = min(args.steps, max(1, capacity - int(caches[0].lengths().max()) - 1) * replicas)
+    n_e2e = min(n_e2e, args.steps)
+    t0.record(stream)
+    for j in range(n_e2e):
+        c = e2e_caches[j % replicas]
+        if int(c.lengths()[0]) >= capacity:
+            break
+        dev_k.copy_(host_news[j][0], non_blocking=True)
+        dev_v.copy_(host_news[j][1], non_blocking=True)
+        dev_q.copy_(host_q, non_blocking=True)
+        c.quantize(dev_k, dev_v)
+        c.decode(dev_q, out)
+        host_out.copy_(out, non_blocking=True)
+        e2e_tokens += w.batch * int(c.lengths()[0])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    e2e_steps = max(1, n_e2e)
+    e2e_value = world * e2e_tokens / (e2e_ms / 1e3) if e2e_ms > 0 else None
+    h2d = host_news[0][0].numel() * host_news[0][0].element_size() * 2 + host_q.numel() * host_q.element_size()
+    d2h = host_out.numel() * host_out.element_size()
+
+    peaks, peak_kind = measured_peaks()
+    bytes_step = w.batch * heads_kv * (lens0 + 1) * per_tok  # packed bytes one decode call reads
+    achieved = bytes_step / (dec_ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    line = {
+        "metric": "quantized-KV decode attention: KV tokens/s and HBM GB/s vs ~8 TB/s peak",
+        "value": value, "unit": "KV tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "n_q_heads": w.n_q_heads,
+                   "n_kv_heads": heads_kv, "head_dim": w.head_dim if w.k_mode != "fp4" else w.latent_dim,
+                   "ctx": w.ctx, "codec": f"K {w.k_mode}{w.k_bits} / V {w.v_mode}{w.v_bits}",
+                   "l2": f"{replicas} cache replicas x {bytes_prefix / 1e6:.1f} MB rotated per step (> 126 MB L2)",
+                   "parallelism": f"replicas{world}"},
+        "hbm_gbs": achieved, "frac_of_8tbs": achieved / 8000.0,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "kvq_decode_attention (split-K decode + reduce)",
+                     "bytes_per_launch": bytes_step, "ms_per_launch": dec_ms},
+        "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps * 3,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1 and w.k_mode != "fp4":
+        pairs = 2
+        P = oracle_prepare(w, pairs, w.ctx)
+        tot, toks_tot, reps = 0.0, 0.0, 0
+        while tot < 10.0 and reps < 200:
+            dt, toks = oracle_step(P)
+            tot, toks_tot, reps = tot + dt, toks_tot + toks, reps + 1
+        line["cpu_baseline"] = {"value": toks_tot / tot, "unit": "KV tokens/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{reps} repetitions of {pairs} (sequence, kv-head) pairs of one decode "
+                                          f"step at ctx {w.ctx} (of {w.batch * heads_kv} pairs per step), fp64 numpy"}
+    if rank == 0:
+        print(json.dumps(line))
+    for c in caches:
+        c.close()
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

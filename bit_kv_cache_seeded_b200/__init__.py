@@ -1,0 +1,262 @@
+"""Python binding of the kvq C ABI (include/kvq.h): argument marshalling only.
+
+Every step of the hot path -- rotation, Lloyd-Max coding, QJL sketch, packing, decode
+attention, split reduce -- runs in the CUDA kernels of ``libkvq.so``. This module loads that
+library (built in-tree by ``bit_kv_cache_seeded_b200.build``) and raises if it is missing or
+if no CUDA device is present when a call needs one; there is no fallback path.
+
+The C functions are exposed under their own names (``kvq_cache_bytes``, ``kvq_cache_init``,
+``kvq_quantize``, ``kvq_workspace_bytes``, ``kvq_decode_attention``, ...), taking torch
+tensors for device buffers. ``KvqCache`` bundles the arena, the host handle and the
+workspace for convenience.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvq.so")
+
+KVQ_OK = 0
+STATUS_NAMES = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED",
+                3: "KVQ_ERR_CAPACITY", 4: "KVQ_ERR_ALIGNMENT", 5: "KVQ_ERR_WORKSPACE",
+                6: "KVQ_ERR_CUDA"}
+MODES = {"lm_qjl": 0, "lm": 1, "sign1": 2, "fp4": 3}
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+# Every symbol include/kvq.h declares.
+EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "kvq_cache_init",
+           "kvq_quantize", "kvq_workspace_bytes", "kvq_decode_attention", "kvq_cache_lengths",
+           "kvq_cache_layout", "kvq_lloyd_max_table", "kvq_cache_destroy",
+           "kvq_debug_quantize_rotated")
+
+
+class KvqError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class kvq_cfg(ctypes.Structure):
+    _fields_ = [("head_dim", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("k_mode", ctypes.c_int32),
+                ("v_mode", ctypes.c_int32), ("k_bits", ctypes.c_int32),
+                ("v_bits", ctypes.c_int32), ("qjl_dim", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float), ("latent_dim", ctypes.c_int32),
+                ("rope_dim", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libkvq.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise OSError(f"{LIB_PATH} not built: run `python -m bit_kv_cache_seeded_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, SZ, VP = ctypes.POINTER, ctypes.c_int32, ctypes.c_size_t, ctypes.c_void_p
+    sig = {
+        "kvq_status_str": ([I32], ctypes.c_char_p),
+        "kvq_cache_bytes": ([P(kvq_cfg), I32, I32, P(SZ)], I32),
+        "kvq_packed_bytes_per_token": ([P(kvq_cfg), P(SZ)], I32),
+        "kvq_cache_init": ([P(VP), P(kvq_cfg), I32, I32, VP, SZ, VP, VP, VP], I32),
+        "kvq_quantize": ([VP, VP, VP, I32, I32, VP, I32, VP], I32),
+        "kvq_workspace_bytes": ([VP, P(SZ)], I32),
+        "kvq_decode_attention": ([VP, VP, I32, VP, VP, SZ, VP], I32),
+        "kvq_cache_lengths": ([VP, VP], I32),
+        "kvq_cache_layout": ([VP, VP, I32], I32),
+        "kvq_lloyd_max_table": ([I32, VP, VP], I32),
+        "kvq_cache_destroy": ([VP], None),
+        "kvq_debug_quantize_rotated": ([VP, VP, I32, VP, VP, VP, VP], I32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != KVQ_OK:
+        raise KvqError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_cfg(head_dim=128, n_q_heads=1, n_kv_heads=1, k_mode="lm_qjl", v_mode="lm_qjl", k_bits=2,
+             v_bits=2, qjl_dim=128, softmax_scale=0.0, latent_dim=0, rope_dim=0) -> kvq_cfg:
+    return kvq_cfg(head_dim, n_q_heads, n_kv_heads, MODES[k_mode], MODES[v_mode], k_bits, v_bits,
+                   qjl_dim, softmax_scale, latent_dim, rope_dim)
+
+
+def cfg_for_workload(w) -> kvq_cfg:
+    """kvq_cfg of a kvq_inputs.Workload."""
+    if w.k_mode == "fp4":
+        return make_cfg(head_dim=w.latent_dim, n_q_heads=w.n_q_heads, n_kv_heads=1, k_mode="fp4",
+                        v_mode="fp4", k_bits=4, v_bits=4, qjl_dim=0, latent_dim=w.latent_dim,
+                        rope_dim=w.rope_dim)
+    return make_cfg(w.head_dim, w.n_q_heads, w.n_kv_heads, w.k_mode, w.v_mode, w.k_bits, w.v_bits,
+                    w.qjl_dim)
+
+
+# ---------------------------------------------------------------- same-name wrappers
+
+def kvq_status_str(status: int) -> str:
+    return load().kvq_status_str(status).decode()
+
+
+def kvq_cache_bytes(cfg: kvq_cfg, batch: int, capacity: int) -> int:
+    out = ctypes.c_size_t()
+    _check("kvq_cache_bytes", load().kvq_cache_bytes(ctypes.byref(cfg), batch, capacity, ctypes.byref(out)))
+    return out.value
+
+
+def kvq_packed_bytes_per_token(cfg: kvq_cfg) -> int:
+    out = ctypes.c_size_t()
+    _check("kvq_packed_bytes_per_token", load().kvq_packed_bytes_per_token(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def kvq_cache_init(cfg: kvq_cfg, batch: int, capacity: int, arena: torch.Tensor, rot_signs=None,
+                   qjl_matrix=None, stream=None) -> ctypes.c_void_p:
+    handle = ctypes.c_void_p()
+    signs = None if rot_signs is None else np.ascontiguousarray(rot_signs, dtype=np.int8)
+    S = None if qjl_matrix is None else np.ascontiguousarray(qjl_matrix, dtype=np.float32)
+    st = load().kvq_cache_init(ctypes.byref(handle), ctypes.byref(cfg), batch, capacity, _ptr(arena),
+                               arena.numel() * arena.element_size(),
+                               None if signs is None else signs.ctypes.data_as(ctypes.c_void_p),
+                               None if S is None else S.ctypes.data_as(ctypes.c_void_p), _stream(stream))
+    _check("kvq_cache_init", st)
+    return handle
+
+
+def kvq_quantize(handle, K: torch.Tensor, V: torch.Tensor, seq_ids=None, stream=None):
+    if K.dtype not in DTYPES or V.dtype != K.dtype:
+        raise TypeError("K and V must both be float32 or bfloat16")
+    if not (K.is_contiguous() and V.is_contiguous()):
+        raise ValueError("K and V must be contiguous")
+    n_seq = K.shape[0]
+    n_new = K.shape[-2]
+    ids = None
+    if seq_ids is not None:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
+        if ids.shape[0] != n_seq:
+            raise ValueError("seq_ids length must match K.shape[0]")
+    st = load().kvq_quantize(handle, _ptr(K), _ptr(V), DTYPES[K.dtype], n_new,
+                             None if ids is None else ids.ctypes.data_as(ctypes.c_void_p), n_seq,
+                             _stream(stream))
+    _check("kvq_quantize", st)
+
+
+def kvq_workspace_bytes(handle) -> int:
+    out = ctypes.c_size_t()
+    _check("kvq_workspace_bytes", load().kvq_workspace_bytes(handle, ctypes.byref(out)))
+    return out.value
+
+
+def kvq_decode_attention(handle, q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                         stream=None):
+    if q.dtype not in DTYPES or out.dtype != torch.float32:
+        raise TypeError("q must be float32/bfloat16 and out float32")
+    if not (q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("q and out must be contiguous")
+    st = load().kvq_decode_attention(handle, _ptr(q), DTYPES[q.dtype], _ptr(out), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("kvq_decode_attention", st)
+
+
+def kvq_cache_lengths(handle, batch: int) -> np.ndarray:
+    lens = np.zeros(batch, dtype=np.int32)
+    _check("kvq_cache_lengths", load().kvq_cache_lengths(handle, lens.ctypes.data_as(ctypes.c_void_p)))
+    return lens
+
+
+def kvq_cache_layout(handle) -> np.ndarray:
+    info = np.zeros(16, dtype=np.int64)
+    _check("kvq_cache_layout", load().kvq_cache_layout(handle, info.ctypes.data_as(ctypes.c_void_p), 16))
+    return info
+
+
+def kvq_lloyd_max_table(bits: int):
+    c = np.zeros(1 << bits, dtype=np.float32)
+    t = np.zeros((1 << bits) - 1, dtype=np.float32)
+    _check("kvq_lloyd_max_table", load().kvq_lloyd_max_table(bits, c.ctypes.data_as(ctypes.c_void_p),
+                                                             t.ctypes.data_as(ctypes.c_void_p)))
+    return c, t
+
+
+def kvq_cache_destroy(handle):
+    if handle:
+        load().kvq_cache_destroy(handle)
+
+
+def kvq_debug_quantize_rotated(handle, u: torch.Tensor, k_bits: int, qjl: bool, stream=None):
+    n = u.shape[0]
+    planes = torch.zeros((n, k_bits, 4), dtype=torch.int32, device=u.device)
+    sketch = torch.zeros((n, 4), dtype=torch.int32, device=u.device) if qjl else None
+    gamma = torch.zeros((n,), dtype=torch.int16, device=u.device) if qjl else None
+    st = load().kvq_debug_quantize_rotated(handle, _ptr(u), n, _ptr(planes), _ptr(sketch), _ptr(gamma),
+                                           _stream(stream))
+    _check("kvq_debug_quantize_rotated", st)
+    return planes, sketch, gamma
+
+
+# ---------------------------------------------------------------- convenience object
+
+class KvqCache:
+    """A packed cache in a torch-allocated device arena, plus its decode workspace."""
+
+    def __init__(self, cfg: kvq_cfg, batch: int, capacity: int, rot_signs=None, qjl_matrix=None,
+                 device="cuda"):
+        if not torch.cuda.is_available():
+            raise RuntimeError("kvq needs a CUDA device")
+        self.cfg, self.batch = cfg, batch
+        nbytes = kvq_cache_bytes(cfg, batch, capacity)
+        self.arena = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.handle = kvq_cache_init(cfg, batch, capacity, self.arena, rot_signs, qjl_matrix)
+        self.workspace = torch.empty(max(16, kvq_workspace_bytes(self.handle)), dtype=torch.uint8,
+                                     device=device)
+        self.out_dim = cfg.latent_dim if cfg.k_mode == MODES["fp4"] else cfg.head_dim
+
+    def quantize(self, K, V, seq_ids=None, stream=None):
+        kvq_quantize(self.handle, K, V, seq_ids, stream)
+
+    def decode(self, q, out=None, stream=None):
+        if out is None:
+            out = torch.empty((self.batch, self.cfg.n_q_heads, self.out_dim), dtype=torch.float32,
+                              device=q.device)
+        kvq_decode_attention(self.handle, q, out, self.workspace, stream)
+        return out
+
+    def lengths(self):
+        return kvq_cache_lengths(self.handle, self.batch)
+
+    def layout(self):
+        return kvq_cache_layout(self.handle)
+
+    def close(self):
+        if self.handle:
+            kvq_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,460 @@
+// Host side of the kvq C ABI: validation, cache layout, tables, split planning, launches.
+// Every entry point validates before launching and reports failures as kvq_status codes.
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "kvq_internal.h"
+
+using namespace kvq;
+
+namespace {
+
+constexpr size_t kArenaAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool is_lm_mode(int m) { return m == KVQ_MODE_LM_QJL || m == KVQ_MODE_LM || m == KVQ_MODE_SIGN1; }
+
+kvq_status validate_cfg(const kvq_cfg* c) {
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  if (c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->n_q_heads % c->n_kv_heads) return KVQ_ERR_INVALID_ARG;
+  if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  if (c->k_mode == KVQ_MODE_FP4 || c->v_mode == KVQ_MODE_FP4) {
+    if (c->k_mode != KVQ_MODE_FP4 || c->v_mode != KVQ_MODE_FP4) return KVQ_ERR_INVALID_ARG;
+    if (c->n_kv_heads != 1) return KVQ_ERR_INVALID_ARG;
+    if (c->latent_dim <= 0 || c->rope_dim < 0) return KVQ_ERR_INVALID_ARG;
+    if (c->latent_dim != 512 || c->rope_dim != 64) return KVQ_ERR_UNSUPPORTED;
+    if (c->n_q_heads != 8 && c->n_q_heads != 16 && c->n_q_heads != 32 && c->n_q_heads != 64)
+      return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+  }
+  if (!is_lm_mode(c->k_mode) || !is_lm_mode(c->v_mode)) return KVQ_ERR_INVALID_ARG;
+  if (c->head_dim != kHeadDim) return c->head_dim > 0 ? KVQ_ERR_UNSUPPORTED : KVQ_ERR_INVALID_ARG;
+  const int modes[2] = {c->k_mode, c->v_mode};
+  const int bits[2] = {c->k_bits, c->v_bits};
+  bool any_qjl = false;
+  for (int i = 0; i < 2; ++i) {
+    if (modes[i] == KVQ_MODE_SIGN1) {
+      if (bits[i] != 1 && bits[i] != 0) return KVQ_ERR_INVALID_ARG;
+    } else if (bits[i] < 1 || bits[i] > kMaxBits) {
+      return KVQ_ERR_INVALID_ARG;
+    }
+    any_qjl |= modes[i] == KVQ_MODE_LM_QJL;
+  }
+  if (any_qjl && c->qjl_dim != kHeadDim) return c->qjl_dim > 0 ? KVQ_ERR_UNSUPPORTED : KVQ_ERR_INVALID_ARG;
+  const int g = c->n_q_heads / c->n_kv_heads;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+SideLayout make_side(int mode, int bits, int qjl_dim) {
+  SideLayout L;
+  L.bits = (mode == KVQ_MODE_SIGN1) ? 1 : bits;
+  L.qjl = mode == KVQ_MODE_LM_QJL;
+  L.m = L.qjl ? qjl_dim : 0;
+  int off = 0;
+  L.off_planes = off;
+  off += L.bits * kTile * (kHeadDim / 8);
+  L.off_sketch = off;
+  off += L.qjl ? kTile * (L.m / 8) : 0;
+  L.off_norm = off;
+  off += kTile * 2;
+  L.off_gamma = off;
+  off += L.qjl ? kTile * 2 : 0;
+  L.tile_bytes = (int)align_up((size_t)off, 16);
+  lloyd_max_f32(L.bits, L.cent, L.thr);
+  return L;
+}
+
+Fp4Layout make_fp4(int latent, int rope) {
+  Fp4Layout F;
+  F.latent = latent;
+  F.rope = rope;
+  F.off_codes = 0;
+  F.off_scales = kTile * latent / 2;
+  F.off_rope = F.off_scales + kTile * latent / 16;
+  F.tile_bytes = (int)align_up((size_t)F.off_rope + (size_t)kTile * rope * 2, 16);
+  return F;
+}
+
+struct Plan {
+  size_t lens_off, signs_off, S_off, St_off, k_off, v_off, total;
+  SideLayout k, v;
+  Fp4Layout fp4;
+  bool fp4_mode;
+  int tiles;
+};
+
+Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
+  Plan P{};
+  P.fp4_mode = c->k_mode == KVQ_MODE_FP4;
+  P.tiles = (capacity + kTile - 1) / kTile;
+  size_t off = 0;
+  P.lens_off = off;
+  off = align_up(off + sizeof(int) * (size_t)batch, kArenaAlign);
+  const size_t pairs = (size_t)batch * c->n_kv_heads;
+  if (P.fp4_mode) {
+    P.fp4 = make_fp4(c->latent_dim, c->rope_dim);
+    P.signs_off = P.S_off = P.St_off = off;
+    P.k_off = off;
+    off = align_up(off + pairs * P.tiles * (size_t)P.fp4.tile_bytes, kArenaAlign);
+    P.v_off = off;
+  } else {
+    P.k = make_side(c->k_mode, c->k_bits, c->qjl_dim);
+    P.v = make_side(c->v_mode, c->v_bits, c->qjl_dim);
+    const size_t m = (P.k.qjl || P.v.qjl) ? (size_t)c->qjl_dim : 0;
+    P.signs_off = off;
+    off = align_up(off + sizeof(float) * kHeadDim, kArenaAlign);
+    P.S_off = off;
+    off = align_up(off + sizeof(float) * m * kHeadDim, kArenaAlign);
+    P.St_off = off;
+    off = align_up(off + sizeof(float) * m * kHeadDim, kArenaAlign);
+    P.k_off = off;
+    off = align_up(off + pairs * P.tiles * (size_t)P.k.tile_bytes, kArenaAlign);
+    P.v_off = off;
+    off = align_up(off + pairs * P.tiles * (size_t)P.v.tile_bytes, kArenaAlign);
+  }
+  P.total = off;
+  return P;
+}
+
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+// Split plan: enough (pair, split) CTAs to fill the GPU several times over, each split a whole
+// number of tiles. max_splits() bounds the split count for every length up to the capacity.
+int split_target(int pairs, int sms) {
+  const int target = 4 * sms;
+  return std::max(1, (target + pairs - 1) / pairs);
+}
+
+void plan_splits(int pairs, int sms, int max_len, int* splits, int* chunk) {
+  const int tiles = std::max(1, (max_len + kTile - 1) / kTile);
+  const int s = std::min(split_target(pairs, sms), tiles);
+  const int chunk_tiles = (tiles + s - 1) / s;
+  *splits = (tiles + chunk_tiles - 1) / chunk_tiles;
+  *chunk = chunk_tiles * kTile;
+}
+
+int max_splits(int pairs, int sms, int tiles) { return std::min(split_target(pairs, sms), std::max(1, tiles)); }
+
+int part_stride(const kvq_cache* c) {
+  if (c->is_fp4) return 2 + c->cfg.latent_dim;
+  return 2 + kHeadDim * (c->v.qjl ? 2 : 1);
+}
+
+size_t workspace_for(const kvq_cache* c, int splits) {
+  return sizeof(float) * (size_t)c->batch * c->cfg.n_q_heads * splits * part_stride(c);
+}
+
+float default_scale(const kvq_cfg& cfg) {
+  if (cfg.softmax_scale > 0.f) return cfg.softmax_scale;
+  const int dqk = (cfg.k_mode == KVQ_MODE_FP4) ? cfg.latent_dim + cfg.rope_dim : cfg.head_dim;
+  return 1.0f / std::sqrt((float)dqk);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_status_str(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "cache capacity exceeded";
+    case KVQ_ERR_ALIGNMENT: return "misaligned pointer";
+    case KVQ_ERR_WORKSPACE: return "buffer too small";
+    case KVQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+kvq_status kvq_cache_bytes(const kvq_cfg* cfg, int32_t batch, int32_t capacity, size_t* bytes) {
+  if (!bytes || batch <= 0 || capacity <= 0) return KVQ_ERR_INVALID_ARG;
+  const kvq_status st = validate_cfg(cfg);
+  if (st != KVQ_OK) return st;
+  *bytes = plan_layout(cfg, batch, capacity).total;
+  return KVQ_OK;
+}
+
+kvq_status kvq_packed_bytes_per_token(const kvq_cfg* cfg, size_t* bytes) {
+  if (!bytes) return KVQ_ERR_INVALID_ARG;
+  const kvq_status st = validate_cfg(cfg);
+  if (st != KVQ_OK) return st;
+  if (cfg->k_mode == KVQ_MODE_FP4) {
+    *bytes = (size_t)cfg->latent_dim / 2 + cfg->latent_dim / 16 + 2 * (size_t)cfg->rope_dim;
+    return KVQ_OK;
+  }
+  size_t b = 0;
+  const int modes[2] = {cfg->k_mode, cfg->v_mode}, bits[2] = {cfg->k_bits, cfg->v_bits};
+  for (int i = 0; i < 2; ++i) {
+    const int nb = modes[i] == KVQ_MODE_SIGN1 ? 1 : bits[i];
+    b += (size_t)nb * kHeadDim / 8 + 2;
+    if (modes[i] == KVQ_MODE_LM_QJL) b += (size_t)cfg->qjl_dim / 8 + 2;
+  }
+  *bytes = b;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_t capacity,
+                          void* dev_mem, size_t dev_bytes, const int8_t* rot_signs,
+                          const float* qjl_matrix, void* stream) {
+  if (!out || !dev_mem || batch <= 0 || capacity <= 0) return KVQ_ERR_INVALID_ARG;
+  *out = nullptr;
+  const kvq_status st = validate_cfg(cfg);
+  if (st != KVQ_OK) return st;
+  if (reinterpret_cast<uintptr_t>(dev_mem) % kArenaAlign) return KVQ_ERR_ALIGNMENT;
+  const Plan P = plan_layout(cfg, batch, capacity);
+  if (dev_bytes < P.total) return KVQ_ERR_WORKSPACE;
+  const bool need_sketch = !P.fp4_mode && (P.k.qjl || P.v.qjl);
+  if (!P.fp4_mode && !rot_signs) return KVQ_ERR_INVALID_ARG;
+  if (need_sketch && !qjl_matrix) return KVQ_ERR_INVALID_ARG;
+  if (!P.fp4_mode)
+    for (int i = 0; i < kHeadDim; ++i)
+      if (rot_signs[i] != 1 && rot_signs[i] != -1) return KVQ_ERR_INVALID_ARG;
+
+  kvq_cache* c = new (std::nothrow) kvq_cache();
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  c->cfg = *cfg;
+  c->batch = batch;
+  c->capacity = P.tiles * kTile;
+  c->tiles_per_seq = P.tiles;
+  c->dev = static_cast<char*>(dev_mem);
+  c->dev_bytes = dev_bytes;
+  c->d_lens = reinterpret_cast<int*>(c->dev + P.lens_off);
+  c->is_fp4 = P.fp4_mode;
+  c->k = P.k;
+  c->v = P.v;
+  c->fp4 = P.fp4;
+  c->d_k = c->dev + P.k_off;
+  c->d_v = c->dev + P.v_off;
+  c->k_region = P.k_off;
+  c->v_region = P.v_off;
+  c->lens.assign(batch, 0);
+  c->sms = device_sms();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(c->d_lens, 0, sizeof(int) * (size_t)batch, s) != cudaSuccess) {
+    delete c;
+    return KVQ_ERR_CUDA;
+  }
+  if (!P.fp4_mode) {
+    c->d_signs = reinterpret_cast<float*>(c->dev + P.signs_off);
+    c->d_S = reinterpret_cast<float*>(c->dev + P.S_off);
+    c->d_St = reinterpret_cast<float*>(c->dev + P.St_off);
+    const size_t m = need_sketch ? (size_t)cfg->qjl_dim : 0;
+    c->h_tables.resize(kHeadDim + 2 * m * kHeadDim);
+    float* hs = c->h_tables.data();
+    for (int i = 0; i < kHeadDim; ++i) hs[i] = (float)rot_signs[i];
+    float* hS = hs + kHeadDim;
+    float* hSt = hS + m * kHeadDim;
+    for (size_t j = 0; j < m; ++j)
+      for (int i = 0; i < kHeadDim; ++i) {
+        hS[j * kHeadDim + i] = qjl_matrix[j * kHeadDim + i];
+        hSt[(size_t)i * m + j] = qjl_matrix[j * kHeadDim + i];
+      }
+    // Synchronous copies: the tables are tiny and this keeps the staging buffer's lifetime
+    // trivially safe.
+    if (cudaMemcpy(c->d_signs, hs, sizeof(float) * kHeadDim, cudaMemcpyHostToDevice) != cudaSuccess ||
+        (m && cudaMemcpy(c->d_S, hS, sizeof(float) * m * kHeadDim, cudaMemcpyHostToDevice) != cudaSuccess) ||
+        (m && cudaMemcpy(c->d_St, hSt, sizeof(float) * m * kHeadDim, cudaMemcpyHostToDevice) != cudaSuccess)) {
+      delete c;
+      return KVQ_ERR_CUDA;
+    }
+  }
+  *out = c;
+  return KVQ_OK;
+}
+
+kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dtype,
+                        int32_t n_new, const int32_t* seq_ids, int32_t n_seq, void* stream) {
+  if (!c || n_new < 0 || n_seq < 0) return KVQ_ERR_INVALID_ARG;
+  if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (n_new == 0 || n_seq == 0) return KVQ_OK;
+  if (!K || !V) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(V)) return KVQ_ERR_ALIGNMENT;
+  if (!seq_ids && n_seq != c->batch) return KVQ_ERR_INVALID_ARG;
+  if (n_seq > c->batch) return KVQ_ERR_INVALID_ARG;
+  std::vector<char> seen(c->batch, 0);
+  for (int i = 0; i < n_seq; ++i) {
+    const int sid = seq_ids ? seq_ids[i] : i;
+    if (sid < 0 || sid >= c->batch || seen[sid]) return KVQ_ERR_INVALID_ARG;
+    seen[sid] = 1;
+    if ((long)c->lens[sid] + n_new > (long)c->capacity) return KVQ_ERR_CAPACITY;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int heads = c->is_fp4 ? 1 : c->cfg.n_kv_heads;
+  const size_t elem = dtype == KVQ_BF16 ? 2 : 4;
+  const size_t per_seq_k = c->is_fp4 ? (size_t)n_new * c->cfg.latent_dim : (size_t)heads * n_new * kHeadDim;
+  const size_t per_seq_v = c->is_fp4 ? (size_t)n_new * c->cfg.rope_dim : per_seq_k;
+  for (int first = 0; first < n_seq; first += kMaxSeqPerLaunch) {
+    const int cnt = std::min(kMaxSeqPerLaunch, n_seq - first);
+    QuantizeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.src[0] = static_cast<const char*>(K) + first * per_seq_k * elem;
+    p.src[1] = static_cast<const char*>(V) + first * per_seq_v * elem;
+    p.bf16 = dtype == KVQ_BF16;
+    p.n_new = n_new;
+    p.n_seq = cnt;
+    p.heads = heads;
+    p.region[0] = c->d_k;
+    p.region[1] = c->d_v;
+    p.tiles_per_seq = c->tiles_per_seq;
+    p.side[0] = c->k;
+    p.side[1] = c->v;
+    p.fp4 = c->fp4;
+    p.signs = c->d_signs;
+    p.St = c->d_St;
+    p.lens = c->d_lens;
+    for (int i = 0; i < cnt; ++i) {
+      const int sid = seq_ids ? seq_ids[first + i] : first + i;
+      p.seq[i] = sid;
+      p.pos[i] = c->lens[sid];
+    }
+    const cudaError_t e = c->is_fp4 ? launch_quantize_fp4(p, s) : launch_quantize_lm(p, 2, s);
+    if (e != cudaSuccess) return KVQ_ERR_CUDA;
+    for (int i = 0; i < cnt; ++i) c->lens[p.seq[i]] += n_new;
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_workspace_bytes(const kvq_cache* c, size_t* bytes) {
+  if (!c || !bytes) return KVQ_ERR_INVALID_ARG;
+  const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
+  *bytes = workspace_for(c, max_splits(pairs, c->sms, c->tiles_per_seq));
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  if (!c || !q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+  if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
+  int max_len = 0;
+  for (int v : c->lens) max_len = std::max(max_len, v);
+  const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
+  int splits, chunk;
+  plan_splits(pairs, c->sms, max_len, &splits, &chunk);
+  if (ws_bytes < workspace_for(c, splits)) return KVQ_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const float log2e = 1.4426950408889634f;
+  if (c->is_fp4) {
+    MlaParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.bf16 = dtype == KVQ_BF16;
+    p.out = out;
+    p.part = static_cast<float*>(workspace);
+    p.B = c->batch;
+    p.Hq = c->cfg.n_q_heads;
+    p.splits = splits;
+    p.chunk = chunk;
+    p.lens = c->d_lens;
+    p.reg = c->d_k;
+    p.tiles_per_seq = c->tiles_per_seq;
+    p.fp4 = c->fp4;
+    p.logit_scale = default_scale(c->cfg) * log2e;
+    if (launch_decode_mla(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (launch_reduce_mla(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+    return KVQ_OK;
+  }
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q;
+  p.bf16 = dtype == KVQ_BF16;
+  p.out = out;
+  p.part = static_cast<float*>(workspace);
+  p.part_stride = part_stride(c);
+  p.B = c->batch;
+  p.Hq = c->cfg.n_q_heads;
+  p.Hkv = c->cfg.n_kv_heads;
+  p.group = p.Hq / p.Hkv;
+  p.splits = splits;
+  p.chunk = chunk;
+  p.lens = c->d_lens;
+  p.kreg = c->d_k;
+  p.vreg = c->d_v;
+  p.tiles_per_seq = c->tiles_per_seq;
+  p.k = c->k;
+  p.v = c->v;
+  p.signs = c->d_signs;
+  p.S = c->d_S;
+  p.St = c->d_St;
+  p.logit_scale = default_scale(c->cfg) * log2e;
+  if (launch_decode_lm(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (launch_reduce_lm(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens) {
+  if (!c || !lens) return KVQ_ERR_INVALID_ARG;
+  for (int i = 0; i < c->batch; ++i) lens[i] = c->lens[i];
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_layout(const kvq_cache* c, int64_t* info, int32_t n_info) {
+  if (!c || !info || n_info < 16) return KVQ_ERR_INVALID_ARG;
+  info[0] = kTile;
+  info[1] = c->is_fp4 ? c->fp4.tile_bytes : c->k.tile_bytes;
+  info[2] = c->is_fp4 ? 0 : c->v.tile_bytes;
+  info[3] = c->tiles_per_seq;
+  info[4] = (int64_t)c->k_region;
+  info[5] = (int64_t)c->v_region;
+  if (c->is_fp4) {
+    info[6] = c->fp4.off_codes;
+    info[7] = c->fp4.off_scales;
+    info[8] = c->fp4.off_rope;
+    for (int i = 9; i < 16; ++i) info[i] = 0;
+    return KVQ_OK;
+  }
+  const SideLayout* sides[2] = {&c->k, &c->v};
+  for (int i = 0; i < 2; ++i) {
+    info[6 + 5 * i] = sides[i]->off_planes;
+    info[7 + 5 * i] = sides[i]->off_sketch;
+    info[8 + 5 * i] = sides[i]->off_norm;
+    info[9 + 5 * i] = sides[i]->off_gamma;
+    info[10 + 5 * i] = sides[i]->bits;
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_lloyd_max_table(int32_t bits, float* centroids, float* thresholds) {
+  if (bits < 1 || bits > kMaxBits || !centroids || !thresholds) return KVQ_ERR_INVALID_ARG;
+  lloyd_max_f32(bits, centroids, thresholds);
+  return KVQ_OK;
+}
+
+void kvq_cache_destroy(kvq_cache* c) { delete c; }
+
+kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_t n,
+                                      uint32_t* planes, uint32_t* sketch, uint16_t* gamma,
+                                      void* stream) {
+  if (!c || c->is_fp4 || n < 0) return KVQ_ERR_INVALID_ARG;
+  if (n == 0) return KVQ_OK;
+  if (!u || !planes || (c->k.qjl && (!sketch || !gamma))) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(u) || !aligned16(planes) || (sketch && !aligned16(sketch))) return KVQ_ERR_ALIGNMENT;
+  QuantizeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.src[0] = u;
+  p.bf16 = 0;
+  p.n_new = n;
+  p.n_seq = 1;
+  p.heads = 1;
+  p.side[0] = c->k;
+  p.St = c->d_St;
+  p.skip_rotation = 1;
+  p.dbg_planes = planes;
+  p.dbg_sketch = sketch;
+  p.dbg_gamma = gamma;
+  if (launch_quantize_lm(p, 1, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
+}  // extern "C"

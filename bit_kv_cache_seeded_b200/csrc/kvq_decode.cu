@@ -1,0 +1,321 @@
+// Split-K decode attention over an LM / LM_QJL / SIGN1 packed cache, and the split reduce.
+//
+// For one (sequence b, kv-head, context chunk) a CTA computes, for the g query heads of the
+// group ("TurboQuant vs OSCAR vs EpiCache", section "Quantization frontiers: TurboQuant and
+// OSCAR" -- logits from the Lloyd-Max centroids plus the unbiased QJL correction):
+//   q_r = R q = H D q / sqrt(d),  s_q = S q_r                       (prologue, per head)
+//   l_t = scale (n_t / sqrt d) [ <q_r, c[code_t]> + sqrt(pi/2)/m gamma_t <s_q, z_t> ]
+//   online softmax in fp32 (base-2 exponent, log2(e) folded into the scale)
+//   o_r   += p_t (n_t / sqrt d) c[code_t]                            (value centroids)
+//   acc_z += p_t (n_t / sqrt d) sqrt(pi/2)/m gamma_t z_t             (value sketch, if any)
+// and writes the partial (m, l, o_r, acc_z). The reduce kernel merges the splits,
+//   M = max m_i, l = sum 2^(m_i - M) l_i, o = sum 2^(m_i - M) o_i / l,
+// folds the value sketch back with S^T acc_z, and undoes the rotation: out = D H o / sqrt(d).
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+__device__ __forceinline__ float load_q(const void* base, size_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  return reinterpret_cast<const float*>(base)[i];
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// exp2 that maps -inf to 0 without producing NaN for (-inf) - (-inf).
+__device__ __forceinline__ float exp2_diff(float a, float b) {
+  return (a == -INFINITY) ? 0.f : exp2f(a - b);
+}
+
+constexpr int kWarps = 4;
+
+// Rotated query of one head into smem: q_s = H D q * coef (coef folds 1/sqrt(d) and scales).
+__device__ void rotate_query(const void* q, size_t base, int bf16, const float* signs, float coef,
+                             float* dst) {
+  const int lane = threadIdx.x & 31;
+  float u[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) u[k] = load_q(q, base + 32 * k + lane, bf16) * signs[32 * k + lane];
+#pragma unroll
+  for (int b = 0; b < 5; ++b) {
+    const bool upper = (lane >> b) & 1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float o = __shfl_xor_sync(0xffffffffu, u[k], 1 << b);
+      u[k] = upper ? o - u[k] : u[k] + o;
+    }
+  }
+  const float a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
+  dst[lane] = (a0 + a2) * coef;
+  dst[64 + lane] = (a0 - a2) * coef;
+  dst[32 + lane] = (a1 + a3) * coef;
+  dst[96 + lane] = (a1 - a3) * coef;
+}
+
+template <int G, int KB, bool KQ, int VB, bool VQ>
+__global__ void __launch_bounds__(kWarps * 32)
+decode_lm_simple(const __grid_constant__ DecodeParams p) {
+  __shared__ float q_s[G][kHeadDim];   // rotated query * scale/sqrt(d) * log2(e) / sqrt(d)
+  __shared__ float s_s[G][kHeadDim];   // sketched query * the same * sqrt(pi/2)/m
+  __shared__ float mrg[kWarps][G][2 + 2 * kHeadDim];
+  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int len = p.lens[b];
+  const int t_begin = split * p.chunk;
+  const int t_end = min(len, t_begin + p.chunk);
+  const float inv_sqrt_d = 0.08838834764831845f;  // 1/sqrt(128)
+
+  // ---- prologue: rotated (and sketched) queries of the group
+  // logit (base 2) = n_t * ( <q_s, c> + gamma_t <s_s, z> ),  q_s = R q * scale*log2e/sqrt(d)
+  const float qcoef = inv_sqrt_d * p.logit_scale * inv_sqrt_d;
+  for (int h = warp; h < G; h += kWarps)
+    rotate_query(p.q, ((size_t)b * p.Hq + hk * G + h) * kHeadDim, p.bf16, p.signs, qcoef, q_s[h]);
+  __syncthreads();
+  if (KQ) {
+    const float kappa = 1.2533141373155003f / (float)p.k.m;  // sqrt(pi/2)/m
+    for (int idx = threadIdx.x; idx < G * kHeadDim; idx += blockDim.x) {
+      const int h = idx / kHeadDim, j = idx % kHeadDim;
+      float acc = 0.f;
+      for (int i = 0; i < kHeadDim; ++i) acc = fmaf(p.St[(size_t)i * p.k.m + j], q_s[h][i], acc);
+      s_s[h][j] = acc * kappa;
+    }
+  }
+  __syncthreads();
+
+  float m_run[G], l_run[G], o[G][4], oz[G][4];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m_run[h] = -INFINITY;
+    l_run[h] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) { o[h][k] = 0.f; oz[h][k] = 0.f; }
+  }
+  const float vkappa = VQ ? 1.2533141373155003f / (float)p.v.m : 0.f;
+
+  const size_t pair = (size_t)b * p.Hkv + hk;
+  for (int tile = t_begin / kTile + warp; tile * kTile < t_end; tile += kWarps) {
+    const int count = min(kTile, t_end - tile * kTile);
+    const bool valid = lane < count;
+    const char* kt = p.kreg + (pair * p.tiles_per_seq + tile) * (size_t)p.k.tile_bytes;
+    const char* vt = p.vreg + (pair * p.tiles_per_seq + tile) * (size_t)p.v.tile_bytes;
+
+    // ---- logits: lane = token
+    float logit[G];
+    {
+      uint4 pl[KB];
+#pragma unroll
+      for (int pp = 0; pp < KB; ++pp)
+        pl[pp] = *reinterpret_cast<const uint4*>(kt + p.k.off_planes + pp * (kTile * 16) + lane * 16);
+      uint4 zz = make_uint4(0, 0, 0, 0);
+      float gam = 0.f;
+      if (KQ) {
+        zz = *reinterpret_cast<const uint4*>(kt + p.k.off_sketch + lane * 16);
+        gam = __half2float(*reinterpret_cast<const __half*>(kt + p.k.off_gamma + lane * 2));
+      }
+      const float nk = __half2float(*reinterpret_cast<const __half*>(kt + p.k.off_norm + lane * 2));
+      float dot[G], dz[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) { dot[h] = 0.f; dz[h] = 0.f; }
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t words[KB];
+#pragma unroll
+        for (int pp = 0; pp < KB; ++pp)
+          words[pp] = (w == 0) ? pl[pp].x : (w == 1) ? pl[pp].y : (w == 2) ? pl[pp].z : pl[pp].w;
+        const uint32_t zword = (w == 0) ? zz.x : (w == 1) ? zz.y : (w == 2) ? zz.z : zz.w;
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {
+          int code = 0;
+#pragma unroll
+          for (int pp = 0; pp < KB; ++pp) code |= ((words[pp] >> i) & 1) << pp;
+          const float c = p.k.cent[code];
+          const int j = 32 * w + i;
+#pragma unroll
+          for (int h = 0; h < G; ++h) dot[h] = fmaf(q_s[h][j], c, dot[h]);
+          if (KQ) {
+            const float zs = ((zword >> i) & 1) ? 1.f : -1.f;
+#pragma unroll
+            for (int h = 0; h < G; ++h) dz[h] = fmaf(s_s[h][j], zs, dz[h]);
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) logit[h] = valid ? nk * (dot[h] + (KQ ? gam * dz[h] : 0.f)) : -INFINITY;
+    }
+
+    // ---- online softmax (per warp, per head)
+    float pw[G], pz[G];
+    const float nv = valid ? __half2float(*reinterpret_cast<const __half*>(vt + p.v.off_norm + lane * 2)) * inv_sqrt_d : 0.f;
+    const float gv = (VQ && valid) ? __half2float(*reinterpret_cast<const __half*>(vt + p.v.off_gamma + lane * 2)) * vkappa : 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float m_new = fmaxf(m_run[h], warp_max(logit[h]));
+      const float corr = exp2_diff(m_run[h], m_new);
+      const float pr = exp2_diff(logit[h], m_new);
+      l_run[h] = l_run[h] * corr + warp_sum(pr);
+      m_run[h] = m_new;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) { o[h][k] *= corr; oz[h][k] *= corr; }
+      pw[h] = pr * nv;
+      pz[h] = pw[h] * gv;
+    }
+
+    // ---- values: lane = coordinate (32k + lane), loop over the tile's tokens
+    for (int t = 0; t < count; ++t) {
+      uint32_t vw[VB][4];
+#pragma unroll
+      for (int pp = 0; pp < VB; ++pp) {
+        const uint4 x = *reinterpret_cast<const uint4*>(vt + p.v.off_planes + pp * (kTile * 16) + t * 16);
+        vw[pp][0] = x.x; vw[pp][1] = x.y; vw[pp][2] = x.z; vw[pp][3] = x.w;
+      }
+      float c[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        int code = 0;
+#pragma unroll
+        for (int pp = 0; pp < VB; ++pp) code |= ((vw[pp][k] >> lane) & 1) << pp;
+        c[k] = p.v.cent[code];
+      }
+      float zs[4] = {0.f, 0.f, 0.f, 0.f};
+      if (VQ) {
+        const uint4 x = *reinterpret_cast<const uint4*>(vt + p.v.off_sketch + t * 16);
+        zs[0] = ((x.x >> lane) & 1) ? 1.f : -1.f;
+        zs[1] = ((x.y >> lane) & 1) ? 1.f : -1.f;
+        zs[2] = ((x.z >> lane) & 1) ? 1.f : -1.f;
+        zs[3] = ((x.w >> lane) & 1) ? 1.f : -1.f;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float pt = __shfl_sync(0xffffffffu, pw[h], t);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[h][k] = fmaf(pt, c[k], o[h][k]);
+        if (VQ) {
+          const float ptz = __shfl_sync(0xffffffffu, pz[h], t);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) oz[h][k] = fmaf(ptz, zs[k], oz[h][k]);
+        }
+      }
+    }
+  }
+
+  // ---- merge the CTA's warps and write the split partial
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    if (lane == 0) { mrg[warp][h][0] = m_run[h]; mrg[warp][h][1] = l_run[h]; }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      mrg[warp][h][2 + 32 * k + lane] = o[h][k];
+      mrg[warp][h][2 + kHeadDim + 32 * k + lane] = oz[h][k];
+    }
+  }
+  __syncthreads();
+  const int width = 2 + (VQ ? 2 : 1) * kHeadDim;
+  for (int idx = threadIdx.x; idx < G * width; idx += blockDim.x) {
+    const int h = idx / width, e = idx % width;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mrg[w][h][0]);
+    float v = 0.f;
+    if (e == 0) {
+      v = M;
+    } else {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += exp2_diff(mrg[w][h][0], M) * mrg[w][h][e];
+    }
+    float* dst = p.part + (((size_t)b * p.Hq + hk * G + h) * p.splits + split) * p.part_stride;
+    dst[e] = v;
+  }
+}
+
+__global__ void __launch_bounds__(kHeadDim)
+reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
+  __shared__ float zs[kHeadDim];
+  __shared__ float xs[kHeadDim];
+  const int row = blockIdx.x;  // b * Hq + hq
+  const int i = threadIdx.x;
+  const float* part = p.part + (size_t)row * p.splits * p.part_stride;
+  float M = -INFINITY;
+  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, part[(size_t)s * p.part_stride]);
+  float L = 0.f, o = 0.f, oz = 0.f;
+  for (int s = 0; s < p.splits; ++s) {
+    const float* ps = part + (size_t)s * p.part_stride;
+    const float w = exp2_diff(ps[0], M);
+    L += w * ps[1];
+    o += w * ps[2 + i];
+    if (vq) oz += w * ps[2 + kHeadDim + i];
+  }
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  o *= inv;
+  if (vq) {
+    zs[i] = oz * inv;
+    __syncthreads();
+    float acc = 0.f;
+    for (int j = 0; j < p.v.m; ++j) acc = fmaf(p.S[(size_t)j * kHeadDim + i], zs[j], acc);
+    o += acc;
+  }
+  // out = D H o / sqrt(d)
+  xs[i] = o;
+  __syncthreads();
+  for (int h = 1; h < kHeadDim; h <<= 1) {
+    const float a = xs[i], bb = xs[i ^ h];
+    __syncthreads();
+    xs[i] = (i & h) ? bb - a : a + bb;
+    __syncthreads();
+  }
+  p.out[(size_t)row * kHeadDim + i] = xs[i] * p.signs[i] * 0.08838834764831845f;
+}
+
+template <int G>
+cudaError_t dispatch_modes(const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  const int kb = p.k.bits, vb = p.v.bits;
+  const bool kq = p.k.qjl, vq = p.v.qjl;
+#define KVQ_CASE(KB, KQ, VB, VQ)                                              \
+  if (kb == KB && kq == KQ && vb == VB && vq == VQ) {                         \
+    decode_lm_simple<G, KB, KQ, VB, VQ><<<grid, kWarps * 32, 0, s>>>(p);      \
+    return cudaGetLastError();                                                \
+  }
+  KVQ_CASE(2, true, 2, true)
+  KVQ_CASE(3, true, 3, false)
+  KVQ_CASE(1, false, 1, false)
+  KVQ_CASE(2, true, 2, false)
+  KVQ_CASE(3, true, 3, true)
+  KVQ_CASE(2, false, 2, false)
+  KVQ_CASE(3, false, 3, false)
+  KVQ_CASE(1, true, 1, false)
+  KVQ_CASE(1, true, 1, true)
+#undef KVQ_CASE
+  return cudaErrorNotSupported;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s) {
+  dim3 grid(p.splits, p.Hkv, p.B);
+  switch (p.group) {
+    case 1: return dispatch_modes<1>(p, grid, s);
+    case 2: return dispatch_modes<2>(p, grid, s);
+    case 4: return dispatch_modes<4>(p, grid, s);
+    case 8: return dispatch_modes<8>(p, grid, s);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s) {
+  reduce_lm<<<p.B * p.Hq, kHeadDim, 0, s>>>(p, p.v.qjl);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

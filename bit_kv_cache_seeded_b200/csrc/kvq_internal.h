@@ -1,0 +1,125 @@
+// Internal definitions shared by the host API and the kernels of the kvq library.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kTile = 32;          // tokens per cache tile
+constexpr int kHeadDim = 128;      // head_dim supported by the rotated (LM/SIGN1) modes
+constexpr int kMaxSeqPerLaunch = 1024;
+constexpr int kMaxBits = 3;
+
+// Where one side (K or V) of an LM/SIGN1 cache keeps its fields inside a 32-token tile.
+struct SideLayout {
+  int bits = 0;         // code bit-planes
+  int qjl = 0;          // 1 if a residual sign sketch is stored
+  int m = 0;            // sketch rows
+  int tile_bytes = 0;
+  int off_planes = 0;   // [bits][32][16 B]
+  int off_sketch = 0;   // [32][m/8 B]
+  int off_norm = 0;     // [32] fp16
+  int off_gamma = 0;    // [32] fp16
+  float cent[8] = {};   // fp32 Lloyd-Max centroids (2^bits, ascending)
+  float thr[7] = {};    // fp32 thresholds (2^bits - 1)
+};
+
+// FP4 latent cache tile: [32][latent/2] codes, [32][latent/16] E4M3 scales, [32][rope] bf16.
+struct Fp4Layout {
+  int latent = 0, rope = 0;
+  int tile_bytes = 0;
+  int off_codes = 0, off_scales = 0, off_rope = 0;
+};
+
+struct QuantizeParams {
+  // LM/SIGN1: src[0] = K, src[1] = V, each [n_seq, heads, n_new, d].
+  // FP4: src[0] = latent [n_seq, n_new, latent], src[1] = rope [n_seq, n_new, rope].
+  const void* src[2];
+  int bf16;
+  int n_new, n_seq, heads;
+  char* region[2];       // side region bases (FP4: region[0] only)
+  int tiles_per_seq;
+  SideLayout side[2];
+  Fp4Layout fp4;
+  const float* signs;    // [d] +-1
+  const float* St;       // [d][m] transposed sketch matrix
+  int* lens;             // device lengths, set to pos + n_new
+  int skip_rotation;     // debug entry: src[0] already rotated and normalised (fp32)
+  uint32_t* dbg_planes;  // debug outputs (skip_rotation only)
+  uint32_t* dbg_sketch;
+  uint16_t* dbg_gamma;
+  int seq[kMaxSeqPerLaunch];
+  int pos[kMaxSeqPerLaunch];
+};
+
+struct DecodeParams {
+  const void* q;          // [B, Hq, d]
+  int bf16;
+  float* out;             // [B, Hq, d]
+  float* part;            // [B, Hq, splits, part_stride]
+  int part_stride;        // 2 + d (+ m with a value sketch)
+  int B, Hq, Hkv, group;
+  int splits, chunk;      // tokens per split (multiple of kTile)
+  const int* lens;
+  const char* kreg;
+  const char* vreg;
+  int tiles_per_seq;
+  SideLayout k, v;
+  const float* signs;     // [d]
+  const float* S;         // [m][d]
+  const float* St;        // [d][m]
+  float logit_scale;      // softmax_scale * log2(e)
+};
+
+struct MlaParams {
+  const void* q;          // [B, Hq, latent + rope]
+  int bf16;
+  float* out;             // [B, Hq, latent]
+  float* part;            // [B, Hq, splits, 2 + latent]
+  int B, Hq;
+  int splits, chunk;
+  const int* lens;
+  const char* reg;
+  int tiles_per_seq;
+  Fp4Layout fp4;
+  float logit_scale;      // softmax_scale * log2(e)
+};
+
+// Launchers (kvq_quantize.cu, kvq_decode.cu, kvq_mla.cu). Return cudaGetLastError().
+cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s);
+cudaError_t launch_quantize_fp4(const QuantizeParams& p, cudaStream_t s);
+cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s);
+cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s);
+
+// Host Lloyd-Max tables (lloyd_max.cpp): fp64 fixed-point iteration rounded to fp32.
+void lloyd_max_f32(int bits, float* centroids, float* thresholds);
+
+}  // namespace kvq
+
+// Host object behind the opaque kvq_cache handle.
+struct kvq_cache {
+  kvq_cfg cfg;
+  int batch = 0, capacity = 0, tiles_per_seq = 0, sms = 148;
+  char* dev = nullptr;
+  size_t dev_bytes = 0;
+  int* d_lens = nullptr;
+  float* d_signs = nullptr;
+  float* d_S = nullptr;
+  float* d_St = nullptr;
+  char* d_k = nullptr;
+  char* d_v = nullptr;
+  size_t k_region = 0, v_region = 0;
+  kvq::SideLayout k, v;
+  kvq::Fp4Layout fp4;
+  bool is_fp4 = false;
+  std::vector<int> lens;
+  std::vector<float> h_tables;  // staging for the asynchronous table copies
+};

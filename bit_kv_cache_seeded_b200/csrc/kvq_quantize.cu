@@ -1,0 +1,221 @@
+// Quantize-and-append kernels.
+//
+// LM / LM_QJL / SIGN1 ("TurboQuant vs OSCAR vs EpiCache", section "Quantization frontiers:
+// TurboQuant and OSCAR"), one warp per vector, lane l holding coordinates 32k + l (k < 4):
+//   1. n = ||x||                                    (warp sum of squares, fp32)
+//   2. y = H D x                                    (sign flip; fast Walsh-Hadamard transform:
+//                                                    5 shuffle stages over the lane bits and
+//                                                    2 in-register stages over k)
+//   3. u = y / n  (= sqrt(d) R x / n with R = H D / sqrt(d))
+//   4. code_j = #{k : u_j >= t_k}                   (fp32 Lloyd-Max thresholds)
+//   5. rho = u - c[code], gamma = ||rho||           (stage-two residual)
+//   6. z_j = [ (S rho)_j >= 0 ]                     (1-bit QJL sketch, j < m)
+//   7. one __ballot_sync per code plane / sketch word gives word k directly (bit l =
+//      coordinate 32k + l), stored with one 16-byte store per plane; fp16 n and gamma.
+//
+// FP4 ("How DeepSeek-V4.1-Flash cut KV cache storage by 4x via CSA2", section "Numerics and
+// hardware efficiency"): one warp per token, lane l owning the 16-channel group l:
+//   s = E4M3_rn_satfinite(amax / 6); q_i = E2M1_rn_satfinite(x_i / s) (IEEE fp32 division);
+//   a zero scale codes the group as zeros; RoPE key copied as bf16.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+__device__ __forceinline__ float load_elem(const void* base, size_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  return reinterpret_cast<const float*>(base)[i];
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+constexpr int kQuantWarps = 8;
+
+__global__ void __launch_bounds__(kQuantWarps * 32)
+quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
+  __shared__ float rho_s[kQuantWarps][kHeadDim];
+  const int side = blockIdx.y;
+  const SideLayout& L = p.side[side];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nthr = L.bits ? (1 << L.bits) - 1 : 0;
+  const long total = (long)p.n_seq * p.heads * p.n_new;
+
+  for (long vec = (long)blockIdx.x * kQuantWarps + warp; vec < total;
+       vec += (long)gridDim.x * kQuantWarps) {
+    const int t = (int)(vec % p.n_new);
+    const int h = (int)((vec / p.n_new) % p.heads);
+    const int s = (int)(vec / ((long)p.n_new * p.heads));
+    const size_t base = (size_t)vec * kHeadDim;  // [n_seq, heads, n_new, d] row-major
+
+    float u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = load_elem(p.src[side], base + 32 * k + lane, p.bf16);
+
+    float n = 0.f;
+    if (!p.skip_rotation) {
+      n = sqrtf(warp_sum(u[0] * u[0] + u[1] * u[1] + u[2] * u[2] + u[3] * u[3]));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) u[k] *= p.signs[32 * k + lane];
+      // Walsh-Hadamard butterflies over index bits 0..4 (lane) and 5..6 (k).
+#pragma unroll
+      for (int b = 0; b < 5; ++b) {
+        const bool upper = (lane >> b) & 1;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float other = __shfl_xor_sync(0xffffffffu, u[k], 1 << b);
+          u[k] = upper ? other - u[k] : u[k] + other;
+        }
+      }
+      const float a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
+      u[0] = a0 + a2; u[2] = a0 - a2; u[1] = a1 + a3; u[3] = a1 - a3;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) u[k] = (n > 0.f) ? u[k] / n : 0.f;
+    }
+
+    int code[4];
+    float rho[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      int c = 0;
+      for (int i = 0; i < nthr; ++i) c += (u[k] >= L.thr[i]) ? 1 : 0;
+      code[k] = c;
+      rho[k] = u[k] - L.cent[c];
+    }
+    uint32_t planes[kMaxBits][4];
+#pragma unroll
+    for (int pp = 0; pp < kMaxBits; ++pp)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        planes[pp][k] = (pp < L.bits) ? __ballot_sync(0xffffffffu, (code[k] >> pp) & 1) : 0u;
+
+    uint32_t zw[4] = {0u, 0u, 0u, 0u};
+    float gamma = 0.f;
+    if (L.qjl) {
+      gamma = sqrtf(warp_sum(rho[0] * rho[0] + rho[1] * rho[1] + rho[2] * rho[2] + rho[3] * rho[3]));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rho_s[warp][32 * k + lane] = rho[k];
+      __syncwarp();
+      float proj[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = 0; i < kHeadDim; ++i) {
+        const float r = rho_s[warp][i];
+        const float* row = p.St + (size_t)i * L.m;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) proj[k] = fmaf(__ldg(row + 32 * k + lane), r, proj[k]);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < 4; ++k) zw[k] = __ballot_sync(0xffffffffu, proj[k] >= 0.f);
+    }
+
+    if (p.skip_rotation) {
+      if (lane < L.bits)
+        *reinterpret_cast<uint4*>(p.dbg_planes + ((size_t)vec * L.bits + lane) * 4) =
+            make_uint4(planes[lane][0], planes[lane][1], planes[lane][2], planes[lane][3]);
+      if (L.qjl && lane == 31)
+        *reinterpret_cast<uint4*>(p.dbg_sketch + (size_t)vec * 4) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+      if (L.qjl && lane == 0) p.dbg_gamma[vec] = __half_as_ushort(__float2half_rn(gamma));
+      continue;
+    }
+
+    const int pos = p.pos[s] + t;
+    const int seq = p.seq[s];
+    const int tile = pos / kTile, slot = pos % kTile;
+    char* tb = p.region[side] +
+               (((size_t)seq * p.heads + h) * p.tiles_per_seq + tile) * (size_t)L.tile_bytes;
+    if (lane < L.bits)
+      *reinterpret_cast<uint4*>(tb + L.off_planes + lane * (kTile * 16) + slot * 16) =
+          make_uint4(planes[lane][0], planes[lane][1], planes[lane][2], planes[lane][3]);
+    if (L.qjl && lane == 31)
+      *reinterpret_cast<uint4*>(tb + L.off_sketch + slot * 16) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+    if (lane == 30) *reinterpret_cast<__half*>(tb + L.off_norm + slot * 2) = __float2half_rn(n);
+    if (L.qjl && lane == 29)
+      *reinterpret_cast<__half*>(tb + L.off_gamma + slot * 2) = __float2half_rn(gamma);
+  }
+
+  if (side == 0 && blockIdx.x == 0 && !p.skip_rotation)
+    for (int i = threadIdx.x; i < p.n_seq; i += blockDim.x) p.lens[p.seq[i]] = p.pos[i] + p.n_new;
+}
+
+// E2M1 code of an fp32 value: nearest grid point of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the
+// even code, saturating at 6; the sign bit is kept even when the magnitude rounds to zero.
+__device__ __forceinline__ uint32_t e2m1_code(float v) {
+  const float a = fabsf(v);
+  uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) +
+               (a >= 3.5f) + (a > 5.0f);
+  return c | (signbit(v) ? 8u : 0u);
+}
+
+__global__ void __launch_bounds__(kQuantWarps * 32)
+quantize_fp4_kernel(const __grid_constant__ QuantizeParams p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const Fp4Layout& F = p.fp4;
+  const long total = (long)p.n_seq * p.n_new;
+  for (long tok = (long)blockIdx.x * kQuantWarps + warp; tok < total;
+       tok += (long)gridDim.x * kQuantWarps) {
+    const int t = (int)(tok % p.n_new);
+    const int s = (int)(tok / p.n_new);
+    const size_t lbase = (size_t)tok * F.latent + 16 * lane;
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = load_elem(p.src[0], lbase + i, p.bf16);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const __nv_fp8_storage_t sc = __nv_cvt_float_to_fp8(amax / 6.0f, __NV_SATFINITE, __NV_E4M3);
+    const float scale = __half2float(__half(__nv_cvt_fp8_to_halfraw(sc, __NV_E4M3)));
+    uint32_t lo = 0u, hi = 0u;
+    if (scale > 0.f) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) lo |= e2m1_code(x[i] / scale) << (4 * i);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) hi |= e2m1_code(x[8 + i] / scale) << (4 * i);
+    }
+    const int pos = p.pos[s] + t, seq = p.seq[s];
+    const int tile = pos / kTile, slot = pos % kTile;
+    char* tb = p.region[0] + ((size_t)seq * p.tiles_per_seq + tile) * (size_t)F.tile_bytes;
+    *reinterpret_cast<uint2*>(tb + F.off_codes + slot * (F.latent / 2) + lane * 8) = make_uint2(lo, hi);
+    tb[F.off_scales + slot * (F.latent / 16) + lane] = (char)sc;
+    // RoPE key: rope bf16 values, 16 bytes per lane for the first rope/8 lanes.
+    if (lane < F.rope / 8) {
+      const size_t rbase = (size_t)tok * F.rope + 8 * lane;
+      __nv_bfloat16 r[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) r[i] = __float2bfloat16_rn(load_elem(p.src[1], rbase + i, p.bf16));
+      *reinterpret_cast<uint4*>(tb + F.off_rope + slot * (F.rope * 2) + lane * 16) =
+          *reinterpret_cast<const uint4*>(r);
+    }
+  }
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.n_seq; i += blockDim.x) p.lens[p.seq[i]] = p.pos[i] + p.n_new;
+}
+
+int grid_for(long work_items, int per_block) {
+  long blocks = (work_items + per_block - 1) / per_block;
+  if (blocks > 148L * 16) blocks = 148L * 16;
+  return blocks < 1 ? 1 : (int)blocks;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s) {
+  const long total = (long)p.n_seq * p.heads * p.n_new;
+  dim3 grid(grid_for(total, kQuantWarps), n_sides);
+  quantize_lm_kernel<<<grid, kQuantWarps * 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_fp4(const QuantizeParams& p, cudaStream_t s) {
+  const long total = (long)p.n_seq * p.n_new;
+  quantize_fp4_kernel<<<grid_for(total, kQuantWarps), kQuantWarps * 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

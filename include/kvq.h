@@ -1,0 +1,162 @@
+/*
+ * kvq.h -- C ABI of a few-bit KV-cache codec with decode attention on the packed cache,
+ * written for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (cited by page title and section):
+ *
+ *  - "TurboQuant vs OSCAR vs EpiCache" (dothoosh.com), section "Quantization frontiers:
+ *    TurboQuant and OSCAR". Stage one rotates each key/value vector at random so that its
+ *    coordinates become close to independent Gaussians, then codes every coordinate with a
+ *    precomputed Lloyd-Max scalar quantizer. Stage two sketches the residual with a 1-bit
+ *    quantized Johnson-Lindenstrauss transform (QJL), which gives an unbiased estimate of the
+ *    attention logit. The same section describes KIVI (keys per channel, values per token).
+ *    The random rotation here is a randomized Hadamard transform R = H D / sqrt(d): D is a
+ *    +-1 diagonal and H the Sylvester-Hadamard matrix (natural order).
+ *  - Same page, section "KV-cache bottleneck": each decode step streams the whole cache, so
+ *    decode attention is bound by HBM bandwidth.
+ *  - "TaSQ 1-bit KV cache compression boosts batch sizes 14x": a cache of one sign bit per
+ *    coordinate (here: rotation, one sign bit per coordinate, an fp16 norm).
+ *  - "How DeepSeek-V4.1-Flash cut KV cache storage by 4x via CSA2", sections "CSA2" (one
+ *    512-dim latent per token shared by every head) and "Numerics and hardware efficiency"
+ *    (FP4 E2M1 storage with one scale per 16 channels; here the scale is an E4M3 byte).
+ *
+ * Conventions for every call:
+ *  - Calls return a kvq_status and never abort or throw. Arguments are validated before any
+ *    launch; a call that fails validation writes nothing.
+ *  - "stream" is a cudaStream_t passed as void* (NULL = legacy default stream). Calls that
+ *    launch work are asynchronous on that stream.
+ *  - Device pointers must be 16-byte aligned (KVQ_ERR_ALIGNMENT otherwise); the cache arena
+ *    must be 256-byte aligned.
+ *  - Ownership: the caller owns every device buffer (cache arena, K/V/q, out, workspace).
+ *    The library owns only the small host object returned by kvq_cache_init. It calls no
+ *    device allocator.
+ *  - Tensors are row-major and contiguous:
+ *      K, V  [n_seq, n_kv_heads, n_new, head_dim]   (f32 or bf16)
+ *      q     [batch, n_q_heads, head_dim]            (f32 or bf16)
+ *      out   [batch, n_q_heads, head_dim]            (f32)
+ *    Query head h uses KV head h / (n_q_heads / n_kv_heads) (grouped-query attention).
+ *    FP4 (MLA) caches instead take latent [n_seq, n_new, latent_dim] as "K" and the RoPE key
+ *    [n_seq, n_new, rope_dim] as "V", the absorbed query q [batch, n_q_heads,
+ *    latent_dim + rope_dim] (latent part first) and give out [batch, n_q_heads, latent_dim].
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, inconsistent configuration */
+  KVQ_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. head_dim != 128) */
+  KVQ_ERR_CAPACITY = 3,     /* append would exceed the cache capacity; nothing written */
+  KVQ_ERR_ALIGNMENT = 4,    /* a pointer is not 16-byte (arena: 256-byte) aligned */
+  KVQ_ERR_WORKSPACE = 5,    /* workspace or arena smaller than the size query returned */
+  KVQ_ERR_CUDA = 6          /* a CUDA launch or copy reported an error */
+} kvq_status;
+
+typedef enum {
+  KVQ_MODE_LM_QJL = 0,  /* rotation + b-bit Lloyd-Max code + 1-bit QJL residual sketch */
+  KVQ_MODE_LM = 1,      /* rotation + b-bit Lloyd-Max code, no sketch */
+  KVQ_MODE_SIGN1 = 2,   /* rotation + one sign bit per coordinate (1-bit Lloyd-Max) */
+  KVQ_MODE_FP4 = 3      /* FP4 E2M1 latent, one E4M3 scale per 16 channels (MLA caches) */
+} kvq_mode;
+
+typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+typedef struct {
+  int32_t head_dim;     /* LM/SIGN1 modes: 128 */
+  int32_t n_q_heads;    /* multiple of n_kv_heads */
+  int32_t n_kv_heads;   /* FP4: 1 (one shared latent) */
+  int32_t k_mode;       /* kvq_mode; FP4 requires k_mode == v_mode == KVQ_MODE_FP4 */
+  int32_t v_mode;
+  int32_t k_bits;       /* Lloyd-Max bits for LM modes: 1, 2 or 3 (SIGN1: 1) */
+  int32_t v_bits;
+  int32_t qjl_dim;      /* sketch rows m; 128 when either side is LM_QJL, else 0 */
+  float softmax_scale;  /* 0 => 1/sqrt(dim of q.k): head_dim, or latent_dim + rope_dim */
+  int32_t latent_dim;   /* FP4 only: 512 */
+  int32_t rope_dim;     /* FP4 only: 64 */
+} kvq_cfg;
+
+typedef struct kvq_cache kvq_cache; /* opaque host object */
+
+/* Human-readable name of a status code (static string). */
+const char* kvq_status_str(kvq_status s);
+
+/* Bytes of device memory a cache of `batch` sequences x `capacity` tokens needs (tables
+ * included). capacity is rounded up internally to a multiple of 32 tokens. */
+kvq_status kvq_cache_bytes(const kvq_cfg* cfg, int32_t batch, int32_t capacity, size_t* bytes);
+
+/* Packed bytes one token occupies per KV head (codes, sketch and norms of K and V; FP4:
+ * latent codes, scales and RoPE key), i.e. the algorithmic bytes decode reads per token. */
+kvq_status kvq_packed_bytes_per_token(const kvq_cfg* cfg, size_t* bytes);
+
+/* Create a cache inside caller-owned device memory `dev_mem` (dev_bytes >= kvq_cache_bytes).
+ * All sequences start empty. rot_signs: host [head_dim] of +1/-1 (the diagonal D), required
+ * for LM/SIGN1 modes. qjl_matrix: host [qjl_dim, head_dim] fp32, row-major, i.i.d. N(0,1)
+ * entries (the sketch matrix S), required when a side is LM_QJL. Both are copied; the
+ * library keeps no pointer to them after the call returns. The copies into dev_mem are
+ * enqueued on `stream`. On success *out owns a host object to free with kvq_cache_destroy. */
+kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_t capacity,
+                          void* dev_mem, size_t dev_bytes, const int8_t* rot_signs,
+                          const float* qjl_matrix, void* stream);
+
+/* Quantize n_new tokens per listed sequence and append them ("kvq_quantize(K or V, cfg) ->
+ * packed codes + norms + sketch"). K, V: device tensors in the layout above. seq_ids: host
+ * array of n_seq distinct sequence indices, or NULL for all sequences in order (then n_seq
+ * must equal batch). Fails with KVQ_ERR_CAPACITY, writing nothing, if any listed sequence
+ * would exceed the capacity. n_new == 0 or n_seq == 0 is a no-op. */
+kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dtype,
+                        int32_t n_new, const int32_t* seq_ids, int32_t n_seq, void* stream);
+
+/* Workspace bytes kvq_decode_attention needs for this cache (split-K partials). */
+kvq_status kvq_workspace_bytes(const kvq_cache* c, size_t* bytes);
+
+/* Decode attention of one query per sequence over the packed cache
+ * ("kvq_decode_attention(q, packed cache, cfg) -> out"). Every query head attends to all
+ * tokens its sequence holds: logits from the codes (plus the QJL correction), softmax in
+ * fp32, values dequantised and accumulated on the fly, split over the context with a
+ * second-pass combine. A sequence with no tokens gets an all-zero output. */
+kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Host copy of the current per-sequence lengths (lens: host array of `batch` entries). */
+kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens);
+
+/* Byte offsets describing the packed layout, for tools that read the arena directly.
+ * info[0..15] receives: tile_tokens, k_tile_bytes, v_tile_bytes, tiles_per_seq,
+ * k_region_offset, v_region_offset, then per side (K at 6, V at 11): planes_offset,
+ * sketch_offset, norm_offset, gamma_offset, planes. Layout of a tile (32 tokens) of one
+ * (sequence, kv-head): [planes][32 tokens][head_dim/8 bytes] code bit-planes (plane p holds
+ * bit p of every code; 32-bit word w of a token's plane holds coordinates 32w..32w+31,
+ * coordinate 32w+i in bit i), then [32][qjl_dim/8] sign words (bit = 1 for a non-negative
+ * projection), then [32] fp16 norms, then [32] fp16 residual norms. Tiles of a (sequence,
+ * kv-head) are consecutive; (sequence, kv-head) pairs follow in row-major order.
+ * FP4: [32][latent_dim/2] codes (channel 2k in the low nibble of byte k), [32][latent_dim/16]
+ * E4M3 scales, [32][rope_dim] bf16 RoPE keys. */
+kvq_status kvq_cache_layout(const kvq_cache* c, int64_t* info, int32_t n_info);
+
+/* The fp32 Gaussian Lloyd-Max table the library quantizes against (bits 1..3): centroids
+ * [2^bits] ascending, thresholds [2^bits - 1] (midpoints). Host arrays. */
+kvq_status kvq_lloyd_max_table(int32_t bits, float* centroids, float* thresholds);
+
+/* Free the host object (the caller still owns and frees the arena). NULL is a no-op. */
+void kvq_cache_destroy(kvq_cache* c);
+
+/* Test entry: code already rotated and normalised vectors u [n, head_dim] (device fp32)
+ * with the cache's key-side quantizer, writing per vector the code planes
+ * [n][k_bits][head_dim/32] u32, the sign words [n][qjl_dim/32] u32 (when the key side has a
+ * sketch) and the fp16 residual norm [n] (as uint16 bits). Output pointers are device. */
+kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_t n,
+                                      uint32_t* planes, uint32_t* sketch, uint16_t* gamma,
+                                      void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

@@ -46,6 +46,20 @@ def dequantize(codes, n16, centroids32, signs, gamma16=None, z=None, S=None) -> 
     return unrotate(dequantize_rotated(codes, n16, centroids32, gamma16, z, S), signs)
 
 
+def dequantize_many(codes, n16, centroids32, signs, gamma16=None, z=None, S=None) -> np.ndarray:
+    """``dequantize`` applied to every row: codes [T, d], n16 [T], gamma16 [T], z [T, m] (0/1)
+    -> x_hat [T, d]. The same arithmetic, written over a token axis."""
+    codes = np.asarray(codes, dtype=np.int64)
+    d = codes.shape[1]
+    est = np.asarray(centroids32, dtype=np.float64)[codes]
+    if z is not None:
+        Sd = np.asarray(S, dtype=np.float64)
+        zpm = 2.0 * np.asarray(z, dtype=np.float64) - 1.0
+        est = est + qjl_constant(Sd.shape[0]) * np.asarray(gamma16, dtype=np.float64)[:, None] * (zpm @ Sd)
+    est = est * (np.asarray(n16, dtype=np.float64) / math.sqrt(d))[:, None]
+    return unrotate(est, signs)
+
+
 def softmax_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float) -> np.ndarray:
     """out = sum_t p_t V_t with p = softmax(scale * K q); two-pass, max-subtracted, fp64.
 
@@ -108,6 +122,30 @@ def decode_attention_rotated(q_heads, codes_k, n16_k, gamma16_k, z_k, codes_v, n
             o_r += Sd.T @ acc_z
         outs.append(unrotate(o_r, signs))
     return np.stack(outs)
+
+
+def fp4_dequantize_many(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """``fp4_dequantize`` applied to every row: packed uint8 [T, C/2], scales uint8 [T, C/16]
+    -> [T, C], through the oracle's own E2M1/E4M3 decode tables."""
+    from .tables import E4M3_TABLE, e2m1_decode
+    e2m1 = np.array([e2m1_decode(n) for n in range(16)])
+    packed = np.asarray(packed, dtype=np.int64)
+    T, half = packed.shape
+    nib = np.empty((T, 2 * half), dtype=np.int64)
+    nib[:, 0::2] = packed & 0xF
+    nib[:, 1::2] = packed >> 4
+    sc = E4M3_TABLE[np.asarray(scales, dtype=np.int64)]
+    return e2m1[nib] * np.repeat(sc, 16, axis=1)
+
+
+def mla_decode_attention_many(q, latent_packed, latent_scales, k_rope, scale, heads=None):
+    """``mla_decode_attention`` over a long context, for the query heads listed in ``heads``
+    (default all): the same keys/values, dequantised once for all tokens."""
+    lat = fp4_dequantize_many(latent_packed, latent_scales)
+    K = np.concatenate([lat, np.asarray(k_rope, dtype=np.float64)], axis=1)
+    q = np.asarray(q, dtype=np.float64)
+    hs = range(q.shape[0]) if heads is None else heads
+    return np.stack([softmax_attention(q[h], K, lat, scale) for h in hs])
 
 
 def mla_decode_attention(q: np.ndarray, latent_packed: np.ndarray, latent_scales: np.ndarray,

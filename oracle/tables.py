@@ -4,6 +4,7 @@ Test infrastructure only (see ``oracle/__init__.py``).
 """
 from __future__ import annotations
 
+import functools
 import math
 
 import numpy as np
@@ -100,8 +101,10 @@ def lloyd_max_tables_f32(bits: int):
 # The random rotation of stage one is realised as R = H D / sqrt(d), D a seeded +-1 diagonal.
 # ---------------------------------------------------------------------------------------------
 
+@functools.lru_cache(maxsize=None)
 def hadamard(d: int) -> np.ndarray:
-    """Explicit d x d Sylvester-Hadamard matrix, entry (-1)^popcount(i & j), as fp64."""
+    """Explicit d x d Sylvester-Hadamard matrix, entry (-1)^popcount(i & j), as fp64
+    (read-only; cached)."""
     if d <= 0 or d & (d - 1):
         raise ValueError("d must be a power of two")
     i = np.arange(d)[:, None]
@@ -111,7 +114,9 @@ def hadamard(d: int) -> np.ndarray:
     while np.any(x):
         pop += x & 1
         x >>= 1
-    return np.where(pop % 2 == 0, 1.0, -1.0)
+    H = np.where(pop % 2 == 0, 1.0, -1.0)
+    H.setflags(write=False)
+    return H
 
 
 # ---------------------------------------------------------------------------------------------

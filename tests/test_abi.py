@@ -1,0 +1,100 @@
+"""The C-ABI library builds, loads and exports every symbol include/kvq.h declares; host-only
+entry points (tables, sizes, validation) behave as documented. No GPU needed."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_kv_cache_seeded_b200 as kvq
+from bit_kv_cache_seeded_b200 import build
+from oracle import tables, sizes
+from kvq_inputs import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return kvq.load()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"\b(kvq_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(kvq.EXPORTS)
+
+
+def test_lloyd_max_table_bit_equal_to_oracle(lib):
+    for bits in (1, 2, 3):
+        c, t = kvq.kvq_lloyd_max_table(bits)
+        oc, ot = tables.lloyd_max_tables_f32(bits)
+        assert c.tobytes() == oc.tobytes()
+        assert t.tobytes() == ot.tobytes()
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_packed_bytes_match_oracle_sizes(lib, name):
+    w = WORKLOADS[name]
+    cfg = kvq.cfg_for_workload(w)
+    got = kvq.kvq_packed_bytes_per_token(cfg)
+    if w.k_mode == "fp4":
+        want = sizes.fp4_token_bytes(w.latent_dim, w.rope_dim)
+    else:
+        want = (sizes.lm_vector_bytes(128, w.k_bits, 128 if w.k_mode == "lm_qjl" else 0)
+                + sizes.lm_vector_bytes(128, w.v_bits, 128 if w.v_mode == "lm_qjl" else 0))
+    assert got == want
+
+
+def test_cache_bytes_scales_with_capacity(lib):
+    cfg = kvq.cfg_for_workload(WORKLOADS["llama8b"])
+    a = kvq.kvq_cache_bytes(cfg, 16, 8192)
+    b = kvq.kvq_cache_bytes(cfg, 16, 8192 + 32)
+    assert b - a == 16 * 8 * 104 * 32
+    assert kvq.kvq_cache_bytes(cfg, 16, 8193) == b  # capacity rounds up to whole tiles
+
+
+def test_validation_errors(lib):
+    bad = kvq.make_cfg(head_dim=64)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_cache_bytes(bad, 1, 32)
+    assert e.value.status == 2  # unsupported
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_cache_bytes(kvq.make_cfg(n_q_heads=3, n_kv_heads=2), 1, 32)
+    assert e.value.status == 1
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_cache_bytes(kvq.make_cfg(k_bits=4), 1, 32)
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_cache_bytes(kvq.make_cfg(k_mode="fp4"), 1, 32)  # fp4 on one side only
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_cache_bytes(kvq.make_cfg(), 0, 32)
+    assert kvq.kvq_status_str(3) == "cache capacity exceeded"
+
+
+def test_init_rejects_null_and_misaligned_before_any_launch(lib):
+    import ctypes
+    cfg = kvq.make_cfg()
+    h = ctypes.c_void_p()
+    signs = np.ones(128, dtype=np.int8)
+    st = lib.kvq_cache_init(ctypes.byref(h), ctypes.byref(cfg), 1, 32, None, 1 << 20,
+                            signs.ctypes.data_as(ctypes.c_void_p), None, None)
+    assert st == 1
+    st = lib.kvq_cache_init(ctypes.byref(h), ctypes.byref(cfg), 1, 32, ctypes.c_void_p(0x1010), 1 << 20,
+                            signs.ctypes.data_as(ctypes.c_void_p), None, None)
+    assert st == 4
+    st = lib.kvq_cache_init(ctypes.byref(h), ctypes.byref(cfg), 1, 32, ctypes.c_void_p(0x10000), 16,
+                            signs.ctypes.data_as(ctypes.c_void_p), None, None)
+    assert st == 5
+    bad_signs = np.zeros(128, dtype=np.int8)
+    S = np.zeros((128, 128), dtype=np.float32)
+    st = lib.kvq_cache_init(ctypes.byref(h), ctypes.byref(cfg), 1, 32, ctypes.c_void_p(0x10000), 1 << 20,
+                            bad_signs.ctypes.data_as(ctypes.c_void_p), S.ctypes.data_as(ctypes.c_void_p), None)
+    assert st == 1

@@ -1,0 +1,240 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the same seeded inputs.
+
+Covers bit-exact packing on shared rotated fp32 inputs, end-to-end codes with the 1e-5
+boundary rule, attention within 2e-3 relative over identical codes for every workload shape
+(small contexts with ragged tails, then sampled pairs at full size), FP4 codes bit-exact, and
+the edge cases: one token, empty sequences, token-by-token appends, capacity overflow.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import bit_kv_cache_seeded_b200 as kvq
+from kvq_inputs import WORKLOADS, generate
+from kvq_inputs.workloads import rotation_and_sketch
+from oracle import codec, tables, attention
+from tests._cache_reader import fp4_fields
+from tests._parity import pair_reference, rel_err, REL_TOL, BOUNDARY
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    kvq.load()
+
+
+def new_cache(w, batch, capacity):
+    signs, S = rotation_and_sketch(w)
+    return kvq.KvqCache(kvq.cfg_for_workload(w), batch, capacity, signs, S), signs, S
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+# ---------------------------------------------------------------- packing on shared u
+
+@pytest.mark.parametrize("bits,qjl", [(2, True), (3, True), (1, False), (3, False)])
+def test_debug_quantize_rotated_bit_exact(bits, qjl):
+    w = WORKLOADS["tiny"].with_(k_bits=bits, v_bits=bits, k_mode="lm_qjl" if qjl else "lm",
+                                v_mode="lm_qjl" if qjl else "lm")
+    cache, signs, S = new_cache(w, 1, 32)
+    c32, t32 = tables.lloyd_max_tables_f32(bits)
+    rng = np.random.default_rng(bits)
+    u = rng.standard_normal((300, 128)).astype(np.float32)
+    u[0, :len(t32)] = t32                       # exactly on thresholds: upper cell
+    u[1, :len(t32)] = np.nextafter(t32, -np.inf)  # just below
+    u[2] = 0.0
+    ut = torch.tensor(u, device=DEV)
+    planes, sketch, gamma = kvq.kvq_debug_quantize_rotated(cache.handle, ut, bits, qjl)
+    torch.cuda.synchronize()
+    planes = planes.cpu().numpy().view(np.uint32)
+    for i in range(u.shape[0]):
+        r = codec.quantize_rotated(u[i].astype(np.float64), bits, c32, t32, S if qjl else None)
+        np.testing.assert_array_equal(planes[i], r["planes"])
+        if qjl:
+            zg = sketch[i].cpu().numpy().view(np.uint32)
+            mism = np.nonzero(codec.unpack_bits(zg, 128) != r["z"])[0]
+            tol = 4 * 128 * 2.0 ** -24 * (np.abs(S.astype(np.float64)) @ np.abs(r["rho"]))
+            assert np.all(np.abs(r["proj"][mism]) < tol[mism])
+            g = float(gamma[i:i + 1].cpu().numpy().view(np.float16)[0])
+            assert abs(g - r["gamma16"]) <= 2.0 ** (math.floor(math.log2(max(r["gamma"], 2 ** -14))) - 10)
+    cache.close()
+
+
+# ---------------------------------------------------------------- decode parity, small contexts
+
+def run_small(name, batch, lens, seed_appends=1):
+    """Quantize lens[b] tokens into sequence b (in `seed_appends` calls), decode, compare every
+    (sequence, kv-head) with the oracle."""
+    w = WORKLOADS[name]
+    T = max(lens)
+    data = generate(w, DEV, seqs=range(batch), ctx=T)
+    cache, signs, S = new_cache(w, batch, T + 40)
+    # append per sequence, in chunks, to exercise positions inside tiles
+    for b in range(batch):
+        L = lens[b]
+        cuts = np.linspace(0, L, seed_appends + 1).astype(int)
+        for a, e in zip(cuts[:-1], cuts[1:]):
+            if e > a:
+                cache.quantize(data["k"][b:b + 1, :, a:e].contiguous(), data["v"][b:b + 1, :, a:e].contiguous(),
+                               seq_ids=[b])
+    assert list(cache.lengths()) == list(lens)
+    out = f64(cache.decode(data["q"]))
+    torch.cuda.synchronize()
+    arena = cache.arena.cpu().numpy()
+    info = cache.layout()
+    stats = {}
+    for b in range(batch):
+        for hk in range(w.n_kv_heads):
+            g = w.group
+            if lens[b] == 0:
+                assert np.all(out[b, hk * g:(hk + 1) * g] == 0)
+                continue
+            ref = pair_reference(w, arena, info, b, hk, lens[b], f64(data["k"][b, hk, :lens[b]]),
+                                 f64(data["v"][b, hk, :lens[b]]), f64(data["q"][b, hk * g:(hk + 1) * g]),
+                                 signs, S, stats)
+            err = rel_err(out[b, hk * g:(hk + 1) * g], ref)
+            assert np.all(err <= REL_TOL), (b, hk, err.max())
+    cache.close()
+    return stats
+
+
+def test_tiny_full():
+    w = WORKLOADS["tiny"]
+    stats = run_small("tiny", 1, [w.ctx])
+    assert stats["code_flips"] <= 1e-3 * stats["coords"]
+
+
+def test_tiny_token_by_token_and_ragged():
+    run_small("tiny", 1, [77], seed_appends=77)
+
+
+@pytest.mark.parametrize("lens", [[1000, 333, 1, 0], [32, 31, 64, 65]])
+def test_llama8b_small_ragged(lens):
+    run_small("llama8b", len(lens), lens, seed_appends=3)
+
+
+def test_llama70b_small():
+    run_small("llama70b", 2, [700, 129], seed_appends=2)
+
+
+def test_onebit_small():
+    run_small("onebit", 3, [500, 1, 257])
+
+
+def test_single_token_equals_dequantised_value():
+    """ctx = 1: softmax weight 1, so every head's output is that token's dequantised value."""
+    run_small("llama8b", 1, [1])
+
+
+# ---------------------------------------------------------------- full-size, sampled pairs
+
+@pytest.mark.parametrize("name", ["llama8b", "llama70b", "onebit"])
+def test_full_size_sampled_pairs(name):
+    w = WORKLOADS[name]
+    torch.cuda.empty_cache()
+    cache, signs, S = new_cache(w, w.batch, w.ctx)
+    # generate and append in slices of sequences to bound memory
+    step = max(1, w.batch // 8)
+    q_all = []
+    sampled = [(0, 0), (w.batch - 1, w.n_kv_heads - 1), (w.batch // 2, w.n_kv_heads // 2)]
+    keep = {}
+    for b0 in range(0, w.batch, step):
+        seqs = list(range(b0, min(w.batch, b0 + step)))
+        data = generate(w, DEV, seqs=seqs)
+        cache.quantize(data["k"], data["v"], seq_ids=seqs)
+        q_all.append(data["q"])
+        for (b, hk) in sampled:
+            if b in seqs:
+                keep[(b, hk)] = (f64(data["k"][b - b0, hk]), f64(data["v"][b - b0, hk]))
+        del data
+    q = torch.cat(q_all)
+    out = f64(cache.decode(q))
+    torch.cuda.synchronize()
+    arena = cache.arena.cpu().numpy()
+    info = cache.layout()
+    stats = {}
+    for (b, hk) in sampled:
+        g = w.group
+        K, V = keep[(b, hk)]
+        ref = pair_reference(w, arena, info, b, hk, w.ctx, K, V, f64(q[b, hk * g:(hk + 1) * g]), signs, S, stats)
+        err = rel_err(out[b, hk * g:(hk + 1) * g], ref)
+        assert np.all(err <= REL_TOL), (name, b, hk, err.max())
+    assert np.all(np.isfinite(out))
+    cache.close()
+
+
+# ---------------------------------------------------------------- FP4 latent cache
+
+def fp4_check(ctx, heads_checked=None, batch=1, lens=None):
+    w = WORKLOADS["mla_fp4"]
+    lens = lens or [ctx] * batch
+    data = generate(w, DEV, seqs=range(batch), ctx=max(lens))
+    cache = kvq.KvqCache(kvq.cfg_for_workload(w), batch, max(lens) + 32)
+    for b in range(batch):
+        if lens[b]:
+            cache.quantize(data["latent"][b:b + 1, :lens[b]].contiguous(), data["rope"][b:b + 1, :lens[b]].contiguous(),
+                           seq_ids=[b])
+    out = f64(cache.decode(data["q"]))
+    torch.cuda.synchronize()
+    arena = cache.arena.cpu().numpy()
+    info = cache.layout()
+    for b in range(batch):
+        if lens[b] == 0:
+            assert np.all(out[b] == 0)
+            continue
+        codes, scales, kr = fp4_fields(arena, info, b, lens[b])
+        lat = f64(data["latent"][b, :lens[b]]).astype(np.float32)
+        # codes: bit-exact against the oracle's own encoding, on sampled tokens
+        idx = np.unique(np.concatenate([np.arange(min(64, lens[b])), np.linspace(0, lens[b] - 1, 64).astype(int)]))
+        for t in idx:
+            pk, sc = codec.fp4_quantize(lat[t])
+            np.testing.assert_array_equal(codes[t], pk)
+            np.testing.assert_array_equal(scales[t], sc)
+        np.testing.assert_array_equal(kr, f64(data["rope"][b, :lens[b]]))
+        heads = heads_checked or list(range(w.n_q_heads))
+        ref = attention.mla_decode_attention_many(f64(data["q"][b]), codes, scales, kr,
+                                                  1.0 / math.sqrt(w.latent_dim + w.rope_dim), heads)
+        err = rel_err(out[b, heads], ref)
+        assert np.all(err <= REL_TOL), err.max()
+    cache.close()
+
+
+def test_fp4_small_ragged():
+    fp4_check(0, batch=3, lens=[1000, 0, 33])
+
+
+def test_fp4_full_context_sampled_heads():
+    fp4_check(WORKLOADS["mla_fp4"].ctx, heads_checked=[0, 21, 63])
+
+
+# ---------------------------------------------------------------- errors
+
+def test_capacity_overflow_writes_nothing():
+    w = WORKLOADS["llama8b"]
+    data = generate(w, DEV, seqs=range(2), ctx=40)
+    cache, _, _ = new_cache(w, 2, 32)
+    cache.quantize(data["k"][:, :, :20].contiguous(), data["v"][:, :, :20].contiguous())
+    before = cache.arena.clone()
+    with pytest.raises(kvq.KvqError) as e:
+        cache.quantize(data["k"][:, :, 20:40].contiguous(), data["v"][:, :, 20:40].contiguous())
+    assert e.value.status == 3
+    torch.cuda.synchronize()
+    assert torch.equal(before, cache.arena)
+    assert list(cache.lengths()) == [20, 20]
+    with pytest.raises(kvq.KvqError) as e:
+        cache.quantize(data["k"][:1, :, :1].contiguous(), data["v"][:1, :, :1].contiguous(), seq_ids=[5])
+    assert e.value.status == 1
+    small = torch.empty(16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_decode_attention(cache.handle, data["q"], torch.empty(2, 32, 128, device=DEV), small)
+    assert e.value.status == 5
+    cache.close()

@@ -420,3 +420,31 @@ def test_packed_sizes_per_workload():
     assert sizes.lm_vector_bytes(128, 3, 128) + sizes.lm_vector_bytes(128, 3, 0) == 118
     assert 2 * sizes.lm_vector_bytes(128, 1, 0) == 36
     assert sizes.fp4_token_bytes(512, 64) == 416
+
+
+# ---------------------------------------------------------------- vectorised forms
+
+def test_vectorised_forms_equal_per_vector_forms():
+    rng = np.random.default_rng(21)
+    d, T = 128, 9
+    signs = rotation_signs(5, d)
+    S = qjl_matrix(6, 128, d)
+    c32, _ = tables.lloyd_max_tables_f32(2)
+    codes = rng.integers(0, 4, size=(T, d))
+    n16 = rng.uniform(1, 30, T)
+    g16 = rng.uniform(0.1, 1, T)
+    z = rng.integers(0, 2, size=(T, 128))
+    many = attention.dequantize_many(codes, n16, c32, signs, g16, z, S)
+    one = np.stack([attention.dequantize(codes[t], n16[t], c32, signs, g16[t], z[t], S) for t in range(T)])
+    np.testing.assert_allclose(many, one, rtol=1e-13, atol=1e-13)
+    packed = rng.integers(0, 256, size=(T, 256)).astype(np.uint8)
+    scales = rng.integers(0, 0x7E, size=(T, 32)).astype(np.uint8)
+    np.testing.assert_array_equal(codec_fp4_rows(packed, scales), attention.fp4_dequantize_many(packed, scales))
+    q = rng.standard_normal((3, 576))
+    kr = rng.standard_normal((T, 64))
+    np.testing.assert_allclose(attention.mla_decode_attention_many(q, packed, scales, kr, 0.04),
+                               attention.mla_decode_attention(q, packed, scales, kr, 0.04), rtol=1e-12)
+
+
+def codec_fp4_rows(packed, scales):
+    return np.stack([codec.fp4_dequantize(packed[t], scales[t]) for t in range(packed.shape[0])])
