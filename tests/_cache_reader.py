@@ -20,7 +20,7 @@ def side_fields(arena: np.ndarray, info, side: int, pair: int, n_tokens: int, m:
     tiles = int(info[3])
     region = int(info[4 + side])
     off_planes, off_sketch, off_norm, off_gamma, bits = (int(v) for v in info[6 + 5 * side: 11 + 5 * side])
-    qjl = off_gamma > off_norm
+    qjl = off_norm > off_sketch  # a side without a sketch has an empty sketch block
     tb = _tiles(arena, region, pair, tiles, tile_bytes, n_tokens)
     nt = tb.shape[0]
     planes = np.ascontiguousarray(tb[:, off_planes:off_planes + bits * TILE * 16]
