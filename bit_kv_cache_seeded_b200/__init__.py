@@ -32,7 +32,7 @@ DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "kvq_cache_init",
            "kvq_quantize", "kvq_workspace_bytes", "kvq_decode_attention", "kvq_cache_lengths",
            "kvq_cache_layout", "kvq_lloyd_max_table", "kvq_cache_destroy",
-           "kvq_debug_quantize_rotated")
+           "kvq_debug_quantize_rotated", "kvq_decode_attention_static")
 
 
 class KvqError(RuntimeError):
@@ -75,6 +75,7 @@ def load() -> ctypes.CDLL:
         "kvq_lloyd_max_table": ([I32, VP, VP], I32),
         "kvq_cache_destroy": ([VP], None),
         "kvq_debug_quantize_rotated": ([VP, VP, I32, VP, VP, VP, VP], I32),
+        "kvq_decode_attention_static": ([VP, VP, I32, VP, VP], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -179,6 +180,16 @@ def kvq_decode_attention(handle, q: torch.Tensor, out: torch.Tensor, workspace: 
     st = load().kvq_decode_attention(handle, _ptr(q), DTYPES[q.dtype], _ptr(out), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check("kvq_decode_attention", st)
+
+
+def kvq_decode_attention_static(handle, q: torch.Tensor, out: torch.Tensor, stream=None):
+    """Decode attention without a workspace (partials in the library's fixed device array)."""
+    if q.dtype not in DTYPES or out.dtype != torch.float32:
+        raise TypeError("q must be float32/bfloat16 and out float32")
+    if not (q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("q and out must be contiguous")
+    st = load().kvq_decode_attention_static(handle, _ptr(q), DTYPES[q.dtype], _ptr(out), _stream(stream))
+    _check("kvq_decode_attention_static", st)
 
 
 def kvq_cache_lengths(handle, batch: int) -> np.ndarray:

@@ -458,3 +458,60 @@ kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free decode entry point.
+//
+// Some callers cannot hand the library a workspace: serving loops that reserve all device
+// memory at start-up and forbid any further allocation on the decode path, hosts whose device
+// memory belongs to another allocator, and code that must not call cudaMalloc because it can
+// synchronize the device. For them kvq_decode_attention_static keeps the split-K partials in
+// the fixed array below instead of a caller workspace.
+//
+// The array is file-scope device memory: every GPU that loads this library holds its 16 MiB
+// until the process exits. Its address is a device address only on the device side; host code
+// gets it once per device from cudaGetSymbolAddress (done by the first call on that device).
+// Nothing in it has to start at zero: each call writes every partial slot it later reads. All
+// calls share it, so two calls that overlap on the GPU (e.g. on different streams) race.
+// ---------------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+constexpr int kMaxDevices = 64;
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) float g_kvq_static_scratch[kStaticScratchBytes / sizeof(float)];
+
+namespace {
+kvq_status static_scratch_for_current_device(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kvq_static_scratch) != cudaSuccess || !p) return KVQ_ERR_CUDA;
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return KVQ_OK;
+}
+}  // namespace
+
+extern "C" kvq_status kvq_decode_attention_static(const kvq_cache* c, const void* q, kvq_dtype dtype,
+                                                  float* out, void* stream) {
+  if (!c || !q || !out) return KVQ_ERR_INVALID_ARG;
+  int max_len = 0;
+  for (int v : c->lens) max_len = std::max(max_len, v);
+  const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
+  int splits, chunk;
+  plan_splits(pairs, c->sms, max_len, &splits, &chunk);
+  if (workspace_for(c, splits) > kStaticScratchBytes) return KVQ_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const kvq_status st = static_scratch_for_current_device(&scratch);
+  if (st != KVQ_OK) return st;
+  return kvq_decode_attention(c, q, dtype, out, scratch, kStaticScratchBytes, stream);
+}

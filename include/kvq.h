@@ -124,6 +124,20 @@ kvq_status kvq_workspace_bytes(const kvq_cache* c, size_t* bytes);
 kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* The same decode attention as kvq_decode_attention, for callers that cannot allocate device
+ * memory on the decode path (serving loops that reserve all memory up front, hosts whose memory
+ * belongs to another allocator, code that must not risk the device synchronisation cudaMalloc
+ * can cause). It takes no workspace and allocates nothing: the split partials go to a fixed
+ * 16 MiB device array inside the library, which every GPU that loads the library keeps until
+ * the process exits. The paper has no counterpart to this call; it is an interface
+ * convenience. Returns KVQ_ERR_WORKSPACE, launching nothing, when the partials of this cache
+ * (batch x n_q_heads x splits x (2 + head_dim [+ qjl_dim]) floats; FP4: 2 + latent_dim) would
+ * exceed 16 MiB. The first call on a device looks up the array's device address (once per
+ * device); make that first call before any stream capture. All calls share the array, so calls
+ * that overlap on the GPU (different streams, or threads) race: order them on one stream. */
+kvq_status kvq_decode_attention_static(const kvq_cache* c, const void* q, kvq_dtype dtype,
+                                       float* out, void* stream);
+
 /* Host copy of the current per-sequence lengths (lens: host array of `batch` entries). */
 kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens);
 
