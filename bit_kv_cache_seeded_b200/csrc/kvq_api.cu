@@ -51,8 +51,9 @@ kvq_status validate_cfg(const kvq_cfg* c) {
   return KVQ_OK;
 }
 
-SideLayout make_side(int mode, int bits, int qjl_dim) {
+SideLayout make_side(int mode, int bits, int qjl_dim, int tokmajor) {
   SideLayout L;
+  L.tokmajor = tokmajor;
   L.bits = (mode == KVQ_MODE_SIGN1) ? 1 : bits;
   L.qjl = mode == KVQ_MODE_LM_QJL;
   L.m = L.qjl ? qjl_dim : 0;
@@ -92,7 +93,7 @@ struct Plan {
 Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
   Plan P{};
   P.fp4_mode = c->k_mode == KVQ_MODE_FP4;
-  P.tiles = (capacity + kTile - 1) / kTile;
+  P.tiles = (capacity + kTile * kTilePair - 1) / (kTile * kTilePair) * kTilePair;
   size_t off = 0;
   P.lens_off = off;
   off = align_up(off + sizeof(int) * (size_t)batch, kArenaAlign);
@@ -104,8 +105,8 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
     off = align_up(off + pairs * P.tiles * (size_t)P.fp4.tile_bytes, kArenaAlign);
     P.v_off = off;
   } else {
-    P.k = make_side(c->k_mode, c->k_bits, c->qjl_dim);
-    P.v = make_side(c->v_mode, c->v_bits, c->qjl_dim);
+    P.k = make_side(c->k_mode, c->k_bits, c->qjl_dim, 1);
+    P.v = make_side(c->v_mode, c->v_bits, c->qjl_dim, 0);
     const size_t m = (P.k.qjl || P.v.qjl) ? (size_t)c->qjl_dim : 0;
     P.signs_off = off;
     off = align_up(off + sizeof(float) * kHeadDim, kArenaAlign);
@@ -128,31 +129,63 @@ int device_sms() {
   return sms > 0 ? sms : 148;
 }
 
-// Split plan: enough (pair, split) CTAs to fill the GPU several times over, each split a whole
-// number of tiles. max_splits() bounds the split count for every length up to the capacity.
-int split_target(int pairs, int sms) {
-  const int target = 4 * sms;
-  return std::max(1, (target + pairs - 1) / pairs);
+// Split plan. Each (pair, split) CTA covers a whole number of 64-token units, at most
+// `max_units` of them. The split count minimises waves x (units per CTA + a fixed per-CTA
+// overhead of 4 units), with `slots` resident CTAs per wave; max_splits() bounds it for every
+// length up to the capacity (it sizes the workspace).
+int max_splits(int pairs, int sms, int tiles, int max_units, int waves_bound) {
+  const int units = std::max(1, tiles / kTilePair);
+  const int need = (units + max_units - 1) / max_units;
+  const int bound = std::max(1, (waves_bound * sms + pairs - 1) / pairs);
+  return std::max(need, std::min(bound, units));
 }
 
-void plan_splits(int pairs, int sms, int max_len, int* splits, int* chunk) {
-  const int tiles = std::max(1, (max_len + kTile - 1) / kTile);
-  const int s = std::min(split_target(pairs, sms), tiles);
-  const int chunk_tiles = (tiles + s - 1) / s;
-  *splits = (tiles + chunk_tiles - 1) / chunk_tiles;
-  *chunk = chunk_tiles * kTile;
+void plan_splits(int pairs, int sms, int slots_per_sm, int max_units, int waves_bound, int max_len,
+                 int* splits, int* chunk) {
+  const int units = std::max(1, (max_len + kTile * kTilePair - 1) / (kTile * kTilePair));
+  const int smin = (units + max_units - 1) / max_units;
+  const int smax = std::min(max_splits(pairs, sms, units * kTilePair, max_units, waves_bound), units);
+  const long slots = (long)sms * slots_per_sm;
+  long best_cost = -1;
+  int best_cu = units;
+  for (int s = std::max(1, smin); s <= std::max(smin, smax); ++s) {
+    const int cu = (units + s - 1) / s;
+    if (cu > max_units) continue;
+    const int ss = (units + cu - 1) / cu;
+    const long waves = ((long)pairs * ss + slots - 1) / slots;
+    const long cost = waves * (cu + 4);
+    if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_cu = cu; }
+  }
+  *splits = (units + best_cu - 1) / best_cu;
+  *chunk = best_cu * kTile * kTilePair;
 }
-
-int max_splits(int pairs, int sms, int tiles) { return std::min(split_target(pairs, sms), std::max(1, tiles)); }
 
 int part_stride(const kvq_cache* c) {
   if (c->is_fp4) return 2 + c->cfg.latent_dim;
   return 2 + kHeadDim * (c->v.qjl ? 2 : 1);
 }
 
-size_t workspace_for(const kvq_cache* c, int splits) {
-  return sizeof(float) * (size_t)c->batch * c->cfg.n_q_heads * splits * part_stride(c);
+int prep_stride(const kvq_cache* c) {
+  if (c->is_fp4) return 0;
+  return mma_prep_bytes(c->k.bits, c->k.qjl, c->cfg.n_q_heads / c->cfg.n_kv_heads);
 }
+
+size_t partials_bytes(const kvq_cache* c, int splits) {
+  return align_up(sizeof(float) * (size_t)c->batch * c->cfg.n_q_heads * splits * part_stride(c), 256);
+}
+
+// Workspace = split partials, then the per-(sequence, kv-head) query tables of the tensor-core path.
+size_t workspace_for(const kvq_cache* c, int splits) {
+  return partials_bytes(c, splits) + (size_t)c->batch * c->cfg.n_kv_heads * prep_stride(c);
+}
+
+int decode_slots_per_sm(const kvq_cache* c) { return c->is_fp4 ? 1 : 4; }
+
+// Largest chunk (in 64-token units) one decode CTA may take.
+int decode_max_units(const kvq_cache* c) { return c->is_fp4 ? (1 << 30) : kChunkMax / (kTile * kTilePair); }
+
+// Upper bound on CTAs per SM considered by the split plan (sizes the workspace).
+int decode_waves_bound(const kvq_cache* c) { return c->is_fp4 ? 2 : 16; }
 
 float default_scale(const kvq_cfg& cfg) {
   if (cfg.softmax_scale > 0.f) return cfg.softmax_scale;
@@ -328,7 +361,7 @@ kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dt
 kvq_status kvq_workspace_bytes(const kvq_cache* c, size_t* bytes) {
   if (!c || !bytes) return KVQ_ERR_INVALID_ARG;
   const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
-  *bytes = workspace_for(c, max_splits(pairs, c->sms, c->tiles_per_seq));
+  *bytes = workspace_for(c, max_splits(pairs, c->sms, c->tiles_per_seq, decode_max_units(c), decode_waves_bound(c)));
   return KVQ_OK;
 }
 
@@ -341,7 +374,8 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
   for (int v : c->lens) max_len = std::max(max_len, v);
   const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
   int splits, chunk;
-  plan_splits(pairs, c->sms, max_len, &splits, &chunk);
+  plan_splits(pairs, c->sms, decode_slots_per_sm(c), decode_max_units(c), decode_waves_bound(c), max_len,
+              &splits, &chunk);
   if (ws_bytes < workspace_for(c, splits)) return KVQ_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const float log2e = 1.4426950408889634f;
@@ -388,6 +422,8 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
   p.S = c->d_S;
   p.St = c->d_St;
   p.logit_scale = default_scale(c->cfg) * log2e;
+  p.qprep = static_cast<unsigned char*>(workspace) + partials_bytes(c, splits);
+  p.qprep_stride = prep_stride(c);
   if (launch_decode_lm(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
   if (launch_reduce_lm(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
   return KVQ_OK;
@@ -508,7 +544,8 @@ extern "C" kvq_status kvq_decode_attention_static(const kvq_cache* c, const void
   for (int v : c->lens) max_len = std::max(max_len, v);
   const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
   int splits, chunk;
-  plan_splits(pairs, c->sms, max_len, &splits, &chunk);
+  plan_splits(pairs, c->sms, decode_slots_per_sm(c), decode_max_units(c), decode_waves_bound(c), max_len,
+              &splits, &chunk);
   if (workspace_for(c, splits) > kStaticScratchBytes) return KVQ_ERR_WORKSPACE;
   void* scratch = nullptr;
   const kvq_status st = static_scratch_for_current_device(&scratch);

@@ -42,6 +42,15 @@ __device__ __forceinline__ float exp2_diff(float a, float b) {
 
 constexpr int kWarps = 4;
 
+// 32-bit word k (coordinates 32k..32k+31) of token slot t of a plane at byte offset `off`.
+__device__ __forceinline__ uint32_t vword(const char* tile, const SideLayout& L, int off, int t, int k) {
+  if (L.tokmajor) return *reinterpret_cast<const uint32_t*>(tile + off + t * 16 + k * 4);
+  uint32_t w = 0;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) w |= (uint32_t)(uint8_t)tile[off + (4 * k + b) * kTile + t] << (8 * b);
+  return w;
+}
+
 // Rotated query of one head into smem: q_s = H D q * coef (coef folds 1/sqrt(d) and scales).
 __device__ void rotate_query(const void* q, size_t base, int bf16, const float* signs, float coef,
                              float* dst) {
@@ -177,10 +186,9 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
     for (int t = 0; t < count; ++t) {
       uint32_t vw[VB][4];
 #pragma unroll
-      for (int pp = 0; pp < VB; ++pp) {
-        const uint4 x = *reinterpret_cast<const uint4*>(vt + p.v.off_planes + pp * (kTile * 16) + t * 16);
-        vw[pp][0] = x.x; vw[pp][1] = x.y; vw[pp][2] = x.z; vw[pp][3] = x.w;
-      }
+      for (int pp = 0; pp < VB; ++pp)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) vw[pp][k] = vword(vt, p.v, p.v.off_planes + pp * (kTile * 16), t, k);
       float c[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -191,11 +199,9 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
       }
       float zs[4] = {0.f, 0.f, 0.f, 0.f};
       if (VQ) {
-        const uint4 x = *reinterpret_cast<const uint4*>(vt + p.v.off_sketch + t * 16);
-        zs[0] = ((x.x >> lane) & 1) ? 1.f : -1.f;
-        zs[1] = ((x.y >> lane) & 1) ? 1.f : -1.f;
-        zs[2] = ((x.z >> lane) & 1) ? 1.f : -1.f;
-        zs[3] = ((x.w >> lane) & 1) ? 1.f : -1.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          zs[k] = ((vword(vt, p.v, p.v.off_sketch, t, k) >> lane) & 1) ? 1.f : -1.f;
       }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -240,42 +246,73 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
   }
 }
 
+// One block per (sequence, kv-head): merge the split partials of the group's G query heads,
+// fold the value sketch back (o_r += S^T acc_z, with S staged in shared memory by cp.async while
+// the partials are merged), undo the rotation (out = D H o_r / sqrt(d)) and write out.
+template <int G>
 __global__ void __launch_bounds__(kHeadDim)
 reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
-  __shared__ float zs[kHeadDim];
-  __shared__ float xs[kHeadDim];
-  const int row = blockIdx.x;  // b * Hq + hq
-  const int i = threadIdx.x;
-  const float* part = p.part + (size_t)row * p.splits * p.part_stride;
-  float M = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, part[(size_t)s * p.part_stride]);
-  float L = 0.f, o = 0.f, oz = 0.f;
-  for (int s = 0; s < p.splits; ++s) {
-    const float* ps = part + (size_t)s * p.part_stride;
-    const float w = exp2_diff(ps[0], M);
-    L += w * ps[1];
-    o += w * ps[2 + i];
-    if (vq) oz += w * ps[2 + kHeadDim + i];
-  }
-  const float inv = (L > 0.f) ? 1.f / L : 0.f;
-  o *= inv;
+  extern __shared__ __align__(16) float rs[];
+  float* S_s = rs;                                   // [m][d] when vq
+  float* az = rs + (vq ? p.v.m * kHeadDim : 0);      // [G][d] merged sketch accumulators
+  float* xs = az + G * kHeadDim;                     // [G][d] rotated-domain outputs
+  const int hk = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
   if (vq) {
-    zs[i] = oz * inv;
-    __syncthreads();
-    float acc = 0.f;
-    for (int j = 0; j < p.v.m; ++j) acc = fmaf(p.S[(size_t)j * kHeadDim + i], zs[j], acc);
-    o += acc;
+    for (int c = i; c < p.v.m * kHeadDim / 4; c += kHeadDim) {
+      const unsigned dst = (unsigned)__cvta_generic_to_shared(S_s + 4 * c);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(p.S + 4 * c));
+    }
+    asm volatile("cp.async.commit_group;\n" ::);
   }
-  // out = D H o / sqrt(d)
-  xs[i] = o;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const size_t row = (size_t)b * p.Hq + hk * G + h;
+    const float* part = p.part + row * p.splits * p.part_stride;
+    float M = -INFINITY;
+    for (int s = 0; s < p.splits; ++s) M = fmaxf(M, part[(size_t)s * p.part_stride]);
+    float L = 0.f, o = 0.f, oz = 0.f;
+    for (int s = 0; s < p.splits; ++s) {
+      const float* ps = part + (size_t)s * p.part_stride;
+      const float w = exp2_diff(ps[0], M);
+      L += w * ps[1];
+      o += w * ps[2 + i];
+      if (vq) oz += w * ps[2 + kHeadDim + i];
+    }
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+    xs[h * kHeadDim + i] = o * inv;
+    az[h * kHeadDim + i] = oz * inv;
+  }
+  if (vq) asm volatile("cp.async.wait_group 0;\n" ::);
   __syncthreads();
-  for (int h = 1; h < kHeadDim; h <<= 1) {
-    const float a = xs[i], bb = xs[i ^ h];
+  if (vq) {
+    float acc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < p.v.m; ++j) {
+      const float sv = S_s[j * kHeadDim + i];
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] = fmaf(sv, az[h * kHeadDim + j], acc[h]);
+    }
     __syncthreads();
-    xs[i] = (i & h) ? bb - a : a + bb;
+#pragma unroll
+    for (int h = 0; h < G; ++h) xs[h * kHeadDim + i] += acc[h];
+  }
+  __syncthreads();
+  // out = D H o_r / sqrt(d): Walsh-Hadamard butterflies in shared memory, all heads at once
+  for (int hb = 1; hb < kHeadDim; hb <<= 1) {
+    float a[G], o2[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) { a[h] = xs[h * kHeadDim + i]; o2[h] = xs[h * kHeadDim + (i ^ hb)]; }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < G; ++h) xs[h * kHeadDim + i] = (i & hb) ? o2[h] - a[h] : a[h] + o2[h];
     __syncthreads();
   }
-  p.out[(size_t)row * kHeadDim + i] = xs[i] * p.signs[i] * 0.08838834764831845f;
+  const float sgn = p.signs[i] * 0.08838834764831845f;
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+    p.out[((size_t)b * p.Hq + hk * G + h) * kHeadDim + i] = xs[h * kHeadDim + i] * sgn;
 }
 
 template <int G>
@@ -303,6 +340,7 @@ cudaError_t dispatch_modes(const DecodeParams& p, dim3 grid, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s) {
+  if (mma_decode_supported(p)) return launch_decode_lm_mma(p, s);
   dim3 grid(p.splits, p.Hkv, p.B);
   switch (p.group) {
     case 1: return dispatch_modes<1>(p, grid, s);
@@ -313,9 +351,23 @@ cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s) {
   }
 }
 
-cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s) {
-  reduce_lm<<<p.B * p.Hq, kHeadDim, 0, s>>>(p, p.v.qjl);
+template <int G>
+cudaError_t launch_reduce_g(const DecodeParams& p, cudaStream_t s) {
+  const size_t smem = sizeof(float) * ((p.v.qjl ? (size_t)p.v.m * kHeadDim : 0) + 2 * G * kHeadDim);
+  cudaError_t e = cudaFuncSetAttribute(reduce_lm<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  reduce_lm<G><<<dim3(p.Hkv, p.B), kHeadDim, smem, s>>>(p, p.v.qjl);
   return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s) {
+  switch (p.group) {
+    case 1: return launch_reduce_g<1>(p, s);
+    case 2: return launch_reduce_g<2>(p, s);
+    case 4: return launch_reduce_g<4>(p, s);
+    case 8: return launch_reduce_g<8>(p, s);
+    default: return cudaErrorNotSupported;
+  }
 }
 
 }  // namespace kvq

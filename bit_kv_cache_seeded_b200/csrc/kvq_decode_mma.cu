@@ -1,0 +1,659 @@
+// Tensor-core split-K decode attention for LM / LM_QJL / SIGN1 caches (query group g <= 4).
+//
+// Same computation as the CUDA-core kernel in kvq_decode.cu ("TurboQuant vs OSCAR vs
+// EpiCache", section "Quantization frontiers: TurboQuant and OSCAR": logits from the
+// Lloyd-Max centroids plus the unbiased QJL correction, softmax, values dequantised on the fly),
+// arranged as exact int8 tensor-core contractions (mma.sync m16n8k32 s8 -> s32) over the packed
+// bit-planes:
+//
+//   * Walsh expansion of the code table. The Lloyd-Max table is odd, so with B_i = 2 b_i - 1:
+//       1 bit : c = a0 B0;   2 bits: c = a0 B0 + a1 B1
+//       3 bits: c = a0 B0 + a1 B1 + a2 B2 + a3 B0B1B2,   B0B1B2 = 2 (b0^b1^b2) - 1
+//     so <q, c[code]> = sum_P 2 a_P <q, b_P> - (sum_P a_P) sum_j q_j over 0/1 "Walsh planes".
+//   * Logits: A = key bits [16 tokens x 32 bits]. Byte i of plane word w holds coordinates
+//     32w + 8i + p in bit p; (w << (7 - p)) & 0x80808080 turns bit p of every byte into the int8
+//     value -128 or 0 (one multiply and one LOP3 per 4 operand bytes). B = the query term
+//     2 a_P q~_j quantised to a 14-bit integer (2 x 7-bit signed digits, one column each).
+//   * Values: A = value bits [16 coordinates x 32 tokens] read from the byte-lane-major value
+//     tile, where 4 tokens of one byte-lane are one 32-bit word: w & (0x01010101 << p) gives the
+//     int8 value 2^p (p < 7) or -128 (p = 7) per byte, i.e. a fixed power of two per row. B = the
+//     softmax weights p_t n_t / sqrt(d) (times sqrt(pi/2)/m gamma_t for the value sketch) as a
+//     21-bit integer relative to the chunk maximum (3 x 7-bit unsigned digits).
+//   * Two passes over a CTA's chunk (at most kChunkMax tokens): pass 1 computes every logit into
+//     shared memory and the chunk's maxima; pass 2 streams the value tiles with the weights
+//     2^(l - M) fixed, so the int32 accumulators are exact and never rescaled.
+//
+// CTA: 4 warps. Pass 1: 64 tokens (two cache tiles) per iteration, warp w owns tokens
+// 16w..16w+15. Pass 2: 64 tokens per iteration, warp w owns bit positions 2w, 2w+1 of every value
+// Walsh plane. cp.async stages both passes. Partials (m, l, o_r, acc_z) are written in the format
+// of the CUDA-core kernel; the same reduce kernel finishes.
+#include <algorithm>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr int kWarpsM = 4;
+constexpr int kThreadsM = kWarpsM * 32;
+constexpr int kCtaTok = 64;
+constexpr int kStagesM = 3;
+constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
+constexpr float kSqrtHalfPi = 1.2533141373155003f;  // sqrt(pi/2)
+constexpr int kQRange = 8191;                        // query term quantised to [-8191, 8191]
+constexpr float kWRange = 2097152.f;                 // weights quantised below 2^21
+
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Bit p of every byte of w as the int8 value -128 (set) or 0 (clear).
+template <int P>
+__device__ __forceinline__ uint32_t bit_to_s8(uint32_t w) {
+  return (P == 7) ? (w & 0x80808080u) : ((w * (1u << (7 - P))) & 0x80808080u);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ float load_q(const void* base, size_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  return reinterpret_cast<const float*>(base)[i];
+}
+
+template <int BITS> struct Walsh { static constexpr int P = BITS == 3 ? 4 : BITS; };
+
+// 32-bit word of Walsh plane P from the stored bit-plane words (parity plane for 3 bits).
+template <int BITS>
+__device__ __forceinline__ uint32_t walsh_word(const uint32_t (&w)[3], int P) {
+  if (BITS == 3 && P == 3) return w[0] ^ w[1] ^ w[2];
+  return w[P];
+}
+
+// Walsh coefficients a_P of an odd b-bit table (codes 2^(b-1).. are the positive half).
+__device__ __forceinline__ void walsh_coeffs(int bits, const float* c, float (&a)[4]) {
+  a[0] = a[1] = a[2] = a[3] = 0.f;
+  if (bits == 1) a[0] = c[1];
+  if (bits == 2) { a[0] = 0.5f * (c[3] - c[2]); a[1] = 0.5f * (c[3] + c[2]); }
+  if (bits == 3) {
+    a[0] = 0.25f * (c[7] - c[6] + c[5] - c[4]);
+    a[1] = 0.25f * (c[7] + c[6] - c[5] - c[4]);
+    a[2] = 0.25f * (c[7] + c[6] + c[5] + c[4]);
+    a[3] = 0.25f * (c[7] - c[6] - c[5] + c[4]);
+  }
+}
+
+template <int G, int KB, bool KQ, int VB, bool VQ>
+struct MmaCfg {
+  static constexpr int KP = Walsh<KB>::P + (KQ ? 1 : 0);  // logit planes (sketch last)
+  static constexpr int VP = Walsh<VB>::P + (VQ ? 1 : 0);  // value planes (sketch last)
+  static constexpr int KNT = (2 * G + 7) / 8;             // logit N-tiles: (head, 2 digits)
+  static constexpr int VNT = (4 * G + 7) / 8;             // value N-tiles: (head, 3 digits + pad)
+  static constexpr int VNCOL = VNT * 8;
+};
+
+// ------------------------------------------------------------------------------------------
+// Prep kernel, once per (sequence, kv-head): the logit-phase B operand.
+//   q~ = H D q * scale*log2(e)/d (rotated query),  s~ = sqrt(pi/2)/m * S q~ (sketched query)
+//   centroid planes: v = 2 a_P q~_j;  sketch plane: v = 2 s~_j
+//   q_int = rint(v * 8191 / vmax_h) (vmax over the centroid planes, separately for the sketch),
+//   digits hi = floor((q_int + 64) / 128), lo = q_int - 128 hi, both in [-64, 64).
+// Layout per pair: [KP][G][2 digits][128 fragment-ordered coordinates] bytes, then [G][4] f32:
+// (s, C, sz, Cz) with s = vmax / (8191 * -128) (the one-hot bytes are -128), C = -(sum_P a_P)
+// sum_j q~_j and Cz = -sum_j s~_j. Fragment order of coordinate j: (j%8)*16 + (j/32)*4 + (j%32)/8.
+// ------------------------------------------------------------------------------------------
+template <int G, int KB, bool KQ>
+__global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constant__ DecodeParams p) {
+  constexpr int KP = Walsh<KB>::P + (KQ ? 1 : 0);
+  constexpr int KWP = Walsh<KB>::P;
+  __shared__ float qf[G][kHeadDim];
+  __shared__ float sf[G][kHeadDim];
+  __shared__ float hc[G][4];
+  extern __shared__ __align__(16) float st_s[];  // [128][m] transposed sketch matrix
+  const int hk = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  unsigned char* out = p.qprep + ((size_t)b * p.Hkv + hk) * p.qprep_stride;
+  if (KQ)
+    for (int c = tid; c < kHeadDim * kHeadDim / 4; c += kThreadsM)
+      reinterpret_cast<float4*>(st_s)[c] = __ldg(reinterpret_cast<const float4*>(p.St) + c);
+  const float qcoef = kInvSqrtD * p.logit_scale * kInvSqrtD;
+  for (int h = warp; h < G; h += kWarpsM) {
+    float u[4];
+    const size_t qb = ((size_t)b * p.Hq + hk * G + h) * kHeadDim;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = load_q(p.q, qb + 32 * k + lane, p.bf16) * p.signs[32 * k + lane];
+#pragma unroll
+    for (int bb = 0; bb < 5; ++bb) {
+      const bool upper = (lane >> bb) & 1;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float o = __shfl_xor_sync(0xffffffffu, u[k], 1 << bb);
+        u[k] = upper ? o - u[k] : u[k] + o;
+      }
+    }
+    const float a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
+    qf[h][lane] = (a0 + a2) * qcoef;
+    qf[h][64 + lane] = (a0 - a2) * qcoef;
+    qf[h][32 + lane] = (a1 + a3) * qcoef;
+    qf[h][96 + lane] = (a1 - a3) * qcoef;
+  }
+  __syncthreads();
+  if (KQ) {
+    const float kappa = kSqrtHalfPi / (float)p.k.m;
+    const int j = tid;  // 128 threads, one sketch row each
+    float acc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 8
+    for (int i = 0; i < kHeadDim; ++i) {
+      const float sv = st_s[i * kHeadDim + j];
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] = fmaf(sv, qf[h][i], acc[h]);
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) sf[h][j] = acc[h] * kappa;
+    __syncthreads();
+  }
+  float ka[4];
+  walsh_coeffs(KB, p.k.cent, ka);
+  if (tid < 2 * G) {
+    const int h = tid >> 1, which = tid & 1;  // 0: centroid planes, 1: sketch plane
+    float mx = 0.f, sum = 0.f;
+    for (int j = 0; j < kHeadDim; ++j) {
+      const float v = which ? sf[h][j] : qf[h][j];
+      mx = fmaxf(mx, fabsf(v));
+      sum += v;
+    }
+    float asum = 0.f, amax = 0.f;
+    for (int P = 0; P < KWP; ++P) { asum += ka[P]; amax = fmaxf(amax, fabsf(ka[P])); }
+    mx *= which ? 2.f : 2.f * amax;  // largest |v| over the planes
+    hc[h][2 * which] = mx > 0.f ? mx : 1.f;
+    hc[h][2 * which + 1] = which ? -sum : -asum * sum;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < KP * G * kHeadDim; idx += kThreadsM) {
+    const int P = idx / (G * kHeadDim), h = (idx / kHeadDim) % G, j = idx % kHeadDim;
+    const bool sk = KQ && P == KP - 1;
+    const float v = sk ? 2.f * sf[h][j] : 2.f * ka[min(P, 3)] * qf[h][j];
+    const int q = __float2int_rn(v * ((float)kQRange / hc[h][sk ? 2 : 0]));
+    const int hi = (q + 64) >> 7, lo = q - 128 * hi;
+    const int pj = (j % 8) * 16 + (j / 32) * 4 + (j % 32) / 8;
+    out[((P * G + h) * 2 + 0) * 128 + pj] = (unsigned char)(signed char)hi;
+    out[((P * G + h) * 2 + 1) * 128 + pj] = (unsigned char)(signed char)lo;
+  }
+  __syncthreads();
+  if (tid < 4 * G) {
+    const int h = tid / 4, k = tid % 4;
+    float v = hc[h][k];
+    if (k == 0 || k == 2) v = v / ((float)kQRange * -128.f);  // integer sum -> query units
+    reinterpret_cast<float*>(out + KP * G * 2 * 128)[tid] = v;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Decode kernel (two passes over the CTA's chunk).
+// ------------------------------------------------------------------------------------------
+template <int G, int KB, bool KQ, int VB, bool VQ>
+__global__ void __launch_bounds__(kThreadsM, 4)
+decode_lm_mma(const __grid_constant__ DecodeParams p) {
+  using C = MmaCfg<G, KB, KQ, VB, VQ>;
+  constexpr int KP = C::KP, VP = C::VP, KNT = C::KNT, VNT = C::VNT, VNCOL = C::VNCOL;
+  constexpr int VWP = Walsh<VB>::P;
+  constexpr int NKIND = VQ ? 2 : 1;
+  constexpr int NTASK = NKIND * G * 16;
+  static_assert(NTASK <= kThreadsM, "one weight task per thread");
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int ktb = p.k.tile_bytes, vtb = p.v.tile_bytes;
+  const int stage_bytes = 2 * max(ktb, vtb);
+  unsigned char* stages = smem;                                            // [kStagesM][2 tiles]
+  float* lgs = reinterpret_cast<float*>(stages + kStagesM * stage_bytes);  // [G][kChunkMax] logits
+  unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * kChunkMax);  // [NKIND][VNCOL][64]
+  float* red = reinterpret_cast<float*>(pdig + NKIND * VNCOL * kCtaTok);       // reductions
+
+  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int len = p.lens[b];
+  const int t_begin = split * p.chunk;
+  const int t_end = min(len, t_begin + p.chunk);
+  const size_t pair = (size_t)b * p.Hkv + hk;
+  const unsigned char* kbase = reinterpret_cast<const unsigned char*>(p.kreg) + pair * p.tiles_per_seq * (size_t)ktb;
+  const unsigned char* vbase = reinterpret_cast<const unsigned char*>(p.vreg) + pair * p.tiles_per_seq * (size_t)vtb;
+  const int n_iter = t_end > t_begin ? (t_end - t_begin + kCtaTok - 1) / kCtaTok : 0;
+
+  // stage loader: the two cache tiles of K (pass 0) or V (pass 1) for iteration `it`
+  auto load_stage = [&](int pass, int it, int slot) {
+    if (it < n_iter) {
+      const int tile0 = (t_begin + it * kCtaTok) / kTile;
+      const int ntiles = (t_begin + it * kCtaTok + kTile < t_end) ? 2 : 1;
+      const int tb = pass ? vtb : ktb;
+      const unsigned char* src = (pass ? vbase : kbase) + (size_t)tile0 * tb;
+      unsigned char* dst = stages + slot * stage_bytes;
+      for (int c = tid; c < ntiles * tb / 16; c += kThreadsM) cp_async16(dst + 16 * c, src + 16 * c);
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int s = 0; s < kStagesM - 1; ++s) load_stage(0, s, s);
+
+  // logit-phase B fragments (query digits) and head constants from the prep area
+  const unsigned char* prep = p.qprep + pair * p.qprep_stride;
+  uint32_t qb[KP][4][KNT][2];
+#pragma unroll
+  for (int P = 0; P < KP; ++P)
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int nt = 0; nt < KNT; ++nt) {
+        const int n = nt * 8 + g, h = n / 2, d = n % 2;  // column = (head, digit)
+        if (h < G) {
+          const unsigned char* row = prep + ((P * G + h) * 2 + d) * 128;
+          qb[P][m][nt][0] = __ldg(reinterpret_cast<const uint32_t*>(row + ((2 * m) * 4 + t) * 4));
+          qb[P][m][nt][1] = __ldg(reinterpret_cast<const uint32_t*>(row + ((2 * m + 1) * 4 + t) * 4));
+        } else {
+          qb[P][m][nt][0] = qb[P][m][nt][1] = 0u;
+        }
+      }
+  // this thread's logit columns (2t, 2t+1) of N-tile nt: digits (hi, lo) of head 4 nt + t
+  const float* hconst = reinterpret_cast<const float*>(prep + KP * G * 2 * 128);
+  float hs[KNT], hc[KNT], hsz[KNT], hcz[KNT];
+#pragma unroll
+  for (int nt = 0; nt < KNT; ++nt) {
+    const int h = min(4 * nt + t, G - 1);
+    hs[nt] = __ldg(hconst + h * 4 + 0);
+    hc[nt] = __ldg(hconst + h * 4 + 1);
+    hsz[nt] = __ldg(hconst + h * 4 + 2);
+    hcz[nt] = __ldg(hconst + h * 4 + 3);
+  }
+  const float vkappa = VQ ? kSqrtHalfPi / (float)p.v.m : 0.f;
+
+  // ================= pass 1: logits of the whole chunk into lgs, running maxima
+  float mrow[KNT];  // max over this thread's logits of head 4 nt + t
+#pragma unroll
+  for (int nt = 0; nt < KNT; ++nt) mrow[nt] = -INFINITY;
+  float wmax = 0.f;  // largest value weight (times max(1, sketch weight)) seen by this thread
+  const int tl = warp * 16;
+  for (int it = 0; it < n_iter; ++it) {
+    load_stage(0, it + kStagesM - 1, (it + kStagesM - 1) % kStagesM);
+    cp_async_wait<kStagesM - 1>();
+    __syncthreads();
+    const unsigned char* kt = stages + (it % kStagesM) * stage_bytes;
+    const int tok0 = it * kCtaTok;  // chunk-relative first token of this iteration
+    const int count = min(kCtaTok, t_end - (t_begin + tok0));
+    {
+      const unsigned char* ktile = kt + (tl / kTile) * ktb;
+      const int s0 = (tl % kTile) + g, s1 = s0 + 8;
+      int acc[KNT][4], accz[KNT][4];
+#pragma unroll
+      for (int nt = 0; nt < KNT; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) { acc[nt][c] = 0; accz[nt][c] = 0; }
+      uint32_t w0[3] = {0u, 0u, 0u}, w1[3] = {0u, 0u, 0u};
+      const unsigned char* kp = ktile + p.k.off_planes + t * 4;
+#pragma unroll
+      for (int pp = 0; pp < KB; ++pp) {
+        w0[pp] = *reinterpret_cast<const uint32_t*>(kp + pp * (kTile * 16) + s0 * 16);
+        w1[pp] = *reinterpret_cast<const uint32_t*>(kp + pp * (kTile * 16) + s1 * 16);
+      }
+#pragma unroll
+      for (int P = 0; P < KP; ++P) {
+        const bool sk = KQ && P == KP - 1;
+        uint32_t x0, x1;
+        if (sk) {
+          x0 = *reinterpret_cast<const uint32_t*>(ktile + p.k.off_sketch + s0 * 16 + t * 4);
+          x1 = *reinterpret_cast<const uint32_t*>(ktile + p.k.off_sketch + s1 * 16 + t * 4);
+        } else {
+          x0 = walsh_word<KB>(w0, P);
+          x1 = walsh_word<KB>(w1, P);
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          uint32_t a0, a1, a2, a3;
+          switch (m) {
+            case 0: a0 = bit_to_s8<0>(x0); a1 = bit_to_s8<0>(x1); a2 = bit_to_s8<1>(x0); a3 = bit_to_s8<1>(x1); break;
+            case 1: a0 = bit_to_s8<2>(x0); a1 = bit_to_s8<2>(x1); a2 = bit_to_s8<3>(x0); a3 = bit_to_s8<3>(x1); break;
+            case 2: a0 = bit_to_s8<4>(x0); a1 = bit_to_s8<4>(x1); a2 = bit_to_s8<5>(x0); a3 = bit_to_s8<5>(x1); break;
+            default: a0 = bit_to_s8<6>(x0); a1 = bit_to_s8<6>(x1); a2 = bit_to_s8<7>(x0); a3 = bit_to_s8<7>(x1); break;
+          }
+#pragma unroll
+          for (int nt = 0; nt < KNT; ++nt) {
+            if (sk) mma_s8(accz[nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+            else mma_s8(acc[nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+          }
+        }
+      }
+      const float nk0 = __half2float(*reinterpret_cast<const __half*>(ktile + p.k.off_norm + s0 * 2));
+      const float nk1 = __half2float(*reinterpret_cast<const __half*>(ktile + p.k.off_norm + s1 * 2));
+      float gk0 = 0.f, gk1 = 0.f;
+      if (KQ) {
+        gk0 = __half2float(*reinterpret_cast<const __half*>(ktile + p.k.off_gamma + s0 * 2));
+        gk1 = __half2float(*reinterpret_cast<const __half*>(ktile + p.k.off_gamma + s1 * 2));
+      }
+      const bool v0 = tl + g < count, v1 = tl + g + 8 < count;
+#pragma unroll
+      for (int nt = 0; nt < KNT; ++nt) {
+        const int h = 4 * nt + t;
+        float l0 = fmaf(hs[nt], (float)(acc[nt][0] * 128 + acc[nt][1]), hc[nt]);
+        float l1 = fmaf(hs[nt], (float)(acc[nt][2] * 128 + acc[nt][3]), hc[nt]);
+        if (KQ) {
+          l0 = fmaf(gk0, fmaf(hsz[nt], (float)(accz[nt][0] * 128 + accz[nt][1]), hcz[nt]), l0);
+          l1 = fmaf(gk1, fmaf(hsz[nt], (float)(accz[nt][2] * 128 + accz[nt][3]), hcz[nt]), l1);
+        }
+        const float lg0 = v0 ? nk0 * l0 : -INFINITY, lg1 = v1 ? nk1 * l1 : -INFINITY;
+        if (h < G) {
+          lgs[h * kChunkMax + tok0 + tl + g] = lg0;
+          lgs[h * kChunkMax + tok0 + tl + g + 8] = lg1;
+        }
+        mrow[nt] = fmaxf(mrow[nt], fmaxf(lg0, lg1));
+      }
+    }
+    // largest value weight: tokens of this iteration, one per thread of warps 0 and 1
+    if (tid < count) {
+      const size_t tok = (size_t)t_begin + tok0 + tid;
+      const unsigned char* vtile = vbase + (tok / kTile) * vtb;
+      float w = __half2float(*reinterpret_cast<const __half*>(vtile + p.v.off_norm + (tok % kTile) * 2)) * kInvSqrtD;
+      if (VQ) w *= fmaxf(1.f, __half2float(*reinterpret_cast<const __half*>(vtile + p.v.off_gamma + (tok % kTile) * 2)) * vkappa);
+      wmax = fmaxf(wmax, w);
+    }
+    __syncthreads();  // the next iteration refills a stage buffer
+  }
+  // prefetch the first value tiles while the maxima are combined
+#pragma unroll
+  for (int s = 0; s < kStagesM - 1; ++s) load_stage(1, s, s);
+
+  // chunk maxima per head, and the weight scale
+  float* hmax = red;                 // [kWarpsM][G]
+  float* wred = red + kWarpsM * G;   // [kWarpsM]
+#pragma unroll
+  for (int nt = 0; nt < KNT; ++nt) {
+    float mx = mrow[nt];
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (g == 0 && 4 * nt + t < G) hmax[warp * G + 4 * nt + t] = mx;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+  if (lane == 0) wred[warp] = wmax;
+  __syncthreads();
+  float wm = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarpsM; ++w) wm = fmaxf(wm, wred[w]);
+  // integer weights below 2^21 (3 x 7-bit digits); a power-of-two scale keeps the digits exact
+  const float wsc = wm > 0.f ? exp2f(floorf(log2f(kWRange / wm)) - 1.f) : 1.f;
+
+  // ================= pass 2: weights -> digits, value contractions
+  const bool has_task = tid < NTASK;
+  const int task_kind = tid / (G * 16), task_h = (tid / 16) % G, task_q = tid % 16;
+  float task_m = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarpsM; ++w) task_m = fmaxf(task_m, hmax[w * G + task_h]);
+  float task_l = 0.f;     // sum of p over this task's tokens
+  long long task_wl = 0;  // sum of the quantised weights (exact)
+  for (int idx = tid; idx < NKIND * VNCOL * kCtaTok / 4; idx += kThreadsM)
+    reinterpret_cast<uint32_t*>(pdig)[idx] = 0u;  // the pad digit and absent heads stay zero
+
+  int vacc[VP][2][VNT][4];
+#pragma unroll
+  for (int P = 0; P < VP; ++P)
+#pragma unroll
+    for (int pi = 0; pi < 2; ++pi)
+#pragma unroll
+      for (int nt = 0; nt < VNT; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) vacc[P][pi][nt][c] = 0;
+  const uint32_t vm0 = 0x01010101u << (2 * warp), vm1 = 0x01010101u << (2 * warp + 1);
+
+  for (int it = 0; it < n_iter; ++it) {
+    load_stage(1, it + kStagesM - 1, (it + kStagesM - 1) % kStagesM);
+    cp_async_wait<kStagesM - 1>();
+    __syncthreads();
+    const unsigned char* vt = stages + (it % kStagesM) * stage_bytes;
+    const int tok0 = it * kCtaTok;
+    const int count = min(kCtaTok, t_end - (t_begin + tok0));
+
+    // weight task: 4 consecutive tokens of one head, one kind
+    if (has_task) {
+      const int T = 4 * task_q;
+      const float4 l4 = *reinterpret_cast<const float4*>(lgs + task_h * kChunkMax + tok0 + T);
+      const unsigned char* vtile = vt + (T / kTile) * vtb;
+      const uint2 nraw = *reinterpret_cast<const uint2*>(vtile + p.v.off_norm + (T % kTile) * 2);
+      const float2 n01 = __half22float2(*reinterpret_cast<const __half2*>(&nraw.x));
+      const float2 n23 = __half22float2(*reinterpret_cast<const __half2*>(&nraw.y));
+      float wv[4] = {n01.x * kInvSqrtD, n01.y * kInvSqrtD, n23.x * kInvSqrtD, n23.y * kInvSqrtD};
+      if (VQ && task_kind == 1) {
+        const uint2 graw = *reinterpret_cast<const uint2*>(vtile + p.v.off_gamma + (T % kTile) * 2);
+        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&graw.x));
+        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&graw.y));
+        wv[0] *= g01.x * vkappa; wv[1] *= g01.y * vkappa; wv[2] *= g23.x * vkappa; wv[3] *= g23.y * vkappa;
+      }
+      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+      uint32_t d0 = 0, d1 = 0, d2 = 0;
+      float psum = 0.f;
+      int qsum = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool ok = T + e < count;
+        const float pe = ok ? exp2f(lv[e] - task_m) : 0.f;
+        psum += pe;
+        const int q = ok ? __float2int_rn(pe * wv[e] * wsc) : 0;  // < 2^21
+        qsum += q;
+        d0 |= (uint32_t)(q >> 14) << (8 * e);
+        d1 |= (uint32_t)((q >> 7) & 127) << (8 * e);
+        d2 |= (uint32_t)(q & 127) << (8 * e);
+      }
+      task_l += psum;
+      task_wl += qsum;
+      unsigned char* col = pdig + (size_t)(task_kind * VNCOL + 4 * task_h) * kCtaTok + T;
+      *reinterpret_cast<uint32_t*>(col) = d0;
+      *reinterpret_cast<uint32_t*>(col + kCtaTok) = d1;
+      *reinterpret_cast<uint32_t*>(col + 2 * kCtaTok) = d2;
+    }
+    __syncthreads();
+
+    // value contractions: positions 2w, 2w+1 of every value Walsh plane
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      if (s * kTile >= count) break;
+      const unsigned char* vtile = vt + s * vtb;
+      uint32_t bm[VNT][2], bz[VNT][2];
+#pragma unroll
+      for (int nt = 0; nt < VNT; ++nt) {
+        const unsigned char* col = pdig + (size_t)(nt * 8 + g) * kCtaTok + s * kTile + 4 * t;
+        bm[nt][0] = *reinterpret_cast<const uint32_t*>(col);
+        bm[nt][1] = *reinterpret_cast<const uint32_t*>(col + 16);
+        if (VQ) {
+          const unsigned char* colz = col + (size_t)VNCOL * kCtaTok;
+          bz[nt][0] = *reinterpret_cast<const uint32_t*>(colz);
+          bz[nt][1] = *reinterpret_cast<const uint32_t*>(colz + 16);
+        }
+      }
+      uint32_t xv[3][4];
+#pragma unroll
+      for (int pp = 0; pp < VB; ++pp) {
+        const unsigned char* pl = vtile + p.v.off_planes + pp * (kTile * 16) + 4 * t;
+        xv[pp][0] = *reinterpret_cast<const uint32_t*>(pl + g * kTile);
+        xv[pp][1] = *reinterpret_cast<const uint32_t*>(pl + (g + 8) * kTile);
+        xv[pp][2] = *reinterpret_cast<const uint32_t*>(pl + g * kTile + 16);
+        xv[pp][3] = *reinterpret_cast<const uint32_t*>(pl + (g + 8) * kTile + 16);
+      }
+#pragma unroll
+      for (int P = 0; P < VP; ++P) {
+        const bool sk = VQ && P == VP - 1;
+        uint32_t x[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          if (sk) {
+            const unsigned char* pl = vtile + p.v.off_sketch + 4 * t;
+            x[r] = *reinterpret_cast<const uint32_t*>(pl + ((r & 1) ? g + 8 : g) * kTile + ((r & 2) ? 16 : 0));
+          } else if (VB == 3 && P == 3) {
+            x[r] = xv[0][r] ^ xv[1][r] ^ xv[2][r];
+          } else {
+            x[r] = xv[P][r];
+          }
+        }
+        const uint32_t a00 = x[0] & vm0, a01 = x[1] & vm0, a02 = x[2] & vm0, a03 = x[3] & vm0;
+        const uint32_t a10 = x[0] & vm1, a11 = x[1] & vm1, a12 = x[2] & vm1, a13 = x[3] & vm1;
+#pragma unroll
+        for (int nt = 0; nt < VNT; ++nt) {
+          const uint32_t b0 = sk ? bz[nt][0] : bm[nt][0], b1 = sk ? bz[nt][1] : bm[nt][1];
+          mma_s8(vacc[P][0][nt], a00, a01, a02, a03, b0, b1);
+          mma_s8(vacc[P][1][nt], a10, a11, a12, a13, b0, b1);
+        }
+      }
+    }
+    __syncthreads();  // the next iteration refills a stage buffer and the digits
+  }
+
+  // ================= finish: per-head sums of p and of the weights, then this warp's rows
+  cp_async_wait<0>();
+  __syncthreads();
+  float* tsum = reinterpret_cast<float*>(stages);  // [kThreadsM][2] (staging reused)
+  float* hsum = tsum + 2 * kThreadsM;               // [3][G]: sum p, sum weights, sum sketch weights
+  tsum[2 * tid] = task_l;
+  tsum[2 * tid + 1] = (float)task_wl;
+  __syncthreads();
+  if (tid < 3 * G) {
+    const int what = tid / G, h = tid % G;
+    const int kind = what == 2 ? 1 : 0;
+    float s2 = 0.f;
+    if (kind < NKIND)
+      for (int q = 0; q < 16; ++q) s2 += tsum[2 * ((kind * G + h) * 16 + q) + (what == 0 ? 0 : 1)];
+    hsum[tid] = s2;
+  }
+  __syncthreads();
+  float va[4];
+  walsh_coeffs(VB, p.v.cent, va);
+  float vasum = 0.f;
+#pragma unroll
+  for (int P = 0; P < VWP; ++P) vasum += va[P];
+  const float inv_w = 1.f / wsc;
+#pragma unroll
+  for (int pi = 0; pi < 2; ++pi) {
+    const int pos = 2 * warp + pi;
+    const float rowinv = (pos == 7 ? -1.f / 128.f : 1.f / (float)(1 << pos)) * inv_w;  // row value 2^p or -128
+#pragma unroll
+    for (int nt = 0; nt < VNT; ++nt) {
+      const int h = 2 * nt + t / 2;
+      // columns (2t, 2t+1): digits (0, 1) for even t, (2, pad) for odd t, of head 2 nt + t / 2
+      const float wd0 = (t & 1) ? 1.f : 16384.f, wd1 = (t & 1) ? 0.f : 128.f;
+      float o0 = 0.f, o1 = 0.f, z0 = 0.f, z1 = 0.f;
+#pragma unroll
+      for (int P = 0; P < VP; ++P) {
+        float r0 = (float)vacc[P][pi][nt][0] * wd0 + (float)vacc[P][pi][nt][1] * wd1;
+        float r1 = (float)vacc[P][pi][nt][2] * wd0 + (float)vacc[P][pi][nt][3] * wd1;
+        r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
+        r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+        const bool sk = VQ && P == VP - 1;
+        if (sk) { z0 = 2.f * r0 * rowinv; z1 = 2.f * r1 * rowinv; }
+        else { o0 = fmaf(2.f * va[min(P, 3)], r0 * rowinv, o0); o1 = fmaf(2.f * va[min(P, 3)], r1 * rowinv, o1); }
+      }
+      if (h < G) {
+        float* dst = p.part + (((size_t)b * p.Hq + hk * G + h) * p.splits + split) * p.part_stride;
+        const int j0 = 8 * g + pos, j1 = 8 * (g + 8) + pos;
+        if ((t & 1) == 0) {
+          const float Wt = hsum[G + h] * inv_w;
+          dst[2 + j0] = o0 - vasum * Wt;
+          dst[2 + j1] = o1 - vasum * Wt;
+        } else if (VQ) {
+          const float Wz = hsum[2 * G + h] * inv_w;
+          dst[2 + kHeadDim + j0] = z0 - Wz;
+          dst[2 + kHeadDim + j1] = z1 - Wz;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    if (tid == h) {
+      float* dst = p.part + (((size_t)b * p.Hq + hk * G + h) * p.splits + split) * p.part_stride;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarpsM; ++w) mx = fmaxf(mx, hmax[w * G + h]);
+      dst[0] = mx;
+      dst[1] = hsum[h];
+    }
+  }
+}
+
+template <int G, int KB, bool KQ, int VB, bool VQ>
+size_t mma_smem_bytes(const DecodeParams& p) {
+  using C = MmaCfg<G, KB, KQ, VB, VQ>;
+  constexpr int NKIND = VQ ? 2 : 1;
+  size_t s = (size_t)kStagesM * 2 * std::max(p.k.tile_bytes, p.v.tile_bytes);
+  s += sizeof(float) * (size_t)G * kChunkMax;
+  s += (size_t)NKIND * C::VNCOL * kCtaTok;
+  s += sizeof(float) * (kWarpsM * G + kWarpsM);
+  return (s + 15) / 16 * 16;
+}
+
+template <int G, int KB, bool KQ, int VB, bool VQ>
+cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s) {
+  const size_t prep_smem = KQ ? sizeof(float) * kHeadDim * kHeadDim : 0;
+  cudaError_t e = cudaFuncSetAttribute(decode_lm_prep<G, KB, KQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)prep_smem);
+  if (e != cudaSuccess) return e;
+  decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv, p.B), kThreadsM, prep_smem, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = mma_smem_bytes<G, KB, KQ, VB, VQ>(p);
+  auto kern = decode_lm_mma<G, KB, KQ, VB, VQ>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(p.splits, p.Hkv, p.B), kThreadsM, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t dispatch_mma_modes(const DecodeParams& p, cudaStream_t s) {
+  const int kb = p.k.bits, vb = p.v.bits;
+  const bool kq = p.k.qjl, vq = p.v.qjl;
+#define KVQ_MMA_CASE(KB, KQ, VB, VQ) \
+  if (kb == KB && kq == KQ && vb == VB && vq == VQ) return launch_mma<G, KB, KQ, VB, VQ>(p, s);
+  KVQ_MMA_CASE(2, true, 2, true)
+  KVQ_MMA_CASE(3, true, 3, false)
+  KVQ_MMA_CASE(1, false, 1, false)
+  KVQ_MMA_CASE(2, true, 2, false)
+  KVQ_MMA_CASE(3, true, 3, true)
+  KVQ_MMA_CASE(2, false, 2, false)
+  KVQ_MMA_CASE(3, false, 3, false)
+#undef KVQ_MMA_CASE
+  return cudaErrorNotSupported;
+}
+
+}  // namespace
+
+int mma_prep_bytes(int k_bits, int k_qjl, int group) {
+  const int kp = (k_bits == 3 ? 4 : k_bits) + (k_qjl ? 1 : 0);
+  const int bytes = kp * group * 2 * 128 + 16 * group;
+  return (bytes + 255) / 256 * 256;
+}
+
+bool mma_decode_supported(const DecodeParams& p) {
+  return (p.group == 1 || p.group == 2 || p.group == 4) && p.chunk % kCtaTok == 0 &&
+         p.chunk <= kChunkMax && p.qprep != nullptr;
+}
+
+cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s) {
+  switch (p.group) {
+    case 1: return dispatch_mma_modes<1>(p, s);
+    case 2: return dispatch_mma_modes<2>(p, s);
+    case 4: return dispatch_mma_modes<4>(p, s);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace kvq

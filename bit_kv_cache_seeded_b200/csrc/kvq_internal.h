@@ -15,15 +15,18 @@ constexpr int kTile = 32;          // tokens per cache tile
 constexpr int kHeadDim = 128;      // head_dim supported by the rotated (LM/SIGN1) modes
 constexpr int kMaxSeqPerLaunch = 1024;
 constexpr int kMaxBits = 3;
+constexpr int kTilePair = 2;      // cache tiles are allocated and split in pairs (64 tokens)
+constexpr int kChunkMax = 2048;   // largest context chunk of one decode CTA (LM tensor-core path)
 
 // Where one side (K or V) of an LM/SIGN1 cache keeps its fields inside a 32-token tile.
 struct SideLayout {
   int bits = 0;         // code bit-planes
   int qjl = 0;          // 1 if a residual sign sketch is stored
+  int tokmajor = 1;     // 1: [32 tokens][16 B] per plane; 0: [16 byte-lanes][32 tokens]
   int m = 0;            // sketch rows
   int tile_bytes = 0;
-  int off_planes = 0;   // [bits][32][16 B]
-  int off_sketch = 0;   // [32][m/8 B]
+  int off_planes = 0;   // [bits][32 x 16 B] (layout per tokmajor)
+  int off_sketch = 0;   // [32 x m/8 B] (layout per tokmajor)
   int off_norm = 0;     // [32] fp16
   int off_gamma = 0;    // [32] fp16
   float cent[8] = {};   // fp32 Lloyd-Max centroids (2^bits, ascending)
@@ -75,6 +78,8 @@ struct DecodeParams {
   const float* S;         // [m][d]
   const float* St;        // [d][m]
   float logit_scale;      // softmax_scale * log2(e)
+  unsigned char* qprep;   // per (sequence, kv-head) query digit tables (tensor-core path)
+  int qprep_stride;       // bytes per (sequence, kv-head)
 };
 
 struct MlaParams {
@@ -95,9 +100,14 @@ struct MlaParams {
 cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s);
 cudaError_t launch_quantize_fp4(const QuantizeParams& p, cudaStream_t s);
 cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s);
+bool mma_decode_supported(const DecodeParams& p);
+int mma_prep_bytes(int k_bits, int k_qjl, int group);  // bytes of one (sequence, kv-head) prep area
+cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s);
+bool mla_mma_supported(const MlaParams& p);
+cudaError_t launch_decode_mla_mma(const MlaParams& p, cudaStream_t s);
 
 // Host Lloyd-Max tables (lloyd_max.cpp): fp64 fixed-point iteration rounded to fp32.
 void lloyd_max_f32(int bits, float* centroids, float* thresholds);

@@ -42,8 +42,14 @@ constexpr int kQuantWarps = 8;
 __global__ void __launch_bounds__(kQuantWarps * 32)
 quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
   __shared__ float rho_s[kQuantWarps][kHeadDim];
+  extern __shared__ __align__(16) float st_s[];  // [d][m] transposed sketch matrix (sketch sides)
   const int side = blockIdx.y;
   const SideLayout& L = p.side[side];
+  if (L.qjl) {
+    for (int c = threadIdx.x; c < kHeadDim * L.m / 4; c += blockDim.x)
+      reinterpret_cast<float4*>(st_s)[c] = __ldg(reinterpret_cast<const float4*>(p.St) + c);
+    __syncthreads();
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nthr = L.bits ? (1 << L.bits) - 1 : 0;
   const long total = (long)p.n_seq * p.heads * p.n_new;
@@ -104,11 +110,12 @@ quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
       for (int k = 0; k < 4; ++k) rho_s[warp][32 * k + lane] = rho[k];
       __syncwarp();
       float proj[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
       for (int i = 0; i < kHeadDim; ++i) {
         const float r = rho_s[warp][i];
-        const float* row = p.St + (size_t)i * L.m;
+        const float* row = st_s + i * L.m;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) proj[k] = fmaf(__ldg(row + 32 * k + lane), r, proj[k]);
+        for (int k = 0; k < 4; ++k) proj[k] = fmaf(row[32 * k + lane], r, proj[k]);
       }
       __syncwarp();
 #pragma unroll
@@ -130,11 +137,21 @@ quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
     const int tile = pos / kTile, slot = pos % kTile;
     char* tb = p.region[side] +
                (((size_t)seq * p.heads + h) * p.tiles_per_seq + tile) * (size_t)L.tile_bytes;
-    if (lane < L.bits)
-      *reinterpret_cast<uint4*>(tb + L.off_planes + lane * (kTile * 16) + slot * 16) =
-          make_uint4(planes[lane][0], planes[lane][1], planes[lane][2], planes[lane][3]);
-    if (L.qjl && lane == 31)
-      *reinterpret_cast<uint4*>(tb + L.off_sketch + slot * 16) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+    if (L.tokmajor) {
+      if (lane < L.bits)
+        *reinterpret_cast<uint4*>(tb + L.off_planes + lane * (kTile * 16) + slot * 16) =
+            make_uint4(planes[lane][0], planes[lane][1], planes[lane][2], planes[lane][3]);
+      if (L.qjl && lane == 31)
+        *reinterpret_cast<uint4*>(tb + L.off_sketch + slot * 16) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+    } else {
+      // byte-lane-major: byte k of a token's 16-byte plane goes to [k][slot]
+      for (int idx = lane; idx < (L.bits + L.qjl) * 16; idx += 32) {
+        const int pp = idx >> 4, k = idx & 15;
+        const uint32_t w = (pp < L.bits) ? planes[pp][k >> 2] : zw[k >> 2];
+        const int off = (pp < L.bits) ? L.off_planes + pp * (kTile * 16) : L.off_sketch;
+        tb[off + k * kTile + slot] = (char)((w >> (8 * (k & 3))) & 0xFFu);
+      }
+    }
     if (lane == 30) *reinterpret_cast<__half*>(tb + L.off_norm + slot * 2) = __float2half_rn(n);
     if (L.qjl && lane == 29)
       *reinterpret_cast<__half*>(tb + L.off_gamma + slot * 2) = __float2half_rn(gamma);
@@ -208,7 +225,12 @@ int grid_for(long work_items, int per_block) {
 cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s) {
   const long total = (long)p.n_seq * p.heads * p.n_new;
   dim3 grid(grid_for(total, kQuantWarps), n_sides);
-  quantize_lm_kernel<<<grid, kQuantWarps * 32, 0, s>>>(p);
+  const bool sketch = p.side[0].qjl || (n_sides > 1 && p.side[1].qjl);
+  const int m = p.side[0].qjl ? p.side[0].m : p.side[1].m;
+  const size_t smem = sketch ? sizeof(float) * kHeadDim * m : 0;
+  cudaError_t e = cudaFuncSetAttribute(quantize_lm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  quantize_lm_kernel<<<grid, kQuantWarps * 32, smem, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -88,7 +88,7 @@ typedef struct kvq_cache kvq_cache; /* opaque host object */
 const char* kvq_status_str(kvq_status s);
 
 /* Bytes of device memory a cache of `batch` sequences x `capacity` tokens needs (tables
- * included). capacity is rounded up internally to a multiple of 32 tokens. */
+ * included). capacity is rounded up internally to a multiple of 64 tokens. */
 kvq_status kvq_cache_bytes(const kvq_cfg* cfg, int32_t batch, int32_t capacity, size_t* bytes);
 
 /* Packed bytes one token occupies per KV head (codes, sketch and norms of K and V; FP4:
@@ -145,11 +145,15 @@ kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens);
  * info[0..15] receives: tile_tokens, k_tile_bytes, v_tile_bytes, tiles_per_seq,
  * k_region_offset, v_region_offset, then per side (K at 6, V at 11): planes_offset,
  * sketch_offset, norm_offset, gamma_offset, planes. Layout of a tile (32 tokens) of one
- * (sequence, kv-head): [planes][32 tokens][head_dim/8 bytes] code bit-planes (plane p holds
- * bit p of every code; 32-bit word w of a token's plane holds coordinates 32w..32w+31,
- * coordinate 32w+i in bit i), then [32][qjl_dim/8] sign words (bit = 1 for a non-negative
- * projection), then [32] fp16 norms, then [32] fp16 residual norms. Tiles of a (sequence,
- * kv-head) are consecutive; (sequence, kv-head) pairs follow in row-major order.
+ * (sequence, kv-head): code bit-planes, then sign words, then [32] fp16 norms, then [32] fp16
+ * residual norms (sides with a sketch). Plane p holds bit p of every code; within a token's
+ * 16-byte plane, 32-bit word w holds coordinates 32w..32w+31, coordinate 32w+i in bit i, i.e.
+ * byte k holds coordinates 8k..8k+7. Sign words use the same order (bit = 1 for a non-negative
+ * projection). Key planes and key sign words are token-major: [planes][32 tokens][16 bytes],
+ * [32][16 bytes]. Value planes and value sign words are byte-lane-major: [planes][16 byte
+ * lanes][32 tokens], [16][32], byte (k, t) being byte k of token t's 16 bytes. Tiles of a
+ * (sequence, kv-head) are consecutive; (sequence, kv-head) pairs follow in row-major order.
+ * Capacity is rounded up to whole pairs of tiles (64 tokens).
  * FP4: [32][latent_dim/2] codes (channel 2k in the low nibble of byte k), [32][latent_dim/16]
  * E4M3 scales, [32][rope_dim] bf16 RoPE keys. */
 kvq_status kvq_cache_layout(const kvq_cache* c, int64_t* info, int32_t n_info);

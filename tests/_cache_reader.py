@@ -23,14 +23,22 @@ def side_fields(arena: np.ndarray, info, side: int, pair: int, n_tokens: int, m:
     qjl = off_norm > off_sketch  # a side without a sketch has an empty sketch block
     tb = _tiles(arena, region, pair, tiles, tile_bytes, n_tokens)
     nt = tb.shape[0]
-    planes = np.ascontiguousarray(tb[:, off_planes:off_planes + bits * TILE * 16]
-                                  .reshape(nt, bits, TILE, 16).transpose(0, 2, 1, 3))
+    # keys: token-major [bits][32 tokens][16 B]; values: byte-lane-major [bits][16][32 tokens]
+    raw = tb[:, off_planes:off_planes + bits * TILE * 16]
+    if side == 0:
+        planes = np.ascontiguousarray(raw.reshape(nt, bits, TILE, 16).transpose(0, 2, 1, 3))
+    else:
+        planes = np.ascontiguousarray(raw.reshape(nt, bits, 16, TILE).transpose(0, 3, 1, 2))
     planes = planes.reshape(nt * TILE, bits, 16).view(np.uint32)[:n_tokens]
     n16 = np.ascontiguousarray(tb[:, off_norm:off_norm + TILE * 2]).view(np.float16).reshape(-1)[:n_tokens]
     sketch, g16 = None, np.zeros(n_tokens)
     if qjl:
-        sketch = np.ascontiguousarray(tb[:, off_sketch:off_sketch + TILE * m // 8]) \
-            .reshape(nt * TILE, m // 8).view(np.uint32)[:n_tokens]
+        raw = tb[:, off_sketch:off_sketch + TILE * m // 8]
+        if side == 0:
+            sk = np.ascontiguousarray(raw).reshape(nt * TILE, m // 8)
+        else:
+            sk = np.ascontiguousarray(raw.reshape(nt, m // 8, TILE).transpose(0, 2, 1)).reshape(nt * TILE, m // 8)
+        sketch = sk.view(np.uint32)[:n_tokens]
         g16 = np.ascontiguousarray(tb[:, off_gamma:off_gamma + TILE * 2]).view(np.float16) \
             .reshape(-1)[:n_tokens].astype(np.float64)
     return planes, sketch, n16.astype(np.float64), g16

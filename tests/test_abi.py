@@ -57,9 +57,9 @@ def test_packed_bytes_match_oracle_sizes(lib, name):
 def test_cache_bytes_scales_with_capacity(lib):
     cfg = kvq.cfg_for_workload(WORKLOADS["llama8b"])
     a = kvq.kvq_cache_bytes(cfg, 16, 8192)
-    b = kvq.kvq_cache_bytes(cfg, 16, 8192 + 32)
-    assert b - a == 16 * 8 * 104 * 32
-    assert kvq.kvq_cache_bytes(cfg, 16, 8193) == b  # capacity rounds up to whole tiles
+    b = kvq.kvq_cache_bytes(cfg, 16, 8192 + 64)
+    assert b - a == 16 * 8 * 104 * 64
+    assert kvq.kvq_cache_bytes(cfg, 16, 8193) == b  # capacity rounds up to whole tile pairs
 
 
 def test_validation_errors(lib):

@@ -220,12 +220,12 @@ def test_fp4_full_context_sampled_heads():
 
 def test_capacity_overflow_writes_nothing():
     w = WORKLOADS["llama8b"]
-    data = generate(w, DEV, seqs=range(2), ctx=40)
-    cache, _, _ = new_cache(w, 2, 32)
+    data = generate(w, DEV, seqs=range(2), ctx=80)
+    cache, _, _ = new_cache(w, 2, 64)  # capacity is whole pairs of 32-token tiles: 64
     cache.quantize(data["k"][:, :, :20].contiguous(), data["v"][:, :, :20].contiguous())
     before = cache.arena.clone()
     with pytest.raises(kvq.KvqError) as e:
-        cache.quantize(data["k"][:, :, 20:40].contiguous(), data["v"][:, :, 20:40].contiguous())
+        cache.quantize(data["k"][:, :, 20:80].contiguous(), data["v"][:, :, 20:80].contiguous())
     assert e.value.status == 3
     torch.cuda.synchronize()
     assert torch.equal(before, cache.arena)
