@@ -34,6 +34,19 @@ from kvq_inputs import WORKLOADS, generate  # noqa: E402
 from kvq_inputs.workloads import rotation_and_sketch  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
+METRIC = "quantized-KV decode attention: KV tokens/s and HBM GB/s vs ~8 TB/s peak"
+UNIT = "KV tokens/s"
+
+
+def workload_config(w, world):
+    """The `config` object of both arms' JSON lines (identical for the same workload)."""
+    fp4 = w.k_mode == "fp4"
+    return {"workload": w.name, "batch": w.batch, "n_q_heads": w.n_q_heads,
+            "n_kv_heads": 1 if fp4 else w.n_kv_heads,
+            "head_dim": w.latent_dim if fp4 else w.head_dim, "ctx": w.ctx,
+            "codec": f"K {w.k_mode}{w.k_bits} / V {w.v_mode}{w.v_bits}",
+            "l2": "inputs larger than L2: cache replicas (> 2.5 x 126 MB in total) rotated per step",
+            "parallelism": f"replicas{world}"}
 
 
 def parse():
@@ -129,14 +142,26 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def _all_reduce(x: float, world: int, op) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
     dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
     t = torch.tensor([x], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Slowest rank's time: the job finishes when the last replica does."""
+    import torch.distributed as dist
+    return _all_reduce(x, world, dist.ReduceOp.MAX if world > 1 else None)
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    """Work done by all ranks together (each rank runs its own replica of the workload)."""
+    import torch.distributed as dist
+    return _all_reduce(x, world, dist.ReduceOp.SUM if world > 1 else None)
 
 
 # ------------------------------------------------------------------ oracle (CPU) timing
@@ -195,7 +220,7 @@ def blas_threads():
 
 def run_reference(args, world, rank):
     w = WORKLOADS[args.workload]
-    metric, unit = "quantized-KV decode attention: KV tokens/s", "KV tokens/s"
+    metric, unit = METRIC, UNIT
     if rank != 0:
         return
     if w.k_mode == "fp4":
@@ -214,7 +239,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name, "batch": w.batch, "ctx": w.ctx},
+            "data": "synthetic", "config": workload_config(w, world),
             "cpu_baseline": {"value": value, "unit": unit, "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -279,6 +304,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kv_tokens = 0
+    launches0 = kvq.kvq_kernel_launches()
     with ClockSampler(torch.cuda.current_device()) as clk:
         start.record(stream)
         for j in range(args.steps):
@@ -287,6 +313,7 @@ def run_ours(args, world, rank, local):
             kv_tokens += w.batch * (int(caches[i % replicas].lengths()[0]))
         end.record(stream)
         torch.cuda.synchronize()
+    launches = kvq.kvq_kernel_launches() - launches0
     barrier(world)
     torch.cuda.synchronize()
     elapsed_ms = start.elapsed_time(end)
@@ -294,7 +321,7 @@ def run_ours(args, world, rank, local):
     elapsed_ms = max_over_ranks(elapsed_ms, world)
     dec_ms = max_over_ranks(dec_ms, world)
     ms_per_step = elapsed_ms / args.steps
-    value = world * kv_tokens / (elapsed_ms / 1e3)
+    value = sum_over_ranks(kv_tokens, world) / (elapsed_ms / 1e3)
 
     # End to end: host (pinned) inputs copied in, result copied out, every step.
     host_news = [(a.cpu().pin_memory(), b.cpu().pin_memory()) for a, b in news[:args.steps]]
@@ -327,7 +354,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world)
     e2e_steps = max(1, n_e2e)
-    e2e_value = world * e2e_tokens / (e2e_ms / 1e3) if e2e_ms > 0 else None
+    e2e_tokens = sum_over_ranks(e2e_tokens, world)
+    e2e_value = e2e_tokens / (e2e_ms / 1e3) if e2e_ms > 0 else None
     h2d = host_news[0][0].numel() * host_news[0][0].element_size() * 2 + host_q.numel() * host_q.element_size()
     d2h = host_out.numel() * host_out.element_size()
 
@@ -336,16 +364,13 @@ def run_ours(args, world, rank, local):
     achieved = bytes_step / (dec_ms / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
     line = {
-        "metric": "quantized-KV decode attention: KV tokens/s and HBM GB/s vs ~8 TB/s peak",
-        "value": value, "unit": "KV tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC,
+        "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "n_q_heads": w.n_q_heads,
-                   "n_kv_heads": heads_kv, "head_dim": w.head_dim if w.k_mode != "fp4" else w.latent_dim,
-                   "ctx": w.ctx, "codec": f"K {w.k_mode}{w.k_bits} / V {w.v_mode}{w.v_bits}",
-                   "l2": f"{replicas} cache replicas x {bytes_prefix / 1e6:.1f} MB rotated per step (> 126 MB L2)",
-                   "parallelism": f"replicas{world}"},
+        "config": workload_config(w, world),
+        "l2_detail": f"{replicas} cache replicas x {bytes_prefix / 1e6:.1f} MB rotated per step",
         "hbm_gbs": achieved, "frac_of_8tbs": achieved / 8000.0,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
@@ -353,7 +378,7 @@ def run_ours(args, world, rank, local):
                      "bytes_per_launch": bytes_step, "ms_per_launch": dec_ms},
         "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": args.steps * 3,
+        "gpu_launches": launches,
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1 and w.k_mode != "fp4":

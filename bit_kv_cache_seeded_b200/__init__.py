@@ -32,7 +32,7 @@ DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "kvq_cache_init",
            "kvq_quantize", "kvq_workspace_bytes", "kvq_decode_attention", "kvq_cache_lengths",
            "kvq_cache_layout", "kvq_lloyd_max_table", "kvq_cache_destroy",
-           "kvq_debug_quantize_rotated", "kvq_decode_attention_static")
+           "kvq_debug_quantize_rotated", "kvq_decode_attention_static", "kvq_kernel_launches")
 
 
 class KvqError(RuntimeError):
@@ -76,6 +76,7 @@ def load() -> ctypes.CDLL:
         "kvq_cache_destroy": ([VP], None),
         "kvq_debug_quantize_rotated": ([VP, VP, I32, VP, VP, VP, VP], I32),
         "kvq_decode_attention_static": ([VP, VP, I32, VP, VP], I32),
+        "kvq_kernel_launches": ([], ctypes.c_uint64),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -215,6 +216,11 @@ def kvq_lloyd_max_table(bits: int):
 def kvq_cache_destroy(handle):
     if handle:
         load().kvq_cache_destroy(handle)
+
+
+def kvq_kernel_launches() -> int:
+    """Kernels the library has enqueued since it was loaded (all threads and devices)."""
+    return int(load().kvq_kernel_launches())
 
 
 def kvq_debug_quantize_rotated(handle, u: torch.Tensor, k_bits: int, qjl: bool, stream=None):

@@ -1,5 +1,6 @@
 // Host side of the kvq C ABI: validation, cache layout, tables, split planning, launches.
 // Every entry point validates before launching and reports failures as kvq_status codes.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -194,6 +195,18 @@ float default_scale(const kvq_cfg& cfg) {
 }
 
 }  // namespace
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+namespace kvq {
+cudaError_t launched() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+}  // namespace kvq
 
 extern "C" {
 
@@ -428,6 +441,8 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
   if (launch_reduce_lm(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }
+
+uint64_t kvq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens) {
   if (!c || !lens) return KVQ_ERR_INVALID_ARG;

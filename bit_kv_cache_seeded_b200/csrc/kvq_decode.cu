@@ -14,6 +14,7 @@
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
 
+#include "kvq_async.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -249,6 +250,9 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
 // One block per (sequence, kv-head): merge the split partials of the group's G query heads,
 // fold the value sketch back (o_r += S^T acc_z, with S staged in shared memory by cp.async while
 // the partials are merged), undo the rotation (out = D H o_r / sqrt(d)) and write out.
+// Thread i owns coordinate i during the merge and the S^T product; the loads of all heads and
+// two splits are issued together so the merge costs a few memory latencies, not one per split.
+// The final Walsh-Hadamard transform runs one warp per head with shuffles.
 template <int G>
 __global__ void __launch_bounds__(kHeadDim)
 reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
@@ -257,62 +261,93 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
   float* az = rs + (vq ? p.v.m * kHeadDim : 0);      // [G][d] merged sketch accumulators
   float* xs = az + G * kHeadDim;                     // [G][d] rotated-domain outputs
   const int hk = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+  const int lane = i & 31, warp = i >> 5;
   if (vq) {
-    for (int c = i; c < p.v.m * kHeadDim / 4; c += kHeadDim) {
-      const unsigned dst = (unsigned)__cvta_generic_to_shared(S_s + 4 * c);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(p.S + 4 * c));
+    for (int c = i; c < p.v.m * kHeadDim / 4; c += kHeadDim) cp_async16(S_s + 4 * c, p.S + 4 * c);
+    cp_async_commit();
+  }
+  // Launched as a programmatic dependent of the decode kernel: S is staged above while that
+  // grid finishes; its partials are read only after this wait.
+  grid_dep_wait();
+  const size_t hstride = (size_t)p.splits * p.part_stride;  // between heads of one row block
+  const float* part0 = p.part + ((size_t)b * p.Hq + hk * G) * hstride;
+  // Online merge over groups of 4 splits: every load of a group (all heads) is issued before
+  // any is used, so the merge costs one memory latency per 4 splits.
+  float M[G], L[G], o[G], oz[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) { M[h] = -INFINITY; L[h] = 0.f; o[h] = 0.f; oz[h] = 0.f; }
+  for (int s0 = 0; s0 < p.splits; s0 += 4) {
+    float mv[4][G], lv[4][G], ov[4][G], zv[4][G];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const bool in = s0 + k < p.splits;
+        const float* ps = part0 + h * hstride + (size_t)(in ? s0 + k : 0) * p.part_stride;
+        mv[k][h] = in ? __ldcg(ps) : -INFINITY;
+        lv[k][h] = in ? __ldcg(ps + 1) : 0.f;
+        ov[k][h] = in ? __ldcg(ps + 2 + i) : 0.f;
+        zv[k][h] = (in && vq) ? __ldcg(ps + 2 + kHeadDim + i) : 0.f;
+      }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float mn = fmaxf(fmaxf(M[h], fmaxf(mv[0][h], mv[1][h])), fmaxf(mv[2][h], mv[3][h]));
+      const float c = exp2_diff(M[h], mn);
+      L[h] *= c; o[h] *= c; oz[h] *= c;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float w = exp2_diff(mv[k][h], mn);
+        L[h] = fmaf(w, lv[k][h], L[h]);
+        o[h] = fmaf(w, ov[k][h], o[h]);
+        oz[h] = fmaf(w, zv[k][h], oz[h]);
+      }
+      M[h] = mn;
     }
-    asm volatile("cp.async.commit_group;\n" ::);
   }
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    const size_t row = (size_t)b * p.Hq + hk * G + h;
-    const float* part = p.part + row * p.splits * p.part_stride;
-    float M = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) M = fmaxf(M, part[(size_t)s * p.part_stride]);
-    float L = 0.f, o = 0.f, oz = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float* ps = part + (size_t)s * p.part_stride;
-      const float w = exp2_diff(ps[0], M);
-      L += w * ps[1];
-      o += w * ps[2 + i];
-      if (vq) oz += w * ps[2 + kHeadDim + i];
-    }
-    const float inv = (L > 0.f) ? 1.f / L : 0.f;
-    xs[h * kHeadDim + i] = o * inv;
-    az[h * kHeadDim + i] = oz * inv;
+    const float inv = (L[h] > 0.f) ? 1.f / L[h] : 0.f;
+    o[h] *= inv;
+    az[h * kHeadDim + i] = oz[h] * inv;
   }
-  if (vq) asm volatile("cp.async.wait_group 0;\n" ::);
-  __syncthreads();
   if (vq) {
-    float acc[G];
+    cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll 4
+    for (int j = 0; j < p.v.m; j += 4) {
+      const float s0 = S_s[j * kHeadDim + i], s1 = S_s[(j + 1) * kHeadDim + i];
+      const float s2 = S_s[(j + 2) * kHeadDim + i], s3 = S_s[(j + 3) * kHeadDim + i];
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < p.v.m; ++j) {
-      const float sv = S_s[j * kHeadDim + i];
-#pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = fmaf(sv, az[h * kHeadDim + j], acc[h]);
+      for (int h = 0; h < G; ++h) {
+        const float4 a = *reinterpret_cast<const float4*>(az + h * kHeadDim + j);
+        o[h] = fmaf(s0, a.x, fmaf(s1, a.y, fmaf(s2, a.z, fmaf(s3, a.w, o[h]))));
+      }
     }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < G; ++h) xs[h * kHeadDim + i] += acc[h];
   }
+#pragma unroll
+  for (int h = 0; h < G; ++h) xs[h * kHeadDim + i] = o[h];
   __syncthreads();
-  // out = D H o_r / sqrt(d): Walsh-Hadamard butterflies in shared memory, all heads at once
-  for (int hb = 1; hb < kHeadDim; hb <<= 1) {
-    float a[G], o2[G];
+  // out = D H o_r / sqrt(d): one warp per head, lane l holding coordinates 32k + l; butterflies
+  // over index bits 0..4 by shuffles, bits 5..6 in registers.
+  for (int h = warp; h < G; h += kHeadDim / 32) {
+    float u[4];
 #pragma unroll
-    for (int h = 0; h < G; ++h) { a[h] = xs[h * kHeadDim + i]; o2[h] = xs[h * kHeadDim + (i ^ hb)]; }
-    __syncthreads();
+    for (int k = 0; k < 4; ++k) u[k] = xs[h * kHeadDim + 32 * k + lane];
 #pragma unroll
-    for (int h = 0; h < G; ++h) xs[h * kHeadDim + i] = (i & hb) ? o2[h] - a[h] : a[h] + o2[h];
-    __syncthreads();
+    for (int bb = 0; bb < 5; ++bb) {
+      const bool upper = (lane >> bb) & 1;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float other = __shfl_xor_sync(0xffffffffu, u[k], 1 << bb);
+        u[k] = upper ? other - u[k] : u[k] + other;
+      }
+    }
+    const float a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
+    u[0] = a0 + a2; u[2] = a0 - a2; u[1] = a1 + a3; u[3] = a1 - a3;
+    float* dst = p.out + ((size_t)b * p.Hq + hk * G + h) * kHeadDim;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dst[32 * k + lane] = u[k] * (p.signs[32 * k + lane] * 0.08838834764831845f);
   }
-  const float sgn = p.signs[i] * 0.08838834764831845f;
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-    p.out[((size_t)b * p.Hq + hk * G + h) * kHeadDim + i] = xs[h * kHeadDim + i] * sgn;
 }
 
 template <int G>
@@ -322,7 +357,7 @@ cudaError_t dispatch_modes(const DecodeParams& p, dim3 grid, cudaStream_t s) {
 #define KVQ_CASE(KB, KQ, VB, VQ)                                              \
   if (kb == KB && kq == KQ && vb == VB && vq == VQ) {                         \
     decode_lm_simple<G, KB, KQ, VB, VQ><<<grid, kWarps * 32, 0, s>>>(p);      \
-    return cudaGetLastError();                                                \
+    return launched();                                                        \
   }
   KVQ_CASE(2, true, 2, true)
   KVQ_CASE(3, true, 3, false)
@@ -356,8 +391,19 @@ cudaError_t launch_reduce_g(const DecodeParams& p, cudaStream_t s) {
   const size_t smem = sizeof(float) * ((p.v.qjl ? (size_t)p.v.m * kHeadDim : 0) + 2 * G * kHeadDim);
   cudaError_t e = cudaFuncSetAttribute(reduce_lm<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  reduce_lm<G><<<dim3(p.Hkv, p.B), kHeadDim, smem, s>>>(p, p.v.qjl);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.Hkv, p.B);
+  cfg.blockDim = dim3(kHeadDim);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, reduce_lm<G>, p, (int)p.v.qjl);
+  if (e != cudaSuccess) return e;
+  return launched();
 }
 
 cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s) {

@@ -32,6 +32,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "kvq_async.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -43,7 +44,10 @@ constexpr int kCtaTok = 64;
 constexpr int kStagesM = 3;
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
 constexpr float kSqrtHalfPi = 1.2533141373155003f;  // sqrt(pi/2)
-constexpr int kQRange = 8191;                        // query term quantised to [-8191, 8191]
+constexpr int kQRange = 32639;                       // query term quantised to [-32639, 32639]
+constexpr int kLgStride = kChunkMax + 8;             // logits row stride (floats): rows on distinct banks
+constexpr int kPdStride = 96;                        // weight-digit row stride (bytes): 64 tokens + pad
+constexpr int kNormBlock = 256;                      // staged value norms / gammas of two cache tiles
 constexpr float kWRange = 2097152.f;                 // weights quantised below 2^21
 
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -61,13 +65,11 @@ __device__ __forceinline__ uint32_t bit_to_s8(uint32_t w) {
   return (P == 7) ? (w & 0x80808080u) : ((w * (1u << (7 - P))) & 0x80808080u);
 }
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 __device__ __forceinline__ float load_q(const void* base, size_t i, int bf16) {
   if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
@@ -109,26 +111,30 @@ struct MmaCfg {
 // Prep kernel, once per (sequence, kv-head): the logit-phase B operand.
 //   q~ = H D q * scale*log2(e)/d (rotated query),  s~ = sqrt(pi/2)/m * S q~ (sketched query)
 //   centroid planes: v = 2 a_P q~_j;  sketch plane: v = 2 s~_j
-//   q_int = rint(v * 8191 / vmax_h) (vmax over the centroid planes, separately for the sketch),
-//   digits hi = floor((q_int + 64) / 128), lo = q_int - 128 hi, both in [-64, 64).
+//   q_int = rint(v * 32639 / vmax_h) (vmax over the centroid planes, separately for the sketch),
+//   digits hi = floor((q_int + 128) / 256) in [-127, 127], lo = q_int - 256 hi in [-128, 128):
+//   two full int8 digits, about 16 bits of the query term.
 // Layout per pair: [KP][G][2 digits][128 fragment-ordered coordinates] bytes, then [G][4] f32:
-// (s, C, sz, Cz) with s = vmax / (8191 * -128) (the one-hot bytes are -128), C = -(sum_P a_P)
+// (s, C, sz, Cz) with s = vmax / (32639 * -128) (the one-hot bytes are -128), C = -(sum_P a_P)
 // sum_j q~_j and Cz = -sum_j s~_j. Fragment order of coordinate j: (j%8)*16 + (j/32)*4 + (j%32)/8.
 // ------------------------------------------------------------------------------------------
 template <int G, int KB, bool KQ>
 __global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constant__ DecodeParams p) {
   constexpr int KP = Walsh<KB>::P + (KQ ? 1 : 0);
   constexpr int KWP = Walsh<KB>::P;
-  __shared__ float qf[G][kHeadDim];
-  __shared__ float sf[G][kHeadDim];
+  __shared__ __align__(16) float qf[G][kHeadDim];
+  __shared__ __align__(16) float sf[G][kHeadDim];
   __shared__ float hc[G][4];
+  __shared__ float qscale[G][2];                 // 32639 / vmax: centroid planes, sketch
   extern __shared__ __align__(16) float st_s[];  // [128][m] transposed sketch matrix
   const int hk = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned char* out = p.qprep + ((size_t)b * p.Hkv + hk) * p.qprep_stride;
-  if (KQ)
-    for (int c = tid; c < kHeadDim * kHeadDim / 4; c += kThreadsM)
-      reinterpret_cast<float4*>(st_s)[c] = __ldg(reinterpret_cast<const float4*>(p.St) + c);
+  if (KQ) {  // staged while the queries are rotated
+    for (int c = tid; c < kHeadDim * kHeadDim / 4; c += kThreadsM) cp_async16(st_s + 4 * c, p.St + 4 * c);
+    cp_async_commit();
+  }
+  grid_dep_launch();  // the decode kernel may be scheduled now; it waits before reading this output
   const float qcoef = kInvSqrtD * p.logit_scale * kInvSqrtD;
   for (int h = warp; h < G; h += kWarpsM) {
     float u[4];
@@ -150,6 +156,7 @@ __global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constan
     qf[h][32 + lane] = (a1 + a3) * qcoef;
     qf[h][96 + lane] = (a1 - a3) * qcoef;
   }
+  if (KQ) cp_async_wait<0>();
   __syncthreads();
   if (KQ) {
     const float kappa = kSqrtHalfPi / (float)p.k.m;
@@ -157,11 +164,15 @@ __global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constan
     float acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < kHeadDim; ++i) {
-      const float sv = st_s[i * kHeadDim + j];
+#pragma unroll 4
+    for (int i = 0; i < kHeadDim; i += 4) {
+      const float s0 = st_s[i * kHeadDim + j], s1 = st_s[(i + 1) * kHeadDim + j];
+      const float s2 = st_s[(i + 2) * kHeadDim + j], s3 = st_s[(i + 3) * kHeadDim + j];
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = fmaf(sv, qf[h][i], acc[h]);
+      for (int h = 0; h < G; ++h) {
+        const float4 qv = *reinterpret_cast<const float4*>(&qf[h][i]);
+        acc[h] = fmaf(s3, qv.w, fmaf(s2, qv.z, fmaf(s1, qv.y, fmaf(s0, qv.x, acc[h]))));
+      }
     }
 #pragma unroll
     for (int h = 0; h < G; ++h) sf[h][j] = acc[h] * kappa;
@@ -169,27 +180,41 @@ __global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constan
   }
   float ka[4];
   walsh_coeffs(KB, p.k.cent, ka);
-  if (tid < 2 * G) {
-    const int h = tid >> 1, which = tid & 1;  // 0: centroid planes, 1: sketch plane
+  for (int task = warp; task < 2 * G; task += kWarpsM) {  // (head, 0: centroid planes / 1: sketch)
+    const int h = task >> 1, which = task & 1;
     float mx = 0.f, sum = 0.f;
-    for (int j = 0; j < kHeadDim; ++j) {
-      const float v = which ? sf[h][j] : qf[h][j];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float v = which ? sf[h][32 * k + lane] : qf[h][32 * k + lane];
       mx = fmaxf(mx, fabsf(v));
       sum += v;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
     float asum = 0.f, amax = 0.f;
+#pragma unroll
     for (int P = 0; P < KWP; ++P) { asum += ka[P]; amax = fmaxf(amax, fabsf(ka[P])); }
     mx *= which ? 2.f : 2.f * amax;  // largest |v| over the planes
-    hc[h][2 * which] = mx > 0.f ? mx : 1.f;
-    hc[h][2 * which + 1] = which ? -sum : -asum * sum;
+    if (lane == 0) {
+      hc[h][2 * which] = mx > 0.f ? mx : 1.f;
+      hc[h][2 * which + 1] = which ? -sum : -asum * sum;
+      qscale[h][which] = (float)kQRange / (mx > 0.f ? mx : 1.f);
+    }
   }
   __syncthreads();
   for (int idx = tid; idx < KP * G * kHeadDim; idx += kThreadsM) {
     const int P = idx / (G * kHeadDim), h = (idx / kHeadDim) % G, j = idx % kHeadDim;
     const bool sk = KQ && P == KP - 1;
-    const float v = sk ? 2.f * sf[h][j] : 2.f * ka[min(P, 3)] * qf[h][j];
-    const int q = __float2int_rn(v * ((float)kQRange / hc[h][sk ? 2 : 0]));
-    const int hi = (q + 64) >> 7, lo = q - 128 * hi;
+    float kaP = ka[0];
+#pragma unroll
+    for (int r = 1; r < 4; ++r)
+      if (P == r) kaP = ka[r];
+    const float v = sk ? 2.f * sf[h][j] : 2.f * kaP * qf[h][j];
+    const int q = __float2int_rn(v * qscale[h][sk ? 1 : 0]);
+    const int hi = (q + 128) >> 8, lo = q - 256 * hi;
     const int pj = (j % 8) * 16 + (j / 32) * 4 + (j % 32) / 8;
     out[((P * G + h) * 2 + 0) * 128 + pj] = (unsigned char)(signed char)hi;
     out[((P * G + h) * 2 + 1) * 128 + pj] = (unsigned char)(signed char)lo;
@@ -217,11 +242,11 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   static_assert(NTASK <= kThreadsM, "one weight task per thread");
   extern __shared__ __align__(16) unsigned char smem[];
   const int ktb = p.k.tile_bytes, vtb = p.v.tile_bytes;
-  const int stage_bytes = 2 * max(ktb, vtb);
-  unsigned char* stages = smem;                                            // [kStagesM][2 tiles]
-  float* lgs = reinterpret_cast<float*>(stages + kStagesM * stage_bytes);  // [G][kChunkMax] logits
-  unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * kChunkMax);  // [NKIND][VNCOL][64]
-  float* red = reinterpret_cast<float*>(pdig + NKIND * VNCOL * kCtaTok);       // reductions
+  const int stage_bytes = max(2 * ktb + kNormBlock, 2 * vtb);
+  unsigned char* stages = smem;                                            // [kStagesM][2 tiles (+ norms)]
+  float* lgs = reinterpret_cast<float*>(stages + kStagesM * stage_bytes);  // [G][kLgStride] logits
+  unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * kLgStride);  // [NKIND][VNCOL][kPdStride]
+  float* red = reinterpret_cast<float*>(pdig + NKIND * VNCOL * kPdStride);     // reductions
 
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -243,6 +268,13 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       const unsigned char* src = (pass ? vbase : kbase) + (size_t)tile0 * tb;
       unsigned char* dst = stages + slot * stage_bytes;
       for (int c = tid; c < ntiles * tb / 16; c += kThreadsM) cp_async16(dst + 16 * c, src + 16 * c);
+      if (!pass && tid < ntiles * 8) {  // value norms (4 x 16 B) and gammas (4 x 16 B) per tile
+        const int tile = tid >> 3, part = tid & 7;
+        if (part < 4 || VQ) {
+          const unsigned char* vs = vbase + (size_t)(tile0 + tile) * vtb + (part < 4 ? p.v.off_norm : p.v.off_gamma) + 16 * (part & 3);
+          cp_async16(dst + 2 * ktb + tile * 128 + 16 * part, vs);
+        }
+      }
     }
     cp_async_commit();
   };
@@ -250,6 +282,9 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   for (int s = 0; s < kStagesM - 1; ++s) load_stage(0, s, s);
 
   // logit-phase B fragments (query digits) and head constants from the prep area
+  // Launched as a programmatic dependent of the prep kernel: the cache tiles staged above were
+  // complete before prep started; the prep output is read only after this wait.
+  grid_dep_wait();
   const unsigned char* prep = p.qprep + pair * p.qprep_stride;
   uint32_t qb[KP][4][KNT][2];
 #pragma unroll
@@ -284,7 +319,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   float mrow[KNT];  // max over this thread's logits of head 4 nt + t
 #pragma unroll
   for (int nt = 0; nt < KNT; ++nt) mrow[nt] = -INFINITY;
-  float wmax = 0.f;  // largest value weight (times max(1, sketch weight)) seen by this thread
+  float wmax = 0.f, wmaxz = 0.f;  // largest value weight of each kind seen by this thread
   const int tl = warp * 16;
   for (int it = 0; it < n_iter; ++it) {
     load_stage(0, it + kStagesM - 1, (it + kStagesM - 1) % kStagesM);
@@ -296,11 +331,13 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     {
       const unsigned char* ktile = kt + (tl / kTile) * ktb;
       const int s0 = (tl % kTile) + g, s1 = s0 + 8;
-      int acc[KNT][4], accz[KNT][4];
+      int acc[4][KNT][4], accz[2][KNT][4];  // independent chains: position pair m (z: m & 1)
 #pragma unroll
-      for (int nt = 0; nt < KNT; ++nt)
+      for (int m = 0; m < 4; ++m)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) { acc[nt][c] = 0; accz[nt][c] = 0; }
+        for (int nt = 0; nt < KNT; ++nt)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) { acc[m][nt][c] = 0; if (m < 2) accz[m][nt][c] = 0; }
       uint32_t w0[3] = {0u, 0u, 0u}, w1[3] = {0u, 0u, 0u};
       const unsigned char* kp = ktile + p.k.off_planes + t * 4;
 #pragma unroll
@@ -330,8 +367,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
           }
 #pragma unroll
           for (int nt = 0; nt < KNT; ++nt) {
-            if (sk) mma_s8(accz[nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
-            else mma_s8(acc[nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+            if (sk) mma_s8(accz[m & 1][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+            else mma_s8(acc[m][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
           }
         }
       }
@@ -346,27 +383,32 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
       for (int nt = 0; nt < KNT; ++nt) {
         const int h = 4 * nt + t;
-        float l0 = fmaf(hs[nt], (float)(acc[nt][0] * 128 + acc[nt][1]), hc[nt]);
-        float l1 = fmaf(hs[nt], (float)(acc[nt][2] * 128 + acc[nt][3]), hc[nt]);
+        int c[4], cz[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          c[e] = (acc[0][nt][e] + acc[1][nt][e]) + (acc[2][nt][e] + acc[3][nt][e]);
+          cz[e] = accz[0][nt][e] + accz[1][nt][e];
+        }
+        float l0 = fmaf(hs[nt], fmaf((float)c[0], 256.f, (float)c[1]), hc[nt]);
+        float l1 = fmaf(hs[nt], fmaf((float)c[2], 256.f, (float)c[3]), hc[nt]);
         if (KQ) {
-          l0 = fmaf(gk0, fmaf(hsz[nt], (float)(accz[nt][0] * 128 + accz[nt][1]), hcz[nt]), l0);
-          l1 = fmaf(gk1, fmaf(hsz[nt], (float)(accz[nt][2] * 128 + accz[nt][3]), hcz[nt]), l1);
+          l0 = fmaf(gk0, fmaf(hsz[nt], fmaf((float)cz[0], 256.f, (float)cz[1]), hcz[nt]), l0);
+          l1 = fmaf(gk1, fmaf(hsz[nt], fmaf((float)cz[2], 256.f, (float)cz[3]), hcz[nt]), l1);
         }
         const float lg0 = v0 ? nk0 * l0 : -INFINITY, lg1 = v1 ? nk1 * l1 : -INFINITY;
         if (h < G) {
-          lgs[h * kChunkMax + tok0 + tl + g] = lg0;
-          lgs[h * kChunkMax + tok0 + tl + g + 8] = lg1;
+          lgs[h * kLgStride + tok0 + tl + g] = lg0;
+          lgs[h * kLgStride + tok0 + tl + g + 8] = lg1;
         }
         mrow[nt] = fmaxf(mrow[nt], fmaxf(lg0, lg1));
       }
     }
     // largest value weight: tokens of this iteration, one per thread of warps 0 and 1
-    if (tid < count) {
-      const size_t tok = (size_t)t_begin + tok0 + tid;
-      const unsigned char* vtile = vbase + (tok / kTile) * vtb;
-      float w = __half2float(*reinterpret_cast<const __half*>(vtile + p.v.off_norm + (tok % kTile) * 2)) * kInvSqrtD;
-      if (VQ) w *= fmaxf(1.f, __half2float(*reinterpret_cast<const __half*>(vtile + p.v.off_gamma + (tok % kTile) * 2)) * vkappa);
+    if (tid < count) {  // staged value norms: [tile][64 B norms | 64 B gammas]
+      const unsigned char* nb = kt + 2 * ktb + (tid / kTile) * 128 + (tid % kTile) * 2;
+      const float w = __half2float(*reinterpret_cast<const __half*>(nb)) * kInvSqrtD;
       wmax = fmaxf(wmax, w);
+      if (VQ) wmaxz = fmaxf(wmaxz, w * (__half2float(*reinterpret_cast<const __half*>(nb + 64)) * vkappa));
     }
     __syncthreads();  // the next iteration refills a stage buffer
   }
@@ -376,7 +418,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 
   // chunk maxima per head, and the weight scale
   float* hmax = red;                 // [kWarpsM][G]
-  float* wred = red + kWarpsM * G;   // [kWarpsM]
+  float* wred = red + kWarpsM * G;   // [2][kWarpsM]: both kinds' weight maxima
 #pragma unroll
   for (int nt = 0; nt < KNT; ++nt) {
     float mx = mrow[nt];
@@ -386,24 +428,30 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     if (g == 0 && 4 * nt + t < G) hmax[warp * G + 4 * nt + t] = mx;
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
-  if (lane == 0) wred[warp] = wmax;
+  for (int o = 16; o > 0; o >>= 1) {
+    wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+    wmaxz = fmaxf(wmaxz, __shfl_xor_sync(0xffffffffu, wmaxz, o));
+  }
+  if (lane == 0) { wred[warp] = wmax; wred[kWarpsM + warp] = wmaxz; }
   __syncthreads();
-  float wm = 0.f;
+  float wm = 0.f, wmz = 0.f;
 #pragma unroll
-  for (int w = 0; w < kWarpsM; ++w) wm = fmaxf(wm, wred[w]);
-  // integer weights below 2^21 (3 x 7-bit digits); a power-of-two scale keeps the digits exact
+  for (int w = 0; w < kWarpsM; ++w) { wm = fmaxf(wm, wred[w]); wmz = fmaxf(wmz, wred[kWarpsM + w]); }
+  // integer weights below 2^21 (3 x 7-bit digits), each kind scaled to its own range by a power
+  // of two (exact digits; the sketch weights are ~sqrt(pi/2) gamma / m of the centroid ones)
   const float wsc = wm > 0.f ? exp2f(floorf(log2f(kWRange / wm)) - 1.f) : 1.f;
+  const float wscz = wmz > 0.f ? exp2f(floorf(log2f(kWRange / wmz)) - 1.f) : 1.f;
 
   // ================= pass 2: weights -> digits, value contractions
   const bool has_task = tid < NTASK;
   const int task_kind = tid / (G * 16), task_h = (tid / 16) % G, task_q = tid % 16;
+  const float task_sc = (VQ && task_kind == 1) ? wscz : wsc;
   float task_m = -INFINITY;
 #pragma unroll
   for (int w = 0; w < kWarpsM; ++w) task_m = fmaxf(task_m, hmax[w * G + task_h]);
   float task_l = 0.f;     // sum of p over this task's tokens
   long long task_wl = 0;  // sum of the quantised weights (exact)
-  for (int idx = tid; idx < NKIND * VNCOL * kCtaTok / 4; idx += kThreadsM)
+  for (int idx = tid; idx < NKIND * VNCOL * kPdStride / 4; idx += kThreadsM)
     reinterpret_cast<uint32_t*>(pdig)[idx] = 0u;  // the pad digit and absent heads stay zero
 
   int vacc[VP][2][VNT][4];
@@ -428,7 +476,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     // weight task: 4 consecutive tokens of one head, one kind
     if (has_task) {
       const int T = 4 * task_q;
-      const float4 l4 = *reinterpret_cast<const float4*>(lgs + task_h * kChunkMax + tok0 + T);
+      const float4 l4 = *reinterpret_cast<const float4*>(lgs + task_h * kLgStride + tok0 + T);
       const unsigned char* vtile = vt + (T / kTile) * vtb;
       const uint2 nraw = *reinterpret_cast<const uint2*>(vtile + p.v.off_norm + (T % kTile) * 2);
       const float2 n01 = __half22float2(*reinterpret_cast<const __half2*>(&nraw.x));
@@ -447,9 +495,9 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const bool ok = T + e < count;
-        const float pe = ok ? exp2f(lv[e] - task_m) : 0.f;
+        const float pe = ok ? ex2(lv[e] - task_m) : 0.f;
         psum += pe;
-        const int q = ok ? __float2int_rn(pe * wv[e] * wsc) : 0;  // < 2^21
+        const int q = ok ? __float2int_rn(pe * wv[e] * task_sc) : 0;  // < 2^21
         qsum += q;
         d0 |= (uint32_t)(q >> 14) << (8 * e);
         d1 |= (uint32_t)((q >> 7) & 127) << (8 * e);
@@ -457,10 +505,10 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       }
       task_l += psum;
       task_wl += qsum;
-      unsigned char* col = pdig + (size_t)(task_kind * VNCOL + 4 * task_h) * kCtaTok + T;
+      unsigned char* col = pdig + (size_t)(task_kind * VNCOL + 4 * task_h) * kPdStride + T;
       *reinterpret_cast<uint32_t*>(col) = d0;
-      *reinterpret_cast<uint32_t*>(col + kCtaTok) = d1;
-      *reinterpret_cast<uint32_t*>(col + 2 * kCtaTok) = d2;
+      *reinterpret_cast<uint32_t*>(col + kPdStride) = d1;
+      *reinterpret_cast<uint32_t*>(col + 2 * kPdStride) = d2;
     }
     __syncthreads();
 
@@ -469,26 +517,29 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     for (int s = 0; s < 2; ++s) {
       if (s * kTile >= count) break;
       const unsigned char* vtile = vt + s * vtb;
+      // K order within a 32-token step: K-index 4t + i <-> token 8t + i, 16 + 4t + i <-> 8t + 4 + i,
+      // so a thread's two 4-token groups are one 64-bit load (bits and digits alike)
       uint32_t bm[VNT][2], bz[VNT][2];
 #pragma unroll
       for (int nt = 0; nt < VNT; ++nt) {
-        const unsigned char* col = pdig + (size_t)(nt * 8 + g) * kCtaTok + s * kTile + 4 * t;
-        bm[nt][0] = *reinterpret_cast<const uint32_t*>(col);
-        bm[nt][1] = *reinterpret_cast<const uint32_t*>(col + 16);
+        const unsigned char* col = pdig + (size_t)(nt * 8 + g) * kPdStride + s * kTile + 8 * t;
+        const uint2 v = *reinterpret_cast<const uint2*>(col);
+        bm[nt][0] = v.x;
+        bm[nt][1] = v.y;
         if (VQ) {
-          const unsigned char* colz = col + (size_t)VNCOL * kCtaTok;
-          bz[nt][0] = *reinterpret_cast<const uint32_t*>(colz);
-          bz[nt][1] = *reinterpret_cast<const uint32_t*>(colz + 16);
+          const uint2 vz = *reinterpret_cast<const uint2*>(col + (size_t)VNCOL * kPdStride);
+          bz[nt][0] = vz.x;
+          bz[nt][1] = vz.y;
         }
       }
       uint32_t xv[3][4];
 #pragma unroll
       for (int pp = 0; pp < VB; ++pp) {
-        const unsigned char* pl = vtile + p.v.off_planes + pp * (kTile * 16) + 4 * t;
-        xv[pp][0] = *reinterpret_cast<const uint32_t*>(pl + g * kTile);
-        xv[pp][1] = *reinterpret_cast<const uint32_t*>(pl + (g + 8) * kTile);
-        xv[pp][2] = *reinterpret_cast<const uint32_t*>(pl + g * kTile + 16);
-        xv[pp][3] = *reinterpret_cast<const uint32_t*>(pl + (g + 8) * kTile + 16);
+        const unsigned char* pl = vtile + p.v.off_planes + pp * (kTile * 16) + 8 * t;
+        const uint2 r0 = *reinterpret_cast<const uint2*>(pl + g * kTile);
+        const uint2 r1 = *reinterpret_cast<const uint2*>(pl + (g + 8) * kTile);
+        xv[pp][0] = r0.x; xv[pp][2] = r0.y;
+        xv[pp][1] = r1.x; xv[pp][3] = r1.y;
       }
 #pragma unroll
       for (int P = 0; P < VP; ++P) {
@@ -497,8 +548,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           if (sk) {
-            const unsigned char* pl = vtile + p.v.off_sketch + 4 * t;
-            x[r] = *reinterpret_cast<const uint32_t*>(pl + ((r & 1) ? g + 8 : g) * kTile + ((r & 2) ? 16 : 0));
+            const unsigned char* pl = vtile + p.v.off_sketch + 8 * t;
+            x[r] = *reinterpret_cast<const uint32_t*>(pl + ((r & 1) ? g + 8 : g) * kTile + ((r & 2) ? 4 : 0));
           } else if (VB == 3 && P == 3) {
             x[r] = xv[0][r] ^ xv[1][r] ^ xv[2][r];
           } else {
@@ -518,6 +569,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     __syncthreads();  // the next iteration refills a stage buffer and the digits
   }
 
+  grid_dep_launch();  // let the split reduce be scheduled; it waits for this grid to finish
   // ================= finish: per-head sums of p and of the weights, then this warp's rows
   cp_async_wait<0>();
   __syncthreads();
@@ -540,11 +592,12 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   float vasum = 0.f;
 #pragma unroll
   for (int P = 0; P < VWP; ++P) vasum += va[P];
-  const float inv_w = 1.f / wsc;
+  const float inv_w = 1.f / wsc, inv_wz = 1.f / wscz;
 #pragma unroll
   for (int pi = 0; pi < 2; ++pi) {
     const int pos = 2 * warp + pi;
-    const float rowinv = (pos == 7 ? -1.f / 128.f : 1.f / (float)(1 << pos)) * inv_w;  // row value 2^p or -128
+    const float rowpos = pos == 7 ? -1.f / 128.f : 1.f / (float)(1 << pos);  // row value 2^p or -128
+    const float rowinv = rowpos * inv_w, rowinvz = rowpos * inv_wz;
 #pragma unroll
     for (int nt = 0; nt < VNT; ++nt) {
       const int h = 2 * nt + t / 2;
@@ -558,7 +611,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
         r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
         const bool sk = VQ && P == VP - 1;
-        if (sk) { z0 = 2.f * r0 * rowinv; z1 = 2.f * r1 * rowinv; }
+        if (sk) { z0 = 2.f * r0 * rowinvz; z1 = 2.f * r1 * rowinvz; }
         else { o0 = fmaf(2.f * va[min(P, 3)], r0 * rowinv, o0); o1 = fmaf(2.f * va[min(P, 3)], r1 * rowinv, o1); }
       }
       if (h < G) {
@@ -569,7 +622,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
           dst[2 + j0] = o0 - vasum * Wt;
           dst[2 + j1] = o1 - vasum * Wt;
         } else if (VQ) {
-          const float Wz = hsum[2 * G + h] * inv_w;
+          const float Wz = hsum[2 * G + h] * inv_wz;
           dst[2 + kHeadDim + j0] = z0 - Wz;
           dst[2 + kHeadDim + j1] = z1 - Wz;
         }
@@ -593,10 +646,10 @@ template <int G, int KB, bool KQ, int VB, bool VQ>
 size_t mma_smem_bytes(const DecodeParams& p) {
   using C = MmaCfg<G, KB, KQ, VB, VQ>;
   constexpr int NKIND = VQ ? 2 : 1;
-  size_t s = (size_t)kStagesM * 2 * std::max(p.k.tile_bytes, p.v.tile_bytes);
-  s += sizeof(float) * (size_t)G * kChunkMax;
-  s += (size_t)NKIND * C::VNCOL * kCtaTok;
-  s += sizeof(float) * (kWarpsM * G + kWarpsM);
+  size_t s = (size_t)kStagesM * std::max(2 * p.k.tile_bytes + kNormBlock, 2 * p.v.tile_bytes);
+  s += sizeof(float) * (size_t)G * kLgStride;
+  s += (size_t)NKIND * C::VNCOL * kPdStride;
+  s += sizeof(float) * (kWarpsM * G + 2 * kWarpsM);
   return (s + 15) / 16 * 16;
 }
 
@@ -607,14 +660,25 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s) {
                                        (int)prep_smem);
   if (e != cudaSuccess) return e;
   decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv, p.B), kThreadsM, prep_smem, s>>>(p);
-  e = cudaGetLastError();
+  e = launched();
   if (e != cudaSuccess) return e;
   const size_t smem = mma_smem_bytes<G, KB, KQ, VB, VQ>(p);
   auto kern = decode_lm_mma<G, KB, KQ, VB, VQ>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(p.splits, p.Hkv, p.B), kThreadsM, smem, s>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.splits, p.Hkv, p.B);
+  cfg.blockDim = dim3(kThreadsM);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e != cudaSuccess) return e;
+  return launched();
 }
 
 template <int G>

@@ -96,7 +96,11 @@ struct MlaParams {
   float logit_scale;      // softmax_scale * log2(e)
 };
 
-// Launchers (kvq_quantize.cu, kvq_decode.cu, kvq_mla.cu). Return cudaGetLastError().
+// Reads cudaGetLastError() right after a kernel launch and, when it is cudaSuccess, adds one to
+// the library's launch counter (kvq_kernel_launches).
+cudaError_t launched();
+
+// Launchers (kvq_quantize.cu, kvq_decode.cu, kvq_mla.cu). Return launched().
 cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s);
 cudaError_t launch_quantize_fp4(const QuantizeParams& p, cudaStream_t s);
 cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s);

@@ -164,7 +164,7 @@ cudaError_t launch_hpw(const MlaParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(decode_mla_simple<HPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   decode_mla_simple<HPW><<<dim3(p.splits, p.B), kMlaThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launched();
 }
 
 }  // namespace
@@ -183,7 +183,7 @@ cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s) {
 
 cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s) {
   reduce_mla<<<p.B * p.Hq, kLat, 0, s>>>(p);
-  return cudaGetLastError();
+  return launched();
 }
 
 }  // namespace kvq

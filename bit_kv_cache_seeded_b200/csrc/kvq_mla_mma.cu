@@ -346,7 +346,7 @@ cudaError_t launch_decode_mla_mma(const MlaParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(decode_mla_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   decode_mla_mma<<<dim3(p.splits, p.B), kThreadsL, smem, s>>>(p);
-  return cudaGetLastError();
+  return launched();
 }
 
 }  // namespace kvq

@@ -21,6 +21,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include "kvq_async.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -37,25 +38,44 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-constexpr int kQuantWarps = 8;
+constexpr int kQuantWarps = 8;  // FP4 kernel: one token per warp
+constexpr int kLmWarps = 4;     // LM kernel: warps per block
 
-__global__ void __launch_bounds__(kQuantWarps * 32)
+// LM quantize. Sides with a sketch: the block's 4 warps share one vector; each redoes steps 1-5
+// (cheap, and it keeps every warp independent), then warp w forms sketch word w, i.e. the 32
+// projections j = 32w + lane, from its own 16 KB column slice of S^T staged in shared memory.
+// Sides without a sketch: one vector per warp.
+__global__ void __launch_bounds__(kLmWarps * 32)
 quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
-  __shared__ float rho_s[kQuantWarps][kHeadDim];
-  extern __shared__ __align__(16) float st_s[];  // [d][m] transposed sketch matrix (sketch sides)
+  __shared__ float rho_s[kLmWarps][kHeadDim];
+  extern __shared__ __align__(16) float st_s[];  // sketch sides: [warp][d][32] columns 32w.. of S^T
   const int side = blockIdx.y;
   const SideLayout& L = p.side[side];
-  if (L.qjl) {
-    for (int c = threadIdx.x; c < kHeadDim * L.m / 4; c += blockDim.x)
-      reinterpret_cast<float4*>(st_s)[c] = __ldg(reinterpret_cast<const float4*>(p.St) + c);
-    __syncthreads();
-  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nthr = L.bits ? (1 << L.bits) - 1 : 0;
+  const bool coop = L.qjl;
   const long total = (long)p.n_seq * p.heads * p.n_new;
+  const long first = coop ? (long)blockIdx.x : (long)blockIdx.x * kLmWarps + warp;
+  const long stride = coop ? (long)gridDim.x : (long)gridDim.x * kLmWarps;
+  float* stw = st_s + warp * kHeadDim * 32;  // stw[i * 32 + l] = S^T[i][32 warp + l] = S[32 warp + l][i]
+  // The slice is staged asynchronously while the first vector's elements are fetched.
+  if (coop && first < total) {
+    for (int c = lane; c < kHeadDim * 8; c += 32) {  // row i = c / 8, 16-byte chunk c % 8 of its 32 floats
+      const int i = c >> 3, ch = c & 7;
+      cp_async16(stw + i * 32 + ch * 4, p.St + (size_t)i * L.m + 32 * warp + ch * 4);
+    }
+    cp_async_commit();
+  }
+  float u_first[4] = {0.f, 0.f, 0.f, 0.f};
+  if (first < total)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u_first[k] = load_elem(p.src[side], (size_t)first * kHeadDim + 32 * k + lane, p.bf16);
+  if (coop) {
+    cp_async_wait<0>();
+    __syncwarp();
+  }
 
-  for (long vec = (long)blockIdx.x * kQuantWarps + warp; vec < total;
-       vec += (long)gridDim.x * kQuantWarps) {
+  for (long vec = first; vec < total; vec += stride) {
     const int t = (int)(vec % p.n_new);
     const int h = (int)((vec / p.n_new) % p.heads);
     const int s = (int)(vec / ((long)p.n_new * p.heads));
@@ -63,7 +83,7 @@ quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
 
     float u[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) u[k] = load_elem(p.src[side], base + 32 * k + lane, p.bf16);
+    for (int k = 0; k < 4; ++k) u[k] = (vec == first) ? u_first[k] : load_elem(p.src[side], base + 32 * k + lane, p.bf16);
 
     float n = 0.f;
     if (!p.skip_rotation) {
@@ -101,34 +121,32 @@ quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
 #pragma unroll
       for (int k = 0; k < 4; ++k)
         planes[pp][k] = (pp < L.bits) ? __ballot_sync(0xffffffffu, (code[k] >> pp) & 1) : 0u;
+    // lane pp < bits stores plane pp (selected without indexing registers by lane)
+    uint4 mine = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int pp = 0; pp < kMaxBits; ++pp)
+      if (lane == pp) mine = make_uint4(planes[pp][0], planes[pp][1], planes[pp][2], planes[pp][3]);
 
-    uint32_t zw[4] = {0u, 0u, 0u, 0u};
+    uint32_t zword = 0u;  // sketch word `warp` (coop sides)
     float gamma = 0.f;
-    if (L.qjl) {
+    if (coop) {
       gamma = sqrtf(warp_sum(rho[0] * rho[0] + rho[1] * rho[1] + rho[2] * rho[2] + rho[3] * rho[3]));
 #pragma unroll
       for (int k = 0; k < 4; ++k) rho_s[warp][32 * k + lane] = rho[k];
       __syncwarp();
-      float proj[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-      for (int i = 0; i < kHeadDim; ++i) {
-        const float r = rho_s[warp][i];
-        const float* row = st_s + i * L.m;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) proj[k] = fmaf(row[32 * k + lane], r, proj[k]);
-      }
+      float proj = 0.f;  // (S rho)_j, j = 32 warp + lane
+#pragma unroll 16
+      for (int i = 0; i < kHeadDim; ++i) proj = fmaf(stw[i * 32 + lane], rho_s[warp][i], proj);
       __syncwarp();
-#pragma unroll
-      for (int k = 0; k < 4; ++k) zw[k] = __ballot_sync(0xffffffffu, proj[k] >= 0.f);
+      zword = __ballot_sync(0xffffffffu, proj >= 0.f);
     }
+    const bool lead = !coop || warp == 0;  // writes the planes and norms of this vector
 
     if (p.skip_rotation) {
-      if (lane < L.bits)
-        *reinterpret_cast<uint4*>(p.dbg_planes + ((size_t)vec * L.bits + lane) * 4) =
-            make_uint4(planes[lane][0], planes[lane][1], planes[lane][2], planes[lane][3]);
-      if (L.qjl && lane == 31)
-        *reinterpret_cast<uint4*>(p.dbg_sketch + (size_t)vec * 4) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
-      if (L.qjl && lane == 0) p.dbg_gamma[vec] = __half_as_ushort(__float2half_rn(gamma));
+      if (lead && lane < L.bits)
+        *reinterpret_cast<uint4*>(p.dbg_planes + ((size_t)vec * L.bits + lane) * 4) = mine;
+      if (coop && lane == 0) p.dbg_sketch[(size_t)vec * 4 + warp] = zword;
+      if (coop && warp == 0 && lane == 1) p.dbg_gamma[vec] = __half_as_ushort(__float2half_rn(gamma));
       continue;
     }
 
@@ -138,22 +156,27 @@ quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
     char* tb = p.region[side] +
                (((size_t)seq * p.heads + h) * p.tiles_per_seq + tile) * (size_t)L.tile_bytes;
     if (L.tokmajor) {
-      if (lane < L.bits)
-        *reinterpret_cast<uint4*>(tb + L.off_planes + lane * (kTile * 16) + slot * 16) =
-            make_uint4(planes[lane][0], planes[lane][1], planes[lane][2], planes[lane][3]);
-      if (L.qjl && lane == 31)
-        *reinterpret_cast<uint4*>(tb + L.off_sketch + slot * 16) = make_uint4(zw[0], zw[1], zw[2], zw[3]);
+      if (lead && lane < L.bits)
+        *reinterpret_cast<uint4*>(tb + L.off_planes + lane * (kTile * 16) + slot * 16) = mine;
+      if (coop && lane == 0) *reinterpret_cast<uint32_t*>(tb + L.off_sketch + slot * 16 + 4 * warp) = zword;
     } else {
       // byte-lane-major: byte k of a token's 16-byte plane goes to [k][slot]
-      for (int idx = lane; idx < (L.bits + L.qjl) * 16; idx += 32) {
-        const int pp = idx >> 4, k = idx & 15;
-        const uint32_t w = (pp < L.bits) ? planes[pp][k >> 2] : zw[k >> 2];
-        const int off = (pp < L.bits) ? L.off_planes + pp * (kTile * 16) : L.off_sketch;
-        tb[off + k * kTile + slot] = (char)((w >> (8 * (k & 3))) & 0xFFu);
+      if (lead && lane < 16) {
+#pragma unroll
+        for (int pp = 0; pp < kMaxBits; ++pp) {
+          if (pp < L.bits) {  // byte `lane` of plane pp: word lane / 4, byte lane % 4
+            const uint32_t lo = (lane & 4) ? planes[pp][1] : planes[pp][0];
+            const uint32_t hi = (lane & 4) ? planes[pp][3] : planes[pp][2];
+            const uint32_t w = (lane & 8) ? hi : lo;
+            tb[L.off_planes + pp * (kTile * 16) + lane * kTile + slot] = (char)((w >> (8 * (lane & 3))) & 0xFFu);
+          }
+        }
       }
+      if (coop && lane < 4)
+        tb[L.off_sketch + (4 * warp + lane) * kTile + slot] = (char)((zword >> (8 * lane)) & 0xFFu);
     }
-    if (lane == 30) *reinterpret_cast<__half*>(tb + L.off_norm + slot * 2) = __float2half_rn(n);
-    if (L.qjl && lane == 29)
+    if (lead && lane == 30) *reinterpret_cast<__half*>(tb + L.off_norm + slot * 2) = __float2half_rn(n);
+    if (coop && warp == 0 && lane == 29)
       *reinterpret_cast<__half*>(tb + L.off_gamma + slot * 2) = __float2half_rn(gamma);
   }
 
@@ -224,20 +247,19 @@ int grid_for(long work_items, int per_block) {
 
 cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s) {
   const long total = (long)p.n_seq * p.heads * p.n_new;
-  dim3 grid(grid_for(total, kQuantWarps), n_sides);
   const bool sketch = p.side[0].qjl || (n_sides > 1 && p.side[1].qjl);
-  const int m = p.side[0].qjl ? p.side[0].m : p.side[1].m;
-  const size_t smem = sketch ? sizeof(float) * kHeadDim * m : 0;
+  dim3 grid(grid_for(total, sketch ? 1 : kLmWarps), n_sides);  // sketch sides: one vector per block
+  const size_t smem = sketch ? sizeof(float) * kHeadDim * kHeadDim : 0;  // m = d = 128
   cudaError_t e = cudaFuncSetAttribute(quantize_lm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  quantize_lm_kernel<<<grid, kQuantWarps * 32, smem, s>>>(p);
-  return cudaGetLastError();
+  quantize_lm_kernel<<<grid, kLmWarps * 32, smem, s>>>(p);
+  return launched();
 }
 
 cudaError_t launch_quantize_fp4(const QuantizeParams& p, cudaStream_t s) {
   const long total = (long)p.n_seq * p.n_new;
   quantize_fp4_kernel<<<grid_for(total, kQuantWarps), kQuantWarps * 32, 0, s>>>(p);
-  return cudaGetLastError();
+  return launched();
 }
 
 }  // namespace kvq

@@ -173,6 +173,13 @@ kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_
                                       uint32_t* planes, uint32_t* sketch, uint16_t* gamma,
                                       void* stream);
 
+/* Diagnostic, with no counterpart in the method: the number of GPU kernels this library has
+ * enqueued successfully since it was loaded, summed over all threads, devices and caches. A
+ * caller reads it before and after a region to learn how many kernels the region launched
+ * (quantize: 1 per call; decode: 3 for LM caches on the tensor-core path, else 2). Host-only;
+ * never fails. */
+uint64_t kvq_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

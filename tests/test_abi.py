@@ -98,3 +98,16 @@ def test_init_rejects_null_and_misaligned_before_any_launch(lib):
     st = lib.kvq_cache_init(ctypes.byref(h), ctypes.byref(cfg), 1, 32, ctypes.c_void_p(0x10000), 1 << 20,
                             bad_signs.ctypes.data_as(ctypes.c_void_p), S.ctypes.data_as(ctypes.c_void_p), None)
     assert st == 1
+
+
+def test_rejected_calls_launch_nothing(lib):
+    """Validation failures return before any kernel is enqueued: the launch counter stays put."""
+    n0 = kvq.kvq_kernel_launches()
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_cache_bytes(kvq.make_cfg(k_bits=4), 1, 32)
+    import ctypes
+    h = ctypes.c_void_p()
+    signs = np.ones(128, dtype=np.int8)
+    assert lib.kvq_cache_init(ctypes.byref(h), ctypes.byref(kvq.make_cfg()), 1, 32, None, 1 << 20,
+                              signs.ctypes.data_as(ctypes.c_void_p), None, None) == 1
+    assert kvq.kvq_kernel_launches() == n0

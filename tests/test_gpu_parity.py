@@ -216,6 +216,29 @@ def test_fp4_full_context_sampled_heads():
     fp4_check(WORKLOADS["mla_fp4"].ctx, heads_checked=[0, 21, 63])
 
 
+# ---------------------------------------------------------------- launch accounting
+
+def test_launch_counts_per_call():
+    """quantize: one kernel; decode: prep + split decode + reduce for LM caches on the tensor-core
+    path (G <= 4), split decode + reduce otherwise (G = 8 and FP4)."""
+    for name, per_decode in (("llama8b", 3), ("llama70b", 2), ("mla_fp4", 2)):
+        w = WORKLOADS[name]
+        data = generate(w, DEV, seqs=range(2), ctx=100)
+        if w.k_mode == "fp4":
+            cache = kvq.KvqCache(kvq.cfg_for_workload(w), 2, 128)
+            a, b = data["latent"], data["rope"]
+        else:
+            cache, _, _ = new_cache(w, 2, 128)
+            a, b = data["k"], data["v"]
+        n0 = kvq.kvq_kernel_launches()
+        cache.quantize(a, b)
+        assert kvq.kvq_kernel_launches() - n0 == 1
+        cache.decode(data["q"])
+        assert kvq.kvq_kernel_launches() - n0 == 1 + per_decode, name
+        torch.cuda.synchronize()
+        cache.close()
+
+
 # ---------------------------------------------------------------- errors
 
 def test_capacity_overflow_writes_nothing():
