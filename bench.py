@@ -60,6 +60,30 @@ def parse():
     return ap.parse_args()
 
 
+# DRAM bytes (read + write) of one launch of the split decode kernel, from an ncu capture of the
+# workload named here. The record only counts while the kernel's sources are the ones captured
+# (their SHA-256 below); after any change the bench reports null until a new capture.
+TRAFFIC = {}
+TRAFFIC_SOURCES = ("bit_kv_cache_seeded_b200/csrc/kvq_decode_mma.cu", "bit_kv_cache_seeded_b200/csrc/kvq_async.cuh",
+                   "bit_kv_cache_seeded_b200/csrc/kvq_internal.h")
+
+
+def kernel_sources_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_record(w):
+    rec = TRAFFIC.get(w.name)
+    if rec is None or rec["sources_sha256"] != kernel_sources_sha():
+        return None
+    return rec["dram_bytes"]
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -209,6 +233,33 @@ def oracle_step(P):
     return dt, len(P["pairs"]) * P["ctx"] / w.n_kv_heads
 
 
+FP4_SAMPLE_CTX = 4096  # tokens of the FP4 latent cache the oracle covers per step
+
+
+def oracle_prepare_fp4(w, ctx):
+    """FP4 latent cache of the first `ctx` tokens of sequence 0, coded by the oracle (untimed)."""
+    from oracle import codec
+    data = generate(w, "cpu", seqs=range(1), ctx=ctx)
+    lat = data["latent"][0].float().numpy()
+    coded = [codec.fp4_quantize(lat[t]) for t in range(ctx - 1)]
+    return dict(w=w, packed=np.stack([c[0] for c in coded]), scales=np.stack([c[1] for c in coded]),
+                new=lat[ctx - 1], rope=data["rope"][0].double().numpy(), q=data["q"][0].double().numpy(),
+                ctx=ctx)
+
+
+def oracle_step_fp4(P):
+    """One oracle decode step over the sample: code the new token, dequantise, attend (all heads)."""
+    from oracle import attention, codec
+    w = P["w"]
+    t0 = time.perf_counter()
+    pk, sc = codec.fp4_quantize(P["new"])
+    packed = np.concatenate([P["packed"], pk[None]])
+    scales = np.concatenate([P["scales"], sc[None]])
+    attention.mla_decode_attention_many(P["q"], packed, scales, P["rope"],
+                                        1.0 / math.sqrt(w.latent_dim + w.rope_dim))
+    return time.perf_counter() - t0, P["ctx"]
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -224,18 +275,19 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     if w.k_mode == "fp4":
-        print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the LM workloads"}))
-        return
-    pairs = 1
-    P = oracle_prepare(w, pairs, w.ctx)
+        P, step_fn = oracle_prepare_fp4(w, FP4_SAMPLE_CTX), oracle_step_fp4
+        sample = f"sequence 0, first {FP4_SAMPLE_CTX} of {w.ctx} tokens, all {w.n_q_heads} heads, per step"
+    else:
+        pairs = 1
+        P, step_fn = oracle_prepare(w, pairs, w.ctx), oracle_step
+        sample = f"{pairs} (sequence, kv-head) pair of {w.batch * w.n_kv_heads} per step, ctx {w.ctx}"
     times = []
     for i in range(args.warmup + args.steps):
-        dt, toks = oracle_step(P)
+        dt, toks = step_fn(P)
         if i >= args.warmup:
             times.append(dt)
     per_step = sum(times) / len(times)
     value = toks / per_step
-    sample = f"{pairs} (sequence, kv-head) pair of {w.batch * w.n_kv_heads} per step, ctx {w.ctx}"
     line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -323,6 +375,19 @@ def run_ours(args, world, rank, local):
     ms_per_step = elapsed_ms / args.steps
     value = sum_over_ranks(kv_tokens, world) / (elapsed_ms / 1e3)
 
+    # Per-kernel device times: the same decode through the measurement entry, which records CUDA
+    # events between its kernels (prep | split kernel | reduce), rotating over the replicas.
+    n_k = min(args.steps, 50)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_k)]
+    torch.cuda.synchronize()
+    for j in range(n_k):
+        c = caches[j % replicas]
+        kvq.kvq_debug_decode_timed(c.handle, q, out, c.workspace, kev[j])
+    torch.cuda.synchronize()
+    kern_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in kev) / n_k for i in range(3)]
+    kern_ms = [max_over_ranks(x, world) for x in kern_ms]
+    lens_k = sum(int(caches[j % replicas].lengths()[0]) for j in range(n_k)) / n_k
+
     # End to end: host (pinned) inputs copied in, result copied out, every step.
     host_news = [(a.cpu().pin_memory(), b.cpu().pin_memory()) for a, b in news[:args.steps]]
     host_q = q.cpu().pin_memory()
@@ -361,7 +426,9 @@ def run_ours(args, world, rank, local):
 
     peaks, peak_kind = measured_peaks()
     bytes_step = w.batch * heads_kv * (lens0 + 1) * per_tok  # packed bytes one decode call reads
-    achieved = bytes_step / (dec_ms / 1e3) / 1e9
+    achieved_call = bytes_step / (dec_ms / 1e3) / 1e9
+    bytes_kernel = w.batch * heads_kv * lens_k * per_tok      # the split kernel's algorithmic bytes
+    achieved = bytes_kernel / (kern_ms[1] / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
     line = {
         "metric": METRIC,
@@ -371,27 +438,34 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": workload_config(w, world),
         "l2_detail": f"{replicas} cache replicas x {bytes_prefix / 1e6:.1f} MB rotated per step",
-        "hbm_gbs": achieved, "frac_of_8tbs": achieved / 8000.0,
+        "hbm_gbs": achieved_call, "frac_of_8tbs": achieved_call / 8000.0,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
-                     "kernel": "kvq_decode_attention (split-K decode + reduce)",
-                     "bytes_per_launch": bytes_step, "ms_per_launch": dec_ms},
+                     "frac": achieved / peak, "traffic": traffic_record(w), "peak_kind": peak_kind,
+                     "kernel": "split decode kernel (decode_lm_mma / decode_mla_mma)",
+                     "bytes_per_launch": bytes_kernel, "ms_per_launch": kern_ms[1]},
+        "decode_call": {"ms": dec_ms, "bytes": bytes_step, "gbs": achieved_call,
+                        "kernels_ms": {"prep": kern_ms[0], "split": kern_ms[1], "reduce": kern_ms[2]}},
         "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
-    if rank == 0 and not args.no_cpu_baseline and world == 1 and w.k_mode != "fp4":
-        pairs = 2
-        P = oracle_prepare(w, pairs, w.ctx)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        if w.k_mode == "fp4":
+            P, step_fn = oracle_prepare_fp4(w, FP4_SAMPLE_CTX), oracle_step_fp4
+            what = f"sequence 0, first {FP4_SAMPLE_CTX} of {w.ctx} tokens, all {w.n_q_heads} heads"
+        else:
+            pairs = 2
+            P, step_fn = oracle_prepare(w, pairs, w.ctx), oracle_step
+            what = (f"{pairs} (sequence, kv-head) pairs at ctx {w.ctx} (of {w.batch * heads_kv} pairs per "
+                    f"step)")
         tot, toks_tot, reps = 0.0, 0.0, 0
         while tot < 10.0 and reps < 200:
-            dt, toks = oracle_step(P)
+            dt, toks = step_fn(P)
             tot, toks_tot, reps = tot + dt, toks_tot + toks, reps + 1
         line["cpu_baseline"] = {"value": toks_tot / tot, "unit": "KV tokens/s", "cores": blas_threads(),
                                 "kind": "oracle",
-                                "sample": f"{reps} repetitions of {pairs} (sequence, kv-head) pairs of one decode "
-                                          f"step at ctx {w.ctx} (of {w.batch * heads_kv} pairs per step), fp64 numpy"}
+                                "sample": f"{reps} repetitions of one decode step over {what}, fp64 numpy"}
     if rank == 0:
         print(json.dumps(line))
     for c in caches:

@@ -32,7 +32,9 @@ DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "kvq_cache_init",
            "kvq_quantize", "kvq_workspace_bytes", "kvq_decode_attention", "kvq_cache_lengths",
            "kvq_cache_layout", "kvq_lloyd_max_table", "kvq_cache_destroy",
-           "kvq_debug_quantize_rotated", "kvq_decode_attention_static", "kvq_kernel_launches")
+           "kvq_debug_quantize_rotated", "kvq_decode_attention_static", "kvq_kernel_launches",
+           "kvq_cache_status", "kvq_debug_decode_unset_wait", "kvq_debug_decode_timed")
+KVQ_STATUS_WAIT_TIMEOUT = 1
 
 
 class KvqError(RuntimeError):
@@ -77,6 +79,9 @@ def load() -> ctypes.CDLL:
         "kvq_debug_quantize_rotated": ([VP, VP, I32, VP, VP, VP, VP], I32),
         "kvq_decode_attention_static": ([VP, VP, I32, VP, VP], I32),
         "kvq_kernel_launches": ([], ctypes.c_uint64),
+        "kvq_cache_status": ([VP, VP, VP], I32),
+        "kvq_debug_decode_unset_wait": ([VP, VP, I32, VP, VP, SZ, ctypes.c_int64, VP], I32),
+        "kvq_debug_decode_timed": ([VP, VP, I32, VP, VP, SZ, VP, VP], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +196,42 @@ def kvq_decode_attention_static(handle, q: torch.Tensor, out: torch.Tensor, stre
         raise ValueError("q and out must be contiguous")
     st = load().kvq_decode_attention_static(handle, _ptr(q), DTYPES[q.dtype], _ptr(out), _stream(stream))
     _check("kvq_decode_attention_static", st)
+
+
+def kvq_cache_status(handle, stream=None) -> int:
+    """The cache's device status word (KVQ_STATUS_* bits); waits for the stream."""
+    v = ctypes.c_int32(0)
+    _check("kvq_cache_status", load().kvq_cache_status(handle, ctypes.byref(v), _stream(stream)))
+    return int(v.value)
+
+
+def kvq_debug_decode_unset_wait(handle, q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                                wait_limit_cycles: int, stream=None):
+    """Test entry: decode with one extra bounded wait on a barrier that nothing completes."""
+    if q.dtype not in DTYPES or out.dtype != torch.float32:
+        raise TypeError("q must be float32/bfloat16 and out float32")
+    if not (q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("q and out must be contiguous")
+    st = load().kvq_debug_decode_unset_wait(handle, _ptr(q), DTYPES[q.dtype], _ptr(out), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(),
+                                            int(wait_limit_cycles), _stream(stream))
+    _check("kvq_debug_decode_unset_wait", st)
+
+
+def kvq_debug_decode_timed(handle, q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, events,
+                           stream=None):
+    """Decode recording 4 torch.cuda.Events: start, after prep, after the split kernel, after reduce."""
+    if q.dtype not in DTYPES or out.dtype != torch.float32:
+        raise TypeError("q must be float32/bfloat16 and out float32")
+    if len(events) != 4:
+        raise ValueError("four events")
+    for e in events:
+        if e.cuda_event == 0:  # torch creates the event lazily, on its first record
+            e.record()
+    arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    st = load().kvq_debug_decode_timed(handle, _ptr(q), DTYPES[q.dtype], _ptr(out), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream(stream), arr)
+    _check("kvq_debug_decode_timed", st)
 
 
 def kvq_cache_lengths(handle, batch: int) -> np.ndarray:

@@ -97,7 +97,7 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
   P.tiles = (capacity + kTile * kTilePair - 1) / (kTile * kTilePair) * kTilePair;
   size_t off = 0;
   P.lens_off = off;
-  off = align_up(off + sizeof(int) * (size_t)batch, kArenaAlign);
+  off = align_up(off + sizeof(int) * ((size_t)batch + kStatusWords), kArenaAlign);
   const size_t pairs = (size_t)batch * c->n_kv_heads;
   if (P.fp4_mode) {
     P.fp4 = make_fp4(c->latent_dim, c->rope_dim);
@@ -276,6 +276,7 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
   c->dev = static_cast<char*>(dev_mem);
   c->dev_bytes = dev_bytes;
   c->d_lens = reinterpret_cast<int*>(c->dev + P.lens_off);
+  c->d_status = c->d_lens + batch;
   c->is_fp4 = P.fp4_mode;
   c->k = P.k;
   c->v = P.v;
@@ -287,7 +288,7 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
   c->lens.assign(batch, 0);
   c->sms = device_sms();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(c->d_lens, 0, sizeof(int) * (size_t)batch, s) != cudaSuccess) {
+  if (cudaMemsetAsync(c->d_lens, 0, sizeof(int) * ((size_t)batch + kStatusWords), s) != cudaSuccess) {
     delete c;
     return KVQ_ERR_CUDA;
   }
@@ -378,8 +379,14 @@ kvq_status kvq_workspace_bytes(const kvq_cache* c, size_t* bytes) {
   return KVQ_OK;
 }
 
-kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
-                                void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// Shared body of kvq_decode_attention and its test entry (debug_unset_wait: every tensor-core
+// decode CTA first waits, bounded by wait_limit cycles, on a barrier that nothing completes).
+kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out, void* workspace,
+                       size_t ws_bytes, void* stream, int debug_unset_wait, long long wait_limit,
+                       const cudaEvent_t* ev = nullptr) {
   if (!c || !q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
   if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
@@ -392,6 +399,8 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
   if (ws_bytes < workspace_for(c, splits)) return KVQ_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const float log2e = 1.4426950408889634f;
+  auto rec = [&](int i) { return !ev || cudaEventRecord(ev[i], s) == cudaSuccess; };
+  if (!rec(0)) return KVQ_ERR_CUDA;
   if (c->is_fp4) {
     MlaParams p;
     std::memset(&p, 0, sizeof(p));
@@ -408,8 +417,8 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
     p.tiles_per_seq = c->tiles_per_seq;
     p.fp4 = c->fp4;
     p.logit_scale = default_scale(c->cfg) * log2e;
-    if (launch_decode_mla(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
-    if (launch_reduce_mla(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (!rec(1) || launch_decode_mla(p, s) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
+    if (launch_reduce_mla(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
     return KVQ_OK;
   }
   DecodeParams p;
@@ -437,8 +446,44 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
   p.logit_scale = default_scale(c->cfg) * log2e;
   p.qprep = static_cast<unsigned char*>(workspace) + partials_bytes(c, splits);
   p.qprep_stride = prep_stride(c);
-  if (launch_decode_lm(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
-  if (launch_reduce_lm(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  p.err = c->d_status;
+  p.wait_limit = wait_limit;
+  p.debug_unset_wait = debug_unset_wait;
+  if (debug_unset_wait && !mma_decode_supported(p)) return KVQ_ERR_UNSUPPORTED;
+  if (launch_decode_lm(p, s, ev ? ev[1] : nullptr) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
+  if (launch_reduce_lm(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles);
+}
+
+kvq_status kvq_debug_decode_unset_wait(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
+                                       void* workspace, size_t ws_bytes, int64_t wait_limit_cycles,
+                                       void* stream) {
+  if (wait_limit_cycles <= 0 || wait_limit_cycles > kWaitLimitCycles) return KVQ_ERR_INVALID_ARG;
+  return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 1, wait_limit_cycles);
+}
+
+kvq_status kvq_debug_decode_timed(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
+                                  void* workspace, size_t ws_bytes, void* stream, void* const* events) {
+  if (!events || !events[0] || !events[1] || !events[2] || !events[3]) return KVQ_ERR_INVALID_ARG;
+  cudaEvent_t ev[4];
+  for (int i = 0; i < 4; ++i) ev[i] = static_cast<cudaEvent_t>(events[i]);
+  return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles, ev);
+}
+
+kvq_status kvq_cache_status(const kvq_cache* c, int32_t* status, void* stream) {
+  if (!c || !status) return KVQ_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(status, c->d_status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }
 

@@ -4,6 +4,8 @@
 // commit groups); other threads see them only after a barrier that follows the wait.
 #pragma once
 
+#include <cstdint>
+
 namespace kvq {
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -13,6 +15,39 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+// Bulk (TMA 1-D) copies global -> shared that complete on an mbarrier. One thread arms the
+// barrier with the byte count it expects (arrive + expect_tx) and issues the copies; every thread
+// then waits on the barrier's phase parity. Addresses and sizes must be multiples of 16 bytes.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+// Makes initialised barriers visible to the bulk-copy unit (before the first copy names them).
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Orders this thread's earlier generic-proxy shared-memory accesses (after a barrier, those of
+// the whole CTA) before later bulk copies into the same buffer.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+// Waits until the barrier's phase with parity `parity` has completed, giving up after `limit`
+// SM clock cycles. Returns false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    if (done) return true;
+    if (clock64() - t0 > limit) return false;
+  }
+}
 
 // Programmatic dependent launch (sm_90+). A kernel launched with programmatic stream
 // serialization may start while its predecessor in the stream is still running; grid_dep_wait()

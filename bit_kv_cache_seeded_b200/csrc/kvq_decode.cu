@@ -374,8 +374,9 @@ cudaError_t dispatch_modes(const DecodeParams& p, dim3 grid, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s) {
-  if (mma_decode_supported(p)) return launch_decode_lm_mma(p, s);
+cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid) {
+  if (mma_decode_supported(p)) return launch_decode_lm_mma(p, s, ev_mid);
+  if (ev_mid && cudaEventRecord(ev_mid, s) != cudaSuccess) return cudaErrorUnknown;
   dim3 grid(p.splits, p.Hkv, p.B);
   switch (p.group) {
     case 1: return dispatch_modes<1>(p, grid, s);

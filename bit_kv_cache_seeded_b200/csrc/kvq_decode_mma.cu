@@ -13,20 +13,24 @@
 //   * Logits: A = key bits [16 tokens x 32 bits]. Byte i of plane word w holds coordinates
 //     32w + 8i + p in bit p; (w << (7 - p)) & 0x80808080 turns bit p of every byte into the int8
 //     value -128 or 0 (one multiply and one LOP3 per 4 operand bytes). B = the query term
-//     2 a_P q~_j quantised to a 14-bit integer (2 x 7-bit signed digits, one column each).
+//     2 a_P q~_j quantised to a 16-bit integer (2 signed 8-bit digits, one column each).
 //   * Values: A = value bits [16 coordinates x 32 tokens] read from the byte-lane-major value
 //     tile, where 4 tokens of one byte-lane are one 32-bit word: w & (0x01010101 << p) gives the
 //     int8 value 2^p (p < 7) or -128 (p = 7) per byte, i.e. a fixed power of two per row. B = the
 //     softmax weights p_t n_t / sqrt(d) (times sqrt(pi/2)/m gamma_t for the value sketch) as a
-//     21-bit integer relative to the chunk maximum (3 x 7-bit unsigned digits).
+//     21-bit integer (3 x 7-bit unsigned digits), each kind scaled by a power of two to its own
+//     chunk maximum.
 //   * Two passes over a CTA's chunk (at most kChunkMax tokens): pass 1 computes every logit into
 //     shared memory and the chunk's maxima; pass 2 streams the value tiles with the weights
 //     2^(l - M) fixed, so the int32 accumulators are exact and never rescaled.
 //
 // CTA: 4 warps. Pass 1: 64 tokens (two cache tiles) per iteration, warp w owns tokens
 // 16w..16w+15. Pass 2: 64 tokens per iteration, warp w owns bit positions 2w, 2w+1 of every value
-// Walsh plane. cp.async stages both passes. Partials (m, l, o_r, acc_z) are written in the format
-// of the CUDA-core kernel; the same reduce kernel finishes.
+// Walsh plane. Both passes stream whole tile pairs through 4 shared-memory stages with bulk
+// (TMA 1-D) copies completing on mbarriers; the value tiles of pass 2 are already in flight during
+// the last iterations of pass 1. Every wait is bounded: a wait that gives up sets bit 0 of the
+// cache's status word. Partials (m, l, o_r, acc_z) are written in the format of the CUDA-core
+// kernel; the same reduce kernel finishes.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -41,14 +45,33 @@ namespace {
 constexpr int kWarpsM = 4;
 constexpr int kThreadsM = kWarpsM * 32;
 constexpr int kCtaTok = 64;
-constexpr int kStagesM = 3;
+constexpr int kStagesM = 4;                          // bulk-copy stages (tile pairs in flight)
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
 constexpr float kSqrtHalfPi = 1.2533141373155003f;  // sqrt(pi/2)
 constexpr int kQRange = 32639;                       // query term quantised to [-32639, 32639]
 constexpr int kLgStride = kChunkMax + 8;             // logits row stride (floats): rows on distinct banks
 constexpr int kPdStride = 96;                        // weight-digit row stride (bytes): 64 tokens + pad
 constexpr int kNormBlock = 256;                      // staged value norms / gammas of two cache tiles
-constexpr float kWRange = 2097152.f;                 // weights quantised below 2^21
+constexpr float kWRange = 8388608.f;                 // weights quantised below 2^23
+constexpr float kRoundBias = 8388608.f;              // x + 2^23 (0 <= x < 2^23): bits = 0x4B000000 | rint(x)
+
+// A int8, B uint8 (the value-phase weight digits are non-negative bytes).
+__device__ __forceinline__ void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte `k` of each of four words, packed into one word (k = 0..3).
+template <int K>
+__device__ __forceinline__ uint32_t pack_byte(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
+  const uint32_t a = __byte_perm(x0, x1, K | ((4 + K) << 4));
+  const uint32_t b = __byte_perm(x2, x3, K | ((4 + K) << 4));
+  return __byte_perm(a, b, 0x5410);
+}
 
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1) {
@@ -238,15 +261,21 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   constexpr int KP = C::KP, VP = C::VP, KNT = C::KNT, VNT = C::VNT, VNCOL = C::VNCOL;
   constexpr int VWP = Walsh<VB>::P;
   constexpr int NKIND = VQ ? 2 : 1;
-  constexpr int NTASK = NKIND * G * 16;
-  static_assert(NTASK <= kThreadsM, "one weight task per thread");
-  extern __shared__ __align__(16) unsigned char smem[];
+  // weight tasks: (head, TPT consecutive tokens), both kinds; spread over all threads
+  constexpr int TPT = (G * kCtaTok) / kThreadsM > 0 ? (G * kCtaTok) / kThreadsM : 1;
+  constexpr int TASKS_PER_HEAD = kCtaTok / TPT;
+  constexpr int NTASK = G * TASKS_PER_HEAD;
+  static_assert(NTASK <= kThreadsM && (TPT == 1 || TPT == 2), "one weight task per thread");
+  constexpr int PDB = NKIND * VNCOL * kPdStride;  // one digit buffer (two: current and next)
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t mbar[kStagesM + 1];  // per stage (+ one nothing completes: test entry)
+  __shared__ int s_fail;                             // a wait of this CTA gave up
   const int ktb = p.k.tile_bytes, vtb = p.v.tile_bytes;
   const int stage_bytes = max(2 * ktb + kNormBlock, 2 * vtb);
   unsigned char* stages = smem;                                            // [kStagesM][2 tiles (+ norms)]
   float* lgs = reinterpret_cast<float*>(stages + kStagesM * stage_bytes);  // [G][kLgStride] logits
-  unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * kLgStride);  // [NKIND][VNCOL][kPdStride]
-  float* red = reinterpret_cast<float*>(pdig + NKIND * VNCOL * kPdStride);     // reductions
+  unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * kLgStride);  // [2][NKIND][VNCOL][kPdStride]
+  float* red = reinterpret_cast<float*>(pdig + 2 * PDB);                      // reductions
 
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -259,27 +288,52 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   const unsigned char* vbase = reinterpret_cast<const unsigned char*>(p.vreg) + pair * p.tiles_per_seq * (size_t)vtb;
   const int n_iter = t_end > t_begin ? (t_end - t_begin + kCtaTok - 1) / kCtaTok : 0;
 
-  // stage loader: the two cache tiles of K (pass 0) or V (pass 1) for iteration `it`
-  auto load_stage = [&](int pass, int it, int slot) {
-    if (it < n_iter) {
-      const int tile0 = (t_begin + it * kCtaTok) / kTile;
-      const int ntiles = (t_begin + it * kCtaTok + kTile < t_end) ? 2 : 1;
-      const int tb = pass ? vtb : ktb;
-      const unsigned char* src = (pass ? vbase : kbase) + (size_t)tile0 * tb;
-      unsigned char* dst = stages + slot * stage_bytes;
-      for (int c = tid; c < ntiles * tb / 16; c += kThreadsM) cp_async16(dst + 16 * c, src + 16 * c);
-      if (!pass && tid < ntiles * 8) {  // value norms (4 x 16 B) and gammas (4 x 16 B) per tile
-        const int tile = tid >> 3, part = tid & 7;
-        if (part < 4 || VQ) {
-          const unsigned char* vs = vbase + (size_t)(tile0 + tile) * vtb + (part < 4 ? p.v.off_norm : p.v.off_gamma) + 16 * (part & 3);
-          cp_async16(dst + 2 * ktb + tile * 128 + 16 * part, vs);
-        }
-      }
-    }
-    cp_async_commit();
-  };
+  // Staging: fill f < n_iter brings the K tile pair of pass-1 iteration f (and the value norms
+  // and sketch norms of the same tokens, for the weight scale); fill n_iter + i brings the V tile
+  // pair of pass-2 iteration i. Fill f goes to stage f % kStagesM and completes phase f / kStagesM
+  // of that stage's barrier. Thread 0 issues the fills as bulk copies; every tile pair is whole
+  // (capacity is a whole number of pairs), so a fill never reads outside its pair's region.
+  const int n_fill = 2 * n_iter;
+  if (tid == 0) {
 #pragma unroll
-  for (int s = 0; s < kStagesM - 1; ++s) load_stage(0, s, s);
+    for (int s = 0; s <= kStagesM; ++s) mbar_init(smem_addr(&mbar[s]), 1);
+    mbar_init_fence();
+    s_fail = 0;
+  }
+  __syncthreads();
+  auto issue = [&](int f) {  // thread 0 only
+    if (f >= n_fill) return;
+    const int slot = f % kStagesM;
+    const uint32_t bar = smem_addr(&mbar[slot]);
+    unsigned char* dst = stages + slot * stage_bytes;
+    fence_proxy_async();  // the stage's previous contents were read by the generic proxy
+    if (f < n_iter) {
+      const int tile0 = (t_begin + f * kCtaTok) / kTile;
+      constexpr uint32_t nb = VQ ? 128u : 64u;  // value norms (+ gammas, contiguous) per tile
+      mbar_arrive_expect_tx(bar, 2u * ktb + 2u * nb);
+      bulk_g2s(smem_addr(dst), kbase + (size_t)tile0 * ktb, 2u * ktb, bar);
+#pragma unroll
+      for (int tile = 0; tile < 2; ++tile)
+        bulk_g2s(smem_addr(dst + 2 * ktb + tile * 128), vbase + (size_t)(tile0 + tile) * vtb + p.v.off_norm, nb, bar);
+    } else {
+      const int tile0 = (t_begin + (f - n_iter) * kCtaTok) / kTile;
+      mbar_arrive_expect_tx(bar, 2u * vtb);
+      bulk_g2s(smem_addr(dst), vbase + (size_t)tile0 * vtb, 2u * vtb, bar);
+    }
+  };
+  auto wait_fill = [&](int f) {  // every thread
+    if (!mbar_wait(smem_addr(&mbar[f % kStagesM]), (uint32_t)(f / kStagesM) & 1u, p.wait_limit)) {
+      s_fail = 1;
+      atomicOr(p.err, 1);
+    }
+  };
+  if (tid == 0)
+#pragma unroll
+    for (int f = 0; f < kStagesM - 1; ++f) issue(f);
+  if (p.debug_unset_wait && !mbar_wait(smem_addr(&mbar[kStagesM]), 0u, p.wait_limit)) {
+    s_fail = 1;
+    atomicOr(p.err, 1);
+  }
 
   // logit-phase B fragments (query digits) and head constants from the prep area
   // Launched as a programmatic dependent of the prep kernel: the cache tiles staged above were
@@ -322,9 +376,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   float wmax = 0.f, wmaxz = 0.f;  // largest value weight of each kind seen by this thread
   const int tl = warp * 16;
   for (int it = 0; it < n_iter; ++it) {
-    load_stage(0, it + kStagesM - 1, (it + kStagesM - 1) % kStagesM);
-    cp_async_wait<kStagesM - 1>();
-    __syncthreads();
+    if (tid == 0) issue(it + kStagesM - 1);
+    wait_fill(it);
     const unsigned char* kt = stages + (it % kStagesM) * stage_bytes;
     const int tok0 = it * kCtaTok;  // chunk-relative first token of this iteration
     const int count = min(kCtaTok, t_end - (t_begin + tok0));
@@ -412,10 +465,6 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     }
     __syncthreads();  // the next iteration refills a stage buffer
   }
-  // prefetch the first value tiles while the maxima are combined
-#pragma unroll
-  for (int s = 0; s < kStagesM - 1; ++s) load_stage(1, s, s);
-
   // chunk maxima per head, and the weight scale
   float* hmax = red;                 // [kWarpsM][G]
   float* wred = red + kWarpsM * G;   // [2][kWarpsM]: both kinds' weight maxima
@@ -433,6 +482,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     wmaxz = fmaxf(wmaxz, __shfl_xor_sync(0xffffffffu, wmaxz, o));
   }
   if (lane == 0) { wred[warp] = wmax; wred[kWarpsM + warp] = wmaxz; }
+  for (int idx = tid; idx < 2 * PDB / 4; idx += kThreadsM)
+    reinterpret_cast<uint32_t*>(pdig)[idx] = 0u;  // the pad digit and absent heads stay zero
   __syncthreads();
   float wm = 0.f, wmz = 0.f;
 #pragma unroll
@@ -444,15 +495,70 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 
   // ================= pass 2: weights -> digits, value contractions
   const bool has_task = tid < NTASK;
-  const int task_kind = tid / (G * 16), task_h = (tid / 16) % G, task_q = tid % 16;
-  const float task_sc = (VQ && task_kind == 1) ? wscz : wsc;
+  const int task_h = min(tid / TASKS_PER_HEAD, G - 1), task_T = TPT * (tid % TASKS_PER_HEAD);
   float task_m = -INFINITY;
 #pragma unroll
   for (int w = 0; w < kWarpsM; ++w) task_m = fmaxf(task_m, hmax[w * G + task_h]);
-  float task_l = 0.f;     // sum of p over this task's tokens
-  long long task_wl = 0;  // sum of the quantised weights (exact)
-  for (int idx = tid; idx < NKIND * VNCOL * kPdStride / 4; idx += kThreadsM)
-    reinterpret_cast<uint32_t*>(pdig)[idx] = 0u;  // the pad digit and absent heads stay zero
+  float task_l = 0.f;                 // sum of p over this task's tokens
+  uint32_t task_wc = 0, task_wz = 0;  // sums of the quantised weights (exact: <= 64 tokens x 2^23)
+
+  // Weight digits of pass-2 iteration `it` into digit buffer it & 1: p = 2^(l - m) for the task's
+  // tokens, then both kinds of value weight; w * scale is rounded by adding 2^23, after which the
+  // float's low three bytes are the integer, i.e. directly its three byte digits. Tokens past the
+  // end have logit -inf (p = 0) and their norms are masked (a tile's tail may hold anything).
+  // Reads the logits and the value norms of fill n_iter + it (which must have landed).
+  auto tasks = [&](int it) {
+    if (!has_task) return;
+    const int tok0 = it * kCtaTok, T = task_T;
+    const int count = min(kCtaTok, t_end - (t_begin + tok0));
+    const unsigned char* vtile = stages + ((n_iter + it) % kStagesM) * stage_bytes + (T / kTile) * vtb;
+    float lv[TPT], wc[TPT], wz[TPT];
+    if (TPT == 2) {
+      const float2 l2 = *reinterpret_cast<const float2*>(lgs + task_h * kLgStride + tok0 + T);
+      const float2 n2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + p.v.off_norm + (T % kTile) * 2));
+      lv[0] = l2.x; lv[TPT - 1] = l2.y; wc[0] = n2.x; wc[TPT - 1] = n2.y;
+      if (VQ) {
+        const float2 g2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + p.v.off_gamma + (T % kTile) * 2));
+        wz[0] = g2.x; wz[TPT - 1] = g2.y;
+      }
+    } else {
+      lv[0] = lgs[task_h * kLgStride + tok0 + T];
+      wc[0] = __half2float(*reinterpret_cast<const __half*>(vtile + p.v.off_norm + (T % kTile) * 2));
+      if (VQ) wz[0] = __half2float(*reinterpret_cast<const __half*>(vtile + p.v.off_gamma + (T % kTile) * 2));
+    }
+    uint32_t bc[TPT], bz[TPT];
+    float psum = 0.f;
+#pragma unroll
+    for (int e = 0; e < TPT; ++e) {
+      const bool ok = T + e < count;
+      const float pe = ex2(lv[e] - task_m);
+      psum += pe;
+      const float n = ok ? wc[e] * (kInvSqrtD * wsc) : 0.f;
+      bc[e] = __float_as_uint(fmaf(pe, n, kRoundBias));
+      task_wc += bc[e] - 0x4B000000u;
+      if (VQ) {
+        const float nz = ok ? wc[e] * wz[e] * (kInvSqrtD * wscz * vkappa) : 0.f;
+        bz[e] = __float_as_uint(fmaf(pe, nz, kRoundBias));
+        task_wz += bz[e] - 0x4B000000u;
+      }
+    }
+    task_l += psum;
+    unsigned char* col = pdig + (it & 1) * PDB + (size_t)(4 * task_h) * kPdStride + T;
+#pragma unroll
+    for (int kind = 0; kind < NKIND; ++kind) {
+      const uint32_t* bw = kind ? bz : bc;
+      unsigned char* ck = col + (size_t)kind * VNCOL * kPdStride;
+      if (TPT == 2) {  // digit rows 0, 1, 2 = bytes 2, 1, 0 of the rounded floats
+        *reinterpret_cast<uint16_t*>(ck) = (uint16_t)__byte_perm(bw[0], bw[TPT - 1], 0x62);
+        *reinterpret_cast<uint16_t*>(ck + kPdStride) = (uint16_t)__byte_perm(bw[0], bw[TPT - 1], 0x51);
+        *reinterpret_cast<uint16_t*>(ck + 2 * kPdStride) = (uint16_t)__byte_perm(bw[0], bw[TPT - 1], 0x40);
+      } else {
+        ck[0] = (unsigned char)(bw[0] >> 16);
+        ck[kPdStride] = (unsigned char)(bw[0] >> 8);
+        ck[2 * kPdStride] = (unsigned char)bw[0];
+      }
+    }
+  };
 
   int vacc[VP][2][VNT][4];
 #pragma unroll
@@ -465,52 +571,23 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         for (int c = 0; c < 4; ++c) vacc[P][pi][nt][c] = 0;
   const uint32_t vm0 = 0x01010101u << (2 * warp), vm1 = 0x01010101u << (2 * warp + 1);
 
+  // Digits of iteration 0, then per iteration: the digits of the next one (all threads) and the
+  // contractions of this one; one barrier per iteration separates the two digit buffers.
+  if (n_iter > 0) {
+    wait_fill(n_iter);
+    tasks(0);
+  }
+  __syncthreads();
   for (int it = 0; it < n_iter; ++it) {
-    load_stage(1, it + kStagesM - 1, (it + kStagesM - 1) % kStagesM);
-    cp_async_wait<kStagesM - 1>();
-    __syncthreads();
-    const unsigned char* vt = stages + (it % kStagesM) * stage_bytes;
+    if (tid == 0) issue(n_iter + it + kStagesM - 1);
+    if (it + 1 < n_iter) {
+      wait_fill(n_iter + it + 1);
+      tasks(it + 1);
+    }
+    const unsigned char* vt = stages + ((n_iter + it) % kStagesM) * stage_bytes;
     const int tok0 = it * kCtaTok;
     const int count = min(kCtaTok, t_end - (t_begin + tok0));
-
-    // weight task: 4 consecutive tokens of one head, one kind
-    if (has_task) {
-      const int T = 4 * task_q;
-      const float4 l4 = *reinterpret_cast<const float4*>(lgs + task_h * kLgStride + tok0 + T);
-      const unsigned char* vtile = vt + (T / kTile) * vtb;
-      const uint2 nraw = *reinterpret_cast<const uint2*>(vtile + p.v.off_norm + (T % kTile) * 2);
-      const float2 n01 = __half22float2(*reinterpret_cast<const __half2*>(&nraw.x));
-      const float2 n23 = __half22float2(*reinterpret_cast<const __half2*>(&nraw.y));
-      float wv[4] = {n01.x * kInvSqrtD, n01.y * kInvSqrtD, n23.x * kInvSqrtD, n23.y * kInvSqrtD};
-      if (VQ && task_kind == 1) {
-        const uint2 graw = *reinterpret_cast<const uint2*>(vtile + p.v.off_gamma + (T % kTile) * 2);
-        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(&graw.x));
-        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(&graw.y));
-        wv[0] *= g01.x * vkappa; wv[1] *= g01.y * vkappa; wv[2] *= g23.x * vkappa; wv[3] *= g23.y * vkappa;
-      }
-      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-      uint32_t d0 = 0, d1 = 0, d2 = 0;
-      float psum = 0.f;
-      int qsum = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool ok = T + e < count;
-        const float pe = ok ? ex2(lv[e] - task_m) : 0.f;
-        psum += pe;
-        const int q = ok ? __float2int_rn(pe * wv[e] * task_sc) : 0;  // < 2^21
-        qsum += q;
-        d0 |= (uint32_t)(q >> 14) << (8 * e);
-        d1 |= (uint32_t)((q >> 7) & 127) << (8 * e);
-        d2 |= (uint32_t)(q & 127) << (8 * e);
-      }
-      task_l += psum;
-      task_wl += qsum;
-      unsigned char* col = pdig + (size_t)(task_kind * VNCOL + 4 * task_h) * kPdStride + T;
-      *reinterpret_cast<uint32_t*>(col) = d0;
-      *reinterpret_cast<uint32_t*>(col + kPdStride) = d1;
-      *reinterpret_cast<uint32_t*>(col + 2 * kPdStride) = d2;
-    }
-    __syncthreads();
+    const unsigned char* pd = pdig + (it & 1) * PDB;
 
     // value contractions: positions 2w, 2w+1 of every value Walsh plane
 #pragma unroll
@@ -522,7 +599,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       uint32_t bm[VNT][2], bz[VNT][2];
 #pragma unroll
       for (int nt = 0; nt < VNT; ++nt) {
-        const unsigned char* col = pdig + (size_t)(nt * 8 + g) * kPdStride + s * kTile + 8 * t;
+        const unsigned char* col = pd + (size_t)(nt * 8 + g) * kPdStride + s * kTile + 8 * t;
         const uint2 v = *reinterpret_cast<const uint2*>(col);
         bm[nt][0] = v.x;
         bm[nt][1] = v.y;
@@ -532,10 +609,11 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
           bz[nt][1] = vz.y;
         }
       }
-      uint32_t xv[3][4];
+      uint32_t xv[4][4];  // code planes, then the sketch plane (same byte-lane-major layout)
 #pragma unroll
-      for (int pp = 0; pp < VB; ++pp) {
-        const unsigned char* pl = vtile + p.v.off_planes + pp * (kTile * 16) + 8 * t;
+      for (int pp = 0; pp < VB + (VQ ? 1 : 0); ++pp) {
+        const unsigned char* pl =
+            vtile + (pp < VB ? p.v.off_planes + pp * (kTile * 16) : p.v.off_sketch) + 8 * t;
         const uint2 r0 = *reinterpret_cast<const uint2*>(pl + g * kTile);
         const uint2 r1 = *reinterpret_cast<const uint2*>(pl + (g + 8) * kTile);
         xv[pp][0] = r0.x; xv[pp][2] = r0.y;
@@ -548,8 +626,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           if (sk) {
-            const unsigned char* pl = vtile + p.v.off_sketch + 8 * t;
-            x[r] = *reinterpret_cast<const uint32_t*>(pl + ((r & 1) ? g + 8 : g) * kTile + ((r & 2) ? 4 : 0));
+            x[r] = xv[VB][r];
           } else if (VB == 3 && P == 3) {
             x[r] = xv[0][r] ^ xv[1][r] ^ xv[2][r];
           } else {
@@ -561,8 +638,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int nt = 0; nt < VNT; ++nt) {
           const uint32_t b0 = sk ? bz[nt][0] : bm[nt][0], b1 = sk ? bz[nt][1] : bm[nt][1];
-          mma_s8(vacc[P][0][nt], a00, a01, a02, a03, b0, b1);
-          mma_s8(vacc[P][1][nt], a10, a11, a12, a13, b0, b1);
+          mma_s8u8(vacc[P][0][nt], a00, a01, a02, a03, b0, b1);
+          mma_s8u8(vacc[P][1][nt], a10, a11, a12, a13, b0, b1);
         }
       }
     }
@@ -571,19 +648,22 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 
   grid_dep_launch();  // let the split reduce be scheduled; it waits for this grid to finish
   // ================= finish: per-head sums of p and of the weights, then this warp's rows
-  cp_async_wait<0>();
+  // Every fill was waited for above; after a wait that gave up, thread 0 waits once more (bounded)
+  // for the last fill of each stage, so no copy is still landing when the stages are reused.
+  if (tid == 0 && s_fail)
+    for (int f = max(0, n_fill - kStagesM); f < n_fill; ++f)
+      mbar_wait(smem_addr(&mbar[f % kStagesM]), (uint32_t)(f / kStagesM) & 1u, p.wait_limit);
   __syncthreads();
-  float* tsum = reinterpret_cast<float*>(stages);  // [kThreadsM][2] (staging reused)
-  float* hsum = tsum + 2 * kThreadsM;               // [3][G]: sum p, sum weights, sum sketch weights
-  tsum[2 * tid] = task_l;
-  tsum[2 * tid + 1] = (float)task_wl;
+  float* tsum = reinterpret_cast<float*>(stages);  // [kThreadsM][3] (staging reused)
+  float* hsum = tsum + 3 * kThreadsM;               // [3][G]: sum p, sum weights, sum sketch weights
+  tsum[3 * tid] = task_l;
+  tsum[3 * tid + 1] = (float)task_wc;
+  tsum[3 * tid + 2] = (float)task_wz;
   __syncthreads();
   if (tid < 3 * G) {
-    const int what = tid / G, h = tid % G;
-    const int kind = what == 2 ? 1 : 0;
+    const int what = tid / G, h = tid % G;  // what: 0 sum p, 1 sum weights, 2 sum sketch weights
     float s2 = 0.f;
-    if (kind < NKIND)
-      for (int q = 0; q < 16; ++q) s2 += tsum[2 * ((kind * G + h) * 16 + q) + (what == 0 ? 0 : 1)];
+    for (int q = 0; q < TASKS_PER_HEAD; ++q) s2 += tsum[3 * (h * TASKS_PER_HEAD + q) + what];
     hsum[tid] = s2;
   }
   __syncthreads();
@@ -601,8 +681,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
     for (int nt = 0; nt < VNT; ++nt) {
       const int h = 2 * nt + t / 2;
-      // columns (2t, 2t+1): digits (0, 1) for even t, (2, pad) for odd t, of head 2 nt + t / 2
-      const float wd0 = (t & 1) ? 1.f : 16384.f, wd1 = (t & 1) ? 0.f : 128.f;
+      // columns (2t, 2t+1): byte digits (2, 1) for even t, (0, pad) for odd t, of head 2 nt + t / 2
+      const float wd0 = (t & 1) ? 1.f : 65536.f, wd1 = (t & 1) ? 0.f : 256.f;
       float o0 = 0.f, o1 = 0.f, z0 = 0.f, z1 = 0.f;
 #pragma unroll
       for (int P = 0; P < VP; ++P) {
@@ -648,13 +728,13 @@ size_t mma_smem_bytes(const DecodeParams& p) {
   constexpr int NKIND = VQ ? 2 : 1;
   size_t s = (size_t)kStagesM * std::max(2 * p.k.tile_bytes + kNormBlock, 2 * p.v.tile_bytes);
   s += sizeof(float) * (size_t)G * kLgStride;
-  s += (size_t)NKIND * C::VNCOL * kPdStride;
+  s += 2 * (size_t)NKIND * C::VNCOL * kPdStride;
   s += sizeof(float) * (kWarpsM * G + 2 * kWarpsM);
   return (s + 15) / 16 * 16;
 }
 
 template <int G, int KB, bool KQ, int VB, bool VQ>
-cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s) {
+cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid) {
   const size_t prep_smem = KQ ? sizeof(float) * kHeadDim * kHeadDim : 0;
   cudaError_t e = cudaFuncSetAttribute(decode_lm_prep<G, KB, KQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep_smem);
@@ -662,6 +742,7 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s) {
   decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv, p.B), kThreadsM, prep_smem, s>>>(p);
   e = launched();
   if (e != cudaSuccess) return e;
+  if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
   const size_t smem = mma_smem_bytes<G, KB, KQ, VB, VQ>(p);
   auto kern = decode_lm_mma<G, KB, KQ, VB, VQ>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -682,11 +763,11 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s) {
 }
 
 template <int G>
-cudaError_t dispatch_mma_modes(const DecodeParams& p, cudaStream_t s) {
+cudaError_t dispatch_mma_modes(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid) {
   const int kb = p.k.bits, vb = p.v.bits;
   const bool kq = p.k.qjl, vq = p.v.qjl;
 #define KVQ_MMA_CASE(KB, KQ, VB, VQ) \
-  if (kb == KB && kq == KQ && vb == VB && vq == VQ) return launch_mma<G, KB, KQ, VB, VQ>(p, s);
+  if (kb == KB && kq == KQ && vb == VB && vq == VQ) return launch_mma<G, KB, KQ, VB, VQ>(p, s, ev_mid);
   KVQ_MMA_CASE(2, true, 2, true)
   KVQ_MMA_CASE(3, true, 3, false)
   KVQ_MMA_CASE(1, false, 1, false)
@@ -711,11 +792,11 @@ bool mma_decode_supported(const DecodeParams& p) {
          p.chunk <= kChunkMax && p.qprep != nullptr;
 }
 
-cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s) {
+cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid) {
   switch (p.group) {
-    case 1: return dispatch_mma_modes<1>(p, s);
-    case 2: return dispatch_mma_modes<2>(p, s);
-    case 4: return dispatch_mma_modes<4>(p, s);
+    case 1: return dispatch_mma_modes<1>(p, s, ev_mid);
+    case 2: return dispatch_mma_modes<2>(p, s, ev_mid);
+    case 4: return dispatch_mma_modes<4>(p, s, ev_mid);
     default: return cudaErrorNotSupported;
   }
 }

@@ -17,6 +17,8 @@ constexpr int kMaxSeqPerLaunch = 1024;
 constexpr int kMaxBits = 3;
 constexpr int kTilePair = 2;      // cache tiles are allocated and split in pairs (64 tokens)
 constexpr int kChunkMax = 2048;   // largest context chunk of one decode CTA (LM tensor-core path)
+constexpr int kStatusWords = 8;   // device status ints kept after the lengths in the arena
+constexpr long long kWaitLimitCycles = 1ll << 31;  // ~1 s at 2 GHz: a staged-data wait gives up
 
 // Where one side (K or V) of an LM/SIGN1 cache keeps its fields inside a 32-token tile.
 struct SideLayout {
@@ -80,6 +82,9 @@ struct DecodeParams {
   float logit_scale;      // softmax_scale * log2(e)
   unsigned char* qprep;   // per (sequence, kv-head) query digit tables (tensor-core path)
   int qprep_stride;       // bytes per (sequence, kv-head)
+  int* err;               // cache status word: bit 0 set when a wait for staged data gave up
+  long long wait_limit;   // SM clock cycles a kernel waits for staged data before giving up
+  int debug_unset_wait;   // test entry: also wait once on a barrier nothing completes
 };
 
 struct MlaParams {
@@ -103,10 +108,12 @@ cudaError_t launched();
 // Launchers (kvq_quantize.cu, kvq_decode.cu, kvq_mla.cu). Return launched().
 cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s);
 cudaError_t launch_quantize_fp4(const QuantizeParams& p, cudaStream_t s);
-cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s);
+// ev_mid (may be null) is recorded between the query prep and the split kernel (right before the
+// split kernel when there is no prep).
+cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid = nullptr);
 bool mma_decode_supported(const DecodeParams& p);
 int mma_prep_bytes(int k_bits, int k_qjl, int group);  // bytes of one (sequence, kv-head) prep area
-cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s);
+cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid);
 cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s);
@@ -125,6 +132,7 @@ struct kvq_cache {
   char* dev = nullptr;
   size_t dev_bytes = 0;
   int* d_lens = nullptr;
+  int* d_status = nullptr;  // kStatusWords device ints after the lengths (zeroed at init)
   float* d_signs = nullptr;
   float* d_S = nullptr;
   float* d_St = nullptr;

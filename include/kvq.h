@@ -138,6 +138,35 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
 kvq_status kvq_decode_attention_static(const kvq_cache* c, const void* q, kvq_dtype dtype,
                                        float* out, void* stream);
 
+/* Bits of the cache's device status word. The tensor-core decode kernel bounds every wait for
+ * staged cache data (about one second of SM clock); a wait that gives up sets
+ * KVQ_STATUS_WAIT_TIMEOUT, the kernel still runs to its end and returns, and the output of that
+ * call is not to be trusted. No kernel sets any other bit. */
+#define KVQ_STATUS_WAIT_TIMEOUT 1
+
+/* Read the cache's device status word (the bits above) into *status (host). Enqueues a 4-byte
+ * copy on `stream` and waits for the stream, so it reports on all work enqueued before it.
+ * Only kvq_cache_init clears the word. Not part of the method: a failure-detection aid. */
+kvq_status kvq_cache_status(const kvq_cache* c, int32_t* status, void* stream);
+
+/* Test entry for the bounded waits (no counterpart in the method): the same call as
+ * kvq_decode_attention, except that every CTA of the tensor-core decode kernel first waits on
+ * a barrier that nothing ever completes, giving up after wait_limit_cycles SM clock cycles
+ * (1 ... 2^31). It then carries on as usual, so the output equals kvq_decode_attention's and
+ * KVQ_STATUS_WAIT_TIMEOUT is set. Caches that decode without that kernel (query groups of 8,
+ * FP4) return KVQ_ERR_UNSUPPORTED and launch nothing. */
+kvq_status kvq_debug_decode_unset_wait(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
+                                       void* workspace, size_t ws_bytes, int64_t wait_limit_cycles,
+                                       void* stream);
+
+/* Measurement entry (no counterpart in the method): kvq_decode_attention, recording four
+ * caller-created CUDA events (cudaEvent_t, passed as void*) on `stream`: events[0] before the
+ * first kernel, events[1] after the query prep (right before the split kernel where there is no
+ * prep), events[2] after the split kernel, events[3] after the reduce. The events sit between the
+ * kernels, so the kernels cannot overlap their neighbours as they do in kvq_decode_attention. */
+kvq_status kvq_debug_decode_timed(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
+                                  void* workspace, size_t ws_bytes, void* stream, void* const* events);
+
 /* Host copy of the current per-sequence lengths (lens: host array of `batch` entries). */
 kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens);
 

@@ -239,6 +239,38 @@ def test_launch_counts_per_call():
         cache.close()
 
 
+# ---------------------------------------------------------------- bounded waits
+
+def test_bounded_wait_sets_status_and_returns():
+    """Every wait of the tensor-core decode kernel is bounded. The test entry adds one wait on a
+    barrier that nothing completes: each CTA gives up after ~1e5 cycles, sets the status bit and
+    carries on, so the call returns, its output equals the plain call's, and the cache reports
+    KVQ_STATUS_WAIT_TIMEOUT. No GPU fault is involved: the wait simply runs out."""
+    w = WORKLOADS["llama8b"]
+    data = generate(w, DEV, seqs=range(2), ctx=300)
+    cache, _, _ = new_cache(w, 2, 320)
+    cache.quantize(data["k"], data["v"])
+    ref = cache.decode(data["q"])
+    assert kvq.kvq_cache_status(cache.handle) == 0
+    out = torch.empty_like(ref)
+    kvq.kvq_debug_decode_unset_wait(cache.handle, data["q"], out, cache.workspace, 100000)
+    assert kvq.kvq_cache_status(cache.handle) == kvq.KVQ_STATUS_WAIT_TIMEOUT
+    assert torch.equal(out, ref)
+    cache.close()
+    # no tensor-core kernel for groups of 8: the test entry refuses and launches nothing
+    w70 = WORKLOADS["llama70b"]
+    d70 = generate(w70, DEV, seqs=range(1), ctx=64)
+    c70, _, _ = new_cache(w70, 1, 64)
+    c70.quantize(d70["k"], d70["v"])
+    n0 = kvq.kvq_kernel_launches()
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_debug_decode_unset_wait(c70.handle, d70["q"], torch.empty(1, 64, 128, device=DEV),
+                                        c70.workspace, 100000)
+    assert e.value.status == 2 and kvq.kvq_kernel_launches() == n0
+    assert kvq.kvq_cache_status(c70.handle) == 0
+    c70.close()
+
+
 # ---------------------------------------------------------------- errors
 
 def test_capacity_overflow_writes_nothing():
