@@ -63,7 +63,11 @@ def parse():
 # DRAM bytes (read + write) of one launch of the split decode kernel, from an ncu capture of the
 # workload named here. The record only counts while the kernel's sources are the ones captured
 # (their SHA-256 below); after any change the bench reports null until a new capture.
-TRAFFIC = {}
+TRAFFIC = {
+    "llama8b": {"kernel": "decode_lm_mma<4, 2, 1, 2, 1>", "dram_bytes": 113742080,  # 109.520896 + 4.221184 MB
+                "profile": "profiles/decode_lm_mma_llama8b.md",
+                "sources_sha256": "316fa78548ffaba5d8778e75a1e0822e2fd7c33d223be9be5d1adb6849f1dfbc"},
+}
 TRAFFIC_SOURCES = ("bit_kv_cache_seeded_b200/csrc/kvq_decode_mma.cu", "bit_kv_cache_seeded_b200/csrc/kvq_async.cuh",
                    "bit_kv_cache_seeded_b200/csrc/kvq_internal.h")
 
