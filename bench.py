@@ -64,9 +64,9 @@ def parse():
 # workload named here. The record only counts while the kernel's sources are the ones captured
 # (their SHA-256 below); after any change the bench reports null until a new capture.
 TRAFFIC = {
-    "llama8b": {"kernel": "decode_lm_mma<4, 2, 1, 2, 1>", "dram_bytes": 113742080,  # 109.520896 + 4.221184 MB
+    "llama8b": {"kernel": "decode_lm_mma<4, 2, 1, 2, 1>", "dram_bytes": 114141696,  # 109.523200 + 4.618496 MB
                 "profile": "profiles/decode_lm_mma_llama8b.md",
-                "sources_sha256": "316fa78548ffaba5d8778e75a1e0822e2fd7c33d223be9be5d1adb6849f1dfbc"},
+                "sources_sha256": "702734a8b3ffe10db97adb712ea7a0b4e75dc5cfde7ca6167719d0043bc49b26"},
 }
 TRAFFIC_SOURCES = ("bit_kv_cache_seeded_b200/csrc/kvq_decode_mma.cu", "bit_kv_cache_seeded_b200/csrc/kvq_async.cuh",
                    "bit_kv_cache_seeded_b200/csrc/kvq_internal.h")
@@ -344,12 +344,13 @@ def run_ours(args, world, rank, local):
     lens0 = int(caches[0].lengths()[0])
 
     def step(i, timed_idx=None):
+        # one decode step through the fused entry: append the new token of every sequence and
+        # attend (kvq_decode_step = kvq_quantize + kvq_decode_attention, prep overlapping the append)
         c = caches[i % replicas]
         k_new, v_new = news[i]
-        c.quantize(k_new, v_new)
         if timed_idx is not None:
             ev[timed_idx][0].record(stream)
-        c.decode(q, out)
+        c.step(k_new, v_new, q, out)
         if timed_idx is not None:
             ev[timed_idx][1].record(stream)
 
@@ -380,7 +381,7 @@ def run_ours(args, world, rank, local):
     value = sum_over_ranks(kv_tokens, world) / (elapsed_ms / 1e3)
 
     # Per-kernel device times: the same decode through the measurement entry, which records CUDA
-    # events between its kernels (prep | split kernel | reduce), rotating over the replicas.
+    # events between its kernels (prep | split kernel | separate reduce, if any), rotating over the replicas.
     n_k = min(args.steps, 50)
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_k)]
     torch.cuda.synchronize()
@@ -415,8 +416,7 @@ def run_ours(args, world, rank, local):
         dev_k.copy_(host_news[j][0], non_blocking=True)
         dev_v.copy_(host_news[j][1], non_blocking=True)
         dev_q.copy_(host_q, non_blocking=True)
-        c.quantize(dev_k, dev_v)
-        c.decode(dev_q, out)
+        c.step(dev_k, dev_v, dev_q, out)
         host_out.copy_(out, non_blocking=True)
         e2e_tokens += w.batch * int(c.lengths()[0])
     t1.record(stream)
@@ -430,10 +430,21 @@ def run_ours(args, world, rank, local):
 
     peaks, peak_kind = measured_peaks()
     bytes_step = w.batch * heads_kv * (lens0 + 1) * per_tok  # packed bytes one decode call reads
-    achieved_call = bytes_step / (dec_ms / 1e3) / 1e9
+    call_ms = sum(kern_ms)  # kvq_decode_attention alone, from the per-kernel events
+    achieved_call = bytes_step / (call_ms / 1e3) / 1e9
     bytes_kernel = w.batch * heads_kv * lens_k * per_tok      # the split kernel's algorithmic bytes
-    achieved = bytes_kernel / (kern_ms[1] / 1e3) / 1e9
-    peak = float(peaks["hbm_gbs"])
+    if w.k_mode == "fp4":
+        # 64 heads x (latent + rope) MACs for the logits and 64 x latent for the values, per token:
+        # a dense contraction (146 GFLOP at 2^20 tokens), so the tensor roofline bounds it. The
+        # kernel runs back to back for tens of ms: the sustained bf16 (= f16) figure applies.
+        flops_kernel = 2.0 * w.batch * w.n_q_heads * (2 * w.latent_dim + w.rope_dim) * lens_k
+        roof = {"bound": "tensor", "achieved": flops_kernel / (kern_ms[1] / 1e3) / 1e12,
+                "peak": float(peaks["bf16_tflops_sustained"]), "unit": "TFLOP/s",
+                "flops_per_launch": flops_kernel, "hbm_gbs_of_kernel": bytes_kernel / (kern_ms[1] / 1e3) / 1e9}
+    else:
+        roof = {"bound": "hbm", "achieved": bytes_kernel / (kern_ms[1] / 1e3) / 1e9,
+                "peak": float(peaks["hbm_gbs"]), "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
     line = {
         "metric": METRIC,
         "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -443,11 +454,11 @@ def run_ours(args, world, rank, local):
         "config": workload_config(w, world),
         "l2_detail": f"{replicas} cache replicas x {bytes_prefix / 1e6:.1f} MB rotated per step",
         "hbm_gbs": achieved_call, "frac_of_8tbs": achieved_call / 8000.0,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic_record(w), "peak_kind": peak_kind,
-                     "kernel": "split decode kernel (decode_lm_mma / decode_mla_mma)",
-                     "bytes_per_launch": bytes_kernel, "ms_per_launch": kern_ms[1]},
-        "decode_call": {"ms": dec_ms, "bytes": bytes_step, "gbs": achieved_call,
+        "roofline": dict(roof, traffic=traffic_record(w), peak_kind=peak_kind,
+                         kernel="split decode kernel (decode_lm_mma / decode_mla_mma)",
+                         bytes_per_launch=bytes_kernel, ms_per_launch=kern_ms[1]),
+        "step_events_ms": dec_ms,
+        "decode_call": {"ms": call_ms, "bytes": bytes_step, "gbs": achieved_call,
                         "kernels_ms": {"prep": kern_ms[0], "split": kern_ms[1], "reduce": kern_ms[2]}},
         "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},

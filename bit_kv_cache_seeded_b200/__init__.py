@@ -33,7 +33,7 @@ EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "k
            "kvq_quantize", "kvq_workspace_bytes", "kvq_decode_attention", "kvq_cache_lengths",
            "kvq_cache_layout", "kvq_lloyd_max_table", "kvq_cache_destroy",
            "kvq_debug_quantize_rotated", "kvq_decode_attention_static", "kvq_kernel_launches",
-           "kvq_cache_status", "kvq_debug_decode_unset_wait", "kvq_debug_decode_timed")
+           "kvq_cache_status", "kvq_debug_decode_unset_wait", "kvq_debug_decode_timed", "kvq_decode_step")
 KVQ_STATUS_WAIT_TIMEOUT = 1
 
 
@@ -82,6 +82,7 @@ def load() -> ctypes.CDLL:
         "kvq_cache_status": ([VP, VP, VP], I32),
         "kvq_debug_decode_unset_wait": ([VP, VP, I32, VP, VP, SZ, ctypes.c_int64, VP], I32),
         "kvq_debug_decode_timed": ([VP, VP, I32, VP, VP, SZ, VP, VP], I32),
+        "kvq_decode_step": ([VP, VP, VP, VP, I32, VP, VP, SZ, VP], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -186,6 +187,20 @@ def kvq_decode_attention(handle, q: torch.Tensor, out: torch.Tensor, workspace: 
     st = load().kvq_decode_attention(handle, _ptr(q), DTYPES[q.dtype], _ptr(out), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check("kvq_decode_attention", st)
+
+
+def kvq_decode_step(handle, K: torch.Tensor, V: torch.Tensor, q: torch.Tensor, out: torch.Tensor,
+                    workspace: torch.Tensor, stream=None):
+    """Append one token per sequence (K, V [B, Hkv, 1, d]; FP4: latent, rope) and decode with q."""
+    if K.dtype != V.dtype or K.dtype != q.dtype or q.dtype not in DTYPES or out.dtype != torch.float32:
+        raise TypeError("K, V and q must share float32/bfloat16; out is float32")
+    if not (K.is_contiguous() and V.is_contiguous() and q.is_contiguous() and out.is_contiguous()):
+        raise ValueError("K, V, q and out must be contiguous")
+    if K.shape[-2] != 1 or V.shape[-2] != 1:
+        raise ValueError("a decode step appends exactly one token per sequence")
+    st = load().kvq_decode_step(handle, _ptr(K), _ptr(V), _ptr(q), DTYPES[q.dtype], _ptr(out), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("kvq_decode_step", st)
 
 
 def kvq_decode_attention_static(handle, q: torch.Tensor, out: torch.Tensor, stream=None):
@@ -294,6 +309,14 @@ class KvqCache:
 
     def quantize(self, K, V, seq_ids=None, stream=None):
         kvq_quantize(self.handle, K, V, seq_ids, stream)
+
+    def step(self, K, V, q, out=None, stream=None):
+        """Append one token per sequence and decode (kvq_decode_step); returns out."""
+        if out is None:
+            out = torch.empty((self.batch, self.cfg.n_q_heads, self.out_dim), dtype=torch.float32,
+                              device=q.device)
+        kvq_decode_step(self.handle, K, V, q, out, self.workspace, stream)
+        return out
 
     def decode(self, q, out=None, stream=None):
         if out is None:

@@ -320,6 +320,42 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
   return KVQ_OK;
 }
 
+}  // extern "C"
+
+namespace {
+// Quantize parameters for sequences [first, first + cnt) of the call (seq_ids may be null: all).
+void fill_quantize(QuantizeParams& p, const kvq_cache* c, const void* K, const void* V, kvq_dtype dtype,
+                   int n_new, const int32_t* seq_ids, int first, int cnt) {
+  const int heads = c->is_fp4 ? 1 : c->cfg.n_kv_heads;
+  const size_t elem = dtype == KVQ_BF16 ? 2 : 4;
+  const size_t per_seq_k = c->is_fp4 ? (size_t)n_new * c->cfg.latent_dim : (size_t)heads * n_new * kHeadDim;
+  const size_t per_seq_v = c->is_fp4 ? (size_t)n_new * c->cfg.rope_dim : per_seq_k;
+  std::memset(&p, 0, sizeof(p));
+  p.src[0] = static_cast<const char*>(K) + first * per_seq_k * elem;
+  p.src[1] = static_cast<const char*>(V) + first * per_seq_v * elem;
+  p.bf16 = dtype == KVQ_BF16;
+  p.n_new = n_new;
+  p.n_seq = cnt;
+  p.heads = heads;
+  p.region[0] = c->d_k;
+  p.region[1] = c->d_v;
+  p.tiles_per_seq = c->tiles_per_seq;
+  p.side[0] = c->k;
+  p.side[1] = c->v;
+  p.fp4 = c->fp4;
+  p.signs = c->d_signs;
+  p.St = c->d_St;
+  p.lens = c->d_lens;
+  for (int i = 0; i < cnt; ++i) {
+    const int sid = seq_ids ? seq_ids[first + i] : first + i;
+    p.seq[i] = sid;
+    p.pos[i] = c->lens[sid];
+  }
+}
+}  // namespace
+
+extern "C" {
+
 kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dtype,
                         int32_t n_new, const int32_t* seq_ids, int32_t n_seq, void* stream) {
   if (!c || n_new < 0 || n_seq < 0) return KVQ_ERR_INVALID_ARG;
@@ -337,34 +373,10 @@ kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dt
     if ((long)c->lens[sid] + n_new > (long)c->capacity) return KVQ_ERR_CAPACITY;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int heads = c->is_fp4 ? 1 : c->cfg.n_kv_heads;
-  const size_t elem = dtype == KVQ_BF16 ? 2 : 4;
-  const size_t per_seq_k = c->is_fp4 ? (size_t)n_new * c->cfg.latent_dim : (size_t)heads * n_new * kHeadDim;
-  const size_t per_seq_v = c->is_fp4 ? (size_t)n_new * c->cfg.rope_dim : per_seq_k;
   for (int first = 0; first < n_seq; first += kMaxSeqPerLaunch) {
     const int cnt = std::min(kMaxSeqPerLaunch, n_seq - first);
     QuantizeParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.src[0] = static_cast<const char*>(K) + first * per_seq_k * elem;
-    p.src[1] = static_cast<const char*>(V) + first * per_seq_v * elem;
-    p.bf16 = dtype == KVQ_BF16;
-    p.n_new = n_new;
-    p.n_seq = cnt;
-    p.heads = heads;
-    p.region[0] = c->d_k;
-    p.region[1] = c->d_v;
-    p.tiles_per_seq = c->tiles_per_seq;
-    p.side[0] = c->k;
-    p.side[1] = c->v;
-    p.fp4 = c->fp4;
-    p.signs = c->d_signs;
-    p.St = c->d_St;
-    p.lens = c->d_lens;
-    for (int i = 0; i < cnt; ++i) {
-      const int sid = seq_ids ? seq_ids[first + i] : first + i;
-      p.seq[i] = sid;
-      p.pos[i] = c->lens[sid];
-    }
+    fill_quantize(p, c, K, V, dtype, n_new, seq_ids, first, cnt);
     const cudaError_t e = c->is_fp4 ? launch_quantize_fp4(p, s) : launch_quantize_lm(p, 2, s);
     if (e != cudaSuccess) return KVQ_ERR_CUDA;
     for (int i = 0; i < cnt; ++i) c->lens[p.seq[i]] += n_new;
@@ -386,7 +398,7 @@ namespace {
 // decode CTA first waits, bounded by wait_limit cycles, on a barrier that nothing completes).
 kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out, void* workspace,
                        size_t ws_bytes, void* stream, int debug_unset_wait, long long wait_limit,
-                       const cudaEvent_t* ev = nullptr) {
+                       const cudaEvent_t* ev = nullptr, const QuantizeParams* qp = nullptr) {
   if (!c || !q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
   if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
@@ -417,6 +429,8 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
     p.tiles_per_seq = c->tiles_per_seq;
     p.fp4 = c->fp4;
     p.logit_scale = default_scale(c->cfg) * log2e;
+    p.err = c->d_status;
+    p.wait_limit = wait_limit;
     if (!rec(1) || launch_decode_mla(p, s) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
     if (launch_reduce_mla(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
     return KVQ_OK;
@@ -449,8 +463,13 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.err = c->d_status;
   p.wait_limit = wait_limit;
   p.debug_unset_wait = debug_unset_wait;
+  if (qp && !mma_decode_supported(p)) {  // no fused front kernel on this path: append first
+    if (launch_quantize_lm(*qp, 2, s) != cudaSuccess) return KVQ_ERR_CUDA;
+    qp = nullptr;
+  }
+  p.cache_after_wait = qp != nullptr;
   if (debug_unset_wait && !mma_decode_supported(p)) return KVQ_ERR_UNSUPPORTED;
-  if (launch_decode_lm(p, s, ev ? ev[1] : nullptr) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
+  if (launch_decode_lm(p, s, ev ? ev[1] : nullptr, qp) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
   if (launch_reduce_lm(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }
@@ -461,6 +480,34 @@ extern "C" {
 kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
                                 void* workspace, size_t ws_bytes, void* stream) {
   return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles);
+}
+
+kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
+                           float* out, void* workspace, size_t ws_bytes, void* stream) {
+  if (!c || !K || !V || !q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+  if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(q) || !aligned16(out) || !aligned16(workspace))
+    return KVQ_ERR_ALIGNMENT;
+  // everything both halves check, with the lengths after the append, before anything is written
+  int max_len = 0;
+  for (int v : c->lens) {
+    if ((long)v + 1 > (long)c->capacity) return KVQ_ERR_CAPACITY;
+    max_len = std::max(max_len, v);
+  }
+  const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
+  int splits, chunk;
+  plan_splits(pairs, c->sms, decode_slots_per_sm(c), decode_max_units(c), decode_waves_bound(c), max_len + 1,
+              &splits, &chunk);
+  if (ws_bytes < workspace_for(c, splits)) return KVQ_ERR_WORKSPACE;
+  if (c->is_fp4 || c->batch > kMaxSeqPerLaunch) {  // no fused front kernel: the two calls in sequence
+    const kvq_status st = kvq_quantize(c, K, V, dtype, 1, nullptr, c->batch, stream);
+    if (st != KVQ_OK) return st;
+    return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles);
+  }
+  QuantizeParams qp;
+  fill_quantize(qp, c, K, V, dtype, 1, nullptr, 0, c->batch);
+  for (int i = 0; i < c->batch; ++i) c->lens[i] += 1;  // the plan of the decode sees the new lengths
+  return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles, nullptr, &qp);
 }
 
 kvq_status kvq_debug_decode_unset_wait(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,

@@ -374,8 +374,9 @@ cudaError_t dispatch_modes(const DecodeParams& p, dim3 grid, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid) {
-  if (mma_decode_supported(p)) return launch_decode_lm_mma(p, s, ev_mid);
+cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
+  if (mma_decode_supported(p)) return launch_decode_lm_mma(p, s, ev_mid, qp);
+  if (qp) return cudaErrorNotSupported;
   if (ev_mid && cudaEventRecord(ev_mid, s) != cudaSuccess) return cudaErrorUnknown;
   dim3 grid(p.splits, p.Hkv, p.B);
   switch (p.group) {

@@ -38,6 +38,7 @@
 
 #include "kvq_async.cuh"
 #include "kvq_internal.h"
+#include "kvq_quantize_lm.cuh"
 
 namespace kvq {
 namespace {
@@ -58,7 +59,7 @@ constexpr float kRoundBias = 8388608.f;              // x + 2^23 (0 <= x < 2^23)
 // A int8, B uint8 (the value-phase weight digits are non-negative bytes).
 __device__ __forceinline__ void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
@@ -75,7 +76,7 @@ __device__ __forceinline__ uint32_t pack_byte(uint32_t x0, uint32_t x1, uint32_t
 
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};\n"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
@@ -121,6 +122,23 @@ __device__ __forceinline__ void walsh_coeffs(int bits, const float* c, float (&a
   }
 }
 
+// Byte layout of one 32-token tile of a side with BITS code planes (and a sketch when QJL), as the
+// host lays it out (kvq_api.cu make_side): planes, sketch words, fp16 norms, fp16 residual norms.
+// Compile-time here so that every shared-memory address in the decode kernel is an immediate
+// offset; launch_mma() refuses a cache whose runtime layout differs.
+template <int BITS, bool QJL>
+struct TileLayout {
+  static constexpr int PLANES = 0;
+  static constexpr int SKETCH = BITS * kTile * 16;
+  static constexpr int NORM = SKETCH + (QJL ? kTile * 16 : 0);
+  static constexpr int GAMMA = NORM + kTile * 2;
+  static constexpr int BYTES = (GAMMA + (QJL ? kTile * 2 : 0) + 15) / 16 * 16;
+  static bool matches(const SideLayout& L) {
+    return L.off_planes == PLANES && L.off_sketch == SKETCH && L.off_norm == NORM &&
+           (!QJL || L.off_gamma == GAMMA) && L.tile_bytes == BYTES && L.bits == BITS && L.qjl == QJL;
+  }
+};
+
 template <int G, int KB, bool KQ, int VB, bool VQ>
 struct MmaCfg {
   static constexpr int KP = Walsh<KB>::P + (KQ ? 1 : 0);  // logit planes (sketch last)
@@ -142,7 +160,7 @@ struct MmaCfg {
 // sum_j q~_j and Cz = -sum_j s~_j. Fragment order of coordinate j: (j%8)*16 + (j/32)*4 + (j%32)/8.
 // ------------------------------------------------------------------------------------------
 template <int G, int KB, bool KQ>
-__global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constant__ DecodeParams p) {
+__device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b) {
   constexpr int KP = Walsh<KB>::P + (KQ ? 1 : 0);
   constexpr int KWP = Walsh<KB>::P;
   __shared__ __align__(16) float qf[G][kHeadDim];
@@ -150,14 +168,12 @@ __global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constan
   __shared__ float hc[G][4];
   __shared__ float qscale[G][2];                 // 32639 / vmax: centroid planes, sketch
   extern __shared__ __align__(16) float st_s[];  // [128][m] transposed sketch matrix
-  const int hk = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned char* out = p.qprep + ((size_t)b * p.Hkv + hk) * p.qprep_stride;
   if (KQ) {  // staged while the queries are rotated
     for (int c = tid; c < kHeadDim * kHeadDim / 4; c += kThreadsM) cp_async16(st_s + 4 * c, p.St + 4 * c);
     cp_async_commit();
   }
-  grid_dep_launch();  // the decode kernel may be scheduled now; it waits before reading this output
   const float qcoef = kInvSqrtD * p.logit_scale * kInvSqrtD;
   for (int h = warp; h < G; h += kWarpsM) {
     float u[4];
@@ -251,6 +267,29 @@ __global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constan
   }
 }
 
+template <int G, int KB, bool KQ>
+__global__ void __launch_bounds__(kThreadsM) decode_lm_prep(const __grid_constant__ DecodeParams p) {
+  grid_dep_launch();  // the decode kernel may be scheduled now; it waits before reading this output
+  prep_block<G, KB, KQ>(p, blockIdx.x, blockIdx.y);
+}
+
+// Front kernel of a fused decode step (kvq_decode_step): blocks 0 .. 2 nq - 1 append the new
+// token of every sequence (K side, then V side: qlm::quantize_lm_block), the remaining B x Hkv
+// blocks compute the query prep. The two parts are independent, so they share one launch and
+// overlap; the decode kernel, a programmatic dependent of this one, waits for all of it.
+template <int G, int KB, bool KQ>
+__global__ void __launch_bounds__(kThreadsM)
+decode_front(const __grid_constant__ QuantizeParams qp, const __grid_constant__ DecodeParams p, int nq) {
+  grid_dep_launch();
+  const int blk = blockIdx.x;
+  if (blk < 2 * nq) {
+    qlm::quantize_lm_block(qp, blk / nq, blk % nq, nq);
+  } else {
+    const int r = blk - 2 * nq;
+    prep_block<G, KB, KQ>(p, r % p.Hkv, r / p.Hkv);
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // Decode kernel (two passes over the CTA's chunk).
 // ------------------------------------------------------------------------------------------
@@ -270,8 +309,10 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t mbar[kStagesM + 1];  // per stage (+ one nothing completes: test entry)
   __shared__ int s_fail;                             // a wait of this CTA gave up
-  const int ktb = p.k.tile_bytes, vtb = p.v.tile_bytes;
-  const int stage_bytes = max(2 * ktb + kNormBlock, 2 * vtb);
+  using KL = TileLayout<KB, KQ>;
+  using VL = TileLayout<VB, VQ>;
+  constexpr int ktb = KL::BYTES, vtb = VL::BYTES;
+  constexpr int stage_bytes = (2 * ktb + kNormBlock > 2 * vtb) ? 2 * ktb + kNormBlock : 2 * vtb;
   unsigned char* stages = smem;                                            // [kStagesM][2 tiles (+ norms)]
   float* lgs = reinterpret_cast<float*>(stages + kStagesM * stage_bytes);  // [G][kLgStride] logits
   unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * kLgStride);  // [2][NKIND][VNCOL][kPdStride]
@@ -280,7 +321,10 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int len = p.lens[b];
+  // In a fused append + decode step the cache (and len) are written by the append kernel that
+  // runs before the prep: everything that reads them waits for the prep (which waits for it).
+  if (p.cache_after_wait) grid_dep_wait();
+  const int len = __ldcg(p.lens + b);  // through L2: a predecessor may have written it
   const int t_begin = split * p.chunk;
   const int t_end = min(len, t_begin + p.chunk);
   const size_t pair = (size_t)b * p.Hkv + hk;
@@ -314,7 +358,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       bulk_g2s(smem_addr(dst), kbase + (size_t)tile0 * ktb, 2u * ktb, bar);
 #pragma unroll
       for (int tile = 0; tile < 2; ++tile)
-        bulk_g2s(smem_addr(dst + 2 * ktb + tile * 128), vbase + (size_t)(tile0 + tile) * vtb + p.v.off_norm, nb, bar);
+        bulk_g2s(smem_addr(dst + 2 * ktb + tile * 128), vbase + (size_t)(tile0 + tile) * vtb + VL::NORM, nb, bar);
     } else {
       const int tile0 = (t_begin + (f - n_iter) * kCtaTok) / kTile;
       mbar_arrive_expect_tx(bar, 2u * vtb);
@@ -322,7 +366,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     }
   };
   auto wait_fill = [&](int f) {  // every thread
-    if (!mbar_wait(smem_addr(&mbar[f % kStagesM]), (uint32_t)(f / kStagesM) & 1u, p.wait_limit)) {
+    const uint32_t bar = smem_addr(&mbar[f % kStagesM]), par = (uint32_t)(f / kStagesM) & 1u;
+    if (!mbar_try(bar, par) && !mbar_wait(bar, par, p.wait_limit)) {
       s_fail = 1;
       atomicOr(p.err, 1);
     }
@@ -335,10 +380,12 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     atomicOr(p.err, 1);
   }
 
-  // logit-phase B fragments (query digits) and head constants from the prep area
+  // logit-phase B fragments (query digits) and head constants from the prep area (written by the
+  // predecessor kernel while this one may already run: loaded through L2, not the read-only path)
   // Launched as a programmatic dependent of the prep kernel: the cache tiles staged above were
-  // complete before prep started; the prep output is read only after this wait.
-  grid_dep_wait();
+  // complete before prep started (unless cache_after_wait, handled above); the prep output is read
+  // only after this wait.
+  if (!p.cache_after_wait) grid_dep_wait();
   const unsigned char* prep = p.qprep + pair * p.qprep_stride;
   uint32_t qb[KP][4][KNT][2];
 #pragma unroll
@@ -350,8 +397,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         const int n = nt * 8 + g, h = n / 2, d = n % 2;  // column = (head, digit)
         if (h < G) {
           const unsigned char* row = prep + ((P * G + h) * 2 + d) * 128;
-          qb[P][m][nt][0] = __ldg(reinterpret_cast<const uint32_t*>(row + ((2 * m) * 4 + t) * 4));
-          qb[P][m][nt][1] = __ldg(reinterpret_cast<const uint32_t*>(row + ((2 * m + 1) * 4 + t) * 4));
+          qb[P][m][nt][0] = __ldcg(reinterpret_cast<const uint32_t*>(row + ((2 * m) * 4 + t) * 4));
+          qb[P][m][nt][1] = __ldcg(reinterpret_cast<const uint32_t*>(row + ((2 * m + 1) * 4 + t) * 4));
         } else {
           qb[P][m][nt][0] = qb[P][m][nt][1] = 0u;
         }
@@ -362,10 +409,10 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
   for (int nt = 0; nt < KNT; ++nt) {
     const int h = min(4 * nt + t, G - 1);
-    hs[nt] = __ldg(hconst + h * 4 + 0);
-    hc[nt] = __ldg(hconst + h * 4 + 1);
-    hsz[nt] = __ldg(hconst + h * 4 + 2);
-    hcz[nt] = __ldg(hconst + h * 4 + 3);
+    hs[nt] = __ldcg(hconst + h * 4 + 0);
+    hc[nt] = __ldcg(hconst + h * 4 + 1);
+    hsz[nt] = __ldcg(hconst + h * 4 + 2);
+    hcz[nt] = __ldcg(hconst + h * 4 + 3);
   }
   const float vkappa = VQ ? kSqrtHalfPi / (float)p.v.m : 0.f;
 
@@ -392,7 +439,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) { acc[m][nt][c] = 0; if (m < 2) accz[m][nt][c] = 0; }
       uint32_t w0[3] = {0u, 0u, 0u}, w1[3] = {0u, 0u, 0u};
-      const unsigned char* kp = ktile + p.k.off_planes + t * 4;
+      const unsigned char* kp = ktile + KL::PLANES + t * 4;
 #pragma unroll
       for (int pp = 0; pp < KB; ++pp) {
         w0[pp] = *reinterpret_cast<const uint32_t*>(kp + pp * (kTile * 16) + s0 * 16);
@@ -403,8 +450,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         const bool sk = KQ && P == KP - 1;
         uint32_t x0, x1;
         if (sk) {
-          x0 = *reinterpret_cast<const uint32_t*>(ktile + p.k.off_sketch + s0 * 16 + t * 4);
-          x1 = *reinterpret_cast<const uint32_t*>(ktile + p.k.off_sketch + s1 * 16 + t * 4);
+          x0 = *reinterpret_cast<const uint32_t*>(ktile + KL::SKETCH + s0 * 16 + t * 4);
+          x1 = *reinterpret_cast<const uint32_t*>(ktile + KL::SKETCH + s1 * 16 + t * 4);
         } else {
           x0 = walsh_word<KB>(w0, P);
           x1 = walsh_word<KB>(w1, P);
@@ -425,12 +472,12 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
           }
         }
       }
-      const float nk0 = __half2float(*reinterpret_cast<const __half*>(ktile + p.k.off_norm + s0 * 2));
-      const float nk1 = __half2float(*reinterpret_cast<const __half*>(ktile + p.k.off_norm + s1 * 2));
+      const float nk0 = __half2float(*reinterpret_cast<const __half*>(ktile + KL::NORM + s0 * 2));
+      const float nk1 = __half2float(*reinterpret_cast<const __half*>(ktile + KL::NORM + s1 * 2));
       float gk0 = 0.f, gk1 = 0.f;
       if (KQ) {
-        gk0 = __half2float(*reinterpret_cast<const __half*>(ktile + p.k.off_gamma + s0 * 2));
-        gk1 = __half2float(*reinterpret_cast<const __half*>(ktile + p.k.off_gamma + s1 * 2));
+        gk0 = __half2float(*reinterpret_cast<const __half*>(ktile + KL::GAMMA + s0 * 2));
+        gk1 = __half2float(*reinterpret_cast<const __half*>(ktile + KL::GAMMA + s1 * 2));
       }
       const bool v0 = tl + g < count, v1 = tl + g + 8 < count;
 #pragma unroll
@@ -442,11 +489,14 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
           c[e] = (acc[0][nt][e] + acc[1][nt][e]) + (acc[2][nt][e] + acc[3][nt][e]);
           cz[e] = accz[0][nt][e] + accz[1][nt][e];
         }
-        float l0 = fmaf(hs[nt], fmaf((float)c[0], 256.f, (float)c[1]), hc[nt]);
-        float l1 = fmaf(hs[nt], fmaf((float)c[2], 256.f, (float)c[3]), hc[nt]);
-        if (KQ) {
-          l0 = fmaf(gk0, fmaf(hsz[nt], fmaf((float)cz[0], 256.f, (float)cz[1]), hcz[nt]), l0);
-          l1 = fmaf(gk1, fmaf(hsz[nt], fmaf((float)cz[2], 256.f, (float)cz[3]), hcz[nt]), l1);
+        // hi * 256 + lo: exact in int32 up to 2 Walsh planes (|hi| < 2^22), else in fp32
+        const float c01 = KB <= 2 ? (float)(c[0] * 256 + c[1]) : fmaf((float)c[0], 256.f, (float)c[1]);
+        const float c23 = KB <= 2 ? (float)(c[2] * 256 + c[3]) : fmaf((float)c[2], 256.f, (float)c[3]);
+        float l0 = fmaf(hs[nt], c01, hc[nt]);
+        float l1 = fmaf(hs[nt], c23, hc[nt]);
+        if (KQ) {  // one sketch plane: |hi| < 2^21
+          l0 = fmaf(gk0, fmaf(hsz[nt], (float)(cz[0] * 256 + cz[1]), hcz[nt]), l0);
+          l1 = fmaf(gk1, fmaf(hsz[nt], (float)(cz[2] * 256 + cz[3]), hcz[nt]), l1);
         }
         const float lg0 = v0 ? nk0 * l0 : -INFINITY, lg1 = v1 ? nk1 * l1 : -INFINITY;
         if (h < G) {
@@ -515,16 +565,16 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     float lv[TPT], wc[TPT], wz[TPT];
     if (TPT == 2) {
       const float2 l2 = *reinterpret_cast<const float2*>(lgs + task_h * kLgStride + tok0 + T);
-      const float2 n2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + p.v.off_norm + (T % kTile) * 2));
+      const float2 n2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::NORM + (T % kTile) * 2));
       lv[0] = l2.x; lv[TPT - 1] = l2.y; wc[0] = n2.x; wc[TPT - 1] = n2.y;
       if (VQ) {
-        const float2 g2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + p.v.off_gamma + (T % kTile) * 2));
+        const float2 g2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::GAMMA + (T % kTile) * 2));
         wz[0] = g2.x; wz[TPT - 1] = g2.y;
       }
     } else {
       lv[0] = lgs[task_h * kLgStride + tok0 + T];
-      wc[0] = __half2float(*reinterpret_cast<const __half*>(vtile + p.v.off_norm + (T % kTile) * 2));
-      if (VQ) wz[0] = __half2float(*reinterpret_cast<const __half*>(vtile + p.v.off_gamma + (T % kTile) * 2));
+      wc[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::NORM + (T % kTile) * 2));
+      if (VQ) wz[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::GAMMA + (T % kTile) * 2));
     }
     uint32_t bc[TPT], bz[TPT];
     float psum = 0.f;
@@ -613,7 +663,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
       for (int pp = 0; pp < VB + (VQ ? 1 : 0); ++pp) {
         const unsigned char* pl =
-            vtile + (pp < VB ? p.v.off_planes + pp * (kTile * 16) : p.v.off_sketch) + 8 * t;
+            vtile + (pp < VB ? VL::PLANES + pp * (kTile * 16) : VL::SKETCH) + 8 * t;
         const uint2 r0 = *reinterpret_cast<const uint2*>(pl + g * kTile);
         const uint2 r1 = *reinterpret_cast<const uint2*>(pl + (g + 8) * kTile);
         xv[pp][0] = r0.x; xv[pp][2] = r0.y;
@@ -720,13 +770,14 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       dst[1] = hsum[h];
     }
   }
+
 }
 
 template <int G, int KB, bool KQ, int VB, bool VQ>
 size_t mma_smem_bytes(const DecodeParams& p) {
   using C = MmaCfg<G, KB, KQ, VB, VQ>;
   constexpr int NKIND = VQ ? 2 : 1;
-  size_t s = (size_t)kStagesM * std::max(2 * p.k.tile_bytes + kNormBlock, 2 * p.v.tile_bytes);
+  size_t s = (size_t)kStagesM * std::max(2 * TileLayout<KB, KQ>::BYTES + kNormBlock, 2 * TileLayout<VB, VQ>::BYTES);
   s += sizeof(float) * (size_t)G * kLgStride;
   s += 2 * (size_t)NKIND * C::VNCOL * kPdStride;
   s += sizeof(float) * (kWarpsM * G + 2 * kWarpsM);
@@ -734,12 +785,21 @@ size_t mma_smem_bytes(const DecodeParams& p) {
 }
 
 template <int G, int KB, bool KQ, int VB, bool VQ>
-cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid) {
+cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
+  if (!TileLayout<KB, KQ>::matches(p.k) || !TileLayout<VB, VQ>::matches(p.v)) return cudaErrorNotSupported;
   const size_t prep_smem = KQ ? sizeof(float) * kHeadDim * kHeadDim : 0;
   cudaError_t e = cudaFuncSetAttribute(decode_lm_prep<G, KB, KQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep_smem);
   if (e != cudaSuccess) return e;
-  decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv, p.B), kThreadsM, prep_smem, s>>>(p);
+  if (qp) {  // fused step: append + prep in one launch
+    const int nq = qlm::blocks_per_side(*qp);
+    const size_t fsmem = std::max(prep_smem, (size_t)sizeof(float) * kHeadDim * kHeadDim);
+    e = cudaFuncSetAttribute(decode_front<G, KB, KQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
+    if (e != cudaSuccess) return e;
+    decode_front<G, KB, KQ><<<2 * nq + p.B * p.Hkv, kThreadsM, fsmem, s>>>(*qp, p, nq);
+  } else {
+    decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv, p.B), kThreadsM, prep_smem, s>>>(p);
+  }
   e = launched();
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
@@ -763,11 +823,11 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid
 }
 
 template <int G>
-cudaError_t dispatch_mma_modes(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid) {
+cudaError_t dispatch_mma_modes(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
   const int kb = p.k.bits, vb = p.v.bits;
   const bool kq = p.k.qjl, vq = p.v.qjl;
 #define KVQ_MMA_CASE(KB, KQ, VB, VQ) \
-  if (kb == KB && kq == KQ && vb == VB && vq == VQ) return launch_mma<G, KB, KQ, VB, VQ>(p, s, ev_mid);
+  if (kb == KB && kq == KQ && vb == VB && vq == VQ) return launch_mma<G, KB, KQ, VB, VQ>(p, s, ev_mid, qp);
   KVQ_MMA_CASE(2, true, 2, true)
   KVQ_MMA_CASE(3, true, 3, false)
   KVQ_MMA_CASE(1, false, 1, false)
@@ -792,11 +852,11 @@ bool mma_decode_supported(const DecodeParams& p) {
          p.chunk <= kChunkMax && p.qprep != nullptr;
 }
 
-cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid) {
+cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
   switch (p.group) {
-    case 1: return dispatch_mma_modes<1>(p, s, ev_mid);
-    case 2: return dispatch_mma_modes<2>(p, s, ev_mid);
-    case 4: return dispatch_mma_modes<4>(p, s, ev_mid);
+    case 1: return dispatch_mma_modes<1>(p, s, ev_mid, qp);
+    case 2: return dispatch_mma_modes<2>(p, s, ev_mid, qp);
+    case 4: return dispatch_mma_modes<4>(p, s, ev_mid, qp);
     default: return cudaErrorNotSupported;
   }
 }

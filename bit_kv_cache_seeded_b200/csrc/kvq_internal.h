@@ -85,6 +85,7 @@ struct DecodeParams {
   int* err;               // cache status word: bit 0 set when a wait for staged data gave up
   long long wait_limit;   // SM clock cycles a kernel waits for staged data before giving up
   int debug_unset_wait;   // test entry: also wait once on a barrier nothing completes
+  int cache_after_wait;   // fused step: the cache is written by this kernel's predecessor (wait first)
 };
 
 struct MlaParams {
@@ -99,6 +100,8 @@ struct MlaParams {
   int tiles_per_seq;
   Fp4Layout fp4;
   float logit_scale;      // softmax_scale * log2(e)
+  int* err;               // cache status word (bit 0: a bounded wait gave up)
+  long long wait_limit;   // SM clock cycles a kernel waits before giving up
 };
 
 // Reads cudaGetLastError() right after a kernel launch and, when it is cudaSuccess, adds one to
@@ -110,14 +113,19 @@ cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_
 cudaError_t launch_quantize_fp4(const QuantizeParams& p, cudaStream_t s);
 // ev_mid (may be null) is recorded between the query prep and the split kernel (right before the
 // split kernel when there is no prep).
-cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid = nullptr);
+// qp (may be null): a fused decode step's append, launched together with the query prep in one
+// kernel (tensor-core path only; the caller checks mma_decode_supported).
+cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid = nullptr,
+                             const QuantizeParams* qp = nullptr);
 bool mma_decode_supported(const DecodeParams& p);
 int mma_prep_bytes(int k_bits, int k_qjl, int group);  // bytes of one (sequence, kv-head) prep area
-cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid);
+cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp);
 cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s);
 bool mla_mma_supported(const MlaParams& p);
+bool mla_umma_supported(const MlaParams& p);
+cudaError_t launch_decode_mla_umma(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_decode_mla_mma(const MlaParams& p, cudaStream_t s);
 
 // Host Lloyd-Max tables (lloyd_max.cpp): fp64 fixed-point iteration rounded to fp32.

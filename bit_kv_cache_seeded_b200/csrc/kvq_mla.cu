@@ -170,6 +170,7 @@ cudaError_t launch_hpw(const MlaParams& p, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s) {
+  if (mla_umma_supported(p)) return launch_decode_mla_umma(p, s);  // 64 heads: tcgen05
   if (mla_mma_supported(p)) return launch_decode_mla_mma(p, s);
   if (p.fp4.latent != kLat || p.fp4.rope != kRope) return cudaErrorNotSupported;
   switch (p.Hq) {

@@ -1,0 +1,461 @@
+// 5th-generation tensor-core (tcgen05, accumulators in tensor memory) split-K decode attention
+// over the FP4 MLA-style latent cache, for 64 query heads.
+//
+// "How DeepSeek-V4.1-Flash cut KV cache storage by 4x via CSA2": one 512-dim latent per token is
+// shared by all heads (section "CSA2") and stored as FP4 E2M1 with one scale per 16 channels
+// (section "Numerics and hardware efficiency"; the scale is an E4M3 byte here). With the absorbed
+// query q = [q_lat ; q_rope] each 64-token tile is two dense contractions:
+//   S   = Q [64 heads x 576] . K^T [576 x 64 tokens]        (tcgen05.mma M=64, N=64, K=16 steps)
+//   O^T += latent_hat^T [512 x 64 tokens] . P^T [64 x 64]   (tcgen05.mma M=128 x 4, N=64)
+// latent_hat = E4M3 scale x E2M1 value is exact in f16; Q's latent part is scaled per head by a
+// power of two into f16 range, its RoPE part stays bf16 (bf16 MMAs into the same accumulator).
+//
+// One CTA per SM (8 warps; warp w reaches tensor-memory lane quarter w % 4), per 64-token
+// iteration:
+//   1. the packed tile pair arrives by bulk copy (double-buffered, mbarrier-completed);
+//   2. all threads dequantise the latent to f16 and copy the RoPE key into shared memory in the
+//      canonical no-swizzle "core matrix" layout (8 rows x 16 B blocks) both MMAs read;
+//   3. thread 0 issues S = Q K^T into tensor memory and commits to an mbarrier;
+//   4. lanes 0..15 of warps 0..3 (the rows of S for an M=64 MMA) load their head's 64 logits,
+//      update a lazily rescaled running maximum (rescale only when it grows by more than 8 in
+//      log2 units), write P = 2^(l - m) (<= 256) as f16 in core-matrix layout;
+//   5. if a head's maximum moved, every thread rescales that head's column of O^T in tensor
+//      memory (load, multiply, store);
+//   6. thread 0 issues O^T += latent^T P^T and commits; the next iteration waits for it before
+//      it overwrites the latent, P or O.
+// Every mbarrier wait is bounded (the cache status word records a wait that gave up). Partials
+// (m, l, o[512]) per (sequence, head, split) go to the workspace in the format of the other
+// MLA kernels; the same reduce kernel finishes.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kvq_async.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace {
+
+constexpr int kThreadsU = 256;          // 8 warps: warp w reaches tensor-memory lanes 32 (w % 4) ..
+constexpr int kTokU = 64;               // tokens per iteration (two cache tiles)
+constexpr int kLatU = 512, kRopeU = 64, kDqU = kLatU + kRopeU;
+constexpr int kHeadsU = 64;
+constexpr int kCore = 128;              // bytes of one core matrix (8 rows x 16 B)
+constexpr float kLazyRescale = 8.f;     // rescale O only when the running max grows by more than this
+constexpr uint32_t kTmemCols = 512;     // allocation: O^T in columns 0..255, S in 256..319
+constexpr uint32_t kColO = 0, kColS = 256;
+
+// Shared-memory layout (bytes). Q: [8 head groups][72 dim chunks] core matrices; LAT: [8 token
+// groups][64 dim chunks]; ROPE: [8 token groups][8 dim chunks]; P: [8 head groups][8 token chunks].
+constexpr int kOffQ = 0;
+constexpr int kSizeQ = kHeadsU * kDqU * 2;              // 73728
+constexpr int kOffLat = kOffQ + kSizeQ;
+constexpr int kSizeLat = kTokU * kLatU * 2;             // 65536
+constexpr int kOffRope = kOffLat + kSizeLat;
+constexpr int kSizeRope = kTokU * kRopeU * 2;           // 8192
+constexpr int kOffP = kOffRope + kSizeRope;
+constexpr int kSizeP = kHeadsU * kTokU * 2;             // 8192
+constexpr int kOffRaw = kOffP + kSizeP;                 // then 2 raw stages of 2 cache tiles
+
+// ---- tcgen05 / descriptor helpers (PTX ISA 8.7+, sm_100a) ----------------------------------
+
+// Shared-memory matrix descriptor, no swizzle: start address, leading-dimension byte offset
+// (between core matrices along K for K-major operands, along K for MN-major ones too: see the
+// call sites), stride-dimension byte offset, version 1 (tcgen05), layout type 0.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
+  return d;
+}
+
+// Instruction descriptor for kind::f16 with fp32 accumulation.
+//   fmt: 0 = f16, 1 = bf16 (A and B alike); a_mn / b_mn: operand is MN-major; M, N: tile shape.
+__host__ __device__ constexpr uint32_t idesc_f16(int fmt, int a_mn, int b_mn, int M, int N) {
+  return (1u << 4)                      // D format: f32
+         | ((uint32_t)fmt << 7)         // A format
+         | ((uint32_t)fmt << 10)        // B format
+         | ((uint32_t)a_mn << 15)       // A major
+         | ((uint32_t)b_mn << 16)       // B major
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Arrives once on the mbarrier when every MMA this thread issued before has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+// 32 lanes x 32 bit, 32 consecutive columns: thread l of the warp gets lane (base lane + l).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// Two E2M1 codes (one byte, channel 2k in the low nibble) to f16x2 (channel 2k in the low half).
+__device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n .reg .b8 b;\n cvt.u8.u32 b, %1;\n cvt.rn.f16x2.e2m1x2 %0, b;\n}\n" : "=r"(r) : "r"(byte));
+  return r;
+}
+// Two E4M3 bytes (low 16 bits) to f16x2.
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;\n" : "=r"(r) : "h"((unsigned short)two));
+  return r;
+}
+// 2^x with the hardware approximation (relative error ~2^-22; 2^-inf = +0).
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// Byte offset of element (row, col) of a 16-bit matrix stored as core matrices with
+// `chunks_per_row` 8-element column chunks per 8-row group: block (row/8, col/8) at
+// ((row/8) * chunks_per_row + col/8) * 128, row % 8 at 16 B, col % 8 at 2 B.
+__device__ __forceinline__ int core_off(int row, int col, int chunks_per_row) {
+  return ((row >> 3) * chunks_per_row + (col >> 3)) * kCore + (row & 7) * 16 + (col & 7) * 2;
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_constant__ MlaParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ __align__(8) uint64_t bar_raw[2];  // a raw stage landed
+  __shared__ __align__(8) uint64_t bar_s;       // S = Q K^T done
+  __shared__ __align__(8) uint64_t bar_o;       // O^T += latent^T P^T done
+  __shared__ uint32_t s_tmem;                   // tensor-memory base address
+  __shared__ float s_alpha[kHeadsU];            // per-head O rescale factor of this iteration
+  __shared__ float s_hsc[kHeadsU];              // per-head power-of-two query scale
+  __shared__ int s_fail;
+
+  const Fp4Layout& F = p.fp4;
+  const int tile_bytes = F.tile_bytes;
+  unsigned char* sQ = smem + kOffQ;
+  unsigned char* sLat = smem + kOffLat;
+  unsigned char* sRope = smem + kOffRope;
+  unsigned char* sP = smem + kOffP;
+  unsigned char* raw = smem + kOffRaw;  // [2 stages][2 cache tiles]
+
+  const int split = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int len = p.lens[b];
+  const int t_begin = split * p.chunk;
+  const int t_end = min(len, t_begin + p.chunk);
+  const int n_iter = t_end > t_begin ? (t_end - t_begin + kTokU - 1) / kTokU : 0;
+  const unsigned char* base = reinterpret_cast<const unsigned char*>(p.reg) + (size_t)b * p.tiles_per_seq * tile_bytes;
+
+  if (tid == 0) {
+    mbar_init(smem_addr(&bar_raw[0]), 1);
+    mbar_init(smem_addr(&bar_raw[1]), 1);
+    mbar_init(smem_addr(&bar_s), 1);
+    mbar_init(smem_addr(&bar_o), 1);
+    mbar_init_fence();
+    s_fail = 0;
+  }
+  if (warp == 0) tmem_alloc(smem_addr(&s_tmem), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint32_t tmem_warp = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's lane quarter
+  const int col_half = warp >> 2;  // O^T columns (heads) 32 col_half .. +31 for rescale and output
+
+  // raw tile pair of iteration `it` into stage it & 1 (whole pairs: capacity is whole pairs)
+  auto issue_raw = [&](int it) {
+    if (it >= n_iter) return;
+    const int tile0 = (t_begin + it * kTokU) / kTile;
+    const uint32_t bar = smem_addr(&bar_raw[it & 1]);
+    fence_proxy_async();
+    mbar_arrive_expect_tx(bar, 2u * tile_bytes);
+    bulk_g2s(smem_addr(raw + (it & 1) * 2 * tile_bytes), base + (size_t)tile0 * tile_bytes, 2u * tile_bytes, bar);
+  };
+  auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_addr(bar);
+    if (!mbar_try(a, parity) && !mbar_wait(a, parity, p.wait_limit)) {
+      s_fail = 1;
+      atomicOr(p.err, 1);
+    }
+  };
+  if (tid == 0) issue_raw(0);
+
+  // ---- Q: per-head power-of-two scale into f16 range; latent part f16, RoPE part bf16, stored
+  // as core matrices [8 head groups][72 dim chunks] (K-major A operand of S = Q K^T)
+  const size_t qbase = (size_t)b * kHeadsU * kDqU;
+  for (int h = warp; h < kHeadsU; h += kThreadsU / 32) {
+    const void* qh = p.bf16 ? (const void*)(reinterpret_cast<const __nv_bfloat16*>(p.q) + qbase + (size_t)h * kDqU)
+                            : (const void*)(reinterpret_cast<const float*>(p.q) + qbase + (size_t)h * kDqU);
+    float mx = 0.f;
+    for (int c = lane; c < kDqU; c += 32) {
+      const float v = p.bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(qh)[c])
+                             : reinterpret_cast<const float*>(qh)[c];
+      mx = fmaxf(mx, fabsf(v));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float sc = mx > 0.f ? exp2f(ceilf(log2f(mx)) - 14.f) : 1.f;
+    if (lane == 0) s_hsc[h] = sc;
+    const float inv = 1.f / sc;
+    for (int c = lane; c < kDqU; c += 32) {
+      const float v = (p.bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(qh)[c])
+                              : reinterpret_cast<const float*>(qh)[c]) * inv;
+      unsigned char* dst = sQ + core_off(h, c, kDqU / 8);
+      if (c < kLatU) *reinterpret_cast<__half*>(dst) = __float2half_rn(v);
+      else *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
+    }
+  }
+  fence_proxy_async();  // Q is read by the tensor cores
+  __syncthreads();
+
+  // softmax state of head 16 warp + lane (lanes 0..15: the rows of an M=64 accumulator)
+  const bool head_lane = warp < 4 && lane < 16;
+  const int my_h = 16 * (warp & 3) + (lane & 15);
+  const float lsc = s_hsc[my_h] * p.logit_scale;
+  float m_used = -INFINITY, l_run = 0.f;
+
+  constexpr uint32_t kIdS = idesc_f16(0, 0, 0, 64, kTokU);       // f16, K-major A and B
+  constexpr uint32_t kIdSr = idesc_f16(1, 0, 0, 64, kTokU);      // bf16 (RoPE part)
+  constexpr uint32_t kIdO = idesc_f16(0, 1, 0, 128, kHeadsU);    // A (latent^T) MN-major
+  const uint32_t aQ = smem_addr(sQ), aLat = smem_addr(sLat), aRope = smem_addr(sRope), aP = smem_addr(sP);
+
+  for (int it = 0; it < n_iter; ++it) {
+    if (tid == 0) issue_raw(it + 1);  // stage (it+1)&1 was last read by the dequant of it-1
+    wait_bar(&bar_raw[it & 1], (uint32_t)(it >> 1) & 1u);
+    if (it > 0) {  // the previous O^T += latent^T P^T must be done before latent, P or O change
+      wait_bar(&bar_o, (uint32_t)(it - 1) & 1u);
+      tc_fence_after();
+    }
+    const unsigned char* rt = raw + (it & 1) * 2 * tile_bytes;
+    const int count = min(kTokU, t_end - (t_begin + it * kTokU));
+
+    // ---- dequantise: thread -> (token tid % 64, channel half tid / 64). The 16-byte code chunks
+    // are visited in a token-skewed order, which keeps both the reads of the packed rows and the
+    // core-matrix writes free of bank conflicts.
+    {
+      const int tok = tid & 63, quarter = tid >> 6, slot = tok & (kTile - 1);  // 128 channels each
+      const unsigned char* ct = rt + (tok / kTile) * tile_bytes;
+      if (tok < count) {
+        const uint2 sc8 = *reinterpret_cast<const uint2*>(ct + F.off_scales + slot * (kLatU / 16) + quarter * 8);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int c = (j + slot) & 3;  // 32-channel chunk of this quarter
+          const uint4 cw = *reinterpret_cast<const uint4*>(ct + F.off_codes + slot * (kLatU / 2) + quarter * 64 + c * 16);
+          const uint32_t sw = (c >> 1) ? sc8.y : sc8.x;
+          const uint32_t s2 = e4m3x2_f16x2((sw >> (16 * (c & 1))) & 0xFFFFu);  // groups 2c, 2c+1
+          const uint32_t slo = s2 & 0xFFFFu, shi = s2 >> 16;
+          const uint32_t bA = slo | (slo << 16), bB = shi | (shi << 16);
+          const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+          uint32_t out[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            out[k] = hmul2u(e2m1x2_f16x2((w4[k >> 2] >> (8 * (k & 3))) & 0xFFu), k < 8 ? bA : bB);
+          const int d0 = 128 * quarter + 32 * c;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(sLat + core_off(tok, d0 + 8 * v, kLatU / 8)) =
+                make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
+        }
+      } else {
+#pragma unroll 4
+        for (int j = 0; j < 16; ++j)
+          *reinterpret_cast<uint4*>(sLat + core_off(tok, 128 * quarter + 8 * j, kLatU / 8)) = make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {  // RoPE key: 64 tokens x 8 chunks of 16 B, chunk order skewed by token
+        const int rtok = tid & 63, dc = ((tid >> 6) + 4 * k + rtok) & 7;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (rtok < count)
+          v = *reinterpret_cast<const uint4*>(rt + (rtok / kTile) * tile_bytes + F.off_rope +
+                                              (rtok & (kTile - 1)) * (kRopeU * 2) + dc * 16);
+        *reinterpret_cast<uint4*>(sRope + core_off(rtok, 8 * dc, kRopeU / 8)) = v;
+      }
+    }
+    fence_proxy_async();  // the tile is read by the tensor cores
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- S = Q K^T (64 heads x 64 tokens, fp32 in tensor memory)
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll 4
+      for (int kk = 0; kk < kLatU / 16; ++kk)
+        umma_f16(tmem + kColS, smem_desc(aQ + kk * 2 * kCore, kCore, (kDqU / 8) * kCore),
+                 smem_desc(aLat + kk * 2 * kCore, kCore, (kLatU / 8) * kCore), kIdS, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < kRopeU / 16; ++kk)
+        umma_f16(tmem + kColS, smem_desc(aQ + (kLatU / 8 + 2 * kk) * kCore, kCore, (kDqU / 8) * kCore),
+                 smem_desc(aRope + kk * 2 * kCore, kCore, (kRopeU / 8) * kCore), kIdSr, 1u);
+      umma_commit(smem_addr(&bar_s));
+    }
+    wait_bar(&bar_s, (uint32_t)it & 1u);
+    tc_fence_after();
+
+    // ---- softmax rows: lanes 0..15 hold head 16 warp + lane (an M=64 accumulator's rows)
+    uint32_t sv0[32], sv1[32];
+    if (warp < 4) {
+      tmem_ld32(tmem_warp + kColS, sv0);
+      tmem_ld32(tmem_warp + kColS + 32, sv1);
+      tmem_wait_ld();
+    }
+    int moved = 0;
+    if (head_lane) {
+      float x[kTokU];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < kTokU; ++t) {
+        const float sv = __uint_as_float(t < 32 ? sv0[t] : sv1[t - 32]);
+        x[t] = t < count ? sv * lsc : -INFINITY;
+        mt = fmaxf(mt, x[t]);
+      }
+      float alpha = 1.f;
+      if (mt > m_used + kLazyRescale || (m_used == -INFINITY && mt > -INFINITY)) {
+        alpha = m_used == -INFINITY ? 0.f : ex2f(m_used - mt);
+        m_used = mt;
+        l_run *= alpha;
+        moved = 1;
+      }
+      s_alpha[my_h] = alpha;
+      float ls = 0.f;
+#pragma unroll
+      for (int tc = 0; tc < kTokU / 8; ++tc) {
+        uint32_t h2[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = ex2f(x[8 * tc + 2 * e] - m_used);  // 2^-inf = +0
+          const float p1 = ex2f(x[8 * tc + 2 * e + 1] - m_used);
+          ls += p0 + p1;
+          const __half2 hp = __floats2half2_rn(p0, p1);
+          h2[e] = *reinterpret_cast<const uint32_t*>(&hp);
+        }
+        *reinterpret_cast<uint4*>(sP + core_off(my_h, 8 * tc, kTokU / 8)) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+      }
+      l_run += ls;
+    }
+    const int any_moved = __syncthreads_or(moved);
+
+    // ---- rescale O^T columns of heads whose maximum moved (not before the first product)
+    if (it > 0 && any_moved) {
+#pragma unroll 1
+      for (int mt4 = 0; mt4 < kLatU / 128; ++mt4) {
+        uint32_t r[32];
+        const uint32_t ta = tmem_warp + kColO + mt4 * kHeadsU + col_half * 32;
+        tmem_ld32(ta, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * s_alpha[col_half * 32 + j]);
+        tmem_st32(ta, r);
+      }
+      tmem_wait_st();
+    }
+    fence_proxy_async();  // P is read by the tensor cores
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- O^T[512 x 64 heads] += latent^T [512 x 64 tokens] P^T [64 tokens x 64 heads]
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int mt4 = 0; mt4 < kLatU / 128; ++mt4)
+#pragma unroll
+        for (int kk = 0; kk < kTokU / 16; ++kk)
+          umma_f16(tmem + kColO + mt4 * kHeadsU,
+                   smem_desc(aLat + (kk * 2 * (kLatU / 8) + mt4 * 16) * kCore, (kLatU / 8) * kCore, kCore),
+                   smem_desc(aP + kk * 2 * kCore, kCore, (kTokU / 8) * kCore), kIdO, (it > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(smem_addr(&bar_o));
+    }
+  }
+
+  // ---- partials (m, l, o) of the 64 heads of this split
+  if (n_iter > 0) {
+    wait_bar(&bar_o, (uint32_t)(n_iter - 1) & 1u);
+    tc_fence_after();
+  }
+  const int stride = 2 + kLatU;
+  float* part = p.part + ((size_t)b * kHeadsU * p.splits + split) * stride;  // head h at + h * splits * stride
+  if (head_lane) {
+    float* d = part + (size_t)my_h * p.splits * stride;
+    d[0] = m_used;
+    d[1] = l_run;
+  }
+#pragma unroll 1
+  for (int mt4 = 0; mt4 < kLatU / 128; ++mt4) {
+    uint32_t r[32];
+    tmem_ld32(tmem_warp + kColO + mt4 * kHeadsU + col_half * 32, r);
+    tmem_wait_ld();
+    const int dim = 128 * mt4 + 32 * (warp & 3) + lane;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      part[(size_t)(col_half * 32 + j) * p.splits * stride + 2 + dim] = n_iter > 0 ? __uint_as_float(r[j]) : 0.f;
+  }
+
+  // ---- teardown: after a wait that gave up, wait once more (bounded) for what may be in flight
+  if (tid == 0 && s_fail) {
+    if (n_iter > 0) mbar_wait(smem_addr(&bar_o), (uint32_t)(n_iter - 1) & 1u, p.wait_limit);
+    for (int it = max(0, n_iter - 2); it < n_iter; ++it)
+      mbar_wait(smem_addr(&bar_raw[it & 1]), (uint32_t)(it >> 1) & 1u, p.wait_limit);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+bool mla_umma_supported(const MlaParams& p) {
+  return p.fp4.latent == kLatU && p.fp4.rope == kRopeU && p.Hq == kHeadsU && p.chunk % kTokU == 0 &&
+         (size_t)kOffRaw + 4 * (size_t)p.fp4.tile_bytes <= 227 * 1024;
+}
+
+cudaError_t launch_decode_mla_umma(const MlaParams& p, cudaStream_t s) {
+  const size_t smem = (size_t)kOffRaw + 4 * (size_t)p.fp4.tile_bytes;
+  cudaError_t e = cudaFuncSetAttribute(decode_mla_umma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  decode_mla_umma<<<dim3(p.splits, p.B), kThreadsU, smem, s>>>(p);
+  return launched();
+}
+
+}  // namespace kvq

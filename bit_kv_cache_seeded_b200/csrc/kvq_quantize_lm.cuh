@@ -1,0 +1,183 @@
+// LM / LM_QJL / SIGN1 quantize-and-append, as a block-level device function so that it can run
+// alone (quantize_lm_kernel) or beside the query prep of a fused decode step (one launch).
+//
+// "TurboQuant vs OSCAR vs EpiCache", section "Quantization frontiers: TurboQuant and OSCAR"; the
+// steps are listed at the top of kvq_quantize.cu.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kvq_async.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+namespace qlm {
+
+__device__ __forceinline__ float load_elem(const void* base, size_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  return reinterpret_cast<const float*>(base)[i];
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+constexpr int kLmWarps = 4;     // LM quantize: warps per block
+
+// Blocks per side of an LM quantize launch: one vector per block on sides with a sketch (the
+// block's warps share it), one per warp otherwise; at most 16 blocks per SM of a B200.
+inline int blocks_per_side(const QuantizeParams& p) {
+  const long total = (long)p.n_seq * p.heads * p.n_new;
+  const bool sketch = p.side[0].qjl || p.side[1].qjl;
+  const long per = sketch ? 1 : kLmWarps;
+  long blocks = (total + per - 1) / per;
+  if (blocks > 148L * 16) blocks = 148L * 16;
+  return blocks < 1 ? 1 : (int)blocks;
+}
+
+// One block of the LM quantize (`blk` of `nblk` blocks of side `side`). Sides with a sketch: the block's 4 warps share one vector; each redoes steps 1-5
+// (cheap, and it keeps every warp independent), then warp w forms sketch word w, i.e. the 32
+// projections j = 32w + lane, from its own 16 KB column slice of S^T staged in shared memory.
+// Sides without a sketch: one vector per warp.
+__device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int side, int blk, int nblk) {
+  __shared__ float rho_s[kLmWarps][kHeadDim];
+  extern __shared__ __align__(16) float st_s[];  // sketch sides: [warp][d][32] columns 32w.. of S^T
+  const SideLayout& L = p.side[side];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nthr = L.bits ? (1 << L.bits) - 1 : 0;
+  const bool coop = L.qjl;
+  const long total = (long)p.n_seq * p.heads * p.n_new;
+  const long first = coop ? (long)blk : (long)blk * kLmWarps + warp;
+  const long stride = coop ? (long)nblk : (long)nblk * kLmWarps;
+  float* stw = st_s + warp * kHeadDim * 32;  // stw[i * 32 + l] = S^T[i][32 warp + l] = S[32 warp + l][i]
+  // The slice is staged asynchronously while the first vector's elements are fetched.
+  if (coop && first < total) {
+    for (int c = lane; c < kHeadDim * 8; c += 32) {  // row i = c / 8, 16-byte chunk c % 8 of its 32 floats
+      const int i = c >> 3, ch = c & 7;
+      cp_async16(stw + i * 32 + ch * 4, p.St + (size_t)i * L.m + 32 * warp + ch * 4);
+    }
+    cp_async_commit();
+  }
+  float u_first[4] = {0.f, 0.f, 0.f, 0.f};
+  if (first < total)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u_first[k] = load_elem(p.src[side], (size_t)first * kHeadDim + 32 * k + lane, p.bf16);
+  if (coop) {
+    cp_async_wait<0>();
+    __syncwarp();
+  }
+
+  for (long vec = first; vec < total; vec += stride) {
+    const int t = (int)(vec % p.n_new);
+    const int h = (int)((vec / p.n_new) % p.heads);
+    const int s = (int)(vec / ((long)p.n_new * p.heads));
+    const size_t base = (size_t)vec * kHeadDim;  // [n_seq, heads, n_new, d] row-major
+
+    float u[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = (vec == first) ? u_first[k] : load_elem(p.src[side], base + 32 * k + lane, p.bf16);
+
+    float n = 0.f;
+    if (!p.skip_rotation) {
+      n = sqrtf(warp_sum(u[0] * u[0] + u[1] * u[1] + u[2] * u[2] + u[3] * u[3]));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) u[k] *= p.signs[32 * k + lane];
+      // Walsh-Hadamard butterflies over index bits 0..4 (lane) and 5..6 (k).
+#pragma unroll
+      for (int b = 0; b < 5; ++b) {
+        const bool upper = (lane >> b) & 1;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float other = __shfl_xor_sync(0xffffffffu, u[k], 1 << b);
+          u[k] = upper ? other - u[k] : u[k] + other;
+        }
+      }
+      const float a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
+      u[0] = a0 + a2; u[2] = a0 - a2; u[1] = a1 + a3; u[3] = a1 - a3;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) u[k] = (n > 0.f) ? u[k] / n : 0.f;
+    }
+
+    int code[4];
+    float rho[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      int c = 0;
+      for (int i = 0; i < nthr; ++i) c += (u[k] >= L.thr[i]) ? 1 : 0;
+      code[k] = c;
+      rho[k] = u[k] - L.cent[c];
+    }
+    uint32_t planes[kMaxBits][4];
+#pragma unroll
+    for (int pp = 0; pp < kMaxBits; ++pp)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        planes[pp][k] = (pp < L.bits) ? __ballot_sync(0xffffffffu, (code[k] >> pp) & 1) : 0u;
+    // lane pp < bits stores plane pp (selected without indexing registers by lane)
+    uint4 mine = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int pp = 0; pp < kMaxBits; ++pp)
+      if (lane == pp) mine = make_uint4(planes[pp][0], planes[pp][1], planes[pp][2], planes[pp][3]);
+
+    uint32_t zword = 0u;  // sketch word `warp` (coop sides)
+    float gamma = 0.f;
+    if (coop) {
+      gamma = sqrtf(warp_sum(rho[0] * rho[0] + rho[1] * rho[1] + rho[2] * rho[2] + rho[3] * rho[3]));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rho_s[warp][32 * k + lane] = rho[k];
+      __syncwarp();
+      float proj = 0.f;  // (S rho)_j, j = 32 warp + lane
+#pragma unroll 16
+      for (int i = 0; i < kHeadDim; ++i) proj = fmaf(stw[i * 32 + lane], rho_s[warp][i], proj);
+      __syncwarp();
+      zword = __ballot_sync(0xffffffffu, proj >= 0.f);
+    }
+    const bool lead = !coop || warp == 0;  // writes the planes and norms of this vector
+
+    if (p.skip_rotation) {
+      if (lead && lane < L.bits)
+        *reinterpret_cast<uint4*>(p.dbg_planes + ((size_t)vec * L.bits + lane) * 4) = mine;
+      if (coop && lane == 0) p.dbg_sketch[(size_t)vec * 4 + warp] = zword;
+      if (coop && warp == 0 && lane == 1) p.dbg_gamma[vec] = __half_as_ushort(__float2half_rn(gamma));
+      continue;
+    }
+
+    const int pos = p.pos[s] + t;
+    const int seq = p.seq[s];
+    const int tile = pos / kTile, slot = pos % kTile;
+    char* tb = p.region[side] +
+               (((size_t)seq * p.heads + h) * p.tiles_per_seq + tile) * (size_t)L.tile_bytes;
+    if (L.tokmajor) {
+      if (lead && lane < L.bits)
+        *reinterpret_cast<uint4*>(tb + L.off_planes + lane * (kTile * 16) + slot * 16) = mine;
+      if (coop && lane == 0) *reinterpret_cast<uint32_t*>(tb + L.off_sketch + slot * 16 + 4 * warp) = zword;
+    } else {
+      // byte-lane-major: byte k of a token's 16-byte plane goes to [k][slot]
+      if (lead && lane < 16) {
+#pragma unroll
+        for (int pp = 0; pp < kMaxBits; ++pp) {
+          if (pp < L.bits) {  // byte `lane` of plane pp: word lane / 4, byte lane % 4
+            const uint32_t lo = (lane & 4) ? planes[pp][1] : planes[pp][0];
+            const uint32_t hi = (lane & 4) ? planes[pp][3] : planes[pp][2];
+            const uint32_t w = (lane & 8) ? hi : lo;
+            tb[L.off_planes + pp * (kTile * 16) + lane * kTile + slot] = (char)((w >> (8 * (lane & 3))) & 0xFFu);
+          }
+        }
+      }
+      if (coop && lane < 4)
+        tb[L.off_sketch + (4 * warp + lane) * kTile + slot] = (char)((zword >> (8 * lane)) & 0xFFu);
+    }
+    if (lead && lane == 30) *reinterpret_cast<__half*>(tb + L.off_norm + slot * 2) = __float2half_rn(n);
+    if (coop && warp == 0 && lane == 29)
+      *reinterpret_cast<__half*>(tb + L.off_gamma + slot * 2) = __float2half_rn(gamma);
+  }
+
+  if (side == 0 && blk == 0 && !p.skip_rotation)
+    for (int i = threadIdx.x; i < p.n_seq; i += blockDim.x) p.lens[p.seq[i]] = p.pos[i] + p.n_new;
+}
+
+}  // namespace qlm
+}  // namespace kvq

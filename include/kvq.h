@@ -124,6 +124,15 @@ kvq_status kvq_workspace_bytes(const kvq_cache* c, size_t* bytes);
 kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* One decode step: append one token to every sequence (K, V as for kvq_quantize with n_new = 1
+ * and all sequences) and run kvq_decode_attention with q over the caches that now include it.
+ * The result equals the two calls in sequence; fusing them lets the query prep run while the
+ * append is still in flight (on the tensor-core path). Everything is validated (capacity,
+ * alignment, workspace for the lengths after the append) before anything is written; on an
+ * error nothing is appended. */
+kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
+                           float* out, void* workspace, size_t ws_bytes, void* stream);
+
 /* The same decode attention as kvq_decode_attention, for callers that cannot allocate device
  * memory on the decode path (serving loops that reserve all memory up front, hosts whose memory
  * belongs to another allocator, code that must not risk the device synchronisation cudaMalloc
@@ -205,8 +214,8 @@ kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_
 /* Diagnostic, with no counterpart in the method: the number of GPU kernels this library has
  * enqueued successfully since it was loaded, summed over all threads, devices and caches. A
  * caller reads it before and after a region to learn how many kernels the region launched
- * (quantize: 1 per call; decode: 3 for LM caches on the tensor-core path, else 2). Host-only;
- * never fails. */
+ * (quantize: 1 per call; decode: 3 per call on the tensor-core path, else 2). Host-only; never
+ * fails. */
 uint64_t kvq_kernel_launches(void);
 
 #ifdef __cplusplus

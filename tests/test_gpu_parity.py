@@ -15,7 +15,7 @@ import bit_kv_cache_seeded_b200 as kvq
 from kvq_inputs import WORKLOADS, generate
 from kvq_inputs.workloads import rotation_and_sketch
 from oracle import codec, tables, attention
-from tests._cache_reader import fp4_fields
+from tests._cache_reader import fp4_fields, side_fields
 from tests._parity import pair_reference, rel_err, REL_TOL, BOUNDARY
 
 pytestmark = pytest.mark.gpu
@@ -174,8 +174,10 @@ def test_full_size_sampled_pairs(name):
 
 # ---------------------------------------------------------------- FP4 latent cache
 
-def fp4_check(ctx, heads_checked=None, batch=1, lens=None):
+def fp4_check(ctx, heads_checked=None, batch=1, lens=None, n_q_heads=None):
     w = WORKLOADS["mla_fp4"]
+    if n_q_heads is not None:
+        w = w.with_(n_q_heads=n_q_heads)
     lens = lens or [ctx] * batch
     data = generate(w, DEV, seqs=range(batch), ctx=max(lens))
     cache = kvq.KvqCache(kvq.cfg_for_workload(w), batch, max(lens) + 32)
@@ -212,6 +214,11 @@ def test_fp4_small_ragged():
     fp4_check(0, batch=3, lens=[1000, 0, 33])
 
 
+def test_fp4_sixteen_heads_ragged():
+    """16 query heads decode on the mma.sync kernel (the tcgen05 kernel is for 64 heads)."""
+    fp4_check(0, batch=2, lens=[700, 65], n_q_heads=16)
+
+
 def test_fp4_full_context_sampled_heads():
     fp4_check(WORKLOADS["mla_fp4"].ctx, heads_checked=[0, 21, 63])
 
@@ -219,8 +226,8 @@ def test_fp4_full_context_sampled_heads():
 # ---------------------------------------------------------------- launch accounting
 
 def test_launch_counts_per_call():
-    """quantize: one kernel; decode: prep + split decode + reduce for LM caches on the tensor-core
-    path (G <= 4), split decode + reduce otherwise (G = 8 and FP4)."""
+    """quantize: one kernel; decode: query prep + split decode + reduce on the tensor-core path
+    (G <= 4), split decode + reduce otherwise (G = 8 and FP4)."""
     for name, per_decode in (("llama8b", 3), ("llama70b", 2), ("mla_fp4", 2)):
         w = WORKLOADS[name]
         data = generate(w, DEV, seqs=range(2), ctx=100)
@@ -237,6 +244,50 @@ def test_launch_counts_per_call():
         assert kvq.kvq_kernel_launches() - n0 == 1 + per_decode, name
         torch.cuda.synchronize()
         cache.close()
+
+
+# ---------------------------------------------------------------- fused decode step
+
+@pytest.mark.parametrize("name", ["llama8b", "onebit", "mla_fp4"])
+def test_decode_step_equals_append_then_decode(name):
+    """kvq_decode_step (append one token, then attend, with the query prep overlapping the append)
+    leaves the same cache and returns the same output as kvq_quantize followed by
+    kvq_decode_attention."""
+    w = WORKLOADS[name]
+    fp4 = w.k_mode == "fp4"
+    B = 3
+    data = generate(w, DEV, seqs=range(B), ctx=200)
+    new = generate(w, DEV, seqs=range(B), step=0)
+    if fp4:
+        a, v, na, nv = data["latent"], data["rope"], new["latent"], new["rope"]
+        mk = lambda: kvq.KvqCache(kvq.cfg_for_workload(w), B, 256)
+    else:
+        a, v, na, nv = data["k"], data["v"], new["k"], new["v"]
+        mk = lambda: new_cache(w, B, 256)[0]
+    c1, c2 = mk(), mk()
+    for c in (c1, c2):
+        c.quantize(a[:, :, :150].contiguous() if not fp4 else a[:, :150].contiguous(),
+                   v[:, :, :150].contiguous() if not fp4 else v[:, :150].contiguous())
+    c1.quantize(na, nv)
+    ref = c1.decode(data["q"])
+    out = c2.step(na, nv, data["q"])
+    torch.cuda.synchronize()
+    assert list(c1.lengths()) == list(c2.lengths()) == [151] * B
+    assert torch.equal(out, ref)
+    # the written part of the caches is identical (tile tails past the lengths are never written)
+    a1, a2, info = c1.arena.cpu().numpy(), c2.arena.cpu().numpy(), c1.layout()
+    if fp4:
+        for b in range(B):
+            for f1, f2 in zip(fp4_fields(a1, info, b, 151), fp4_fields(a2, info, b, 151)):
+                np.testing.assert_array_equal(f1, f2)
+    else:
+        for pair in range(B * w.n_kv_heads):
+            for side in (0, 1):
+                for f1, f2 in zip(side_fields(a1, info, side, pair, 151), side_fields(a2, info, side, pair, 151)):
+                    if f1 is not None:
+                        np.testing.assert_array_equal(f1[:151], f2[:151])
+    c1.close()
+    c2.close()
 
 
 # ---------------------------------------------------------------- bounded waits
