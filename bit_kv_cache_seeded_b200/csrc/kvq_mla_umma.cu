@@ -12,17 +12,19 @@
 //
 // One CTA per SM (8 warps; warp w reaches tensor-memory lane quarter w % 4), per 64-token
 // iteration:
-//   1. the packed tile pair arrives by bulk copy (double-buffered, mbarrier-completed);
-//   2. all threads dequantise the latent to f16 and copy the RoPE key into shared memory in the
-//      canonical no-swizzle "core matrix" layout (8 rows x 16 B blocks) both MMAs read;
-//   3. thread 0 issues S = Q K^T into tensor memory and commits to an mbarrier;
-//   4. lanes 0..15 of warps 0..3 (the rows of S for an M=64 MMA) load their head's 64 logits,
+//   1. every thread holds its share of the next tile's packed data in registers (loaded one tile
+//      ahead) and dequantises it to f16, with the RoPE key, into the free one of two shared-memory
+//      buffers in the canonical no-swizzle "core matrix" layout (8 rows x 16 B blocks) that both
+//      MMAs read; this overlaps S of the current tile on the tensor cores;
+//   2. thread 0 issues S = Q K^T into tensor memory and commits to an mbarrier (for the next tile
+//      right after the current tile's O^T product);
+//   3. lanes 0..15 of warps 0..3 (the rows of S for an M=64 MMA) load their head's 64 logits,
 //      update a lazily rescaled running maximum (rescale only when it grows by more than 8 in
 //      log2 units), write P = 2^(l - m) (<= 256) as f16 in core-matrix layout;
-//   5. if a head's maximum moved, every thread rescales that head's column of O^T in tensor
+//   4. if a head's maximum moved, every thread rescales that head's column of O^T in tensor
 //      memory (load, multiply, store);
-//   6. thread 0 issues O^T += latent^T P^T and commits; the next iteration waits for it before
-//      it overwrites the latent, P or O.
+//   5. thread 0 issues O^T += latent^T P^T and commits; the next iteration waits for it before
+//      it overwrites that latent buffer, P or O.
 // Every mbarrier wait is bounded (the cache status word records a wait that gave up). Partials
 // (m, l, o[512]) per (sequence, head, split) go to the workspace in the format of the other
 // MLA kernels; the same reduce kernel finishes.
@@ -44,17 +46,18 @@ constexpr float kLazyRescale = 8.f;     // rescale O only when the running max g
 constexpr uint32_t kTmemCols = 512;     // allocation: O^T in columns 0..255, S in 256..319
 constexpr uint32_t kColO = 0, kColS = 256;
 
-// Shared-memory layout (bytes). Q: [8 head groups][72 dim chunks] core matrices; LAT: [8 token
-// groups][64 dim chunks]; ROPE: [8 token groups][8 dim chunks]; P: [8 head groups][8 token chunks].
+// Shared-memory layout (bytes). Q: [8 head groups][72 dim chunks] core matrices; LAT (x2): [8 token
+// groups][64 dim chunks]; ROPE (x2): [8 token groups][8 dim chunks]; P: [8 head groups][8 token
+// chunks]. The latent/RoPE buffers alternate between tiles.
 constexpr int kOffQ = 0;
 constexpr int kSizeQ = kHeadsU * kDqU * 2;              // 73728
-constexpr int kOffLat = kOffQ + kSizeQ;
+constexpr int kOffLat = kOffQ + kSizeQ;                 // [2 buffers]
 constexpr int kSizeLat = kTokU * kLatU * 2;             // 65536
-constexpr int kOffRope = kOffLat + kSizeLat;
+constexpr int kOffRope = kOffLat + 2 * kSizeLat;        // [2 buffers]
 constexpr int kSizeRope = kTokU * kRopeU * 2;           // 8192
-constexpr int kOffP = kOffRope + kSizeRope;
+constexpr int kOffP = kOffRope + 2 * kSizeRope;
 constexpr int kSizeP = kHeadsU * kTokU * 2;             // 8192
-constexpr int kOffRaw = kOffP + kSizeP;                 // then 2 raw stages of 2 cache tiles
+constexpr int kSmemU = kOffP + kSizeP;                  // 229376
 
 // ---- tcgen05 / descriptor helpers (PTX ISA 8.7+, sm_100a) ----------------------------------
 
@@ -160,24 +163,80 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
+// Packed data of one 64-token tile that one thread dequantises: token tid % 64, channels
+// 128 (tid / 64) .. +127 (64 code bytes, 8 scale bytes) and two 16-byte RoPE chunks. Loaded straight
+// from global memory into registers one tile ahead of its use.
+struct TileRegs {
+  uint4 codes[4];
+  uint2 scales;
+  uint4 rope[2];
+};
+
+__device__ __forceinline__ void load_tile(TileRegs& r, const unsigned char* base, const Fp4Layout& F, int tile_bytes,
+                                          int t0, int count, int tid) {
+  const int tok = tid & 63, quarter = tid >> 6, slot = tok & (kTile - 1);
+  if (tok < count) {
+    const unsigned char* ct = base + (size_t)((t0 >> 5) + (tok >> 5)) * tile_bytes;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // chunk order skewed by token: see dequant_tile
+      const int c = (j + slot) & 3;
+      r.codes[j] = *reinterpret_cast<const uint4*>(ct + F.off_codes + slot * (kLatU / 2) + quarter * 64 + c * 16);
+    }
+    r.scales = *reinterpret_cast<const uint2*>(ct + F.off_scales + slot * (kLatU / 16) + quarter * 8);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int dc = (quarter + 4 * k + tok) & 7;
+      r.rope[k] = *reinterpret_cast<const uint4*>(ct + F.off_rope + slot * (kRopeU * 2) + dc * 16);
+    }
+  } else {  // zero codes and scales dequantise to zeros
+#pragma unroll
+    for (int j = 0; j < 4; ++j) r.codes[j] = make_uint4(0, 0, 0, 0);
+    r.scales = make_uint2(0, 0);
+    r.rope[0] = r.rope[1] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Dequantise one thread's share of a tile into core-matrix layout. The chunk order is skewed by
+// token so that the 8 rows of each core matrix are written by 8 consecutive lanes (no conflicts).
+__device__ __forceinline__ void dequant_tile(const TileRegs& r, unsigned char* lat, unsigned char* rope, int tid) {
+  const int tok = tid & 63, quarter = tid >> 6, slot = tok & (kTile - 1);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int c = (j + slot) & 3;  // 32-channel chunk of this quarter: groups 2c, 2c+1
+    const uint32_t sw = (c >> 1) ? r.scales.y : r.scales.x;
+    const uint32_t s2 = e4m3x2_f16x2((sw >> (16 * (c & 1))) & 0xFFFFu);
+    const uint32_t slo = s2 & 0xFFFFu, shi = s2 >> 16;
+    const uint32_t bA = slo | (slo << 16), bB = shi | (shi << 16);
+    const uint32_t w4[4] = {r.codes[j].x, r.codes[j].y, r.codes[j].z, r.codes[j].w};
+    uint32_t out[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      out[k] = hmul2u(e2m1x2_f16x2((w4[k >> 2] >> (8 * (k & 3))) & 0xFFu), k < 8 ? bA : bB);
+    const int d0 = 128 * quarter + 32 * c;
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      *reinterpret_cast<uint4*>(lat + core_off(tok, d0 + 8 * v, kLatU / 8)) =
+          make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int dc = (quarter + 4 * k + tok) & 7;
+    *reinterpret_cast<uint4*>(rope + core_off(tok, 8 * dc, kRopeU / 8)) = r.rope[k];
+  }
+}
+
 __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_constant__ MlaParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t bar_raw[2];  // a raw stage landed
-  __shared__ __align__(8) uint64_t bar_s;       // S = Q K^T done
-  __shared__ __align__(8) uint64_t bar_o;       // O^T += latent^T P^T done
-  __shared__ uint32_t s_tmem;                   // tensor-memory base address
-  __shared__ float s_alpha[kHeadsU];            // per-head O rescale factor of this iteration
-  __shared__ float s_hsc[kHeadsU];              // per-head power-of-two query scale
+  __shared__ __align__(8) uint64_t bar_s;  // S = Q K^T done (all earlier MMAs too)
+  __shared__ __align__(8) uint64_t bar_o;  // O^T += latent^T P^T done (all earlier MMAs too)
+  __shared__ uint32_t s_tmem;              // tensor-memory base address
+  __shared__ float s_alpha[kHeadsU];       // per-head O rescale factor of this iteration
+  __shared__ float s_hsc[kHeadsU];         // per-head power-of-two query scale
   __shared__ int s_fail;
 
   const Fp4Layout& F = p.fp4;
   const int tile_bytes = F.tile_bytes;
   unsigned char* sQ = smem + kOffQ;
-  unsigned char* sLat = smem + kOffLat;
-  unsigned char* sRope = smem + kOffRope;
-  unsigned char* sP = smem + kOffP;
-  unsigned char* raw = smem + kOffRaw;  // [2 stages][2 cache tiles]
-
   const int split = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int len = p.lens[b];
@@ -185,10 +244,9 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
   const int t_end = min(len, t_begin + p.chunk);
   const int n_iter = t_end > t_begin ? (t_end - t_begin + kTokU - 1) / kTokU : 0;
   const unsigned char* base = reinterpret_cast<const unsigned char*>(p.reg) + (size_t)b * p.tiles_per_seq * tile_bytes;
+  auto tile_count = [&](int it) { return min(kTokU, t_end - (t_begin + it * kTokU)); };
 
   if (tid == 0) {
-    mbar_init(smem_addr(&bar_raw[0]), 1);
-    mbar_init(smem_addr(&bar_raw[1]), 1);
     mbar_init(smem_addr(&bar_s), 1);
     mbar_init(smem_addr(&bar_o), 1);
     mbar_init_fence();
@@ -201,16 +259,6 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
   const uint32_t tmem = s_tmem;
   const uint32_t tmem_warp = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // this warp's lane quarter
   const int col_half = warp >> 2;  // O^T columns (heads) 32 col_half .. +31 for rescale and output
-
-  // raw tile pair of iteration `it` into stage it & 1 (whole pairs: capacity is whole pairs)
-  auto issue_raw = [&](int it) {
-    if (it >= n_iter) return;
-    const int tile0 = (t_begin + it * kTokU) / kTile;
-    const uint32_t bar = smem_addr(&bar_raw[it & 1]);
-    fence_proxy_async();
-    mbar_arrive_expect_tx(bar, 2u * tile_bytes);
-    bulk_g2s(smem_addr(raw + (it & 1) * 2 * tile_bytes), base + (size_t)tile0 * tile_bytes, 2u * tile_bytes, bar);
-  };
   auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
     const uint32_t a = smem_addr(bar);
     if (!mbar_try(a, parity) && !mbar_wait(a, parity, p.wait_limit)) {
@@ -218,7 +266,9 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
       atomicOr(p.err, 1);
     }
   };
-  if (tid == 0) issue_raw(0);
+
+  TileRegs regs;
+  if (n_iter > 0) load_tile(regs, base, F, tile_bytes, t_begin, tile_count(0), tid);
 
   // ---- Q: per-head power-of-two scale into f16 range; latent part f16, RoPE part bf16, stored
   // as core matrices [8 head groups][72 dim chunks] (K-major A operand of S = Q K^T)
@@ -245,10 +295,14 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
       else *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(v);
     }
   }
-  fence_proxy_async();  // Q is read by the tensor cores
+  // first tile into buffer 0, then fetch the second
+  if (n_iter > 0) dequant_tile(regs, smem + kOffLat, smem + kOffRope, tid);
+  if (n_iter > 1) load_tile(regs, base, F, tile_bytes, t_begin + kTokU, tile_count(1), tid);
+  fence_proxy_async();  // Q and the first tile are read by the tensor cores
+  tc_fence_before();
   __syncthreads();
 
-  // softmax state of head 16 warp + lane (lanes 0..15: the rows of an M=64 accumulator)
+  // softmax state of head 16 warp + lane (warps 0..3, lanes 0..15: the rows of an M=64 accumulator)
   const bool head_lane = warp < 4 && lane < 16;
   const int my_h = 16 * (warp & 3) + (lane & 15);
   const float lsc = s_hsc[my_h] * p.logit_scale;
@@ -257,81 +311,52 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
   constexpr uint32_t kIdS = idesc_f16(0, 0, 0, 64, kTokU);       // f16, K-major A and B
   constexpr uint32_t kIdSr = idesc_f16(1, 0, 0, 64, kTokU);      // bf16 (RoPE part)
   constexpr uint32_t kIdO = idesc_f16(0, 1, 0, 128, kHeadsU);    // A (latent^T) MN-major
-  const uint32_t aQ = smem_addr(sQ), aLat = smem_addr(sLat), aRope = smem_addr(sRope), aP = smem_addr(sP);
+  const uint32_t aQ = smem_addr(sQ), aP = smem_addr(smem + kOffP);
+  auto issue_s = [&](int buf) {  // S = Q K^T over latent/RoPE buffer `buf`
+    const uint32_t aLat = smem_addr(smem + kOffLat + buf * kSizeLat), aRope = smem_addr(smem + kOffRope + buf * kSizeRope);
+#pragma unroll 4
+    for (int kk = 0; kk < kLatU / 16; ++kk)
+      umma_f16(tmem + kColS, smem_desc(aQ + kk * 2 * kCore, kCore, (kDqU / 8) * kCore),
+               smem_desc(aLat + kk * 2 * kCore, kCore, (kLatU / 8) * kCore), kIdS, kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < kRopeU / 16; ++kk)
+      umma_f16(tmem + kColS, smem_desc(aQ + (kLatU / 8 + 2 * kk) * kCore, kCore, (kDqU / 8) * kCore),
+               smem_desc(aRope + kk * 2 * kCore, kCore, (kRopeU / 8) * kCore), kIdSr, 1u);
+    umma_commit(smem_addr(&bar_s));
+  };
+  auto issue_o = [&](int buf, bool first) {  // O^T += latent^T P^T over buffer `buf`
+    const uint32_t aLat = smem_addr(smem + kOffLat + buf * kSizeLat);
+#pragma unroll
+    for (int mt4 = 0; mt4 < kLatU / 128; ++mt4)
+#pragma unroll
+      for (int kk = 0; kk < kTokU / 16; ++kk)
+        umma_f16(tmem + kColO + mt4 * kHeadsU,
+                 smem_desc(aLat + (kk * 2 * (kLatU / 8) + mt4 * 16) * kCore, (kLatU / 8) * kCore, kCore),
+                 smem_desc(aP + kk * 2 * kCore, kCore, (kTokU / 8) * kCore), kIdO, (!first || kk > 0) ? 1u : 0u);
+    umma_commit(smem_addr(&bar_o));
+  };
+  if (tid == 0 && n_iter > 0) {
+    tc_fence_after();
+    issue_s(0);
+  }
 
   for (int it = 0; it < n_iter; ++it) {
-    if (tid == 0) issue_raw(it + 1);  // stage (it+1)&1 was last read by the dequant of it-1
-    wait_bar(&bar_raw[it & 1], (uint32_t)(it >> 1) & 1u);
-    if (it > 0) {  // the previous O^T += latent^T P^T must be done before latent, P or O change
+    const int buf = it & 1;
+    const int count = tile_count(it);
+    // PV(it-1) read the other latent buffer and P, and wrote O^T: wait for it before any of them
+    // changes; then the next tile goes into the other buffer while S(it) runs on the tensor cores
+    if (it > 0) {
       wait_bar(&bar_o, (uint32_t)(it - 1) & 1u);
       tc_fence_after();
     }
-    const unsigned char* rt = raw + (it & 1) * 2 * tile_bytes;
-    const int count = min(kTokU, t_end - (t_begin + it * kTokU));
-
-    // ---- dequantise: thread -> (token tid % 64, channel half tid / 64). The 16-byte code chunks
-    // are visited in a token-skewed order, which keeps both the reads of the packed rows and the
-    // core-matrix writes free of bank conflicts.
-    {
-      const int tok = tid & 63, quarter = tid >> 6, slot = tok & (kTile - 1);  // 128 channels each
-      const unsigned char* ct = rt + (tok / kTile) * tile_bytes;
-      if (tok < count) {
-        const uint2 sc8 = *reinterpret_cast<const uint2*>(ct + F.off_scales + slot * (kLatU / 16) + quarter * 8);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = (j + slot) & 3;  // 32-channel chunk of this quarter
-          const uint4 cw = *reinterpret_cast<const uint4*>(ct + F.off_codes + slot * (kLatU / 2) + quarter * 64 + c * 16);
-          const uint32_t sw = (c >> 1) ? sc8.y : sc8.x;
-          const uint32_t s2 = e4m3x2_f16x2((sw >> (16 * (c & 1))) & 0xFFFFu);  // groups 2c, 2c+1
-          const uint32_t slo = s2 & 0xFFFFu, shi = s2 >> 16;
-          const uint32_t bA = slo | (slo << 16), bB = shi | (shi << 16);
-          const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
-          uint32_t out[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-            out[k] = hmul2u(e2m1x2_f16x2((w4[k >> 2] >> (8 * (k & 3))) & 0xFFu), k < 8 ? bA : bB);
-          const int d0 = 128 * quarter + 32 * c;
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            *reinterpret_cast<uint4*>(sLat + core_off(tok, d0 + 8 * v, kLatU / 8)) =
-                make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
-        }
-      } else {
-#pragma unroll 4
-        for (int j = 0; j < 16; ++j)
-          *reinterpret_cast<uint4*>(sLat + core_off(tok, 128 * quarter + 8 * j, kLatU / 8)) = make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {  // RoPE key: 64 tokens x 8 chunks of 16 B, chunk order skewed by token
-        const int rtok = tid & 63, dc = ((tid >> 6) + 4 * k + rtok) & 7;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (rtok < count)
-          v = *reinterpret_cast<const uint4*>(rt + (rtok / kTile) * tile_bytes + F.off_rope +
-                                              (rtok & (kTile - 1)) * (kRopeU * 2) + dc * 16);
-        *reinterpret_cast<uint4*>(sRope + core_off(rtok, 8 * dc, kRopeU / 8)) = v;
-      }
-    }
-    fence_proxy_async();  // the tile is read by the tensor cores
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- S = Q K^T (64 heads x 64 tokens, fp32 in tensor memory)
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll 4
-      for (int kk = 0; kk < kLatU / 16; ++kk)
-        umma_f16(tmem + kColS, smem_desc(aQ + kk * 2 * kCore, kCore, (kDqU / 8) * kCore),
-                 smem_desc(aLat + kk * 2 * kCore, kCore, (kLatU / 8) * kCore), kIdS, kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < kRopeU / 16; ++kk)
-        umma_f16(tmem + kColS, smem_desc(aQ + (kLatU / 8 + 2 * kk) * kCore, kCore, (kDqU / 8) * kCore),
-                 smem_desc(aRope + kk * 2 * kCore, kCore, (kRopeU / 8) * kCore), kIdSr, 1u);
-      umma_commit(smem_addr(&bar_s));
+    if (it + 1 < n_iter) {
+      dequant_tile(regs, smem + kOffLat + (buf ^ 1) * kSizeLat, smem + kOffRope + (buf ^ 1) * kSizeRope, tid);
+      if (it + 2 < n_iter) load_tile(regs, base, F, tile_bytes, t_begin + (it + 2) * kTokU, tile_count(it + 2), tid);
     }
     wait_bar(&bar_s, (uint32_t)it & 1u);
     tc_fence_after();
 
-    // ---- softmax rows: lanes 0..15 hold head 16 warp + lane (an M=64 accumulator's rows)
+    // ---- softmax rows: lanes 0..15 of warps 0..3 hold head 16 warp + lane
     uint32_t sv0[32], sv1[32];
     if (warp < 4) {
       tmem_ld32(tmem_warp + kColS, sv0);
@@ -349,7 +374,7 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
         mt = fmaxf(mt, x[t]);
       }
       float alpha = 1.f;
-      if (mt > m_used + kLazyRescale || (m_used == -INFINITY && mt > -INFINITY)) {
+      if (mt > m_used + kLazyRescale) {  // also the first tile (m_used = -inf)
         alpha = m_used == -INFINITY ? 0.f : ex2f(m_used - mt);
         m_used = mt;
         l_run *= alpha;
@@ -368,7 +393,7 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
           const __half2 hp = __floats2half2_rn(p0, p1);
           h2[e] = *reinterpret_cast<const uint32_t*>(&hp);
         }
-        *reinterpret_cast<uint4*>(sP + core_off(my_h, 8 * tc, kTokU / 8)) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+        *reinterpret_cast<uint4*>(smem + kOffP + core_off(my_h, 8 * tc, kTokU / 8)) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
       }
       l_run += ls;
     }
@@ -388,21 +413,15 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
       }
       tmem_wait_st();
     }
-    fence_proxy_async();  // P is read by the tensor cores
+    fence_proxy_async();  // P and the next tile are read by the tensor cores
     tc_fence_before();
     __syncthreads();
 
-    // ---- O^T[512 x 64 heads] += latent^T [512 x 64 tokens] P^T [64 tokens x 64 heads]
+    // ---- O^T += latent^T P^T for this tile, then S for the next one
     if (tid == 0) {
       tc_fence_after();
-#pragma unroll
-      for (int mt4 = 0; mt4 < kLatU / 128; ++mt4)
-#pragma unroll
-        for (int kk = 0; kk < kTokU / 16; ++kk)
-          umma_f16(tmem + kColO + mt4 * kHeadsU,
-                   smem_desc(aLat + (kk * 2 * (kLatU / 8) + mt4 * 16) * kCore, (kLatU / 8) * kCore, kCore),
-                   smem_desc(aP + kk * 2 * kCore, kCore, (kTokU / 8) * kCore), kIdO, (it > 0 || kk > 0) ? 1u : 0u);
-      umma_commit(smem_addr(&bar_o));
+      issue_o(buf, it == 0);
+      if (it + 1 < n_iter) issue_s(buf ^ 1);
     }
   }
 
@@ -429,12 +448,8 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
       part[(size_t)(col_half * 32 + j) * p.splits * stride + 2 + dim] = n_iter > 0 ? __uint_as_float(r[j]) : 0.f;
   }
 
-  // ---- teardown: after a wait that gave up, wait once more (bounded) for what may be in flight
-  if (tid == 0 && s_fail) {
-    if (n_iter > 0) mbar_wait(smem_addr(&bar_o), (uint32_t)(n_iter - 1) & 1u, p.wait_limit);
-    for (int it = max(0, n_iter - 2); it < n_iter; ++it)
-      mbar_wait(smem_addr(&bar_raw[it & 1]), (uint32_t)(it >> 1) & 1u, p.wait_limit);
-  }
+  // ---- teardown: after a wait that gave up, wait once more (bounded) for the last MMAs
+  if (tid == 0 && s_fail && n_iter > 0) mbar_wait(smem_addr(&bar_o), (uint32_t)(n_iter - 1) & 1u, p.wait_limit);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -446,12 +461,11 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
 }  // namespace
 
 bool mla_umma_supported(const MlaParams& p) {
-  return p.fp4.latent == kLatU && p.fp4.rope == kRopeU && p.Hq == kHeadsU && p.chunk % kTokU == 0 &&
-         (size_t)kOffRaw + 4 * (size_t)p.fp4.tile_bytes <= 227 * 1024;
+  return p.fp4.latent == kLatU && p.fp4.rope == kRopeU && p.Hq == kHeadsU && p.chunk % kTokU == 0;
 }
 
 cudaError_t launch_decode_mla_umma(const MlaParams& p, cudaStream_t s) {
-  const size_t smem = (size_t)kOffRaw + 4 * (size_t)p.fp4.tile_bytes;
+  const size_t smem = kSmemU;
   cudaError_t e = cudaFuncSetAttribute(decode_mla_umma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   decode_mla_umma<<<dim3(p.splits, p.B), kThreadsU, smem, s>>>(p);
