@@ -256,8 +256,8 @@ def kvq_cache_lengths(handle, batch: int) -> np.ndarray:
 
 
 def kvq_cache_layout(handle) -> np.ndarray:
-    info = np.zeros(16, dtype=np.int64)
-    _check("kvq_cache_layout", load().kvq_cache_layout(handle, info.ctypes.data_as(ctypes.c_void_p), 16))
+    info = np.zeros(18, dtype=np.int64)
+    _check("kvq_cache_layout", load().kvq_cache_layout(handle, info.ctypes.data_as(ctypes.c_void_p), 18))
     return info
 
 

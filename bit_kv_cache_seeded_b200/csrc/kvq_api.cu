@@ -52,9 +52,9 @@ kvq_status validate_cfg(const kvq_cfg* c) {
   return KVQ_OK;
 }
 
-SideLayout make_side(int mode, int bits, int qjl_dim, int tokmajor) {
+SideLayout make_side(int mode, int bits, int qjl_dim, int order) {
   SideLayout L;
-  L.tokmajor = tokmajor;
+  L.order = order;
   L.bits = (mode == KVQ_MODE_SIGN1) ? 1 : bits;
   L.qjl = mode == KVQ_MODE_LM_QJL;
   L.m = L.qjl ? qjl_dim : 0;
@@ -106,8 +106,10 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
     off = align_up(off + pairs * P.tiles * (size_t)P.fp4.tile_bytes, kArenaAlign);
     P.v_off = off;
   } else {
-    P.k = make_side(c->k_mode, c->k_bits, c->qjl_dim, 1);
-    P.v = make_side(c->v_mode, c->v_bits, c->qjl_dim, 0);
+    P.v = make_side(c->v_mode, c->v_bits, c->qjl_dim, kOrderByteLane);
+    P.k = make_side(c->k_mode, c->k_bits, c->qjl_dim, kOrderToken);
+    if (mma_modes_supported(c->n_q_heads / c->n_kv_heads, P.k.bits, P.k.qjl, P.v.bits, P.v.qjl))
+      P.k.order = kOrderOctet;
     const size_t m = (P.k.qjl || P.v.qjl) ? (size_t)c->qjl_dim : 0;
     P.signs_off = off;
     off = align_up(off + sizeof(float) * kHeadDim, kArenaAlign);
@@ -132,8 +134,8 @@ int device_sms() {
 
 // Split plan. Each (pair, split) CTA covers a whole number of 64-token units, at most
 // `max_units` of them. The split count minimises waves x (units per CTA + a fixed per-CTA
-// overhead of 4 units), with `slots` resident CTAs per wave; max_splits() bounds it for every
-// length up to the capacity (it sizes the workspace).
+// overhead of 4 units), with slots_per_sm(units per CTA) resident CTAs per SM in a wave;
+// max_splits() bounds it for every length up to the capacity (it sizes the workspace).
 int max_splits(int pairs, int sms, int tiles, int max_units, int waves_bound) {
   const int units = std::max(1, tiles / kTilePair);
   const int need = (units + max_units - 1) / max_units;
@@ -141,18 +143,19 @@ int max_splits(int pairs, int sms, int tiles, int max_units, int waves_bound) {
   return std::max(need, std::min(bound, units));
 }
 
-void plan_splits(int pairs, int sms, int slots_per_sm, int max_units, int waves_bound, int max_len,
+template <class SlotsFn>
+void plan_splits(int pairs, int sms, const SlotsFn& slots_per_sm, int max_units, int waves_bound, int max_len,
                  int* splits, int* chunk) {
   const int units = std::max(1, (max_len + kTile * kTilePair - 1) / (kTile * kTilePair));
   const int smin = (units + max_units - 1) / max_units;
   const int smax = std::min(max_splits(pairs, sms, units * kTilePair, max_units, waves_bound), units);
-  const long slots = (long)sms * slots_per_sm;
   long best_cost = -1;
   int best_cu = units;
   for (int s = std::max(1, smin); s <= std::max(smin, smax); ++s) {
     const int cu = (units + s - 1) / s;
     if (cu > max_units) continue;
     const int ss = (units + cu - 1) / cu;
+    const long slots = (long)sms * slots_per_sm(cu);
     const long waves = ((long)pairs * ss + slots - 1) / slots;
     const long cost = waves * (cu + 4);
     if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_cu = cu; }
@@ -180,7 +183,15 @@ size_t workspace_for(const kvq_cache* c, int splits) {
   return partials_bytes(c, splits) + (size_t)c->batch * c->cfg.n_kv_heads * prep_stride(c);
 }
 
-int decode_slots_per_sm(const kvq_cache* c) { return c->is_fp4 ? 1 : 4; }
+// Resident decode CTAs per SM for a chunk of `units` 64-token units: one for the MLA kernel, the
+// tensor-core kernel's shared-memory and register limit for query groups of 1, 2 or 4, else 4.
+int decode_slots_per_sm(const kvq_cache* c, int units) {
+  if (c->is_fp4) return 1;
+  const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
+  if (group == 1 || group == 2 || group == 4)
+    return lm_mma_slots_per_sm(group, c->k, c->v, units * kTile * kTilePair);
+  return 4;
+}
 
 // Largest chunk (in 64-token units) one decode CTA may take.
 int decode_max_units(const kvq_cache* c) { return c->is_fp4 ? (1 << 30) : kChunkMax / (kTile * kTilePair); }
@@ -406,7 +417,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   for (int v : c->lens) max_len = std::max(max_len, v);
   const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
   int splits, chunk;
-  plan_splits(pairs, c->sms, decode_slots_per_sm(c), decode_max_units(c), decode_waves_bound(c), max_len,
+  plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len,
               &splits, &chunk);
   if (ws_bytes < workspace_for(c, splits)) return KVQ_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -496,7 +507,7 @@ kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const voi
   }
   const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
   int splits, chunk;
-  plan_splits(pairs, c->sms, decode_slots_per_sm(c), decode_max_units(c), decode_waves_bound(c), max_len + 1,
+  plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len + 1,
               &splits, &chunk);
   if (ws_bytes < workspace_for(c, splits)) return KVQ_ERR_WORKSPACE;
   if (c->is_fp4 || c->batch > kMaxSeqPerLaunch) {  // no fused front kernel: the two calls in sequence
@@ -544,6 +555,9 @@ kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens) {
 
 kvq_status kvq_cache_layout(const kvq_cache* c, int64_t* info, int32_t n_info) {
   if (!c || !info || n_info < 16) return KVQ_ERR_INVALID_ARG;
+  if (n_info > 16) info[16] = c->is_fp4 ? 0 : c->k.order;
+  if (n_info > 17) info[17] = c->is_fp4 ? 0 : c->v.order;
+  for (int i = 18; i < n_info; ++i) info[i] = 0;
   info[0] = kTile;
   info[1] = c->is_fp4 ? c->fp4.tile_bytes : c->k.tile_bytes;
   info[2] = c->is_fp4 ? 0 : c->v.tile_bytes;
@@ -591,6 +605,7 @@ kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_
   p.n_seq = 1;
   p.heads = 1;
   p.side[0] = c->k;
+  p.signs = c->d_signs;
   p.St = c->d_St;
   p.skip_rotation = 1;
   p.dbg_planes = planes;
@@ -651,7 +666,7 @@ extern "C" kvq_status kvq_decode_attention_static(const kvq_cache* c, const void
   for (int v : c->lens) max_len = std::max(max_len, v);
   const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
   int splits, chunk;
-  plan_splits(pairs, c->sms, decode_slots_per_sm(c), decode_max_units(c), decode_waves_bound(c), max_len,
+  plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len,
               &splits, &chunk);
   if (workspace_for(c, splits) > kStaticScratchBytes) return KVQ_ERR_WORKSPACE;
   void* scratch = nullptr;

@@ -43,9 +43,10 @@ __device__ __forceinline__ float exp2_diff(float a, float b) {
 
 constexpr int kWarps = 4;
 
-// 32-bit word k (coordinates 32k..32k+31) of token slot t of a plane at byte offset `off`.
+// 32-bit word k (coordinates 32k..32k+31) of token slot t of a plane at byte offset `off`
+// (token or byte-lane order: the caches this kernel decodes never hold octet order).
 __device__ __forceinline__ uint32_t vword(const char* tile, const SideLayout& L, int off, int t, int k) {
-  if (L.tokmajor) return *reinterpret_cast<const uint32_t*>(tile + off + t * 16 + k * 4);
+  if (L.order == kOrderToken) return *reinterpret_cast<const uint32_t*>(tile + off + t * 16 + k * 4);
   uint32_t w = 0;
 #pragma unroll
   for (int b = 0; b < 4; ++b) w |= (uint32_t)(uint8_t)tile[off + (4 * k + b) * kTile + t] << (8 * b);
@@ -247,92 +248,105 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
   }
 }
 
-// One block per (sequence, kv-head): merge the split partials of the group's G query heads,
-// fold the value sketch back (o_r += S^T acc_z, with S staged in shared memory by cp.async while
-// the partials are merged), undo the rotation (out = D H o_r / sqrt(d)) and write out.
-// Thread i owns coordinate i during the merge and the S^T product; the loads of all heads and
-// two splits are issued together so the merge costs a few memory latencies, not one per split.
-// The final Walsh-Hadamard transform runs one warp per head with shuffles.
+// One block per (sequence, kv-head), 128 threads per query head of the group. Merge: thread
+// (h, i) merges head h's split partials at coordinate i (the loads of 4 splits issued together,
+// one memory latency per 4 splits). Value sketch fold-back, o_r += S^T acc_z, with S staged in
+// shared memory by cp.async while the partials are merged: thread (q, i) sums the rows j of
+// quarter q (of G) for all G heads at once, so each staged S element is read once; the G partial
+// sums of a head meet in shared memory. Warp h then undoes the rotation of head h
+// (out = D H o_r / sqrt(d)) with shuffles and writes it out.
 template <int G>
-__global__ void __launch_bounds__(kHeadDim)
+__global__ void __launch_bounds__(G * kHeadDim)
 reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
+  constexpr int kSplitBatch = 4;
+  constexpr int kRows = kHeadDim / G;                 // sketch rows per thread in the fold-back
   extern __shared__ __align__(16) float rs[];
   float* S_s = rs;                                   // [m][d] when vq
-  float* az = rs + (vq ? p.v.m * kHeadDim : 0);      // [G][d] merged sketch accumulators
+  float* az = rs + (vq ? p.v.m * kHeadDim : 0);      // [m][G] merged sketch accumulators
   float* xs = az + G * kHeadDim;                     // [G][d] rotated-domain outputs
-  const int hk = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
-  const int lane = i & 31, warp = i >> 5;
+  float* red = xs + G * kHeadDim;                    // [G quarters][G heads][d] fold-back partials
+  const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int h = tid / kHeadDim, i = tid % kHeadDim;
+  const int lane = tid & 31, warp = tid >> 5;
   if (vq) {
-    for (int c = i; c < p.v.m * kHeadDim / 4; c += kHeadDim) cp_async16(S_s + 4 * c, p.S + 4 * c);
+    for (int c = tid; c < p.v.m * kHeadDim / 4; c += G * kHeadDim) cp_async16(S_s + 4 * c, p.S + 4 * c);
     cp_async_commit();
   }
+  float sg[4];  // the output rotation's signs and scale (warps 0..G-1), fetched while waiting
+#pragma unroll
+  for (int k = 0; k < 4; ++k) sg[k] = warp < G ? p.signs[32 * k + lane] * 0.08838834764831845f : 0.f;
   // Launched as a programmatic dependent of the decode kernel: S is staged above while that
   // grid finishes; its partials are read only after this wait.
   grid_dep_wait();
-  const size_t hstride = (size_t)p.splits * p.part_stride;  // between heads of one row block
-  const float* part0 = p.part + ((size_t)b * p.Hq + hk * G) * hstride;
-  // Online merge over groups of 4 splits: every load of a group (all heads) is issued before
-  // any is used, so the merge costs one memory latency per 4 splits.
-  float M[G], L[G], o[G], oz[G];
+  const float* part = p.part + ((size_t)b * p.Hq + hk * G + h) * (size_t)p.splits * p.part_stride;
+  float M = -INFINITY, L = 0.f, o = 0.f, oz = 0.f;
+  for (int s0 = 0; s0 < p.splits; s0 += kSplitBatch) {
+    float mv[kSplitBatch], lv[kSplitBatch], ov[kSplitBatch], zv[kSplitBatch];
 #pragma unroll
-  for (int h = 0; h < G; ++h) { M[h] = -INFINITY; L[h] = 0.f; o[h] = 0.f; oz[h] = 0.f; }
-  for (int s0 = 0; s0 < p.splits; s0 += 4) {
-    float mv[4][G], lv[4][G], ov[4][G], zv[4][G];
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const bool in = s0 + k < p.splits;
-        const float* ps = part0 + h * hstride + (size_t)(in ? s0 + k : 0) * p.part_stride;
-        mv[k][h] = in ? __ldcg(ps) : -INFINITY;
-        lv[k][h] = in ? __ldcg(ps + 1) : 0.f;
-        ov[k][h] = in ? __ldcg(ps + 2 + i) : 0.f;
-        zv[k][h] = (in && vq) ? __ldcg(ps + 2 + kHeadDim + i) : 0.f;
-      }
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float mn = fmaxf(fmaxf(M[h], fmaxf(mv[0][h], mv[1][h])), fmaxf(mv[2][h], mv[3][h]));
-      const float c = exp2_diff(M[h], mn);
-      L[h] *= c; o[h] *= c; oz[h] *= c;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float w = exp2_diff(mv[k][h], mn);
-        L[h] = fmaf(w, lv[k][h], L[h]);
-        o[h] = fmaf(w, ov[k][h], o[h]);
-        oz[h] = fmaf(w, zv[k][h], oz[h]);
-      }
-      M[h] = mn;
+    for (int k = 0; k < kSplitBatch; ++k) {
+      const bool in = s0 + k < p.splits;
+      const float* ps = part + (size_t)(in ? s0 + k : 0) * p.part_stride;
+      mv[k] = in ? __ldcg(ps) : -INFINITY;
+      lv[k] = in ? __ldcg(ps + 1) : 0.f;
+      ov[k] = in ? __ldcg(ps + 2 + i) : 0.f;
+      zv[k] = (in && vq) ? __ldcg(ps + 2 + kHeadDim + i) : 0.f;
     }
-  }
+    float mn = M;
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const float inv = (L[h] > 0.f) ? 1.f / L[h] : 0.f;
-    o[h] *= inv;
-    az[h * kHeadDim + i] = oz[h] * inv;
+    for (int k = 0; k < kSplitBatch; ++k) mn = fmaxf(mn, mv[k]);
+    const float c = exp2_diff(M, mn);
+    L *= c; o *= c; oz *= c;
+#pragma unroll
+    for (int k = 0; k < kSplitBatch; ++k) {
+      const float w = exp2_diff(mv[k], mn);
+      L = fmaf(w, lv[k], L);
+      o = fmaf(w, ov[k], o);
+      oz = fmaf(w, zv[k], oz);
+    }
+    M = mn;
   }
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  o *= inv;
   if (vq) {
+    az[i * G + h] = oz * inv;
     cp_async_wait<0>();
     __syncthreads();
-#pragma unroll 4
-    for (int j = 0; j < p.v.m; j += 4) {
-      const float s0 = S_s[j * kHeadDim + i], s1 = S_s[(j + 1) * kHeadDim + i];
-      const float s2 = S_s[(j + 2) * kHeadDim + i], s3 = S_s[(j + 3) * kHeadDim + i];
+    const int q = h;  // this thread's quarter of the sketch rows
+    float acc[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float4 a = *reinterpret_cast<const float4*>(az + h * kHeadDim + j);
-        o[h] = fmaf(s0, a.x, fmaf(s1, a.y, fmaf(s2, a.z, fmaf(s3, a.w, o[h]))));
+    for (int hh = 0; hh < G; ++hh) acc[hh] = 0.f;
+#pragma unroll 8
+    for (int j = q * kRows; j < (q + 1) * kRows; ++j) {
+      const float sv = S_s[j * kHeadDim + i];
+      if (G >= 4) {
+#pragma unroll
+        for (int h4 = 0; h4 < G; h4 += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(az + j * G + h4);
+          acc[h4] = fmaf(sv, a.x, acc[h4]);
+          acc[h4 + 1] = fmaf(sv, a.y, acc[h4 + 1]);
+          acc[h4 + 2] = fmaf(sv, a.z, acc[h4 + 2]);
+          acc[h4 + 3] = fmaf(sv, a.w, acc[h4 + 3]);
+        }
+      } else {
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) acc[hh] = fmaf(sv, az[j * G + hh], acc[hh]);
       }
     }
-  }
 #pragma unroll
-  for (int h = 0; h < G; ++h) xs[h * kHeadDim + i] = o[h];
+    for (int hh = 0; hh < G; ++hh) red[(q * G + hh) * kHeadDim + i] = acc[hh];
+    __syncthreads();
+#pragma unroll
+    for (int qq = 0; qq < G; ++qq) o += red[(qq * G + h) * kHeadDim + i];
+  }
+  xs[h * kHeadDim + i] = o;
   __syncthreads();
-  // out = D H o_r / sqrt(d): one warp per head, lane l holding coordinates 32k + l; butterflies
-  // over index bits 0..4 by shuffles, bits 5..6 in registers.
-  for (int h = warp; h < G; h += kHeadDim / 32) {
+  // lane l of warp h holds coordinates 32k + l; butterflies over index bits 0..4 by shuffles,
+  // bits 5..6 in registers.
+  if (warp < G) {
+    const int hh = warp;
     float u[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) u[k] = xs[h * kHeadDim + 32 * k + lane];
+    for (int k = 0; k < 4; ++k) u[k] = xs[hh * kHeadDim + 32 * k + lane];
 #pragma unroll
     for (int bb = 0; bb < 5; ++bb) {
       const bool upper = (lane >> bb) & 1;
@@ -344,9 +358,9 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
     }
     const float a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
     u[0] = a0 + a2; u[2] = a0 - a2; u[1] = a1 + a3; u[3] = a1 - a3;
-    float* dst = p.out + ((size_t)b * p.Hq + hk * G + h) * kHeadDim;
+    float* dst = p.out + ((size_t)b * p.Hq + hk * G + hh) * kHeadDim;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) dst[32 * k + lane] = u[k] * (p.signs[32 * k + lane] * 0.08838834764831845f);
+    for (int k = 0; k < 4; ++k) dst[32 * k + lane] = u[k] * sg[k];
   }
 }
 
@@ -390,12 +404,13 @@ cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t 
 
 template <int G>
 cudaError_t launch_reduce_g(const DecodeParams& p, cudaStream_t s) {
-  const size_t smem = sizeof(float) * ((p.v.qjl ? (size_t)p.v.m * kHeadDim : 0) + 2 * G * kHeadDim);
+  const size_t smem = sizeof(float) * ((p.v.qjl ? (size_t)p.v.m * kHeadDim : 0) + 2 * G * kHeadDim +
+                                      (size_t)G * G * kHeadDim);
   cudaError_t e = cudaFuncSetAttribute(reduce_lm<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.Hkv, p.B);
-  cfg.blockDim = dim3(kHeadDim);
+  cfg.blockDim = dim3(G * kHeadDim);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

@@ -10,10 +10,11 @@
 //       1 bit : c = a0 B0;   2 bits: c = a0 B0 + a1 B1
 //       3 bits: c = a0 B0 + a1 B1 + a2 B2 + a3 B0B1B2,   B0B1B2 = 2 (b0^b1^b2) - 1
 //     so <q, c[code]> = sum_P 2 a_P <q, b_P> - (sum_P a_P) sum_j q_j over 0/1 "Walsh planes".
-//   * Logits: A = key bits [16 tokens x 32 bits]. Byte i of plane word w holds coordinates
-//     32w + 8i + p in bit p; (w << (7 - p)) & 0x80808080 turns bit p of every byte into the int8
-//     value -128 or 0 (one multiply and one LOP3 per 4 operand bytes). B = the query term
-//     2 a_P q~_j quantised to a 16-bit integer (2 signed 8-bit digits, one column each).
+//   * Logits: A = key bits [16 tokens x 32 coordinates] from the octet-ordered key tile, where a
+//     byte holds one coordinate of 8 consecutive tokens: w & (0x01010101 << g) keeps token g of
+//     the octet in every byte, the int8 value 2^g (g < 7) or -128 (g = 7), one LOP3 per 4 operand
+//     bytes and a fixed power of two per row. B = the query term 2 a_P q~_j quantised to a
+//     16-bit integer (2 signed 8-bit digits, one column each).
 //   * Values: A = value bits [16 coordinates x 32 tokens] read from the byte-lane-major value
 //     tile, where 4 tokens of one byte-lane are one 32-bit word: w & (0x01010101 << p) gives the
 //     int8 value 2^p (p < 7) or -128 (p = 7) per byte, i.e. a fixed power of two per row. B = the
@@ -47,10 +48,12 @@ constexpr int kWarpsM = 4;
 constexpr int kThreadsM = kWarpsM * 32;
 constexpr int kCtaTok = 64;
 constexpr int kStagesM = 4;                          // bulk-copy stages (tile pairs in flight)
+constexpr int kMinBlocksM = 4;                       // resident CTAs per SM the registers are sized for
+constexpr int kSmemPerSm = 233472;                   // shared memory per SM (228 KB)
+constexpr int kSmemReserved = 1024 + 128;            // per CTA: the runtime's reserve + static arrays
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
 constexpr float kSqrtHalfPi = 1.2533141373155003f;  // sqrt(pi/2)
 constexpr int kQRange = 32639;                       // query term quantised to [-32639, 32639]
-constexpr int kLgStride = kChunkMax + 8;             // logits row stride (floats): rows on distinct banks
 constexpr int kPdStride = 96;                        // weight-digit row stride (bytes): 64 tokens + pad
 constexpr int kNormBlock = 256;                      // staged value norms / gammas of two cache tiles
 constexpr float kWRange = 8388608.f;                 // weights quantised below 2^23
@@ -148,6 +151,18 @@ struct MmaCfg {
   static constexpr int VNCOL = VNT * 8;
 };
 
+// Dynamic shared memory of one decode CTA: the staging ring, the chunk's logits, the two weight
+// digit buffers and the reduction scratch.
+size_t mma_smem_bytes(int group, const SideLayout& k, const SideLayout& v, int chunk) {
+  const int nkind = v.qjl ? 2 : 1;
+  const int vncol = ((4 * group + 7) / 8) * 8;
+  size_t s = (size_t)kStagesM * std::max(2 * k.tile_bytes + kNormBlock, 2 * v.tile_bytes);
+  s += sizeof(float) * (size_t)group * (chunk + 8);
+  s += 2 * (size_t)nkind * vncol * kPdStride;
+  s += sizeof(float) * (kWarpsM * group + 2 * kWarpsM);
+  return (s + 15) / 16 * 16;
+}
+
 // ------------------------------------------------------------------------------------------
 // Prep kernel, once per (sequence, kv-head): the logit-phase B operand.
 //   q~ = H D q * scale*log2(e)/d (rotated query),  s~ = sqrt(pi/2)/m * S q~ (sketched query)
@@ -157,7 +172,8 @@ struct MmaCfg {
 //   two full int8 digits, about 16 bits of the query term.
 // Layout per pair: [KP][G][2 digits][128 fragment-ordered coordinates] bytes, then [G][4] f32:
 // (s, C, sz, Cz) with s = vmax / (32639 * -128) (the one-hot bytes are -128), C = -(sum_P a_P)
-// sum_j q~_j and Cz = -sum_j s~_j. Fragment order of coordinate j: (j%8)*16 + (j/32)*4 + (j%32)/8.
+// sum_j q~_j and Cz = -sum_j s~_j. Coordinates in natural order: the decode kernel's operand byte
+// k of coordinate block m is coordinate 32m + k.
 // ------------------------------------------------------------------------------------------
 template <int G, int KB, bool KQ>
 __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b) {
@@ -170,16 +186,20 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b)
   extern __shared__ __align__(16) float st_s[];  // [128][m] transposed sketch matrix
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned char* out = p.qprep + ((size_t)b * p.Hkv + hk) * p.qprep_stride;
+  static_assert(G <= kWarpsM, "one query head per warp");
+  const int h0 = warp;  // this warp's query head (h0 < G)
+  float u[4];
+  if (h0 < G) {  // requested before the sketch matrix is staged
+    const size_t qb = ((size_t)b * p.Hq + hk * G + h0) * kHeadDim;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) u[k] = load_q(p.q, qb + 32 * k + lane, p.bf16) * p.signs[32 * k + lane];
+  }
   if (KQ) {  // staged while the queries are rotated
     for (int c = tid; c < kHeadDim * kHeadDim / 4; c += kThreadsM) cp_async16(st_s + 4 * c, p.St + 4 * c);
     cp_async_commit();
   }
   const float qcoef = kInvSqrtD * p.logit_scale * kInvSqrtD;
-  for (int h = warp; h < G; h += kWarpsM) {
-    float u[4];
-    const size_t qb = ((size_t)b * p.Hq + hk * G + h) * kHeadDim;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) u[k] = load_q(p.q, qb + 32 * k + lane, p.bf16) * p.signs[32 * k + lane];
+  if (h0 < G) {
 #pragma unroll
     for (int bb = 0; bb < 5; ++bb) {
       const bool upper = (lane >> bb) & 1;
@@ -190,31 +210,35 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b)
       }
     }
     const float a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
-    qf[h][lane] = (a0 + a2) * qcoef;
-    qf[h][64 + lane] = (a0 - a2) * qcoef;
-    qf[h][32 + lane] = (a1 + a3) * qcoef;
-    qf[h][96 + lane] = (a1 - a3) * qcoef;
+    qf[h0][lane] = (a0 + a2) * qcoef;
+    qf[h0][64 + lane] = (a0 - a2) * qcoef;
+    qf[h0][32 + lane] = (a1 + a3) * qcoef;
+    qf[h0][96 + lane] = (a1 - a3) * qcoef;
   }
   if (KQ) cp_async_wait<0>();
   __syncthreads();
   if (KQ) {
     const float kappa = kSqrtHalfPi / (float)p.k.m;
-    const int j = tid;  // 128 threads, one sketch row each
-    float acc[G];
+    const int j = tid;  // 128 threads, one sketch row each; two halves of the sum as separate chains
+    float acc[2][G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < kHeadDim; i += 4) {
-      const float s0 = st_s[i * kHeadDim + j], s1 = st_s[(i + 1) * kHeadDim + j];
-      const float s2 = st_s[(i + 2) * kHeadDim + j], s3 = st_s[(i + 3) * kHeadDim + j];
+    for (int h = 0; h < G; ++h) acc[0][h] = acc[1][h] = 0.f;
+#pragma unroll 2
+    for (int i = 0; i < kHeadDim / 2; i += 4) {
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float4 qv = *reinterpret_cast<const float4*>(&qf[h][i]);
-        acc[h] = fmaf(s3, qv.w, fmaf(s2, qv.z, fmaf(s1, qv.y, fmaf(s0, qv.x, acc[h]))));
+      for (int hf = 0; hf < 2; ++hf) {
+        const int ii = i + hf * (kHeadDim / 2);
+        const float s0 = st_s[ii * kHeadDim + j], s1 = st_s[(ii + 1) * kHeadDim + j];
+        const float s2 = st_s[(ii + 2) * kHeadDim + j], s3 = st_s[(ii + 3) * kHeadDim + j];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float4 qv = *reinterpret_cast<const float4*>(&qf[h][ii]);
+          acc[hf][h] = fmaf(s3, qv.w, fmaf(s2, qv.z, fmaf(s1, qv.y, fmaf(s0, qv.x, acc[hf][h]))));
+        }
       }
     }
 #pragma unroll
-    for (int h = 0; h < G; ++h) sf[h][j] = acc[h] * kappa;
+    for (int h = 0; h < G; ++h) sf[h][j] = (acc[0][h] + acc[1][h]) * kappa;
     __syncthreads();
   }
   float ka[4];
@@ -244,19 +268,28 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b)
     }
   }
   __syncthreads();
-  for (int idx = tid; idx < KP * G * kHeadDim; idx += kThreadsM) {
-    const int P = idx / (G * kHeadDim), h = (idx / kHeadDim) % G, j = idx % kHeadDim;
+  // four consecutive coordinates per step: their hi and lo digits are one 32-bit store each
+  for (int idx = tid; idx < KP * G * (kHeadDim / 4); idx += kThreadsM) {
+    const int P = idx / (G * (kHeadDim / 4)), h = (idx / (kHeadDim / 4)) % G, j0 = 4 * (idx % (kHeadDim / 4));
     const bool sk = KQ && P == KP - 1;
     float kaP = ka[0];
 #pragma unroll
     for (int r = 1; r < 4; ++r)
       if (P == r) kaP = ka[r];
-    const float v = sk ? 2.f * sf[h][j] : 2.f * kaP * qf[h][j];
-    const int q = __float2int_rn(v * qscale[h][sk ? 1 : 0]);
-    const int hi = (q + 128) >> 8, lo = q - 256 * hi;
-    const int pj = (j % 8) * 16 + (j / 32) * 4 + (j % 32) / 8;
-    out[((P * G + h) * 2 + 0) * 128 + pj] = (unsigned char)(signed char)hi;
-    out[((P * G + h) * 2 + 1) * 128 + pj] = (unsigned char)(signed char)lo;
+    const float4 src = sk ? *reinterpret_cast<const float4*>(&sf[h][j0]) : *reinterpret_cast<const float4*>(&qf[h][j0]);
+    const float mul = (sk ? 2.f : 2.f * kaP);
+    const float qs = qscale[h][sk ? 1 : 0];
+    const float vv[4] = {src.x, src.y, src.z, src.w};
+    uint32_t hw = 0u, lw = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int q = __float2int_rn((mul * vv[e]) * qs);
+      const int hi = (q + 128) >> 8, lo = q - 256 * hi;
+      hw |= (uint32_t)(hi & 0xFF) << (8 * e);
+      lw |= (uint32_t)(lo & 0xFF) << (8 * e);
+    }
+    *reinterpret_cast<uint32_t*>(out + ((P * G + h) * 2 + 0) * 128 + j0) = hw;
+    *reinterpret_cast<uint32_t*>(out + ((P * G + h) * 2 + 1) * 128 + j0) = lw;
   }
   __syncthreads();
   if (tid < 4 * G) {
@@ -294,7 +327,7 @@ decode_front(const __grid_constant__ QuantizeParams qp, const __grid_constant__ 
 // Decode kernel (two passes over the CTA's chunk).
 // ------------------------------------------------------------------------------------------
 template <int G, int KB, bool KQ, int VB, bool VQ>
-__global__ void __launch_bounds__(kThreadsM, 4)
+__global__ void __launch_bounds__(kThreadsM, kMinBlocksM)
 decode_lm_mma(const __grid_constant__ DecodeParams p) {
   using C = MmaCfg<G, KB, KQ, VB, VQ>;
   constexpr int KP = C::KP, VP = C::VP, KNT = C::KNT, VNT = C::VNT, VNCOL = C::VNCOL;
@@ -313,9 +346,11 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   using VL = TileLayout<VB, VQ>;
   constexpr int ktb = KL::BYTES, vtb = VL::BYTES;
   constexpr int stage_bytes = (2 * ktb + kNormBlock > 2 * vtb) ? 2 * ktb + kNormBlock : 2 * vtb;
+  // logits row stride (floats): chunk + 8 with the chunk a multiple of 64, so rows start on distinct banks
+  const int lgst = p.chunk + 8;
   unsigned char* stages = smem;                                            // [kStagesM][2 tiles (+ norms)]
-  float* lgs = reinterpret_cast<float*>(stages + kStagesM * stage_bytes);  // [G][kLgStride] logits
-  unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * kLgStride);  // [2][NKIND][VNCOL][kPdStride]
+  float* lgs = reinterpret_cast<float*>(stages + kStagesM * stage_bytes);  // [G][lgst] logits
+  unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * lgst);  // [2][NKIND][VNCOL][kPdStride]
   float* red = reinterpret_cast<float*>(pdig + 2 * PDB);                      // reductions
 
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
@@ -405,13 +440,16 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       }
   // this thread's logit columns (2t, 2t+1) of N-tile nt: digits (hi, lo) of head 4 nt + t
   const float* hconst = reinterpret_cast<const float*>(prep + KP * G * 2 * 128);
+  // Rows g, g + 8 of the key contraction carry operand bytes 2^g (g < 7) or -128 (g = 7); the
+  // head scales are in units of the -128 byte, so this thread's rows rescale them by rowf.
+  const float rowf = g == 7 ? 1.f : -128.f / (float)(1 << g);
   float hs[KNT], hc[KNT], hsz[KNT], hcz[KNT];
 #pragma unroll
   for (int nt = 0; nt < KNT; ++nt) {
     const int h = min(4 * nt + t, G - 1);
-    hs[nt] = __ldcg(hconst + h * 4 + 0);
+    hs[nt] = __ldcg(hconst + h * 4 + 0) * rowf;
     hc[nt] = __ldcg(hconst + h * 4 + 1);
-    hsz[nt] = __ldcg(hconst + h * 4 + 2);
+    hsz[nt] = __ldcg(hconst + h * 4 + 2) * rowf;
     hcz[nt] = __ldcg(hconst + h * 4 + 3);
   }
   const float vkappa = VQ ? kSqrtHalfPi / (float)p.v.m : 0.f;
@@ -429,46 +467,61 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     const int tok0 = it * kCtaTok;  // chunk-relative first token of this iteration
     const int count = min(kCtaTok, t_end - (t_begin + tok0));
     {
+      // Key bits in octet order: warp w's tokens 16w..16w+15 are octets o0, o0 + 1 of tile w / 2.
+      // Row g of the contraction is token 8 o0 + g, row g + 8 token 8 (o0 + 1) + g: both keep bit g
+      // of every byte, so one mask makes an operand register and every value of the row is 2^g
+      // (-128 for g = 7), a per-row scale folded into the head constants below.
       const unsigned char* ktile = kt + (tl / kTile) * ktb;
       const int s0 = (tl % kTile) + g, s1 = s0 + 8;
-      int acc[4][KNT][4], accz[2][KNT][4];  // independent chains: position pair m (z: m & 1)
+      const int o0 = (tl % kTile) / 8;
+      const uint32_t mg = 0x01010101u << g;
+      int acc[4][KNT][4], accz[2][KNT][4];  // independent chains: coordinate block m (z: m & 1)
 #pragma unroll
       for (int m = 0; m < 4; ++m)
 #pragma unroll
         for (int nt = 0; nt < KNT; ++nt)
 #pragma unroll
           for (int c = 0; c < 4; ++c) { acc[m][nt][c] = 0; if (m < 2) accz[m][nt][c] = 0; }
-      uint32_t w0[3] = {0u, 0u, 0u}, w1[3] = {0u, 0u, 0u};
-      const unsigned char* kp = ktile + KL::PLANES + t * 4;
+      // this thread's words of octet o: 8t + 2m + h, m = 0..3, h = 0..1 (32 contiguous bytes)
+      const unsigned char* kp = ktile + KL::PLANES + o0 * 128 + t * 32;
 #pragma unroll
-      for (int pp = 0; pp < KB; ++pp) {
-        w0[pp] = *reinterpret_cast<const uint32_t*>(kp + pp * (kTile * 16) + s0 * 16);
-        w1[pp] = *reinterpret_cast<const uint32_t*>(kp + pp * (kTile * 16) + s1 * 16);
-      }
+      for (int mp = 0; mp < 2; ++mp) {  // coordinate blocks 2 mp, 2 mp + 1: one 16-byte load per octet
+        uint4 wa[KB + (KQ ? 1 : 0)], wb[KB + (KQ ? 1 : 0)];  // octets o0, o0 + 1
 #pragma unroll
-      for (int P = 0; P < KP; ++P) {
-        const bool sk = KQ && P == KP - 1;
-        uint32_t x0, x1;
-        if (sk) {
-          x0 = *reinterpret_cast<const uint32_t*>(ktile + KL::SKETCH + s0 * 16 + t * 4);
-          x1 = *reinterpret_cast<const uint32_t*>(ktile + KL::SKETCH + s1 * 16 + t * 4);
-        } else {
-          x0 = walsh_word<KB>(w0, P);
-          x1 = walsh_word<KB>(w1, P);
+        for (int pp = 0; pp < KB + (KQ ? 1 : 0); ++pp) {
+          const int off = (pp < KB ? pp * (kTile * 16) : KL::SKETCH - KL::PLANES) + mp * 16;
+          wa[pp] = *reinterpret_cast<const uint4*>(kp + off);
+          wb[pp] = *reinterpret_cast<const uint4*>(kp + off + 128);
         }
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          uint32_t a0, a1, a2, a3;
-          switch (m) {
-            case 0: a0 = bit_to_s8<0>(x0); a1 = bit_to_s8<0>(x1); a2 = bit_to_s8<1>(x0); a3 = bit_to_s8<1>(x1); break;
-            case 1: a0 = bit_to_s8<2>(x0); a1 = bit_to_s8<2>(x1); a2 = bit_to_s8<3>(x0); a3 = bit_to_s8<3>(x1); break;
-            case 2: a0 = bit_to_s8<4>(x0); a1 = bit_to_s8<4>(x1); a2 = bit_to_s8<5>(x0); a3 = bit_to_s8<5>(x1); break;
-            default: a0 = bit_to_s8<6>(x0); a1 = bit_to_s8<6>(x1); a2 = bit_to_s8<7>(x0); a3 = bit_to_s8<7>(x1); break;
-          }
+        for (int mm = 0; mm < 2; ++mm) {
+          const int m = 2 * mp + mm;
 #pragma unroll
-          for (int nt = 0; nt < KNT; ++nt) {
-            if (sk) mma_s8(accz[m & 1][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
-            else mma_s8(acc[m][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+          for (int P = 0; P < KP; ++P) {
+            const bool sk = KQ && P == KP - 1;
+            uint32_t xa0, xa1, xb0, xb1;  // (octet a / b, h = 0 / 1) words of coordinate block m
+            auto pick = [&](int pp, uint32_t& a0w, uint32_t& a1w, uint32_t& b0w, uint32_t& b1w) {
+              a0w = mm ? wa[pp].z : wa[pp].x; a1w = mm ? wa[pp].w : wa[pp].y;
+              b0w = mm ? wb[pp].z : wb[pp].x; b1w = mm ? wb[pp].w : wb[pp].y;
+            };
+            if (sk) {
+              pick(KB, xa0, xa1, xb0, xb1);
+            } else if (KB == 3 && P == 3) {  // parity plane
+              uint32_t c0, c1, c2, c3;
+              pick(0, xa0, xa1, xb0, xb1);
+              pick(1, c0, c1, c2, c3);
+              xa0 ^= c0; xa1 ^= c1; xb0 ^= c2; xb1 ^= c3;
+              pick(KB - 1, c0, c1, c2, c3);
+              xa0 ^= c0; xa1 ^= c1; xb0 ^= c2; xb1 ^= c3;
+            } else {
+              pick(P < KB ? P : 0, xa0, xa1, xb0, xb1);
+            }
+            const uint32_t a0 = xa0 & mg, a1 = xb0 & mg, a2 = xa1 & mg, a3 = xb1 & mg;
+#pragma unroll
+            for (int nt = 0; nt < KNT; ++nt) {
+              if (sk) mma_s8(accz[m & 1][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+              else mma_s8(acc[m][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+            }
           }
         }
       }
@@ -500,8 +553,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         }
         const float lg0 = v0 ? nk0 * l0 : -INFINITY, lg1 = v1 ? nk1 * l1 : -INFINITY;
         if (h < G) {
-          lgs[h * kLgStride + tok0 + tl + g] = lg0;
-          lgs[h * kLgStride + tok0 + tl + g + 8] = lg1;
+          lgs[h * lgst + tok0 + tl + g] = lg0;
+          lgs[h * lgst + tok0 + tl + g + 8] = lg1;
         }
         mrow[nt] = fmaxf(mrow[nt], fmaxf(lg0, lg1));
       }
@@ -564,7 +617,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     const unsigned char* vtile = stages + ((n_iter + it) % kStagesM) * stage_bytes + (T / kTile) * vtb;
     float lv[TPT], wc[TPT], wz[TPT];
     if (TPT == 2) {
-      const float2 l2 = *reinterpret_cast<const float2*>(lgs + task_h * kLgStride + tok0 + T);
+      const float2 l2 = *reinterpret_cast<const float2*>(lgs + task_h * lgst + tok0 + T);
       const float2 n2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::NORM + (T % kTile) * 2));
       lv[0] = l2.x; lv[TPT - 1] = l2.y; wc[0] = n2.x; wc[TPT - 1] = n2.y;
       if (VQ) {
@@ -572,7 +625,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         wz[0] = g2.x; wz[TPT - 1] = g2.y;
       }
     } else {
-      lv[0] = lgs[task_h * kLgStride + tok0 + T];
+      lv[0] = lgs[task_h * lgst + tok0 + T];
       wc[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::NORM + (T % kTile) * 2));
       if (VQ) wz[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::GAMMA + (T % kTile) * 2));
     }
@@ -774,19 +827,9 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 }
 
 template <int G, int KB, bool KQ, int VB, bool VQ>
-size_t mma_smem_bytes(const DecodeParams& p) {
-  using C = MmaCfg<G, KB, KQ, VB, VQ>;
-  constexpr int NKIND = VQ ? 2 : 1;
-  size_t s = (size_t)kStagesM * std::max(2 * TileLayout<KB, KQ>::BYTES + kNormBlock, 2 * TileLayout<VB, VQ>::BYTES);
-  s += sizeof(float) * (size_t)G * kLgStride;
-  s += 2 * (size_t)NKIND * C::VNCOL * kPdStride;
-  s += sizeof(float) * (kWarpsM * G + 2 * kWarpsM);
-  return (s + 15) / 16 * 16;
-}
-
-template <int G, int KB, bool KQ, int VB, bool VQ>
 cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
   if (!TileLayout<KB, KQ>::matches(p.k) || !TileLayout<VB, VQ>::matches(p.v)) return cudaErrorNotSupported;
+  if (p.k.order != kOrderOctet || p.v.order != kOrderByteLane) return cudaErrorNotSupported;
   const size_t prep_smem = KQ ? sizeof(float) * kHeadDim * kHeadDim : 0;
   cudaError_t e = cudaFuncSetAttribute(decode_lm_prep<G, KB, KQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep_smem);
@@ -803,7 +846,7 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid
   e = launched();
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
-  const size_t smem = mma_smem_bytes<G, KB, KQ, VB, VQ>(p);
+  const size_t smem = mma_smem_bytes(G, p.k, p.v, p.chunk);
   auto kern = decode_lm_mma<G, KB, KQ, VB, VQ>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -845,6 +888,21 @@ int mma_prep_bytes(int k_bits, int k_qjl, int group) {
   const int kp = (k_bits == 3 ? 4 : k_bits) + (k_qjl ? 1 : 0);
   const int bytes = kp * group * 2 * 128 + 16 * group;
   return (bytes + 255) / 256 * 256;
+}
+
+bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl) {
+  if (group != 1 && group != 2 && group != 4) return false;
+  // the (K bits, K sketch, V bits, V sketch) instances of dispatch_mma_modes
+  static const int kModes[][4] = {{2, 1, 2, 1}, {3, 1, 3, 0}, {1, 0, 1, 0}, {2, 1, 2, 0},
+                                  {3, 1, 3, 1}, {2, 0, 2, 0}, {3, 0, 3, 0}};
+  for (const auto& m : kModes)
+    if (m[0] == k_bits && m[1] == (k_qjl ? 1 : 0) && m[2] == v_bits && m[3] == (v_qjl ? 1 : 0)) return true;
+  return false;
+}
+
+int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk) {
+  const size_t per = mma_smem_bytes(group, k, v, chunk) + kSmemReserved;
+  return std::max(1, std::min(kMinBlocksM, (int)(kSmemPerSm / per)));
 }
 
 bool mma_decode_supported(const DecodeParams& p) {

@@ -20,15 +20,26 @@ constexpr int kChunkMax = 2048;   // largest context chunk of one decode CTA (LM
 constexpr int kStatusWords = 8;   // device status ints kept after the lengths in the arena
 constexpr long long kWaitLimitCycles = 1ll << 31;  // ~1 s at 2 GHz: a staged-data wait gives up
 
+// Orders of the 512 bytes of one plane (or of the sign words) of a 32-token tile. A token's 128
+// bits are 16 bytes, byte k holding coordinates 8k..8k+7 (coordinate 8k + i in bit i).
+//   kOrderByteLane: [16 byte-lanes][32 tokens] (values).
+//   kOrderToken:    [32 tokens][16 B] (keys decoded on CUDA cores).
+//   kOrderOctet:    bit-transposed for the tensor-core key contraction: [4 octets][32 words],
+//                   octet o = tokens 8o..8o+7; word x = 8t + 2m + h, byte i of it covers
+//                   coordinate 32m + 16h + 4t + i, bit j of that byte is token 8o + j.
+constexpr int kOrderByteLane = 0;
+constexpr int kOrderToken = 1;
+constexpr int kOrderOctet = 2;
+
 // Where one side (K or V) of an LM/SIGN1 cache keeps its fields inside a 32-token tile.
 struct SideLayout {
   int bits = 0;         // code bit-planes
   int qjl = 0;          // 1 if a residual sign sketch is stored
-  int tokmajor = 1;     // 1: [32 tokens][16 B] per plane; 0: [16 byte-lanes][32 tokens]
+  int order = 1;        // plane / sign-word order within a tile: one of the kOrder* below
   int m = 0;            // sketch rows
   int tile_bytes = 0;
-  int off_planes = 0;   // [bits][32 x 16 B] (layout per tokmajor)
-  int off_sketch = 0;   // [32 x m/8 B] (layout per tokmajor)
+  int off_planes = 0;   // [bits][512 B] (layout per order)
+  int off_sketch = 0;   // [m/8 x 32 B] (layout per order)
   int off_norm = 0;     // [32] fp16
   int off_gamma = 0;    // [32] fp16
   float cent[8] = {};   // fp32 Lloyd-Max centroids (2^bits, ascending)
@@ -118,6 +129,12 @@ cudaError_t launch_quantize_fp4(const QuantizeParams& p, cudaStream_t s);
 cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid = nullptr,
                              const QuantizeParams* qp = nullptr);
 bool mma_decode_supported(const DecodeParams& p);
+// Resident CTAs per SM of the tensor-core decode kernel for a chunk of `chunk` tokens (shared
+// memory and registers), as the split plan counts them.
+int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk);
+// True when the tensor-core decode kernel handles this query group and code combination (the
+// cache then stores its keys in kOrderOctet).
+bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl);
 int mma_prep_bytes(int k_bits, int k_qjl, int group);  // bytes of one (sequence, kv-head) prep area
 cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp);
 cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s);

@@ -27,6 +27,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 constexpr int kLmWarps = 4;     // LM quantize: warps per block
 
+// Bits 0..3 of x moved to bits 0, 8, 16, 24.
+__device__ __forceinline__ uint32_t spread_nibble(uint32_t x) {
+  return (x & 1u) | ((x & 2u) << 7) | ((x & 4u) << 14) | ((x & 8u) << 21);
+}
+
 // Blocks per side of an LM quantize launch: one vector per block on sides with a sketch (the
 // block's warps share it), one per warp otherwise; at most 16 blocks per SM of a B200.
 inline int blocks_per_side(const QuantizeParams& p) {
@@ -43,7 +48,7 @@ inline int blocks_per_side(const QuantizeParams& p) {
 // projections j = 32w + lane, from its own 16 KB column slice of S^T staged in shared memory.
 // Sides without a sketch: one vector per warp.
 __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int side, int blk, int nblk) {
-  __shared__ float rho_s[kLmWarps][kHeadDim];
+  __shared__ __align__(16) float rho_s[kLmWarps][kHeadDim];
   extern __shared__ __align__(16) float st_s[];  // sketch sides: [warp][d][32] columns 32w.. of S^T
   const SideLayout& L = p.side[side];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -61,14 +66,20 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
     }
     cp_async_commit();
   }
+  // Everything the first vector needs from global memory is requested before the staged slice
+  // is waited for (which happens only right before the sketch product).
   float u_first[4] = {0.f, 0.f, 0.f, 0.f};
   if (first < total)
 #pragma unroll
     for (int k = 0; k < 4; ++k) u_first[k] = load_elem(p.src[side], (size_t)first * kHeadDim + 32 * k + lane, p.bf16);
-  if (coop) {
-    cp_async_wait<0>();
-    __syncwarp();
-  }
+  float sg[4];  // rotation signs (the debug entry's inputs are already rotated: none read)
+#pragma unroll
+  for (int k = 0; k < 4; ++k) sg[k] = p.skip_rotation ? 1.f : p.signs[32 * k + lane];
+  // the table in registers: thresholds (unused ones +inf), centroid c held by lane c % 8
+  float thr[7];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) thr[i] = i < nthr ? L.thr[i] : INFINITY;
+  const float cent_lane = L.cent[(lane & 7) <= nthr ? (lane & 7) : 0];
 
   for (long vec = first; vec < total; vec += stride) {
     const int t = (int)(vec % p.n_new);
@@ -84,7 +95,7 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
     if (!p.skip_rotation) {
       n = sqrtf(warp_sum(u[0] * u[0] + u[1] * u[1] + u[2] * u[2] + u[3] * u[3]));
 #pragma unroll
-      for (int k = 0; k < 4; ++k) u[k] *= p.signs[32 * k + lane];
+      for (int k = 0; k < 4; ++k) u[k] *= sg[k];
       // Walsh-Hadamard butterflies over index bits 0..4 (lane) and 5..6 (k).
 #pragma unroll
       for (int b = 0; b < 5; ++b) {
@@ -106,9 +117,10 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       int c = 0;
-      for (int i = 0; i < nthr; ++i) c += (u[k] >= L.thr[i]) ? 1 : 0;
+#pragma unroll
+      for (int i = 0; i < 7; ++i) c += (u[k] >= thr[i]) ? 1 : 0;
       code[k] = c;
-      rho[k] = u[k] - L.cent[c];
+      rho[k] = u[k] - __shfl_sync(0xffffffffu, cent_lane, c);
     }
     uint32_t planes[kMaxBits][4];
 #pragma unroll
@@ -129,9 +141,18 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
 #pragma unroll
       for (int k = 0; k < 4; ++k) rho_s[warp][32 * k + lane] = rho[k];
       __syncwarp();
-      float proj = 0.f;  // (S rho)_j, j = 32 warp + lane
-#pragma unroll 16
-      for (int i = 0; i < kHeadDim; ++i) proj = fmaf(stw[i * 32 + lane], rho_s[warp][i], proj);
+      if (vec == first) cp_async_wait<0>();  // the staged slice (requested at the start)
+      __syncwarp();
+      float pr[4] = {0.f, 0.f, 0.f, 0.f};  // (S rho)_j, j = 32 warp + lane: four partial chains
+#pragma unroll 8
+      for (int i = 0; i < kHeadDim; i += 4) {
+        const float4 r = *reinterpret_cast<const float4*>(&rho_s[warp][i]);
+        pr[0] = fmaf(stw[i * 32 + lane], r.x, pr[0]);
+        pr[1] = fmaf(stw[(i + 1) * 32 + lane], r.y, pr[1]);
+        pr[2] = fmaf(stw[(i + 2) * 32 + lane], r.z, pr[2]);
+        pr[3] = fmaf(stw[(i + 3) * 32 + lane], r.w, pr[3]);
+      }
+      const float proj = (pr[0] + pr[1]) + (pr[2] + pr[3]);
       __syncwarp();
       zword = __ballot_sync(0xffffffffu, proj >= 0.f);
     }
@@ -150,10 +171,36 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
     const int tile = pos / kTile, slot = pos % kTile;
     char* tb = p.region[side] +
                (((size_t)seq * p.heads + h) * p.tiles_per_seq + tile) * (size_t)L.tile_bytes;
-    if (L.tokmajor) {
+    if (L.order == kOrderToken) {
       if (lead && lane < L.bits)
         *reinterpret_cast<uint4*>(tb + L.off_planes + lane * (kTile * 16) + slot * 16) = mine;
       if (coop && lane == 0) *reinterpret_cast<uint32_t*>(tb + L.off_sketch + slot * 16 + 4 * warp) = zword;
+    } else if (L.order == kOrderOctet) {
+      // bit (slot % 8) of each byte of word x = 8t + 2m + h of octet slot / 8; byte i of the word
+      // is coordinate 32m + 16h + 4t + i. Neighbouring tokens share the words, so this token's bits
+      // are cleared and set with atomics (other tokens' bits are never touched).
+      const uint32_t jmask = 0x01010101u << (slot & 7);
+      uint32_t* octet = reinterpret_cast<uint32_t*>(tb) + (slot >> 3) * 32;
+      if (lead) {  // lane = word x of every plane
+        const int wt = lane >> 3, wm = (lane >> 1) & 3, wh = lane & 1;
+#pragma unroll
+        for (int pp = 0; pp < kMaxBits; ++pp) {
+          if (pp < L.bits) {
+            const uint32_t src = wm == 0 ? planes[pp][0] : wm == 1 ? planes[pp][1] : wm == 2 ? planes[pp][2] : planes[pp][3];
+            const uint32_t bits4 = (src >> (16 * wh + 4 * wt)) & 0xFu;
+            uint32_t* w = octet + (L.off_planes + pp * (kTile * 16)) / 4 + lane;
+            atomicAnd(w, ~jmask);
+            atomicOr(w, spread_nibble(bits4) << (slot & 7));
+          }
+        }
+      }
+      if (coop && lane < 8) {  // sign word `warp` is coordinate block m = warp: words 8t + 2 warp + h
+        const int wt = lane >> 1, wh = lane & 1;
+        const uint32_t bits4 = (zword >> (16 * wh + 4 * wt)) & 0xFu;
+        uint32_t* w = octet + L.off_sketch / 4 + 8 * wt + 2 * warp + wh;
+        atomicAnd(w, ~jmask);
+        atomicOr(w, spread_nibble(bits4) << (slot & 7));
+      }
     } else {
       // byte-lane-major: byte k of a token's 16-byte plane goes to [k][slot]
       if (lead && lane < 16) {

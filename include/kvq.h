@@ -182,16 +182,19 @@ kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens);
 /* Byte offsets describing the packed layout, for tools that read the arena directly.
  * info[0..15] receives: tile_tokens, k_tile_bytes, v_tile_bytes, tiles_per_seq,
  * k_region_offset, v_region_offset, then per side (K at 6, V at 11): planes_offset,
- * sketch_offset, norm_offset, gamma_offset, planes. Layout of a tile (32 tokens) of one
- * (sequence, kv-head): code bit-planes, then sign words, then [32] fp16 norms, then [32] fp16
- * residual norms (sides with a sketch). Plane p holds bit p of every code; within a token's
- * 16-byte plane, 32-bit word w holds coordinates 32w..32w+31, coordinate 32w+i in bit i, i.e.
- * byte k holds coordinates 8k..8k+7. Sign words use the same order (bit = 1 for a non-negative
- * projection). Key planes and key sign words are token-major: [planes][32 tokens][16 bytes],
- * [32][16 bytes]. Value planes and value sign words are byte-lane-major: [planes][16 byte
- * lanes][32 tokens], [16][32], byte (k, t) being byte k of token t's 16 bytes. Tiles of a
- * (sequence, kv-head) are consecutive; (sequence, kv-head) pairs follow in row-major order.
- * Capacity is rounded up to whole pairs of tiles (64 tokens).
+ * sketch_offset, norm_offset, gamma_offset, planes; with n_info >= 18 also info[16], info[17]:
+ * the order of the K and V planes (0 byte-lane, 1 token, 2 octet). Layout of a tile (32 tokens)
+ * of one (sequence, kv-head): code bit-planes (512 bytes each), then sign words (512 bytes),
+ * then [32] fp16 norms, then [32] fp16 residual norms (sides with a sketch). Plane p holds bit p
+ * of every code; a token's 128 bits of a plane are 16 bytes, byte k holding coordinates
+ * 8k..8k+7 (coordinate 8k+i in bit i); sign words use the same order (bit = 1 for a
+ * non-negative projection). The three orders of those bytes within a plane or the sign block:
+ *   byte-lane (values): [16 byte lanes][32 tokens], byte (k, t) = byte k of token t;
+ *   token (keys of query groups the tensor-core kernel does not decode): [32 tokens][16 bytes];
+ *   octet (all other keys): [4 octets][32 words of 4 bytes], octet o = tokens 8o..8o+7; byte i
+ *   of word x = 8t + 2m + h covers coordinate 32m + 16h + 4t + i, bit j of it is token 8o + j.
+ * Tiles of a (sequence, kv-head) are consecutive; (sequence, kv-head) pairs follow in row-major
+ * order. Capacity is rounded up to whole pairs of tiles (64 tokens).
  * FP4: [32][latent_dim/2] codes (channel 2k in the low nibble of byte k), [32][latent_dim/16]
  * E4M3 scales, [32][rope_dim] bf16 RoPE keys. */
 kvq_status kvq_cache_layout(const kvq_cache* c, int64_t* info, int32_t n_info);

@@ -13,6 +13,24 @@ def _tiles(arena: np.ndarray, region: int, pair: int, tiles: int, tile_bytes: in
     return arena[start:start + nt * tile_bytes].reshape(nt, tile_bytes)
 
 
+ORDER_BYTE_LANE, ORDER_TOKEN, ORDER_OCTET = 0, 1, 2
+
+
+def _octet_to_token_major(raw: np.ndarray, nt: int, nplanes: int) -> np.ndarray:
+    """Octet-ordered planes [nt, nplanes * 512] bytes -> token-major uint8 [nt, nplanes, 32, 16].
+
+    Octet order: [4 octets][32 words]; word x = 8t + 2m + h, byte i of it is coordinate
+    32m + 16h + 4t + i, bit j of that byte is token 8 * octet + j."""
+    B = raw.reshape(nt, nplanes, 4, 32, 4)
+    x = np.arange(32)
+    coord = (32 * ((x // 2) % 4) + 16 * (x % 2) + 4 * (x // 8))[:, None] + np.arange(4)[None, :]
+    bits = (B[..., None] >> np.arange(8, dtype=np.uint8)) & 1          # [nt, np, o, x, i, j]
+    per_tok = np.zeros((nt, nplanes, 4, 8, 128), dtype=np.uint8)       # [nt, np, o, j, coord]
+    per_tok[..., coord] = bits.transpose(0, 1, 2, 5, 3, 4)
+    per_tok = per_tok.reshape(nt, nplanes, 32, 16, 8)                  # coordinate 8k + b
+    return (per_tok << np.arange(8, dtype=np.uint8)).sum(axis=-1).astype(np.uint8)
+
+
 def side_fields(arena: np.ndarray, info, side: int, pair: int, n_tokens: int, m: int = 128):
     """planes uint32 [T, bits, 4], sketch uint32 [T, m/32] (or None), n16, gamma16 float64 [T]
     for one (sequence, kv-head) pair index (b * Hkv + h) and its first n_tokens tokens."""
@@ -23,9 +41,13 @@ def side_fields(arena: np.ndarray, info, side: int, pair: int, n_tokens: int, m:
     qjl = off_norm > off_sketch  # a side without a sketch has an empty sketch block
     tb = _tiles(arena, region, pair, tiles, tile_bytes, n_tokens)
     nt = tb.shape[0]
-    # keys: token-major [bits][32 tokens][16 B]; values: byte-lane-major [bits][16][32 tokens]
+    # keys: token-major [bits][32 tokens][16 B] or octet order (info[16]); values: byte-lane-major
+    # [bits][16][32 tokens]
+    order = (int(info[16]) if len(info) > 16 else ORDER_TOKEN) if side == 0 else ORDER_BYTE_LANE
     raw = tb[:, off_planes:off_planes + bits * TILE * 16]
-    if side == 0:
+    if order == ORDER_OCTET:
+        planes = np.ascontiguousarray(_octet_to_token_major(raw, nt, bits).transpose(0, 2, 1, 3))
+    elif order == ORDER_TOKEN:
         planes = np.ascontiguousarray(raw.reshape(nt, bits, TILE, 16).transpose(0, 2, 1, 3))
     else:
         planes = np.ascontiguousarray(raw.reshape(nt, bits, 16, TILE).transpose(0, 3, 1, 2))
@@ -34,7 +56,9 @@ def side_fields(arena: np.ndarray, info, side: int, pair: int, n_tokens: int, m:
     sketch, g16 = None, np.zeros(n_tokens)
     if qjl:
         raw = tb[:, off_sketch:off_sketch + TILE * m // 8]
-        if side == 0:
+        if order == ORDER_OCTET:
+            sk = np.ascontiguousarray(_octet_to_token_major(raw, nt, 1)).reshape(nt * TILE, m // 8)
+        elif order == ORDER_TOKEN:
             sk = np.ascontiguousarray(raw).reshape(nt * TILE, m // 8)
         else:
             sk = np.ascontiguousarray(raw.reshape(nt, m // 8, TILE).transpose(0, 2, 1)).reshape(nt * TILE, m // 8)
