@@ -357,6 +357,8 @@ void fill_quantize(QuantizeParams& p, const kvq_cache* c, const void* K, const v
   p.signs = c->d_signs;
   p.St = c->d_St;
   p.lens = c->d_lens;
+  p.err = c->d_status;
+  p.wait_limit = kWaitLimitCycles;
   for (int i = 0; i < cnt; ++i) {
     const int sid = seq_ids ? seq_ids[first + i] : first + i;
     p.seq[i] = sid;
@@ -607,6 +609,8 @@ kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_
   p.side[0] = c->k;
   p.signs = c->d_signs;
   p.St = c->d_St;
+  p.err = c->d_status;
+  p.wait_limit = kWaitLimitCycles;
   p.skip_rotation = 1;
   p.dbg_planes = planes;
   p.dbg_sketch = sketch;

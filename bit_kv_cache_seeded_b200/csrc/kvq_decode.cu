@@ -268,6 +268,7 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
   const int hk = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int h = tid / kHeadDim, i = tid % kHeadDim;
   const int lane = tid & 31, warp = tid >> 5;
+  grid_dep_launch();  // a following fused step's first kernel may start its setup now
   if (vq) {
     for (int c = tid; c < p.v.m * kHeadDim / 4; c += G * kHeadDim) cp_async16(S_s + 4 * c, p.S + 4 * c);
     cp_async_commit();

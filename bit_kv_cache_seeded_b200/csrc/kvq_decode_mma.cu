@@ -183,20 +183,29 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b)
   __shared__ __align__(16) float sf[G][kHeadDim];
   __shared__ float hc[G][4];
   __shared__ float qscale[G][2];                 // 32639 / vmax: centroid planes, sketch
+  __shared__ __align__(8) uint64_t st_bar;       // completes when S^T has landed
   extern __shared__ __align__(16) float st_s[];  // [128][m] transposed sketch matrix
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned char* out = p.qprep + ((size_t)b * p.Hkv + hk) * p.qprep_stride;
   static_assert(G <= kWarpsM, "one query head per warp");
   const int h0 = warp;  // this warp's query head (h0 < G)
+  if (KQ && tid == 0) {  // one bulk copy, landing while the queries are rotated
+    const uint32_t bar = smem_addr(&st_bar);
+    mbar_init(bar, 1);
+    mbar_init_fence();
+    constexpr uint32_t kQuarter = kHeadDim * kHeadDim / 4;  // floats in a quarter of S^T (16 KB)
+    mbar_arrive_expect_tx(bar, 4u * kQuarter * 4u);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) bulk_g2s(smem_addr(st_s + c * kQuarter), p.St + c * kQuarter, kQuarter * 4u, bar);
+  }
   float u[4];
-  if (h0 < G) {  // requested before the sketch matrix is staged
+  // Launched as a programmatic dependent (fused decode step): the query may come from the
+  // preceding kernel, so wait for it (the sketch matrix requested above is the cache's own).
+  grid_dep_wait();
+  if (h0 < G) {
     const size_t qb = ((size_t)b * p.Hq + hk * G + h0) * kHeadDim;
 #pragma unroll
     for (int k = 0; k < 4; ++k) u[k] = load_q(p.q, qb + 32 * k + lane, p.bf16) * p.signs[32 * k + lane];
-  }
-  if (KQ) {  // staged while the queries are rotated
-    for (int c = tid; c < kHeadDim * kHeadDim / 4; c += kThreadsM) cp_async16(st_s + 4 * c, p.St + 4 * c);
-    cp_async_commit();
   }
   const float qcoef = kInvSqrtD * p.logit_scale * kInvSqrtD;
   if (h0 < G) {
@@ -215,8 +224,12 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b)
     qf[h0][32 + lane] = (a1 + a3) * qcoef;
     qf[h0][96 + lane] = (a1 - a3) * qcoef;
   }
-  if (KQ) cp_async_wait<0>();
-  __syncthreads();
+  __syncthreads();  // the rotated queries; the barrier below was initialised before this
+  bool st_failed = false;
+  if (KQ && !mbar_try(smem_addr(&st_bar), 0u) && !mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit)) {
+    st_failed = true;
+    atomicOr(p.err, 1);
+  }
   if (KQ) {
     const float kappa = kSqrtHalfPi / (float)p.k.m;
     const int j = tid;  // 128 threads, one sketch row each; two halves of the sum as separate chains
@@ -292,6 +305,7 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b)
     *reinterpret_cast<uint32_t*>(out + ((P * G + h) * 2 + 1) * 128 + j0) = lw;
   }
   __syncthreads();
+  if (st_failed) mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit);  // nothing may land after exit
   if (tid < 4 * G) {
     const int h = tid / 4, k = tid % 4;
     float v = hc[h][k];
@@ -839,7 +853,20 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid
     const size_t fsmem = std::max(prep_smem, (size_t)sizeof(float) * kHeadDim * kHeadDim);
     e = cudaFuncSetAttribute(decode_front<G, KB, KQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem);
     if (e != cudaSuccess) return e;
-    decode_front<G, KB, KQ><<<2 * nq + p.B * p.Hkv, kThreadsM, fsmem, s>>>(*qp, p, nq);
+    // a programmatic dependent of whatever precedes it: its launch and setup overlap that
+    // kernel's tail, and it waits for it before reading inputs
+    cudaLaunchConfig_t fc = {};
+    fc.gridDim = dim3(2 * nq + p.B * p.Hkv);
+    fc.blockDim = dim3(kThreadsM);
+    fc.dynamicSmemBytes = fsmem;
+    fc.stream = s;
+    cudaLaunchAttribute fa[1];
+    fa[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    fa[0].val.programmaticStreamSerializationAllowed = 1;
+    fc.attrs = fa;
+    fc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&fc, decode_front<G, KB, KQ>, *qp, p, nq);
+    if (e != cudaSuccess) return e;
   } else {
     decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv, p.B), kThreadsM, prep_smem, s>>>(p);
   }

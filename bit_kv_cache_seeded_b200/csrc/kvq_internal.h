@@ -16,7 +16,8 @@ constexpr int kHeadDim = 128;      // head_dim supported by the rotated (LM/SIGN
 constexpr int kMaxSeqPerLaunch = 1024;
 constexpr int kMaxBits = 3;
 constexpr int kTilePair = 2;      // cache tiles are allocated and split in pairs (64 tokens)
-constexpr int kChunkMax = 2048;   // largest context chunk of one decode CTA (LM tensor-core path)
+constexpr int kChunkMax = 2240;   // largest context chunk of one decode CTA (LM tensor-core path): its
+                                  // logits still leave room for four CTAs per SM (query group 4)
 constexpr int kStatusWords = 8;   // device status ints kept after the lengths in the arena
 constexpr long long kWaitLimitCycles = 1ll << 31;  // ~1 s at 2 GHz: a staged-data wait gives up
 
@@ -70,6 +71,8 @@ struct QuantizeParams {
   uint32_t* dbg_planes;  // debug outputs (skip_rotation only)
   uint32_t* dbg_sketch;
   uint16_t* dbg_gamma;
+  int* err;              // cache status word: bit 0 set when a wait for staged data gave up
+  long long wait_limit;  // SM clock cycles a block waits for staged data before giving up
   int seq[kMaxSeqPerLaunch];
   int pos[kMaxSeqPerLaunch];
 };

@@ -43,13 +43,15 @@ inline int blocks_per_side(const QuantizeParams& p) {
   return blocks < 1 ? 1 : (int)blocks;
 }
 
-// One block of the LM quantize (`blk` of `nblk` blocks of side `side`). Sides with a sketch: the block's 4 warps share one vector; each redoes steps 1-5
-// (cheap, and it keeps every warp independent), then warp w forms sketch word w, i.e. the 32
-// projections j = 32w + lane, from its own 16 KB column slice of S^T staged in shared memory.
+// One block of the LM quantize (`blk` of `nblk` blocks of side `side`). Sides with a sketch: the
+// block's 4 warps share one vector; each redoes steps 1-5 (cheap, and it keeps every warp
+// independent), then warp w forms sketch word w, i.e. the 32 projections j = 32w + lane, from
+// columns 32w.. of S^T, which one bulk copy brings into shared memory while steps 1-5 run.
 // Sides without a sketch: one vector per warp.
 __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int side, int blk, int nblk) {
   __shared__ __align__(16) float rho_s[kLmWarps][kHeadDim];
-  extern __shared__ __align__(16) float st_s[];  // sketch sides: [warp][d][32] columns 32w.. of S^T
+  __shared__ __align__(8) uint64_t st_bar;       // completes when S^T has landed
+  extern __shared__ __align__(16) float st_s[];  // sketch sides: S^T [d][m], m = d = 128
   const SideLayout& L = p.side[side];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nthr = L.bits ? (1 << L.bits) - 1 : 0;
@@ -57,17 +59,26 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
   const long total = (long)p.n_seq * p.heads * p.n_new;
   const long first = coop ? (long)blk : (long)blk * kLmWarps + warp;
   const long stride = coop ? (long)nblk : (long)nblk * kLmWarps;
-  float* stw = st_s + warp * kHeadDim * 32;  // stw[i * 32 + l] = S^T[i][32 warp + l] = S[32 warp + l][i]
-  // The slice is staged asynchronously while the first vector's elements are fetched.
-  if (coop && first < total) {
-    for (int c = lane; c < kHeadDim * 8; c += 32) {  // row i = c / 8, 16-byte chunk c % 8 of its 32 floats
-      const int i = c >> 3, ch = c & 7;
-      cp_async16(stw + i * 32 + ch * 4, p.St + (size_t)i * L.m + 32 * warp + ch * 4);
+  const bool staged = coop && first < total;  // the same for every thread of the block
+  bool st_failed = false;
+  if (staged) {
+    if (threadIdx.x == 0) {
+      const uint32_t bar = smem_addr(&st_bar);
+      mbar_init(bar, 1);
+      mbar_init_fence();
+      constexpr uint32_t kQuarter = kHeadDim * kHeadDim / 4;  // floats in a quarter of S^T (16 KB)
+      mbar_arrive_expect_tx(bar, 4u * kQuarter * 4u);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) bulk_g2s(smem_addr(st_s + c * kQuarter), p.St + c * kQuarter, kQuarter * 4u, bar);
     }
-    cp_async_commit();
+    __syncthreads();  // the barrier is initialised before anyone waits on it
   }
+  const float* stw = st_s + 32 * warp + lane;  // stw[i * d] = S^T[i][32 warp + lane] = S[32 warp + lane][i]
   // Everything the first vector needs from global memory is requested before the staged slice
   // is waited for (which happens only right before the sketch product).
+  // Launched as a programmatic dependent (fused decode step): everything above reads only the
+  // cache's own constants; the inputs may come from the preceding kernel, so wait for it here.
+  grid_dep_wait();
   float u_first[4] = {0.f, 0.f, 0.f, 0.f};
   if (first < total)
 #pragma unroll
@@ -141,16 +152,20 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
 #pragma unroll
       for (int k = 0; k < 4; ++k) rho_s[warp][32 * k + lane] = rho[k];
       __syncwarp();
-      if (vec == first) cp_async_wait<0>();  // the staged slice (requested at the start)
+      if (vec == first && !mbar_try(smem_addr(&st_bar), 0u) &&
+          !mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit)) {  // S^T (requested at the start)
+        st_failed = true;
+        atomicOr(p.err, 1);
+      }
       __syncwarp();
       float pr[4] = {0.f, 0.f, 0.f, 0.f};  // (S rho)_j, j = 32 warp + lane: four partial chains
 #pragma unroll 8
       for (int i = 0; i < kHeadDim; i += 4) {
         const float4 r = *reinterpret_cast<const float4*>(&rho_s[warp][i]);
-        pr[0] = fmaf(stw[i * 32 + lane], r.x, pr[0]);
-        pr[1] = fmaf(stw[(i + 1) * 32 + lane], r.y, pr[1]);
-        pr[2] = fmaf(stw[(i + 2) * 32 + lane], r.z, pr[2]);
-        pr[3] = fmaf(stw[(i + 3) * 32 + lane], r.w, pr[3]);
+        pr[0] = fmaf(stw[i * kHeadDim], r.x, pr[0]);
+        pr[1] = fmaf(stw[(i + 1) * kHeadDim], r.y, pr[1]);
+        pr[2] = fmaf(stw[(i + 2) * kHeadDim], r.z, pr[2]);
+        pr[3] = fmaf(stw[(i + 3) * kHeadDim], r.w, pr[3]);
       }
       const float proj = (pr[0] + pr[1]) + (pr[2] + pr[3]);
       __syncwarp();
@@ -222,6 +237,8 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
       *reinterpret_cast<__half*>(tb + L.off_gamma + slot * 2) = __float2half_rn(gamma);
   }
 
+  // a wait that gave up: the copy may still be landing, so wait for it (bounded) before leaving
+  if (st_failed) mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit);
   if (side == 0 && blk == 0 && !p.skip_rotation)
     for (int i = threadIdx.x; i < p.n_seq; i += blockDim.x) p.lens[p.seq[i]] = p.pos[i] + p.n_new;
 }
