@@ -28,6 +28,10 @@ __device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
 }
+// One plain arrival on the barrier (release semantics at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
 // Orders this thread's earlier generic-proxy shared-memory accesses (after a barrier, those of
 // the whole CTA) before later bulk copies into the same buffer.
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
@@ -45,14 +49,15 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the barrier's phase with parity `parity` has completed, giving up after `limit`
-// SM clock cycles. Returns false if it gave up.
+// SM clock cycles. Returns false if it gave up. Each try_wait may suspend the thread (up to the
+// hint, 100 us) until the phase completes, so a waiting warp takes no issue slots meanwhile.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit) {
   const long long t0 = clock64();
   while (true) {
     uint32_t done;
     asm volatile(
-        "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n selp.u32 %0, 1, 0, q;\n}\n"
-        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+        "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2, %3;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(done) : "r"(bar), "r"(parity), "r"(100000u) : "memory");
     if (done) return true;
     if (clock64() - t0 > limit) return false;
   }
