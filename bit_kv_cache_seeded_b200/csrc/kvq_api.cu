@@ -169,10 +169,26 @@ int part_stride(const kvq_cache* c) {
   return 2 + kHeadDim * (c->v.qjl ? 2 : 1);
 }
 
-int prep_stride(const kvq_cache* c) {
-  if (c->is_fp4) return 0;
-  return mma_prep_bytes(c->k.bits, c->k.qjl, c->cfg.n_q_heads / c->cfg.n_kv_heads);
+// Tensor-core decode: CTAs per (sequence, kv-head, split), each taking at most 4 query heads
+// (1 on every other path).
+int decode_hsplit(const kvq_cache* c) {
+  if (c->is_fp4) return 1;
+  const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
+  if (!mma_modes_supported(group, c->k.bits, c->k.qjl, c->v.bits, c->v.qjl)) return 1;
+  return group > 4 ? group / 4 : 1;
 }
+
+// Query prep area of one piece of a query group (tensor-core path), and of a whole (sequence,
+// kv-head): decode_hsplit pieces.
+int prep_piece_stride(const kvq_cache* c) {
+  if (c->is_fp4) return 0;
+  const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
+  return mma_prep_bytes(c->k.bits, c->k.qjl, group / decode_hsplit(c));
+}
+int prep_stride(const kvq_cache* c) { return prep_piece_stride(c) * decode_hsplit(c); }
+
+// Rows of the decode grid the split plan spreads over the SMs: (sequence, kv-head, piece).
+int decode_rows(const kvq_cache* c) { return c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads * decode_hsplit(c)); }
 
 size_t partials_bytes(const kvq_cache* c, int splits) {
   return align_up(sizeof(float) * (size_t)c->batch * c->cfg.n_q_heads * splits * part_stride(c), 256);
@@ -399,7 +415,7 @@ kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dt
 
 kvq_status kvq_workspace_bytes(const kvq_cache* c, size_t* bytes) {
   if (!c || !bytes) return KVQ_ERR_INVALID_ARG;
-  const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
+  const int pairs = decode_rows(c);
   *bytes = workspace_for(c, max_splits(pairs, c->sms, c->tiles_per_seq, decode_max_units(c), decode_waves_bound(c)));
   return KVQ_OK;
 }
@@ -417,7 +433,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
   int max_len = 0;
   for (int v : c->lens) max_len = std::max(max_len, v);
-  const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
+  const int pairs = decode_rows(c);
   int splits, chunk;
   plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len,
               &splits, &chunk);
@@ -472,7 +488,8 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.St = c->d_St;
   p.logit_scale = default_scale(c->cfg) * log2e;
   p.qprep = static_cast<unsigned char*>(workspace) + partials_bytes(c, splits);
-  p.qprep_stride = prep_stride(c);
+  p.hsplit = decode_hsplit(c);
+  p.qprep_stride = prep_piece_stride(c);
   p.err = c->d_status;
   p.wait_limit = wait_limit;
   p.debug_unset_wait = debug_unset_wait;
@@ -507,7 +524,7 @@ kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const voi
     if ((long)v + 1 > (long)c->capacity) return KVQ_ERR_CAPACITY;
     max_len = std::max(max_len, v);
   }
-  const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
+  const int pairs = decode_rows(c);
   int splits, chunk;
   plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len + 1,
               &splits, &chunk);
@@ -668,7 +685,7 @@ extern "C" kvq_status kvq_decode_attention_static(const kvq_cache* c, const void
   if (!c || !q || !out) return KVQ_ERR_INVALID_ARG;
   int max_len = 0;
   for (int v : c->lens) max_len = std::max(max_len, v);
-  const int pairs = c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads);
+  const int pairs = decode_rows(c);
   int splits, chunk;
   plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len,
               &splits, &chunk);

@@ -176,7 +176,7 @@ size_t mma_smem_bytes(int group, const SideLayout& k, const SideLayout& v, int c
 // k of coordinate block m is coordinate 32m + k.
 // ------------------------------------------------------------------------------------------
 template <int G, int KB, bool KQ>
-__device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b) {
+__device__ __forceinline__ void prep_block(const DecodeParams& p, int vk, int b) {
   constexpr int KP = Walsh<KB>::P + (KQ ? 1 : 0);
   constexpr int KWP = Walsh<KB>::P;
   __shared__ __align__(16) float qf[G][kHeadDim];
@@ -186,7 +186,10 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b)
   __shared__ __align__(8) uint64_t st_bar;       // completes when S^T has landed
   extern __shared__ __align__(16) float st_s[];  // [128][m] transposed sketch matrix
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  unsigned char* out = p.qprep + ((size_t)b * p.Hkv + hk) * p.qprep_stride;
+  // piece `half` (of p.hsplit) of kv-head hk's query group: query heads h_first .. h_first + G - 1
+  const int hk = vk / p.hsplit, half = vk % p.hsplit;
+  const int h_first = hk * p.group + half * G;
+  unsigned char* out = p.qprep + (((size_t)b * p.Hkv + hk) * p.hsplit + half) * p.qprep_stride;
   static_assert(G <= kWarpsM, "one query head per warp");
   const int h0 = warp;  // this warp's query head (h0 < G)
   if (KQ && tid == 0) {  // one bulk copy, landing while the queries are rotated
@@ -203,7 +206,7 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int hk, int b)
   // preceding kernel, so wait for it (the sketch matrix requested above is the cache's own).
   grid_dep_wait();
   if (h0 < G) {
-    const size_t qb = ((size_t)b * p.Hq + hk * G + h0) * kHeadDim;
+    const size_t qb = ((size_t)b * p.Hq + h_first + h0) * kHeadDim;
 #pragma unroll
     for (int k = 0; k < 4; ++k) u[k] = load_q(p.q, qb + 32 * k + lane, p.bf16) * p.signs[32 * k + lane];
   }
@@ -333,7 +336,7 @@ decode_front(const __grid_constant__ QuantizeParams qp, const __grid_constant__ 
     qlm::quantize_lm_block(qp, blk / nq, blk % nq, nq);
   } else {
     const int r = blk - 2 * nq;
-    prep_block<G, KB, KQ>(p, r % p.Hkv, r / p.Hkv);
+    prep_block<G, KB, KQ>(p, r % (p.Hkv * p.hsplit), r / (p.Hkv * p.hsplit));
   }
 }
 
@@ -367,7 +370,10 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * lgst);  // [2][NKIND][VNCOL][kPdStride]
   float* red = reinterpret_cast<float*>(pdig + 2 * PDB);                      // reductions
 
-  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, b = blockIdx.z;
+  // blockIdx.y: piece `half` of kv-head hk's query group (p.hsplit pieces of G heads)
+  const int hk = blockIdx.y / p.hsplit, half = blockIdx.y % p.hsplit;
+  const int h_first = hk * p.group + half * G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   // In a fused append + decode step the cache (and len) are written by the append kernel that
@@ -435,7 +441,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   // complete before prep started (unless cache_after_wait, handled above); the prep output is read
   // only after this wait.
   if (!p.cache_after_wait) grid_dep_wait();
-  const unsigned char* prep = p.qprep + pair * p.qprep_stride;
+  const unsigned char* prep = p.qprep + (pair * p.hsplit + half) * p.qprep_stride;
   uint32_t qb[KP][4][KNT][2];
 #pragma unroll
   for (int P = 0; P < KP; ++P)
@@ -812,7 +818,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         else { o0 = fmaf(2.f * va[min(P, 3)], r0 * rowinv, o0); o1 = fmaf(2.f * va[min(P, 3)], r1 * rowinv, o1); }
       }
       if (h < G) {
-        float* dst = p.part + (((size_t)b * p.Hq + hk * G + h) * p.splits + split) * p.part_stride;
+        float* dst = p.part + (((size_t)b * p.Hq + h_first + h) * p.splits + split) * p.part_stride;
         const int j0 = 8 * g + pos, j1 = 8 * (g + 8) + pos;
         if ((t & 1) == 0) {
           const float Wt = hsum[G + h] * inv_w;
@@ -829,7 +835,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     if (tid == h) {
-      float* dst = p.part + (((size_t)b * p.Hq + hk * G + h) * p.splits + split) * p.part_stride;
+      float* dst = p.part + (((size_t)b * p.Hq + h_first + h) * p.splits + split) * p.part_stride;
       float mx = -INFINITY;
 #pragma unroll
       for (int w = 0; w < kWarpsM; ++w) mx = fmaxf(mx, hmax[w * G + h]);
@@ -856,7 +862,7 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid
     // a programmatic dependent of whatever precedes it: its launch and setup overlap that
     // kernel's tail, and it waits for it before reading inputs
     cudaLaunchConfig_t fc = {};
-    fc.gridDim = dim3(2 * nq + p.B * p.Hkv);
+    fc.gridDim = dim3(2 * nq + p.B * p.Hkv * p.hsplit);
     fc.blockDim = dim3(kThreadsM);
     fc.dynamicSmemBytes = fsmem;
     fc.stream = s;
@@ -868,7 +874,7 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid
     e = cudaLaunchKernelEx(&fc, decode_front<G, KB, KQ>, *qp, p, nq);
     if (e != cudaSuccess) return e;
   } else {
-    decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv, p.B), kThreadsM, prep_smem, s>>>(p);
+    decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv * p.hsplit, p.B), kThreadsM, prep_smem, s>>>(p);
   }
   e = launched();
   if (e != cudaSuccess) return e;
@@ -878,7 +884,7 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.splits, p.Hkv, p.B);
+  cfg.gridDim = dim3(p.splits, p.Hkv * p.hsplit, p.B);
   cfg.blockDim = dim3(kThreadsM);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -918,7 +924,7 @@ int mma_prep_bytes(int k_bits, int k_qjl, int group) {
 }
 
 bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl) {
-  if (group != 1 && group != 2 && group != 4) return false;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return false;
   // the (K bits, K sketch, V bits, V sketch) instances of dispatch_mma_modes
   static const int kModes[][4] = {{2, 1, 2, 1}, {3, 1, 3, 0}, {1, 0, 1, 0}, {2, 1, 2, 0},
                                   {3, 1, 3, 1}, {2, 0, 2, 0}, {3, 0, 3, 0}};
@@ -928,12 +934,13 @@ bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl
 }
 
 int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk) {
-  const size_t per = mma_smem_bytes(group, k, v, chunk) + kSmemReserved;
+  const size_t per = mma_smem_bytes(std::min(group, 4), k, v, chunk) + kSmemReserved;
   return std::max(1, std::min(kMinBlocksM, (int)(kSmemPerSm / per)));
 }
 
 bool mma_decode_supported(const DecodeParams& p) {
-  return (p.group == 1 || p.group == 2 || p.group == 4) && p.chunk % kCtaTok == 0 &&
+  if (!mma_modes_supported(p.group, p.k.bits, p.k.qjl, p.v.bits, p.v.qjl) || p.k.order != kOrderOctet) return false;
+  return (p.group == 1 || p.group == 2 || p.group == 4 || (p.group == 8 && p.hsplit == 2)) && p.chunk % kCtaTok == 0 &&
          p.chunk <= kChunkMax && p.qprep != nullptr;
 }
 
@@ -942,6 +949,7 @@ cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEven
     case 1: return dispatch_mma_modes<1>(p, s, ev_mid, qp);
     case 2: return dispatch_mma_modes<2>(p, s, ev_mid, qp);
     case 4: return dispatch_mma_modes<4>(p, s, ev_mid, qp);
+    case 8: return dispatch_mma_modes<4>(p, s, ev_mid, qp);  // two pieces of 4 heads
     default: return cudaErrorNotSupported;
   }
 }

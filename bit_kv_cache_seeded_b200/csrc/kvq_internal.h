@@ -84,6 +84,7 @@ struct DecodeParams {
   float* part;            // [B, Hq, splits, part_stride]
   int part_stride;        // 2 + d (+ m with a value sketch)
   int B, Hq, Hkv, group;
+  int hsplit;             // tensor-core path: CTAs per (sequence, kv-head, split), G = group / hsplit heads each
   int splits, chunk;      // tokens per split (multiple of kTile)
   const int* lens;
   const char* kreg;

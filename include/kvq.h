@@ -162,8 +162,8 @@ kvq_status kvq_cache_status(const kvq_cache* c, int32_t* status, void* stream);
  * kvq_decode_attention, except that every CTA of the tensor-core decode kernel first waits on
  * a barrier that nothing ever completes, giving up after wait_limit_cycles SM clock cycles
  * (1 ... 2^31). It then carries on as usual, so the output equals kvq_decode_attention's and
- * KVQ_STATUS_WAIT_TIMEOUT is set. Caches that decode without that kernel (query groups of 8,
- * FP4) return KVQ_ERR_UNSUPPORTED and launch nothing. */
+ * KVQ_STATUS_WAIT_TIMEOUT is set. Caches that decode without that kernel (FP4, and LM code
+ * combinations it has no instance for) return KVQ_ERR_UNSUPPORTED and launch nothing. */
 kvq_status kvq_debug_decode_unset_wait(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
                                        void* workspace, size_t ws_bytes, int64_t wait_limit_cycles,
                                        void* stream);

@@ -71,10 +71,10 @@ def test_debug_quantize_rotated_bit_exact(bits, qjl):
 
 # ---------------------------------------------------------------- decode parity, small contexts
 
-def run_small(name, batch, lens, seed_appends=1):
+def run_small(name, batch, lens, seed_appends=1, w=None):
     """Quantize lens[b] tokens into sequence b (in `seed_appends` calls), decode, compare every
     (sequence, kv-head) with the oracle."""
-    w = WORKLOADS[name]
+    w = w if w is not None else WORKLOADS[name]
     T = max(lens)
     data = generate(w, DEV, seqs=range(batch), ctx=T)
     cache, signs, S = new_cache(w, batch, T + 40)
@@ -115,6 +115,13 @@ def test_tiny_full():
 
 def test_tiny_token_by_token_and_ragged():
     run_small("tiny", 1, [77], seed_appends=77)
+
+
+def test_cuda_core_code_combination():
+    """1-bit keys with a sketch and 1-bit values without: a combination the tensor-core kernel has
+    no instance for, decoded by the CUDA-core kernel (token-ordered keys)."""
+    w = WORKLOADS["tiny"].with_(k_bits=1, v_bits=1, k_mode="lm_qjl", v_mode="lm", n_q_heads=4, n_kv_heads=1)
+    run_small("tiny", 2, [300, 65], seed_appends=2, w=w)
 
 
 @pytest.mark.parametrize("lens", [[1000, 333, 1, 0], [32, 31, 64, 65]])
@@ -227,8 +234,8 @@ def test_fp4_full_context_sampled_heads():
 
 def test_launch_counts_per_call():
     """quantize: one kernel; decode: query prep + split decode + reduce on the tensor-core path
-    (G <= 4), split decode + reduce otherwise (G = 8 and FP4)."""
-    for name, per_decode in (("llama8b", 3), ("llama70b", 2), ("mla_fp4", 2)):
+    (query groups of 8 as two pieces of 4 heads), split decode + reduce for FP4."""
+    for name, per_decode in (("llama8b", 3), ("llama70b", 3), ("mla_fp4", 2)):
         w = WORKLOADS[name]
         data = generate(w, DEV, seqs=range(2), ctx=100)
         if w.k_mode == "fp4":
@@ -308,18 +315,19 @@ def test_bounded_wait_sets_status_and_returns():
     assert kvq.kvq_cache_status(cache.handle) == kvq.KVQ_STATUS_WAIT_TIMEOUT
     assert torch.equal(out, ref)
     cache.close()
-    # no tensor-core kernel for groups of 8: the test entry refuses and launches nothing
-    w70 = WORKLOADS["llama70b"]
-    d70 = generate(w70, DEV, seqs=range(1), ctx=64)
-    c70, _, _ = new_cache(w70, 1, 64)
-    c70.quantize(d70["k"], d70["v"])
+    # a code combination only the CUDA-core kernel decodes (1-bit keys with a sketch, 1-bit values
+    # without): the test entry refuses and launches nothing
+    w1 = WORKLOADS["tiny"].with_(k_bits=1, v_bits=1, k_mode="lm_qjl", v_mode="lm")
+    d1 = generate(w1, DEV, seqs=range(1), ctx=64)
+    c1, _, _ = new_cache(w1, 1, 64)
+    c1.quantize(d1["k"], d1["v"])
     n0 = kvq.kvq_kernel_launches()
     with pytest.raises(kvq.KvqError) as e:
-        kvq.kvq_debug_decode_unset_wait(c70.handle, d70["q"], torch.empty(1, 64, 128, device=DEV),
-                                        c70.workspace, 100000)
+        kvq.kvq_debug_decode_unset_wait(c1.handle, d1["q"], torch.empty(1, 1, 128, device=DEV),
+                                        c1.workspace, 100000)
     assert e.value.status == 2 and kvq.kvq_kernel_launches() == n0
-    assert kvq.kvq_cache_status(c70.handle) == 0
-    c70.close()
+    assert kvq.kvq_cache_status(c1.handle) == 0
+    c1.close()
 
 
 # ---------------------------------------------------------------- errors
