@@ -378,21 +378,29 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   const int g = lane >> 2, t = lane & 3;
   // In a fused append + decode step the cache (and len) are written by the append kernel that
   // runs before the prep: everything that reads them waits for the prep (which waits for it).
-  if (p.cache_after_wait) grid_dep_wait();
-  const int len = __ldcg(p.lens + b);  // through L2: a predecessor may have written it
   const int t_begin = split * p.chunk;
-  const int t_end = min(len, t_begin + p.chunk);
   const size_t pair = (size_t)b * p.Hkv + hk;
   const unsigned char* kbase = reinterpret_cast<const unsigned char*>(p.kreg) + pair * p.tiles_per_seq * (size_t)ktb;
   const unsigned char* vbase = reinterpret_cast<const unsigned char*>(p.vreg) + pair * p.tiles_per_seq * (size_t)vtb;
-  const int n_iter = t_end > t_begin ? (t_end - t_begin + kCtaTok - 1) / kCtaTok : 0;
+  // In a fused append + decode step the predecessor appends the token at the old length and sets
+  // the new one, so a length read before waiting for it is either value. When the first
+  // kStagesM - 1 fills end below the old length under both readings, they hold no token the
+  // predecessor writes: they are issued before the wait (`early`), the rest after it.
+  int len = __ldcg(p.lens + b);  // through L2: a predecessor may write it
+  const bool early = p.cache_after_wait && t_begin + kCtaTok * (kStagesM - 1) < len;
+  if (p.cache_after_wait && !early) {
+    grid_dep_wait();
+    len = __ldcg(p.lens + b);
+  }
+  int t_end = min(len, t_begin + p.chunk);
+  int n_iter = t_end > t_begin ? (t_end - t_begin + kCtaTok - 1) / kCtaTok : 0;
 
   // Staging: fill f < n_iter brings the K tile pair of pass-1 iteration f (and the value norms
   // and sketch norms of the same tokens, for the weight scale); fill n_iter + i brings the V tile
   // pair of pass-2 iteration i. Fill f goes to stage f % kStagesM and completes phase f / kStagesM
   // of that stage's barrier. Thread 0 issues the fills as bulk copies; every tile pair is whole
   // (capacity is a whole number of pairs), so a fill never reads outside its pair's region.
-  const int n_fill = 2 * n_iter;
+  int n_fill = 2 * n_iter;
   if (tid == 0) {
 #pragma unroll
     for (int s = 0; s <= kStagesM; ++s) mbar_init(smem_addr(&mbar[s]), 1);
@@ -429,7 +437,14 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   };
   if (tid == 0)
 #pragma unroll
-    for (int f = 0; f < kStagesM - 1; ++f) issue(f);
+    for (int f = 0; f < kStagesM - 1; ++f) issue(f);  // early: key fills whatever the final length
+  if (early) {  // the final length, now that the predecessor has finished
+    grid_dep_wait();
+    len = __ldcg(p.lens + b);
+    t_end = min(len, t_begin + p.chunk);
+    n_iter = t_end > t_begin ? (t_end - t_begin + kCtaTok - 1) / kCtaTok : 0;
+    n_fill = 2 * n_iter;
+  }
   if (p.debug_unset_wait && !mbar_wait(smem_addr(&mbar[kStagesM]), 0u, p.wait_limit)) {
     s_fail = 1;
     atomicOr(p.err, 1);
