@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--workload", default="llama8b", choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ctx", type=int, default=0,
+                    help="context length override (smaller cases for profiling); default: the workload's")
     return ap.parse_args()
 
 
@@ -83,7 +85,7 @@ def kernel_sources_sha():
 
 def traffic_record(w):
     rec = TRAFFIC.get(w.name)
-    if rec is None or rec["sources_sha256"] != kernel_sources_sha():
+    if rec is None or rec["sources_sha256"] != kernel_sources_sha() or w.ctx != WORKLOADS[w.name].ctx:
         return None
     return rec["dram_bytes"]
 
@@ -275,6 +277,8 @@ def blas_threads():
 
 def run_reference(args, world, rank):
     w = WORKLOADS[args.workload]
+    if args.ctx > 0:
+        w = w.with_(ctx=args.ctx)
     metric, unit = METRIC, UNIT
     if rank != 0:
         return
@@ -308,6 +312,8 @@ def run_ours(args, world, rank, local):
     import bit_kv_cache_seeded_b200 as kvq
     kvq.load()
     w = WORKLOADS[args.workload]
+    if args.ctx > 0:
+        w = w.with_(ctx=args.ctx)
     dev = f"cuda:{local}"
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
