@@ -410,12 +410,12 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   __syncthreads();
   auto issue = [&](int f) {  // thread 0 only
     if (f >= n_fill) return;
-    const int slot = f % kStagesM;
+    const int slot = (unsigned)f % kStagesM;
     const uint32_t bar = smem_addr(&mbar[slot]);
     unsigned char* dst = stages + slot * stage_bytes;
     fence_proxy_async();  // the stage's previous contents were read by the generic proxy
     if (f < n_iter) {
-      const int tile0 = (t_begin + f * kCtaTok) / kTile;
+      const int tile0 = (unsigned)(t_begin + f * kCtaTok) / kTile;
       constexpr uint32_t nb = VQ ? 128u : 64u;  // value norms (+ gammas, contiguous) per tile
       mbar_arrive_expect_tx(bar, 2u * ktb + 2u * nb);
       bulk_g2s(smem_addr(dst), kbase + (size_t)tile0 * ktb, 2u * ktb, bar);
@@ -423,13 +423,13 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       for (int tile = 0; tile < 2; ++tile)
         bulk_g2s(smem_addr(dst + 2 * ktb + tile * 128), vbase + (size_t)(tile0 + tile) * vtb + VL::NORM, nb, bar);
     } else {
-      const int tile0 = (t_begin + (f - n_iter) * kCtaTok) / kTile;
+      const int tile0 = (unsigned)(t_begin + (f - n_iter) * kCtaTok) / kTile;
       mbar_arrive_expect_tx(bar, 2u * vtb);
       bulk_g2s(smem_addr(dst), vbase + (size_t)tile0 * vtb, 2u * vtb, bar);
     }
   };
   auto wait_fill = [&](int f) {  // every thread
-    const uint32_t bar = smem_addr(&mbar[f % kStagesM]), par = (uint32_t)(f / kStagesM) & 1u;
+    const uint32_t bar = smem_addr(&mbar[(unsigned)f % kStagesM]), par = ((unsigned)f / kStagesM) & 1u;
     if (!mbar_try(bar, par) && !mbar_wait(bar, par, p.wait_limit)) {
       s_fail = 1;
       atomicOr(p.err, 1);
@@ -498,7 +498,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   for (int it = 0; it < n_iter; ++it) {
     if (tid == 0) issue(it + kStagesM - 1);
     wait_fill(it);
-    const unsigned char* kt = stages + (it % kStagesM) * stage_bytes;
+    const unsigned char* kt = stages + ((unsigned)it % kStagesM) * stage_bytes;
     const int tok0 = it * kCtaTok;  // chunk-relative first token of this iteration
     const int count = min(kCtaTok, t_end - (t_begin + tok0));
     {
@@ -649,20 +649,20 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     if (!has_task) return;
     const int tok0 = it * kCtaTok, T = task_T;
     const int count = min(kCtaTok, t_end - (t_begin + tok0));
-    const unsigned char* vtile = stages + ((n_iter + it) % kStagesM) * stage_bytes + (T / kTile) * vtb;
+    const unsigned char* vtile = stages + ((unsigned)(n_iter + it) % kStagesM) * stage_bytes + ((unsigned)T / kTile) * vtb;
     float lv[TPT], wc[TPT], wz[TPT];
     if (TPT == 2) {
       const float2 l2 = *reinterpret_cast<const float2*>(lgs + task_h * lgst + tok0 + T);
-      const float2 n2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::NORM + (T % kTile) * 2));
+      const float2 n2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::NORM + ((unsigned)T % kTile) * 2));
       lv[0] = l2.x; lv[TPT - 1] = l2.y; wc[0] = n2.x; wc[TPT - 1] = n2.y;
       if (VQ) {
-        const float2 g2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::GAMMA + (T % kTile) * 2));
+        const float2 g2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::GAMMA + ((unsigned)T % kTile) * 2));
         wz[0] = g2.x; wz[TPT - 1] = g2.y;
       }
     } else {
       lv[0] = lgs[task_h * lgst + tok0 + T];
-      wc[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::NORM + (T % kTile) * 2));
-      if (VQ) wz[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::GAMMA + (T % kTile) * 2));
+      wc[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::NORM + ((unsigned)T % kTile) * 2));
+      if (VQ) wz[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::GAMMA + ((unsigned)T % kTile) * 2));
     }
     uint32_t bc[TPT], bz[TPT];
     float psum = 0.f;
@@ -722,15 +722,12 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       wait_fill(n_iter + it + 1);
       tasks(it + 1);
     }
-    const unsigned char* vt = stages + ((n_iter + it) % kStagesM) * stage_bytes;
-    const int tok0 = it * kCtaTok;
-    const int count = min(kCtaTok, t_end - (t_begin + tok0));
+    const unsigned char* vt = stages + ((unsigned)(n_iter + it) % kStagesM) * stage_bytes;
     const unsigned char* pd = pdig + (it & 1) * PDB;
 
     // value contractions: positions 2w, 2w+1 of every value Walsh plane
 #pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      if (s * kTile >= count) break;
+    for (int s = 0; s < 2; ++s) {  // a step past the end adds nothing: its weights are zero
       const unsigned char* vtile = vt + s * vtb;
       // K order within a 32-token step: K-index 4t + i <-> token 8t + i, 16 + 4t + i <-> 8t + 4 + i,
       // so a thread's two 4-token groups are one 64-bit load (bits and digits alike)
@@ -790,7 +787,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   // for the last fill of each stage, so no copy is still landing when the stages are reused.
   if (tid == 0 && s_fail)
     for (int f = max(0, n_fill - kStagesM); f < n_fill; ++f)
-      mbar_wait(smem_addr(&mbar[f % kStagesM]), (uint32_t)(f / kStagesM) & 1u, p.wait_limit);
+      mbar_wait(smem_addr(&mbar[(unsigned)f % kStagesM]), ((unsigned)f / kStagesM) & 1u, p.wait_limit);
   __syncthreads();
   float* tsum = reinterpret_cast<float*>(stages);  // [kThreadsM][3] (staging reused)
   float* hsum = tsum + 3 * kThreadsM;               // [3][G]: sum p, sum weights, sum sketch weights
