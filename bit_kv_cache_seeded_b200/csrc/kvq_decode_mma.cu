@@ -510,13 +510,13 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       const int s0 = (tl % kTile) + g, s1 = s0 + 8;
       const int o0 = (tl % kTile) / 8;
       const uint32_t mg = 0x01010101u << g;
-      int acc[4][KNT][4], accz[2][KNT][4];  // independent chains: coordinate block m (z: m & 1)
+      int acc[2][KNT][4], accz[2][KNT][4];  // independent chains: coordinate block parity m & 1
 #pragma unroll
       for (int m = 0; m < 4; ++m)
 #pragma unroll
         for (int nt = 0; nt < KNT; ++nt)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) { acc[m][nt][c] = 0; if (m < 2) accz[m][nt][c] = 0; }
+          for (int c = 0; c < 4; ++c) { if (m < 2) { acc[m][nt][c] = 0; accz[m][nt][c] = 0; } }
       // this thread's words of octet o: 8t + 2m + h, m = 0..3, h = 0..1 (32 contiguous bytes)
       const unsigned char* kp = ktile + KL::PLANES + o0 * 128 + t * 32;
 #pragma unroll
@@ -555,7 +555,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
             for (int nt = 0; nt < KNT; ++nt) {
               if (sk) mma_s8(accz[m & 1][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
-              else mma_s8(acc[m][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+              else mma_s8(acc[m & 1][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
             }
           }
         }
@@ -574,7 +574,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         int c[4], cz[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          c[e] = (acc[0][nt][e] + acc[1][nt][e]) + (acc[2][nt][e] + acc[3][nt][e]);
+          c[e] = acc[0][nt][e] + acc[1][nt][e];
           cz[e] = accz[0][nt][e] + accz[1][nt][e];
         }
         // hi * 256 + lo: exact in int32 up to 2 Walsh planes (|hi| < 2^22), else in fp32
