@@ -71,7 +71,7 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
 #pragma unroll
       for (int c = 0; c < 4; ++c) bulk_g2s(smem_addr(st_s + c * kQuarter), p.St + c * kQuarter, kQuarter * 4u, bar);
     }
-    __syncthreads();  // the barrier is initialised before anyone waits on it
+    // no block barrier here: the one before the first wait below publishes the initialisation
   }
   const float* stw = st_s + 32 * warp + lane;  // stw[i * d] = S^T[i][32 warp + lane] = S[32 warp + lane][i]
   // Everything the first vector needs from global memory is requested before the staged slice
@@ -152,6 +152,7 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
 #pragma unroll
       for (int k = 0; k < 4; ++k) rho_s[warp][32 * k + lane] = rho[k];
       __syncwarp();
+      if (vec == first) __syncthreads();  // st_bar was initialised (by thread 0) before anyone waits
       if (vec == first && !mbar_try(smem_addr(&st_bar), 0u) &&
           !mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit)) {  // S^T (requested at the start)
         st_failed = true;
