@@ -508,7 +508,10 @@ def run_ours(args, world, rank, local):
         "metric": METRIC,
         "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "scaling": "weak", "vs_baseline": None,
+        # the contractions' operand / accumulation types: exact int8 tensor-core products with int32
+        # sums and fp32 softmax (LM), f16/bf16 tcgen05 products with fp32 accumulators (FP4 latent)
+        "dtype": "f16/f32" if w.k_mode == "fp4" else "s8/s32/f32",
         "data": "synthetic",
         "config": workload_config(w, world),
         "l2_detail": f"{replicas} cache replicas x {bytes_prefix / 1e6:.1f} MB rotated per step",
