@@ -255,7 +255,7 @@ def test_launch_counts_per_call():
 
 # ---------------------------------------------------------------- fused decode step
 
-@pytest.mark.parametrize("name", ["llama8b", "onebit", "mla_fp4"])
+@pytest.mark.parametrize("name", ["llama8b", "llama70b", "onebit", "mla_fp4"])
 def test_decode_step_equals_append_then_decode(name):
     """kvq_decode_step (append one token, then attend, with the query prep overlapping the append)
     leaves the same cache and returns the same output as kvq_quantize followed by
@@ -293,6 +293,30 @@ def test_decode_step_equals_append_then_decode(name):
                 for f1, f2 in zip(side_fields(a1, info, side, pair, 151), side_fields(a2, info, side, pair, 151)):
                     if f1 is not None:
                         np.testing.assert_array_equal(f1[:151], f2[:151])
+    c1.close()
+    c2.close()
+
+
+def test_decode_step_ragged_long():
+    """Ragged lengths long enough that most splits issue their first key fills before waiting for
+    the append: the fused step still equals append-then-decode, and matches the oracle."""
+    w = WORKLOADS["llama8b"]
+    B, lens = 3, [1000, 333, 700]
+    T = max(lens)
+    data = generate(w, DEV, seqs=range(B), ctx=T)
+    new = generate(w, DEV, seqs=range(B), step=0)
+    c1, signs, S = new_cache(w, B, T + 64)
+    c2, _, _ = new_cache(w, B, T + 64)
+    for c in (c1, c2):
+        for b in range(B):
+            c.quantize(data["k"][b:b + 1, :, :lens[b]].contiguous(), data["v"][b:b + 1, :, :lens[b]].contiguous(),
+                       seq_ids=[b])
+    c1.quantize(new["k"], new["v"])
+    ref = c1.decode(data["q"])
+    out = c2.step(new["k"], new["v"], data["q"])
+    torch.cuda.synchronize()
+    assert list(c2.lengths()) == [n + 1 for n in lens]
+    assert torch.equal(out, ref)
     c1.close()
     c2.close()
 
