@@ -68,7 +68,7 @@ def parse():
 TRAFFIC = {
     "llama8b": {"kernel": "decode_lm_mma<4, 2, 1, 2, 1>", "dram_bytes": 113382912,  # 109.512704 + 3.870208 MB
                 "profile": "profiles/decode_lm_mma_llama8b.md",
-                "sources_sha256": "bf0f6b4b39b302209cd82dda1d489ecd99a13b3c7a177fd99834afcdda98e8e8"},
+                "sources_sha256": "4898861750d5ee9a9bfa1b72b124014c1836d9446cde511be9a6c58cd6270560"},
 }
 TRAFFIC_SOURCES = ("bit_kv_cache_seeded_b200/csrc/kvq_decode_mma.cu", "bit_kv_cache_seeded_b200/csrc/kvq_async.cuh",
                    "bit_kv_cache_seeded_b200/csrc/kvq_internal.h")

@@ -1,4 +1,5 @@
-// Tensor-core split-K decode attention for LM / LM_QJL / SIGN1 caches (query group g <= 4).
+// Tensor-core split-K decode attention for LM / LM_QJL / SIGN1 caches (up to 4 query heads per
+// CTA; a query group of 8 runs as two pieces of 4 heads).
 //
 // Same computation as the CUDA-core kernel in kvq_decode.cu ("TurboQuant vs OSCAR vs
 // EpiCache", section "Quantization frontiers: TurboQuant and OSCAR": logits from the
@@ -19,7 +20,7 @@
 //     tile, where 4 tokens of one byte-lane are one 32-bit word: w & (0x01010101 << p) gives the
 //     int8 value 2^p (p < 7) or -128 (p = 7) per byte, i.e. a fixed power of two per row. B = the
 //     softmax weights p_t n_t / sqrt(d) (times sqrt(pi/2)/m gamma_t for the value sketch) as a
-//     21-bit integer (3 x 7-bit unsigned digits), each kind scaled by a power of two to its own
+//     23-bit integer (3 unsigned byte digits), each kind scaled by a power of two to its own
 //     chunk maximum.
 //   * Two passes over a CTA's chunk (at most kChunkMax tokens): pass 1 computes every logit into
 //     shared memory and the chunk's maxima; pass 2 streams the value tiles with the weights
