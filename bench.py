@@ -68,7 +68,7 @@ def parse():
 TRAFFIC = {
     "llama8b": {"kernel": "decode_lm_mma<4, 2, 1, 2, 1>", "dram_bytes": 113382912,  # 109.512704 + 3.870208 MB
                 "profile": "profiles/decode_lm_mma_llama8b.md",
-                "sources_sha256": "4898861750d5ee9a9bfa1b72b124014c1836d9446cde511be9a6c58cd6270560"},
+                "sources_sha256": "a506daec4d4b17781042b53742a2e8ff7d574e27935e60a922a432e57279fa2f"},
 }
 TRAFFIC_SOURCES = ("bit_kv_cache_seeded_b200/csrc/kvq_decode_mma.cu", "bit_kv_cache_seeded_b200/csrc/kvq_async.cuh",
                    "bit_kv_cache_seeded_b200/csrc/kvq_internal.h")

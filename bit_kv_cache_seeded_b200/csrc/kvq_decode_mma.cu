@@ -627,7 +627,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   float wm = 0.f, wmz = 0.f;
 #pragma unroll
   for (int w = 0; w < kWarpsM; ++w) { wm = fmaxf(wm, wred[w]); wmz = fmaxf(wmz, wred[kWarpsM + w]); }
-  // integer weights below 2^21 (3 x 7-bit digits), each kind scaled to its own range by a power
+  // integer weights below 2^23 (3 byte digits), each kind scaled to its own range by a power
   // of two (exact digits; the sketch weights are ~sqrt(pi/2) gamma / m of the centroid ones)
   const float wsc = wm > 0.f ? exp2f(floorf(log2f(kWRange / wm)) - 1.f) : 1.f;
   const float wscz = wmz > 0.f ? exp2f(floorf(log2f(kWRange / wmz)) - 1.f) : 1.f;
