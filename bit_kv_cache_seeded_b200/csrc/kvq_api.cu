@@ -7,8 +7,11 @@
 #include <vector>
 
 #include "kvq_internal.h"
+#include "kvq_plan.h"
 
 using namespace kvq;
+
+static_assert(kTile * kTilePair == kPlanUnitTokens && kTilePair == kPlanUnitTiles, "split unit = two tiles");
 
 namespace {
 
@@ -130,38 +133,6 @@ int device_sms() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   return sms > 0 ? sms : 148;
-}
-
-// Split plan. Each (pair, split) CTA covers a whole number of 64-token units, at most
-// `max_units` of them. The split count minimises waves x (units per CTA + a fixed per-CTA
-// overhead of 4 units), with slots_per_sm(units per CTA) resident CTAs per SM in a wave;
-// max_splits() bounds it for every length up to the capacity (it sizes the workspace).
-int max_splits(int pairs, int sms, int tiles, int max_units, int waves_bound) {
-  const int units = std::max(1, tiles / kTilePair);
-  const int need = (units + max_units - 1) / max_units;
-  const int bound = std::max(1, (waves_bound * sms + pairs - 1) / pairs);
-  return std::max(need, std::min(bound, units));
-}
-
-template <class SlotsFn>
-void plan_splits(int pairs, int sms, const SlotsFn& slots_per_sm, int max_units, int waves_bound, int max_len,
-                 int* splits, int* chunk) {
-  const int units = std::max(1, (max_len + kTile * kTilePair - 1) / (kTile * kTilePair));
-  const int smin = (units + max_units - 1) / max_units;
-  const int smax = std::min(max_splits(pairs, sms, units * kTilePair, max_units, waves_bound), units);
-  long best_cost = -1;
-  int best_cu = units;
-  for (int s = std::max(1, smin); s <= std::max(smin, smax); ++s) {
-    const int cu = (units + s - 1) / s;
-    if (cu > max_units) continue;
-    const int ss = (units + cu - 1) / cu;
-    const long slots = (long)sms * slots_per_sm(cu);
-    const long waves = ((long)pairs * ss + slots - 1) / slots;
-    const long cost = waves * (cu + 4);
-    if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_cu = cu; }
-  }
-  *splits = (units + best_cu - 1) / best_cu;
-  *chunk = best_cu * kTile * kTilePair;
 }
 
 int part_stride(const kvq_cache* c) {
