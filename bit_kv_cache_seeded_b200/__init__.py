@@ -33,7 +33,8 @@ EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "k
            "kvq_quantize", "kvq_workspace_bytes", "kvq_decode_attention", "kvq_cache_lengths",
            "kvq_cache_layout", "kvq_lloyd_max_table", "kvq_cache_destroy",
            "kvq_debug_quantize_rotated", "kvq_decode_attention_static", "kvq_kernel_launches",
-           "kvq_cache_status", "kvq_debug_decode_unset_wait", "kvq_debug_decode_timed", "kvq_decode_step")
+           "kvq_cache_status", "kvq_debug_decode_unset_wait", "kvq_debug_decode_timed", "kvq_decode_step",
+           "kvq_step_staging_bytes", "kvq_decode_step_host")
 KVQ_STATUS_WAIT_TIMEOUT = 1
 
 
@@ -83,6 +84,8 @@ def load() -> ctypes.CDLL:
         "kvq_debug_decode_unset_wait": ([VP, VP, I32, VP, VP, SZ, ctypes.c_int64, VP], I32),
         "kvq_debug_decode_timed": ([VP, VP, I32, VP, VP, SZ, VP, VP], I32),
         "kvq_decode_step": ([VP, VP, VP, VP, I32, VP, VP, SZ, VP], I32),
+        "kvq_step_staging_bytes": ([VP, I32, P(SZ)], I32),
+        "kvq_decode_step_host": ([VP, VP, VP, VP, I32, VP, VP, SZ, VP, SZ, VP], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -203,6 +206,27 @@ def kvq_decode_step(handle, K: torch.Tensor, V: torch.Tensor, q: torch.Tensor, o
     _check("kvq_decode_step", st)
 
 
+def kvq_step_staging_bytes(handle, dtype) -> int:
+    n = ctypes.c_size_t(0)
+    _check("kvq_step_staging_bytes", load().kvq_step_staging_bytes(handle, DTYPES[dtype], ctypes.byref(n)))
+    return n.value
+
+
+def kvq_decode_step_host(handle, K: torch.Tensor, V: torch.Tensor, q: torch.Tensor, dtype, out: torch.Tensor,
+                         staging: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """kvq_decode_step from host memory: K, V, q and out are CPU tensors (pinned for asynchronous
+    copies) holding the bytes of the layouts kvq_decode_step takes, inputs of type `dtype`; out is
+    valid once the stream reaches the end of the call's work."""
+    for t in (K, V, q, out):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("kvq_decode_step_host takes contiguous host tensors")
+    st = load().kvq_decode_step_host(handle, _ptr(K), _ptr(V), _ptr(q), DTYPES[dtype], _ptr(out), _ptr(staging),
+                                     staging.numel() * staging.element_size(), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("kvq_decode_step_host", st)
+    return out
+
+
 def kvq_decode_attention_static(handle, q: torch.Tensor, out: torch.Tensor, stream=None):
     """Decode attention without a workspace (partials in the library's fixed device array)."""
     if q.dtype not in DTYPES or out.dtype != torch.float32:
@@ -317,6 +341,16 @@ class KvqCache:
                               device=q.device)
         kvq_decode_step(self.handle, K, V, q, out, self.workspace, stream)
         return out
+
+    def step_host(self, K, V, q, out=None, stream=None):
+        """step() with host (CPU) inputs and output: one call enqueues the input copies, the step
+        and the output copy on the stream; returns out (valid after the stream reaches it)."""
+        if out is None:
+            out = torch.empty((self.batch, self.cfg.n_q_heads, self.out_dim), dtype=torch.float32).pin_memory()
+        need = kvq_step_staging_bytes(self.handle, q.dtype)
+        if getattr(self, "staging", None) is None or self.staging.numel() < need:
+            self.staging = torch.empty(need, dtype=torch.uint8, device=self.workspace.device)
+        return kvq_decode_step_host(self.handle, K, V, q, q.dtype, out, self.staging, self.workspace, stream)
 
     def decode(self, q, out=None, stream=None):
         if out is None:

@@ -4,6 +4,8 @@
 #include <cmath>
 #include <cstring>
 #include <new>
+#include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "kvq_internal.h"
@@ -511,6 +513,132 @@ kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const voi
   return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles, nullptr, &qp);
 }
 
+}  // extern "C"
+
+namespace {
+// Byte sizes of one step's K, V, q and out, and their offsets in the staging buffer: two input
+// slots (K, V, q each), then the output.
+struct StepStaging {
+  size_t n[4] = {};    // K, V, q, out
+  size_t off[4] = {};  // within an input slot (out: within the buffer)
+  size_t slot = 0;     // bytes of one input slot
+  size_t total = 0;
+};
+StepStaging step_staging(const kvq_cache* c, kvq_dtype dtype) {
+  const size_t elem = dtype == KVQ_BF16 ? 2 : 4, B = (size_t)c->batch, Hq = (size_t)c->cfg.n_q_heads;
+  StepStaging S;
+  if (c->is_fp4) {
+    S.n[0] = B * c->cfg.latent_dim * elem;
+    S.n[1] = B * c->cfg.rope_dim * elem;
+    S.n[2] = B * Hq * (size_t)(c->cfg.latent_dim + c->cfg.rope_dim) * elem;
+    S.n[3] = B * Hq * (size_t)c->cfg.latent_dim * sizeof(float);
+  } else {
+    S.n[0] = S.n[1] = B * (size_t)c->cfg.n_kv_heads * kHeadDim * elem;
+    S.n[2] = B * Hq * kHeadDim * elem;
+    S.n[3] = B * Hq * kHeadDim * sizeof(float);
+  }
+  for (int i = 0; i < 3; ++i) {
+    S.off[i] = S.slot;
+    S.slot = align_up(S.slot + S.n[i], 256);
+  }
+  S.off[3] = 2 * S.slot;
+  S.total = align_up(S.off[3] + S.n[3], 256);
+  return S;
+}
+
+// Per cache: the copy stream of kvq_decode_step_host and, per input slot, the events "inputs
+// landed" (copy stream) and "step done reading them" (caller's stream). Created at the first
+// call, released by kvq_cache_destroy.
+struct HostStep {
+  cudaStream_t copy = nullptr;
+  cudaEvent_t landed[2] = {}, done[2] = {};
+  unsigned long long calls = 0;
+};
+std::mutex g_host_step_mu;
+std::unordered_map<const kvq_cache*, HostStep> g_host_step;
+
+void release_host_step(HostStep& h) {
+  for (int i = 0; i < 2; ++i) {
+    if (h.landed[i]) cudaEventDestroy(h.landed[i]);
+    if (h.done[i]) cudaEventDestroy(h.done[i]);
+  }
+  if (h.copy) cudaStreamDestroy(h.copy);
+  h = HostStep{};
+}
+
+HostStep* host_step_state(const kvq_cache* c) {
+  std::lock_guard<std::mutex> lock(g_host_step_mu);
+  HostStep& h = g_host_step[c];
+  if (h.copy) return &h;
+  bool ok = cudaStreamCreateWithFlags(&h.copy, cudaStreamNonBlocking) == cudaSuccess;
+  for (int i = 0; i < 2 && ok; ++i)
+    ok = cudaEventCreateWithFlags(&h.landed[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&h.done[i], cudaEventDisableTiming) == cudaSuccess;
+  if (ok) return &h;
+  release_host_step(h);
+  g_host_step.erase(c);
+  return nullptr;
+}
+
+void forget_host_step(const kvq_cache* c) {
+  std::lock_guard<std::mutex> lock(g_host_step_mu);
+  auto it = g_host_step.find(c);
+  if (it == g_host_step.end()) return;
+  release_host_step(it->second);
+  g_host_step.erase(it);
+}
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_step_staging_bytes(const kvq_cache* c, kvq_dtype dtype, size_t* bytes) {
+  if (!c || !bytes || (dtype != KVQ_F32 && dtype != KVQ_BF16)) return KVQ_ERR_INVALID_ARG;
+  *bytes = step_staging(c, dtype).total;
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_step_host(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
+                                float* out, void* staging, size_t staging_bytes, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  if (!c || !K || !V || !q || !out || !staging || !workspace) return KVQ_ERR_INVALID_ARG;
+  if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(staging) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
+  const StepStaging S = step_staging(c, dtype);
+  if (staging_bytes < S.total) return KVQ_ERR_INVALID_ARG;
+  // what kvq_decode_step would refuse, refused before any copy
+  int max_len = 0;
+  for (int v : c->lens) {
+    if ((long)v + 1 > (long)c->capacity) return KVQ_ERR_CAPACITY;
+    max_len = std::max(max_len, v);
+  }
+  int splits, chunk;
+  plan_splits(decode_rows(c), c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c),
+              decode_waves_bound(c), max_len + 1, &splits, &chunk);
+  if (ws_bytes < workspace_for(c, splits)) return KVQ_ERR_WORKSPACE;
+  HostStep* h = host_step_state(c);
+  if (!h) return KVQ_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int slot = (int)(h->calls & 1);
+  char* in = static_cast<char*>(staging) + slot * S.slot;
+  char* dout = static_cast<char*>(staging) + S.off[3];
+  // the inputs cross on the copy stream once the step two calls back has read this slot, while
+  // the previous step may still run; the step waits for them on the caller's stream
+  if (cudaStreamWaitEvent(h->copy, h->done[slot], 0) != cudaSuccess) return KVQ_ERR_CUDA;
+  const void* src[3] = {K, V, q};
+  for (int i = 0; i < 3; ++i)
+    if (cudaMemcpyAsync(in + S.off[i], src[i], S.n[i], cudaMemcpyHostToDevice, h->copy) != cudaSuccess)
+      return KVQ_ERR_CUDA;
+  if (cudaEventRecord(h->landed[slot], h->copy) != cudaSuccess || cudaStreamWaitEvent(s, h->landed[slot], 0) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  const kvq_status r = kvq_decode_step(c, in + S.off[0], in + S.off[1], in + S.off[2], dtype,
+                                       reinterpret_cast<float*>(dout), workspace, ws_bytes, stream);
+  if (r != KVQ_OK) return r;
+  ++h->calls;
+  if (cudaEventRecord(h->done[slot], s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaMemcpyAsync(out, dout, S.n[3], cudaMemcpyDeviceToHost, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
 kvq_status kvq_debug_decode_unset_wait(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
                                        void* workspace, size_t ws_bytes, int64_t wait_limit_cycles,
                                        void* stream) {
@@ -578,7 +706,11 @@ kvq_status kvq_lloyd_max_table(int32_t bits, float* centroids, float* thresholds
   return KVQ_OK;
 }
 
-void kvq_cache_destroy(kvq_cache* c) { delete c; }
+void kvq_cache_destroy(kvq_cache* c) {
+  if (!c) return;
+  forget_host_step(c);
+  delete c;
+}
 
 kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_t n,
                                       uint32_t* planes, uint32_t* sketch, uint16_t* gamma,
@@ -624,7 +756,6 @@ kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_
 // Nothing in it has to start at zero: each call writes every partial slot it later reads. All
 // calls share it, so two calls that overlap on the GPU (e.g. on different streams) race.
 // ---------------------------------------------------------------------------------------------
-#include <mutex>
 
 namespace {
 constexpr size_t kStaticScratchBytes = size_t(16) << 20;

@@ -133,6 +133,29 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
 kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
                            float* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* Device bytes of the staging buffer kvq_decode_step_host needs for inputs of type dtype: two
+ * input slots (one step's K and V with n_new = 1 for all sequences, and q), then out; each region
+ * 256-byte aligned. */
+kvq_status kvq_step_staging_bytes(const kvq_cache* c, kvq_dtype dtype, size_t* bytes);
+
+/* kvq_decode_step with its inputs and output in HOST memory (layouts as for kvq_decode_step;
+ * dtype f32 or bf16; out [batch, n_q_heads, head_dim] f32, or latent_dim for FP4). The copies of
+ * K, V and q run on a copy stream the library keeps for the cache (created at the first call,
+ * released by kvq_cache_destroy), into the input slot of `staging` the step two calls back has
+ * finished with, so they overlap the previous step. The step waits for them on `stream`, and the
+ * copy of out back to host memory follows it on `stream`; the call returns without waiting, and
+ * out is valid once `stream` has reached that point. staging: device, 16-byte aligned, at least
+ * kvq_step_staging_bytes, used by nothing else while steps are in flight. Host inputs must be
+ * complete when the call is made (not pending writes of GPU work) and unchanged until `stream`
+ * has passed the call; pinned (page-locked) memory keeps the copies asynchronous, pageable memory
+ * makes the runtime stage them. Everything kvq_decode_step checks is checked before the first
+ * copy, so those errors enqueue nothing; KVQ_ERR_CUDA means a copy, event or launch failed,
+ * possibly after earlier copies were enqueued. The paper has no counterpart; it keeps a serving
+ * loop to one call per step. */
+kvq_status kvq_decode_step_host(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
+                                float* out, void* staging, size_t staging_bytes, void* workspace,
+                                size_t ws_bytes, void* stream);
+
 /* The same decode attention as kvq_decode_attention, for callers that cannot allocate device
  * memory on the decode path (serving loops that reserve all memory up front, hosts whose memory
  * belongs to another allocator, code that must not risk the device synchronisation cudaMalloc

@@ -321,6 +321,48 @@ def test_decode_step_ragged_long():
     c2.close()
 
 
+@pytest.mark.parametrize("name,pinned", [("llama8b", True), ("llama70b", False), ("mla_fp4", True)])
+def test_decode_step_host_equals_device_step(name, pinned):
+    """kvq_decode_step_host (inputs and output in host memory, copies enqueued by the library)
+    appends the same tokens and returns the same output as kvq_decode_step on device buffers."""
+    w = WORKLOADS[name]
+    fp4 = w.k_mode == "fp4"
+    B = 3
+    data = generate(w, DEV, seqs=range(B), ctx=256)
+    mk = (lambda: kvq.KvqCache(kvq.cfg_for_workload(w), B, 256)) if fp4 else (lambda: new_cache(w, B, 256)[0])
+    a, v = (data["latent"], data["rope"]) if fp4 else (data["k"], data["v"])
+    c1, c2 = mk(), mk()
+    for c in (c1, c2):
+        c.quantize(a[:, :150].contiguous() if fp4 else a[:, :, :150].contiguous(),
+                   v[:, :150].contiguous() if fp4 else v[:, :, :150].contiguous())
+    host = lambda t: t.cpu().pin_memory() if pinned else t.cpu()
+    # four steps enqueued back to back (inputs of step j + 1 cross while step j runs), then compared
+    refs, outs, keep = [], [], []
+    for step in range(4):
+        new = generate(w, DEV, seqs=range(B), step=step)
+        na, nv = (new["latent"], new["rope"]) if fp4 else (new["k"], new["v"])
+        refs.append(c1.step(na, nv, data["q"]).clone())
+        keep.append((host(na), host(nv), host(data["q"])))
+    torch.cuda.synchronize()
+    for step in range(4):
+        outs.append(host(torch.empty(refs[0].shape, dtype=torch.float32)))
+        c2.step_host(*keep[step], outs[step])
+    torch.cuda.synchronize()
+    for step in range(4):
+        assert torch.equal(outs[step], refs[step].cpu()), (name, step)
+    assert list(c1.lengths()) == list(c2.lengths()) == [154] * B
+    # a step past the capacity is refused before anything is copied or appended
+    full = mk()
+    full.quantize(a[:, :256].contiguous() if fp4 else a[:, :, :256].contiguous(),
+                  v[:, :256].contiguous() if fp4 else v[:, :, :256].contiguous())
+    with pytest.raises(kvq.KvqError) as e:
+        full.step_host(*keep[0], host(torch.empty(refs[0].shape, dtype=torch.float32)))
+    assert e.value.status == 3  # KVQ_ERR_CAPACITY
+    assert list(full.lengths()) == [256] * B
+    for c in (c1, c2, full):
+        c.close()
+
+
 # ---------------------------------------------------------------- bounded waits
 
 def test_bounded_wait_sets_status_and_returns():
