@@ -216,7 +216,8 @@ def kvq_decode_step_host(handle, K: torch.Tensor, V: torch.Tensor, q: torch.Tens
                          staging: torch.Tensor, workspace: torch.Tensor, stream=None):
     """kvq_decode_step from host memory: K, V, q and out are CPU tensors (pinned for asynchronous
     copies) holding the bytes of the layouts kvq_decode_step takes, inputs of type `dtype`; out is
-    valid once the stream reaches the end of the call's work."""
+    valid once the stream reaches the end of the call's work. The sizes are the caller's to get
+    right (KvqCache.step_host checks them)."""
     for t in (K, V, q, out):
         if t.is_cuda or not t.is_contiguous():
             raise ValueError("kvq_decode_step_host takes contiguous host tensors")
@@ -347,6 +348,16 @@ class KvqCache:
         and the output copy on the stream; returns out (valid after the stream reaches it)."""
         if out is None:
             out = torch.empty((self.batch, self.cfg.n_q_heads, self.out_dim), dtype=torch.float32).pin_memory()
+        # the library cannot see host buffer sizes: check them here
+        B, Hq, cfg = self.batch, self.cfg.n_q_heads, self.cfg
+        if cfg.k_mode == MODES["fp4"]:
+            want = (B * cfg.latent_dim, B * cfg.rope_dim, B * Hq * (cfg.latent_dim + cfg.rope_dim))
+        else:
+            want = (B * cfg.n_kv_heads * cfg.head_dim,) * 2 + (B * Hq * cfg.head_dim,)
+        if tuple(t.numel() for t in (K, V, q)) != want or K.dtype != q.dtype or V.dtype != q.dtype:
+            raise ValueError(f"step_host: K, V, q must hold {want} elements of one dtype")
+        if out.dtype != torch.float32 or out.numel() != B * Hq * self.out_dim:
+            raise ValueError("step_host: out must be float32 [batch, n_q_heads, out_dim]")
         need = kvq_step_staging_bytes(self.handle, q.dtype)
         if getattr(self, "staging", None) is None or self.staging.numel() < need:
             self.staging = torch.empty(need, dtype=torch.uint8, device=self.workspace.device)

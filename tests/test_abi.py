@@ -111,3 +111,23 @@ def test_rejected_calls_launch_nothing(lib):
     assert lib.kvq_cache_init(ctypes.byref(h), ctypes.byref(kvq.make_cfg()), 1, 32, None, 1 << 20,
                               signs.ctypes.data_as(ctypes.c_void_p), None, None) == 1
     assert kvq.kvq_kernel_launches() == n0
+
+
+def test_step_host_checks_host_buffer_sizes(lib):
+    """KvqCache.step_host refuses host tensors whose sizes do not match the cache's step layout
+    (the library cannot see host buffer sizes) before anything reaches the library; the C entry
+    refuses a null cache."""
+    import torch
+    cache = object.__new__(kvq.KvqCache)
+    cache.batch, cache.cfg, cache.out_dim, cache.handle = 3, kvq.make_cfg(n_q_heads=32, n_kv_heads=8), 128, None
+    K = torch.zeros(3, 8, 1, 128, dtype=torch.bfloat16)
+    q = torch.zeros(3, 32, 128, dtype=torch.bfloat16)
+    out = torch.zeros(3, 32, 128)
+    n0 = kvq.kvq_kernel_launches()
+    for bad in ((K[:2], K, q, out), (K, K, q[:, :16], out), (K, K.float(), q, out), (K, K, q, out[:1]),
+                (K, K, q, out.double())):
+        with pytest.raises(ValueError):
+            cache.step_host(*bad)
+    with pytest.raises(kvq.KvqError):  # sizes right: the library itself refuses the null cache
+        cache.step_host(K, K, q, out)
+    assert kvq.kvq_kernel_launches() == n0
