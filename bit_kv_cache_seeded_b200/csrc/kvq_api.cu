@@ -630,22 +630,12 @@ kvq_status kvq_decode_step_host(kvq_cache* c, const void* K, const void* V, cons
       return KVQ_ERR_CUDA;
   if (cudaEventRecord(h->landed[slot], h->copy) != cudaSuccess || cudaStreamWaitEvent(s, h->landed[slot], 0) != cudaSuccess)
     return KVQ_ERR_CUDA;
-  // Page-locked host memory is mapped into the device's address space: the reduce writes the
-  // output there directly. Other host memory gets a copy from the staging buffer after the step.
-  float* mapped = nullptr;
-  cudaPointerAttributes pa;
-  if (cudaPointerGetAttributes(&pa, out) == cudaSuccess) {
-    if (pa.type == cudaMemoryTypeHost && pa.devicePointer && aligned16(pa.devicePointer))
-      mapped = static_cast<float*>(pa.devicePointer);
-  } else {
-    cudaGetLastError();  // plain pageable memory: clear the lookup's error
-  }
   const kvq_status r = kvq_decode_step(c, in + S.off[0], in + S.off[1], in + S.off[2], dtype,
-                                       mapped ? mapped : reinterpret_cast<float*>(dout), workspace, ws_bytes, stream);
+                                       reinterpret_cast<float*>(dout), workspace, ws_bytes, stream);
   if (r != KVQ_OK) return r;
   ++h->calls;
   if (cudaEventRecord(h->done[slot], s) != cudaSuccess) return KVQ_ERR_CUDA;
-  if (!mapped && cudaMemcpyAsync(out, dout, S.n[3], cudaMemcpyDeviceToHost, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (cudaMemcpyAsync(out, dout, S.n[3], cudaMemcpyDeviceToHost, s) != cudaSuccess) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }
 

@@ -142,10 +142,9 @@ kvq_status kvq_step_staging_bytes(const kvq_cache* c, kvq_dtype dtype, size_t* b
  * dtype f32 or bf16; out [batch, n_q_heads, head_dim] f32, or latent_dim for FP4). The copies of
  * K, V and q run on a copy stream the library keeps for the cache (created at the first call,
  * released by kvq_cache_destroy), into the input slot of `staging` the step two calls back has
- * finished with, so they overlap the previous step. The step waits for them on `stream`. When out
- * is page-locked host memory (mapped into the device's address space) the step writes it
- * directly; otherwise a copy back from the staging buffer follows the step on `stream`. The call
- * returns without waiting, and out is valid once `stream` has reached the end of its work. staging: device, 16-byte aligned, at least
+ * finished with, so they overlap the previous step. The step waits for them on `stream`, and the
+ * copy of out back to host memory follows it on `stream`; the call returns without waiting, and
+ * out is valid once `stream` has reached that point. staging: device, 16-byte aligned, at least
  * kvq_step_staging_bytes, used by nothing else while steps are in flight. Host inputs must be
  * complete when the call is made (not pending writes of GPU work) and unchanged until `stream`
  * has passed the call; pinned (page-locked) memory keeps the copies asynchronous, pageable memory
