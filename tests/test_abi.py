@@ -131,3 +131,47 @@ def test_step_host_checks_host_buffer_sizes(lib):
     with pytest.raises(kvq.KvqError):  # sizes right: the library itself refuses the null cache
         cache.step_host(K, K, q, out)
     assert kvq.kvq_kernel_launches() == n0
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "kvq.h"
+int main(void) {
+  float c[8], t[7];
+  size_t bytes = 0;
+  kvq_cfg cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.head_dim = 128; cfg.n_q_heads = 32; cfg.n_kv_heads = 8; cfg.k_mode = KVQ_MODE_LM_QJL;
+  cfg.v_mode = KVQ_MODE_LM_QJL; cfg.k_bits = 2; cfg.v_bits = 2; cfg.qjl_dim = 128;
+  if (kvq_lloyd_max_table(2, c, t) != KVQ_OK) return 1;
+  if (kvq_lloyd_max_table(4, c, t) != KVQ_ERR_INVALID_ARG) return 2;
+  if (kvq_packed_bytes_per_token(&cfg, &bytes) != KVQ_OK) return 3;
+  if (kvq_decode_step_host(NULL, NULL, NULL, NULL, KVQ_BF16, NULL, NULL, 0, NULL, 0, NULL) != KVQ_ERR_INVALID_ARG) return 4;
+  printf("%s|%zu|%.6f\n", kvq_status_str(KVQ_ERR_CAPACITY), bytes, c[3]);
+  return 0;
+}
+"""
+
+
+def test_plain_c_client_links_and_runs(lib, tmp_path):
+    """A C99 program that includes kvq.h, links libkvq.so and calls its host-only entries: the
+    boundary is usable without C++ or Python."""
+    import subprocess
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(kvq.LIB_PATH)
+    try:
+        subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                        "-L", libdir, "-lkvq", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       check=True, capture_output=True, text=True)
+    except FileNotFoundError:
+        pytest.skip("gcc not available")
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stdout + out.stderr
+    name, nbytes, c3 = out.stdout.strip().split("|")
+    cfg = kvq.make_cfg(head_dim=128, n_q_heads=32, n_kv_heads=8, k_bits=2, v_bits=2, qjl_dim=128)
+    assert name == kvq.kvq_status_str(3)
+    assert int(nbytes) == kvq.kvq_packed_bytes_per_token(cfg)
+    assert abs(float(c3) - float(kvq.kvq_lloyd_max_table(2)[0][3])) < 1e-6
