@@ -104,6 +104,14 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _on_device(fn: str, **tensors):
+    """Device entry points take device pointers: a host tensor would reach a kernel as an address
+    it cannot read, so refuse it here."""
+    for name, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{fn}: {name} must be a CUDA tensor")
+
+
 def _stream(stream=None):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -146,6 +154,7 @@ def kvq_packed_bytes_per_token(cfg: kvq_cfg) -> int:
 
 def kvq_cache_init(cfg: kvq_cfg, batch: int, capacity: int, arena: torch.Tensor, rot_signs=None,
                    qjl_matrix=None, stream=None) -> ctypes.c_void_p:
+    _on_device("kvq_cache_init", arena=arena)
     handle = ctypes.c_void_p()
     signs = None if rot_signs is None else np.ascontiguousarray(rot_signs, dtype=np.int8)
     S = None if qjl_matrix is None else np.ascontiguousarray(qjl_matrix, dtype=np.float32)
@@ -158,6 +167,7 @@ def kvq_cache_init(cfg: kvq_cfg, batch: int, capacity: int, arena: torch.Tensor,
 
 
 def kvq_quantize(handle, K: torch.Tensor, V: torch.Tensor, seq_ids=None, stream=None):
+    _on_device("kvq_quantize", K=K, V=V)
     if K.dtype not in DTYPES or V.dtype != K.dtype:
         raise TypeError("K and V must both be float32 or bfloat16")
     if not (K.is_contiguous() and V.is_contiguous()):
@@ -183,6 +193,7 @@ def kvq_workspace_bytes(handle) -> int:
 
 def kvq_decode_attention(handle, q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
                          stream=None):
+    _on_device("kvq_decode_attention", q=q, out=out, workspace=workspace)
     if q.dtype not in DTYPES or out.dtype != torch.float32:
         raise TypeError("q must be float32/bfloat16 and out float32")
     if not (q.is_contiguous() and out.is_contiguous()):
@@ -195,6 +206,7 @@ def kvq_decode_attention(handle, q: torch.Tensor, out: torch.Tensor, workspace: 
 def kvq_decode_step(handle, K: torch.Tensor, V: torch.Tensor, q: torch.Tensor, out: torch.Tensor,
                     workspace: torch.Tensor, stream=None):
     """Append one token per sequence (K, V [B, Hkv, 1, d]; FP4: latent, rope) and decode with q."""
+    _on_device("kvq_decode_step", K=K, V=V, q=q, out=out, workspace=workspace)
     if K.dtype != V.dtype or K.dtype != q.dtype or q.dtype not in DTYPES or out.dtype != torch.float32:
         raise TypeError("K, V and q must share float32/bfloat16; out is float32")
     if not (K.is_contiguous() and V.is_contiguous() and q.is_contiguous() and out.is_contiguous()):
@@ -230,6 +242,7 @@ def kvq_decode_step_host(handle, K: torch.Tensor, V: torch.Tensor, q: torch.Tens
 
 def kvq_decode_attention_static(handle, q: torch.Tensor, out: torch.Tensor, stream=None):
     """Decode attention without a workspace (partials in the library's fixed device array)."""
+    _on_device("kvq_decode_attention_static", q=q, out=out)
     if q.dtype not in DTYPES or out.dtype != torch.float32:
         raise TypeError("q must be float32/bfloat16 and out float32")
     if not (q.is_contiguous() and out.is_contiguous()):
@@ -248,6 +261,7 @@ def kvq_cache_status(handle, stream=None) -> int:
 def kvq_debug_decode_unset_wait(handle, q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
                                 wait_limit_cycles: int, stream=None):
     """Test entry: decode with one extra bounded wait on a barrier that nothing completes."""
+    _on_device("kvq_debug_decode_unset_wait", q=q, out=out, workspace=workspace)
     if q.dtype not in DTYPES or out.dtype != torch.float32:
         raise TypeError("q must be float32/bfloat16 and out float32")
     if not (q.is_contiguous() and out.is_contiguous()):
@@ -261,6 +275,7 @@ def kvq_debug_decode_unset_wait(handle, q: torch.Tensor, out: torch.Tensor, work
 def kvq_debug_decode_timed(handle, q: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, events,
                            stream=None):
     """Decode recording 4 torch.cuda.Events: start, after prep, after the split kernel, after reduce."""
+    _on_device("kvq_debug_decode_timed", q=q, out=out, workspace=workspace)
     if q.dtype not in DTYPES or out.dtype != torch.float32:
         raise TypeError("q must be float32/bfloat16 and out float32")
     if len(events) != 4:
@@ -305,6 +320,7 @@ def kvq_kernel_launches() -> int:
 
 
 def kvq_debug_quantize_rotated(handle, u: torch.Tensor, k_bits: int, qjl: bool, stream=None):
+    _on_device("kvq_debug_quantize_rotated", u=u)
     n = u.shape[0]
     planes = torch.zeros((n, k_bits, 4), dtype=torch.int32, device=u.device)
     sketch = torch.zeros((n, 4), dtype=torch.int32, device=u.device) if qjl else None
@@ -332,11 +348,37 @@ class KvqCache:
                                      device=device)
         self.out_dim = cfg.latent_dim if cfg.k_mode == MODES["fp4"] else cfg.head_dim
 
+    # Shapes the library reads and writes; it cannot see tensor extents, so they are checked here.
+    def _kv_shapes(self, n_seq: int, n_new: int):
+        cfg = self.cfg
+        if cfg.k_mode == MODES["fp4"]:
+            return (n_seq, n_new, cfg.latent_dim), (n_seq, n_new, cfg.rope_dim)
+        kv = (n_seq, cfg.n_kv_heads, n_new, cfg.head_dim)
+        return kv, kv
+
+    def _check_kv(self, fn, K, V, n_seq, n_new):
+        if K.dim() < 2 or (tuple(K.shape), tuple(V.shape)) != self._kv_shapes(n_seq, n_new):
+            raise ValueError(f"{fn}: K, V must be {self._kv_shapes(n_seq, n_new)}, got {tuple(K.shape)}, {tuple(V.shape)}")
+
+    def _check_q_out(self, fn, q, out):
+        cfg = self.cfg
+        dq = cfg.latent_dim + cfg.rope_dim if cfg.k_mode == MODES["fp4"] else cfg.head_dim
+        if tuple(q.shape) != (self.batch, cfg.n_q_heads, dq):
+            raise ValueError(f"{fn}: q must be {(self.batch, cfg.n_q_heads, dq)}, got {tuple(q.shape)}")
+        if out is not None and tuple(out.shape) != (self.batch, cfg.n_q_heads, self.out_dim):
+            raise ValueError(f"{fn}: out must be {(self.batch, cfg.n_q_heads, self.out_dim)}")
+
     def quantize(self, K, V, seq_ids=None, stream=None):
+        n_seq = K.shape[0] if K.dim() else 0
+        if seq_ids is None and n_seq > self.batch:
+            raise ValueError("quantize: more sequences than the cache holds")
+        self._check_kv("quantize", K, V, n_seq, K.shape[-2] if K.dim() >= 2 else 0)
         kvq_quantize(self.handle, K, V, seq_ids, stream)
 
     def step(self, K, V, q, out=None, stream=None):
         """Append one token per sequence and decode (kvq_decode_step); returns out."""
+        self._check_kv("step", K, V, self.batch, 1)
+        self._check_q_out("step", q, out)
         if out is None:
             out = torch.empty((self.batch, self.cfg.n_q_heads, self.out_dim), dtype=torch.float32,
                               device=q.device)
@@ -364,6 +406,7 @@ class KvqCache:
         return kvq_decode_step_host(self.handle, K, V, q, q.dtype, out, self.staging, self.workspace, stream)
 
     def decode(self, q, out=None, stream=None):
+        self._check_q_out("decode", q, out)
         if out is None:
             out = torch.empty((self.batch, self.cfg.n_q_heads, self.out_dim), dtype=torch.float32,
                               device=q.device)

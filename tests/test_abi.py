@@ -175,3 +175,31 @@ def test_plain_c_client_links_and_runs(lib, tmp_path):
     assert name == kvq.kvq_status_str(3)
     assert int(nbytes) == kvq.kvq_packed_bytes_per_token(cfg)
     assert abs(float(c3) - float(kvq.kvq_lloyd_max_table(2)[0][3])) < 1e-6
+
+
+def test_binding_refuses_host_tensors_and_wrong_shapes(lib):
+    """The library reads device pointers with the extents the cache's configuration implies; the
+    binding refuses host tensors at every device entry and KvqCache refuses shapes that do not
+    match its configuration, before anything reaches the library."""
+    import torch
+    cache = object.__new__(kvq.KvqCache)
+    cache.batch, cache.cfg, cache.out_dim, cache.handle = 2, kvq.make_cfg(n_q_heads=8, n_kv_heads=2), 128, None
+    cache.workspace = torch.zeros(16, dtype=torch.uint8)
+    K = torch.zeros(2, 2, 5, 128)
+    q = torch.zeros(2, 8, 128)
+    n0 = kvq.kvq_kernel_launches()
+    bad_shapes = [lambda: cache.quantize(K, K[:, :1]), lambda: cache.quantize(torch.zeros(3, 2, 5, 128), torch.zeros(3, 2, 5, 128)),
+                  lambda: cache.quantize(K[..., :64], K[..., :64]), lambda: cache.decode(q[:, :4]),
+                  lambda: cache.decode(q, torch.zeros(2, 8, 64)), lambda: cache.step(K, K, q),
+                  lambda: cache.step(K[:, :, :1], K[:, :, :1], q[:1])]
+    for call in bad_shapes:
+        with pytest.raises(ValueError, match="must be|more sequences"):
+            call()
+    host = [lambda: cache.quantize(K, K), lambda: cache.decode(q, torch.zeros(2, 8, 128)),
+            lambda: cache.step(K[:, :, :1].contiguous(), K[:, :, :1].contiguous(), q, torch.zeros(2, 8, 128)),
+            lambda: kvq.kvq_decode_attention_static(None, q, torch.zeros(2, 8, 128)),
+            lambda: kvq.kvq_cache_init(kvq.make_cfg(), 1, 32, torch.zeros(16, dtype=torch.uint8))]
+    for call in host:
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
+    assert kvq.kvq_kernel_launches() == n0
