@@ -68,6 +68,7 @@ def resolve_side(x, planes_g, sketch_g, n16_g, g16_g, bits, signs, S, stats):
         zd = z_o != z_g
         assert np.all(np.abs(proj[zd]) < tol[zd]), "sketch bit differs away from zero"
         stats["sketch_flips"] = stats.get("sketch_flips", 0) + int(zd.sum())
+        stats["sketch_bits"] = stats.get("sketch_bits", 0) + zd.size
         z = z_g
     return codes, n16, g16, z
 
@@ -89,6 +90,18 @@ def pair_reference(w, arena, info, b, hk, T, K, V, q, signs, S, stats):
     Kh = attention.dequantize_many(codes_k, n16k, ck, signs, g16k, zk, kq)
     Vh = attention.dequantize_many(codes_v, n16v, cv, signs, g16v, zv, vq)
     return attention.decode_attention(q, Kh, Vh, 1.0 / math.sqrt(w.head_dim))
+
+
+MAX_FLIP_RATE = 1e-3     # rounding-level code / sign decisions allowed, per decision compared
+
+
+def check_flip_rates(stats, where=""):
+    """Bound how often the rounding-level exceptions above were taken: at most MAX_FLIP_RATE of
+    the codes and of the sketch sign bits compared may differ from the oracle's decision."""
+    print(f"{where}: code flips {stats.get('code_flips', 0)}/{stats.get('coords', 0)}, "
+          f"sketch flips {stats.get('sketch_flips', 0)}/{stats.get('sketch_bits', 0)}")
+    assert stats.get("code_flips", 0) <= MAX_FLIP_RATE * max(1, stats.get("coords", 0)), stats
+    assert stats.get("sketch_flips", 0) <= MAX_FLIP_RATE * max(1, stats.get("sketch_bits", 0)), stats
 
 
 def rel_err(out, ref):

@@ -16,7 +16,7 @@ from kvq_inputs import WORKLOADS, generate
 from kvq_inputs.workloads import rotation_and_sketch
 from oracle import codec, tables, attention
 from tests._cache_reader import fp4_fields, side_fields
-from tests._parity import pair_reference, rel_err, REL_TOL, BOUNDARY
+from tests._parity import pair_reference, rel_err, REL_TOL, BOUNDARY, check_flip_rates
 
 pytestmark = pytest.mark.gpu
 
@@ -56,6 +56,7 @@ def test_debug_quantize_rotated_bit_exact(bits, qjl):
     planes, sketch, gamma = kvq.kvq_debug_quantize_rotated(cache.handle, ut, bits, qjl)
     torch.cuda.synchronize()
     planes = planes.cpu().numpy().view(np.uint32)
+    flips = 0
     for i in range(u.shape[0]):
         r = codec.quantize_rotated(u[i].astype(np.float64), bits, c32, t32, S if qjl else None)
         np.testing.assert_array_equal(planes[i], r["planes"])
@@ -64,8 +65,11 @@ def test_debug_quantize_rotated_bit_exact(bits, qjl):
             mism = np.nonzero(codec.unpack_bits(zg, 128) != r["z"])[0]
             tol = 4 * 128 * 2.0 ** -24 * (np.abs(S.astype(np.float64)) @ np.abs(r["rho"]))
             assert np.all(np.abs(r["proj"][mism]) < tol[mism])
+            flips += len(mism)
             g = float(gamma[i:i + 1].cpu().numpy().view(np.float16)[0])
             assert abs(g - r["gamma16"]) <= 2.0 ** (math.floor(math.log2(max(r["gamma"], 2 ** -14))) - 10)
+    print(f"sign bits differing inside the fp32 bound: {flips} of {u.shape[0] * 128}")
+    assert flips <= 1e-3 * u.shape[0] * 128
     cache.close()
 
 
@@ -104,6 +108,7 @@ def run_small(name, batch, lens, seed_appends=1, w=None):
             err = rel_err(out[b, hk * g:(hk + 1) * g], ref)
             assert np.all(err <= REL_TOL), (b, hk, err.max())
     cache.close()
+    check_flip_rates(stats, w.name)
     return stats
 
 
@@ -176,6 +181,7 @@ def test_full_size_sampled_pairs(name):
         err = rel_err(out[b, hk * g:(hk + 1) * g], ref)
         assert np.all(err <= REL_TOL), (name, b, hk, err.max())
     assert np.all(np.isfinite(out))
+    check_flip_rates(stats, name)
     cache.close()
 
 

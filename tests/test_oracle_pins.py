@@ -448,3 +448,82 @@ def test_vectorised_forms_equal_per_vector_forms():
 
 def codec_fp4_rows(packed, scales):
     return np.stack([codec.fp4_dequantize(packed[t], scales[t]) for t in range(packed.shape[0])])
+
+
+# ---------------------------------------------------------------- MLA decode, hand-worked
+
+def _mla_golden_cases(golden):
+    """Cases of tests/golden/mla_hand_example.txt as (q, packed, scales, k_rope, expected out)."""
+    cases, cur = {}, None
+    for row in golden("mla_hand_example.txt"):
+        kind = row[0]
+        if kind == "case":
+            T, H = int(row[3]), int(row[4])
+            cur = dict(packed=np.zeros((T, 256), np.uint8), scales=np.full((T, 32), 0x38, np.uint8),
+                       rope=np.zeros((T, 64)), q=np.zeros((H, 576)), out=np.zeros((H, 512)))
+            cases[row[1]] = cur
+        elif kind == "byte":
+            cur["packed"][int(row[1]), int(row[2])] = int(row[3], 16)
+        elif kind == "scale":
+            cur["scales"][int(row[1]), int(row[2])] = int(row[3], 16)
+        elif kind == "rope":
+            cur["rope"][int(row[1]), int(row[2])] = float(row[3])
+        elif kind == "qlat":
+            cur["q"][int(row[1]), int(row[2])] = float(row[3])
+        elif kind == "qrope":
+            cur["q"][int(row[1]), 512 + int(row[2])] = float(row[3])
+        elif kind == "out":
+            cur["out"][int(row[1]), int(row[2])] = float(row[3])
+    return cases
+
+
+def _mla_matches_golden(fn, golden):
+    """True when fn(q, packed, scales, k_rope, scale) reproduces every hand-worked case."""
+    for name, c in _mla_golden_cases(golden).items():
+        got = np.asarray(fn(c["q"], c["packed"], c["scales"], c["rope"], 1.0 / 24.0))
+        if got.shape != c["out"].shape or not np.allclose(got, c["out"], rtol=1e-13, atol=1e-15):
+            return False
+    return True
+
+
+def test_mla_decode_attention_hand_worked(golden):
+    cases = _mla_golden_cases(golden)
+    assert set(cases) == {"two", "rope_only", "zero_latent"}
+    for name, c in cases.items():
+        got = attention.mla_decode_attention(c["q"], c["packed"], c["scales"], c["rope"], 1.0 / 24.0)
+        np.testing.assert_allclose(got, c["out"], rtol=1e-13, atol=1e-15, err_msg=name)
+        many = attention.mla_decode_attention_many(c["q"], c["packed"], c["scales"], c["rope"], 1.0 / 24.0)
+        np.testing.assert_allclose(many, c["out"], rtol=1e-13, atol=1e-15, err_msg=name)
+    # the scale is 1/sqrt(latent + rope) = 1/24 for the 512 + 64 configuration
+    assert 1.0 / math.sqrt(512 + 64) == 1.0 / 24.0
+
+
+def test_mla_hand_worked_cases_reject_plausible_mistakes(golden):
+    """Planted mistakes in a copy of the oracle's MLA decode: each must fail the hand-worked cases."""
+    def keys_values(packed, scales, rope):
+        lat = np.stack([codec.fp4_dequantize(packed[t], scales[t]) for t in range(packed.shape[0])])
+        return lat, np.asarray(rope, np.float64)
+
+    def dropped_rope(q, packed, scales, rope, scale):
+        lat, _ = keys_values(packed, scales, rope)
+        return np.stack([attention.softmax_attention(qh[:512], lat, lat, scale) for qh in q])
+
+    def rope_in_values(q, packed, scales, rope, scale):
+        lat, kr = keys_values(packed, scales, rope)
+        K = np.concatenate([lat, kr], axis=1)
+        V = lat + np.pad(kr, ((0, 0), (0, 448)))
+        return np.stack([attention.softmax_attention(qh, K, V, scale) for qh in q])
+
+    def latent_only_scale(q, packed, scales, rope, scale):
+        lat, kr = keys_values(packed, scales, rope)
+        K = np.concatenate([lat, kr], axis=1)
+        return np.stack([attention.softmax_attention(qh, K, lat, 1.0 / math.sqrt(512)) for qh in q])
+
+    def sign_dropped(q, packed, scales, rope, scale):
+        lat, kr = keys_values(packed & 0x77, scales, rope)
+        K = np.concatenate([lat, kr], axis=1)
+        return np.stack([attention.softmax_attention(qh, K, lat, scale) for qh in q])
+
+    assert _mla_matches_golden(attention.mla_decode_attention, golden)
+    for bad in (dropped_rope, rope_in_values, latent_only_scale, sign_dropped):
+        assert not _mla_matches_golden(bad, golden), bad.__name__
