@@ -34,7 +34,7 @@ EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "k
            "kvq_cache_layout", "kvq_lloyd_max_table", "kvq_cache_destroy",
            "kvq_debug_quantize_rotated", "kvq_decode_attention_static", "kvq_kernel_launches",
            "kvq_cache_status", "kvq_debug_decode_unset_wait", "kvq_debug_decode_timed", "kvq_decode_step",
-           "kvq_step_staging_bytes", "kvq_decode_step_host")
+           "kvq_step_staging_bytes", "kvq_decode_step_host", "kvq_draw_rotation_signs", "kvq_draw_qjl_matrix")
 KVQ_STATUS_WAIT_TIMEOUT = 1
 
 
@@ -50,7 +50,8 @@ class kvq_cfg(ctypes.Structure):
                 ("v_mode", ctypes.c_int32), ("k_bits", ctypes.c_int32),
                 ("v_bits", ctypes.c_int32), ("qjl_dim", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("latent_dim", ctypes.c_int32),
-                ("rope_dim", ctypes.c_int32)]
+                ("rope_dim", ctypes.c_int32), ("rot_per_head", ctypes.c_int32),
+                ("rot_seed", ctypes.c_uint64), ("qjl_seed", ctypes.c_uint64)]
 
 
 _lib = None
@@ -86,6 +87,8 @@ def load() -> ctypes.CDLL:
         "kvq_decode_step": ([VP, VP, VP, VP, I32, VP, VP, SZ, VP], I32),
         "kvq_step_staging_bytes": ([VP, I32, P(SZ)], I32),
         "kvq_decode_step_host": ([VP, VP, VP, VP, I32, VP, VP, SZ, VP, SZ, VP], I32),
+        "kvq_draw_rotation_signs": ([ctypes.c_uint64, I32, VP], I32),
+        "kvq_draw_qjl_matrix": ([ctypes.c_uint64, I32, I32, VP], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -119,19 +122,35 @@ def _stream(stream=None):
 
 
 def make_cfg(head_dim=128, n_q_heads=1, n_kv_heads=1, k_mode="lm_qjl", v_mode="lm_qjl", k_bits=2,
-             v_bits=2, qjl_dim=128, softmax_scale=0.0, latent_dim=0, rope_dim=0) -> kvq_cfg:
+             v_bits=2, qjl_dim=128, softmax_scale=0.0, latent_dim=0, rope_dim=0, rot_per_head=0,
+             rot_seed=0, qjl_seed=0) -> kvq_cfg:
     return kvq_cfg(head_dim, n_q_heads, n_kv_heads, MODES[k_mode], MODES[v_mode], k_bits, v_bits,
-                   qjl_dim, softmax_scale, latent_dim, rope_dim)
+                   qjl_dim, softmax_scale, latent_dim, rope_dim, int(rot_per_head), rot_seed, qjl_seed)
 
 
 def cfg_for_workload(w) -> kvq_cfg:
-    """kvq_cfg of a kvq_inputs.Workload."""
+    """kvq_cfg of a kvq_inputs.Workload (its seeds included)."""
     if w.k_mode == "fp4":
         return make_cfg(head_dim=w.latent_dim, n_q_heads=w.n_q_heads, n_kv_heads=1, k_mode="fp4",
                         v_mode="fp4", k_bits=4, v_bits=4, qjl_dim=0, latent_dim=w.latent_dim,
                         rope_dim=w.rope_dim)
     return make_cfg(w.head_dim, w.n_q_heads, w.n_kv_heads, w.k_mode, w.v_mode, w.k_bits, w.v_bits,
-                    w.qjl_dim)
+                    w.qjl_dim, rot_per_head=int(getattr(w, "rot_per_head", False)), rot_seed=w.rot_seed,
+                    qjl_seed=w.qjl_seed)
+
+
+def kvq_draw_rotation_signs(seed: int, n: int) -> np.ndarray:
+    """The library's seeded +-1 draws (int8 [n]), as kvq_cache_init makes them from a seed."""
+    out = np.zeros(n, dtype=np.int8)
+    _check("kvq_draw_rotation_signs", load().kvq_draw_rotation_signs(seed, n, out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
+def kvq_draw_qjl_matrix(seed: int, m: int, d: int) -> np.ndarray:
+    """The library's seeded Gaussian sketch matrix (float32 [m, d])."""
+    out = np.zeros((m, d), dtype=np.float32)
+    _check("kvq_draw_qjl_matrix", load().kvq_draw_qjl_matrix(seed, m, d, out.ctypes.data_as(ctypes.c_void_p)))
+    return out
 
 
 # ---------------------------------------------------------------- same-name wrappers

@@ -29,7 +29,9 @@ kvq_status validate_cfg(const kvq_cfg* c) {
   if (!c) return KVQ_ERR_INVALID_ARG;
   if (c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->n_q_heads % c->n_kv_heads) return KVQ_ERR_INVALID_ARG;
   if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  if (c->rot_per_head != 0 && c->rot_per_head != 1) return KVQ_ERR_INVALID_ARG;
   if (c->k_mode == KVQ_MODE_FP4 || c->v_mode == KVQ_MODE_FP4) {
+    if (c->rot_per_head) return KVQ_ERR_INVALID_ARG;  // the FP4 latent is not rotated
     if (c->k_mode != KVQ_MODE_FP4 || c->v_mode != KVQ_MODE_FP4) return KVQ_ERR_INVALID_ARG;
     if (c->n_kv_heads != 1) return KVQ_ERR_INVALID_ARG;
     if (c->latent_dim <= 0 || c->rope_dim < 0) return KVQ_ERR_INVALID_ARG;
@@ -117,7 +119,7 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
       P.k.order = kOrderOctet;
     const size_t m = (P.k.qjl || P.v.qjl) ? (size_t)c->qjl_dim : 0;
     P.signs_off = off;
-    off = align_up(off + sizeof(float) * kHeadDim, kArenaAlign);
+    off = align_up(off + sizeof(float) * kHeadDim * (c->rot_per_head ? c->n_kv_heads : 1), kArenaAlign);
     P.S_off = off;
     off = align_up(off + sizeof(float) * m * kHeadDim, kArenaAlign);
     P.St_off = off;
@@ -135,6 +137,13 @@ int device_sms() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   return sms > 0 ? sms : 148;
+}
+
+// Calls that launch work must run with the cache's device current: its arena, tables and the
+// kernels' launches all belong to that device.
+bool on_cache_device(const kvq_cache* c) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == c->device;
 }
 
 int part_stride(const kvq_cache* c) {
@@ -198,12 +207,16 @@ float default_scale(const kvq_cfg& cfg) {
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
+thread_local uint64_t t_launches = 0;  // this thread's successful launches (a call's own kernels)
 }  // namespace
 
 namespace kvq {
 cudaError_t launched() {
   const cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e == cudaSuccess) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    ++t_launches;
+  }
   return e;
 }
 }  // namespace kvq
@@ -261,11 +274,22 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
   const Plan P = plan_layout(cfg, batch, capacity);
   if (dev_bytes < P.total) return KVQ_ERR_WORKSPACE;
   const bool need_sketch = !P.fp4_mode && (P.k.qjl || P.v.qjl);
-  if (!P.fp4_mode && !rot_signs) return KVQ_ERR_INVALID_ARG;
-  if (need_sketch && !qjl_matrix) return KVQ_ERR_INVALID_ARG;
-  if (!P.fp4_mode)
-    for (int i = 0; i < kHeadDim; ++i)
-      if (rot_signs[i] != 1 && rot_signs[i] != -1) return KVQ_ERR_INVALID_ARG;
+  const int n_signs = P.fp4_mode ? 0 : kHeadDim * (cfg->rot_per_head ? cfg->n_kv_heads : 1);
+  // the method's random draws: the caller's arrays, else the configuration's seeds
+  std::vector<int8_t> drawn_signs;
+  std::vector<float> drawn_S;
+  if (!P.fp4_mode && !rot_signs) {
+    drawn_signs.resize(n_signs);
+    if (kvq_draw_rotation_signs(cfg->rot_seed, n_signs, drawn_signs.data()) != KVQ_OK) return KVQ_ERR_INVALID_ARG;
+    rot_signs = drawn_signs.data();
+  }
+  if (need_sketch && !qjl_matrix) {
+    drawn_S.resize((size_t)cfg->qjl_dim * kHeadDim);
+    if (kvq_draw_qjl_matrix(cfg->qjl_seed, cfg->qjl_dim, kHeadDim, drawn_S.data()) != KVQ_OK) return KVQ_ERR_INVALID_ARG;
+    qjl_matrix = drawn_S.data();
+  }
+  for (int i = 0; i < n_signs; ++i)
+    if (rot_signs[i] != 1 && rot_signs[i] != -1) return KVQ_ERR_INVALID_ARG;
 
   kvq_cache* c = new (std::nothrow) kvq_cache();
   if (!c) return KVQ_ERR_INVALID_ARG;
@@ -287,6 +311,11 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
   c->v_region = P.v_off;
   c->lens.assign(batch, 0);
   c->sms = device_sms();
+  if (cudaGetDevice(&c->device) != cudaSuccess) {
+    delete c;
+    return KVQ_ERR_CUDA;
+  }
+  c->signs_stride = cfg->rot_per_head ? kHeadDim : 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(c->d_lens, 0, sizeof(int) * ((size_t)batch + kStatusWords), s) != cudaSuccess) {
     delete c;
@@ -297,10 +326,10 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
     c->d_S = reinterpret_cast<float*>(c->dev + P.S_off);
     c->d_St = reinterpret_cast<float*>(c->dev + P.St_off);
     const size_t m = need_sketch ? (size_t)cfg->qjl_dim : 0;
-    c->h_tables.resize(kHeadDim + 2 * m * kHeadDim);
+    c->h_tables.resize(n_signs + 2 * m * kHeadDim);
     float* hs = c->h_tables.data();
-    for (int i = 0; i < kHeadDim; ++i) hs[i] = (float)rot_signs[i];
-    float* hS = hs + kHeadDim;
+    for (int i = 0; i < n_signs; ++i) hs[i] = (float)rot_signs[i];
+    float* hS = hs + n_signs;
     float* hSt = hS + m * kHeadDim;
     for (size_t j = 0; j < m; ++j)
       for (int i = 0; i < kHeadDim; ++i) {
@@ -309,7 +338,7 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
       }
     // Synchronous copies: the tables are tiny and this keeps the staging buffer's lifetime
     // trivially safe.
-    if (cudaMemcpy(c->d_signs, hs, sizeof(float) * kHeadDim, cudaMemcpyHostToDevice) != cudaSuccess ||
+    if (cudaMemcpy(c->d_signs, hs, sizeof(float) * n_signs, cudaMemcpyHostToDevice) != cudaSuccess ||
         (m && cudaMemcpy(c->d_S, hS, sizeof(float) * m * kHeadDim, cudaMemcpyHostToDevice) != cudaSuccess) ||
         (m && cudaMemcpy(c->d_St, hSt, sizeof(float) * m * kHeadDim, cudaMemcpyHostToDevice) != cudaSuccess)) {
       delete c;
@@ -344,6 +373,7 @@ void fill_quantize(QuantizeParams& p, const kvq_cache* c, const void* K, const v
   p.side[1] = c->v;
   p.fp4 = c->fp4;
   p.signs = c->d_signs;
+  p.signs_stride = c->signs_stride;
   p.St = c->d_St;
   p.lens = c->d_lens;
   p.err = c->d_status;
@@ -367,6 +397,7 @@ kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dt
   if (!aligned16(K) || !aligned16(V)) return KVQ_ERR_ALIGNMENT;
   if (!seq_ids && n_seq != c->batch) return KVQ_ERR_INVALID_ARG;
   if (n_seq > c->batch) return KVQ_ERR_INVALID_ARG;
+  if (!on_cache_device(c)) return KVQ_ERR_INVALID_ARG;
   std::vector<char> seen(c->batch, 0);
   for (int i = 0; i < n_seq; ++i) {
     const int sid = seq_ids ? seq_ids[i] : i;
@@ -404,6 +435,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   if (!c || !q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
   if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
+  if (!on_cache_device(c)) return KVQ_ERR_INVALID_ARG;
   int max_len = 0;
   for (int v : c->lens) max_len = std::max(max_len, v);
   const int pairs = decode_rows(c);
@@ -457,6 +489,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.k = c->k;
   p.v = c->v;
   p.signs = c->d_signs;
+  p.signs_stride = c->signs_stride;
   p.S = c->d_S;
   p.St = c->d_St;
   p.logit_scale = default_scale(c->cfg) * log2e;
@@ -491,6 +524,7 @@ kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const voi
   if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(K) || !aligned16(V) || !aligned16(q) || !aligned16(out) || !aligned16(workspace))
     return KVQ_ERR_ALIGNMENT;
+  if (!on_cache_device(c)) return KVQ_ERR_INVALID_ARG;
   // everything both halves check, with the lengths after the append, before anything is written
   int max_len = 0;
   for (int v : c->lens) {
@@ -510,7 +544,13 @@ kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const voi
   QuantizeParams qp;
   fill_quantize(qp, c, K, V, dtype, 1, nullptr, 0, c->batch);
   for (int i = 0; i < c->batch; ++i) c->lens[i] += 1;  // the plan of the decode sees the new lengths
-  return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles, nullptr, &qp);
+  const uint64_t launches0 = t_launches;
+  const kvq_status st = decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles, nullptr, &qp);
+  // The append is the step's first kernel: if nothing was launched, nothing was appended and the
+  // host lengths go back. (A failure of a later kernel leaves the append enqueued.)
+  if (st != KVQ_OK && t_launches == launches0)
+    for (int i = 0; i < c->batch; ++i) c->lens[i] -= 1;
+  return st;
 }
 
 }  // extern "C"
@@ -752,9 +792,12 @@ kvq_status kvq_debug_quantize_rotated(const kvq_cache* c, const float* u, int32_
 //
 // The array is file-scope device memory: every GPU that loads this library holds its 16 MiB
 // until the process exits. Its address is a device address only on the device side; host code
-// gets it once per device from cudaGetSymbolAddress (done by the first call on that device).
-// Nothing in it has to start at zero: each call writes every partial slot it later reads. All
-// calls share it, so two calls that overlap on the GPU (e.g. on different streams) race.
+// gets it from cudaGetSymbolAddress with the cache's device current. A call outside stream
+// capture looks the address up again (a context that was reset and re-created reloads the module,
+// and the array may move); a call on a capturing stream, which may not trigger a module load, uses
+// the address the last uncaptured call on that device found. Nothing in it has to start at zero:
+// each call writes every partial slot it later reads. All calls share it, so two calls that
+// overlap on the GPU (e.g. on different streams) race.
 // ---------------------------------------------------------------------------------------------
 
 namespace {
@@ -767,15 +810,19 @@ void* g_static_scratch_ptr[kMaxDevices] = {};
 static __device__ __align__(256) float g_kvq_static_scratch[kStaticScratchBytes / sizeof(float)];
 
 namespace {
-kvq_status static_scratch_for_current_device(void** out) {
+kvq_status static_scratch_for_current_device(cudaStream_t s, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return KVQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (!g_static_scratch_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_kvq_static_scratch) != cudaSuccess || !p) return KVQ_ERR_CUDA;
     g_static_scratch_ptr[dev] = p;
+  } else if (!g_static_scratch_ptr[dev]) {
+    return KVQ_ERR_CUDA;  // no uncaptured call has looked the address up on this device yet
   }
   *out = g_static_scratch_ptr[dev];
   return KVQ_OK;
@@ -785,6 +832,7 @@ kvq_status static_scratch_for_current_device(void** out) {
 extern "C" kvq_status kvq_decode_attention_static(const kvq_cache* c, const void* q, kvq_dtype dtype,
                                                   float* out, void* stream) {
   if (!c || !q || !out) return KVQ_ERR_INVALID_ARG;
+  if (!on_cache_device(c)) return KVQ_ERR_INVALID_ARG;
   int max_len = 0;
   for (int v : c->lens) max_len = std::max(max_len, v);
   const int pairs = decode_rows(c);
@@ -793,7 +841,7 @@ extern "C" kvq_status kvq_decode_attention_static(const kvq_cache* c, const void
               &splits, &chunk);
   if (workspace_for(c, splits) > kStaticScratchBytes) return KVQ_ERR_WORKSPACE;
   void* scratch = nullptr;
-  const kvq_status st = static_scratch_for_current_device(&scratch);
+  const kvq_status st = static_scratch_for_current_device(reinterpret_cast<cudaStream_t>(stream), &scratch);
   if (st != KVQ_OK) return st;
   return kvq_decode_attention(c, q, dtype, out, scratch, kStaticScratchBytes, stream);
 }

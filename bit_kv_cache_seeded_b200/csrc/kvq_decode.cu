@@ -93,7 +93,7 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
   // logit (base 2) = n_t * ( <q_s, c> + gamma_t <s_s, z> ),  q_s = R q * scale*log2e/sqrt(d)
   const float qcoef = inv_sqrt_d * p.logit_scale * inv_sqrt_d;
   for (int h = warp; h < G; h += kWarps)
-    rotate_query(p.q, ((size_t)b * p.Hq + hk * G + h) * kHeadDim, p.bf16, p.signs, qcoef, q_s[h]);
+    rotate_query(p.q, ((size_t)b * p.Hq + hk * G + h) * kHeadDim, p.bf16, p.signs + hk * p.signs_stride, qcoef, q_s[h]);
   __syncthreads();
   if (KQ) {
     const float kappa = 1.2533141373155003f / (float)p.k.m;  // sqrt(pi/2)/m
@@ -275,7 +275,7 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
   }
   float sg[4];  // the output rotation's signs and scale (warps 0..G-1), fetched while waiting
 #pragma unroll
-  for (int k = 0; k < 4; ++k) sg[k] = warp < G ? p.signs[32 * k + lane] * 0.08838834764831845f : 0.f;
+  for (int k = 0; k < 4; ++k) sg[k] = warp < G ? p.signs[hk * p.signs_stride + 32 * k + lane] * 0.08838834764831845f : 0.f;
   // Launched as a programmatic dependent of the decode kernel: S is staged above while that
   // grid finishes; its partials are read only after this wait.
   grid_dep_wait();

@@ -209,7 +209,7 @@ __device__ __forceinline__ void prep_block(const DecodeParams& p, int vk, int b)
   if (h0 < G) {
     const size_t qb = ((size_t)b * p.Hq + h_first + h0) * kHeadDim;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) u[k] = load_q(p.q, qb + 32 * k + lane, p.bf16) * p.signs[32 * k + lane];
+    for (int k = 0; k < 4; ++k) u[k] = load_q(p.q, qb + 32 * k + lane, p.bf16) * p.signs[hk * p.signs_stride + 32 * k + lane];
   }
   const float qcoef = kInvSqrtD * p.logit_scale * kInvSqrtD;
   if (h0 < G) {

@@ -64,7 +64,8 @@ struct QuantizeParams {
   int tiles_per_seq;
   SideLayout side[2];
   Fp4Layout fp4;
-  const float* signs;    // [d] +-1
+  const float* signs;    // [d] +-1 (per-head rotation: [heads][d])
+  int signs_stride;      // 0: one diagonal for every head; d: head h reads signs + h * d
   const float* St;       // [d][m] transposed sketch matrix
   int* lens;             // device lengths, set to pos + n_new
   int skip_rotation;     // debug entry: src[0] already rotated and normalised (fp32)
@@ -91,7 +92,8 @@ struct DecodeParams {
   const char* vreg;
   int tiles_per_seq;
   SideLayout k, v;
-  const float* signs;     // [d]
+  const float* signs;     // [d] (per-head rotation: [Hkv][d])
+  int signs_stride;       // 0: one diagonal for every kv-head; d: kv-head hk reads signs + hk * d
   const float* S;         // [m][d]
   const float* St;        // [d][m]
   float logit_scale;      // softmax_scale * log2(e)
@@ -158,6 +160,8 @@ void lloyd_max_f32(int bits, float* centroids, float* thresholds);
 struct kvq_cache {
   kvq_cfg cfg;
   int batch = 0, capacity = 0, tiles_per_seq = 0, sms = 148;
+  int signs_stride = 0;     // 0, or kHeadDim when every kv-head has its own rotation diagonal
+  int device = -1;          // the CUDA device whose memory holds the arena (current at init)
   char* dev = nullptr;
   size_t dev_bytes = 0;
   int* d_lens = nullptr;

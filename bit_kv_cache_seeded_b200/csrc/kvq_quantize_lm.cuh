@@ -84,8 +84,10 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
 #pragma unroll
     for (int k = 0; k < 4; ++k) u_first[k] = load_elem(p.src[side], (size_t)first * kHeadDim + 32 * k + lane, p.bf16);
   float sg[4];  // rotation signs (the debug entry's inputs are already rotated: none read)
+  int sg_head = 0;  // the head whose diagonal sg holds (per-head rotation)
+  if (first < total) sg_head = (int)((first / p.n_new) % p.heads);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) sg[k] = p.skip_rotation ? 1.f : p.signs[32 * k + lane];
+  for (int k = 0; k < 4; ++k) sg[k] = p.skip_rotation ? 1.f : p.signs[sg_head * p.signs_stride + 32 * k + lane];
   // the table in registers: thresholds (unused ones +inf), centroid c held by lane c % 8
   float thr[7];
 #pragma unroll
@@ -102,6 +104,11 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
 #pragma unroll
     for (int k = 0; k < 4; ++k) u[k] = (vec == first) ? u_first[k] : load_elem(p.src[side], base + 32 * k + lane, p.bf16);
 
+    if (p.signs_stride && h != sg_head && !p.skip_rotation) {  // per-head rotation: this head's diagonal
+      sg_head = h;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sg[k] = p.signs[h * p.signs_stride + 32 * k + lane];
+    }
     float n = 0.f;
     if (!p.skip_rotation) {
       n = sqrtf(warp_sum(u[0] * u[0] + u[1] * u[1] + u[2] * u[2] + u[3] * u[3]));

@@ -23,6 +23,9 @@
  * Conventions for every call:
  *  - Calls return a kvq_status and never abort or throw. Arguments are validated before any
  *    launch; a call that fails validation writes nothing.
+ *  - A cache belongs to the CUDA device that was current when kvq_cache_init ran; calls that
+ *    launch work on it return KVQ_ERR_INVALID_ARG, launching nothing, unless that device is
+ *    current.
  *  - "stream" is a cudaStream_t passed as void* (NULL = legacy default stream). Calls that
  *    launch work are asynchronous on that stream.
  *  - Device pointers must be 16-byte aligned (KVQ_ERR_ALIGNMENT otherwise); the cache arena
@@ -80,9 +83,29 @@ typedef struct {
   float softmax_scale;  /* 0 => 1/sqrt(dim of q.k): head_dim, or latent_dim + rope_dim */
   int32_t latent_dim;   /* FP4 only: 512 */
   int32_t rope_dim;     /* FP4 only: 64 */
+  int32_t rot_per_head; /* LM/SIGN1: 0 = one diagonal D for every KV head; 1 = KV head h has its own
+                           D_h (draws h*head_dim .. h*head_dim + head_dim - 1 of rot_seed). FP4: 0 */
+  uint64_t rot_seed;    /* seed of the rotation's +-1 diagonal (used when kvq_cache_init gets no
+                           rot_signs): see kvq_draw_rotation_signs */
+  uint64_t qjl_seed;    /* seed of the sketch matrix S (used when kvq_cache_init gets no qjl_matrix):
+                           see kvq_draw_qjl_matrix */
 } kvq_cfg;
 
 typedef struct kvq_cache kvq_cache; /* opaque host object */
+
+/* The seeded draws, host-only (they fix what kvq_cache_init draws when given no arrays). With the
+ * counter-based generator
+ *   mix(z)  = z ^= z >> 30; z *= 0xBF58476D1CE4E5B9; z ^= z >> 27; z *= 0x94D049BB133111EB;
+ *             z ^= z >> 31                                   (splitmix64 finaliser, mod 2^64)
+ *   h(s, i) = mix(s + (i + 1) * 0x9E3779B97F4A7C15)            (draw i of stream s)
+ *   U(s, i) = (h(s, i) >> 11) * 2^-53                          (uniform in [0, 1))
+ * kvq_draw_rotation_signs writes out[i] = -1 if h(seed, i) is odd, else +1, for i < n.
+ * kvq_draw_qjl_matrix writes the row-major [m][d] matrix with entry k = j*d + i equal to the fp32
+ * rounding of the Box-Muller normal sqrt(-2 log1p(-U(seed, 2k))) cos(2 pi U(seed, 2k + 1)),
+ * computed in double precision with the C library's log1p, sqrt and cos. KVQ_ERR_INVALID_ARG for a
+ * null pointer or a non-positive size. */
+kvq_status kvq_draw_rotation_signs(uint64_t seed, int32_t n, int8_t* out);
+kvq_status kvq_draw_qjl_matrix(uint64_t seed, int32_t m, int32_t d, float* out);
 
 /* Human-readable name of a status code (static string). */
 const char* kvq_status_str(kvq_status s);
@@ -96,11 +119,17 @@ kvq_status kvq_cache_bytes(const kvq_cfg* cfg, int32_t batch, int32_t capacity, 
 kvq_status kvq_packed_bytes_per_token(const kvq_cfg* cfg, size_t* bytes);
 
 /* Create a cache inside caller-owned device memory `dev_mem` (dev_bytes >= kvq_cache_bytes).
- * All sequences start empty. rot_signs: host [head_dim] of +1/-1 (the diagonal D), required
- * for LM/SIGN1 modes. qjl_matrix: host [qjl_dim, head_dim] fp32, row-major, i.i.d. N(0,1)
- * entries (the sketch matrix S), required when a side is LM_QJL. Both are copied; the
- * library keeps no pointer to them after the call returns. The copies into dev_mem are
- * enqueued on `stream`. On success *out owns a host object to free with kvq_cache_destroy. */
+ * All sequences start empty. The method's two random draws ("TurboQuant vs OSCAR vs EpiCache",
+ * section "Quantization frontiers: TurboQuant and OSCAR": a data-oblivious random rotation, and a
+ * Gaussian matrix for the 1-bit QJL sketch) come from the configuration's seeds, or from the
+ * caller:
+ *   rot_signs: NULL = draw D from cfg->rot_seed (kvq_draw_rotation_signs); else host +1/-1 values,
+ *              [head_dim] or, with cfg->rot_per_head, [n_kv_heads][head_dim]. LM/SIGN1 modes only.
+ *   qjl_matrix: NULL = draw S from cfg->qjl_seed (kvq_draw_qjl_matrix); else host
+ *              [qjl_dim, head_dim] fp32, row-major. Used when a side is LM_QJL.
+ * Given arrays are copied; the library keeps no pointer to them after the call returns. The
+ * copies into dev_mem are enqueued on `stream`. On success *out owns a host object to free with
+ * kvq_cache_destroy. */
 kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_t capacity,
                           void* dev_mem, size_t dev_bytes, const int8_t* rot_signs,
                           const float* qjl_matrix, void* stream);
@@ -109,7 +138,9 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
  * packed codes + norms + sketch"). K, V: device tensors in the layout above. seq_ids: host
  * array of n_seq distinct sequence indices, or NULL for all sequences in order (then n_seq
  * must equal batch). Fails with KVQ_ERR_CAPACITY, writing nothing, if any listed sequence
- * would exceed the capacity. n_new == 0 or n_seq == 0 is a no-op. */
+ * would exceed the capacity. n_new == 0 or n_seq == 0 is a no-op. The listed sequences are
+ * appended by one launch per 1024 of them; KVQ_ERR_CUDA means one of those launches failed: the
+ * sequences of the launches before it were appended, and kvq_cache_lengths counts exactly those. */
 kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dtype,
                         int32_t n_new, const int32_t* seq_ids, int32_t n_seq, void* stream);
 
@@ -128,8 +159,10 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
  * and all sequences) and run kvq_decode_attention with q over the caches that now include it.
  * The result equals the two calls in sequence; fusing them lets the query prep run while the
  * append is still in flight (on the tensor-core path). Everything is validated (capacity,
- * alignment, workspace for the lengths after the append) before anything is written; on an
- * error nothing is appended. */
+ * alignment, workspace for the lengths after the append) before anything is written; a call that
+ * fails validation appends nothing. KVQ_ERR_CUDA: if the append's launch failed, nothing was
+ * appended and the lengths are unchanged; if a later kernel's launch failed, the append is
+ * enqueued and the lengths include it. */
 kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
                            float* out, void* workspace, size_t ws_bytes, void* stream);
 
@@ -164,9 +197,12 @@ kvq_status kvq_decode_step_host(kvq_cache* c, const void* K, const void* V, cons
  * the process exits. The paper has no counterpart to this call; it is an interface
  * convenience. Returns KVQ_ERR_WORKSPACE, launching nothing, when the partials of this cache
  * (batch x n_q_heads x splits x (2 + head_dim [+ qjl_dim]) floats; FP4: 2 + latent_dim) would
- * exceed 16 MiB. The first call on a device looks up the array's device address (once per
- * device); make that first call before any stream capture. All calls share the array, so calls
- * that overlap on the GPU (different streams, or threads) race: order them on one stream. */
+ * exceed 16 MiB. A call looks up the array's device address on the cache's device (outside stream
+ * capture, on every call, so that a device reset and re-created context are followed); a call on
+ * a capturing stream reuses the address found by the last uncaptured call on that device, so
+ * make the first call on a device before any stream capture (otherwise KVQ_ERR_CUDA). All calls
+ * share the array, so calls that overlap on the GPU (different streams, or threads) race: order
+ * them on one stream. */
 kvq_status kvq_decode_attention_static(const kvq_cache* c, const void* q, kvq_dtype dtype,
                                        float* out, void* stream);
 

@@ -6,7 +6,8 @@ Generator definition (fixed here, used by everything):
   h(s, i)  = mix(s + (i + 1) * 0x9E3779B97F4A7C15)           (the i-th draw of stream s)
   U(s, i)  = (h(s, i) >> 11) * 2^-53                           (uniform in [0, 1))
 
-Rotation signs: D_i = -1 if h(rot_seed, i) & 1 else +1, i < d.
+Rotation signs: D_i = -1 if h(rot_seed, i) & 1 else +1, i < d (per-head rotation: head h takes
+                i = h d .. h d + d - 1).
 QJL matrix:     S[j, i] = fp32( sqrt(-2 ln(1 - U(s, 2k))) cos(2 pi U(s, 2k + 1)) ), k = j d + i.
 """
 from __future__ import annotations
@@ -36,6 +37,12 @@ def rotation_signs(rot_seed: int, d: int) -> np.ndarray:
     """+-1 diagonal of the randomized Hadamard rotation, int8 [d]."""
     bit = splitmix64(rot_seed, np.arange(d, dtype=np.uint64)) & np.uint64(1)
     return np.where(bit == 1, -1, 1).astype(np.int8)
+
+
+def rotation_signs_per_head(rot_seed: int, heads: int, d: int) -> np.ndarray:
+    """One +-1 diagonal per KV head, int8 [heads, d]: head h takes draws h*d .. h*d + d - 1 of the
+    same stream (head 0's diagonal is rotation_signs(rot_seed, d))."""
+    return rotation_signs(rot_seed, heads * d).reshape(heads, d)
 
 
 def qjl_matrix(qjl_seed: int, m: int, d: int) -> np.ndarray:

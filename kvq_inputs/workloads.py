@@ -27,7 +27,7 @@ from dataclasses import dataclass, replace
 import numpy as np
 import torch
 
-from .rng import rotation_signs, qjl_matrix
+from .rng import rotation_signs, rotation_signs_per_head, qjl_matrix
 
 
 @dataclass(frozen=True)
@@ -50,6 +50,7 @@ class Workload:
     key_factor: float = 1.0    # outlier multiplier
     latent_dim: int = 0
     rope_dim: int = 0
+    rot_per_head: bool = False  # one rotation diagonal per KV head
 
     @property
     def data_seed(self) -> int:
@@ -110,8 +111,10 @@ def channel_scales(w: Workload, which: str) -> np.ndarray:
 
 
 def rotation_and_sketch(w: Workload):
-    """The method's random draws for this workload: (signs int8 [d], S float32 [m, d] or None)."""
-    signs = rotation_signs(w.rot_seed, w.head_dim)
+    """The method's random draws for this workload: (signs int8 [d] -- or [n_kv_heads, d] with a
+    per-head rotation --, S float32 [m, d] or None)."""
+    signs = (rotation_signs_per_head(w.rot_seed, w.n_kv_heads, w.head_dim) if w.rot_per_head
+             else rotation_signs(w.rot_seed, w.head_dim))
     S = qjl_matrix(w.qjl_seed, w.qjl_dim, w.head_dim) if w.qjl_dim else None
     return signs, S
 

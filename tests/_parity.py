@@ -79,6 +79,8 @@ def pair_reference(w, arena, info, b, hk, T, K, V, q, signs, S, stats):
     K, V: [T, d] fp64 inputs of that pair; q: [g, d] fp64 query heads of the group.
     """
     pair = b * w.n_kv_heads + hk
+    if np.ndim(signs) == 2:  # one rotation diagonal per kv-head
+        signs = signs[hk]
     kp, ks, kn, kg = side_fields(arena, info, 0, pair, T)
     vp, vs, vn, vg = side_fields(arena, info, 1, pair, T)
     kq = S if ks is not None else None

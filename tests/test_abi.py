@@ -148,7 +148,21 @@ int main(void) {
   if (kvq_lloyd_max_table(4, c, t) != KVQ_ERR_INVALID_ARG) return 2;
   if (kvq_packed_bytes_per_token(&cfg, &bytes) != KVQ_OK) return 3;
   if (kvq_decode_step_host(NULL, NULL, NULL, NULL, KVQ_BF16, NULL, NULL, 0, NULL, 0, NULL) != KVQ_ERR_INVALID_ARG) return 4;
-  printf("%s|%zu|%.6f\n", kvq_status_str(KVQ_ERR_CAPACITY), bytes, c[3]);
+  /* the seeded draws a cache makes from cfg.rot_seed / cfg.qjl_seed when given no arrays */
+  cfg.rot_seed = 0x5EED00A4ull; cfg.qjl_seed = 0x5EED005Bull;
+  {
+    static int8_t d[128];
+    static float s[128 * 128];
+    long sum = 0;
+    double ssum = 0.0;
+    int i;
+    if (kvq_draw_rotation_signs(cfg.rot_seed, 128, d) != KVQ_OK) return 5;
+    if (kvq_draw_qjl_matrix(cfg.qjl_seed, 128, 128, s) != KVQ_OK) return 6;
+    if (kvq_draw_qjl_matrix(cfg.qjl_seed, 0, 128, s) != KVQ_ERR_INVALID_ARG) return 7;
+    for (i = 0; i < 128; ++i) sum += (long)d[i] * (i + 1);
+    for (i = 0; i < 128 * 128; ++i) ssum += (double)s[i] * (double)((i % 97) + 1);
+    printf("%s|%zu|%.6f|%ld|%.17g|%.9g\n", kvq_status_str(KVQ_ERR_CAPACITY), bytes, c[3], sum, ssum, (double)s[12345]);
+  }
   return 0;
 }
 """
@@ -170,7 +184,13 @@ def test_plain_c_client_links_and_runs(lib, tmp_path):
         pytest.skip("gcc not available")
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert out.returncode == 0, out.stdout + out.stderr
-    name, nbytes, c3 = out.stdout.strip().split("|")
+    name, nbytes, c3, dsum, ssum, s12345 = out.stdout.strip().split("|")
+    from kvq_inputs import rotation_signs, qjl_matrix
+    d = rotation_signs(0x5EED00A4, 128).astype(np.int64)
+    S = qjl_matrix(0x5EED005B, 128, 128).astype(np.float64).reshape(-1)
+    assert int(dsum) == int(np.sum(d * np.arange(1, 129)))
+    assert np.float32(float(s12345)) == np.float32(S[12345])
+    assert abs(float(ssum) - float(np.sum(S * ((np.arange(S.size) % 97) + 1)))) < 1e-6 * np.sum(np.abs(S)) * 97
     cfg = kvq.make_cfg(head_dim=128, n_q_heads=32, n_kv_heads=8, k_bits=2, v_bits=2, qjl_dim=128)
     assert name == kvq.kvq_status_str(3)
     assert int(nbytes) == kvq.kvq_packed_bytes_per_token(cfg)
@@ -203,3 +223,32 @@ def test_binding_refuses_host_tensors_and_wrong_shapes(lib):
         with pytest.raises(ValueError, match="CUDA tensor"):
             call()
     assert kvq.kvq_kernel_launches() == n0
+
+
+@pytest.mark.parametrize("seed", [0, 1, 0x5EED00A5, 0x5EED005A, 0xFFFFFFFFFFFFFFFF, 0x0123456789ABCDEF])
+def test_seeded_draws_are_the_generator_bit_for_bit(lib, seed):
+    """The library's host draws (what kvq_cache_init uses when it gets seeds and no arrays) equal
+    the seeded generator's, bit for bit: rotation signs over several heads' worth of counters, and
+    the Box-Muller sketch matrix."""
+    from kvq_inputs import rotation_signs, qjl_matrix
+    from kvq_inputs.rng import rotation_signs_per_head
+    np.testing.assert_array_equal(kvq.kvq_draw_rotation_signs(seed, 1024), rotation_signs(seed, 1024))
+    np.testing.assert_array_equal(kvq.kvq_draw_rotation_signs(seed, 8 * 128).reshape(8, 128),
+                                  rotation_signs_per_head(seed, 8, 128))
+    a = kvq.kvq_draw_qjl_matrix(seed, 128, 128)
+    b = qjl_matrix(seed, 128, 128)
+    np.testing.assert_array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def test_cfg_struct_layout_matches_header(lib):
+    """The ctypes mirror of kvq_cfg has the C layout: 12 int32-sized fields, then two uint64 seeds."""
+    import ctypes
+    assert ctypes.sizeof(kvq.kvq_cfg) == 64
+    assert kvq.kvq_cfg.rot_seed.offset == 48 and kvq.kvq_cfg.qjl_seed.offset == 56
+    cfg = kvq.make_cfg(rot_per_head=2)
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_cache_bytes(cfg, 1, 32)
+    fp4 = kvq.make_cfg(head_dim=512, n_q_heads=64, k_mode="fp4", v_mode="fp4", k_bits=4, v_bits=4, qjl_dim=0,
+                       latent_dim=512, rope_dim=64, rot_per_head=1)
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_cache_bytes(fp4, 1, 32)

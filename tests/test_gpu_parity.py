@@ -424,3 +424,36 @@ def test_capacity_overflow_writes_nothing():
         kvq.kvq_decode_attention(cache.handle, data["q"], torch.empty(2, 32, 128, device=DEV), small)
     assert e.value.status == 5
     cache.close()
+
+
+# ---------------------------------------------------------------- seeded draws inside the library
+
+def test_seeded_cache_equals_cache_from_explicit_tables():
+    """A cache given only the configuration's seeds draws the same rotation signs and sketch matrix
+    as the seeded generator: both arenas are byte-identical after the same appends, and decode gives
+    identical outputs."""
+    w = WORKLOADS["llama8b"].with_(batch=2)
+    data = generate(w, DEV, seqs=range(2), ctx=200)
+    signs, S = rotation_and_sketch(w)
+    explicit = kvq.KvqCache(kvq.cfg_for_workload(w), 2, 256, signs, S)
+    seeded = kvq.KvqCache(kvq.cfg_for_workload(w), 2, 256)  # no arrays: drawn from cfg seeds
+    for c in (explicit, seeded):
+        c.quantize(data["k"], data["v"])
+    a = explicit.decode(data["q"])
+    b = seeded.decode(data["q"])
+    torch.cuda.synchronize()
+    assert torch.equal(explicit.arena, seeded.arena)
+    assert torch.equal(a, b)
+    explicit.close()
+    seeded.close()
+
+
+def test_per_head_rotation_parity():
+    """Every kv-head with its own rotation diagonal (drawn from the same seed stream): codes and
+    attention against the oracle, which rotates each head with that head's diagonal."""
+    w = WORKLOADS["llama8b"].with_(rot_per_head=True)
+    signs, _ = rotation_and_sketch(w)
+    assert signs.shape == (w.n_kv_heads, w.head_dim) and not np.all(signs[0] == signs[1])
+    run_small("llama8b", 2, [300, 97], seed_appends=2, w=w)
+    w70 = WORKLOADS["llama70b"].with_(rot_per_head=True)
+    run_small("llama70b", 1, [260], w=w70)

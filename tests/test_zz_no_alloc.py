@@ -46,3 +46,24 @@ def test_static_scratch_decode_matches_workspace_decode():
         err = np.max(np.abs(o - r), axis=-1) / np.max(np.abs(r), axis=-1)
         assert np.all(np.isfinite(o)) and np.all(err <= REL_TOL), err.max()
     cache.close()
+
+
+def test_static_scratch_refuses_partials_beyond_its_size():
+    """A cache whose split partials cannot fit the fixed array (batch 512, 64 query heads: 512 x 64 x
+    (2 + 128) floats already at one split, about 17 MB) is refused with KVQ_ERR_WORKSPACE, and the
+    output buffer is left untouched."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    lib = kvq.load()
+    w = WORKLOADS["llama70b"].with_(batch=512)
+    signs, S = rotation_and_sketch(w)
+    cache = kvq.KvqCache(kvq.cfg_for_workload(w), 512, 64, signs, S)
+    q = torch.randn(512, 64, 128, device="cuda").to(torch.bfloat16)
+    out = torch.full((512, 64, 128), 7.0, device="cuda")
+    st = lib.kvq_decode_attention_static(cache.handle, ctypes.c_void_p(q.data_ptr()), 1,
+                                         ctypes.c_void_p(out.data_ptr()),
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert st == 5, kvq.kvq_status_str(st)  # KVQ_ERR_WORKSPACE
+    assert torch.all(out == 7.0)
+    cache.close()
