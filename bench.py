@@ -54,7 +54,9 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="llama8b", choices=list(WORKLOADS))
+    ap.add_argument("--workload", default="llama70b", choices=list(WORKLOADS),
+                    help="headline workload (default: the largest single-GPU configuration, 1.98 GB per step)")
+    ap.add_argument("--only", action="store_true", help="time the headline workload alone")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ctx", type=int, default=0,
@@ -62,16 +64,21 @@ def parse():
     return ap.parse_args()
 
 
-# DRAM bytes (read + write) of one launch of the split decode kernel, from an ncu capture of the
-# workload named here. The record only counts while the kernel's sources are the ones captured
-# (their SHA-256 below); after any change the bench reports null until a new capture.
-TRAFFIC = {
-    "llama8b": {"kernel": "decode_lm_mma<4, 2, 1, 2, 1>", "dram_bytes": 113382912,  # 109.512704 + 3.870208 MB
-                "profile": "profiles/decode_lm_mma_llama8b.md",
-                "sources_sha256": "a506daec4d4b17781042b53742a2e8ff7d574e27935e60a922a432e57279fa2f"},
+# The dominant (split decode) kernel of each workload.
+KERNEL_NAMES = {
+    "tiny": "decode_lm_mma<1, 2, 1, 2, 1>", "llama8b": "decode_lm_mma<4, 2, 1, 2, 1>",
+    "llama70b": "decode_lm_mma<4, 3, 1, 3, 0>", "onebit": "decode_lm_mma<4, 1, 0, 1, 0>",
+    "mla_fp4": "decode_mla_umma",
 }
+EXTRA_WORKLOADS = ("llama8b", "onebit", "mla_fp4", "llama70b")
+
+# DRAM bytes (read + write) of one launch of the split decode kernel, and the load efficiency of its
+# packed streams, from ncu captures (full size, or a smaller context scaled to the full launch by the
+# tokens processed). A record only counts while the kernel's sources are the ones captured (their
+# SHA-256 below); after any change the bench reports null until a new capture.
+TRAFFIC = {}
 TRAFFIC_SOURCES = ("bit_kv_cache_seeded_b200/csrc/kvq_decode_mma.cu", "bit_kv_cache_seeded_b200/csrc/kvq_async.cuh",
-                   "bit_kv_cache_seeded_b200/csrc/kvq_internal.h")
+                   "bit_kv_cache_seeded_b200/csrc/kvq_internal.h", "bit_kv_cache_seeded_b200/csrc/kvq_mla_umma.cu")
 
 
 def kernel_sources_sha():
@@ -87,7 +94,7 @@ def traffic_record(w):
     rec = TRAFFIC.get(w.name)
     if rec is None or rec["sources_sha256"] != kernel_sources_sha() or w.ctx != WORKLOADS[w.name].ctx:
         return None
-    return rec["dram_bytes"]
+    return rec
 
 
 def measured_peaks():
@@ -308,57 +315,73 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(args, world, rank, local):
-    import bit_kv_cache_seeded_b200 as kvq
-    kvq.load()
-    w = WORKLOADS[args.workload]
-    if args.ctx > 0:
-        w = w.with_(ctx=args.ctx)
-    dev = f"cuda:{local}"
-    torch.cuda.set_device(dev)
+def cpu_baseline(w, seconds):
+    """The oracle, as it stands, on a bounded sample of workload w, scaled to KV tokens/s."""
+    if w.k_mode == "fp4":
+        P, step_fn = oracle_prepare_fp4(w, FP4_SAMPLE_CTX), oracle_step_fp4
+        what = f"sequence 0, first {FP4_SAMPLE_CTX} of {w.ctx} tokens, all {w.n_q_heads} heads"
+    else:
+        pairs = 2
+        P, step_fn = oracle_prepare(w, pairs, w.ctx), oracle_step
+        what = f"{pairs} (sequence, kv-head) pairs at ctx {w.ctx} (of {w.batch * w.n_kv_heads} pairs per step)"
+    tot, toks_tot, reps = 0.0, 0.0, 0
+    while tot < seconds and reps < 200:
+        dt, toks = step_fn(P)
+        tot, toks_tot, reps = tot + dt, toks_tot + toks, reps + 1
+    return {"value": toks_tot / tot, "unit": "KV tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{reps} repetitions of one decode step over {what}, fp64 numpy"}
+
+
+def measure(kvq, w, args, world, dev):
+    """One workload: device-resident timed steps, per-kernel times, end-to-end steps through the
+    host-buffer call. Returns the fields of its JSON line (without cpu_baseline)."""
     stream = torch.cuda.current_stream()
     cfg = kvq.cfg_for_workload(w)
-    signs, S = (None, None) if w.k_mode == "fp4" else rotation_and_sketch(w)
     per_tok = kvq.kvq_packed_bytes_per_token(cfg)
     heads_kv = 1 if w.k_mode == "fp4" else w.n_kv_heads
     bytes_prefix = w.batch * heads_kv * w.ctx * per_tok
     replicas = max(2, math.ceil(2.5 * L2_BYTES / max(bytes_prefix, 1)))
     n_steps = args.warmup + args.steps
-    capacity = w.ctx + n_steps
+    n_e2e = args.steps
+    capacity = w.ctx + n_steps + n_e2e + 1
 
-    # Prefix of ctx - 1 tokens in every replica (identical content), built in sequence slices.
-    caches = [kvq.KvqCache(cfg, w.batch, capacity, signs, S, device=dev) for _ in range(replicas)]
+    # Prefix of ctx - 1 tokens in every replica (identical content), built in sequence slices. The
+    # caches draw their rotation signs and sketch matrix from the configuration's seeds.
+    caches = [kvq.KvqCache(cfg, w.batch, capacity, device=dev) for _ in range(replicas)]
     step_b = max(1, w.batch // 8)
     q = None
+    a_name, b_name = ("latent", "rope") if w.k_mode == "fp4" else ("k", "v")
+    q_ms = 0.0  # device time of the first replica's prefill appends (all sequences, ctx - 1 tokens)
     for b0 in range(0, w.batch, step_b):
         seqs = list(range(b0, min(w.batch, b0 + step_b)))
         d = generate(w, dev, seqs=seqs, ctx=w.ctx - 1)
-        a, bb = ("latent", "rope") if w.k_mode == "fp4" else ("k", "v")
-        for c in caches:
-            c.quantize(d[a], d[bb], seq_ids=seqs)
+        for ci, c in enumerate(caches):
+            if ci == 0:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            c.quantize(d[a_name], d[b_name], seq_ids=seqs)
+            if ci == 0:
+                e1.record(stream)
+                e1.synchronize()
+                q_ms += e0.elapsed_time(e1)
         q = d["q"] if q is None else torch.cat([q, d["q"]])
         del d
-    # New tokens of every step, resident in HBM.
+    n_vec = w.batch * (w.ctx - 1) * (1 if w.k_mode == "fp4" else 2 * w.n_kv_heads)
+    # New tokens of every step, resident in HBM (the e2e steps draw theirs on the host).
     news = []
     for s in range(n_steps):
         d = generate(w, dev, step=s)
-        news.append((d["latent"], d["rope"]) if w.k_mode == "fp4" else (d["k"], d["v"]))
+        news.append((d[a_name], d[b_name]))
     out = torch.empty((w.batch, w.n_q_heads, caches[0].out_dim), dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
-
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     lens0 = int(caches[0].lengths()[0])
 
-    def step(i, timed_idx=None):
+    def step(i):
         # one decode step through the fused entry: append the new token of every sequence and
         # attend (kvq_decode_step = kvq_quantize + kvq_decode_attention, prep overlapping the append)
         c = caches[i % replicas]
         k_new, v_new = news[i % len(news)]
-        if timed_idx is not None:
-            ev[timed_idx][0].record(stream)
         c.step(k_new, v_new, q, out)
-        if timed_idx is not None:
-            ev[timed_idx][1].record(stream)
 
     for i in range(args.warmup):
         step(i)
@@ -381,25 +404,13 @@ def run_ours(args, world, rank, local):
     launches = kvq.kvq_kernel_launches() - launches0
     barrier(world)
     torch.cuda.synchronize()
-    elapsed_ms = start.elapsed_time(end)
-    # one step alone, bracketed by its own events (a few steps after the timed ones)
-    n_ev = min(args.steps, 20)
-    base = args.warmup + args.steps
-    for j in range(n_ev):
-        if int(caches[(base + j) % replicas].lengths()[0]) >= capacity:
-            n_ev = j
-            break
-        step(base + j, j)
-    torch.cuda.synchronize()
-    dec_ms = sum(a.elapsed_time(b) for a, b in ev[:n_ev]) / max(1, n_ev)
-    elapsed_ms = max_over_ranks(elapsed_ms, world)
-    dec_ms = max_over_ranks(dec_ms, world)
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), world)
     ms_per_step = elapsed_ms / args.steps
     value = sum_over_ranks(kv_tokens, world) / (elapsed_ms / 1e3)
 
     # Per-kernel device times: the same decode through the measurement entry, which records CUDA
-    # events between its kernels (prep | split kernel | separate reduce, if any), rotating over the replicas.
-    n_k = min(args.steps, 50)
+    # events between its kernels (prep | split kernel | reduce), rotating over the replicas.
+    n_k = min(max(args.steps, 10), 50)
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_k)]
     torch.cuda.synchronize()
     for j in range(n_k):
@@ -410,82 +421,40 @@ def run_ours(args, world, rank, local):
     kern_ms = [max_over_ranks(x, world) for x in kern_ms]
     lens_k = sum(int(caches[j % replicas].lengths()[0]) for j in range(n_k)) / n_k
 
-    # End to end: host (pinned) inputs copied in, result copied out, every step. A step's new
-    # keys, values and query sit in one pinned buffer and cross in one copy; the device tensors
-    # handed to the library are views of one device buffer.
-    def as_bytes(t):
-        return t.contiguous().view(torch.uint8).reshape(-1)
-    parts = [news[0][0], news[0][1], q]
-    sizes = [x.numel() * x.element_size() for x in parts]
-    slots = [(n + 255) // 256 * 256 for n in sizes]  # each part 256-byte aligned in the buffer
-
-    def packed(a, b):
-        buf = torch.zeros(sum(slots), dtype=torch.uint8)
-        o = 0
-        for x, n, sl in zip((a, b, q), sizes, slots):
-            buf[o:o + n] = as_bytes(x.cpu())
-            o += sl
-        return buf.pin_memory()
-    host_in = [packed(a, b) for a, b in news[:args.steps]]
-    offs = [0, slots[0], slots[0] + slots[1]]
-    # Two sets of device buffers: the inputs of step j + 1 cross on a copy stream while step j
-    # runs, and step j's output comes back on the copy stream once step j is done.
-    dev_ins = [torch.empty(sum(slots), dtype=torch.uint8, device=q.device) for _ in range(2)]
-    views = [tuple(d[o:o + n].view(x.dtype).view(x.shape) for o, n, x in zip(offs, sizes, parts)) for d in dev_ins]
-    outs = [torch.empty_like(out) for _ in range(2)]
-    host_outs = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    host_out = host_outs[0]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    cs = torch.cuda.Stream(device=q.device)   # host -> device
-    cs_out = torch.cuda.Stream(device=q.device)  # device -> host (both directions at once)
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    e2e_caches = caches  # continue appending after the timed run (capacity allows warmup+steps)
+    # End to end through the library's host-buffer call (kvq_decode_step_host): every step's new
+    # keys, values and query start in pinned host memory and its output ends there. The library
+    # copies the inputs in on its own stream (overlapping the previous step) and the output out on
+    # another (overlapping the next step); each call records an event after its output copy, and
+    # the closing event waits for the last ones, so the timed region spans every copy.
+    host_news = []
+    for s in range(n_e2e):
+        k_new, v_new = news[s % len(news)]
+        host_news.append((k_new.cpu().pin_memory(), v_new.cpu().pin_memory()))
+    q_host = q.cpu().pin_memory()
+    host_outs = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    out_events = [torch.cuda.Event() for _ in range(n_e2e)]
+    for c in caches:  # one untimed call per cache: its staging buffer and copy streams now exist
+        c.step_host(*host_news[0], q_host, host_outs[0])
+    e2e_tokens = 0
     torch.cuda.synchronize()
     barrier(world)
+    torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    e2e_tokens = 0
-    n_e2e = min(args.steps, max(1, capacity - int(caches[0].lengths().max()) - 1) * replicas)
-    n_e2e = min(n_e2e, args.steps)
-
-    def copy_in(j):  # on the copy stream, once step j - 2 (same buffers) is done
-        with torch.cuda.stream(cs):
-            if j >= 2:
-                cs.wait_event(ev_done[j % 2])
-            dev_ins[j % 2].copy_(host_in[j], non_blocking=True)
-            ev_in[j % 2].record(cs)
-
     t0.record(stream)
-    cs.wait_stream(stream)
-    cs_out.wait_stream(stream)
-    copy_in(0)
     for j in range(n_e2e):
-        c = e2e_caches[j % replicas]
-        if int(c.lengths()[0]) >= capacity:
-            break
-        if j + 1 < n_e2e:
-            copy_in(j + 1)
-        stream.wait_event(ev_in[j % 2])
-        if j >= 2:
-            stream.wait_event(ev_out[j % 2])  # step j - 2's output has left outs[j % 2]
-        c.step(*views[j % 2], outs[j % 2])
-        ev_done[j % 2].record(stream)
-        with torch.cuda.stream(cs_out):
-            cs_out.wait_event(ev_done[j % 2])
-            host_outs[j % 2].copy_(outs[j % 2], non_blocking=True)
-            ev_out[j % 2].record(cs_out)
+        c = caches[j % replicas]
+        c.step_host(*host_news[j], q_host, host_outs[j % 2], out_event=out_events[j])
         e2e_tokens += w.batch * int(c.lengths()[0])
-    stream.wait_stream(cs)
-    stream.wait_stream(cs_out)
+    for e in out_events[-2:]:
+        stream.wait_event(e)
     t1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world)
-    e2e_steps = max(1, n_e2e)
     e2e_tokens = sum_over_ranks(e2e_tokens, world)
     e2e_value = e2e_tokens / (e2e_ms / 1e3) if e2e_ms > 0 else None
-    h2d = host_in[0].numel()
-    d2h = host_out.numel() * host_out.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in (*host_news[0], q_host))
+    d2h = host_outs[0].numel() * host_outs[0].element_size()
 
     peaks, peak_kind = measured_peaks()
     bytes_step = w.batch * heads_kv * (lens0 + 1) * per_tok  # packed bytes one decode call reads
@@ -504,49 +473,66 @@ def run_ours(args, world, rank, local):
         roof = {"bound": "hbm", "achieved": bytes_kernel / (kern_ms[1] / 1e3) / 1e9,
                 "peak": float(peaks["hbm_gbs"]), "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    tr = traffic_record(w)
     line = {
-        "metric": METRIC,
-        "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
+        "value": value, "ms_per_step": ms_per_step,
         # the contractions' operand / accumulation types: exact int8 tensor-core products with int32
         # sums and fp32 softmax (LM), f16/bf16 tcgen05 products with fp32 accumulators (FP4 latent)
         "dtype": "f16/f32" if w.k_mode == "fp4" else "s8/s32/f32",
-        "data": "synthetic",
         "config": workload_config(w, world),
         "l2_detail": f"{replicas} cache replicas x {bytes_prefix / 1e6:.1f} MB rotated per step",
         "hbm_gbs": achieved_call, "frac_of_8tbs": achieved_call / 8000.0,
-        "roofline": dict(roof, traffic=traffic_record(w), peak_kind=peak_kind,
-                         kernel="split decode kernel (decode_lm_mma / decode_mla_mma)",
-                         bytes_per_launch=bytes_kernel, ms_per_launch=kern_ms[1]),
-        "step_events_ms": dec_ms,
+        "roofline": dict(roof, traffic=None if tr is None else tr["dram_bytes"], peak_kind=peak_kind,
+                         kernel=KERNEL_NAMES[w.name],
+                         bytes_per_launch=bytes_kernel, ms_per_launch=kern_ms[1],
+                         load_efficiency=None if tr is None else tr["load_efficiency"]),
         "decode_call": {"ms": call_ms, "bytes": bytes_step, "gbs": achieved_call,
                         "kernels_ms": {"prep": kern_ms[0], "split": kern_ms[1], "reduce": kern_ms[2]}},
         "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": n_e2e,
+                "path": "kvq_decode_step_host: pinned host inputs and output, library copy streams"},
         "gpu_launches": launches,
         "clocks": clk.summary(),
+        # prefill-rate append (kvq_quantize with ctx - 1 tokens per sequence, in 8 calls of batch/8
+        # sequences): vectors = K and V vectors of every kv-head (FP4: latent tokens)
+        "quantize": {"vectors": n_vec, "ms": q_ms, "vectors_per_s": n_vec / (q_ms / 1e3) if q_ms > 0 else None,
+                     "input_gbs": n_vec * (w.latent_dim + w.rope_dim if w.k_mode == "fp4" else w.head_dim) * 2
+                     / (q_ms / 1e3) / 1e9 if q_ms > 0 else None},
     }
-    if rank == 0 and not args.no_cpu_baseline and world == 1:
-        if w.k_mode == "fp4":
-            P, step_fn = oracle_prepare_fp4(w, FP4_SAMPLE_CTX), oracle_step_fp4
-            what = f"sequence 0, first {FP4_SAMPLE_CTX} of {w.ctx} tokens, all {w.n_q_heads} heads"
-        else:
-            pairs = 2
-            P, step_fn = oracle_prepare(w, pairs, w.ctx), oracle_step
-            what = (f"{pairs} (sequence, kv-head) pairs at ctx {w.ctx} (of {w.batch * heads_kv} pairs per "
-                    f"step)")
-        tot, toks_tot, reps = 0.0, 0.0, 0
-        while tot < 10.0 and reps < 200:
-            dt, toks = step_fn(P)
-            tot, toks_tot, reps = tot + dt, toks_tot + toks, reps + 1
-        line["cpu_baseline"] = {"value": toks_tot / tot, "unit": "KV tokens/s", "cores": blas_threads(),
-                                "kind": "oracle",
-                                "sample": f"{reps} repetitions of one decode step over {what}, fp64 numpy"}
-    if rank == 0:
-        print(json.dumps(line))
     for c in caches:
         c.close()
+    del caches, news, host_news
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return line
+
+
+def run_ours(args, world, rank, local):
+    import bit_kv_cache_seeded_b200 as kvq
+    kvq.load()
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    if args.ctx > 0:
+        w = w.with_(ctx=args.ctx)
+    head = measure(kvq, w, args, world, dev)
+    line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "data": "synthetic"}
+    line.update({k: v for k, v in head.items() if k not in ("value", "ms_per_step")})
+    # the other full-size workloads, each with its own roofline and CPU baseline (one GPU only:
+    # a scaling run times the headline workload alone)
+    extra = [] if (world > 1 or args.ctx > 0 or args.only) else [n for n in EXTRA_WORKLOADS if n != w.name]
+    if extra:
+        line["workloads"] = {}
+        for name in extra:
+            line["workloads"][name] = measure(kvq, WORKLOADS[name], args, world, dev)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, 10.0)
+        for name in extra:
+            line["workloads"][name]["cpu_baseline"] = cpu_baseline(WORKLOADS[name], 3.0)
+    if rank == 0:
+        print(json.dumps(line))
 
 
 def main():

@@ -34,7 +34,8 @@ EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "k
            "kvq_cache_layout", "kvq_lloyd_max_table", "kvq_cache_destroy",
            "kvq_debug_quantize_rotated", "kvq_decode_attention_static", "kvq_kernel_launches",
            "kvq_cache_status", "kvq_debug_decode_unset_wait", "kvq_debug_decode_timed", "kvq_decode_step",
-           "kvq_step_staging_bytes", "kvq_decode_step_host", "kvq_draw_rotation_signs", "kvq_draw_qjl_matrix")
+           "kvq_step_staging_bytes", "kvq_decode_step_host", "kvq_draw_rotation_signs", "kvq_draw_qjl_matrix",
+           "kvq_partial_floats", "kvq_decode_partials", "kvq_combine_partials")
 KVQ_STATUS_WAIT_TIMEOUT = 1
 
 
@@ -86,9 +87,12 @@ def load() -> ctypes.CDLL:
         "kvq_debug_decode_timed": ([VP, VP, I32, VP, VP, SZ, VP, VP], I32),
         "kvq_decode_step": ([VP, VP, VP, VP, I32, VP, VP, SZ, VP], I32),
         "kvq_step_staging_bytes": ([VP, I32, P(SZ)], I32),
-        "kvq_decode_step_host": ([VP, VP, VP, VP, I32, VP, VP, SZ, VP, SZ, VP], I32),
+        "kvq_decode_step_host": ([VP, VP, VP, VP, I32, VP, VP, SZ, VP, SZ, VP, VP], I32),
         "kvq_draw_rotation_signs": ([ctypes.c_uint64, I32, VP], I32),
         "kvq_draw_qjl_matrix": ([ctypes.c_uint64, I32, I32, VP], I32),
+        "kvq_partial_floats": ([VP, P(I32)], I32),
+        "kvq_decode_partials": ([VP, VP, I32, VP, VP, SZ, VP], I32),
+        "kvq_combine_partials": ([VP, I32, I32, I32, I32, VP, VP], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -222,6 +226,39 @@ def kvq_decode_attention(handle, q: torch.Tensor, out: torch.Tensor, workspace: 
     _check("kvq_decode_attention", st)
 
 
+def kvq_partial_floats(handle) -> int:
+    n = ctypes.c_int32(0)
+    _check("kvq_partial_floats", load().kvq_partial_floats(handle, ctypes.byref(n)))
+    return int(n.value)
+
+
+def kvq_decode_partials(handle, q: torch.Tensor, partials: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """Softmax state of this cache's tokens: partials [batch, n_q_heads, 2 + dv] float32 (m, l, o)."""
+    _on_device("kvq_decode_partials", q=q, partials=partials, workspace=workspace)
+    if q.dtype not in DTYPES or partials.dtype != torch.float32:
+        raise TypeError("q must be float32/bfloat16 and partials float32")
+    if not (q.is_contiguous() and partials.is_contiguous()):
+        raise ValueError("q and partials must be contiguous")
+    st = load().kvq_decode_partials(handle, _ptr(q), DTYPES[q.dtype], _ptr(partials), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("kvq_decode_partials", st)
+
+
+def kvq_combine_partials(partials: torch.Tensor, out: torch.Tensor, stream=None):
+    """Merge partials [n_parts, batch, n_q_heads, 2 + dv] into out [batch, n_q_heads, dv]."""
+    _on_device("kvq_combine_partials", partials=partials, out=out)
+    if partials.dtype != torch.float32 or out.dtype != torch.float32:
+        raise TypeError("partials and out must be float32")
+    if partials.dim() != 4 or out.dim() != 3 or tuple(partials.shape[1:3]) != tuple(out.shape[:2]) \
+            or partials.shape[3] != out.shape[2] + 2:
+        raise ValueError("partials must be [n_parts, batch, n_q_heads, 2 + dv] for out [batch, n_q_heads, dv]")
+    if not (partials.is_contiguous() and out.is_contiguous()):
+        raise ValueError("partials and out must be contiguous")
+    n, B, H, S = partials.shape
+    _check("kvq_combine_partials", load().kvq_combine_partials(_ptr(partials), n, B, H, S - 2, _ptr(out),
+                                                               _stream(stream)))
+
+
 def kvq_decode_step(handle, K: torch.Tensor, V: torch.Tensor, q: torch.Tensor, out: torch.Tensor,
                     workspace: torch.Tensor, stream=None):
     """Append one token per sequence (K, V [B, Hkv, 1, d]; FP4: latent, rope) and decode with q."""
@@ -244,17 +281,24 @@ def kvq_step_staging_bytes(handle, dtype) -> int:
 
 
 def kvq_decode_step_host(handle, K: torch.Tensor, V: torch.Tensor, q: torch.Tensor, dtype, out: torch.Tensor,
-                         staging: torch.Tensor, workspace: torch.Tensor, stream=None):
+                         staging: torch.Tensor, workspace: torch.Tensor, stream=None, out_event=None):
     """kvq_decode_step from host memory: K, V, q and out are CPU tensors (pinned for asynchronous
-    copies) holding the bytes of the layouts kvq_decode_step takes, inputs of type `dtype`; out is
-    valid once the stream reaches the end of the call's work. The sizes are the caller's to get
-    right (KvqCache.step_host checks them)."""
+    copies) holding the bytes of the layouts kvq_decode_step takes, inputs of type `dtype`. Without
+    out_event, out is valid once the stream reaches the end of the call's work; with a
+    torch.cuda.Event, the library records it after the output copy (on its own copy stream) and the
+    stream does not wait: out is valid once the event has completed. The sizes are the caller's to
+    get right (KvqCache.step_host checks them)."""
     for t in (K, V, q, out):
         if t.is_cuda or not t.is_contiguous():
             raise ValueError("kvq_decode_step_host takes contiguous host tensors")
+    ev = None
+    if out_event is not None:
+        if out_event.cuda_event == 0:  # torch creates the event lazily, on its first record
+            out_event.record()
+        ev = ctypes.c_void_p(out_event.cuda_event)
     st = load().kvq_decode_step_host(handle, _ptr(K), _ptr(V), _ptr(q), DTYPES[dtype], _ptr(out), _ptr(staging),
                                      staging.numel() * staging.element_size(), _ptr(workspace),
-                                     workspace.numel() * workspace.element_size(), _stream(stream))
+                                     workspace.numel() * workspace.element_size(), _stream(stream), ev)
     _check("kvq_decode_step_host", st)
     return out
 
@@ -404,9 +448,10 @@ class KvqCache:
         kvq_decode_step(self.handle, K, V, q, out, self.workspace, stream)
         return out
 
-    def step_host(self, K, V, q, out=None, stream=None):
+    def step_host(self, K, V, q, out=None, stream=None, out_event=None):
         """step() with host (CPU) inputs and output: one call enqueues the input copies, the step
-        and the output copy on the stream; returns out (valid after the stream reaches it)."""
+        and the output copy; returns out (valid after the stream reaches it, or, with out_event,
+        once that event has completed)."""
         if out is None:
             out = torch.empty((self.batch, self.cfg.n_q_heads, self.out_dim), dtype=torch.float32).pin_memory()
         # the library cannot see host buffer sizes: check them here
@@ -422,7 +467,8 @@ class KvqCache:
         need = kvq_step_staging_bytes(self.handle, q.dtype)
         if getattr(self, "staging", None) is None or self.staging.numel() < need:
             self.staging = torch.empty(need, dtype=torch.uint8, device=self.workspace.device)
-        return kvq_decode_step_host(self.handle, K, V, q, q.dtype, out, self.staging, self.workspace, stream)
+        return kvq_decode_step_host(self.handle, K, V, q, q.dtype, out, self.staging, self.workspace, stream,
+                                    out_event)
 
     def decode(self, q, out=None, stream=None):
         self._check_q_out("decode", q, out)
@@ -431,6 +477,17 @@ class KvqCache:
                               device=q.device)
         kvq_decode_attention(self.handle, q, out, self.workspace, stream)
         return out
+
+    def decode_partials(self, q, partials=None, stream=None):
+        """Softmax state of this cache's tokens (kvq_decode_partials): [batch, n_q_heads, 2 + dv]."""
+        self._check_q_out("decode_partials", q, None)
+        n = kvq_partial_floats(self.handle)
+        if partials is None:
+            partials = torch.empty((self.batch, self.cfg.n_q_heads, n), dtype=torch.float32, device=q.device)
+        if tuple(partials.shape) != (self.batch, self.cfg.n_q_heads, n):
+            raise ValueError(f"decode_partials: partials must be {(self.batch, self.cfg.n_q_heads, n)}")
+        kvq_decode_partials(self.handle, q, partials, self.workspace, stream)
+        return partials
 
     def lengths(self):
         return kvq_cache_lengths(self.handle, self.batch)

@@ -2,6 +2,7 @@
 // Every entry point validates before launching and reports failures as kvq_status codes.
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <mutex>
@@ -151,8 +152,9 @@ int part_stride(const kvq_cache* c) {
   return 2 + kHeadDim * (c->v.qjl ? 2 : 1);
 }
 
-// Tensor-core decode: CTAs per (sequence, kv-head, split), each taking at most 4 query heads
-// (1 on every other path).
+// Query prep pieces per (sequence, kv-head) on the tensor-core paths: at most 4 query heads each
+// (1 on every other path). The mma.sync kernel also runs one CTA per piece; the tcgen05 kernel
+// takes all pieces of a kv-head in one CTA.
 int decode_hsplit(const kvq_cache* c) {
   if (c->is_fp4) return 1;
   const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
@@ -169,8 +171,11 @@ int prep_piece_stride(const kvq_cache* c) {
 }
 int prep_stride(const kvq_cache* c) { return prep_piece_stride(c) * decode_hsplit(c); }
 
-// Rows of the decode grid the split plan spreads over the SMs: (sequence, kv-head, piece).
-int decode_rows(const kvq_cache* c) { return c->batch * (c->is_fp4 ? 1 : c->cfg.n_kv_heads * decode_hsplit(c)); }
+// Rows of the decode grid the split plan spreads over the SMs: (sequence, kv-head[, piece]).
+int decode_rows(const kvq_cache* c) {
+  if (c->is_fp4) return c->batch;
+  return c->batch * c->cfg.n_kv_heads * (c->tc ? 1 : decode_hsplit(c));
+}
 
 size_t partials_bytes(const kvq_cache* c, int splits) {
   return align_up(sizeof(float) * (size_t)c->batch * c->cfg.n_q_heads * splits * part_stride(c), 256);
@@ -184,7 +189,7 @@ size_t workspace_for(const kvq_cache* c, int splits) {
 // Resident decode CTAs per SM for a chunk of `units` 64-token units: one for the MLA kernel, the
 // tensor-core kernel's shared-memory and register limit for query groups of 1, 2 or 4, else 4.
 int decode_slots_per_sm(const kvq_cache* c, int units) {
-  if (c->is_fp4) return 1;
+  if (c->is_fp4 || c->tc) return 1;
   const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
   if (group == 1 || group == 2 || group == 4)
     return lm_mma_slots_per_sm(group, c->k, c->v, units * kTile * kTilePair);
@@ -192,7 +197,19 @@ int decode_slots_per_sm(const kvq_cache* c, int units) {
 }
 
 // Largest chunk (in 64-token units) one decode CTA may take.
-int decode_max_units(const kvq_cache* c) { return c->is_fp4 ? (1 << 30) : kChunkMax / (kTile * kTilePair); }
+int decode_max_units(const kvq_cache* c) {
+  if (c->is_fp4) return 1 << 30;
+  if (c->tc) return tc_chunk_max(c->cfg.n_q_heads / c->cfg.n_kv_heads) / (kTile * kTilePair);
+  return kChunkMax / (kTile * kTilePair);
+}
+
+// The LM decode kernel a cache uses: the tcgen05 kernel where it has an instance, unless the
+// environment variable KVQ_DECODE_KERNEL is "mma" (the mma.sync kernel, for comparison).
+bool choose_tc(const kvq_cfg& cfg, const SideLayout& k, const SideLayout& v) {
+  const char* e = std::getenv("KVQ_DECODE_KERNEL");
+  if (e && std::strcmp(e, "mma") == 0) return false;
+  return k.order == kOrderOctet && tc_modes_supported(cfg.n_q_heads / cfg.n_kv_heads, k.bits, k.qjl, v.bits, v.qjl);
+}
 
 // Upper bound on CTAs per SM considered by the split plan (sizes the workspace).
 int decode_waves_bound(const kvq_cache* c) { return c->is_fp4 ? 2 : 16; }
@@ -316,6 +333,7 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
     return KVQ_ERR_CUDA;
   }
   c->signs_stride = cfg->rot_per_head ? kHeadDim : 0;
+  c->tc = !P.fp4_mode && choose_tc(*cfg, P.k, P.v);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(c->d_lens, 0, sizeof(int) * ((size_t)batch + kStatusWords), s) != cudaSuccess) {
     delete c;
@@ -431,10 +449,11 @@ namespace {
 // decode CTA first waits, bounded by wait_limit cycles, on a barrier that nothing completes).
 kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out, void* workspace,
                        size_t ws_bytes, void* stream, int debug_unset_wait, long long wait_limit,
-                       const cudaEvent_t* ev = nullptr, const QuantizeParams* qp = nullptr) {
-  if (!c || !q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+                       const cudaEvent_t* ev = nullptr, const QuantizeParams* qp = nullptr, float* pout = nullptr) {
+  if (!c || !q || (!out && !pout) || !workspace) return KVQ_ERR_INVALID_ARG;
   if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
+  if (!aligned16(q) || !aligned16(out ? (const void*)out : (const void*)pout) || !aligned16(workspace))
+    return KVQ_ERR_ALIGNMENT;
   if (!on_cache_device(c)) return KVQ_ERR_INVALID_ARG;
   int max_len = 0;
   for (int v : c->lens) max_len = std::max(max_len, v);
@@ -453,6 +472,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
     p.q = q;
     p.bf16 = dtype == KVQ_BF16;
     p.out = out;
+    p.pout = pout;
     p.part = static_cast<float*>(workspace);
     p.B = c->batch;
     p.Hq = c->cfg.n_q_heads;
@@ -474,6 +494,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.q = q;
   p.bf16 = dtype == KVQ_BF16;
   p.out = out;
+  p.pout = pout;
   p.part = static_cast<float*>(workspace);
   p.part_stride = part_stride(c);
   p.B = c->batch;
@@ -499,12 +520,14 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.err = c->d_status;
   p.wait_limit = wait_limit;
   p.debug_unset_wait = debug_unset_wait;
-  if (qp && !mma_decode_supported(p)) {  // no fused front kernel on this path: append first
+  p.use_tc = c->tc ? 1 : 0;
+  const bool tensor_path = p.use_tc ? tc_decode_supported(p) : mma_decode_supported(p);
+  if (qp && !tensor_path) {  // no fused front kernel on this path: append first
     if (launch_quantize_lm(*qp, 2, s) != cudaSuccess) return KVQ_ERR_CUDA;
     qp = nullptr;
   }
   p.cache_after_wait = qp != nullptr;
-  if (debug_unset_wait && !mma_decode_supported(p)) return KVQ_ERR_UNSUPPORTED;
+  if (debug_unset_wait && !tensor_path) return KVQ_ERR_UNSUPPORTED;
   if (launch_decode_lm(p, s, ev ? ev[1] : nullptr, qp) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
   if (launch_reduce_lm(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
   return KVQ_OK;
@@ -516,6 +539,29 @@ extern "C" {
 kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,
                                 void* workspace, size_t ws_bytes, void* stream) {
   return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles);
+}
+
+kvq_status kvq_partial_floats(const kvq_cache* c, int32_t* floats) {
+  if (!c || !floats) return KVQ_ERR_INVALID_ARG;
+  *floats = 2 + (c->is_fp4 ? c->cfg.latent_dim : kHeadDim);
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_partials(const kvq_cache* c, const void* q, kvq_dtype dtype, float* partials,
+                               void* workspace, size_t ws_bytes, void* stream) {
+  if (!partials) return KVQ_ERR_INVALID_ARG;
+  return decode_impl(c, q, dtype, nullptr, workspace, ws_bytes, stream, 0, kWaitLimitCycles, nullptr, nullptr,
+                     partials);
+}
+
+kvq_status kvq_combine_partials(const float* partials, int32_t n_parts, int32_t batch, int32_t n_q_heads,
+                                int32_t dv, float* out, void* stream) {
+  if (!partials || !out || n_parts < 1 || batch < 1 || n_q_heads < 1 || dv < 1) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(partials) || !aligned16(out)) return KVQ_ERR_ALIGNMENT;
+  const long rows = (long)batch * n_q_heads;
+  if (rows > (1l << 31) - 1) return KVQ_ERR_INVALID_ARG;
+  return launch_combine_partials(partials, n_parts, (int)rows, dv, out, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
@@ -557,11 +603,12 @@ kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const voi
 
 namespace {
 // Byte sizes of one step's K, V, q and out, and their offsets in the staging buffer: two input
-// slots (K, V, q each), then the output.
+// slots (K, V, q each), then two output slots.
 struct StepStaging {
   size_t n[4] = {};    // K, V, q, out
-  size_t off[4] = {};  // within an input slot (out: within the buffer)
+  size_t off[4] = {};  // within an input slot (out: the first output slot, within the buffer)
   size_t slot = 0;     // bytes of one input slot
+  size_t out_slot = 0; // bytes of one output slot
   size_t total = 0;
 };
 StepStaging step_staging(const kvq_cache* c, kvq_dtype dtype) {
@@ -582,16 +629,17 @@ StepStaging step_staging(const kvq_cache* c, kvq_dtype dtype) {
     S.slot = align_up(S.slot + S.n[i], 256);
   }
   S.off[3] = 2 * S.slot;
-  S.total = align_up(S.off[3] + S.n[3], 256);
+  S.out_slot = align_up(S.n[3], 256);
+  S.total = S.off[3] + 2 * S.out_slot;
   return S;
 }
 
-// Per cache: the copy stream of kvq_decode_step_host and, per input slot, the events "inputs
-// landed" (copy stream) and "step done reading them" (caller's stream). Created at the first
-// call, released by kvq_cache_destroy.
+// Per cache: the two copy streams of kvq_decode_step_host (host -> device inputs, device -> host
+// output) and, per slot, the events "inputs landed" (input stream), "step done" (caller's stream)
+// and "output copied" (output stream). Created at the first call, released by kvq_cache_destroy.
 struct HostStep {
-  cudaStream_t copy = nullptr;
-  cudaEvent_t landed[2] = {}, done[2] = {};
+  cudaStream_t copy = nullptr, copy_out = nullptr;
+  cudaEvent_t landed[2] = {}, done[2] = {}, copied[2] = {};
   unsigned long long calls = 0;
 };
 std::mutex g_host_step_mu;
@@ -601,8 +649,10 @@ void release_host_step(HostStep& h) {
   for (int i = 0; i < 2; ++i) {
     if (h.landed[i]) cudaEventDestroy(h.landed[i]);
     if (h.done[i]) cudaEventDestroy(h.done[i]);
+    if (h.copied[i]) cudaEventDestroy(h.copied[i]);
   }
   if (h.copy) cudaStreamDestroy(h.copy);
+  if (h.copy_out) cudaStreamDestroy(h.copy_out);
   h = HostStep{};
 }
 
@@ -610,10 +660,12 @@ HostStep* host_step_state(const kvq_cache* c) {
   std::lock_guard<std::mutex> lock(g_host_step_mu);
   HostStep& h = g_host_step[c];
   if (h.copy) return &h;
-  bool ok = cudaStreamCreateWithFlags(&h.copy, cudaStreamNonBlocking) == cudaSuccess;
+  bool ok = cudaStreamCreateWithFlags(&h.copy, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&h.copy_out, cudaStreamNonBlocking) == cudaSuccess;
   for (int i = 0; i < 2 && ok; ++i)
     ok = cudaEventCreateWithFlags(&h.landed[i], cudaEventDisableTiming) == cudaSuccess &&
-         cudaEventCreateWithFlags(&h.done[i], cudaEventDisableTiming) == cudaSuccess;
+         cudaEventCreateWithFlags(&h.done[i], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&h.copied[i], cudaEventDisableTiming) == cudaSuccess;
   if (ok) return &h;
   release_host_step(h);
   g_host_step.erase(c);
@@ -639,7 +691,7 @@ kvq_status kvq_step_staging_bytes(const kvq_cache* c, kvq_dtype dtype, size_t* b
 
 kvq_status kvq_decode_step_host(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
                                 float* out, void* staging, size_t staging_bytes, void* workspace,
-                                size_t ws_bytes, void* stream) {
+                                size_t ws_bytes, void* stream, void* out_event) {
   if (!c || !K || !V || !q || !out || !staging || !workspace) return KVQ_ERR_INVALID_ARG;
   if (dtype != KVQ_F32 && dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(staging) || !aligned16(workspace)) return KVQ_ERR_ALIGNMENT;
@@ -660,23 +712,29 @@ kvq_status kvq_decode_step_host(kvq_cache* c, const void* K, const void* V, cons
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int slot = (int)(h->calls & 1);
   char* in = static_cast<char*>(staging) + slot * S.slot;
-  char* dout = static_cast<char*>(staging) + S.off[3];
-  // the inputs cross on the copy stream once the step two calls back has read this slot, while
-  // the previous step may still run; the step waits for them on the caller's stream
+  char* dout = static_cast<char*>(staging) + S.off[3] + slot * S.out_slot;
+  // the inputs cross on the input stream once the step two calls back has read this slot, while
+  // the previous step may still run; the step waits for them on the caller's stream, and for the
+  // output copy of the step two calls back to have left this output slot
   if (cudaStreamWaitEvent(h->copy, h->done[slot], 0) != cudaSuccess) return KVQ_ERR_CUDA;
   const void* src[3] = {K, V, q};
   for (int i = 0; i < 3; ++i)
     if (cudaMemcpyAsync(in + S.off[i], src[i], S.n[i], cudaMemcpyHostToDevice, h->copy) != cudaSuccess)
       return KVQ_ERR_CUDA;
-  if (cudaEventRecord(h->landed[slot], h->copy) != cudaSuccess || cudaStreamWaitEvent(s, h->landed[slot], 0) != cudaSuccess)
+  if (cudaEventRecord(h->landed[slot], h->copy) != cudaSuccess || cudaStreamWaitEvent(s, h->landed[slot], 0) != cudaSuccess ||
+      cudaStreamWaitEvent(s, h->copied[slot], 0) != cudaSuccess)
     return KVQ_ERR_CUDA;
   const kvq_status r = kvq_decode_step(c, in + S.off[0], in + S.off[1], in + S.off[2], dtype,
                                        reinterpret_cast<float*>(dout), workspace, ws_bytes, stream);
   if (r != KVQ_OK) return r;
   ++h->calls;
-  if (cudaEventRecord(h->done[slot], s) != cudaSuccess) return KVQ_ERR_CUDA;
-  if (cudaMemcpyAsync(out, dout, S.n[3], cudaMemcpyDeviceToHost, s) != cudaSuccess) return KVQ_ERR_CUDA;
-  return KVQ_OK;
+  // the output leaves on the output stream, overlapping the caller's next step
+  if (cudaEventRecord(h->done[slot], s) != cudaSuccess || cudaStreamWaitEvent(h->copy_out, h->done[slot], 0) != cudaSuccess ||
+      cudaMemcpyAsync(out, dout, S.n[3], cudaMemcpyDeviceToHost, h->copy_out) != cudaSuccess ||
+      cudaEventRecord(h->copied[slot], h->copy_out) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  if (out_event) return cudaEventRecord(static_cast<cudaEvent_t>(out_event), h->copy_out) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  return cudaStreamWaitEvent(s, h->copied[slot], 0) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 kvq_status kvq_debug_decode_unset_wait(const kvq_cache* c, const void* q, kvq_dtype dtype, float* out,

@@ -306,7 +306,9 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
     }
     M = mn;
   }
-  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  // the normalisation by L, unless the call asks for the merged softmax state (m, l, unnormalised
+  // o), whose Sᵀ fold and inverse rotation are linear and apply the same way
+  const float inv = p.pout ? 1.f : (L > 0.f) ? 1.f / L : 0.f;
   o *= inv;
   if (vq) {
     az[i * G + h] = oz * inv;
@@ -359,9 +361,15 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
     }
     const float a0 = u[0] + u[1], a1 = u[0] - u[1], a2 = u[2] + u[3], a3 = u[2] - u[3];
     u[0] = a0 + a2; u[2] = a0 - a2; u[1] = a1 + a3; u[3] = a1 - a3;
-    float* dst = p.out + ((size_t)b * p.Hq + hk * G + hh) * kHeadDim;
+    float* dst = p.pout ? p.pout + ((size_t)b * p.Hq + hk * G + hh) * (2 + kHeadDim) + 2
+                        : p.out + ((size_t)b * p.Hq + hk * G + hh) * kHeadDim;
 #pragma unroll
     for (int k = 0; k < 4; ++k) dst[32 * k + lane] = u[k] * sg[k];
+  }
+  if (p.pout && i == 0) {  // the head's running maximum (log2 units) and sum of weights
+    float* st = p.pout + ((size_t)b * p.Hq + hk * G + h) * (2 + kHeadDim);
+    st[0] = M;
+    st[1] = L;
   }
 }
 
@@ -390,6 +398,7 @@ cudaError_t dispatch_modes(const DecodeParams& p, dim3 grid, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
+  if (p.use_tc) return tc_decode_supported(p) ? launch_decode_lm_tc(p, s, ev_mid, qp) : cudaErrorNotSupported;
   if (mma_decode_supported(p)) return launch_decode_lm_mma(p, s, ev_mid, qp);
   if (qp) return cudaErrorNotSupported;
   if (ev_mid && cudaEventRecord(ev_mid, s) != cudaSuccess) return cudaErrorUnknown;

@@ -41,9 +41,12 @@
 #include "kvq_async.cuh"
 #include "kvq_internal.h"
 #include "kvq_quantize_lm.cuh"
+#include "kvq_lm_common.cuh"
 
 namespace kvq {
 namespace {
+
+using namespace lmc;
 
 constexpr int kWarpsM = 4;
 constexpr int kThreadsM = kWarpsM * 32;
@@ -52,13 +55,8 @@ constexpr int kStagesM = 4;                          // bulk-copy stages (tile p
 constexpr int kMinBlocksM = 4;                       // resident CTAs per SM the registers are sized for
 constexpr int kSmemPerSm = 233472;                   // shared memory per SM (228 KB)
 constexpr int kSmemReserved = 1024 + 128;            // per CTA: the runtime's reserve + static arrays
-constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
-constexpr float kSqrtHalfPi = 1.2533141373155003f;  // sqrt(pi/2)
-constexpr int kQRange = 32639;                       // query term quantised to [-32639, 32639]
 constexpr int kPdStride = 96;                        // weight-digit row stride (bytes): 64 tokens + pad
 constexpr int kNormBlock = 256;                      // staged value norms / gammas of two cache tiles
-constexpr float kWRange = 8388608.f;                 // weights quantised below 2^23
-constexpr float kRoundBias = 8388608.f;              // x + 2^23 (0 <= x < 2^23): bits = 0x4B000000 | rint(x)
 
 // A int8, B uint8 (the value-phase weight digits are non-negative bytes).
 __device__ __forceinline__ void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -92,56 +90,6 @@ template <int P>
 __device__ __forceinline__ uint32_t bit_to_s8(uint32_t w) {
   return (P == 7) ? (w & 0x80808080u) : ((w * (1u << (7 - P))) & 0x80808080u);
 }
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.f32 %0, %1;\n" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ float load_q(const void* base, size_t i, int bf16) {
-  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
-  return reinterpret_cast<const float*>(base)[i];
-}
-
-template <int BITS> struct Walsh { static constexpr int P = BITS == 3 ? 4 : BITS; };
-
-// 32-bit word of Walsh plane P from the stored bit-plane words (parity plane for 3 bits).
-template <int BITS>
-__device__ __forceinline__ uint32_t walsh_word(const uint32_t (&w)[3], int P) {
-  if (BITS == 3 && P == 3) return w[0] ^ w[1] ^ w[2];
-  return w[P];
-}
-
-// Walsh coefficients a_P of an odd b-bit table (codes 2^(b-1).. are the positive half).
-__device__ __forceinline__ void walsh_coeffs(int bits, const float* c, float (&a)[4]) {
-  a[0] = a[1] = a[2] = a[3] = 0.f;
-  if (bits == 1) a[0] = c[1];
-  if (bits == 2) { a[0] = 0.5f * (c[3] - c[2]); a[1] = 0.5f * (c[3] + c[2]); }
-  if (bits == 3) {
-    a[0] = 0.25f * (c[7] - c[6] + c[5] - c[4]);
-    a[1] = 0.25f * (c[7] + c[6] - c[5] - c[4]);
-    a[2] = 0.25f * (c[7] + c[6] + c[5] + c[4]);
-    a[3] = 0.25f * (c[7] - c[6] - c[5] + c[4]);
-  }
-}
-
-// Byte layout of one 32-token tile of a side with BITS code planes (and a sketch when QJL), as the
-// host lays it out (kvq_api.cu make_side): planes, sketch words, fp16 norms, fp16 residual norms.
-// Compile-time here so that every shared-memory address in the decode kernel is an immediate
-// offset; launch_mma() refuses a cache whose runtime layout differs.
-template <int BITS, bool QJL>
-struct TileLayout {
-  static constexpr int PLANES = 0;
-  static constexpr int SKETCH = BITS * kTile * 16;
-  static constexpr int NORM = SKETCH + (QJL ? kTile * 16 : 0);
-  static constexpr int GAMMA = NORM + kTile * 2;
-  static constexpr int BYTES = (GAMMA + (QJL ? kTile * 2 : 0) + 15) / 16 * 16;
-  static bool matches(const SideLayout& L) {
-    return L.off_planes == PLANES && L.off_sketch == SKETCH && L.off_norm == NORM &&
-           (!QJL || L.off_gamma == GAMMA) && L.tile_bytes == BYTES && L.bits == BITS && L.qjl == QJL;
-  }
-};
 
 template <int G, int KB, bool KQ, int VB, bool VQ>
 struct MmaCfg {
@@ -859,10 +807,9 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 
 }
 
-template <int G, int KB, bool KQ, int VB, bool VQ>
-cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
-  if (!TileLayout<KB, KQ>::matches(p.k) || !TileLayout<VB, VQ>::matches(p.v)) return cudaErrorNotSupported;
-  if (p.k.order != kOrderOctet || p.v.order != kOrderByteLane) return cudaErrorNotSupported;
+// Query prep of a decode call, or the fused step's front kernel (append + query prep) when qp is given.
+template <int G, int KB, bool KQ>
+cudaError_t launch_prep(const DecodeParams& p, cudaStream_t s, const QuantizeParams* qp) {
   const size_t prep_smem = KQ ? sizeof(float) * kHeadDim * kHeadDim : 0;
   cudaError_t e = cudaFuncSetAttribute(decode_lm_prep<G, KB, KQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep_smem);
@@ -889,7 +836,14 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid
   } else {
     decode_lm_prep<G, KB, KQ><<<dim3(p.Hkv * p.hsplit, p.B), kThreadsM, prep_smem, s>>>(p);
   }
-  e = launched();
+  return launched();
+}
+
+template <int G, int KB, bool KQ, int VB, bool VQ>
+cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
+  if (!TileLayout<KB, KQ>::matches(p.k) || !TileLayout<VB, VQ>::matches(p.v)) return cudaErrorNotSupported;
+  if (p.k.order != kOrderOctet || p.v.order != kOrderByteLane) return cudaErrorNotSupported;
+  cudaError_t e = launch_prep<G, KB, KQ>(p, s, qp);
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
   const size_t smem = mma_smem_bytes(G, p.k, p.v, p.chunk);
@@ -928,7 +882,28 @@ cudaError_t dispatch_mma_modes(const DecodeParams& p, cudaStream_t s, cudaEvent_
   return cudaErrorNotSupported;
 }
 
+template <int G>
+cudaError_t dispatch_prep(const DecodeParams& p, cudaStream_t s, const QuantizeParams* qp) {
+  const int kb = p.k.bits;
+  const bool kq = p.k.qjl;
+  if (kb == 1 && !kq) return launch_prep<G, 1, false>(p, s, qp);
+  if (kb == 2 && kq) return launch_prep<G, 2, true>(p, s, qp);
+  if (kb == 2 && !kq) return launch_prep<G, 2, false>(p, s, qp);
+  if (kb == 3 && kq) return launch_prep<G, 3, true>(p, s, qp);
+  if (kb == 3 && !kq) return launch_prep<G, 3, false>(p, s, qp);
+  return cudaErrorNotSupported;
+}
+
 }  // namespace
+
+cudaError_t launch_lm_query_prep(const DecodeParams& p, cudaStream_t s, const QuantizeParams* qp) {
+  switch (p.group / p.hsplit) {  // heads of one prep piece
+    case 1: return dispatch_prep<1>(p, s, qp);
+    case 2: return dispatch_prep<2>(p, s, qp);
+    case 4: return dispatch_prep<4>(p, s, qp);
+    default: return cudaErrorNotSupported;
+  }
+}
 
 int mma_prep_bytes(int k_bits, int k_qjl, int group) {
   const int kp = (k_bits == 3 ? 4 : k_bits) + (k_qjl ? 1 : 0);

@@ -82,6 +82,7 @@ struct DecodeParams {
   const void* q;          // [B, Hq, d]
   int bf16;
   float* out;             // [B, Hq, d]
+  float* pout;            // instead of out: merged softmax state [B, Hq, 2 + d] (m, l, unnormalised o)
   float* part;            // [B, Hq, splits, part_stride]
   int part_stride;        // 2 + d (+ m with a value sketch)
   int B, Hq, Hkv, group;
@@ -103,12 +104,14 @@ struct DecodeParams {
   long long wait_limit;   // SM clock cycles a kernel waits for staged data before giving up
   int debug_unset_wait;   // test entry: also wait once on a barrier nothing completes
   int cache_after_wait;   // fused step: the cache is written by this kernel's predecessor (wait first)
+  int use_tc;             // decode on the tcgen05 kernel (one CTA per sequence, kv-head and split)
 };
 
 struct MlaParams {
   const void* q;          // [B, Hq, latent + rope]
   int bf16;
   float* out;             // [B, Hq, latent]
+  float* pout;            // instead of out: merged softmax state [B, Hq, 2 + latent]
   float* part;            // [B, Hq, splits, 2 + latent]
   int B, Hq;
   int splits, chunk;
@@ -144,10 +147,21 @@ bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl
 int mma_prep_bytes(int k_bits, int k_qjl, int group);  // bytes of one (sequence, kv-head) prep area
 cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp);
 cudaError_t launch_reduce_lm(const DecodeParams& p, cudaStream_t s);
+// Query prep of the tensor-core paths in pieces of group / hsplit heads (or, with qp, the fused
+// step's front kernel: append + query prep), as one launch.
+cudaError_t launch_lm_query_prep(const DecodeParams& p, cudaStream_t s, const QuantizeParams* qp);
+// The tcgen05 decode kernel (kvq_decode_tc.cu): one CTA per (sequence, kv-head, split) with all
+// query heads of the group. tc_supported: this group and code combination have an instance.
+bool tc_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl);
+bool tc_decode_supported(const DecodeParams& p);
+int tc_chunk_max(int group);     // largest chunk (tokens) of one CTA
+cudaError_t launch_decode_lm_tc(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp);
 cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s);
 bool mla_mma_supported(const MlaParams& p);
 bool mla_umma_supported(const MlaParams& p);
+// Log-sum-exp merge of n_parts softmax states [n_parts][rows][2 + dv] into out [rows][dv] (kvq_combine.cu).
+cudaError_t launch_combine_partials(const float* parts, int n_parts, int rows, int dv, float* out, cudaStream_t s);
 cudaError_t launch_decode_mla_umma(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_decode_mla_mma(const MlaParams& p, cudaStream_t s);
 
@@ -162,6 +176,7 @@ struct kvq_cache {
   int batch = 0, capacity = 0, tiles_per_seq = 0, sms = 148;
   int signs_stride = 0;     // 0, or kHeadDim when every kv-head has its own rotation diagonal
   int device = -1;          // the CUDA device whose memory holds the arena (current at init)
+  bool tc = false;          // LM decode runs on the tcgen05 kernel (else mma.sync / CUDA cores)
   char* dev = nullptr;
   size_t dev_bytes = 0;
   int* d_lens = nullptr;

@@ -151,6 +151,15 @@ __global__ void __launch_bounds__(kLat) reduce_mla(const __grid_constant__ MlaPa
     L += w * ps[1];
     o += w * ps[2 + c];
   }
+  if (p.pout) {  // merged softmax state: running maximum (log2 units), sum of weights, unnormalised o
+    float* st = p.pout + (size_t)row * stride;
+    st[2 + c] = o;
+    if (c == 0) {
+      st[0] = M;
+      st[1] = L;
+    }
+    return;
+  }
   p.out[(size_t)row * kLat + c] = (L > 0.f) ? o / L : 0.f;
 }
 

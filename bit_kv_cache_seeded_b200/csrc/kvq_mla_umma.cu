@@ -33,6 +33,7 @@
 
 #include "kvq_async.cuh"
 #include "kvq_internal.h"
+#include "kvq_tcgen05.cuh"
 
 namespace kvq {
 namespace {
@@ -59,70 +60,16 @@ constexpr int kOffP = kOffRope + 2 * kSizeRope;
 constexpr int kSizeP = kHeadsU * kTokU * 2;             // 8192
 constexpr int kSmemU = kOffP + kSizeP;                  // 229376
 
-// ---- tcgen05 / descriptor helpers (PTX ISA 8.7+, sm_100a) ----------------------------------
-
-// Shared-memory matrix descriptor, no swizzle: start address, leading-dimension byte offset
-// (between core matrices along K for K-major operands, along K for MN-major ones too: see the
-// call sites), stride-dimension byte offset, version 1 (tcgen05), layout type 0.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
-  return d;
-}
-
-// Instruction descriptor for kind::f16 with fp32 accumulation.
-//   fmt: 0 = f16, 1 = bf16 (A and B alike); a_mn / b_mn: operand is MN-major; M, N: tile shape.
-__host__ __device__ constexpr uint32_t idesc_f16(int fmt, int a_mn, int b_mn, int M, int N) {
-  return (1u << 4)                      // D format: f32
-         | ((uint32_t)fmt << 7)         // A format
-         | ((uint32_t)fmt << 10)        // B format
-         | ((uint32_t)a_mn << 15)       // A major
-         | ((uint32_t)b_mn << 16)       // B major
-         | ((uint32_t)(N >> 3) << 17)   // N / 8
-         | ((uint32_t)(M >> 4) << 24);  // M / 16
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
-}
-// Arrives once on the mbarrier when every MMA this thread issued before has completed.
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-
-// 32 lanes x 32 bit, 32 consecutive columns: thread l of the warp gets lane (base lane + l).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
-      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+using tc::smem_desc;
+using tc::idesc_f16;
+using tc::umma_f16;
+using tc::tmem_ld32;
+using tc::tmem_st32;
+__device__ __forceinline__ void umma_commit(uint32_t bar) { tc::commit(bar); }
+__device__ __forceinline__ void tc_fence_before() { tc::fence_before(); }
+__device__ __forceinline__ void tc_fence_after() { tc::fence_after(); }
+__device__ __forceinline__ void tmem_wait_ld() { tc::wait_ld(); }
+__device__ __forceinline__ void tmem_wait_st() { tc::wait_st(); }
 
 // Two E2M1 codes (one byte, channel 2k in the low nibble) to f16x2 (channel 2k in the low half).
 __device__ __forceinline__ uint32_t e2m1x2_f16x2(uint32_t byte) {
@@ -154,14 +101,8 @@ __device__ __forceinline__ int core_off(int row, int col, int chunks_per_row) {
   return ((row >> 3) * chunks_per_row + (col >> 3)) * kCore + (row & 7) * 16 + (col & 7) * 2;
 }
 
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(dst_smem), "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
-}
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) { tc::alloc(dst_smem, ncols); }
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) { tc::dealloc(taddr, ncols); }
 
 // Packed data of one 64-token tile that one thread dequantises: token tid % 64, channels
 // 128 (tid / 64) .. +127 (64 code bytes, 8 scale bytes) and two 16-byte RoPE chunks. Loaded straight

@@ -17,6 +17,8 @@
 // hardware efficiency"): one warp per token, lane l owning the 16-channel group l:
 //   s = E4M3_rn_satfinite(amax / 6); q_i = E2M1_rn_satfinite(x_i / s) (IEEE fp32 division);
 //   a zero scale codes the group as zeros; RoPE key copied as bf16.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -24,11 +26,13 @@
 #include "kvq_async.cuh"
 #include "kvq_internal.h"
 #include "kvq_quantize_lm.cuh"
+#include "kvq_quantize_tile.cuh"
 
 namespace kvq {
 namespace {
 
 constexpr int kQuantWarps = 8;  // FP4 kernel: one token per warp
+constexpr int kTileQuantizeMinTokens = 16;  // appends of at least this many tokens per sequence use the tile kernel
 using qlm::kLmWarps;
 using qlm::load_elem;
 
@@ -36,6 +40,16 @@ using qlm::load_elem;
 __global__ void __launch_bounds__(qlm::kLmWarps * 32)
 quantize_lm_kernel(const __grid_constant__ QuantizeParams p) {
   qlm::quantize_lm_block(p, blockIdx.y, blockIdx.x, gridDim.x);
+}
+
+// Prefill-rate LM quantize: grid (blocks, sides); tiles of one side per block (kvq_quantize_tile.cuh).
+__global__ void __launch_bounds__(qtile::kThreads)
+quantize_lm_tile_kernel(const __grid_constant__ QuantizeParams p) {
+  extern __shared__ __align__(16) unsigned char qt_smem[];
+  const bool sketch = p.side[0].qjl || p.side[1].qjl;
+  qtile::Smem& sm = *reinterpret_cast<qtile::Smem*>(qt_smem);
+  float* st_s = reinterpret_cast<float*>(qt_smem + sizeof(qtile::Smem));
+  qtile::quantize_tiles(p, blockIdx.y, sketch ? st_s : nullptr, sm);
 }
 
 // E2M1 code of an fp32 value: nearest grid point of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the
@@ -100,6 +114,17 @@ int grid_for(long work_items, int per_block) {
 }  // namespace
 
 cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s) {
+  if (n_sides == 2 && !p.skip_rotation && p.n_new >= kTileQuantizeMinTokens) {
+    // appends of many tokens per sequence: whole tiles per block, 16-byte stores, S^T staged once
+    const bool sketch = p.side[0].qjl || p.side[1].qjl;
+    const long tiles = (long)p.n_seq * p.heads * qtile::max_tiles(p.n_new);
+    const size_t smem = qtile::smem_bytes(sketch);
+    cudaError_t e = cudaFuncSetAttribute(quantize_lm_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int blocks = (int)std::min<long>(tiles, 148L * 2);
+    quantize_lm_tile_kernel<<<dim3(blocks, 2), qtile::kThreads, smem, s>>>(p);
+    return launched();
+  }
   QuantizeParams q = p;
   if (n_sides < 2) q.side[1] = q.side[0];  // the block count looks at both sides
   const bool sketch = p.side[0].qjl || (n_sides > 1 && p.side[1].qjl);

@@ -166,18 +166,44 @@ kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dty
 kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
                            float* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* Context-parallel decode ("How DeepSeek-V4.1-Flash cut KV cache storage by 4x via CSA2", section
+ * "CSA2": the long-context MLA cache; here its context can be split over caches on several GPUs).
+ * Each shard -- a cache holding a disjoint part of every sequence's tokens, with the same
+ * configuration and seeds -- computes the softmax state of its part, the shards exchange those
+ * states (a few KB per sequence, e.g. with an NCCL all-gather), and any of them merges them:
+ *   kvq_partial_floats: floats per (sequence, query head) of a state, 2 + dv (dv = head_dim, or
+ *     latent_dim for FP4).
+ *   kvq_decode_partials: as kvq_decode_attention, but writes partials [batch, n_q_heads, 2 + dv]
+ *     (device, f32): m (the largest logit times log2 e), l = sum 2^(logit log2 e - m) and the
+ *     unnormalised output o = sum 2^(...) v_hat (in the original, unrotated domain). A sequence with
+ *     no tokens gives m = -inf, l = 0, o = 0.
+ *   kvq_combine_partials: partials [n_parts][batch, n_q_heads, 2 + dv] (device, contiguous) ->
+ *     out [batch, n_q_heads, dv] = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i, M = max_i m_i
+ *     (all-zero where every part is empty). Needs no cache; runs on the current device.
+ * Merging the states of disjoint shards equals decoding over their union, up to rounding. */
+kvq_status kvq_partial_floats(const kvq_cache* c, int32_t* floats);
+kvq_status kvq_decode_partials(const kvq_cache* c, const void* q, kvq_dtype dtype, float* partials,
+                               void* workspace, size_t ws_bytes, void* stream);
+kvq_status kvq_combine_partials(const float* partials, int32_t n_parts, int32_t batch, int32_t n_q_heads,
+                                int32_t dv, float* out, void* stream);
+
 /* Device bytes of the staging buffer kvq_decode_step_host needs for inputs of type dtype: two
- * input slots (one step's K and V with n_new = 1 for all sequences, and q), then out; each region
- * 256-byte aligned. */
+ * input slots (one step's K and V with n_new = 1 for all sequences, and q), then two output slots;
+ * each region 256-byte aligned. */
 kvq_status kvq_step_staging_bytes(const kvq_cache* c, kvq_dtype dtype, size_t* bytes);
 
 /* kvq_decode_step with its inputs and output in HOST memory (layouts as for kvq_decode_step;
- * dtype f32 or bf16; out [batch, n_q_heads, head_dim] f32, or latent_dim for FP4). The copies of
- * K, V and q run on a copy stream the library keeps for the cache (created at the first call,
- * released by kvq_cache_destroy), into the input slot of `staging` the step two calls back has
- * finished with, so they overlap the previous step. The step waits for them on `stream`, and the
- * copy of out back to host memory follows it on `stream`; the call returns without waiting, and
- * out is valid once `stream` has reached that point. staging: device, 16-byte aligned, at least
+ * dtype f32 or bf16; out [batch, n_q_heads, head_dim] f32, or latent_dim for FP4). The library
+ * keeps two copy streams for the cache (created at the first call, released by
+ * kvq_cache_destroy). The copies of K, V and q run on the first, into the input slot of `staging`
+ * the step two calls back has finished with, so they overlap the previous step; the step waits
+ * for them on `stream`. The copy of out back to host memory runs on the second stream once the
+ * step is done, from one of two output slots, so it overlaps the next step. The call returns
+ * without waiting. out_event NULL: `stream` also waits for that output copy, and out is valid
+ * once `stream` has reached the end of the call's work. out_event a caller-created cudaEvent_t
+ * (passed as void*): the library records it after the output copy and `stream` does not wait;
+ * out is valid once the event has completed (cudaEventSynchronize, or a stream waiting on it).
+ * staging: device, 16-byte aligned, at least
  * kvq_step_staging_bytes, used by nothing else while steps are in flight. Host inputs must be
  * complete when the call is made (not pending writes of GPU work) and unchanged until `stream`
  * has passed the call; pinned (page-locked) memory keeps the copies asynchronous, pageable memory
@@ -187,7 +213,7 @@ kvq_status kvq_step_staging_bytes(const kvq_cache* c, kvq_dtype dtype, size_t* b
  * loop to one call per step. */
 kvq_status kvq_decode_step_host(kvq_cache* c, const void* K, const void* V, const void* q, kvq_dtype dtype,
                                 float* out, void* staging, size_t staging_bytes, void* workspace,
-                                size_t ws_bytes, void* stream);
+                                size_t ws_bytes, void* stream, void* out_event);
 
 /* The same decode attention as kvq_decode_attention, for callers that cannot allocate device
  * memory on the decode path (serving loops that reserve all memory up front, hosts whose memory

@@ -75,6 +75,32 @@ def softmax_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float)
     return (w[:, None] * V).sum(axis=0) / w.sum()
 
 
+def softmax_state(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float):
+    """Softmax state of attention over one part of a context, fp64: (m, l, o) with
+    m = max_t l_t, l = sum_t exp(l_t - m), o = sum_t exp(l_t - m) V_t, l_t = scale <q, K_t>.
+    A part with no tokens has the state (-inf, 0, 0)."""
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    if K.shape[0] == 0:
+        return -math.inf, 0.0, np.zeros(V.shape[1])
+    logits = scale * (K @ np.asarray(q, dtype=np.float64))
+    m = float(np.max(logits))
+    w = np.exp(logits - m)
+    return m, float(w.sum()), (w[:, None] * V).sum(axis=0)
+
+
+def merge_softmax_states(states):
+    """Softmax attention over the union of disjoint context parts from their states:
+    out = sum_i exp(m_i - M) o_i / sum_i exp(m_i - M) l_i, M = max_i m_i (zeros if every part is
+    empty)."""
+    M = max(m for m, _, _ in states)
+    if M == -math.inf:
+        return np.zeros_like(states[0][2])
+    num = sum(math.exp(m - M) * o for m, _, o in states if m != -math.inf)
+    den = sum(math.exp(m - M) * l for m, l, _ in states if m != -math.inf)
+    return num / den
+
+
 def decode_attention(q_heads: np.ndarray, K_hat: np.ndarray, V_hat: np.ndarray,
                      scale: float) -> np.ndarray:
     """GQA decode for one (sequence, kv-head): every query head of the group attends to the same

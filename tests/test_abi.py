@@ -147,7 +147,7 @@ int main(void) {
   if (kvq_lloyd_max_table(2, c, t) != KVQ_OK) return 1;
   if (kvq_lloyd_max_table(4, c, t) != KVQ_ERR_INVALID_ARG) return 2;
   if (kvq_packed_bytes_per_token(&cfg, &bytes) != KVQ_OK) return 3;
-  if (kvq_decode_step_host(NULL, NULL, NULL, NULL, KVQ_BF16, NULL, NULL, 0, NULL, 0, NULL) != KVQ_ERR_INVALID_ARG) return 4;
+  if (kvq_decode_step_host(NULL, NULL, NULL, NULL, KVQ_BF16, NULL, NULL, 0, NULL, 0, NULL, NULL) != KVQ_ERR_INVALID_ARG) return 4;
   /* the seeded draws a cache makes from cfg.rot_seed / cfg.qjl_seed when given no arrays */
   cfg.rot_seed = 0x5EED00A4ull; cfg.qjl_seed = 0x5EED005Bull;
   {

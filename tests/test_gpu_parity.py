@@ -350,9 +350,14 @@ def test_decode_step_host_equals_device_step(name, pinned):
         refs.append(c1.step(na, nv, data["q"]).clone())
         keep.append((host(na), host(nv), host(data["q"])))
     torch.cuda.synchronize()
+    # odd steps hand the library an event to record after the output copy (the stream does not
+    # wait for that copy); even steps let the stream wait for it
+    events = [torch.cuda.Event() if step % 2 else None for step in range(4)]
     for step in range(4):
         outs.append(host(torch.empty(refs[0].shape, dtype=torch.float32)))
-        c2.step_host(*keep[step], outs[step])
+        c2.step_host(*keep[step], outs[step], out_event=events[step])
+    events[3].synchronize()
+    assert torch.equal(outs[3], refs[3].cpu()), (name, 3)
     torch.cuda.synchronize()
     for step in range(4):
         assert torch.equal(outs[step], refs[step].cpu()), (name, step)
@@ -457,3 +462,74 @@ def test_per_head_rotation_parity():
     run_small("llama8b", 2, [300, 97], seed_appends=2, w=w)
     w70 = WORKLOADS["llama70b"].with_(rot_per_head=True)
     run_small("llama70b", 1, [260], w=w70)
+
+
+# ---------------------------------------------------------------- prefill-rate quantize
+
+@pytest.mark.parametrize("name", ["llama8b", "llama70b", "onebit"])
+def test_tile_quantize_equals_token_by_token(name):
+    """Appends of many tokens (whole tiles built in shared memory, 16-byte stores) store the same
+    codes and norms as token-by-token appends (per-vector kernel, atomics), also for tiles a call
+    only partly covers; sketch sign bits may differ only where the two fp32 summation orders
+    disagree on a projection's sign, which the oracle parity bounds, here at most 1e-3 of them."""
+    w = WORKLOADS[name].with_(batch=2)
+    data = generate(w, DEV, seqs=range(2), ctx=150)
+    tiles, tokens = new_cache(w, 2, 192)[0], new_cache(w, 2, 192)[0]
+    # tile path: 37 tokens (a partial tile), then 113 more (starting inside that tile)
+    for a, e in ((0, 37), (37, 150)):
+        tiles.quantize(data["k"][:, :, a:e].contiguous(), data["v"][:, :, a:e].contiguous())
+    for t in range(150):
+        tokens.quantize(data["k"][:, :, t:t + 1].contiguous(), data["v"][:, :, t:t + 1].contiguous())
+    torch.cuda.synchronize()
+    A, B = tiles.arena.cpu().numpy(), tokens.arena.cpu().numpy()
+    info = tiles.layout()
+    assert list(tiles.lengths()) == list(tokens.lengths()) == [150, 150]
+    flips = bits = 0
+    for pair in range(2 * w.n_kv_heads):
+        for side in (0, 1):
+            pa, sa, na, ga = side_fields(A, info, side, pair, 150)
+            pb, sb, nb, gb = side_fields(B, info, side, pair, 150)
+            np.testing.assert_array_equal(pa, pb)
+            np.testing.assert_array_equal(na, nb)
+            if sa is not None:
+                np.testing.assert_array_equal(ga, gb)
+                d = np.unpackbits(np.bitwise_xor(sa, sb).view(np.uint8))
+                flips += int(d.sum())
+                bits += d.size
+    assert flips <= 1e-3 * max(bits, 1), (flips, bits)
+    tiles.close()
+    tokens.close()
+
+
+# ---------------------------------------------------------------- the two LM decode kernels
+
+@pytest.mark.parametrize("name,lens", [("llama8b", [700, 65]), ("llama70b", [1000, 129]), ("onebit", [300, 1])])
+def test_mma_sync_kernel_parity(name, lens, monkeypatch):
+    """The mma.sync decode kernel (chosen with KVQ_DECODE_KERNEL=mma at cache creation) against the
+    oracle, as the tcgen05 kernel is by default."""
+    monkeypatch.setenv("KVQ_DECODE_KERNEL", "mma")
+    run_small(name, len(lens), lens, seed_appends=2)
+
+
+@pytest.mark.parametrize("name", ["llama8b", "llama70b", "onebit"])
+def test_tcgen05_and_mma_sync_kernels_agree(name, monkeypatch):
+    """Both LM decode kernels on the same cache contents: outputs within the attention tolerance of
+    each other, over contexts that span several iterations with a ragged tail."""
+    w = WORKLOADS[name].with_(batch=3)
+    lens = [1500, 700, 64]
+    data = generate(w, DEV, seqs=range(3), ctx=max(lens))
+    monkeypatch.setenv("KVQ_DECODE_KERNEL", "mma")
+    c_mma = new_cache(w, 3, 1536)[0]
+    monkeypatch.delenv("KVQ_DECODE_KERNEL")
+    c_tc = new_cache(w, 3, 1536)[0]
+    for c in (c_mma, c_tc):
+        for b, L in enumerate(lens):
+            c.quantize(data["k"][b:b + 1, :, :L].contiguous(), data["v"][b:b + 1, :, :L].contiguous(), seq_ids=[b])
+    a = f64(c_mma.decode(data["q"]))
+    t = f64(c_tc.decode(data["q"]))
+    torch.cuda.synchronize()
+    assert np.array_equal(c_mma.arena.cpu().numpy(), c_tc.arena.cpu().numpy())
+    err = rel_err(t.reshape(-1, t.shape[-1]), a.reshape(-1, a.shape[-1]))
+    assert np.all(err <= REL_TOL), err.max()
+    c_mma.close()
+    c_tc.close()

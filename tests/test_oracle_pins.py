@@ -527,3 +527,27 @@ def test_mla_hand_worked_cases_reject_plausible_mistakes(golden):
     assert _mla_matches_golden(attention.mla_decode_attention, golden)
     for bad in (dropped_rope, rope_in_values, latent_only_scale, sign_dropped):
         assert not _mla_matches_golden(bad, golden), bad.__name__
+
+
+# ---------------------------------------------------------------- context-parallel merge
+
+def test_merged_softmax_states_equal_attention_over_the_union():
+    """Splitting a context into disjoint parts (including empty ones and a part of one token) and
+    merging the parts' softmax states reproduces attention over the whole context (a closed-form
+    identity of the softmax); a single part reproduces it trivially; all-empty gives zeros."""
+    rng = np.random.default_rng(31)
+    T, d = 97, 16
+    K = rng.standard_normal((T, d)) * 3
+    V = rng.standard_normal((T, 5))
+    q = rng.standard_normal(d)
+    full = attention.softmax_attention(q, K, V, 0.7)
+    for cuts in ([0, 97], [0, 40, 97], [0, 0, 1, 50, 50, 97], [0, 96, 97]):
+        states = [attention.softmax_state(q, K[a:b], V[a:b], 0.7) for a, b in zip(cuts[:-1], cuts[1:])]
+        np.testing.assert_allclose(attention.merge_softmax_states(states), full, rtol=1e-12, atol=1e-14)
+    m, l, o = attention.softmax_state(q, K[:0], V[:0], 0.7)
+    assert m == -math.inf and l == 0.0 and np.all(o == 0)
+    assert np.all(attention.merge_softmax_states([(m, l, o), (m, l, o)]) == 0)
+    # a planted mistake: merging without the exp(m_i - M) weights fails the identity
+    states = [attention.softmax_state(q, K[a:b], V[a:b], 0.7) for a, b in ((0, 40), (40, 97))]
+    wrong = sum(o for _, _, o in states) / sum(l for _, l, _ in states)
+    assert not np.allclose(wrong, full, rtol=1e-6)
