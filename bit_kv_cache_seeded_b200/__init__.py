@@ -52,7 +52,8 @@ class kvq_cfg(ctypes.Structure):
                 ("v_bits", ctypes.c_int32), ("qjl_dim", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("latent_dim", ctypes.c_int32),
                 ("rope_dim", ctypes.c_int32), ("rot_per_head", ctypes.c_int32),
-                ("rot_seed", ctypes.c_uint64), ("qjl_seed", ctypes.c_uint64)]
+                ("rot_seed", ctypes.c_uint64), ("qjl_seed", ctypes.c_uint64),
+                ("sink_tokens", ctypes.c_int32), ("recent_tokens", ctypes.c_int32)]
 
 
 _lib = None
@@ -127,9 +128,10 @@ def _stream(stream=None):
 
 def make_cfg(head_dim=128, n_q_heads=1, n_kv_heads=1, k_mode="lm_qjl", v_mode="lm_qjl", k_bits=2,
              v_bits=2, qjl_dim=128, softmax_scale=0.0, latent_dim=0, rope_dim=0, rot_per_head=0,
-             rot_seed=0, qjl_seed=0) -> kvq_cfg:
+             rot_seed=0, qjl_seed=0, sink_tokens=0, recent_tokens=0) -> kvq_cfg:
     return kvq_cfg(head_dim, n_q_heads, n_kv_heads, MODES[k_mode], MODES[v_mode], k_bits, v_bits,
-                   qjl_dim, softmax_scale, latent_dim, rope_dim, int(rot_per_head), rot_seed, qjl_seed)
+                   qjl_dim, softmax_scale, latent_dim, rope_dim, int(rot_per_head), rot_seed, qjl_seed,
+                   sink_tokens, recent_tokens)
 
 
 def cfg_for_workload(w) -> kvq_cfg:
@@ -140,7 +142,8 @@ def cfg_for_workload(w) -> kvq_cfg:
                         rope_dim=w.rope_dim)
     return make_cfg(w.head_dim, w.n_q_heads, w.n_kv_heads, w.k_mode, w.v_mode, w.k_bits, w.v_bits,
                     w.qjl_dim, rot_per_head=int(getattr(w, "rot_per_head", False)), rot_seed=w.rot_seed,
-                    qjl_seed=w.qjl_seed)
+                    qjl_seed=w.qjl_seed, sink_tokens=getattr(w, "sink_tokens", 0),
+                    recent_tokens=getattr(w, "recent_tokens", 0))
 
 
 def kvq_draw_rotation_signs(seed: int, n: int) -> np.ndarray:
@@ -359,8 +362,8 @@ def kvq_cache_lengths(handle, batch: int) -> np.ndarray:
 
 
 def kvq_cache_layout(handle) -> np.ndarray:
-    info = np.zeros(18, dtype=np.int64)
-    _check("kvq_cache_layout", load().kvq_cache_layout(handle, info.ctypes.data_as(ctypes.c_void_p), 18))
+    info = np.zeros(22, dtype=np.int64)
+    _check("kvq_cache_layout", load().kvq_cache_layout(handle, info.ctypes.data_as(ctypes.c_void_p), 22))
     return info
 
 

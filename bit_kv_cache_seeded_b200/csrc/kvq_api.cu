@@ -31,8 +31,11 @@ kvq_status validate_cfg(const kvq_cfg* c) {
   if (c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->n_q_heads % c->n_kv_heads) return KVQ_ERR_INVALID_ARG;
   if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return KVQ_ERR_INVALID_ARG;
   if (c->rot_per_head != 0 && c->rot_per_head != 1) return KVQ_ERR_INVALID_ARG;
+  if (c->sink_tokens < 0 || c->recent_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  if (c->sink_tokens + (long)c->recent_tokens > 1024) return KVQ_ERR_UNSUPPORTED;
   if (c->k_mode == KVQ_MODE_FP4 || c->v_mode == KVQ_MODE_FP4) {
     if (c->rot_per_head) return KVQ_ERR_INVALID_ARG;  // the FP4 latent is not rotated
+    if (c->sink_tokens || c->recent_tokens) return KVQ_ERR_UNSUPPORTED;
     if (c->k_mode != KVQ_MODE_FP4 || c->v_mode != KVQ_MODE_FP4) return KVQ_ERR_INVALID_ARG;
     if (c->n_kv_heads != 1) return KVQ_ERR_INVALID_ARG;
     if (c->latent_dim <= 0 || c->rope_dim < 0) return KVQ_ERR_INVALID_ARG;
@@ -92,7 +95,7 @@ Fp4Layout make_fp4(int latent, int rope) {
 }
 
 struct Plan {
-  size_t lens_off, signs_off, S_off, St_off, k_off, v_off, total;
+  size_t lens_off, signs_off, S_off, St_off, k_off, v_off, win_off, total;
   SideLayout k, v;
   Fp4Layout fp4;
   bool fp4_mode;
@@ -104,8 +107,8 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
   P.fp4_mode = c->k_mode == KVQ_MODE_FP4;
   P.tiles = (capacity + kTile * kTilePair - 1) / (kTile * kTilePair) * kTilePair;
   size_t off = 0;
-  P.lens_off = off;
-  off = align_up(off + sizeof(int) * ((size_t)batch + kStatusWords), kArenaAlign);
+  P.lens_off = off;  // lengths, status words, history lengths (window caches)
+  off = align_up(off + sizeof(int) * (2 * (size_t)batch + kStatusWords), kArenaAlign);
   const size_t pairs = (size_t)batch * c->n_kv_heads;
   if (P.fp4_mode) {
     P.fp4 = make_fp4(c->latent_dim, c->rope_dim);
@@ -129,6 +132,9 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
     off = align_up(off + pairs * P.tiles * (size_t)P.k.tile_bytes, kArenaAlign);
     P.v_off = off;
     off = align_up(off + pairs * P.tiles * (size_t)P.v.tile_bytes, kArenaAlign);
+    // mixed-precision window: bf16 K then V, [pairs][sink + recent][d] each
+    P.win_off = off;
+    off = align_up(off + 2 * pairs * ((size_t)c->sink_tokens + c->recent_tokens) * kHeadDim * 2, kArenaAlign);
   }
   P.total = off;
   return P;
@@ -182,9 +188,24 @@ size_t partials_bytes(const kvq_cache* c, int splits) {
 }
 
 // Workspace = split partials, then the per-(sequence, kv-head) query tables of the tensor-core path.
-size_t workspace_for(const kvq_cache* c, int splits) {
-  return partials_bytes(c, splits) + (size_t)c->batch * c->cfg.n_kv_heads * prep_stride(c);
+bool has_window(const kvq_cache* c) { return c->sink > 0 || c->recent > 0; }
+
+// Bytes of the window's softmax states [B][Hq][part_stride] (window caches), 256-aligned.
+size_t window_state_bytes(const kvq_cache* c) {
+  return has_window(c) ? align_up(sizeof(float) * (size_t)c->batch * c->cfg.n_q_heads * part_stride(c), 256) : 0;
 }
+
+// Workspace = split partials, the per-(sequence, kv-head) query tables of the tensor-core paths,
+// the window's softmax states.
+size_t prep_bytes_total(const kvq_cache* c) {
+  return align_up((size_t)c->batch * c->cfg.n_kv_heads * prep_stride(c), 256);
+}
+size_t workspace_for(const kvq_cache* c, int splits) {
+  return partials_bytes(c, splits) + prep_bytes_total(c) + window_state_bytes(c);
+}
+
+// The lengths the split plan and the split kernels see: the coded history on window caches.
+const std::vector<int>& coded_lens(const kvq_cache* c) { return has_window(c) ? c->hlens : c->lens; }
 
 // Resident decode CTAs per SM for a chunk of `units` 64-token units: one for the MLA kernel, the
 // tensor-core kernel's shared-memory and register limit for query groups of 1, 2 or 4, else 4.
@@ -335,7 +356,12 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
   c->signs_stride = cfg->rot_per_head ? kHeadDim : 0;
   c->tc = !P.fp4_mode && choose_tc(*cfg, P.k, P.v);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(c->d_lens, 0, sizeof(int) * ((size_t)batch + kStatusWords), s) != cudaSuccess) {
+  c->sink = P.fp4_mode ? 0 : cfg->sink_tokens;
+  c->recent = P.fp4_mode ? 0 : cfg->recent_tokens;
+  c->d_hlens = c->d_status + kStatusWords;
+  c->hlens.assign(batch, 0);
+  if (!P.fp4_mode) c->d_win = reinterpret_cast<uint16_t*>(c->dev + P.win_off);
+  if (cudaMemsetAsync(c->d_lens, 0, sizeof(int) * (2 * (size_t)batch + kStatusWords), s) != cudaSuccess) {
     delete c;
     return KVQ_ERR_CUDA;
   }
@@ -404,6 +430,48 @@ void fill_quantize(QuantizeParams& p, const kvq_cache* c, const void* K, const v
 }
 }  // namespace
 
+namespace {
+// Append to a mixed-precision window cache: per launch of up to kMaxSeqPerLaunch sequences, first
+// code the tokens that leave the window into the history (from the bf16 ring, or from the input when
+// the call appends more tokens than the window holds), then write the new tokens that stay in the
+// window. Sequence slots [first, first + cnt) of the call.
+kvq_status quantize_window(kvq_cache* c, const void* K, const void* V, kvq_dtype dtype, int n_new,
+                           const int32_t* seq_ids, int first, int cnt, cudaStream_t s) {
+  QuantizeParams p;
+  fill_quantize(p, c, K, V, dtype, n_new, seq_ids, first, cnt);
+  const size_t pairs_kv = (size_t)c->batch * c->cfg.n_kv_heads;
+  const int slots = c->sink + c->recent;
+  p.ring[0] = c->d_win;
+  p.ring[1] = c->d_win + pairs_kv * (size_t)slots * kHeadDim;
+  p.win_sink = c->sink;
+  p.win_recent = c->recent;
+  p.win_slots = slots;
+  p.src_rows = n_new;
+  int max_cnt = 0;
+  std::vector<int> h1(cnt);
+  for (int i = 0; i < cnt; ++i) {
+    const int T0 = c->lens[p.seq[i]], T1 = T0 + n_new;
+    const int H0 = std::max(0, T0 - c->recent - c->sink);
+    h1[i] = std::max(0, T1 - c->recent - c->sink);
+    p.total0[i] = T0;
+    p.pos[i] = H0;
+    p.cnt[i] = h1[i] - H0;
+    max_cnt = std::max(max_cnt, p.cnt[i]);
+  }
+  if (max_cnt > 0) {  // history appends (reads the ring before the window write below overwrites it)
+    QuantizeParams ph = p;
+    ph.win_src = 1;
+    ph.n_new = max_cnt;
+    ph.lens = c->d_hlens;
+    if (launch_quantize_lm(ph, 2, s) != cudaSuccess) return KVQ_ERR_CUDA;
+    for (int i = 0; i < cnt; ++i) c->hlens[p.seq[i]] = h1[i];
+  }
+  if (launch_window_write(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  for (int i = 0; i < cnt; ++i) c->lens[p.seq[i]] += n_new;
+  return KVQ_OK;
+}
+}  // namespace
+
 extern "C" {
 
 kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dtype,
@@ -426,6 +494,11 @@ kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dt
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   for (int first = 0; first < n_seq; first += kMaxSeqPerLaunch) {
     const int cnt = std::min(kMaxSeqPerLaunch, n_seq - first);
+    if (has_window(c)) {
+      const kvq_status st = quantize_window(c, K, V, dtype, n_new, seq_ids, first, cnt, s);
+      if (st != KVQ_OK) return st;
+      continue;
+    }
     QuantizeParams p;
     fill_quantize(p, c, K, V, dtype, n_new, seq_ids, first, cnt);
     const cudaError_t e = c->is_fp4 ? launch_quantize_fp4(p, s) : launch_quantize_lm(p, 2, s);
@@ -456,7 +529,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
     return KVQ_ERR_ALIGNMENT;
   if (!on_cache_device(c)) return KVQ_ERR_INVALID_ARG;
   int max_len = 0;
-  for (int v : c->lens) max_len = std::max(max_len, v);
+  for (int v : coded_lens(c)) max_len = std::max(max_len, v);
   const int pairs = decode_rows(c);
   int splits, chunk;
   plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len,
@@ -503,7 +576,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.group = p.Hq / p.Hkv;
   p.splits = splits;
   p.chunk = chunk;
-  p.lens = c->d_lens;
+  p.lens = has_window(c) ? c->d_hlens : c->d_lens;
   p.kreg = c->d_k;
   p.vreg = c->d_v;
   p.tiles_per_seq = c->tiles_per_seq;
@@ -521,6 +594,17 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.wait_limit = wait_limit;
   p.debug_unset_wait = debug_unset_wait;
   p.use_tc = c->tc ? 1 : 0;
+  if (has_window(c)) {
+    const size_t pairs_kv = (size_t)c->batch * c->cfg.n_kv_heads;
+    p.wk = c->d_win;
+    p.wv = c->d_win + pairs_kv * (size_t)(c->sink + c->recent) * kHeadDim;
+    p.win_sink = c->sink;
+    p.win_recent = c->recent;
+    p.win_slots = c->sink + c->recent;
+    p.tot_lens = c->d_lens;
+    p.wpart = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + partials_bytes(c, splits) +
+                                       prep_bytes_total(c));
+  }
   const bool tensor_path = p.use_tc ? tc_decode_supported(p) : mma_decode_supported(p);
   if (qp && !tensor_path) {  // no fused front kernel on this path: append first
     if (launch_quantize_lm(*qp, 2, s) != cudaSuccess) return KVQ_ERR_CUDA;
@@ -529,6 +613,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.cache_after_wait = qp != nullptr;
   if (debug_unset_wait && !tensor_path) return KVQ_ERR_UNSUPPORTED;
   if (launch_decode_lm(p, s, ev ? ev[1] : nullptr, qp) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
+  if (p.wpart && launch_window_decode(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
   if (launch_reduce_lm(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }
@@ -575,14 +660,14 @@ kvq_status kvq_decode_step(kvq_cache* c, const void* K, const void* V, const voi
   int max_len = 0;
   for (int v : c->lens) {
     if ((long)v + 1 > (long)c->capacity) return KVQ_ERR_CAPACITY;
-    max_len = std::max(max_len, v);
   }
+  for (int v : coded_lens(c)) max_len = std::max(max_len, v);
   const int pairs = decode_rows(c);
   int splits, chunk;
   plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len + 1,
               &splits, &chunk);
   if (ws_bytes < workspace_for(c, splits)) return KVQ_ERR_WORKSPACE;
-  if (c->is_fp4 || c->batch > kMaxSeqPerLaunch) {  // no fused front kernel: the two calls in sequence
+  if (c->is_fp4 || c->batch > kMaxSeqPerLaunch || has_window(c)) {  // no fused front kernel: the two calls in sequence
     const kvq_status st = kvq_quantize(c, K, V, dtype, 1, nullptr, c->batch, stream);
     if (st != KVQ_OK) return st;
     return decode_impl(c, q, dtype, out, workspace, ws_bytes, stream, 0, kWaitLimitCycles);
@@ -699,10 +784,9 @@ kvq_status kvq_decode_step_host(kvq_cache* c, const void* K, const void* V, cons
   if (staging_bytes < S.total) return KVQ_ERR_INVALID_ARG;
   // what kvq_decode_step would refuse, refused before any copy
   int max_len = 0;
-  for (int v : c->lens) {
+  for (int v : c->lens)
     if ((long)v + 1 > (long)c->capacity) return KVQ_ERR_CAPACITY;
-    max_len = std::max(max_len, v);
-  }
+  for (int v : coded_lens(c)) max_len = std::max(max_len, v);
   int splits, chunk;
   plan_splits(decode_rows(c), c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c),
               decode_waves_bound(c), max_len + 1, &splits, &chunk);
@@ -774,6 +858,12 @@ kvq_status kvq_cache_layout(const kvq_cache* c, int64_t* info, int32_t n_info) {
   if (n_info > 16) info[16] = c->is_fp4 ? 0 : c->k.order;
   if (n_info > 17) info[17] = c->is_fp4 ? 0 : c->v.order;
   for (int i = 18; i < n_info; ++i) info[i] = 0;
+  if (n_info > 21) {
+    info[18] = c->d_win ? (int64_t)(reinterpret_cast<char*>(c->d_win) - c->dev) : 0;
+    info[19] = c->sink + c->recent;
+    info[20] = c->sink;
+    info[21] = c->recent;
+  }
   info[0] = kTile;
   info[1] = c->is_fp4 ? c->fp4.tile_bytes : c->k.tile_bytes;
   info[2] = c->is_fp4 ? 0 : c->v.tile_bytes;
@@ -892,7 +982,7 @@ extern "C" kvq_status kvq_decode_attention_static(const kvq_cache* c, const void
   if (!c || !q || !out) return KVQ_ERR_INVALID_ARG;
   if (!on_cache_device(c)) return KVQ_ERR_INVALID_ARG;
   int max_len = 0;
-  for (int v : c->lens) max_len = std::max(max_len, v);
+  for (int v : coded_lens(c)) max_len = std::max(max_len, v);
   const int pairs = decode_rows(c);
   int splits, chunk;
   plan_splits(pairs, c->sms, [c](int u) { return decode_slots_per_sm(c, u); }, decode_max_units(c), decode_waves_bound(c), max_len,

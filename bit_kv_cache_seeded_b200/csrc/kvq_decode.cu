@@ -306,6 +306,15 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
     }
     M = mn;
   }
+  if (p.wpart) {  // the mixed-precision window's state, one more part of the same softmax
+    const float* ws = p.wpart + ((size_t)b * p.Hq + hk * G + h) * p.part_stride;
+    const float wm = __ldcg(ws), mn = fmaxf(M, wm);
+    const float c = exp2_diff(M, mn), w = exp2_diff(wm, mn);
+    L = fmaf(w, __ldcg(ws + 1), L * c);
+    o = fmaf(w, __ldcg(ws + 2 + i), o * c);
+    oz = fmaf(w, vq ? __ldcg(ws + 2 + kHeadDim + i) : 0.f, oz * c);
+    M = mn;
+  }
   // the normalisation by L, unless the call asks for the merged softmax state (m, l, unnormalised
   // o), whose Sᵀ fold and inverse rotation are linear and apply the same way
   const float inv = p.pout ? 1.f : (L > 0.f) ? 1.f / L : 0.f;

@@ -76,6 +76,15 @@ struct QuantizeParams {
   long long wait_limit;  // SM clock cycles a block waits for staged data before giving up
   int seq[kMaxSeqPerLaunch];
   int pos[kMaxSeqPerLaunch];
+  // Mixed-precision window caches. History appends (win_src): sequence s takes cnt[s] tokens, history
+  // positions pos[s] ..; the token at sequence position sink + pos[s] + t comes from the bf16 ring
+  // when it is below total0[s] (the length before the call), else from input row
+  // (that position - total0[s]) of the call's src_rows rows. Window writes use total0 the same way.
+  int win_src;
+  const uint16_t* ring[2];  // bf16 window of K and V: [n_seq][heads][win_slots][d]
+  int win_sink, win_recent, win_slots, src_rows;
+  int total0[kMaxSeqPerLaunch];
+  int cnt[kMaxSeqPerLaunch];
 };
 
 struct DecodeParams {
@@ -105,6 +114,14 @@ struct DecodeParams {
   int debug_unset_wait;   // test entry: also wait once on a barrier nothing completes
   int cache_after_wait;   // fused step: the cache is written by this kernel's predecessor (wait first)
   int use_tc;             // decode on the tcgen05 kernel (one CTA per sequence, kv-head and split)
+  // mixed-precision window: bf16 K and V of the sink and recent tokens, [B][Hkv][win_slots][d] each;
+  // lens above counts the coded history only, tot_lens every token; wpart [B][Hq][part_stride] gets
+  // the window's softmax state, which the reduce merges with the splits' (null: no window)
+  const uint16_t* wk;
+  const uint16_t* wv;
+  int win_sink, win_recent, win_slots;
+  const int* tot_lens;
+  float* wpart;
 };
 
 struct MlaParams {
@@ -161,6 +178,10 @@ cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s);
 bool mla_mma_supported(const MlaParams& p);
 bool mla_umma_supported(const MlaParams& p);
 // Log-sum-exp merge of n_parts softmax states [n_parts][rows][2 + dv] into out [rows][dv] (kvq_combine.cu).
+// Mixed-precision window (kvq_window.cu): bf16 writes of appended tokens that stay in the window,
+// and the window's softmax state for decode.
+cudaError_t launch_window_write(const QuantizeParams& p, cudaStream_t s);
+cudaError_t launch_window_decode(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_combine_partials(const float* parts, int n_parts, int rows, int dv, float* out, cudaStream_t s);
 cudaError_t launch_decode_mla_umma(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_decode_mla_mma(const MlaParams& p, cudaStream_t s);
@@ -177,6 +198,10 @@ struct kvq_cache {
   int signs_stride = 0;     // 0, or kHeadDim when every kv-head has its own rotation diagonal
   int device = -1;          // the CUDA device whose memory holds the arena (current at init)
   bool tc = false;          // LM decode runs on the tcgen05 kernel (else mma.sync / CUDA cores)
+  int sink = 0, recent = 0; // mixed-precision window (0, 0: none)
+  int* d_hlens = nullptr;   // window caches: coded history length per sequence (the decode kernels' lens)
+  uint16_t* d_win = nullptr;// window caches: bf16 K then V window, [batch][kv-heads][sink + recent][d] each
+  std::vector<int> hlens;   // host mirror of d_hlens
   char* dev = nullptr;
   size_t dev_bytes = 0;
   int* d_lens = nullptr;

@@ -27,6 +27,27 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 constexpr int kLmWarps = 4;     // LM quantize: warps per block
 
+// Where vector t of sequence slot s, head h of an LM quantize call starts, and whether it is bf16.
+// Plain calls: row t of the [n_seq, heads, n_new, d] input. History appends of a window cache: the
+// token at sequence position sink + pos[s] + t, from the bf16 ring below the old length, else from
+// the input (rows of src_rows per (sequence, head)).
+__device__ __forceinline__ const void* vector_src(const QuantizeParams& p, int side, int s, int h, int t, int& bf16) {
+  bf16 = p.bf16;
+  if (!p.win_src) {
+    const size_t elem = p.bf16 ? 2 : 4;
+    return static_cast<const char*>(p.src[side]) + ((((size_t)s * p.heads + h) * p.n_new + t) * kHeadDim) * elem;
+  }
+  const int pos = p.win_sink + p.pos[s] + t;
+  if (pos < p.total0[s]) {
+    bf16 = 1;
+    const int slot = p.win_sink + (pos - p.win_sink) % p.win_recent;
+    return p.ring[side] + (((size_t)p.seq[s] * p.heads + h) * p.win_slots + slot) * kHeadDim;
+  }
+  const size_t elem = p.bf16 ? 2 : 4;
+  return static_cast<const char*>(p.src[side]) +
+         ((((size_t)s * p.heads + h) * p.src_rows + (pos - p.total0[s])) * kHeadDim) * elem;
+}
+
 // Bits 0..3 of x moved to bits 0, 8, 16, 24.
 __device__ __forceinline__ uint32_t spread_nibble(uint32_t x) {
   return (x & 1u) | ((x & 2u) << 7) | ((x & 4u) << 14) | ((x & 8u) << 21);
@@ -80,9 +101,10 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
   // cache's own constants; the inputs may come from the preceding kernel, so wait for it here.
   grid_dep_wait();
   float u_first[4] = {0.f, 0.f, 0.f, 0.f};
-  if (first < total)
+  if (first < total && !p.win_src)
 #pragma unroll
     for (int k = 0; k < 4; ++k) u_first[k] = load_elem(p.src[side], (size_t)first * kHeadDim + 32 * k + lane, p.bf16);
+  bool block_synced = false;  // the block barrier before the first wait for S^T has been passed
   float sg[4];  // rotation signs (the debug entry's inputs are already rotated: none read)
   int sg_head = 0;  // the head whose diagonal sg holds (per-head rotation)
   if (first < total) sg_head = (int)((first / p.n_new) % p.heads);
@@ -98,11 +120,18 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
     const int t = (int)(vec % p.n_new);
     const int h = (int)((vec / p.n_new) % p.heads);
     const int s = (int)(vec / ((long)p.n_new * p.heads));
-    const size_t base = (size_t)vec * kHeadDim;  // [n_seq, heads, n_new, d] row-major
+    if (p.win_src && t >= p.cnt[s]) continue;  // uniform over the vector's warp (block: coop sides)
 
     float u[4];
+    if (vec == first && !p.win_src) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) u[k] = (vec == first) ? u_first[k] : load_elem(p.src[side], base + 32 * k + lane, p.bf16);
+      for (int k = 0; k < 4; ++k) u[k] = u_first[k];
+    } else {
+      int vb16;
+      const void* src = vector_src(p, side, s, h, t, vb16);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) u[k] = load_elem(src, 32 * k + lane, vb16);
+    }
 
     if (p.signs_stride && h != sg_head && !p.skip_rotation) {  // per-head rotation: this head's diagonal
       sg_head = h;
@@ -159,11 +188,13 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
 #pragma unroll
       for (int k = 0; k < 4; ++k) rho_s[warp][32 * k + lane] = rho[k];
       __syncwarp();
-      if (vec == first) __syncthreads();  // st_bar was initialised (by thread 0) before anyone waits
-      if (vec == first && !mbar_try(smem_addr(&st_bar), 0u) &&
-          !mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit)) {  // S^T (requested at the start)
-        st_failed = true;
-        atomicOr(p.err, 1);
+      if (!block_synced) {
+        __syncthreads();  // st_bar was initialised (by thread 0) before anyone waits
+        if (!mbar_try(smem_addr(&st_bar), 0u) && !mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit)) {
+          st_failed = true;  // S^T (requested at the start)
+          atomicOr(p.err, 1);
+        }
+        block_synced = true;
       }
       __syncwarp();
       float pr[4] = {0.f, 0.f, 0.f, 0.f};  // (S rho)_j, j = 32 warp + lane: four partial chains
@@ -245,10 +276,12 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
       *reinterpret_cast<__half*>(tb + L.off_gamma + slot * 2) = __float2half_rn(gamma);
   }
 
-  // a wait that gave up: the copy may still be landing, so wait for it (bounded) before leaving
-  if (st_failed) mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit);
+  // a wait that gave up: the copy may still be landing, so wait for it (bounded) before leaving; a
+  // staged block whose vectors were all skipped still waits for its copy
+  if (st_failed || (staged && !block_synced && threadIdx.x == 0)) mbar_wait(smem_addr(&st_bar), 0u, p.wait_limit);
   if (side == 0 && blk == 0 && !p.skip_rotation)
-    for (int i = threadIdx.x; i < p.n_seq; i += blockDim.x) p.lens[p.seq[i]] = p.pos[i] + p.n_new;
+    for (int i = threadIdx.x; i < p.n_seq; i += blockDim.x)
+      p.lens[p.seq[i]] = p.pos[i] + (p.win_src ? p.cnt[i] : p.n_new);
 }
 
 }  // namespace qlm

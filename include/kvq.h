@@ -89,6 +89,12 @@ typedef struct {
                            rot_signs): see kvq_draw_rotation_signs */
   uint64_t qjl_seed;    /* seed of the sketch matrix S (used when kvq_cache_init gets no qjl_matrix):
                            see kvq_draw_qjl_matrix */
+  int32_t sink_tokens;  /* LM/SIGN1 mixed-precision window ("TurboQuant vs OSCAR vs EpiCache", section
+                           "Quantization frontiers: TurboQuant and OSCAR": sink and recent tokens stay
+                           BF16, the history is quantized): the first sink_tokens tokens of a sequence */
+  int32_t recent_tokens;/* and its last recent_tokens tokens are kept as bf16 K and V; the tokens in
+                           between are coded as above. 0 and 0 = no window (every token coded).
+                           sink_tokens + recent_tokens <= 1024. FP4: both 0 */
 } kvq_cfg;
 
 typedef struct kvq_cache kvq_cache; /* opaque host object */
@@ -268,7 +274,10 @@ kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens);
  * info[0..15] receives: tile_tokens, k_tile_bytes, v_tile_bytes, tiles_per_seq,
  * k_region_offset, v_region_offset, then per side (K at 6, V at 11): planes_offset,
  * sketch_offset, norm_offset, gamma_offset, planes; with n_info >= 18 also info[16], info[17]:
- * the order of the K and V planes (0 byte-lane, 1 token, 2 octet). Layout of a tile (32 tokens)
+ * the order of the K and V planes (0 byte-lane, 1 token, 2 octet); with n_info >= 22 also info[18..21]:
+ * the byte offset of the mixed-precision window (bf16 K then V, [batch][n_kv_heads][slots][head_dim]
+ * each), slots = sink + recent, sink, recent (zeros without a window). On a window cache the tiles
+ * hold the coded history: history token i is sequence position sink + i. Layout of a tile (32 tokens)
  * of one (sequence, kv-head): code bit-planes (512 bytes each), then sign words (512 bytes),
  * then [32] fp16 norms, then [32] fp16 residual norms (sides with a sketch). Plane p holds bit p
  * of every code; a token's 128 bits of a plane are 16 bytes, byte k holding coordinates

@@ -51,6 +51,8 @@ class Workload:
     latent_dim: int = 0
     rope_dim: int = 0
     rot_per_head: bool = False  # one rotation diagonal per KV head
+    sink_tokens: int = 0        # mixed-precision window: first tokens kept in bf16
+    recent_tokens: int = 0      # and last tokens kept in bf16
 
     @property
     def data_seed(self) -> int:

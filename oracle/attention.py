@@ -150,6 +150,37 @@ def decode_attention_rotated(q_heads, codes_k, n16_k, gamma16_k, z_k, codes_v, n
     return np.stack(outs)
 
 
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round fp32/fp64 values to bfloat16 (round to nearest, ties to even), returned as fp64: the
+    precision the full-precision window of a mixed-precision cache keeps its tokens in."""
+    import torch
+    return torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def window_segments(T: int, sink: int, recent: int):
+    """Token ranges of a mixed-precision cache of T tokens ("TurboQuant vs OSCAR vs EpiCache",
+    section "Quantization frontiers: TurboQuant and OSCAR", OSCAR's mixed-precision paged memory:
+    sink tokens and recent tokens stay in BF16, the history in between is quantized):
+    sink = [0, min(T, sink)), history = [sink, max(sink, T - recent)), recent = [max(sink, T - recent), T)."""
+    s_end = min(T, sink)
+    r_begin = max(sink, T - recent) if T > sink else s_end
+    return (0, s_end), (s_end, max(s_end, r_begin)), (max(s_end, r_begin), T)
+
+
+def window_decode_attention(q_heads: np.ndarray, K: np.ndarray, V: np.ndarray, sink: int, recent: int,
+                            K_hist_hat: np.ndarray, V_hist_hat: np.ndarray, scale: float) -> np.ndarray:
+    """Decode over a mixed-precision cache: keys and values of the sink and recent tokens are the
+    inputs rounded to bf16, those of the history tokens are their dequantised estimates
+    (K_hist_hat / V_hist_hat, one row per history token in order); softmax attention over all of them.
+    q_heads [g, d], K, V [T, d] (inputs) -> out [g, d]."""
+    T = K.shape[0]
+    (s0, s1), (h0, h1), (r0, r1) = window_segments(T, sink, recent)
+    assert K_hist_hat.shape[0] == h1 - h0 and V_hist_hat.shape[0] == h1 - h0
+    Keff = np.concatenate([bf16_round(K[s0:s1]), np.asarray(K_hist_hat, np.float64), bf16_round(K[r0:r1])])
+    Veff = np.concatenate([bf16_round(V[s0:s1]), np.asarray(V_hist_hat, np.float64), bf16_round(V[r0:r1])])
+    return decode_attention(q_heads, Keff, Veff, scale)
+
+
 def fp4_dequantize_many(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
     """``fp4_dequantize`` applied to every row: packed uint8 [T, C/2], scales uint8 [T, C/16]
     -> [T, C], through the oracle's own E2M1/E4M3 decode tables."""

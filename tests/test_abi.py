@@ -241,10 +241,16 @@ def test_seeded_draws_are_the_generator_bit_for_bit(lib, seed):
 
 
 def test_cfg_struct_layout_matches_header(lib):
-    """The ctypes mirror of kvq_cfg has the C layout: 12 int32-sized fields, then two uint64 seeds."""
+    """The ctypes mirror of kvq_cfg has the C layout: 12 int32-sized fields, two uint64 seeds, then the
+    two window sizes."""
     import ctypes
-    assert ctypes.sizeof(kvq.kvq_cfg) == 64
+    assert ctypes.sizeof(kvq.kvq_cfg) == 72
     assert kvq.kvq_cfg.rot_seed.offset == 48 and kvq.kvq_cfg.qjl_seed.offset == 56
+    assert kvq.kvq_cfg.sink_tokens.offset == 64 and kvq.kvq_cfg.recent_tokens.offset == 68
+    with pytest.raises(kvq.KvqError):  # window over 1024 tokens
+        kvq.kvq_cache_bytes(kvq.make_cfg(sink_tokens=64, recent_tokens=1000), 1, 32)
+    assert kvq.kvq_cache_bytes(kvq.make_cfg(sink_tokens=64, recent_tokens=256), 2, 64) > \
+        kvq.kvq_cache_bytes(kvq.make_cfg(), 2, 64) + 2 * 2 * 320 * 128 * 2 - 1
     cfg = kvq.make_cfg(rot_per_head=2)
     with pytest.raises(kvq.KvqError):
         kvq.kvq_cache_bytes(cfg, 1, 32)

@@ -551,3 +551,49 @@ def test_merged_softmax_states_equal_attention_over_the_union():
     states = [attention.softmax_state(q, K[a:b], V[a:b], 0.7) for a, b in ((0, 40), (40, 97))]
     wrong = sum(o for _, _, o in states) / sum(l for _, l, _ in states)
     assert not np.allclose(wrong, full, rtol=1e-6)
+
+
+# ---------------------------------------------------------------- mixed-precision window
+
+def test_window_segments_partition_the_context():
+    for T in (0, 1, 31, 64, 65, 300, 320, 321, 5000):
+        for sink, recent in ((64, 256), (0, 32), (32, 0), (0, 0), (7, 9)):
+            (s0, s1), (h0, h1), (r0, r1) = attention.window_segments(T, sink, recent)
+            assert s0 == 0 and s1 == h0 and h1 == r0 and r1 == T
+            assert s1 - s0 == min(T, sink) and r1 - r0 <= recent and h1 - h0 == max(0, T - sink - recent)
+
+
+def test_window_fraction_matches_the_page():
+    """OSCAR keeps sink and recent tokens in BF16: "only 0.24% of tokens" at a 128k context (TQ
+    page, OSCAR bullet). The window this library uses by default, 64 sink + 256 recent tokens,
+    gives that fraction at 128 x 1024 tokens."""
+    (s0, s1), _, (r0, r1) = attention.window_segments(128 * 1024, 64, 256)
+    frac = 100.0 * ((s1 - s0) + (r1 - r0)) / (128 * 1024)
+    assert round(frac, 2) == 0.24
+
+
+def test_window_attention_special_cases():
+    """No window: the plain attention over the dequantised cache. Everything in the window: plain
+    attention over the bf16-rounded inputs (checked against torch's SDPA in fp64)."""
+    import torch
+    rng = np.random.default_rng(5)
+    T, d = 40, 8
+    K, V = rng.standard_normal((T, d)), rng.standard_normal((T, d))
+    Kh, Vh = K + 0.01 * rng.standard_normal((T, d)), V + 0.01 * rng.standard_normal((T, d))
+    q = rng.standard_normal((2, d))
+    out = attention.window_decode_attention(q, K, V, 0, 0, Kh, Vh, 0.3)
+    np.testing.assert_allclose(out, attention.decode_attention(q, Kh, Vh, 0.3), rtol=1e-13)
+    out = attention.window_decode_attention(q, K, V, 8, 64, Kh[:0], Vh[:0], 0.3)
+    Kb, Vb = attention.bf16_round(K), attention.bf16_round(V)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[:, None, :], torch.tensor(Kb)[None].expand(2, T, d), torch.tensor(Vb)[None].expand(2, T, d),
+        scale=0.3)[:, 0].numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-12)
+    # bf16 rounding is round-to-nearest-even on the 8-bit significand
+    assert attention.bf16_round(np.array([1.0 + 2 ** -8]))[0] == 1.0
+    assert attention.bf16_round(np.array([1.0 + 3 * 2 ** -8]))[0] == 1.0 + 2 ** -6
+    # a mixed case: sink 4, recent 6 over 40 tokens -> 30 history rows from the estimates
+    out = attention.window_decode_attention(q, K, V, 4, 6, Kh[4:34], Vh[4:34], 0.3)
+    Keff = np.concatenate([attention.bf16_round(K[:4]), Kh[4:34], attention.bf16_round(K[34:])])
+    Veff = np.concatenate([attention.bf16_round(V[:4]), Vh[4:34], attention.bf16_round(V[34:])])
+    np.testing.assert_allclose(out, attention.decode_attention(q, Keff, Veff, 0.3), rtol=1e-13)
