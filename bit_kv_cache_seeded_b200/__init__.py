@@ -35,7 +35,8 @@ EXPORTS = ("kvq_status_str", "kvq_cache_bytes", "kvq_packed_bytes_per_token", "k
            "kvq_debug_quantize_rotated", "kvq_decode_attention_static", "kvq_kernel_launches",
            "kvq_cache_status", "kvq_debug_decode_unset_wait", "kvq_debug_decode_timed", "kvq_decode_step",
            "kvq_step_staging_bytes", "kvq_decode_step_host", "kvq_draw_rotation_signs", "kvq_draw_qjl_matrix",
-           "kvq_partial_floats", "kvq_decode_partials", "kvq_combine_partials")
+           "kvq_partial_floats", "kvq_decode_partials", "kvq_combine_partials",
+           "kvq_cache_bytes_paged", "kvq_cache_init_paged")
 KVQ_STATUS_WAIT_TIMEOUT = 1
 
 
@@ -92,6 +93,8 @@ def load() -> ctypes.CDLL:
         "kvq_draw_rotation_signs": ([ctypes.c_uint64, I32, VP], I32),
         "kvq_draw_qjl_matrix": ([ctypes.c_uint64, I32, I32, VP], I32),
         "kvq_partial_floats": ([VP, P(I32)], I32),
+        "kvq_cache_bytes_paged": ([P(kvq_cfg), I32, I32, P(SZ)], I32),
+        "kvq_cache_init_paged": ([P(VP), P(kvq_cfg), I32, I32, I32, VP, VP, SZ, VP, VP, VP], I32),
         "kvq_decode_partials": ([VP, VP, I32, VP, VP, SZ, VP], I32),
         "kvq_combine_partials": ([VP, I32, I32, I32, I32, VP, VP], I32),
     }
@@ -189,6 +192,30 @@ def kvq_cache_init(cfg: kvq_cfg, batch: int, capacity: int, arena: torch.Tensor,
                                None if signs is None else signs.ctypes.data_as(ctypes.c_void_p),
                                None if S is None else S.ctypes.data_as(ctypes.c_void_p), _stream(stream))
     _check("kvq_cache_init", st)
+    return handle
+
+
+def kvq_cache_bytes_paged(cfg: kvq_cfg, batch: int, n_pages: int) -> int:
+    out = ctypes.c_size_t()
+    _check("kvq_cache_bytes_paged", load().kvq_cache_bytes_paged(ctypes.byref(cfg), batch, n_pages, ctypes.byref(out)))
+    return out.value
+
+
+def kvq_cache_init_paged(cfg: kvq_cfg, batch: int, n_pages: int, block_table: torch.Tensor, arena: torch.Tensor,
+                         rot_signs=None, qjl_matrix=None, stream=None) -> ctypes.c_void_p:
+    """A paged cache: block_table int32 CUDA tensor [batch, pages_per_seq] (the caller keeps it)."""
+    _on_device("kvq_cache_init_paged", arena=arena, block_table=block_table)
+    if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != batch \
+            or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 [batch, pages_per_seq] tensor")
+    handle = ctypes.c_void_p()
+    signs = None if rot_signs is None else np.ascontiguousarray(rot_signs, dtype=np.int8)
+    S = None if qjl_matrix is None else np.ascontiguousarray(qjl_matrix, dtype=np.float32)
+    st = load().kvq_cache_init_paged(ctypes.byref(handle), ctypes.byref(cfg), batch, block_table.shape[1], n_pages,
+                                     _ptr(block_table), _ptr(arena), arena.numel() * arena.element_size(),
+                                     None if signs is None else signs.ctypes.data_as(ctypes.c_void_p),
+                                     None if S is None else S.ctypes.data_as(ctypes.c_void_p), _stream(stream))
+    _check("kvq_cache_init_paged", st)
     return handle
 
 
@@ -362,8 +389,8 @@ def kvq_cache_lengths(handle, batch: int) -> np.ndarray:
 
 
 def kvq_cache_layout(handle) -> np.ndarray:
-    info = np.zeros(22, dtype=np.int64)
-    _check("kvq_cache_layout", load().kvq_cache_layout(handle, info.ctypes.data_as(ctypes.c_void_p), 22))
+    info = np.zeros(24, dtype=np.int64)
+    _check("kvq_cache_layout", load().kvq_cache_layout(handle, info.ctypes.data_as(ctypes.c_void_p), 24))
     return info
 
 
@@ -400,16 +427,26 @@ def kvq_debug_quantize_rotated(handle, u: torch.Tensor, k_bits: int, qjl: bool, 
 # ---------------------------------------------------------------- convenience object
 
 class KvqCache:
-    """A packed cache in a torch-allocated device arena, plus its decode workspace."""
+    """A packed cache in a torch-allocated device arena, plus its decode workspace.
+
+    With block_table (an int32 CUDA tensor [batch, pages_per_seq]) and n_pages, the cache is paged:
+    its tiles live in a pool of n_pages pages of 64 tokens and the table names the page of each
+    64-token page of a sequence; the caller owns the table and fills it before tokens reach a page."""
 
     def __init__(self, cfg: kvq_cfg, batch: int, capacity: int, rot_signs=None, qjl_matrix=None,
-                 device="cuda"):
+                 device="cuda", block_table=None, n_pages=0):
         if not torch.cuda.is_available():
             raise RuntimeError("kvq needs a CUDA device")
         self.cfg, self.batch = cfg, batch
-        nbytes = kvq_cache_bytes(cfg, batch, capacity)
-        self.arena = torch.empty(nbytes, dtype=torch.uint8, device=device)
-        self.handle = kvq_cache_init(cfg, batch, capacity, self.arena, rot_signs, qjl_matrix)
+        if block_table is None:
+            nbytes = kvq_cache_bytes(cfg, batch, capacity)
+            self.arena = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            self.handle = kvq_cache_init(cfg, batch, capacity, self.arena, rot_signs, qjl_matrix)
+        else:
+            self.block_table = block_table
+            nbytes = kvq_cache_bytes_paged(cfg, batch, n_pages)
+            self.arena = torch.empty(nbytes, dtype=torch.uint8, device=device)
+            self.handle = kvq_cache_init_paged(cfg, batch, n_pages, block_table, self.arena, rot_signs, qjl_matrix)
         self.workspace = torch.empty(max(16, kvq_workspace_bytes(self.handle)), dtype=torch.uint8,
                                      device=device)
         self.out_dim = cfg.latent_dim if cfg.k_mode == MODES["fp4"] else cfg.head_dim

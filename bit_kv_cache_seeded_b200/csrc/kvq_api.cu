@@ -102,7 +102,9 @@ struct Plan {
   int tiles;
 };
 
-Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
+// n_pages > 0: a paged cache whose regions are a pool of n_pages pages (two tiles of every kv-head)
+// instead of batch x kv-heads x tiles contiguous tiles.
+Plan plan_layout(const kvq_cfg* c, int batch, int capacity, int n_pages = 0) {
   Plan P{};
   P.fp4_mode = c->k_mode == KVQ_MODE_FP4;
   P.tiles = (capacity + kTile * kTilePair - 1) / (kTile * kTilePair) * kTilePair;
@@ -110,11 +112,13 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
   P.lens_off = off;  // lengths, status words, history lengths (window caches)
   off = align_up(off + sizeof(int) * (2 * (size_t)batch + kStatusWords), kArenaAlign);
   const size_t pairs = (size_t)batch * c->n_kv_heads;
+  // tiles a region holds: every (sequence, kv-head)'s own, or the page pool's
+  const size_t region_tiles = n_pages > 0 ? (size_t)n_pages * c->n_kv_heads * kTilePair : pairs * P.tiles;
   if (P.fp4_mode) {
     P.fp4 = make_fp4(c->latent_dim, c->rope_dim);
     P.signs_off = P.S_off = P.St_off = off;
     P.k_off = off;
-    off = align_up(off + pairs * P.tiles * (size_t)P.fp4.tile_bytes, kArenaAlign);
+    off = align_up(off + region_tiles * (size_t)P.fp4.tile_bytes, kArenaAlign);
     P.v_off = off;
   } else {
     P.v = make_side(c->v_mode, c->v_bits, c->qjl_dim, kOrderByteLane);
@@ -129,9 +133,9 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity) {
     P.St_off = off;
     off = align_up(off + sizeof(float) * m * kHeadDim, kArenaAlign);
     P.k_off = off;
-    off = align_up(off + pairs * P.tiles * (size_t)P.k.tile_bytes, kArenaAlign);
+    off = align_up(off + region_tiles * (size_t)P.k.tile_bytes, kArenaAlign);
     P.v_off = off;
-    off = align_up(off + pairs * P.tiles * (size_t)P.v.tile_bytes, kArenaAlign);
+    off = align_up(off + region_tiles * (size_t)P.v.tile_bytes, kArenaAlign);
     // mixed-precision window: bf16 K then V, [pairs][sink + recent][d] each
     P.win_off = off;
     off = align_up(off + 2 * pairs * ((size_t)c->sink_tokens + c->recent_tokens) * kHeadDim * 2, kArenaAlign);
@@ -301,15 +305,28 @@ kvq_status kvq_packed_bytes_per_token(const kvq_cfg* cfg, size_t* bytes) {
   return KVQ_OK;
 }
 
-kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_t capacity,
-                          void* dev_mem, size_t dev_bytes, const int8_t* rot_signs,
-                          const float* qjl_matrix, void* stream) {
+kvq_status kvq_cache_bytes_paged(const kvq_cfg* cfg, int32_t batch, int32_t n_pages, size_t* bytes) {
+  if (!bytes || batch <= 0 || n_pages <= 0) return KVQ_ERR_INVALID_ARG;
+  const kvq_status st = validate_cfg(cfg);
+  if (st != KVQ_OK) return st;
+  if (cfg->k_mode == KVQ_MODE_FP4) return KVQ_ERR_UNSUPPORTED;
+  *bytes = plan_layout(cfg, batch, kTile * kTilePair, n_pages).total;
+  return KVQ_OK;
+}
+
+}  // extern "C"
+
+namespace {
+kvq_status cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_t capacity, void* dev_mem,
+                      size_t dev_bytes, const int8_t* rot_signs, const float* qjl_matrix, void* stream,
+                      const int32_t* table, int32_t pages_per_seq, int32_t n_pages) {
   if (!out || !dev_mem || batch <= 0 || capacity <= 0) return KVQ_ERR_INVALID_ARG;
   *out = nullptr;
   const kvq_status st = validate_cfg(cfg);
   if (st != KVQ_OK) return st;
   if (reinterpret_cast<uintptr_t>(dev_mem) % kArenaAlign) return KVQ_ERR_ALIGNMENT;
-  const Plan P = plan_layout(cfg, batch, capacity);
+  if (table && cfg->k_mode == KVQ_MODE_FP4) return KVQ_ERR_UNSUPPORTED;
+  const Plan P = plan_layout(cfg, batch, capacity, table ? n_pages : 0);
   if (dev_bytes < P.total) return KVQ_ERR_WORKSPACE;
   const bool need_sketch = !P.fp4_mode && (P.k.qjl || P.v.qjl);
   const int n_signs = P.fp4_mode ? 0 : kHeadDim * (cfg->rot_per_head ? cfg->n_kv_heads : 1);
@@ -356,6 +373,9 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
   c->signs_stride = cfg->rot_per_head ? kHeadDim : 0;
   c->tc = !P.fp4_mode && choose_tc(*cfg, P.k, P.v);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  c->table = table;
+  c->pages_per_seq = table ? pages_per_seq : 0;
+  c->n_pages = table ? n_pages : 0;
   c->sink = P.fp4_mode ? 0 : cfg->sink_tokens;
   c->recent = P.fp4_mode ? 0 : cfg->recent_tokens;
   c->d_hlens = c->d_status + kStatusWords;
@@ -392,6 +412,25 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
   *out = c;
   return KVQ_OK;
 }
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_t capacity,
+                          void* dev_mem, size_t dev_bytes, const int8_t* rot_signs,
+                          const float* qjl_matrix, void* stream) {
+  return cache_init(out, cfg, batch, capacity, dev_mem, dev_bytes, rot_signs, qjl_matrix, stream, nullptr, 0, 0);
+}
+
+kvq_status kvq_cache_init_paged(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_t pages_per_seq,
+                                int32_t n_pages, const int32_t* block_table, void* dev_mem, size_t dev_bytes,
+                                const int8_t* rot_signs, const float* qjl_matrix, void* stream) {
+  if (!block_table || pages_per_seq <= 0 || n_pages <= 0) return KVQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(block_table) % 4) return KVQ_ERR_ALIGNMENT;
+  if ((long)pages_per_seq * kTile * kTilePair > (1l << 30)) return KVQ_ERR_INVALID_ARG;
+  return cache_init(out, cfg, batch, pages_per_seq * kTile * kTilePair, dev_mem, dev_bytes, rot_signs, qjl_matrix,
+                    stream, block_table, pages_per_seq, n_pages);
+}
 
 }  // extern "C"
 
@@ -413,6 +452,9 @@ void fill_quantize(QuantizeParams& p, const kvq_cache* c, const void* K, const v
   p.region[0] = c->d_k;
   p.region[1] = c->d_v;
   p.tiles_per_seq = c->tiles_per_seq;
+  p.table = c->table;
+  p.pages_per_seq = c->pages_per_seq;
+  p.n_pages = c->n_pages;
   p.side[0] = c->k;
   p.side[1] = c->v;
   p.fp4 = c->fp4;
@@ -580,6 +622,9 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.kreg = c->d_k;
   p.vreg = c->d_v;
   p.tiles_per_seq = c->tiles_per_seq;
+  p.table = c->table;
+  p.pages_per_seq = c->pages_per_seq;
+  p.n_pages = c->n_pages;
   p.k = c->k;
   p.v = c->v;
   p.signs = c->d_signs;
@@ -863,6 +908,10 @@ kvq_status kvq_cache_layout(const kvq_cache* c, int64_t* info, int32_t n_info) {
     info[19] = c->sink + c->recent;
     info[20] = c->sink;
     info[21] = c->recent;
+  }
+  if (n_info > 23) {
+    info[22] = c->pages_per_seq;
+    info[23] = c->n_pages;
   }
   info[0] = kTile;
   info[1] = c->is_fp4 ? c->fp4.tile_bytes : c->k.tile_bytes;

@@ -16,6 +16,7 @@
 
 #include "kvq_async.cuh"
 #include "kvq_internal.h"
+#include "kvq_tiles.cuh"
 
 namespace kvq {
 namespace {
@@ -116,12 +117,12 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
   }
   const float vkappa = VQ ? 1.2533141373155003f / (float)p.v.m : 0.f;
 
-  const size_t pair = (size_t)b * p.Hkv + hk;
   for (int tile = t_begin / kTile + warp; tile * kTile < t_end; tile += kWarps) {
     const int count = min(kTile, t_end - tile * kTile);
     const bool valid = lane < count;
-    const char* kt = p.kreg + (pair * p.tiles_per_seq + tile) * (size_t)p.k.tile_bytes;
-    const char* vt = p.vreg + (pair * p.tiles_per_seq + tile) * (size_t)p.v.tile_bytes;
+    const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk, tile, p.err);
+    const char* kt = p.kreg + (size_t)ti * p.k.tile_bytes;
+    const char* vt = p.vreg + (size_t)ti * p.v.tile_bytes;
 
     // ---- logits: lane = token
     float logit[G];

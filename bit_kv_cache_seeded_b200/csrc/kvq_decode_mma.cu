@@ -42,6 +42,7 @@
 #include "kvq_internal.h"
 #include "kvq_quantize_lm.cuh"
 #include "kvq_lm_common.cuh"
+#include "kvq_tiles.cuh"
 
 namespace kvq {
 namespace {
@@ -329,8 +330,12 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   // runs before the prep: everything that reads them waits for the prep (which waits for it).
   const int t_begin = split * p.chunk;
   const size_t pair = (size_t)b * p.Hkv + hk;
-  const unsigned char* kbase = reinterpret_cast<const unsigned char*>(p.kreg) + pair * p.tiles_per_seq * (size_t)ktb;
-  const unsigned char* vbase = reinterpret_cast<const unsigned char*>(p.vreg) + pair * p.tiles_per_seq * (size_t)vtb;
+  const unsigned char* kreg = reinterpret_cast<const unsigned char*>(p.kreg);
+  const unsigned char* vreg = reinterpret_cast<const unsigned char*>(p.vreg);
+  // index of a tile pair's first tile (contiguous, or the block table's page)
+  auto pair_index = [&](int tile0) {
+    return tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk, tile0, p.err);
+  };
   // In a fused append + decode step the predecessor appends the token at the old length and sets
   // the new one, so a length read before waiting for it is either value. When the first
   // kStagesM - 1 fills end below the old length under both readings, they hold no token the
@@ -364,17 +369,17 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     unsigned char* dst = stages + slot * stage_bytes;
     fence_proxy_async();  // the stage's previous contents were read by the generic proxy
     if (f < n_iter) {
-      const int tile0 = (unsigned)(t_begin + f * kCtaTok) / kTile;
+      const long ti = pair_index((unsigned)(t_begin + f * kCtaTok) / kTile);
       constexpr uint32_t nb = VQ ? 128u : 64u;  // value norms (+ gammas, contiguous) per tile
       mbar_arrive_expect_tx(bar, 2u * ktb + 2u * nb);
-      bulk_g2s(smem_addr(dst), kbase + (size_t)tile0 * ktb, 2u * ktb, bar);
+      bulk_g2s(smem_addr(dst), kreg + (size_t)ti * ktb, 2u * ktb, bar);
 #pragma unroll
       for (int tile = 0; tile < 2; ++tile)
-        bulk_g2s(smem_addr(dst + 2 * ktb + tile * 128), vbase + (size_t)(tile0 + tile) * vtb + VL::NORM, nb, bar);
+        bulk_g2s(smem_addr(dst + 2 * ktb + tile * 128), vreg + (size_t)(ti + tile) * vtb + VL::NORM, nb, bar);
     } else {
-      const int tile0 = (unsigned)(t_begin + (f - n_iter) * kCtaTok) / kTile;
+      const long ti = pair_index((unsigned)(t_begin + (f - n_iter) * kCtaTok) / kTile);
       mbar_arrive_expect_tx(bar, 2u * vtb);
-      bulk_g2s(smem_addr(dst), vbase + (size_t)tile0 * vtb, 2u * vtb, bar);
+      bulk_g2s(smem_addr(dst), vreg + (size_t)ti * vtb, 2u * vtb, bar);
     }
   };
   auto wait_fill = [&](int f) {  // every thread

@@ -39,6 +39,7 @@
 #include "kvq_internal.h"
 #include "kvq_lm_common.cuh"
 #include "kvq_tcgen05.cuh"
+#include "kvq_tiles.cuh"
 
 namespace kvq {
 namespace {
@@ -120,8 +121,12 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
   const int t_begin = split * p.chunk;
   const size_t pair = (size_t)b * p.Hkv + hk;
   const int h_first = hk * p.group;
-  const unsigned char* kbase = reinterpret_cast<const unsigned char*>(p.kreg) + pair * p.tiles_per_seq * (size_t)ktb;
-  const unsigned char* vbase = reinterpret_cast<const unsigned char*>(p.vreg) + pair * p.tiles_per_seq * (size_t)vtb;
+  const unsigned char* kreg = reinterpret_cast<const unsigned char*>(p.kreg);
+  const unsigned char* vreg = reinterpret_cast<const unsigned char*>(p.vreg);
+  // index of a tile pair's first tile (contiguous, or the block table's page)
+  auto pair_index = [&](int tile0) {
+    return tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk, tile0, p.err);
+  };
   // fused append + decode step: see decode_lm_mma (a length read before the wait is either value)
   int len = __ldcg(p.lens + b);
   const bool early = p.cache_after_wait && t_begin + kTokT * (kStagesT - 1) < len;
@@ -164,12 +169,16 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
     if (f < n_iter) {
       constexpr uint32_t nb = VQ ? 128u : 64u;  // value norms (+ gammas, contiguous) per tile
       mbar_arrive_expect_tx(bar, (uint32_t)npairs * 2u * (ktb + nb));
-      bulk_g2s(smem_addr(dst), kbase + (size_t)tile0 * ktb, (uint32_t)npairs * 2u * ktb, bar);
-      for (int t = 0; t < 2 * npairs; ++t)
-        bulk_g2s(smem_addr(dst + 4 * ktb + t * 128), vbase + (size_t)(tile0 + t) * vtb + VL::NORM, nb, bar);
+      for (int j = 0; j < npairs; ++j) {
+        const long ti = pair_index(tile0 + 2 * j);
+        bulk_g2s(smem_addr(dst + 2 * j * ktb), kreg + (size_t)ti * ktb, 2u * ktb, bar);
+        for (int t = 0; t < 2; ++t)
+          bulk_g2s(smem_addr(dst + 4 * ktb + (2 * j + t) * 128), vreg + (size_t)(ti + t) * vtb + VL::NORM, nb, bar);
+      }
     } else {
       mbar_arrive_expect_tx(bar, (uint32_t)npairs * 2u * vtb);
-      bulk_g2s(smem_addr(dst), vbase + (size_t)tile0 * vtb, (uint32_t)npairs * 2u * vtb, bar);
+      for (int j = 0; j < npairs; ++j)
+        bulk_g2s(smem_addr(dst + 2 * j * vtb), vreg + (size_t)pair_index(tile0 + 2 * j) * vtb, 2u * vtb, bar);
     }
   };
   auto fail = [&]() {

@@ -62,6 +62,8 @@ struct QuantizeParams {
   int n_new, n_seq, heads;
   char* region[2];       // side region bases (FP4: region[0] only)
   int tiles_per_seq;
+  const int* table;      // paged regions: block table [batch][pages_per_seq] (null: contiguous)
+  int pages_per_seq, n_pages;
   SideLayout side[2];
   Fp4Layout fp4;
   const float* signs;    // [d] +-1 (per-head rotation: [heads][d])
@@ -101,6 +103,8 @@ struct DecodeParams {
   const char* kreg;
   const char* vreg;
   int tiles_per_seq;
+  const int* table;       // paged regions: block table [B][pages_per_seq] (null: contiguous)
+  int pages_per_seq, n_pages;
   SideLayout k, v;
   const float* signs;     // [d] (per-head rotation: [Hkv][d])
   int signs_stride;       // 0: one diagonal for every kv-head; d: kv-head hk reads signs + hk * d
@@ -199,6 +203,8 @@ struct kvq_cache {
   int device = -1;          // the CUDA device whose memory holds the arena (current at init)
   bool tc = false;          // LM decode runs on the tcgen05 kernel (else mma.sync / CUDA cores)
   int sink = 0, recent = 0; // mixed-precision window (0, 0: none)
+  const int* table = nullptr;  // paged caches: caller's device block table [batch][pages_per_seq]
+  int pages_per_seq = 0, n_pages = 0;
   int* d_hlens = nullptr;   // window caches: coded history length per sequence (the decode kernels' lens)
   uint16_t* d_win = nullptr;// window caches: bf16 K then V window, [batch][kv-heads][sink + recent][d] each
   std::vector<int> hlens;   // host mirror of d_hlens

@@ -10,6 +10,7 @@
 
 #include "kvq_async.cuh"
 #include "kvq_internal.h"
+#include "kvq_tiles.cuh"
 
 namespace kvq {
 namespace qlm {
@@ -223,8 +224,12 @@ __device__ __forceinline__ void quantize_lm_block(const QuantizeParams& p, int s
     const int pos = p.pos[s] + t;
     const int seq = p.seq[s];
     const int tile = pos / kTile, slot = pos % kTile;
-    char* tb = p.region[side] +
-               (((size_t)seq * p.heads + h) * p.tiles_per_seq + tile) * (size_t)L.tile_bytes;
+    const long ti = tile_index(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.heads, seq, h, tile);
+    if (ti < 0) {  // the block table names no page for this token: nothing is written
+      if (threadIdx.x % 32 == 0) atomicOr(p.err, kStatusBadPage);
+      continue;
+    }
+    char* tb = p.region[side] + (size_t)ti * L.tile_bytes;
     if (L.order == kOrderToken) {
       if (lead && lane < L.bits)
         *reinterpret_cast<uint4*>(tb + L.off_planes + lane * (kTile * 16) + slot * 16) = mine;

@@ -22,6 +22,7 @@
 #include "kvq_async.cuh"
 #include "kvq_internal.h"
 #include "kvq_quantize_lm.cuh"
+#include "kvq_tiles.cuh"
 
 namespace kvq {
 namespace qtile {
@@ -74,7 +75,12 @@ __device__ void quantize_tiles(const QuantizeParams& p, int side, float* st_s, S
     const int t0 = tile * kTile;
     if (t0 >= pos0 + p.n_new) continue;  // the same for the whole block
     const int lo = max(t0, pos0) - t0, hi = min(t0 + kTile, pos0 + p.n_new) - t0;
-    char* tb = p.region[side] + (((size_t)p.seq[s] * p.heads + h) * p.tiles_per_seq + tile) * (size_t)L.tile_bytes;
+    const long ti = tile_index(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.heads, p.seq[s], h, tile);
+    if (ti < 0) {  // the block table names no page for this tile: nothing is written
+      if (tid == 0) atomicOr(p.err, kStatusBadPage);
+      continue;  // the same for the whole block
+    }
+    char* tb = p.region[side] + (size_t)ti * L.tile_bytes;
     // a tile whose first tokens are already stored: start from its current bytes
     if (lo > 0)
       for (int c = tid; c < L.tile_bytes / 16; c += kThreads)

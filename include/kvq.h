@@ -140,6 +140,22 @@ kvq_status kvq_cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, in
                           void* dev_mem, size_t dev_bytes, const int8_t* rot_signs,
                           const float* qjl_matrix, void* stream);
 
+/* Paged cache ("TurboQuant vs OSCAR vs EpiCache", OSCAR: fused kernels compatible with paged
+ * attention and the prefix cache). The tiles of an LM/SIGN1 cache live in a pool of n_pages pages;
+ * a page holds 64 consecutive tokens of one sequence for every kv-head (two tiles of K and of V per
+ * kv-head). block_table: DEVICE int32 [batch][pages_per_seq], owned by the caller, giving the pool
+ * page of each 64-token page of each sequence; capacity = 64 pages_per_seq tokens. The caller fills
+ * the entries of the pages a call appends to before the call, and keeps the table unchanged while
+ * work that reads it is in flight; sequences may share pages that hold identical tokens (a common
+ * prefix) as long as nothing appends into a shared page. The kernels check every entry they use: one
+ * that is not a page of the pool (< 0 or >= n_pages) sets KVQ_STATUS_BAD_PAGE; appends then write
+ * nothing for that page and decode reads page 0 in its place. kvq_cache_bytes_paged gives the arena
+ * size (table excluded); the rest is as for kvq_cache_init. FP4 caches: KVQ_ERR_UNSUPPORTED. */
+kvq_status kvq_cache_bytes_paged(const kvq_cfg* cfg, int32_t batch, int32_t n_pages, size_t* bytes);
+kvq_status kvq_cache_init_paged(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_t pages_per_seq,
+                                int32_t n_pages, const int32_t* block_table, void* dev_mem, size_t dev_bytes,
+                                const int8_t* rot_signs, const float* qjl_matrix, void* stream);
+
 /* Quantize n_new tokens per listed sequence and append them ("kvq_quantize(K or V, cfg) ->
  * packed codes + norms + sketch"). K, V: device tensors in the layout above. seq_ids: host
  * array of n_seq distinct sequence indices, or NULL for all sequences in order (then n_seq
@@ -241,8 +257,9 @@ kvq_status kvq_decode_attention_static(const kvq_cache* c, const void* q, kvq_dt
 /* Bits of the cache's device status word. The tensor-core decode kernel bounds every wait for
  * staged cache data (about one second of SM clock); a wait that gives up sets
  * KVQ_STATUS_WAIT_TIMEOUT, the kernel still runs to its end and returns, and the output of that
- * call is not to be trusted. No kernel sets any other bit. */
+ * call is not to be trusted. KVQ_STATUS_BAD_PAGE: see kvq_cache_init_paged. */
 #define KVQ_STATUS_WAIT_TIMEOUT 1
+#define KVQ_STATUS_BAD_PAGE 2  /* a paged cache's block table named no page of the pool */
 
 /* Read the cache's device status word (the bits above) into *status (host). Enqueues a 4-byte
  * copy on `stream` and waits for the stream, so it reports on all work enqueued before it.
@@ -277,7 +294,9 @@ kvq_status kvq_cache_lengths(const kvq_cache* c, int32_t* lens);
  * the order of the K and V planes (0 byte-lane, 1 token, 2 octet); with n_info >= 22 also info[18..21]:
  * the byte offset of the mixed-precision window (bf16 K then V, [batch][n_kv_heads][slots][head_dim]
  * each), slots = sink + recent, sink, recent (zeros without a window). On a window cache the tiles
- * hold the coded history: history token i is sequence position sink + i. Layout of a tile (32 tokens)
+ * hold the coded history: history token i is sequence position sink + i; with n_info >= 24 also
+ * info[22], info[23]: pages_per_seq and n_pages of a paged cache (zeros otherwise: tiles contiguous).
+ * Layout of a tile (32 tokens)
  * of one (sequence, kv-head): code bit-planes (512 bytes each), then sign words (512 bytes),
  * then [32] fp16 norms, then [32] fp16 residual norms (sides with a sketch). Plane p holds bit p
  * of every code; a token's 128 bits of a plane are 16 bytes, byte k holding coordinates
