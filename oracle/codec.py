@@ -193,3 +193,64 @@ def fp4_dequantize(packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
         nib = (packed[j // 2] >> (4 * (j % 2))) & 0xF
         out[j] = e4m3_decode(int(scales[j // FP4_GROUP])) * e2m1_decode(int(nib))
     return out
+
+
+# ---- KIVI-style asymmetric integer codes ------------------------------------------------------
+#
+# "TurboQuant vs OSCAR vs EpiCache", section "Quantization frontiers: TurboQuant and OSCAR": KIVI
+# quantizes keys per channel (keys have fixed outlier channels across tokens) and values per token.
+# The pages give neither the group size nor the rounding; the readings used here:
+#   * asymmetric b-bit integers: for a group of numbers x, z = min x and s = (max x - min x)/(2^b - 1),
+#     both rounded once to fp16 (round to nearest even, saturating at 65504); the code of x is
+#     rint((x - z) / s) clipped to [0, 2^b - 1], with the subtraction and the IEEE division in fp32
+#     and rint rounding ties to even; s = 0 codes every x as 0. The estimate is z + s * code;
+#   * keys: one (s, z) per channel over a group of KIVI_KEY_GROUP consecutive tokens;
+#   * values: one (s, z) per token over its head_dim channels;
+#   * the tokens of a sequence's last, incomplete key group stay in bf16 (keys and values) until
+#     the group is complete.
+
+KIVI_KEY_GROUP = 128
+
+
+def _f16_sat(x):
+    x = np.asarray(x, dtype=np.float32)
+    return np.clip(x, -65504.0, 65504.0).astype(np.float16)
+
+
+def kivi_params(lo: np.ndarray, hi: np.ndarray, bits: int):
+    """fp16 scale and zero of a group from its fp32 minimum and maximum."""
+    lo = np.asarray(lo, dtype=np.float32)
+    hi = np.asarray(hi, dtype=np.float32)
+    s16 = _f16_sat((hi - lo) / np.float32((1 << bits) - 1))
+    z16 = _f16_sat(lo)
+    return s16, z16
+
+
+def kivi_code(x: np.ndarray, s16: np.ndarray, z16: np.ndarray, bits: int) -> np.ndarray:
+    """Codes of fp32 values x against (broadcast) fp16 scale and zero, fp32 arithmetic."""
+    x = np.asarray(x, dtype=np.float32)
+    s = np.asarray(s16, dtype=np.float32)
+    z = np.asarray(z16, dtype=np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.rint((x - z) / np.where(s > 0, s, np.float32(1.0)))
+    q = np.where(s > 0, q, 0)
+    return np.clip(q, 0, (1 << bits) - 1).astype(np.int64)
+
+
+def kivi_quantize_keys(K: np.ndarray, bits: int = 2):
+    """One key group: K [T, d] (fp32 values) -> codes [T, d], s16 [d], z16 [d] (per channel)."""
+    K = np.asarray(K, dtype=np.float32)
+    s16, z16 = kivi_params(K.min(axis=0), K.max(axis=0), bits)
+    return kivi_code(K, s16[None, :], z16[None, :], bits), s16, z16
+
+
+def kivi_quantize_values(V: np.ndarray, bits: int = 2):
+    """Values V [T, d] (fp32 values) -> codes [T, d], s16 [T], z16 [T] (per token)."""
+    V = np.asarray(V, dtype=np.float32)
+    s16, z16 = kivi_params(V.min(axis=1), V.max(axis=1), bits)
+    return kivi_code(V, s16[:, None], z16[:, None], bits), s16, z16
+
+
+def kivi_dequantize(codes: np.ndarray, s16, z16) -> np.ndarray:
+    """z + s * code in fp64 (s16, z16 broadcast against codes)."""
+    return np.asarray(z16, dtype=np.float64) + np.asarray(s16, dtype=np.float64) * np.asarray(codes, dtype=np.float64)

@@ -597,3 +597,51 @@ def test_window_attention_special_cases():
     Keff = np.concatenate([attention.bf16_round(K[:4]), Kh[4:34], attention.bf16_round(K[34:])])
     Veff = np.concatenate([attention.bf16_round(V[:4]), Vh[4:34], attention.bf16_round(V[34:])])
     np.testing.assert_allclose(out, attention.decode_attention(q, Keff, Veff, 0.3), rtol=1e-13)
+
+
+# ---------------------------------------------------------------- KIVI-style codes
+
+def test_kivi_hand_worked(golden):
+    rows = golden("kivi_example.txt")
+    X, S, Z, C, E = [], [], [], [], []
+    for r in rows:
+        parts = " ".join(r[1:]).split("|")
+        X.append([float(v) for v in parts[0].split()])
+        s, z = (float(v) for v in parts[1].split())
+        S.append(s), Z.append(z)
+        C.append([int(v) for v in parts[2].split()])
+        E.append([float(v) for v in parts[3].split()])
+    K = np.array(X).T  # [4 tokens, 5 channels]: one key group, per-channel parameters
+    codes, s16, z16 = codec.kivi_quantize_keys(K)
+    np.testing.assert_array_equal(s16.astype(np.float64), S)
+    np.testing.assert_array_equal(z16.astype(np.float64), Z)
+    np.testing.assert_array_equal(codes.T, C)
+    np.testing.assert_array_equal(codec.kivi_dequantize(codes, s16[None], z16[None]).T, E)
+    # the same numbers as values of 5 tokens (per-token parameters) give the same codes
+    vc, vs, vz = codec.kivi_quantize_values(np.array(X))
+    np.testing.assert_array_equal(vc, C)
+    np.testing.assert_array_equal(vs.astype(np.float64), S)
+
+
+def test_kivi_error_bound_and_grid_round_trip():
+    """|x - x_hat| <= s/2 plus the fp16 rounding of z and s (per channel for keys, per token for
+    values); values on the grid z + s k with fp16 z and s come back exactly."""
+    rng = np.random.default_rng(12)
+    K = (rng.standard_normal((128, 64)) * np.exp(rng.uniform(-2, 3, 64))[None]).astype(np.float32)
+    codes, s16, z16 = codec.kivi_quantize_keys(K)
+    err = np.abs(codec.kivi_dequantize(codes, s16[None], z16[None]) - K)
+    s = s16.astype(np.float64)
+    span = K.max(0) - K.min(0)
+    slack = 2.0 ** -10 * (np.abs(K.min(0)) + 3 * span / 3)  # fp16 rounding of z and of s times the code
+    assert np.all(err <= s[None] / 2 + slack[None] + 1e-7)
+    z = np.float16(-1.25)
+    sc = np.float16(0.375)
+    grid = (np.float32(z) + np.float32(sc) * rng.integers(0, 4, (50, 8))).astype(np.float32)
+    grid[0], grid[1] = np.float32(z), np.float32(z) + 3 * np.float32(sc)  # min and max present
+    c, s2, z2 = codec.kivi_quantize_keys(grid)
+    np.testing.assert_array_equal(codec.kivi_dequantize(c, s2[None], z2[None]), grid.astype(np.float64))
+    V = rng.standard_normal((40, 128)).astype(np.float32)
+    vc, vs, vz = codec.kivi_quantize_values(V)
+    verr = np.abs(codec.kivi_dequantize(vc, vs[:, None], vz[:, None]) - V)
+    vspan = V.max(1) - V.min(1)
+    assert np.all(verr <= vs.astype(np.float64)[:, None] / 2 + 2.0 ** -10 * (np.abs(V.min(1)) + vspan)[:, None] + 1e-7)
