@@ -25,7 +25,7 @@ KVQ_OK = 0
 STATUS_NAMES = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_UNSUPPORTED",
                 3: "KVQ_ERR_CAPACITY", 4: "KVQ_ERR_ALIGNMENT", 5: "KVQ_ERR_WORKSPACE",
                 6: "KVQ_ERR_CUDA"}
-MODES = {"lm_qjl": 0, "lm": 1, "sign1": 2, "fp4": 3}
+MODES = {"lm_qjl": 0, "lm": 1, "sign1": 2, "fp4": 3, "kivi": 4}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 
 # Every symbol include/kvq.h declares.

@@ -44,6 +44,14 @@ kvq_status validate_cfg(const kvq_cfg* c) {
       return KVQ_ERR_UNSUPPORTED;
     return KVQ_OK;
   }
+  if (c->k_mode == KVQ_MODE_KIVI || c->v_mode == KVQ_MODE_KIVI) {
+    if (c->k_mode != c->v_mode || c->k_bits != 2 || c->v_bits != 2) return KVQ_ERR_UNSUPPORTED;
+    if (c->head_dim != kHeadDim) return c->head_dim > 0 ? KVQ_ERR_UNSUPPORTED : KVQ_ERR_INVALID_ARG;
+    if (c->rot_per_head || c->sink_tokens || c->recent_tokens) return KVQ_ERR_INVALID_ARG;
+    const int g = c->n_q_heads / c->n_kv_heads;
+    if (g != 1 && g != 2 && g != 4 && g != 8) return KVQ_ERR_UNSUPPORTED;
+    return KVQ_OK;
+  }
   if (!is_lm_mode(c->k_mode) || !is_lm_mode(c->v_mode)) return KVQ_ERR_INVALID_ARG;
   if (c->head_dim != kHeadDim) return c->head_dim > 0 ? KVQ_ERR_UNSUPPORTED : KVQ_ERR_INVALID_ARG;
   const int modes[2] = {c->k_mode, c->v_mode};
@@ -83,6 +91,23 @@ SideLayout make_side(int mode, int bits, int qjl_dim, int order) {
   return L;
 }
 
+// KIVI sides: two code bit-planes; keys in octet order with an (unused) norm slot, values in
+// byte-lane order with per-token fp16 scale (norm slot) and zero (gamma slot).
+SideLayout make_kivi_side(bool values) {
+  SideLayout L;
+  L.bits = 2;
+  L.qjl = 0;
+  L.order = values ? kOrderByteLane : kOrderOctet;
+  L.off_planes = 0;
+  L.off_sketch = 2 * kTile * (kHeadDim / 8);
+  L.off_norm = L.off_sketch;
+  L.off_gamma = L.off_norm + kTile * 2;
+  L.tile_bytes = (int)align_up((size_t)L.off_norm + kTile * 2 * (values ? 2 : 1), 16);
+  return L;
+}
+
+constexpr int kKiviGroupTokens = 128;  // KIVI key group (four tiles)
+
 Fp4Layout make_fp4(int latent, int rope) {
   Fp4Layout F;
   F.latent = latent;
@@ -95,7 +120,8 @@ Fp4Layout make_fp4(int latent, int rope) {
 }
 
 struct Plan {
-  size_t lens_off, signs_off, S_off, St_off, k_off, v_off, win_off, total;
+  size_t lens_off, signs_off, S_off, St_off, k_off, v_off, win_off, kstats_off, total;
+  bool kivi;
   SideLayout k, v;
   Fp4Layout fp4;
   bool fp4_mode;
@@ -107,7 +133,9 @@ struct Plan {
 Plan plan_layout(const kvq_cfg* c, int batch, int capacity, int n_pages = 0) {
   Plan P{};
   P.fp4_mode = c->k_mode == KVQ_MODE_FP4;
-  P.tiles = (capacity + kTile * kTilePair - 1) / (kTile * kTilePair) * kTilePair;
+  P.kivi = c->k_mode == KVQ_MODE_KIVI;
+  const int unit = P.kivi ? kKiviGroupTokens : kTile * kTilePair;  // capacity granule
+  P.tiles = (capacity + unit - 1) / unit * (unit / kTile);
   size_t off = 0;
   P.lens_off = off;  // lengths, status words, history lengths (window caches)
   off = align_up(off + sizeof(int) * (2 * (size_t)batch + kStatusWords), kArenaAlign);
@@ -121,10 +149,15 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity, int n_pages = 0) {
     off = align_up(off + region_tiles * (size_t)P.fp4.tile_bytes, kArenaAlign);
     P.v_off = off;
   } else {
-    P.v = make_side(c->v_mode, c->v_bits, c->qjl_dim, kOrderByteLane);
-    P.k = make_side(c->k_mode, c->k_bits, c->qjl_dim, kOrderToken);
-    if (mma_modes_supported(c->n_q_heads / c->n_kv_heads, P.k.bits, P.k.qjl, P.v.bits, P.v.qjl))
-      P.k.order = kOrderOctet;
+    if (P.kivi) {
+      P.v = make_kivi_side(true);
+      P.k = make_kivi_side(false);
+    } else {
+      P.v = make_side(c->v_mode, c->v_bits, c->qjl_dim, kOrderByteLane);
+      P.k = make_side(c->k_mode, c->k_bits, c->qjl_dim, kOrderToken);
+      if (mma_modes_supported(c->n_q_heads / c->n_kv_heads, P.k.bits, P.k.qjl, P.v.bits, P.v.qjl))
+        P.k.order = kOrderOctet;
+    }
     const size_t m = (P.k.qjl || P.v.qjl) ? (size_t)c->qjl_dim : 0;
     P.signs_off = off;
     off = align_up(off + sizeof(float) * kHeadDim * (c->rot_per_head ? c->n_kv_heads : 1), kArenaAlign);
@@ -136,9 +169,13 @@ Plan plan_layout(const kvq_cfg* c, int batch, int capacity, int n_pages = 0) {
     off = align_up(off + region_tiles * (size_t)P.k.tile_bytes, kArenaAlign);
     P.v_off = off;
     off = align_up(off + region_tiles * (size_t)P.v.tile_bytes, kArenaAlign);
-    // mixed-precision window: bf16 K then V, [pairs][sink + recent][d] each
+    // mixed-precision window (KIVI: the incomplete key group): bf16 K then V, [pairs][slots][d] each
+    const size_t slots = P.kivi ? kKiviGroupTokens : (size_t)c->sink_tokens + c->recent_tokens;
     P.win_off = off;
-    off = align_up(off + 2 * pairs * ((size_t)c->sink_tokens + c->recent_tokens) * kHeadDim * 2, kArenaAlign);
+    off = align_up(off + 2 * pairs * slots * kHeadDim * 2, kArenaAlign);
+    // KIVI key statistics: [pairs][groups][2][d] fp16
+    P.kstats_off = off;
+    if (P.kivi) off = align_up(off + pairs * (size_t)(P.tiles / 4) * 2 * kHeadDim * 2, kArenaAlign);
   }
   P.total = off;
   return P;
@@ -166,7 +203,7 @@ int part_stride(const kvq_cache* c) {
 // (1 on every other path). The mma.sync kernel also runs one CTA per piece; the tcgen05 kernel
 // takes all pieces of a kv-head in one CTA.
 int decode_hsplit(const kvq_cache* c) {
-  if (c->is_fp4) return 1;
+  if (c->is_fp4 || c->kivi) return 1;
   const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
   if (!mma_modes_supported(group, c->k.bits, c->k.qjl, c->v.bits, c->v.qjl)) return 1;
   return group > 4 ? group / 4 : 1;
@@ -192,7 +229,7 @@ size_t partials_bytes(const kvq_cache* c, int splits) {
 }
 
 // Workspace = split partials, then the per-(sequence, kv-head) query tables of the tensor-core path.
-bool has_window(const kvq_cache* c) { return c->sink > 0 || c->recent > 0; }
+bool has_window(const kvq_cache* c) { return c->sink > 0 || c->recent > 0 || c->kivi; }
 
 // Bytes of the window's softmax states [B][Hq][part_stride] (window caches), 256-aligned.
 size_t window_state_bytes(const kvq_cache* c) {
@@ -215,6 +252,7 @@ const std::vector<int>& coded_lens(const kvq_cache* c) { return has_window(c) ? 
 // tensor-core kernel's shared-memory and register limit for query groups of 1, 2 or 4, else 4.
 int decode_slots_per_sm(const kvq_cache* c, int units) {
   if (c->is_fp4 || c->tc) return 1;
+  if (c->kivi) return 8;
   const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
   if (group == 1 || group == 2 || group == 4)
     return lm_mma_slots_per_sm(group, c->k, c->v, units * kTile * kTilePair);
@@ -294,6 +332,10 @@ kvq_status kvq_packed_bytes_per_token(const kvq_cfg* cfg, size_t* bytes) {
     *bytes = (size_t)cfg->latent_dim / 2 + cfg->latent_dim / 16 + 2 * (size_t)cfg->rope_dim;
     return KVQ_OK;
   }
+  if (cfg->k_mode == KVQ_MODE_KIVI) {  // per side: codes, plus (K) statistics per 128 tokens or (V) s, z
+    *bytes = 2 * ((size_t)cfg->k_bits * kHeadDim / 8 + 4);
+    return KVQ_OK;
+  }
   size_t b = 0;
   const int modes[2] = {cfg->k_mode, cfg->v_mode}, bits[2] = {cfg->k_bits, cfg->v_bits};
   for (int i = 0; i < 2; ++i) {
@@ -371,13 +413,19 @@ kvq_status cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_
     return KVQ_ERR_CUDA;
   }
   c->signs_stride = cfg->rot_per_head ? kHeadDim : 0;
-  c->tc = !P.fp4_mode && choose_tc(*cfg, P.k, P.v);
+  c->tc = !P.fp4_mode && !P.kivi && choose_tc(*cfg, P.k, P.v);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   c->table = table;
   c->pages_per_seq = table ? pages_per_seq : 0;
   c->n_pages = table ? n_pages : 0;
   c->sink = P.fp4_mode ? 0 : cfg->sink_tokens;
   c->recent = P.fp4_mode ? 0 : cfg->recent_tokens;
+  c->kivi = P.kivi;
+  if (P.kivi) {
+    c->recent = kKiviGroupTokens;  // the window slots hold the incomplete last key group
+    c->d_kstats = c->dev + P.kstats_off;
+    c->groups_per_seq = P.tiles / 4;
+  }
   c->d_hlens = c->d_status + kStatusWords;
   c->hlens.assign(batch, 0);
   if (!P.fp4_mode) c->d_win = reinterpret_cast<uint16_t*>(c->dev + P.win_off);
@@ -512,6 +560,39 @@ kvq_status quantize_window(kvq_cache* c, const void* K, const void* V, kvq_dtype
   for (int i = 0; i < cnt; ++i) c->lens[p.seq[i]] += n_new;
   return KVQ_OK;
 }
+// Append to a KIVI cache: code every 128-token key group the call completes (from the bf16 window
+// and the input), then write the call's tokens that are in the new incomplete group to the window.
+kvq_status quantize_kivi(kvq_cache* c, const void* K, const void* V, kvq_dtype dtype, int n_new,
+                         const int32_t* seq_ids, int first, int cnt, cudaStream_t s) {
+  QuantizeParams p;
+  fill_quantize(p, c, K, V, dtype, n_new, seq_ids, first, cnt);
+  const size_t pairs_kv = (size_t)c->batch * c->cfg.n_kv_heads;
+  p.ring[0] = c->d_win;
+  p.ring[1] = c->d_win + pairs_kv * (size_t)kKiviGroupTokens * kHeadDim;
+  p.win_sink = 0;
+  p.win_recent = kKiviGroupTokens;
+  p.win_slots = kKiviGroupTokens;
+  p.win_kivi = 1;
+  p.kstats = c->d_kstats;
+  p.groups_per_seq = c->groups_per_seq;
+  int max_groups = 0;
+  for (int i = 0; i < cnt; ++i) {
+    const int T0 = c->lens[p.seq[i]];
+    p.total0[i] = T0;
+    max_groups = std::max(max_groups, (T0 + n_new) / kKiviGroupTokens - T0 / kKiviGroupTokens);
+  }
+  if (max_groups > 0) {  // reads the window before the write below overwrites it
+    QuantizeParams pg = p;
+    pg.lens = c->d_hlens;
+    if (launch_kivi_groups(pg, max_groups, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  }
+  if (launch_window_write(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  for (int i = 0; i < cnt; ++i) {
+    c->lens[p.seq[i]] += n_new;
+    c->hlens[p.seq[i]] = c->lens[p.seq[i]] / kKiviGroupTokens * kKiviGroupTokens;
+  }
+  return KVQ_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -536,6 +617,11 @@ kvq_status kvq_quantize(kvq_cache* c, const void* K, const void* V, kvq_dtype dt
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   for (int first = 0; first < n_seq; first += kMaxSeqPerLaunch) {
     const int cnt = std::min(kMaxSeqPerLaunch, n_seq - first);
+    if (c->kivi) {
+      const kvq_status st = quantize_kivi(c, K, V, dtype, n_new, seq_ids, first, cnt, s);
+      if (st != KVQ_OK) return st;
+      continue;
+    }
     if (has_window(c)) {
       const kvq_status st = quantize_window(c, K, V, dtype, n_new, seq_ids, first, cnt, s);
       if (st != KVQ_OK) return st;
@@ -649,6 +735,15 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
     p.tot_lens = c->d_lens;
     p.wpart = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + partials_bytes(c, splits) +
                                        prep_bytes_total(c));
+    p.win_kivi = c->kivi ? 1 : 0;
+    p.kstats = c->d_kstats;
+    p.groups_per_seq = c->groups_per_seq;
+  }
+  if (c->kivi) {  // KIVI: the split kernel over the coded groups, the window, the reduce (no rotation)
+    if (!rec(1) || launch_decode_kivi(p, s) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
+    if (launch_window_decode(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (launch_reduce_lm(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
+    return KVQ_OK;
   }
   const bool tensor_path = p.use_tc ? tc_decode_supported(p) : mma_decode_supported(p);
   if (qp && !tensor_path) {  // no fused front kernel on this path: append first

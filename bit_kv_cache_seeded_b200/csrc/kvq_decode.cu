@@ -354,8 +354,14 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
   xs[h * kHeadDim + i] = o;
   __syncthreads();
   // lane l of warp h holds coordinates 32k + l; butterflies over index bits 0..4 by shuffles,
-  // bits 5..6 in registers.
-  if (warp < G) {
+  // bits 5..6 in registers. KIVI caches are not rotated: the output is o itself.
+  if (p.win_kivi && warp < G) {
+    const int hh = warp;
+    float* dst = p.pout ? p.pout + ((size_t)b * p.Hq + hk * G + hh) * (2 + kHeadDim) + 2
+                        : p.out + ((size_t)b * p.Hq + hk * G + hh) * kHeadDim;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dst[32 * k + lane] = xs[hh * kHeadDim + 32 * k + lane];
+  } else if (warp < G) {
     const int hh = warp;
     float u[4];
 #pragma unroll

@@ -85,6 +85,9 @@ struct QuantizeParams {
   int win_src;
   const uint16_t* ring[2];  // bf16 window of K and V: [n_seq][heads][win_slots][d]
   int win_sink, win_recent, win_slots, src_rows;
+  int win_kivi;             // KIVI caches: the window is the incomplete last key group (T % 128 tokens)
+  char* kstats;             // KIVI caches: per (sequence, kv-head, 128-token group) fp16 key scales, zeros [2][d]
+  int groups_per_seq;
   int total0[kMaxSeqPerLaunch];
   int cnt[kMaxSeqPerLaunch];
 };
@@ -126,6 +129,9 @@ struct DecodeParams {
   int win_sink, win_recent, win_slots;
   const int* tot_lens;
   float* wpart;
+  int win_kivi;            // KIVI caches: window = the incomplete last key group; outputs not rotated
+  const char* kstats;      // KIVI caches: [B][Hkv][groups][2][d] fp16 key scales, zeros
+  int groups_per_seq;
 };
 
 struct MlaParams {
@@ -185,6 +191,9 @@ bool mla_umma_supported(const MlaParams& p);
 // Mixed-precision window (kvq_window.cu): bf16 writes of appended tokens that stay in the window,
 // and the window's softmax state for decode.
 cudaError_t launch_window_write(const QuantizeParams& p, cudaStream_t s);
+// KIVI caches (kvq_kivi.cu): code every 128-token group an append completes (tail and input rows).
+cudaError_t launch_kivi_groups(const QuantizeParams& p, int max_groups, cudaStream_t s);
+cudaError_t launch_decode_kivi(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_window_decode(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_combine_partials(const float* parts, int n_parts, int rows, int dv, float* out, cudaStream_t s);
 cudaError_t launch_decode_mla_umma(const MlaParams& p, cudaStream_t s);
@@ -208,6 +217,9 @@ struct kvq_cache {
   int* d_hlens = nullptr;   // window caches: coded history length per sequence (the decode kernels' lens)
   uint16_t* d_win = nullptr;// window caches: bf16 K then V window, [batch][kv-heads][sink + recent][d] each
   std::vector<int> hlens;   // host mirror of d_hlens
+  bool kivi = false;        // KIVI codes (no rotation); the window is the incomplete last key group
+  char* d_kstats = nullptr; // KIVI: [batch][kv-heads][groups][2][d] fp16 key scales and zeros
+  int groups_per_seq = 0;
   char* dev = nullptr;
   size_t dev_bytes = 0;
   int* d_lens = nullptr;

@@ -39,7 +39,9 @@ __global__ void __launch_bounds__(kWinThreads) window_write(const __grid_constan
     const int pos = p.total0[s] + t, end = p.total0[s] + p.n_new;
     int slot;
     if (pos < p.win_sink) slot = pos;
-    else if (p.win_recent > 0 && pos >= max(p.win_sink, end - p.win_recent)) slot = p.win_sink + (pos - p.win_sink) % p.win_recent;
+    else if (p.win_kivi && pos >= end - end % p.win_recent) slot = pos % p.win_recent;  // incomplete group
+    else if (!p.win_kivi && p.win_recent > 0 && pos >= max(p.win_sink, end - p.win_recent))
+      slot = p.win_sink + (pos - p.win_sink) % p.win_recent;
     else continue;  // this token was coded into the history
     const size_t in = (size_t)vec * kHeadDim + 4 * lane;
     const size_t out = (((size_t)p.seq[s] * p.heads + h) * p.win_slots + slot) * kHeadDim + 4 * lane;
@@ -69,7 +71,7 @@ __global__ void __launch_bounds__(kWinThreads) window_decode(const __grid_consta
   const int G = p.group;
   const int T = p.tot_lens[b];
   const int s_end = min(T, p.win_sink);
-  const int r_begin = T > p.win_sink ? max(p.win_sink, T - p.win_recent) : s_end;
+  const int r_begin = p.win_kivi ? T - T % p.win_recent : T > p.win_sink ? max(p.win_sink, T - p.win_recent) : s_end;
   const int n_sink = s_end, n_tok = s_end + (T - r_begin);
   auto slot_of = [&](int i) { return i < n_sink ? i : p.win_sink + (r_begin + (i - n_sink) - p.win_sink) % p.win_recent; };
   const size_t pair = (size_t)b * p.Hkv + hk;
@@ -121,9 +123,21 @@ __global__ void __launch_bounds__(kWinThreads) window_decode(const __grid_consta
     float acc = 0.f;
     for (int i = 0; i < n_tok; ++i)
       acc = fmaf(lg[h][i], __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(vw)[(size_t)slot_of(i) * kHeadDim + j]), acc);
-    os[h][j] = acc * sg[j];
+    os[h][j] = p.win_kivi ? acc : acc * sg[j];
   }
   __syncthreads();
+  if (p.win_kivi) {  // KIVI caches are not rotated: the state stays in the original domain
+    for (int idx = tid; idx < G * kHeadDim; idx += kWinThreads) {
+      const int h = idx / kHeadDim, j = idx % kHeadDim;
+      p.wpart[((size_t)b * p.Hq + hk * G + h) * p.part_stride + 2 + j] = os[h][j];
+    }
+    if (tid < G) {
+      float* dst = p.wpart + ((size_t)b * p.Hq + hk * G + tid) * p.part_stride;
+      dst[0] = n_tok > 0 ? stat[tid][0] : -INFINITY;
+      dst[1] = n_tok > 0 ? stat[tid][1] : 0.f;
+    }
+    return;
+  }
   // o_r = H (D o) / sqrt(d): warp h, lane l holds coordinates 32k + l
   if (warp < G) {
     float u[4];

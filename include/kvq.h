@@ -66,7 +66,10 @@ typedef enum {
   KVQ_MODE_LM_QJL = 0,  /* rotation + b-bit Lloyd-Max code + 1-bit QJL residual sketch */
   KVQ_MODE_LM = 1,      /* rotation + b-bit Lloyd-Max code, no sketch */
   KVQ_MODE_SIGN1 = 2,   /* rotation + one sign bit per coordinate (1-bit Lloyd-Max) */
-  KVQ_MODE_FP4 = 3      /* FP4 E2M1 latent, one E4M3 scale per 16 channels (MLA caches) */
+  KVQ_MODE_FP4 = 3,     /* FP4 E2M1 latent, one E4M3 scale per 16 channels (MLA caches) */
+  KVQ_MODE_KIVI = 4     /* KIVI-style asymmetric integers, no rotation: keys per channel over groups of 128
+                           tokens, values per token (k_mode == v_mode, k_bits == v_bits == 2). The
+                           tokens of a sequence's incomplete last key group stay bf16 until it fills */
 } kvq_mode;
 
 typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
