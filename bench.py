@@ -30,7 +30,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from kvq_inputs import WORKLOADS, generate  # noqa: E402
+from kvq_inputs import WORKLOADS, VARIANTS, generate  # noqa: E402
 from kvq_inputs.workloads import rotation_and_sketch  # noqa: E402
 
 L2_BYTES = 126 * 2 ** 20
@@ -46,7 +46,9 @@ def workload_config(w, world):
             "head_dim": w.latent_dim if fp4 else w.head_dim, "ctx": w.ctx,
             "codec": f"K {w.k_mode}{w.k_bits} / V {w.v_mode}{w.v_bits}",
             "l2": "inputs larger than L2: cache replicas (> 2.5 x 126 MB in total) rotated per step",
-            "parallelism": f"replicas{world}"}
+            "parallelism": f"replicas{world}",
+            **({"window": {"sink": w.sink_tokens, "recent": w.recent_tokens}} if (w.sink_tokens or w.recent_tokens) else {}),
+            **({"paged": "64-token pages, shuffled pool"} if w.paged else {})}
 
 
 def parse():
@@ -69,8 +71,23 @@ KERNEL_NAMES = {
     "tiny": "decode_lm_mma<1, 2, 1, 2, 1>", "llama8b": "decode_lm_mma<4, 2, 1, 2, 1>",
     "llama70b": "decode_lm_mma<4, 3, 1, 3, 0>", "onebit": "decode_lm_mma<4, 1, 0, 1, 0>",
     "mla_fp4": "decode_mla_umma",
+    "llama8b_kivi": "decode_kivi<4>", "llama8b_window": "decode_lm_tc<4, 2, 1, 2, 1> + window_decode",
+    "llama8b_paged": "decode_lm_tc<4, 2, 1, 2, 1> (paged)",
 }
-EXTRA_WORKLOADS = ("llama8b", "onebit", "mla_fp4", "llama70b")
+EXTRA_WORKLOADS = ("llama8b", "onebit", "mla_fp4", "llama70b", "llama8b_kivi", "llama8b_window", "llama8b_paged")
+
+
+def workload(name):
+    return WORKLOADS[name] if name in WORKLOADS else VARIANTS[name]
+
+
+def coded_len(w, L):
+    """Tokens of a sequence of length L that the split kernel reads (the coded history)."""
+    if w.k_mode == "kivi":
+        return L // 128 * 128
+    if w.sink_tokens or w.recent_tokens:
+        return max(0, L - w.sink_tokens - w.recent_tokens)
+    return L
 
 # DRAM bytes (read + write) of one launch of the split decode kernel, and the load efficiency of its
 # packed streams, from ncu captures (full size, or a smaller context scaled to the full launch by the
@@ -347,7 +364,14 @@ def measure(kvq, w, args, world, dev):
 
     # Prefix of ctx - 1 tokens in every replica (identical content), built in sequence slices. The
     # caches draw their rotation signs and sketch matrix from the configuration's seeds.
-    caches = [kvq.KvqCache(cfg, w.batch, capacity, device=dev) for _ in range(replicas)]
+    def make_cache(r):
+        if not w.paged:
+            return kvq.KvqCache(cfg, w.batch, capacity, device=dev)
+        pps = (capacity + 63) // 64  # pages of 64 tokens per sequence, shuffled over the pool
+        perm = torch.randperm(w.batch * pps, generator=torch.Generator().manual_seed(r)).to(torch.int32)
+        table = perm.reshape(w.batch, pps).to(dev)
+        return kvq.KvqCache(cfg, w.batch, 0, device=dev, block_table=table, n_pages=w.batch * pps)
+    caches = [make_cache(r) for r in range(replicas)]
     step_b = max(1, w.batch // 8)
     q = None
     a_name, b_name = ("latent", "rope") if w.k_mode == "fp4" else ("k", "v")
@@ -367,6 +391,8 @@ def measure(kvq, w, args, world, dev):
         q = d["q"] if q is None else torch.cat([q, d["q"]])
         del d
     n_vec = w.batch * (w.ctx - 1) * (1 if w.k_mode == "fp4" else 2 * w.n_kv_heads)
+    if w.k_mode != "fp4":  # vectors actually coded by the prefill (the window keeps the rest in bf16)
+        n_vec = w.batch * coded_len(w, w.ctx - 1) * 2 * w.n_kv_heads
     # New tokens of every step, resident in HBM (the e2e steps draw theirs on the host).
     news = []
     for s in range(n_steps):
@@ -419,7 +445,7 @@ def measure(kvq, w, args, world, dev):
     torch.cuda.synchronize()
     kern_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in kev) / n_k for i in range(3)]
     kern_ms = [max_over_ranks(x, world) for x in kern_ms]
-    lens_k = sum(int(caches[j % replicas].lengths()[0]) for j in range(n_k)) / n_k
+    lens_k = sum(coded_len(w, int(caches[j % replicas].lengths()[0])) for j in range(n_k)) / n_k
 
     # End to end through the library's host-buffer call (kvq_decode_step_host): every step's new
     # keys, values and query start in pinned host memory and its output ends there. The library
@@ -457,7 +483,7 @@ def measure(kvq, w, args, world, dev):
     d2h = host_outs[0].numel() * host_outs[0].element_size()
 
     peaks, peak_kind = measured_peaks()
-    bytes_step = w.batch * heads_kv * (lens0 + 1) * per_tok  # packed bytes one decode call reads
+    bytes_step = w.batch * heads_kv * coded_len(w, lens0 + 1) * per_tok  # packed bytes one decode call reads
     call_ms = sum(kern_ms)  # kvq_decode_attention alone, from the per-kernel events
     achieved_call = bytes_step / (call_ms / 1e3) / 1e9
     bytes_kernel = w.batch * heads_kv * lens_k * per_tok      # the split kernel's algorithmic bytes
@@ -526,11 +552,12 @@ def run_ours(args, world, rank, local):
     if extra:
         line["workloads"] = {}
         for name in extra:
-            line["workloads"][name] = measure(kvq, WORKLOADS[name], args, world, dev)
+            line["workloads"][name] = measure(kvq, workload(name), args, world, dev)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, 10.0)
         for name in extra:
-            line["workloads"][name]["cpu_baseline"] = cpu_baseline(WORKLOADS[name], 3.0)
+            if name in WORKLOADS:  # the variants' oracle is the same decode over another codec
+                line["workloads"][name]["cpu_baseline"] = cpu_baseline(WORKLOADS[name], 3.0)
     if rank == 0:
         print(json.dumps(line))
 

@@ -12,4 +12,4 @@ bench) and the CPU oracle consume, so that both see identical inputs:
   drawn with torch's seeded generators on whatever device the caller names.
 """
 from .rng import splitmix64, uniform53, rotation_signs, qjl_matrix  # noqa: F401
-from .workloads import WORKLOADS, Workload, get_workload, generate  # noqa: F401
+from .workloads import WORKLOADS, VARIANTS, Workload, get_workload, generate  # noqa: F401

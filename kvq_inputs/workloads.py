@@ -53,6 +53,7 @@ class Workload:
     rot_per_head: bool = False  # one rotation diagonal per KV head
     sink_tokens: int = 0        # mixed-precision window: first tokens kept in bf16
     recent_tokens: int = 0      # and last tokens kept in bf16
+    paged: bool = False         # cache tiles in a shuffled pool of 64-token pages (block table)
 
     @property
     def data_seed(self) -> int:
@@ -92,8 +93,18 @@ WORKLOADS = {
 }
 
 
+# Variants of the 8B-shaped layer for the codec features beside the main path: the KIVI-style codec,
+# OSCAR's mixed-precision window (64 sink + 256 recent tokens in bf16: 0.24% of a 128k context), and
+# a paged cache (pages of 64 tokens in a shuffled pool).
+VARIANTS = {
+    "llama8b_kivi": WORKLOADS["llama8b"].with_(name="llama8b_kivi", k_mode="kivi", v_mode="kivi", qjl_dim=0),
+    "llama8b_window": WORKLOADS["llama8b"].with_(name="llama8b_window", sink_tokens=64, recent_tokens=256),
+    "llama8b_paged": WORKLOADS["llama8b"].with_(name="llama8b_paged", paged=True),
+}
+
+
 def get_workload(name: str) -> Workload:
-    return WORKLOADS[name]
+    return WORKLOADS[name] if name in WORKLOADS else VARIANTS[name]
 
 
 # ---- fixed per-(kv-head, channel) structure ------------------------------------------------
