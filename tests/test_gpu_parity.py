@@ -533,3 +533,52 @@ def test_tcgen05_and_mma_sync_kernels_agree(name, monkeypatch):
     assert np.all(err <= REL_TOL), err.max()
     c_mma.close()
     c_tc.close()
+
+
+# ---------------------------------------------------------------- instances and edge cases
+
+def test_query_group_of_two():
+    w = WORKLOADS["llama8b"].with_(n_q_heads=16)
+    run_small("llama8b", 2, [900, 65], seed_appends=2, w=w)
+
+
+@pytest.mark.parametrize("heads", [8, 32])
+def test_fp4_mma_sync_head_counts(heads):
+    """8 and 32 query heads decode on the mma.sync MLA kernel (64 on tcgen05, 16 tested above)."""
+    fp4_check(0, batch=2, lens=[900, 33], n_q_heads=heads)
+
+
+@pytest.mark.parametrize("kb,kq,vb,vq", [(2, True, 2, False), (3, True, 3, True), (2, False, 2, False),
+                                         (3, False, 3, False)])
+def test_other_code_combinations(kb, kq, vb, vq):
+    w = WORKLOADS["llama8b"].with_(k_bits=kb, v_bits=vb, k_mode="lm_qjl" if kq else "lm",
+                                   v_mode="lm_qjl" if vq else "lm", qjl_dim=128 if (kq or vq) else 0)
+    run_small("llama8b", 2, [700, 100], seed_appends=2, w=w)
+    w8 = WORKLOADS["llama70b"].with_(k_bits=kb, v_bits=vb, k_mode="lm_qjl" if kq else "lm",
+                                     v_mode="lm_qjl" if vq else "lm", qjl_dim=128 if (kq or vq) else 0)
+    run_small("llama70b", 1, [400], w=w8)
+
+
+def test_zero_key_and_value_vectors():
+    """A zero key (norm 0: no logit contribution, n = 0 stored) and a zero value, end to end."""
+    w = WORKLOADS["llama8b"].with_(batch=2)
+    T = 300
+    data = generate(w, DEV, seqs=range(2), ctx=T)
+    data["k"][0, 1, 7] = 0
+    data["v"][0, 1, 9] = 0
+    data["k"][1, :, 100] = 0
+    data["v"][1, :, 100] = 0
+    cache, signs, S = new_cache(w, 2, T + 32)
+    cache.quantize(data["k"], data["v"])
+    out = f64(cache.decode(data["q"]))
+    torch.cuda.synchronize()
+    arena, info = cache.arena.cpu().numpy(), cache.layout()
+    stats = {}
+    for b, hk in ((0, 1), (1, 3)):
+        g = w.group
+        ref = pair_reference(w, arena, info, b, hk, T, f64(data["k"][b, hk]), f64(data["v"][b, hk]),
+                             f64(data["q"][b, hk * g:(hk + 1) * g]), signs, S, stats)
+        assert np.all(rel_err(out[b, hk * g:(hk + 1) * g], ref) <= REL_TOL)
+    _, _, kn, _ = side_fields(arena, info, 0, 0 * w.n_kv_heads + 1, T)
+    assert kn[7] == 0
+    cache.close()
