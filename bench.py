@@ -71,8 +71,8 @@ KERNEL_NAMES = {
     "tiny": "decode_lm_mma<1, 2, 1, 2, 1>", "llama8b": "decode_lm_mma<4, 2, 1, 2, 1>",
     "llama70b": "decode_lm_mma<4, 3, 1, 3, 0>", "onebit": "decode_lm_mma<4, 1, 0, 1, 0>",
     "mla_fp4": "decode_mla_umma",
-    "llama8b_kivi": "decode_kivi<4>", "llama8b_window": "decode_lm_tc<4, 2, 1, 2, 1> + window_decode",
-    "llama8b_paged": "decode_lm_tc<4, 2, 1, 2, 1> (paged)",
+    "llama8b_kivi": "decode_lm_tc<4, 2, 0, 2, 0, kivi>", "llama8b_window": "decode_lm_mma<4, 2, 1, 2, 1> + window_decode",
+    "llama8b_paged": "decode_lm_mma<4, 2, 1, 2, 1> (paged)",
 }
 EXTRA_WORKLOADS = ("llama8b", "onebit", "mla_fp4", "llama70b", "llama8b_kivi", "llama8b_window", "llama8b_paged")
 

@@ -251,7 +251,7 @@ const std::vector<int>& coded_lens(const kvq_cache* c) { return has_window(c) ? 
 // Resident decode CTAs per SM for a chunk of `units` 64-token units: one for the MLA kernel, the
 // tensor-core kernel's shared-memory and register limit for query groups of 1, 2 or 4, else 4.
 int decode_slots_per_sm(const kvq_cache* c, int units) {
-  if (c->is_fp4 || c->tc) return 1;
+  if (c->is_fp4 || c->tc || c->kivi_tc) return 1;
   if (c->kivi) return 8;
   const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
   if (group == 1 || group == 2 || group == 4)
@@ -262,15 +262,15 @@ int decode_slots_per_sm(const kvq_cache* c, int units) {
 // Largest chunk (in 64-token units) one decode CTA may take.
 int decode_max_units(const kvq_cache* c) {
   if (c->is_fp4) return 1 << 30;
-  if (c->tc) return tc_chunk_max(c->cfg.n_q_heads / c->cfg.n_kv_heads) / (kTile * kTilePair);
+  if (c->tc || c->kivi_tc) return tc_chunk_max(c->cfg.n_q_heads / c->cfg.n_kv_heads) / (kTile * kTilePair);
   return kChunkMax / (kTile * kTilePair);
 }
 
-// The LM decode kernel a cache uses: the tcgen05 kernel where it has an instance, unless the
-// environment variable KVQ_DECODE_KERNEL is "mma" (the mma.sync kernel, for comparison).
+// The LM decode kernel a cache uses: the mma.sync kernel (measured faster), or the tcgen05 kernel
+// when the environment variable KVQ_DECODE_KERNEL is "tc" at cache creation.
 bool choose_tc(const kvq_cfg& cfg, const SideLayout& k, const SideLayout& v) {
   const char* e = std::getenv("KVQ_DECODE_KERNEL");
-  if (e && std::strcmp(e, "mma") == 0) return false;
+  if (!e || std::strcmp(e, "tc") != 0) return false;
   return k.order == kOrderOctet && tc_modes_supported(cfg.n_q_heads / cfg.n_kv_heads, k.bits, k.qjl, v.bits, v.qjl);
 }
 
@@ -414,6 +414,10 @@ kvq_status cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_
   }
   c->signs_stride = cfg->rot_per_head ? kHeadDim : 0;
   c->tc = !P.fp4_mode && !P.kivi && choose_tc(*cfg, P.k, P.v);
+  {
+    const char* e = std::getenv("KVQ_DECODE_KERNEL");
+    c->kivi_tc = P.kivi && !(e && (std::strcmp(e, "mma") == 0 || std::strcmp(e, "cuda") == 0));
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   c->table = table;
   c->pages_per_seq = table ? pages_per_seq : 0;
@@ -740,7 +744,12 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
     p.groups_per_seq = c->groups_per_seq;
   }
   if (c->kivi) {  // KIVI: the split kernel over the coded groups, the window, the reduce (no rotation)
-    if (!rec(1) || launch_decode_kivi(p, s) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
+    if (c->kivi_tc && p.chunk % (2 * kTile * kTilePair)) {  // whole 128-token key groups per CTA
+      p.chunk += kTile * kTilePair;
+      p.splits = std::max(1, (max_len + p.chunk - 1) / p.chunk);
+    }
+    if (!rec(1) || (c->kivi_tc ? launch_decode_kivi_tc(p, s) : launch_decode_kivi(p, s)) != cudaSuccess || !rec(2))
+      return KVQ_ERR_CUDA;
     if (launch_window_decode(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
     if (launch_reduce_lm(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
     return KVQ_OK;

@@ -32,6 +32,7 @@
 // Partials (m, l, o_r, acc_z) are written in the format of the other LM kernels; the same reduce
 // kernel finishes.
 #include <algorithm>
+#include <type_traits>
 
 #include <cuda_fp16.h>
 
@@ -53,7 +54,20 @@ constexpr uint32_t kTmemColsT = 512;
 constexpr int kNormBlockT = 4 * 128;   // staged value norms (+ residual norms) of four tiles
 constexpr int kKN = 16;                // key-phase N: (head, digit) columns, padded
 
-template <int G, int KB, bool KQ, int VB, bool VQ>
+// KIVI value tile: two code planes (byte-lane order), per-token fp16 scale and zero.
+struct KiviVTile {
+  static constexpr int PLANES = 0, SKETCH = 2 * kTile * 16, NORM = SKETCH, GAMMA = NORM + kTile * 2;
+  static constexpr int BYTES = GAMMA + kTile * 2;
+  static bool matches(const SideLayout& L) {
+    return L.off_planes == PLANES && L.off_norm == NORM && L.off_gamma == GAMMA && L.tile_bytes == BYTES && L.bits == 2 &&
+           !L.qjl;
+  }
+};
+constexpr int kKiviStats = 2 * kHeadDim * 2;  // a key group's fp16 scales and zeros
+
+// KV: the KIVI instance (2-bit unsigned codes b0 + 2 b1 instead of Walsh planes; per-group query
+// digits; per-token value scale and zero; no rotation).
+template <int G, int KB, bool KQ, int VB, bool VQ, bool KV = false>
 struct TcCfg {
   static constexpr int KWP = Walsh<KB>::P, KP = KWP + (KQ ? 1 : 0);  // key planes (sketch last)
   static constexpr int VWP = Walsh<VB>::P, VP = VWP + (VQ ? 1 : 0);  // value planes (sketch last)
@@ -71,10 +85,11 @@ struct TcCfg {
   static constexpr int NTASK = G * kTokT / TPT;         // weight tasks per iteration (<= threads)
   static_assert(NTASK <= kThreadsT && TPT <= 4, "one weight task per thread");
   using KL = TileLayout<KB, KQ>;
-  using VL = TileLayout<VB, VQ>;
-  static constexpr int STAGE = ((4 * KL::BYTES + kNormBlockT > 4 * VL::BYTES ? 4 * KL::BYTES + kNormBlockT
-                                                                             : 4 * VL::BYTES) + 127) / 128 * 128;
-  static constexpr int BK = KP * kKN * 128;  // query digits: [KP][16 rows][128 K bytes] core matrices
+  using VL = std::conditional_t<KV, KiviVTile, TileLayout<VB, VQ>>;
+  static constexpr int KSTAGE = 4 * KL::BYTES + kNormBlockT + (KV ? kKiviStats : 0);
+  static constexpr int STAGE = ((KSTAGE > 4 * VL::BYTES ? KSTAGE : 4 * VL::BYTES) + 127) / 128 * 128;
+  // query digits: [KP][16 rows][128 K bytes] core matrices (KIVI: two buffers, rebuilt per group)
+  static constexpr int BK = (KV ? 2 : 1) * KP * kKN * 128;
   static constexpr int BV = VN * kTokT;      // one weight-digit buffer: [VN rows][128 tokens]
 };
 
@@ -86,7 +101,7 @@ __host__ __device__ inline int tc_logit_stride(int chunk) { return (chunk + kTok
 template <class C>
 size_t tc_smem_bytes(int G, int chunk) {
   return (size_t)kStagesT * C::STAGE + C::BK + 2 * C::BV + sizeof(float) * (size_t)G * tc_logit_stride(chunk) +
-         sizeof(float) * (size_t)(8 * G + 16 + 3 * kThreadsT);
+         sizeof(float) * (size_t)(8 * G + 16 + 4 * kThreadsT) + sizeof(float) * (size_t)G * (kHeadDim + 4 + 24);
 }
 
 // Byte offset of (row n, K index k) in a K-major operand of core matrices with `kchunks` 16-byte K
@@ -95,9 +110,9 @@ __device__ __forceinline__ int core_off(int n, int k, int kchunks) {
   return ((n >> 3) * kchunks + (k >> 4)) * 128 + (n & 7) * 16 + (k & 15);
 }
 
-template <int G, int KB, bool KQ, int VB, bool VQ>
+template <int G, int KB, bool KQ, int VB, bool VQ, bool KV>
 __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_constant__ DecodeParams p) {
-  using C = TcCfg<G, KB, KQ, VB, VQ>;
+  using C = TcCfg<G, KB, KQ, VB, VQ, KV>;
   using KL = typename C::KL;
   using VL = typename C::VL;
   constexpr int KP = C::KP, KWP = C::KWP, VP = C::VP, VWP = C::VWP, NK0 = C::NK0, GH = C::GH, TPT = C::TPT;
@@ -113,7 +128,12 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
   unsigned char* bk = stages + kStagesT * C::STAGE;
   unsigned char* bv = bk + C::BK;
   float* lgs = reinterpret_cast<float*>(bv + 2 * C::BV);
-  float* red = lgs + G * lgst;  // [8][G] maxima | [16] weight maxima | [3][threads] task sums
+  float* red = lgs + G * lgst;  // [8][G] maxima | [16] weight maxima | [4][threads] task sums
+  // KIVI: q * scale * log2(e) [G][d], per-iteration head scales and offsets [2][G] each, reductions [8][G] x 2
+  float* qsm = red + 8 * G + 16 + 4 * kThreadsT;
+  float* hsk = qsm + G * kHeadDim;
+  float* hck = hsk + 2 * G;
+  float* kred = hck + 2 * G;
 
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -168,7 +188,10 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
     fence_proxy_async();  // the stage's previous contents were read by the generic proxy
     if (f < n_iter) {
       constexpr uint32_t nb = VQ ? 128u : 64u;  // value norms (+ gammas, contiguous) per tile
-      mbar_arrive_expect_tx(bar, (uint32_t)npairs * 2u * (ktb + nb));
+      mbar_arrive_expect_tx(bar, (uint32_t)npairs * 2u * (ktb + nb) + (KV ? (uint32_t)kKiviStats : 0u));
+      if (KV)  // the key group's statistics (iterations are whole 128-token groups)
+        bulk_g2s(smem_addr(dst + 4 * ktb + kNormBlockT),
+                 p.kstats + (pair * p.groups_per_seq + (unsigned)t0 / kTokT) * (size_t)kKiviStats, kKiviStats, bar);
       for (int j = 0; j < npairs; ++j) {
         const long ti = pair_index(tile0 + 2 * j);
         bulk_g2s(smem_addr(dst + 2 * j * ktb), kreg + (size_t)ti * ktb, 2u * ktb, bar);
@@ -210,7 +233,13 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
   // ---- B_k: query digits of every plane in the octet words' byte order. K index 4x + i is byte i
   // of word x = 8t + 2m + hh, i.e. coordinate 32m + 16hh + 4t + i; row n = 2 h + digit.
   const int npiece = p.hsplit, gp = G / npiece;  // prep pieces of gp heads
-  for (int idx = tid; idx < KP * kKN * 32; idx += kThreadsT) {
+  if (KV) {  // KIVI: the query itself; its digits are rebuilt per key group below
+    for (int idx = tid; idx < G * kHeadDim; idx += kThreadsT)
+      qsm[idx] = load_q(p.q, ((size_t)b * p.Hq + h_first + idx / kHeadDim) * kHeadDim + idx % kHeadDim, p.bf16) *
+                 p.logit_scale;
+    for (int idx = tid; idx < C::BK / 4; idx += kThreadsT) reinterpret_cast<uint32_t*>(bk)[idx] = 0u;
+  }
+  for (int idx = tid; idx < (KV ? 0 : KP * kKN * 32); idx += kThreadsT) {
     const int P = idx / (kKN * 32), n = (idx / 32) % kKN, x = idx % 32;
     uint32_t v = 0u;
     if (n < 2 * G) {
@@ -226,6 +255,8 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
   float hs[GH], hc[GH], hsz[GH], hcz[GH];
 #pragma unroll
   for (int i = 0; i < GH; ++i) {
+    hs[i] = hc[i] = hsz[i] = hcz[i] = 0.f;
+    if (KV) continue;
     const int h = min(hf * GH + i, G - 1), pc = h / gp, hp = h % gp;
     const float* hconst =
         reinterpret_cast<const float*>(p.qprep + (pair * npiece + pc) * p.qprep_stride + KP * gp * 2 * 128);
@@ -298,6 +329,16 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
       const int c0 = (int)dm[2 * j], c1 = (int)dm[2 * j + 1];
       // hi * 256 + lo: exact in int32 up to 2 Walsh planes, else in fp32
       const float cc = KB <= 2 ? (float)(c0 * 256 + c1) : fmaf((float)c0, 256.f, (float)c1);
+      if (KV) {  // KIVI: this group's digit scale and zero-point offset; no per-token norm
+        const int hh = min(h, G - 1);
+        const float lk = fmaf(hsk[(i & 1) * G + hh] * rowf, cc, hck[(i & 1) * G + hh]);
+        const float lgk = valid ? lk : -INFINITY;
+        if (h < G) {
+          lgs[h * lgst + tok] = lgk;
+          mrow[j] = fmaxf(mrow[j], lgk);
+        }
+        continue;
+      }
       float l = fmaf(hs[j] * rowf, cc, hc[j]);
       if (KQ) {
         const int z0 = (int)dz[2 * j], z1 = (int)dz[2 * j + 1];
@@ -319,12 +360,74 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
     const unsigned char* kt = stages + ((unsigned)it % kStagesT) * C::STAGE;
     // this thread's token row: tile qtr, octet `oct` (words of every plane at stride 512)
     const unsigned char* krow = kt + qtr * ktb + oct * 128;
+    if (KV) {
+      // KIVI: the query digits of this key group, B_P[j] = 2^P q_j s_j (codes b0 + 2 b1), 16-bit
+      // integers relative to the head's largest |2 q_j s_j|, into buffer it & 1; the head's offset
+      // sum_j q_j z_j. Thread: coordinate j = tid % 128, heads tid / 128, + 2, ..
+      const __half* st = reinterpret_cast<const __half*>(kt + 4 * ktb + kNormBlockT);
+      const int j = tid & (kHeadDim - 1), h0 = tid >> 7;
+      const float sj = __half2float(st[j]), zj = __half2float(st[kHeadDim + j]);
+      constexpr int HT = (G + 1) / 2;
+      float vq[HT];
+#pragma unroll
+      for (int u = 0; u < HT; ++u) {
+        const int h = h0 + 2 * u;
+        float a = 0.f, c = 0.f;
+        vq[u] = 0.f;
+        if (h < G) {
+          vq[u] = qsm[h * kHeadDim + j] * sj;
+          a = fabsf(vq[u]);
+          c = qsm[h * kHeadDim + j] * zj;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+          c += __shfl_xor_sync(0xffffffffu, c, o);
+        }
+        if (lane == 0 && h < G) {
+          kred[warp * G + h] = a;
+          kred[8 * G + warp * G + h] = c;
+        }
+      }
+      __syncthreads();
+      if (tid < G) {  // head tid: warps 4 (tid & 1) .. +3 covered its coordinates
+        const int w0 = 4 * (tid & 1);
+        float a = 0.f, c = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          a = fmaxf(a, kred[(w0 + w) * G + tid]);
+          c += kred[8 * G + (w0 + w) * G + tid];
+        }
+        const float vmax = 2.f * a;
+        hsk[(it & 1) * G + tid] = (vmax > 0.f ? vmax : 1.f) / ((float)kQRange * -128.f);
+        hck[(it & 1) * G + tid] = c;
+        kred[16 * G + tid] = (float)kQRange / (vmax > 0.f ? vmax : 1.f);
+      }
+      __syncthreads();
+      // K index of coordinate j = 32 m + 16 hh + 4 t + i: 4 (8 t + 2 m + hh) + i
+      const int kidx = 4 * (8 * ((j >> 2) & 3) + 2 * (j >> 5) + ((j >> 4) & 1)) + (j & 3);
+      unsigned char* bkb = bk + (it & 1) * (KP * kKN * 128);
+#pragma unroll
+      for (int u = 0; u < HT; ++u) {
+        const int h = h0 + 2 * u;
+        if (h >= G) continue;
+        const float qs = kred[16 * G + h];
+#pragma unroll
+        for (int P = 0; P < 2; ++P) {
+          const int q = __float2int_rn((float)(1 << P) * vq[u] * qs);
+          const int hi = (q + 128) >> 8, lo = q - 256 * hi;
+          bkb[P * (kKN * 128) + core_off(2 * h, kidx, 8)] = (unsigned char)(hi & 0xFF);
+          bkb[P * (kKN * 128) + core_off(2 * h + 1, kidx, 8)] = (unsigned char)(lo & 0xFF);
+        }
+      }
+      fence_proxy_async();  // the digits are read by the tensor cores after the barrier below
+    }
     expand(krow, abuf, KP, KWP, KB, KL::SKETCH, kmask, 16);
     const float nk = __half2float(*reinterpret_cast<const __half*>(kt + qtr * ktb + KL::NORM + lane * 2));
     const float gk = KQ ? __half2float(*reinterpret_cast<const __half*>(kt + qtr * ktb + KL::GAMMA + lane * 2)) : 0.f;
     if (tid < kTokT && t_begin + it * kTokT + tid < t_end) {  // largest value weight of each kind
       const unsigned char* nb = kt + 4 * ktb + (tid / kTile) * 128 + (tid % kTile) * 2;
-      const float w = __half2float(*reinterpret_cast<const __half*>(nb)) * kInvSqrtD;
+      const float w = __half2float(*reinterpret_cast<const __half*>(nb)) * (KV ? 1.f : kInvSqrtD);
       wmax = fmaxf(wmax, w);
       if (VQ) wmaxz = fmaxf(wmaxz, w * (__half2float(*reinterpret_cast<const __half*>(nb + 64)) * (kSqrtHalfPi / (float)p.v.m)));
     }
@@ -335,7 +438,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
       tc::fence_after();
       const uint32_t a0 = tmem + C::COL_A + abuf * C::APL * 32;
       const uint32_t dk = tmem + C::COL_DK + (it & 1) * 2 * kKN;
-      const uint32_t bk0 = smem_addr(bk);
+      const uint32_t bk0 = smem_addr(bk) + (KV ? (it & 1) * (KP * kKN * 128) : 0);
 #pragma unroll
       for (int P = 0; P < KP; ++P) {
         const bool sk = KQ && P == KP - 1;
@@ -386,7 +489,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
   if (has_task)
     for (int w = 0; w < 8; ++w)
       if ((w >> 2) * GH <= task_h && task_h < (w >> 2) * GH + GH) task_m = fmaxf(task_m, hmax[w * G + task_h]);
-  float task_l = 0.f;
+  float task_l = 0.f, task_zs = 0.f;  // task_zs (KIVI): sum of p_t z_t
   uint32_t task_wc = 0, task_wz = 0;
   // value rows: coordinate 32 qtr + lane = byte lane (4 qtr + lane / 8), bit lane % 8
   const int vlane = 4 * qtr + (lane >> 3);
@@ -415,8 +518,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
         const float pe = ok ? ex2(lv - task_m) : 0.f;
         psum += pe;
         const float nrm = ok ? __half2float(*reinterpret_cast<const __half*>(vtile + VL::NORM + (T % kTile) * 2)) : 0.f;
-        bc[e] = __float_as_uint(fmaf(pe, nrm * (kInvSqrtD * wsc), kRoundBias));
+        bc[e] = __float_as_uint(fmaf(pe, nrm * ((KV ? 1.f : kInvSqrtD) * wsc), kRoundBias));
         task_wc += bc[e] - 0x4B000000u;
+        if (KV && ok) task_zs = fmaf(pe, __half2float(*reinterpret_cast<const __half*>(vtile + VL::GAMMA + (T % kTile) * 2)), task_zs);
         if (VQ) {
           const float gz = ok ? __half2float(*reinterpret_cast<const __half*>(vtile + VL::GAMMA + (T % kTile) * 2)) : 0.f;
           bz[e] = __float_as_uint(fmaf(pe, nrm * gz * (kInvSqrtD * wscz * vkappa), kRoundBias));
@@ -508,8 +612,9 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
   tsum[tid] = task_l;
   tsum[kThreadsT + tid] = (float)task_wc;
   tsum[2 * kThreadsT + tid] = (float)task_wz;
+  tsum[3 * kThreadsT + tid] = task_zs;
   __syncthreads();
-  float* hsum = hmax;  // [3][G] (the maxima are folded into registers first)
+  float* hsum = hmax;  // [4][G] (the maxima are folded into registers first)
   float mfin[GH];
 #pragma unroll
   for (int j = 0; j < GH; ++j) {
@@ -520,7 +625,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
     mfin[j] = mx;
   }
   __syncthreads();
-  if (tid < 3 * G) {
+  if (tid < 4 * G) {
     const int what = tid / G, h = tid % G;
     float s2 = 0.f;
     for (int q = 0; q < kTokT / TPT; ++q) s2 += tsum[what * kThreadsT + h * (kTokT / TPT) + q];
@@ -533,6 +638,11 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
   float vasum = 0.f;
 #pragma unroll
   for (int P = 0; P < VWP; ++P) vasum += va[P];
+  if (KV) {  // KIVI codes b0 + 2 b1: plane coefficients 1 and 2, no Walsh offset
+    va[0] = 0.5f;
+    va[1] = 1.f;
+    vasum = 0.f;
+  }
   const int j_c = 32 * qtr + lane;                  // this thread's coordinate row
   const float rowpos = 1.f / (float)(1 << jbit);    // row value 2^p (u8)
   const float rowinv = rowpos / wsc, rowinvz = rowpos / wscz;
@@ -564,7 +674,7 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
     const int h = hf * GH + j;
     if (h < G) {
       float* dst = p.part + (((size_t)b * p.Hq + h_first + h) * p.splits + split) * p.part_stride;
-      dst[2 + j_c] = o[j] - vasum * (hsum[G + h] / wsc);
+      dst[2 + j_c] = KV ? o[j] + hsum[3 * G + h] : o[j] - vasum * (hsum[G + h] / wsc);
       if (VQ) dst[2 + kHeadDim + j_c] = z[j] - hsum[2 * G + h] / wscz;
       if (lane == 0 && qtr == 0) {
         dst[0] = mfin[j];
@@ -584,16 +694,16 @@ __global__ void __launch_bounds__(kThreadsT, 1) decode_lm_tc(const __grid_consta
   }
 }
 
-template <int G, int KB, bool KQ, int VB, bool VQ>
+template <int G, int KB, bool KQ, int VB, bool VQ, bool KV = false>
 cudaError_t launch_tc(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
-  using C = TcCfg<G, KB, KQ, VB, VQ>;
+  using C = TcCfg<G, KB, KQ, VB, VQ, KV>;
   if (!C::KL::matches(p.k) || !C::VL::matches(p.v)) return cudaErrorNotSupported;
   if (p.k.order != kOrderOctet || p.v.order != kOrderByteLane) return cudaErrorNotSupported;
-  cudaError_t e = launch_lm_query_prep(p, s, qp);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!KV && (e = launch_lm_query_prep(p, s, qp)) != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
   const size_t smem = tc_smem_bytes<C>(G, p.chunk);
-  auto kern = decode_lm_tc<G, KB, KQ, VB, VQ>;
+  auto kern = decode_lm_tc<G, KB, KQ, VB, VQ, KV>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -641,6 +751,17 @@ bool tc_decode_supported(const DecodeParams& p) {
   return tc_modes_supported(p.group, p.k.bits, p.k.qjl, p.v.bits, p.v.qjl) && p.k.order == kOrderOctet &&
          p.chunk % 64 == 0 && p.chunk <= tc_chunk_max(p.group) && p.qprep != nullptr &&
          p.hsplit == (p.group > 4 ? 2 : 1);
+}
+
+cudaError_t launch_decode_kivi_tc(const DecodeParams& p, cudaStream_t s) {
+  if (p.chunk % kTokT) return cudaErrorNotSupported;  // iterations are whole key groups
+  switch (p.group) {
+    case 1: return launch_tc<1, 2, false, 2, false, true>(p, s, nullptr, nullptr);
+    case 2: return launch_tc<2, 2, false, 2, false, true>(p, s, nullptr, nullptr);
+    case 4: return launch_tc<4, 2, false, 2, false, true>(p, s, nullptr, nullptr);
+    case 8: return launch_tc<8, 2, false, 2, false, true>(p, s, nullptr, nullptr);
+    default: return cudaErrorNotSupported;
+  }
 }
 
 cudaError_t launch_decode_lm_tc(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {

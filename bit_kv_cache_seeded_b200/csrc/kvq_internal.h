@@ -183,6 +183,8 @@ bool tc_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl)
 bool tc_decode_supported(const DecodeParams& p);
 int tc_chunk_max(int group);     // largest chunk (tokens) of one CTA
 cudaError_t launch_decode_lm_tc(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp);
+// The tcgen05 kernel's KIVI instance (chunks of whole 128-token key groups).
+cudaError_t launch_decode_kivi_tc(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s);
 bool mla_mma_supported(const MlaParams& p);
@@ -218,6 +220,7 @@ struct kvq_cache {
   uint16_t* d_win = nullptr;// window caches: bf16 K then V window, [batch][kv-heads][sink + recent][d] each
   std::vector<int> hlens;   // host mirror of d_hlens
   bool kivi = false;        // KIVI codes (no rotation); the window is the incomplete last key group
+  bool kivi_tc = false;     // KIVI decode on the tcgen05 kernel (else the CUDA-core kernel)
   char* d_kstats = nullptr; // KIVI: [batch][kv-heads][groups][2][d] fp16 key scales and zeros
   int groups_per_seq = 0;
   char* dev = nullptr;

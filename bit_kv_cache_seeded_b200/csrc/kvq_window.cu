@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kWinThreads) window_write(const __grid_constan
 // recent tokens, in the split kernels' partial format (logits in log2 units; o in the rotated domain,
 // o_r = H D o / sqrt(d), so that the reduce's inverse rotation brings it back; no sketch part).
 __global__ void __launch_bounds__(kWinThreads) window_decode(const __grid_constant__ DecodeParams p) {
-  __shared__ float qs[kWinMaxG][kHeadDim];
+  __shared__ __align__(16) float qs[kWinMaxG][kHeadDim];
   __shared__ float lg[kWinMaxG][kWinMaxTokens];
   __shared__ float stat[kWinMaxG][2];  // max, sum
   __shared__ float os[kWinMaxG][kHeadDim];
@@ -82,21 +82,21 @@ __global__ void __launch_bounds__(kWinThreads) window_decode(const __grid_consta
     qs[h][j] = load_in(p.q, ((size_t)b * p.Hq + hk * G + h) * kHeadDim + j, p.bf16) * p.logit_scale;
   }
   __syncthreads();
-  // logits: token i by thread i (strided), all heads
-  for (int i = tid; i < n_tok; i += kWinThreads) {
-    const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(kw + (size_t)slot_of(i) * kHeadDim);
-    float acc[kWinMaxG];
+  // logits: token i by warp i % 8 (lane l: coordinates 4l .. 4l + 3), all heads, warp sums
+  const int nw = kWinThreads / 32;
+  for (int i = warp; i < n_tok; i += nw) {
+    const uint2 k4 = *reinterpret_cast<const uint2*>(kw + (size_t)slot_of(i) * kHeadDim + 4 * lane);
+    const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k4.x));
+    const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k4.y));
 #pragma unroll
-    for (int h = 0; h < kWinMaxG; ++h) acc[h] = 0.f;
-    for (int j2 = 0; j2 < kHeadDim / 2; ++j2) {
-      const float2 k2 = __bfloat1622float2(kr[j2]);
+    for (int h = 0; h < kWinMaxG; ++h) {
+      if (h >= G) break;
+      const float4 q4 = *reinterpret_cast<const float4*>(&qs[h][4 * lane]);
+      float v = fmaf(k23.y, q4.w, fmaf(k23.x, q4.z, fmaf(k01.y, q4.y, k01.x * q4.x)));
 #pragma unroll
-      for (int h = 0; h < kWinMaxG; ++h)
-        if (h < G) acc[h] = fmaf(k2.y, qs[h][2 * j2 + 1], fmaf(k2.x, qs[h][2 * j2], acc[h]));
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) lg[h][i] = v;
     }
-#pragma unroll
-    for (int h = 0; h < kWinMaxG; ++h)
-      if (h < G) lg[h][i] = acc[h];
   }
   __syncthreads();
   // per head: max, then weights 2^(l - m) in place and their sum (warp h)
@@ -116,14 +116,30 @@ __global__ void __launch_bounds__(kWinThreads) window_decode(const __grid_consta
     if (lane == 0) { stat[warp][0] = mx; stat[warp][1] = sm; }
   }
   __syncthreads();
-  // o[h][j] = sum_i w_i v_ij, signs applied (D o) for the rotation below
-  const float* sg = p.signs + hk * p.signs_stride;
-  for (int idx = tid; idx < G * kHeadDim; idx += kWinThreads) {
-    const int h = idx / kHeadDim, j = idx % kHeadDim;
-    float acc = 0.f;
-    for (int i = 0; i < n_tok; ++i)
-      acc = fmaf(lg[h][i], __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(vw)[(size_t)slot_of(i) * kHeadDim + j]), acc);
-    os[h][j] = p.win_kivi ? acc : acc * sg[j];
+  // o[h][j] = sum_i w_i v_ij: thread (j, half) takes every other token and all heads, loading each
+  // value element once; the two halves meet in shared memory. Signs applied (D o) for the rotation.
+  {
+    const int j = tid & (kHeadDim - 1), half = tid >> 7;
+    float acc[kWinMaxG];
+#pragma unroll
+    for (int h = 0; h < kWinMaxG; ++h) acc[h] = 0.f;
+    const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(vw);
+    for (int i = half; i < n_tok; i += 2) {
+      const float v = __bfloat162float(vb[(size_t)slot_of(i) * kHeadDim + j]);
+#pragma unroll
+      for (int h = 0; h < kWinMaxG; ++h)
+        if (h < G) acc[h] = fmaf(lg[h][i], v, acc[h]);
+    }
+    if (half == 1)
+#pragma unroll
+      for (int h = 0; h < kWinMaxG; ++h)
+        if (h < G) os[h][j] = acc[h];
+    __syncthreads();
+    const float* sg = p.signs + hk * p.signs_stride;
+    if (half == 0)
+#pragma unroll
+      for (int h = 0; h < kWinMaxG; ++h)
+        if (h < G) os[h][j] = p.win_kivi ? acc[h] + os[h][j] : (acc[h] + os[h][j]) * sg[j];
   }
   __syncthreads();
   if (p.win_kivi) {  // KIVI caches are not rotated: the state stays in the original domain

@@ -96,8 +96,13 @@ def key_stats(cache, arena, pair, g):
     return st[:128], st[128:]
 
 
+@pytest.mark.parametrize("kernel", ["tc", "cuda"])
 @pytest.mark.parametrize("name,lens", [("llama8b", [1000, 128, 127, 0]), ("llama70b", [700, 300]), ("tiny", [1024])])
-def test_kivi_prefill(name, lens):
+def test_kivi_prefill(name, lens, kernel, monkeypatch):
+    """Both KIVI decode kernels: the tcgen05 instance (default) and the CUDA-core one
+    (KVQ_DECODE_KERNEL=cuda)."""
+    if kernel == "cuda":
+        monkeypatch.setenv("KVQ_DECODE_KERNEL", "cuda")
     w = kivi_workload(name, len(lens))
     data = generate(w, DEV, seqs=range(len(lens)), ctx=max(lens))
     cache = kvq.KvqCache(kvq.cfg_for_workload(w), len(lens), max(lens) + 128)

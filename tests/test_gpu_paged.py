@@ -11,6 +11,7 @@ import torch
 import bit_kv_cache_seeded_b200 as kvq
 from kvq_inputs import WORKLOADS, generate
 from kvq_inputs.workloads import rotation_and_sketch
+from tests._cache_reader import side_fields
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -21,6 +22,14 @@ def _lib():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     kvq.load()
+
+
+def contiguous_info(info, side, ntiles):
+    """Layout info of a buffer holding just one (sequence, kv-head)'s ntiles tiles of one side at 0."""
+    i = np.array(info, copy=True)
+    i[3] = ntiles
+    i[4 + side] = 0
+    return i
 
 
 @pytest.mark.parametrize("name,lens", [("llama8b", [900, 64, 1]), ("llama70b", [700, 130]), ("onebit", [333, 64])])
@@ -43,7 +52,8 @@ def test_shuffled_pages_equal_contiguous(name, lens):
     o1, o2 = paged.decode(data["q"]), flat.decode(data["q"])
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
-    # every tile that holds tokens is byte-identical
+    # every stored token's fields are identical: its tile found through the block table in the pool,
+    # at its contiguous place in the other cache (bytes past a sequence's last token not compared)
     ip, ic = paged.layout(), flat.layout()
     A, B = paged.arena.cpu().numpy(), flat.arena.cpu().numpy()
     tiles_per_seq = int(ic[3])
@@ -51,10 +61,16 @@ def test_shuffled_pages_equal_contiguous(name, lens):
         tb = int(ic[1 + side])
         for b, L in enumerate(lens):
             for h in range(w.n_kv_heads):
-                for t in range((L + 31) // 32):
-                    pc = int(ic[4 + side]) + ((b * w.n_kv_heads + h) * tiles_per_seq + t) * tb
-                    pp = int(ip[4 + side]) + ((int(perm[b, t // 2]) * w.n_kv_heads + h) * 2 + t % 2) * tb
-                    np.testing.assert_array_equal(A[pp:pp + tb], B[pc:pc + tb])
+                ntiles = (L + 31) // 32
+                flat_tiles = np.stack([B[int(ic[4 + side]) + ((b * w.n_kv_heads + h) * tiles_per_seq + t) * tb:][:tb]
+                                       for t in range(ntiles)])
+                paged_tiles = np.stack([A[int(ip[4 + side]) + ((int(perm[b, t // 2]) * w.n_kv_heads + h) * 2 + t % 2) * tb:][:tb]
+                                        for t in range(ntiles)])
+                fa = side_fields(paged_tiles.reshape(-1), contiguous_info(ic, side, ntiles), side, 0, L)
+                fb = side_fields(flat_tiles.reshape(-1), contiguous_info(ic, side, ntiles), side, 0, L)
+                for x, y in zip(fa, fb):
+                    if x is not None:
+                        np.testing.assert_array_equal(x, y)
     assert kvq.kvq_cache_status(paged.handle) == 0
     paged.close()
     flat.close()
