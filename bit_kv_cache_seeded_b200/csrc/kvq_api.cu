@@ -221,7 +221,7 @@ int prep_stride(const kvq_cache* c) { return prep_piece_stride(c) * decode_hspli
 // Rows of the decode grid the split plan spreads over the SMs: (sequence, kv-head[, piece]).
 int decode_rows(const kvq_cache* c) {
   if (c->is_fp4) return c->batch;
-  return c->batch * c->cfg.n_kv_heads * (c->tc ? 1 : decode_hsplit(c));
+  return c->batch * c->cfg.n_kv_heads;  // every LM kernel takes all query heads of a kv-head per CTA
 }
 
 size_t partials_bytes(const kvq_cache* c, int splits) {
@@ -254,7 +254,7 @@ int decode_slots_per_sm(const kvq_cache* c, int units) {
   if (c->is_fp4 || c->tc || c->kivi_tc) return 1;
   if (c->kivi) return 8;
   const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
-  if (group == 1 || group == 2 || group == 4)
+  if (group == 1 || group == 2 || group == 4 || group == 8)
     return lm_mma_slots_per_sm(group, c->k, c->v, units * kTile * kTilePair);
   return 4;
 }

@@ -92,13 +92,20 @@ __device__ __forceinline__ uint32_t bit_to_s8(uint32_t w) {
   return (P == 7) ? (w & 0x80808080u) : ((w * (1u << (7 - P))) & 0x80808080u);
 }
 
+// Warps of a decode CTA: 4, or 8 for a query group of 8 (one CTA per kv-head: warps w and w + 4
+// take the same tokens for heads 0-3 and 4-7 in pass 1, and one value bit position each in pass 2).
+template <int G> struct Warps { static constexpr int N = G > 4 ? 8 : 4; };
+
 template <int G, int KB, bool KQ, int VB, bool VQ>
 struct MmaCfg {
+  static constexpr int NW = Warps<G>::N, NT = NW * 32;
+  static constexpr int GW = G > 4 ? 4 : G;                // heads of one warp's logits
   static constexpr int KP = Walsh<KB>::P + (KQ ? 1 : 0);  // logit planes (sketch last)
   static constexpr int VP = Walsh<VB>::P + (VQ ? 1 : 0);  // value planes (sketch last)
-  static constexpr int KNT = (2 * G + 7) / 8;             // logit N-tiles: (head, 2 digits)
+  static constexpr int KNT = (2 * GW + 7) / 8;            // logit N-tiles: (head, 2 digits)
   static constexpr int VNT = (4 * G + 7) / 8;             // value N-tiles: (head, 3 digits + pad)
   static constexpr int VNCOL = VNT * 8;
+  static constexpr int PPW = 8 / NW;                      // value bit positions per warp
 };
 
 // Dynamic shared memory of one decode CTA: the staging ring, the chunk's logits, the two weight
@@ -106,10 +113,11 @@ struct MmaCfg {
 size_t mma_smem_bytes(int group, const SideLayout& k, const SideLayout& v, int chunk) {
   const int nkind = v.qjl ? 2 : 1;
   const int vncol = ((4 * group + 7) / 8) * 8;
+  const int nw = group > 4 ? 8 : 4;
   size_t s = (size_t)kStagesM * std::max(2 * k.tile_bytes + kNormBlock, 2 * v.tile_bytes);
   s += sizeof(float) * (size_t)group * (chunk + 8);
   s += 2 * (size_t)nkind * vncol * kPdStride;
-  s += sizeof(float) * (kWarpsM * group + 2 * kWarpsM);
+  s += sizeof(float) * (nw * group + 2 * nw);
   return (s + 15) / 16 * 16;
 }
 
@@ -294,17 +302,18 @@ decode_front(const __grid_constant__ QuantizeParams qp, const __grid_constant__ 
 // Decode kernel (two passes over the CTA's chunk).
 // ------------------------------------------------------------------------------------------
 template <int G, int KB, bool KQ, int VB, bool VQ>
-__global__ void __launch_bounds__(kThreadsM, kMinBlocksM)
+__global__ void __launch_bounds__(Warps<G>::N * 32, 16 / Warps<G>::N)
 decode_lm_mma(const __grid_constant__ DecodeParams p) {
   using C = MmaCfg<G, KB, KQ, VB, VQ>;
   constexpr int KP = C::KP, VP = C::VP, KNT = C::KNT, VNT = C::VNT, VNCOL = C::VNCOL;
+  constexpr int NW = C::NW, NT = C::NT, GW = C::GW, PPW = C::PPW;
   constexpr int VWP = Walsh<VB>::P;
   constexpr int NKIND = VQ ? 2 : 1;
   // weight tasks: (head, TPT consecutive tokens), both kinds; spread over all threads
-  constexpr int TPT = (G * kCtaTok) / kThreadsM > 0 ? (G * kCtaTok) / kThreadsM : 1;
+  constexpr int TPT = (G * kCtaTok) / NT > 0 ? (G * kCtaTok) / NT : 1;
   constexpr int TASKS_PER_HEAD = kCtaTok / TPT;
   constexpr int NTASK = G * TASKS_PER_HEAD;
-  static_assert(NTASK <= kThreadsM && (TPT == 1 || TPT == 2), "one weight task per thread");
+  static_assert(NTASK <= NT && (TPT == 1 || TPT == 2), "one weight task per thread");
   constexpr int PDB = NKIND * VNCOL * kPdStride;  // one digit buffer (two: current and next)
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ __align__(8) uint64_t mbar[kStagesM + 1];  // per stage (+ one nothing completes: test entry)
@@ -321,10 +330,13 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   float* red = reinterpret_cast<float*>(pdig + 2 * PDB);                      // reductions
 
   const int split = blockIdx.x, b = blockIdx.z;
-  // blockIdx.y: piece `half` of kv-head hk's query group (p.hsplit pieces of G heads)
-  const int hk = blockIdx.y / p.hsplit, half = blockIdx.y % p.hsplit;
+  // blockIdx.y: piece `half` of kv-head hk's query group (p.hsplit pieces of G heads); a CTA of 8
+  // heads takes the whole group (both prep pieces, one per warp half)
+  const int npc = G > 4 ? 1 : p.hsplit;
+  const int hk = blockIdx.y / npc, half = blockIdx.y % npc;
   const int h_first = hk * p.group + half * G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hb = G > 4 ? 4 * (warp >> 2) : 0;  // first head of this warp's logits
   const int g = lane >> 2, t = lane & 3;
   // In a fused append + decode step the cache (and len) are written by the append kernel that
   // runs before the prep: everything that reads them waits for the prep (which waits for it).
@@ -410,7 +422,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   // complete before prep started (unless cache_after_wait, handled above); the prep output is read
   // only after this wait.
   if (!p.cache_after_wait) grid_dep_wait();
-  const unsigned char* prep = p.qprep + (pair * p.hsplit + half) * p.qprep_stride;
+  const unsigned char* prep = p.qprep + (pair * p.hsplit + (G > 4 ? (warp >> 2) : half)) * p.qprep_stride;
   uint32_t qb[KP][4][KNT][2];
 #pragma unroll
   for (int P = 0; P < KP; ++P)
@@ -418,9 +430,9 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     for (int m = 0; m < 4; ++m)
 #pragma unroll
       for (int nt = 0; nt < KNT; ++nt) {
-        const int n = nt * 8 + g, h = n / 2, d = n % 2;  // column = (head, digit)
-        if (h < G) {
-          const unsigned char* row = prep + ((P * G + h) * 2 + d) * 128;
+        const int n = nt * 8 + g, h = n / 2, d = n % 2;  // column = (head of this warp, digit)
+        if (h < GW) {
+          const unsigned char* row = prep + ((P * GW + h) * 2 + d) * 128;
           qb[P][m][nt][0] = __ldcg(reinterpret_cast<const uint32_t*>(row + ((2 * m) * 4 + t) * 4));
           qb[P][m][nt][1] = __ldcg(reinterpret_cast<const uint32_t*>(row + ((2 * m + 1) * 4 + t) * 4));
         } else {
@@ -428,14 +440,14 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         }
       }
   // this thread's logit columns (2t, 2t+1) of N-tile nt: digits (hi, lo) of head 4 nt + t
-  const float* hconst = reinterpret_cast<const float*>(prep + KP * G * 2 * 128);
+  const float* hconst = reinterpret_cast<const float*>(prep + KP * GW * 2 * 128);
   // Rows g, g + 8 of the key contraction carry operand bytes 2^g (g < 7) or -128 (g = 7); the
   // head scales are in units of the -128 byte, so this thread's rows rescale them by rowf.
   const float rowf = g == 7 ? 1.f : -128.f / (float)(1 << g);
   float hs[KNT], hc[KNT], hsz[KNT], hcz[KNT];
 #pragma unroll
   for (int nt = 0; nt < KNT; ++nt) {
-    const int h = min(4 * nt + t, G - 1);
+    const int h = min(4 * nt + t, GW - 1);
     hs[nt] = __ldcg(hconst + h * 4 + 0) * rowf;
     hc[nt] = __ldcg(hconst + h * 4 + 1);
     hsz[nt] = __ldcg(hconst + h * 4 + 2) * rowf;
@@ -448,7 +460,11 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
 #pragma unroll
   for (int nt = 0; nt < KNT; ++nt) mrow[nt] = -INFINITY;
   float wmax = 0.f, wmaxz = 0.f;  // largest value weight of each kind seen by this thread
-  const int tl = warp * 16;
+  const int tl = (warp & 3) * 16;
+  // chunk maxima per (warp, head): warps write the heads they own, -inf elsewhere
+  float* hmax = red;                 // [NW][G]
+  float* wred = red + NW * G;        // [2][NW]: both kinds' weight maxima
+  for (int i = tid; i < NW * G; i += NT) hmax[i] = -INFINITY;
   for (int it = 0; it < n_iter; ++it) {
     if (tid == 0) issue(it + kStagesM - 1);
     wait_fill(it);
@@ -541,9 +557,9 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
           l1 = fmaf(gk1, fmaf(hsz[nt], (float)(cz[2] * 256 + cz[3]), hcz[nt]), l1);
         }
         const float lg0 = v0 ? nk0 * l0 : -INFINITY, lg1 = v1 ? nk1 * l1 : -INFINITY;
-        if (h < G) {
-          lgs[h * lgst + tok0 + tl + g] = lg0;
-          lgs[h * lgst + tok0 + tl + g + 8] = lg1;
+        if (h < GW) {
+          lgs[(hb + h) * lgst + tok0 + tl + g] = lg0;
+          lgs[(hb + h) * lgst + tok0 + tl + g + 8] = lg1;
         }
         mrow[nt] = fmaxf(mrow[nt], fmaxf(lg0, lg1));
       }
@@ -558,28 +574,26 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     __syncthreads();  // the next iteration refills a stage buffer
   }
   // chunk maxima per head, and the weight scale
-  float* hmax = red;                 // [kWarpsM][G]
-  float* wred = red + kWarpsM * G;   // [2][kWarpsM]: both kinds' weight maxima
 #pragma unroll
   for (int nt = 0; nt < KNT; ++nt) {
     float mx = mrow[nt];
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    if (g == 0 && 4 * nt + t < G) hmax[warp * G + 4 * nt + t] = mx;
+    if (g == 0 && 4 * nt + t < GW) hmax[warp * G + hb + 4 * nt + t] = mx;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
     wmaxz = fmaxf(wmaxz, __shfl_xor_sync(0xffffffffu, wmaxz, o));
   }
-  if (lane == 0) { wred[warp] = wmax; wred[kWarpsM + warp] = wmaxz; }
-  for (int idx = tid; idx < 2 * PDB / 4; idx += kThreadsM)
+  if (lane == 0) { wred[warp] = wmax; wred[NW + warp] = wmaxz; }
+  for (int idx = tid; idx < 2 * PDB / 4; idx += NT)
     reinterpret_cast<uint32_t*>(pdig)[idx] = 0u;  // the pad digit and absent heads stay zero
   __syncthreads();
   float wm = 0.f, wmz = 0.f;
 #pragma unroll
-  for (int w = 0; w < kWarpsM; ++w) { wm = fmaxf(wm, wred[w]); wmz = fmaxf(wmz, wred[kWarpsM + w]); }
+  for (int w = 0; w < NW; ++w) { wm = fmaxf(wm, wred[w]); wmz = fmaxf(wmz, wred[NW + w]); }
   // integer weights below 2^23 (3 byte digits), each kind scaled to its own range by a power
   // of two (exact digits; the sketch weights are ~sqrt(pi/2) gamma / m of the centroid ones)
   const float wsc = wm > 0.f ? exp2f(floorf(log2f(kWRange / wm)) - 1.f) : 1.f;
@@ -590,7 +604,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   const int task_h = min(tid / TASKS_PER_HEAD, G - 1), task_T = TPT * (tid % TASKS_PER_HEAD);
   float task_m = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < kWarpsM; ++w) task_m = fmaxf(task_m, hmax[w * G + task_h]);
+  for (int w = 0; w < NW; ++w) task_m = fmaxf(task_m, hmax[w * G + task_h]);
   float task_l = 0.f;                 // sum of p over this task's tokens
   uint32_t task_wc = 0, task_wz = 0;  // sums of the quantised weights (exact: <= 64 tokens x 2^23)
 
@@ -652,16 +666,16 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     }
   };
 
-  int vacc[VP][2][VNT][4];
+  int vacc[VP][PPW][VNT][4];
 #pragma unroll
   for (int P = 0; P < VP; ++P)
 #pragma unroll
-    for (int pi = 0; pi < 2; ++pi)
+    for (int pi = 0; pi < PPW; ++pi)
 #pragma unroll
       for (int nt = 0; nt < VNT; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) vacc[P][pi][nt][c] = 0;
-  const uint32_t vm0 = 0x01010101u << (2 * warp), vm1 = 0x01010101u << (2 * warp + 1);
+  const uint32_t vm0 = 0x01010101u << (PPW * warp), vm1 = 0x01010101u << (PPW * warp + PPW - 1);
 
   // Digits of iteration 0, then per iteration: the digits of the next one (all threads) and the
   // contractions of this one; one barrier per iteration separates the two digit buffers.
@@ -728,7 +742,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         for (int nt = 0; nt < VNT; ++nt) {
           const uint32_t b0 = sk ? bz[nt][0] : bm[nt][0], b1 = sk ? bz[nt][1] : bm[nt][1];
           mma_s8u8(vacc[P][0][nt], a00, a01, a02, a03, b0, b1);
-          mma_s8u8(vacc[P][1][nt], a10, a11, a12, a13, b0, b1);
+          if (PPW > 1) mma_s8u8(vacc[P][PPW - 1][nt], a10, a11, a12, a13, b0, b1);
         }
       }
     }
@@ -743,8 +757,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     for (int f = max(0, n_fill - kStagesM); f < n_fill; ++f)
       mbar_wait(smem_addr(&mbar[(unsigned)f % kStagesM]), ((unsigned)f / kStagesM) & 1u, p.wait_limit);
   __syncthreads();
-  float* tsum = reinterpret_cast<float*>(stages);  // [kThreadsM][3] (staging reused)
-  float* hsum = tsum + 3 * kThreadsM;               // [3][G]: sum p, sum weights, sum sketch weights
+  float* tsum = reinterpret_cast<float*>(stages);  // [NT][3] (staging reused)
+  float* hsum = tsum + 3 * NT;                      // [3][G]: sum p, sum weights, sum sketch weights
   tsum[3 * tid] = task_l;
   tsum[3 * tid + 1] = (float)task_wc;
   tsum[3 * tid + 2] = (float)task_wz;
@@ -763,8 +777,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   for (int P = 0; P < VWP; ++P) vasum += va[P];
   const float inv_w = 1.f / wsc, inv_wz = 1.f / wscz;
 #pragma unroll
-  for (int pi = 0; pi < 2; ++pi) {
-    const int pos = 2 * warp + pi;
+  for (int pi = 0; pi < PPW; ++pi) {
+    const int pos = PPW * warp + pi;
     const float rowpos = pos == 7 ? -1.f / 128.f : 1.f / (float)(1 << pos);  // row value 2^p or -128
     const float rowinv = rowpos * inv_w, rowinvz = rowpos * inv_wz;
 #pragma unroll
@@ -804,7 +818,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       float* dst = p.part + (((size_t)b * p.Hq + h_first + h) * p.splits + split) * p.part_stride;
       float mx = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kWarpsM; ++w) mx = fmaxf(mx, hmax[w * G + h]);
+      for (int w = 0; w < NW; ++w) mx = fmaxf(mx, hmax[w * G + h]);
       dst[0] = mx;
       dst[1] = hsum[h];
     }
@@ -848,7 +862,7 @@ template <int G, int KB, bool KQ, int VB, bool VQ>
 cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
   if (!TileLayout<KB, KQ>::matches(p.k) || !TileLayout<VB, VQ>::matches(p.v)) return cudaErrorNotSupported;
   if (p.k.order != kOrderOctet || p.v.order != kOrderByteLane) return cudaErrorNotSupported;
-  cudaError_t e = launch_prep<G, KB, KQ>(p, s, qp);
+  cudaError_t e = launch_prep<(G > 4 ? 4 : G), KB, KQ>(p, s, qp);  // query prep in pieces of <= 4 heads
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
   const size_t smem = mma_smem_bytes(G, p.k, p.v, p.chunk);
@@ -856,8 +870,8 @@ cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.splits, p.Hkv * p.hsplit, p.B);
-  cfg.blockDim = dim3(kThreadsM);
+  cfg.gridDim = dim3(p.splits, p.Hkv * (G > 4 ? 1 : p.hsplit), p.B);
+  cfg.blockDim = dim3(MmaCfg<G, KB, KQ, VB, VQ>::NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -927,8 +941,9 @@ bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl
 }
 
 int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk) {
-  const size_t per = mma_smem_bytes(std::min(group, 4), k, v, chunk) + kSmemReserved;
-  return std::max(1, std::min(kMinBlocksM, (int)(kSmemPerSm / per)));
+  const size_t per = mma_smem_bytes(group, k, v, chunk) + kSmemReserved;
+  const int by_regs = group > 4 ? kMinBlocksM / 2 : kMinBlocksM;  // 8-warp CTAs: half as many
+  return std::max(1, std::min(by_regs, (int)(kSmemPerSm / per)));
 }
 
 bool mma_decode_supported(const DecodeParams& p) {
@@ -942,7 +957,7 @@ cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEven
     case 1: return dispatch_mma_modes<1>(p, s, ev_mid, qp);
     case 2: return dispatch_mma_modes<2>(p, s, ev_mid, qp);
     case 4: return dispatch_mma_modes<4>(p, s, ev_mid, qp);
-    case 8: return dispatch_mma_modes<4>(p, s, ev_mid, qp);  // two pieces of 4 heads
+    case 8: return dispatch_mma_modes<8>(p, s, ev_mid, qp);  // one CTA of 8 warps per kv-head
     default: return cudaErrorNotSupported;
   }
 }
