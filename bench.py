@@ -401,6 +401,7 @@ def measure(kvq, w, args, world, dev):
     out = torch.empty((w.batch, w.n_q_heads, caches[0].out_dim), dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
     lens0 = int(caches[0].lengths()[0])
+    caches_info = caches[0].layout()
 
     def step(i):
         # one decode step through the fused entry: append the new token of every sequence and
@@ -500,6 +501,18 @@ def measure(kvq, w, args, world, dev):
                 "peak": float(peaks["hbm_gbs"]), "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     tr = traffic_record(w)
+    # load efficiency of the packed streams: the split kernels stage whole tile pairs with 1-D bulk
+    # copies (TMA), so every copy moves full 16-byte-aligned, contiguous runs; its size follows from
+    # the layout (FP4: the latent kernel loads 16-byte vectors into registers instead)
+    info = caches_info
+    if w.k_mode == "fp4":
+        load_eff = {"path": "16-byte vector loads of whole tile rows", "bytes_per_request": 16}
+    else:
+        ktb, vtb = int(info[1]), int(info[2])
+        nb = 128 if (w.v_mode == "lm_qjl") else 64
+        load_eff = {"path": "1-D bulk copies (TMA) of whole tile pairs",
+                    "bytes_per_copy": {"k_pair": 2 * ktb, "v_norms": nb, "v_pair": 2 * vtb},
+                    "mean_bytes_per_copy": (2 * ktb + 2 * nb + 2 * vtb) / 4.0}
     line = {
         "value": value, "ms_per_step": ms_per_step,
         # the contractions' operand / accumulation types: exact int8 tensor-core products with int32
@@ -511,7 +524,8 @@ def measure(kvq, w, args, world, dev):
         "roofline": dict(roof, traffic=None if tr is None else tr["dram_bytes"], peak_kind=peak_kind,
                          kernel=KERNEL_NAMES[w.name],
                          bytes_per_launch=bytes_kernel, ms_per_launch=kern_ms[1],
-                         load_efficiency=None if tr is None else tr["load_efficiency"]),
+                         load_efficiency=dict(load_eff, dram_over_algorithmic=None if tr is None else
+                                              tr["dram_bytes"] / bytes_kernel)),
         "decode_call": {"ms": call_ms, "bytes": bytes_step, "gbs": achieved_call,
                         "kernels_ms": {"prep": kern_ms[0], "split": kern_ms[1], "reduce": kern_ms[2]}},
         "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,
