@@ -345,8 +345,20 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   const unsigned char* kreg = reinterpret_cast<const unsigned char*>(p.kreg);
   const unsigned char* vreg = reinterpret_cast<const unsigned char*>(p.vreg);
   // index of a tile pair's first tile (contiguous, or the block table's page)
-  auto pair_index = [&](int tile0) {
-    return tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk, tile0, p.err);
+  // paged caches: the block-table entries of this CTA's chunk, read once into shared memory (the
+  // fill issue path then does no global load); chunks are at most kChunkMax tokens
+  __shared__ int s_pages[kChunkMax / kCtaTok + 1];
+  if (p.table)
+    for (int i = threadIdx.x; i <= p.chunk / kCtaTok && (t_begin / kCtaTok + i) < p.pages_per_seq; i += blockDim.x)
+      s_pages[i] = __ldcg(p.table + (size_t)b * p.pages_per_seq + t_begin / kCtaTok + i);
+  auto pair_index = [&](int tile0) -> long {
+    if (!p.table) return ((long)b * p.Hkv + hk) * p.tiles_per_seq + tile0;
+    const int page = s_pages[tile0 / 2 - t_begin / kCtaTok];
+    if (page < 0 || page >= p.n_pages) {
+      atomicOr(p.err, kStatusBadPage);
+      return (long)hk * 2;
+    }
+    return ((long)page * p.Hkv + hk) * 2;
   };
   // In a fused append + decode step the predecessor appends the token at the old length and sets
   // the new one, so a length read before waiting for it is either value. When the first

@@ -84,18 +84,26 @@ __global__ void __launch_bounds__(kWinThreads) window_decode(const __grid_consta
   __syncthreads();
   // logits: token i by warp i % 8 (lane l: coordinates 4l .. 4l + 3), all heads, warp sums
   const int nw = kWinThreads / 32;
-  for (int i = warp; i < n_tok; i += nw) {
-    const uint2 k4 = *reinterpret_cast<const uint2*>(kw + (size_t)slot_of(i) * kHeadDim + 4 * lane);
-    const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k4.x));
-    const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k4.y));
+  constexpr int kBatch = 4;  // tokens per warp step: their key loads are in flight together
+  for (int i0 = warp * kBatch; i0 < n_tok; i0 += nw * kBatch) {
+    uint2 k4[kBatch];
 #pragma unroll
-    for (int h = 0; h < kWinMaxG; ++h) {
-      if (h >= G) break;
-      const float4 q4 = *reinterpret_cast<const float4*>(&qs[h][4 * lane]);
-      float v = fmaf(k23.y, q4.w, fmaf(k23.x, q4.z, fmaf(k01.y, q4.y, k01.x * q4.x)));
+    for (int u = 0; u < kBatch; ++u)
+      k4[u] = i0 + u < n_tok ? *reinterpret_cast<const uint2*>(kw + (size_t)slot_of(i0 + u) * kHeadDim + 4 * lane)
+                             : make_uint2(0u, 0u);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) lg[h][i] = v;
+    for (int u = 0; u < kBatch; ++u) {
+      const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k4[u].x));
+      const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&k4[u].y));
+#pragma unroll
+      for (int h = 0; h < kWinMaxG; ++h) {
+        if (h >= G) break;
+        const float4 q4 = *reinterpret_cast<const float4*>(&qs[h][4 * lane]);
+        float v = fmaf(k23.y, q4.w, fmaf(k23.x, q4.z, fmaf(k01.y, q4.y, k01.x * q4.x)));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && i0 + u < n_tok) lg[h][i0 + u] = v;
+      }
     }
   }
   __syncthreads();
@@ -124,11 +132,22 @@ __global__ void __launch_bounds__(kWinThreads) window_decode(const __grid_consta
 #pragma unroll
     for (int h = 0; h < kWinMaxG; ++h) acc[h] = 0.f;
     const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(vw);
-    for (int i = half; i < n_tok; i += 2) {
-      const float v = __bfloat162float(vb[(size_t)slot_of(i) * kHeadDim + j]);
+    constexpr int kVBatch = 8;  // value loads in flight together
+    for (int i0 = half; i0 < n_tok; i0 += 2 * kVBatch) {
+      float v[kVBatch];
 #pragma unroll
-      for (int h = 0; h < kWinMaxG; ++h)
-        if (h < G) acc[h] = fmaf(lg[h][i], v, acc[h]);
+      for (int u = 0; u < kVBatch; ++u) {
+        const int i = i0 + 2 * u;
+        v[u] = i < n_tok ? __bfloat162float(vb[(size_t)slot_of(i) * kHeadDim + j]) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kVBatch; ++u) {
+        const int i = i0 + 2 * u;
+        if (i < n_tok)
+#pragma unroll
+          for (int h = 0; h < kWinMaxG; ++h)
+            if (h < G) acc[h] = fmaf(lg[h][i], v[u], acc[h]);
+      }
     }
     if (half == 1)
 #pragma unroll
