@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="llama70b", choices=list(WORKLOADS),
+    ap.add_argument("--workload", default="llama70b", choices=list(WORKLOADS) + list(VARIANTS),
                     help="headline workload (default: the largest single-GPU configuration, 1.98 GB per step)")
     ap.add_argument("--only", action="store_true", help="time the headline workload alone")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -109,7 +109,7 @@ def kernel_sources_sha():
 
 def traffic_record(w):
     rec = TRAFFIC.get(w.name)
-    if rec is None or rec["sources_sha256"] != kernel_sources_sha() or w.ctx != WORKLOADS[w.name].ctx:
+    if rec is None or rec["sources_sha256"] != kernel_sources_sha() or w.ctx != workload(w.name).ctx:
         return None
     return rec
 
@@ -300,7 +300,7 @@ def blas_threads():
 
 
 def run_reference(args, world, rank):
-    w = WORKLOADS[args.workload]
+    w = workload(args.workload)
     if args.ctx > 0:
         w = w.with_(ctx=args.ctx)
     metric, unit = METRIC, UNIT
@@ -552,7 +552,7 @@ def run_ours(args, world, rank, local):
     kvq.load()
     dev = f"cuda:{local}"
     torch.cuda.set_device(dev)
-    w = WORKLOADS[args.workload]
+    w = workload(args.workload)
     if args.ctx > 0:
         w = w.with_(ctx=args.ctx)
     head = measure(kvq, w, args, world, dev)
