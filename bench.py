@@ -69,9 +69,10 @@ def parse():
 # The dominant (split decode) kernel of each workload.
 KERNEL_NAMES = {
     "tiny": "decode_lm_mma<1, 2, 1, 2, 1>", "llama8b": "decode_lm_mma<4, 2, 1, 2, 1>",
-    "llama70b": "decode_lm_mma<4, 3, 1, 3, 0>", "onebit": "decode_lm_mma<4, 1, 0, 1, 0>",
+    "llama70b": "decode_lm_mma<8, 3, 1, 3, 0>", "onebit": "decode_lm_mma<4, 1, 0, 1, 0>",
     "mla_fp4": "decode_mla_umma",
-    "llama8b_kivi": "decode_lm_tc<4, 2, 0, 2, 0, kivi>", "llama8b_window": "decode_lm_mma<4, 2, 1, 2, 1> + window_decode",
+    "llama8b_kivi": "decode_lm_mma<4, 2, 0, 2, 0, kivi> (key-group splits + window parts)",
+    "llama8b_window": "decode_lm_mma<4, 2, 1, 2, 1> (history splits + window parts)",
     "llama8b_paged": "decode_lm_mma<4, 2, 1, 2, 1> (paged)",
 }
 EXTRA_WORKLOADS = ("llama8b", "onebit", "mla_fp4", "llama70b", "llama8b_kivi", "llama8b_window", "llama8b_paged")
@@ -88,6 +89,15 @@ def coded_len(w, L):
     if w.sink_tokens or w.recent_tokens:
         return max(0, L - w.sink_tokens - w.recent_tokens)
     return L
+
+
+def window_len(w, L):
+    """bf16 window tokens of a sequence of length L (sink + recent; KIVI: the incomplete group)."""
+    if w.k_mode == "kivi":
+        return L % 128
+    if w.sink_tokens or w.recent_tokens:
+        return min(L, w.sink_tokens) + (min(w.recent_tokens, L - w.sink_tokens) if L > w.sink_tokens else 0)
+    return 0
 
 # DRAM bytes (read + write) of one launch of the split decode kernel, and the load efficiency of its
 # packed streams, from ncu captures (full size, or a smaller context scaled to the full launch by the
@@ -484,10 +494,14 @@ def measure(kvq, w, args, world, dev):
     d2h = host_outs[0].numel() * host_outs[0].element_size()
 
     peaks, peak_kind = measured_peaks()
-    bytes_step = w.batch * heads_kv * coded_len(w, lens0 + 1) * per_tok  # packed bytes one decode call reads
+    # bytes one decode call reads: packed history + bf16 K and V of the window
+    bytes_step = w.batch * heads_kv * (coded_len(w, lens0 + 1) * per_tok + window_len(w, lens0 + 1) * 4 * w.head_dim)
     call_ms = sum(kern_ms)  # kvq_decode_attention alone, from the per-kernel events
     achieved_call = bytes_step / (call_ms / 1e3) / 1e9
     bytes_kernel = w.batch * heads_kv * lens_k * per_tok      # the split kernel's algorithmic bytes
+    if w.k_mode == "kivi" or w.sink_tokens or w.recent_tokens:  # its extra CTAs read the bf16 window
+        win_k = sum(window_len(w, int(caches[j % replicas].lengths()[0])) for j in range(n_k)) / n_k
+        bytes_kernel += w.batch * heads_kv * win_k * 4 * w.head_dim
     if w.k_mode == "fp4":
         # 64 heads x (latent + rope) MACs for the logits and 64 x latent for the values, per token:
         # a dense contraction (146 GFLOP at 2^20 tokens), so the tensor roofline bounds it. The

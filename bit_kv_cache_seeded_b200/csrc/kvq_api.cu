@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "kvq_internal.h"
+#include "kvq_window.cuh"
 #include "kvq_plan.h"
 
 using namespace kvq;
@@ -231,9 +232,11 @@ size_t partials_bytes(const kvq_cache* c, int splits) {
 // Workspace = split partials, then the per-(sequence, kv-head) query tables of the tensor-core path.
 bool has_window(const kvq_cache* c) { return c->sink > 0 || c->recent > 0 || c->kivi; }
 
-// Bytes of the window's softmax states [B][Hq][part_stride] (window caches), 256-aligned.
+// Bytes of the window's softmax states [B][Hq][parts][part_stride] (window caches), 256-aligned.
 size_t window_state_bytes(const kvq_cache* c) {
-  return has_window(c) ? align_up(sizeof(float) * (size_t)c->batch * c->cfg.n_q_heads * part_stride(c), 256) : 0;
+  if (!has_window(c)) return 0;
+  const size_t parts = window_parts(c->sink + c->recent);
+  return align_up(sizeof(float) * (size_t)c->batch * c->cfg.n_q_heads * parts * part_stride(c), 256);
 }
 
 // Workspace = split partials, the per-(sequence, kv-head) query tables of the tensor-core paths,
@@ -252,10 +255,10 @@ const std::vector<int>& coded_lens(const kvq_cache* c) { return has_window(c) ? 
 // tensor-core kernel's shared-memory and register limit for query groups of 1, 2 or 4, else 4.
 int decode_slots_per_sm(const kvq_cache* c, int units) {
   if (c->is_fp4 || c->tc || c->kivi_tc) return 1;
-  if (c->kivi) return 8;
+  if (c->kivi_cuda) return 8;
   const int group = c->cfg.n_q_heads / c->cfg.n_kv_heads;
   if (group == 1 || group == 2 || group == 4 || group == 8)
-    return lm_mma_slots_per_sm(group, c->k, c->v, units * kTile * kTilePair);
+    return lm_mma_slots_per_sm(group, c->k, c->v, units * kTile * kTilePair, c->kivi);
   return 4;
 }
 
@@ -263,6 +266,7 @@ int decode_slots_per_sm(const kvq_cache* c, int units) {
 int decode_max_units(const kvq_cache* c) {
   if (c->is_fp4) return 1 << 30;
   if (c->tc || c->kivi_tc) return tc_chunk_max(c->cfg.n_q_heads / c->cfg.n_kv_heads) / (kTile * kTilePair);
+  if (c->kivi) return kChunkMax / (kTile * kTilePair) / 2 * 2;  // rounded up to whole key groups below
   return kChunkMax / (kTile * kTilePair);
 }
 
@@ -416,7 +420,10 @@ kvq_status cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_
   c->tc = !P.fp4_mode && !P.kivi && choose_tc(*cfg, P.k, P.v);
   {
     const char* e = std::getenv("KVQ_DECODE_KERNEL");
-    c->kivi_tc = P.kivi && !(e && (std::strcmp(e, "mma") == 0 || std::strcmp(e, "cuda") == 0));
+    // KIVI decode: the mma.sync kernel, or (KVQ_DECODE_KERNEL at cache creation) "tc" the tcgen05
+    // kernel, "cuda" the CUDA-core kernel
+    c->kivi_tc = P.kivi && e && std::strcmp(e, "tc") == 0;
+    c->kivi_cuda = P.kivi && e && std::strcmp(e, "cuda") == 0;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   c->table = table;
@@ -739,18 +746,23 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
     p.tot_lens = c->d_lens;
     p.wpart = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + partials_bytes(c, splits) +
                                        prep_bytes_total(c));
+    p.win_parts = window_parts(p.win_slots);
     p.win_kivi = c->kivi ? 1 : 0;
     p.kstats = c->d_kstats;
     p.groups_per_seq = c->groups_per_seq;
   }
   if (c->kivi) {  // KIVI: the split kernel over the coded groups, the window, the reduce (no rotation)
-    if (c->kivi_tc && p.chunk % (2 * kTile * kTilePair)) {  // whole 128-token key groups per CTA
+    if (!c->kivi_cuda && p.chunk % (2 * kTile * kTilePair)) {  // whole 128-token key groups per CTA
       p.chunk += kTile * kTilePair;
       p.splits = std::max(1, (max_len + p.chunk - 1) / p.chunk);
     }
-    if (!rec(1) || (c->kivi_tc ? launch_decode_kivi_tc(p, s) : launch_decode_kivi(p, s)) != cudaSuccess || !rec(2))
-      return KVQ_ERR_CUDA;
-    if (launch_window_decode(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+    p.win_fused = !c->kivi_tc && !c->kivi_cuda;  // the mma.sync kernel's extra CTAs take the window
+    if (!rec(1)) return KVQ_ERR_CUDA;
+    const cudaError_t e = c->kivi_tc ? launch_decode_kivi_tc(p, s)
+                          : c->kivi_cuda ? launch_decode_kivi(p, s)
+                                         : launch_decode_kivi_mma(p, s);
+    if (e != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
+    if (!p.win_fused && launch_window_decode(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
     if (launch_reduce_lm(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
     return KVQ_OK;
   }
@@ -761,8 +773,9 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   }
   p.cache_after_wait = qp != nullptr;
   if (debug_unset_wait && !tensor_path) return KVQ_ERR_UNSUPPORTED;
+  p.win_fused = p.wpart && tensor_path && !p.use_tc;  // the mma.sync split kernel takes the window parts
   if (launch_decode_lm(p, s, ev ? ev[1] : nullptr, qp) != cudaSuccess || !rec(2)) return KVQ_ERR_CUDA;
-  if (p.wpart && launch_window_decode(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
+  if (p.wpart && !p.win_fused && launch_window_decode(p, s) != cudaSuccess) return KVQ_ERR_CUDA;
   if (launch_reduce_lm(p, s) != cudaSuccess || !rec(3)) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }

@@ -280,42 +280,38 @@ reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
   // Launched as a programmatic dependent of the decode kernel: S is staged above while that
   // grid finishes; its partials are read only after this wait.
   grid_dep_wait();
-  const float* part = p.part + ((size_t)b * p.Hq + hk * G + h) * (size_t)p.splits * p.part_stride;
   float M = -INFINITY, L = 0.f, o = 0.f, oz = 0.f;
-  for (int s0 = 0; s0 < p.splits; s0 += kSplitBatch) {
-    float mv[kSplitBatch], lv[kSplitBatch], ov[kSplitBatch], zv[kSplitBatch];
+  // fold n consecutive states [n][part_stride] into (M, L, o, oz), kSplitBatch loads in flight
+  auto merge = [&](const float* part, int n) {
+    for (int s0 = 0; s0 < n; s0 += kSplitBatch) {
+      float mv[kSplitBatch], lv[kSplitBatch], ov[kSplitBatch], zv[kSplitBatch];
 #pragma unroll
-    for (int k = 0; k < kSplitBatch; ++k) {
-      const bool in = s0 + k < p.splits;
-      const float* ps = part + (size_t)(in ? s0 + k : 0) * p.part_stride;
-      mv[k] = in ? __ldcg(ps) : -INFINITY;
-      lv[k] = in ? __ldcg(ps + 1) : 0.f;
-      ov[k] = in ? __ldcg(ps + 2 + i) : 0.f;
-      zv[k] = (in && vq) ? __ldcg(ps + 2 + kHeadDim + i) : 0.f;
+      for (int k = 0; k < kSplitBatch; ++k) {
+        const bool in = s0 + k < n;
+        const float* ps = part + (size_t)(in ? s0 + k : 0) * p.part_stride;
+        mv[k] = in ? __ldcg(ps) : -INFINITY;
+        lv[k] = in ? __ldcg(ps + 1) : 0.f;
+        ov[k] = in ? __ldcg(ps + 2 + i) : 0.f;
+        zv[k] = (in && vq) ? __ldcg(ps + 2 + kHeadDim + i) : 0.f;
+      }
+      float mn = M;
+#pragma unroll
+      for (int k = 0; k < kSplitBatch; ++k) mn = fmaxf(mn, mv[k]);
+      const float c = exp2_diff(M, mn);
+      L *= c; o *= c; oz *= c;
+#pragma unroll
+      for (int k = 0; k < kSplitBatch; ++k) {
+        const float w = exp2_diff(mv[k], mn);
+        L = fmaf(w, lv[k], L);
+        o = fmaf(w, ov[k], o);
+        oz = fmaf(w, zv[k], oz);
+      }
+      M = mn;
     }
-    float mn = M;
-#pragma unroll
-    for (int k = 0; k < kSplitBatch; ++k) mn = fmaxf(mn, mv[k]);
-    const float c = exp2_diff(M, mn);
-    L *= c; o *= c; oz *= c;
-#pragma unroll
-    for (int k = 0; k < kSplitBatch; ++k) {
-      const float w = exp2_diff(mv[k], mn);
-      L = fmaf(w, lv[k], L);
-      o = fmaf(w, ov[k], o);
-      oz = fmaf(w, zv[k], oz);
-    }
-    M = mn;
-  }
-  if (p.wpart) {  // the mixed-precision window's state, one more part of the same softmax
-    const float* ws = p.wpart + ((size_t)b * p.Hq + hk * G + h) * p.part_stride;
-    const float wm = __ldcg(ws), mn = fmaxf(M, wm);
-    const float c = exp2_diff(M, mn), w = exp2_diff(wm, mn);
-    L = fmaf(w, __ldcg(ws + 1), L * c);
-    o = fmaf(w, __ldcg(ws + 2 + i), o * c);
-    oz = fmaf(w, vq ? __ldcg(ws + 2 + kHeadDim + i) : 0.f, oz * c);
-    M = mn;
-  }
+  };
+  merge(p.part + ((size_t)b * p.Hq + hk * G + h) * (size_t)p.splits * p.part_stride, p.splits);
+  // the mixed-precision window's parts: more terms of the same softmax
+  if (p.wpart) merge(p.wpart + ((size_t)b * p.Hq + hk * G + h) * (size_t)p.win_parts * p.part_stride, p.win_parts);
   // the normalisation by L, unless the call asks for the merged softmax state (m, l, unnormalised
   // o), whose Sᵀ fold and inverse rotation are linear and apply the same way
   const float inv = p.pout ? 1.f : (L > 0.f) ? 1.f / L : 0.f;

@@ -34,6 +34,7 @@
 // cache's status word. Partials (m, l, o_r, acc_z) are written in the format of the CUDA-core
 // kernel; the same reduce kernel finishes.
 #include <algorithm>
+#include <type_traits>
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -43,6 +44,7 @@
 #include "kvq_quantize_lm.cuh"
 #include "kvq_lm_common.cuh"
 #include "kvq_tiles.cuh"
+#include "kvq_window.cuh"
 
 namespace kvq {
 namespace {
@@ -103,21 +105,23 @@ struct MmaCfg {
   static constexpr int KP = Walsh<KB>::P + (KQ ? 1 : 0);  // logit planes (sketch last)
   static constexpr int VP = Walsh<VB>::P + (VQ ? 1 : 0);  // value planes (sketch last)
   static constexpr int KNT = (2 * GW + 7) / 8;            // logit N-tiles: (head, 2 digits)
-  static constexpr int VNT = (4 * G + 7) / 8;             // value N-tiles: (head, 3 digits + pad)
+  static constexpr int VNT = (3 * G + 7) / 8;             // value N-tiles: (head, 3 digits), column 3h + d
   static constexpr int VNCOL = VNT * 8;
   static constexpr int PPW = 8 / NW;                      // value bit positions per warp
 };
 
 // Dynamic shared memory of one decode CTA: the staging ring, the chunk's logits, the two weight
 // digit buffers and the reduction scratch.
-size_t mma_smem_bytes(int group, const SideLayout& k, const SideLayout& v, int chunk) {
+size_t mma_smem_bytes(int group, const SideLayout& k, const SideLayout& v, int chunk, bool kivi) {
   const int nkind = v.qjl ? 2 : 1;
-  const int vncol = ((4 * group + 7) / 8) * 8;
+  const int vncol = ((3 * group + 7) / 8) * 8;
   const int nw = group > 4 ? 8 : 4;
-  size_t s = (size_t)kStagesM * std::max(2 * k.tile_bytes + kNormBlock, 2 * v.tile_bytes);
+  size_t s = (size_t)kStagesM * std::max(2 * k.tile_bytes + kNormBlock + (kivi ? kKiviStats : 0), 2 * v.tile_bytes);
   s += sizeof(float) * (size_t)group * (chunk + 8);
   s += 2 * (size_t)nkind * vncol * kPdStride;
   s += sizeof(float) * (nw * group + 2 * nw);
+  if (kivi)  // query, the group's two-plane digit table, head constants
+    s += sizeof(float) * (size_t)group * kHeadDim + 2 * (size_t)group * 2 * kHeadDim + sizeof(float) * 2 * group;
   return (s + 15) / 16 * 16;
 }
 
@@ -301,7 +305,7 @@ decode_front(const __grid_constant__ QuantizeParams qp, const __grid_constant__ 
 // ------------------------------------------------------------------------------------------
 // Decode kernel (two passes over the CTA's chunk).
 // ------------------------------------------------------------------------------------------
-template <int G, int KB, bool KQ, int VB, bool VQ>
+template <int G, int KB, bool KQ, int VB, bool VQ, bool KV>
 __global__ void __launch_bounds__(Warps<G>::N * 32, 16 / Warps<G>::N)
 decode_lm_mma(const __grid_constant__ DecodeParams p) {
   using C = MmaCfg<G, KB, KQ, VB, VQ>;
@@ -319,22 +323,43 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   __shared__ __align__(8) uint64_t mbar[kStagesM + 1];  // per stage (+ one nothing completes: test entry)
   __shared__ int s_fail;                             // a wait of this CTA gave up
   using KL = TileLayout<KB, KQ>;
-  using VL = TileLayout<VB, VQ>;
+  using VL = std::conditional_t<KV, KiviVTile, TileLayout<VB, VQ>>;
   constexpr int ktb = KL::BYTES, vtb = VL::BYTES;
-  constexpr int stage_bytes = (2 * ktb + kNormBlock > 2 * vtb) ? 2 * ktb + kNormBlock : 2 * vtb;
+  // K stage: the key tile pair, the value norms of its tokens (KIVI: scales), and for KIVI the
+  // statistics of the key group the pair starts (when it starts one)
+  constexpr int kstage = 2 * ktb + kNormBlock + (KV ? kKiviStats : 0);
+  constexpr int stage_bytes = (kstage > 2 * vtb) ? kstage : 2 * vtb;
   // logits row stride (floats): chunk + 8 with the chunk a multiple of 64, so rows start on distinct banks
   const int lgst = p.chunk + 8;
   unsigned char* stages = smem;                                            // [kStagesM][2 tiles (+ norms)]
   float* lgs = reinterpret_cast<float*>(stages + kStagesM * stage_bytes);  // [G][lgst] logits
   unsigned char* pdig = reinterpret_cast<unsigned char*>(lgs + G * lgst);  // [2][NKIND][VNCOL][kPdStride]
   float* red = reinterpret_cast<float*>(pdig + 2 * PDB);                      // reductions
+  // KIVI: the query in log2 logit units [G][d]; the current key group's query digits [KP][G][2][d]
+  // (bytes; words permuted for load_qb), per head (scale, offset) [G][2]
+  float* kq = red + (NW * G + 2 * NW);
+  unsigned char* ktab = reinterpret_cast<unsigned char*>(kq + G * kHeadDim);
+  float* kcon = reinterpret_cast<float*>(ktab + KP * G * 2 * kHeadDim);
 
-  const int split = blockIdx.x, b = blockIdx.z;
-  // blockIdx.y: piece `half` of kv-head hk's query group (p.hsplit pieces of G heads); a CTA of 8
-  // heads takes the whole group (both prep pieces, one per warp half)
+  // One-dimensional grid: the split CTAs (split fastest, then row y, then sequence), then the
+  // window parts' CTAs in the same order (mixed-precision caches), which the block scheduler
+  // places last: they fill the slots the split CTAs leave free.
+  // Row y: piece `half` of kv-head hk's query group (p.hsplit pieces of G heads); a CTA of 8 heads
+  // takes the whole group (both prep pieces, one per warp half).
   const int npc = G > 4 ? 1 : p.hsplit;
-  const int hk = blockIdx.y / npc, half = blockIdx.y % npc;
+  const int n_rows = p.Hkv * npc;
+  const int n_split_ctas = p.splits * n_rows * p.B;
+  const bool win_cta = (int)blockIdx.x >= n_split_ctas;
+  const int bx = win_cta ? (int)blockIdx.x - n_split_ctas : (int)blockIdx.x;
+  const int nx = win_cta ? p.win_parts : p.splits;
+  const int split = bx % nx, row = (bx / nx) % n_rows, b = bx / (nx * n_rows);
+  const int hk = row / npc, half = row % npc;
   const int h_first = hk * p.group + half * G;
+  if (win_cta) {  // a window part: no staging, no barrier below
+    grid_dep_wait();
+    window_part<NW, G>(p, b, hk, half * G, split, reinterpret_cast<float*>(smem));
+    return;
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int hb = G > 4 ? 4 * (warp >> 2) : 0;  // first head of this warp's logits
   const int g = lane >> 2, t = lane & 3;
@@ -395,11 +420,16 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     if (f < n_iter) {
       const long ti = pair_index((unsigned)(t_begin + f * kCtaTok) / kTile);
       constexpr uint32_t nb = VQ ? 128u : 64u;  // value norms (+ gammas, contiguous) per tile
-      mbar_arrive_expect_tx(bar, 2u * ktb + 2u * nb);
+      const int t0 = t_begin + f * kCtaTok;
+      const bool stats = KV && t0 % kKiviGroup == 0;  // KIVI: the pair starts a key group
+      mbar_arrive_expect_tx(bar, 2u * ktb + 2u * nb + (stats ? (uint32_t)kKiviStats : 0u));
       bulk_g2s(smem_addr(dst), kreg + (size_t)ti * ktb, 2u * ktb, bar);
 #pragma unroll
       for (int tile = 0; tile < 2; ++tile)
         bulk_g2s(smem_addr(dst + 2 * ktb + tile * 128), vreg + (size_t)(ti + tile) * vtb + VL::NORM, nb, bar);
+      if (stats)
+        bulk_g2s(smem_addr(dst + 2 * ktb + kNormBlock),
+                 p.kstats + (pair * p.groups_per_seq + t0 / kKiviGroup) * (size_t)kKiviStats, kKiviStats, bar);
     } else {
       const long ti = pair_index((unsigned)(t_begin + (f - n_iter) * kCtaTok) / kTile);
       mbar_arrive_expect_tx(bar, 2u * vtb);
@@ -434,36 +464,55 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   // complete before prep started (unless cache_after_wait, handled above); the prep output is read
   // only after this wait.
   if (!p.cache_after_wait) grid_dep_wait();
-  const unsigned char* prep = p.qprep + (pair * p.hsplit + (G > 4 ? (warp >> 2) : half)) * p.qprep_stride;
+  // Query digit table rows: [KP][heads th][2 digits][128 coordinates] bytes from head h_off on (the
+  // prep area in global memory, or the KIVI group's table in shared memory)
   uint32_t qb[KP][4][KNT][2];
+  auto load_qb = [&](const unsigned char* tab, int th, int h_off) {
 #pragma unroll
-  for (int P = 0; P < KP; ++P)
-#pragma unroll
-    for (int m = 0; m < 4; ++m)
+    for (int P = 0; P < KP; ++P)
 #pragma unroll
       for (int nt = 0; nt < KNT; ++nt) {
         const int n = nt * 8 + g, h = n / 2, d = n % 2;  // column = (head of this warp, digit)
-        if (h < GW) {
-          const unsigned char* row = prep + ((P * GW + h) * 2 + d) * 128;
-          qb[P][m][nt][0] = __ldcg(reinterpret_cast<const uint32_t*>(row + ((2 * m) * 4 + t) * 4));
-          qb[P][m][nt][1] = __ldcg(reinterpret_cast<const uint32_t*>(row + ((2 * m + 1) * 4 + t) * 4));
+        const uint32_t* row = reinterpret_cast<const uint32_t*>(tab + ((P * th + h_off + min(h, GW - 1)) * 2 + d) * 128);
+        if constexpr (KV) {  // KIVI's table keeps word x at (x % 4) * 8 + x / 4: two 16-byte loads
+          const uint4 w0 = *reinterpret_cast<const uint4*>(row + t * 8);
+          const uint4 w1 = *reinterpret_cast<const uint4*>(row + t * 8 + 4);
+          const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            qb[P][m][nt][0] = h < GW ? w[2 * m] : 0u;
+            qb[P][m][nt][1] = h < GW ? w[2 * m + 1] : 0u;
+          }
         } else {
-          qb[P][m][nt][0] = qb[P][m][nt][1] = 0u;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            qb[P][m][nt][0] = h < GW ? __ldcg(row + (2 * m) * 4 + t) : 0u;
+            qb[P][m][nt][1] = h < GW ? __ldcg(row + (2 * m + 1) * 4 + t) : 0u;
+          }
         }
       }
-  // this thread's logit columns (2t, 2t+1) of N-tile nt: digits (hi, lo) of head 4 nt + t
-  const float* hconst = reinterpret_cast<const float*>(prep + KP * GW * 2 * 128);
+  };
   // Rows g, g + 8 of the key contraction carry operand bytes 2^g (g < 7) or -128 (g = 7); the
   // head scales are in units of the -128 byte, so this thread's rows rescale them by rowf.
   const float rowf = g == 7 ? 1.f : -128.f / (float)(1 << g);
+  // this thread's logit columns (2t, 2t+1) of N-tile nt: digits (hi, lo) of head 4 nt + t
   float hs[KNT], hc[KNT], hsz[KNT], hcz[KNT];
+  if (!KV) {
+    const unsigned char* prep = p.qprep + (pair * p.hsplit + (G > 4 ? (warp >> 2) : half)) * p.qprep_stride;
+    load_qb(prep, GW, 0);
+    const float* hconst = reinterpret_cast<const float*>(prep + KP * GW * 2 * 128);
 #pragma unroll
-  for (int nt = 0; nt < KNT; ++nt) {
-    const int h = min(4 * nt + t, GW - 1);
-    hs[nt] = __ldcg(hconst + h * 4 + 0) * rowf;
-    hc[nt] = __ldcg(hconst + h * 4 + 1);
-    hsz[nt] = __ldcg(hconst + h * 4 + 2) * rowf;
-    hcz[nt] = __ldcg(hconst + h * 4 + 3);
+    for (int nt = 0; nt < KNT; ++nt) {
+      const int h = min(4 * nt + t, GW - 1);
+      hs[nt] = __ldcg(hconst + h * 4 + 0) * rowf;
+      hc[nt] = __ldcg(hconst + h * 4 + 1);
+      hsz[nt] = __ldcg(hconst + h * 4 + 2) * rowf;
+      hcz[nt] = __ldcg(hconst + h * 4 + 3);
+    }
+  } else {  // KIVI: the query itself; the digits follow per key group
+    for (int i = tid; i < G * kHeadDim; i += NT)
+      kq[i] = load_q(p.q, ((size_t)b * p.Hq + h_first + i / kHeadDim) * kHeadDim + i % kHeadDim, p.bf16) * p.logit_scale;
+    __syncthreads();  // the group builds read other threads' coordinates
   }
   const float vkappa = VQ ? kSqrtHalfPi / (float)p.v.m : 0.f;
 
@@ -483,6 +532,65 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     const unsigned char* kt = stages + ((unsigned)it % kStagesM) * stage_bytes;
     const int tok0 = it * kCtaTok;  // chunk-relative first token of this iteration
     const int count = min(kCtaTok, t_end - (t_begin + tok0));
+    if (KV && (t_begin + tok0) % kKiviGroup == 0) {
+      // KIVI key group: logit = sum_j q_j (s_j code_j + z_j) with code = b0 + 2 b1, so plane P's
+      // query term is 2^P q_j s_j (a 16-bit integer relative to the head's largest |2 q_j s_j|,
+      // as two digits) and the head's offset is sum_j q_j z_j. Warp h builds head h: lane l takes
+      // coordinates 4l .. 4l + 3, i.e. word x = l of each digit row, stored where load_qb reads it
+      // with two 16-byte loads (word x at (x % 4) * 8 + x / 4).
+      const __half* st = reinterpret_cast<const __half*>(kt + 2 * ktb + kNormBlock);
+      const uint2 s4 = *reinterpret_cast<const uint2*>(st + 4 * lane);
+      const uint2 z4 = *reinterpret_cast<const uint2*>(st + kHeadDim + 4 * lane);
+      const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&s4.x));
+      const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&s4.y));
+      const float2 z01 = __half22float2(*reinterpret_cast<const __half2*>(&z4.x));
+      const float2 z23 = __half22float2(*reinterpret_cast<const __half2*>(&z4.y));
+      const float sv[4] = {s01.x, s01.y, s23.x, s23.y}, zv[4] = {z01.x, z01.y, z23.x, z23.y};
+      const int wpos = (lane & 3) * 8 + (lane >> 2);
+      for (int h = warp; h < G; h += NW) {
+        const float4 q4 = *reinterpret_cast<const float4*>(kq + h * kHeadDim + 4 * lane);
+        const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+        float x[4], a = 0.f, c = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[e] = qv[e] * sv[e];
+          a = fmaxf(a, fabsf(x[e]));
+          c = fmaf(qv[e], zv[e], c);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+          c += __shfl_xor_sync(0xffffffffu, c, o);
+        }
+        const float vmax = a > 0.f ? 2.f * a : 1.f;
+        const float qsc = (float)kQRange / vmax;
+#pragma unroll
+        for (int P = 0; P < KP; ++P) {
+          uint32_t hw = 0u, lw = 0u;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int q = __float2int_rn(((float)(1 << P) * x[e]) * qsc);
+            const int hi = (q + 128) >> 8, lo = q - 256 * hi;
+            hw |= (uint32_t)(hi & 0xFF) << (8 * e);
+            lw |= (uint32_t)(lo & 0xFF) << (8 * e);
+          }
+          reinterpret_cast<uint32_t*>(ktab + ((P * G + h) * 2 + 0) * kHeadDim)[wpos] = hw;
+          reinterpret_cast<uint32_t*>(ktab + ((P * G + h) * 2 + 1) * kHeadDim)[wpos] = lw;
+        }
+        if (lane == 0) {
+          kcon[2 * h] = vmax / ((float)kQRange * -128.f);
+          kcon[2 * h + 1] = c;
+        }
+      }
+      __syncthreads();
+      load_qb(ktab, G, hb);
+#pragma unroll
+      for (int nt = 0; nt < KNT; ++nt) {
+        const int h = hb + min(4 * nt + t, GW - 1);
+        hs[nt] = kcon[2 * h] * rowf;
+        hc[nt] = kcon[2 * h + 1];
+      }
+    }
     {
       // Key bits in octet order: warp w's tokens 16w..16w+15 are octets o0, o0 + 1 of tile w / 2.
       // Row g of the contraction is token 8 o0 + g, row g + 8 token 8 (o0 + 1) + g: both keep bit g
@@ -568,7 +676,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
           l0 = fmaf(gk0, fmaf(hsz[nt], (float)(cz[0] * 256 + cz[1]), hcz[nt]), l0);
           l1 = fmaf(gk1, fmaf(hsz[nt], (float)(cz[2] * 256 + cz[3]), hcz[nt]), l1);
         }
-        const float lg0 = v0 ? nk0 * l0 : -INFINITY, lg1 = v1 ? nk1 * l1 : -INFINITY;
+        // (KIVI keys have no per-token norm)
+        const float lg0 = v0 ? (KV ? l0 : nk0 * l0) : -INFINITY, lg1 = v1 ? (KV ? l1 : nk1 * l1) : -INFINITY;
         if (h < GW) {
           lgs[(hb + h) * lgst + tok0 + tl + g] = lg0;
           lgs[(hb + h) * lgst + tok0 + tl + g + 8] = lg1;
@@ -579,7 +688,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
     // largest value weight: tokens of this iteration, one per thread of warps 0 and 1
     if (tid < count) {  // staged value norms: [tile][64 B norms | 64 B gammas]
       const unsigned char* nb = kt + 2 * ktb + (tid / kTile) * 128 + (tid % kTile) * 2;
-      const float w = __half2float(*reinterpret_cast<const __half*>(nb)) * kInvSqrtD;
+      const float w = __half2float(*reinterpret_cast<const __half*>(nb)) * (KV ? 1.f : kInvSqrtD);
       wmax = fmaxf(wmax, w);
       if (VQ) wmaxz = fmaxf(wmaxz, w * (__half2float(*reinterpret_cast<const __half*>(nb + 64)) * vkappa));
     }
@@ -619,6 +728,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   for (int w = 0; w < NW; ++w) task_m = fmaxf(task_m, hmax[w * G + task_h]);
   float task_l = 0.f;                 // sum of p over this task's tokens
   uint32_t task_wc = 0, task_wz = 0;  // sums of the quantised weights (exact: <= 64 tokens x 2^23)
+  float task_pz = 0.f;                // KIVI: sum of p z over this task's tokens (value zero points)
 
   // Weight digits of pass-2 iteration `it` into digit buffer it & 1: p = 2^(l - m) for the task's
   // tokens, then both kinds of value weight; w * scale is rounded by adding 2^23, after which the
@@ -635,14 +745,14 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       const float2 l2 = *reinterpret_cast<const float2*>(lgs + task_h * lgst + tok0 + T);
       const float2 n2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::NORM + ((unsigned)T % kTile) * 2));
       lv[0] = l2.x; lv[TPT - 1] = l2.y; wc[0] = n2.x; wc[TPT - 1] = n2.y;
-      if (VQ) {
+      if (VQ || KV) {
         const float2 g2 = __half22float2(*reinterpret_cast<const __half2*>(vtile + VL::GAMMA + ((unsigned)T % kTile) * 2));
         wz[0] = g2.x; wz[TPT - 1] = g2.y;
       }
     } else {
       lv[0] = lgs[task_h * lgst + tok0 + T];
       wc[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::NORM + ((unsigned)T % kTile) * 2));
-      if (VQ) wz[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::GAMMA + ((unsigned)T % kTile) * 2));
+      if (VQ || KV) wz[0] = __half2float(*reinterpret_cast<const __half*>(vtile + VL::GAMMA + ((unsigned)T % kTile) * 2));
     }
     uint32_t bc[TPT], bz[TPT];
     float psum = 0.f;
@@ -651,9 +761,10 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       const bool ok = T + e < count;
       const float pe = ex2(lv[e] - task_m);
       psum += pe;
-      const float n = ok ? wc[e] * (kInvSqrtD * wsc) : 0.f;
+      const float n = ok ? wc[e] * ((KV ? 1.f : kInvSqrtD) * wsc) : 0.f;
       bc[e] = __float_as_uint(fmaf(pe, n, kRoundBias));
       task_wc += bc[e] - 0x4B000000u;
+      if (KV && ok) task_pz = fmaf(pe, wz[e], task_pz);
       if (VQ) {
         const float nz = ok ? wc[e] * wz[e] * (kInvSqrtD * wscz * vkappa) : 0.f;
         bz[e] = __float_as_uint(fmaf(pe, nz, kRoundBias));
@@ -661,7 +772,7 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       }
     }
     task_l += psum;
-    unsigned char* col = pdig + (it & 1) * PDB + (size_t)(4 * task_h) * kPdStride + T;
+    unsigned char* col = pdig + (it & 1) * PDB + (size_t)(3 * task_h) * kPdStride + T;
 #pragma unroll
     for (int kind = 0; kind < NKIND; ++kind) {
       const uint32_t* bw = kind ? bz : bc;
@@ -773,10 +884,10 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   float* hsum = tsum + 3 * NT;                      // [3][G]: sum p, sum weights, sum sketch weights
   tsum[3 * tid] = task_l;
   tsum[3 * tid + 1] = (float)task_wc;
-  tsum[3 * tid + 2] = (float)task_wz;
+  tsum[3 * tid + 2] = KV ? task_pz : (float)task_wz;
   __syncthreads();
   if (tid < 3 * G) {
-    const int what = tid / G, h = tid % G;  // what: 0 sum p, 1 sum weights, 2 sum sketch weights
+    const int what = tid / G, h = tid % G;  // what: 0 sum p, 1 sum weights, 2 sum sketch weights (KIVI: p z)
     float s2 = 0.f;
     for (int q = 0; q < TASKS_PER_HEAD; ++q) s2 += tsum[3 * (h * TASKS_PER_HEAD + q) + what];
     hsum[tid] = s2;
@@ -787,39 +898,58 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
   float vasum = 0.f;
 #pragma unroll
   for (int P = 0; P < VWP; ++P) vasum += va[P];
+  if (KV) {  // KIVI codes b0 + 2 b1 on 0/1 planes: 2 va_P = 2^P, no Walsh offset
+    va[0] = 0.5f;
+    va[1] = 1.f;
+    vasum = 0.f;
+  }
   const float inv_w = 1.f / wsc, inv_wz = 1.f / wscz;
+  // Column c = 3h + d of the value contraction holds byte digit d (weight 2^16, 2^8, 1) of head h,
+  // on lane 4g + (c % 8) / 2 (register pair c / 8, element c % 2): the quad of lanes 4g .. 4g + 3
+  // holds every column of rows g and g + 8, so each head's three digits are gathered by shuffles
+  // (a fixed summation order) and lane 4g + h % 4 writes the head's coordinates.
+  float offs[G], offz[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    offs[h] = KV ? hsum[2 * G + h] : -vasum * hsum[G + h] * inv_w;  // KIVI: sum_t p_t z_t
+    offz[h] = VQ ? -hsum[2 * G + h] * inv_wz : 0.f;
+  }
 #pragma unroll
   for (int pi = 0; pi < PPW; ++pi) {
     const int pos = PPW * warp + pi;
     const float rowpos = pos == 7 ? -1.f / 128.f : 1.f / (float)(1 << pos);  // row value 2^p or -128
     const float rowinv = rowpos * inv_w, rowinvz = rowpos * inv_wz;
 #pragma unroll
-    for (int nt = 0; nt < VNT; ++nt) {
-      const int h = 2 * nt + t / 2;
-      // columns (2t, 2t+1): byte digits (2, 1) for even t, (0, pad) for odd t, of head 2 nt + t / 2
-      const float wd0 = (t & 1) ? 1.f : 65536.f, wd1 = (t & 1) ? 0.f : 256.f;
-      float o0 = 0.f, o1 = 0.f, z0 = 0.f, z1 = 0.f;
+    for (int rr = 0; rr < 2; ++rr) {
+      const int j = 8 * (g + 8 * rr) + pos;  // coordinate of row g (rr = 0) or g + 8
+      float vo[VNT][2], vz[VNT][2];  // this lane's columns, planes folded
 #pragma unroll
-      for (int P = 0; P < VP; ++P) {
-        float r0 = (float)vacc[P][pi][nt][0] * wd0 + (float)vacc[P][pi][nt][1] * wd1;
-        float r1 = (float)vacc[P][pi][nt][2] * wd0 + (float)vacc[P][pi][nt][3] * wd1;
-        r0 += __shfl_xor_sync(0xffffffffu, r0, 1);
-        r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
-        const bool sk = VQ && P == VP - 1;
-        if (sk) { z0 = 2.f * r0 * rowinvz; z1 = 2.f * r1 * rowinvz; }
-        else { o0 = fmaf(2.f * va[min(P, 3)], r0 * rowinv, o0); o1 = fmaf(2.f * va[min(P, 3)], r1 * rowinv, o1); }
-      }
-      if (h < G) {
-        float* dst = p.part + (((size_t)b * p.Hq + h_first + h) * p.splits + split) * p.part_stride;
-        const int j0 = 8 * g + pos, j1 = 8 * (g + 8) + pos;
-        if ((t & 1) == 0) {
-          const float Wt = hsum[G + h] * inv_w;
-          dst[2 + j0] = o0 - vasum * Wt;
-          dst[2 + j1] = o1 - vasum * Wt;
-        } else if (VQ) {
-          const float Wz = hsum[2 * G + h] * inv_wz;
-          dst[2 + kHeadDim + j0] = z0 - Wz;
-          dst[2 + kHeadDim + j1] = z1 - Wz;
+      for (int nt = 0; nt < VNT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float o = 0.f, z = 0.f;
+#pragma unroll
+          for (int P = 0; P < VP; ++P) {
+            const float r = (float)vacc[P][pi][nt][2 * rr + e];
+            if (VQ && P == VP - 1) z = 2.f * r;
+            else o = fmaf(2.f * va[min(P, 3)], r, o);
+          }
+          vo[nt][e] = o;
+          vz[nt][e] = z;
+        }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float dg[3], dz[3];
+#pragma unroll
+        for (int d = 0; d < 3; ++d) {
+          const int c = 3 * h + d, src = (lane & ~3) | ((c & 7) >> 1);
+          dg[d] = __shfl_sync(0xffffffffu, vo[c >> 3][c & 1], src);
+          if (VQ) dz[d] = __shfl_sync(0xffffffffu, vz[c >> 3][c & 1], src);
+        }
+        if ((lane & 3) == (h & 3)) {
+          float* dst = p.part + (((size_t)b * p.Hq + h_first + h) * p.splits + split) * p.part_stride;
+          dst[2 + j] = fmaf(fmaf(dg[0], 65536.f, dg[1] * 256.f) + dg[2], rowinv, offs[h]);
+          if (VQ) dst[2 + kHeadDim + j] = fmaf(fmaf(dz[0], 65536.f, dz[1] * 256.f) + dz[2], rowinvz, offz[h]);
         }
       }
     }
@@ -870,19 +1000,27 @@ cudaError_t launch_prep(const DecodeParams& p, cudaStream_t s, const QuantizePar
   return launched();
 }
 
-template <int G, int KB, bool KQ, int VB, bool VQ>
+template <int G, int KB, bool KQ, int VB, bool VQ, bool KV = false>
 cudaError_t launch_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
-  if (!TileLayout<KB, KQ>::matches(p.k) || !TileLayout<VB, VQ>::matches(p.v)) return cudaErrorNotSupported;
+  using VL = std::conditional_t<KV, KiviVTile, TileLayout<VB, VQ>>;
+  if (!TileLayout<KB, KQ>::matches(p.k) || !VL::matches(p.v)) return cudaErrorNotSupported;
   if (p.k.order != kOrderOctet || p.v.order != kOrderByteLane) return cudaErrorNotSupported;
-  cudaError_t e = launch_prep<(G > 4 ? 4 : G), KB, KQ>(p, s, qp);  // query prep in pieces of <= 4 heads
-  if (e != cudaSuccess) return e;
+  if (KV && (p.chunk % kKiviGroup || qp)) return cudaErrorNotSupported;  // whole key groups per CTA
+  cudaError_t e = cudaSuccess;
+  // query prep in pieces of <= 4 heads (KIVI: none; the CTAs build each key group's digits)
+  if (!KV && (e = launch_prep<(G > 4 ? 4 : G), KB, KQ>(p, s, qp)) != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
-  const size_t smem = mma_smem_bytes(G, p.k, p.v, p.chunk);
-  auto kern = decode_lm_mma<G, KB, KQ, VB, VQ>;
+  size_t smem = mma_smem_bytes(G, p.k, p.v, p.chunk, KV);
+  if (p.win_fused) smem = std::max(smem, sizeof(float) * window_smem_floats<MmaCfg<G, KB, KQ, VB, VQ>::NW, G>());
+  auto kern = decode_lm_mma<G, KB, KQ, VB, VQ, KV>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.splits, p.Hkv * (G > 4 ? 1 : p.hsplit), p.B);
+  // split CTAs, then the window parts' CTAs (mixed-precision caches), in one dimension
+  const long rows = (long)p.Hkv * (G > 4 ? 1 : p.hsplit) * p.B;
+  const long ctas = rows * (p.splits + (p.win_fused ? p.win_parts : 0));
+  if (ctas > 0x7fffffffL) return cudaErrorInvalidValue;
+  cfg.gridDim = dim3((unsigned)ctas);
   cfg.blockDim = dim3(MmaCfg<G, KB, KQ, VB, VQ>::NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -952,8 +1090,8 @@ bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl
   return false;
 }
 
-int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk) {
-  const size_t per = mma_smem_bytes(group, k, v, chunk) + kSmemReserved;
+int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk, bool kivi) {
+  const size_t per = mma_smem_bytes(group, k, v, chunk, kivi) + kSmemReserved;
   const int by_regs = group > 4 ? kMinBlocksM / 2 : kMinBlocksM;  // 8-warp CTAs: half as many
   return std::max(1, std::min(by_regs, (int)(kSmemPerSm / per)));
 }
@@ -962,6 +1100,16 @@ bool mma_decode_supported(const DecodeParams& p) {
   if (!mma_modes_supported(p.group, p.k.bits, p.k.qjl, p.v.bits, p.v.qjl) || p.k.order != kOrderOctet) return false;
   return (p.group == 1 || p.group == 2 || p.group == 4 || (p.group == 8 && p.hsplit == 2)) && p.chunk % kCtaTok == 0 &&
          p.chunk <= kChunkMax && p.qprep != nullptr;
+}
+
+cudaError_t launch_decode_kivi_mma(const DecodeParams& p, cudaStream_t s) {
+  switch (p.group) {
+    case 1: return launch_mma<1, 2, false, 2, false, true>(p, s, nullptr, nullptr);
+    case 2: return launch_mma<2, 2, false, 2, false, true>(p, s, nullptr, nullptr);
+    case 4: return launch_mma<4, 2, false, 2, false, true>(p, s, nullptr, nullptr);
+    case 8: return launch_mma<8, 2, false, 2, false, true>(p, s, nullptr, nullptr);
+    default: return cudaErrorNotSupported;
+  }
 }
 
 cudaError_t launch_decode_lm_mma(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {

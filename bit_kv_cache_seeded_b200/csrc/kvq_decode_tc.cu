@@ -54,16 +54,6 @@ constexpr uint32_t kTmemColsT = 512;
 constexpr int kNormBlockT = 4 * 128;   // staged value norms (+ residual norms) of four tiles
 constexpr int kKN = 16;                // key-phase N: (head, digit) columns, padded
 
-// KIVI value tile: two code planes (byte-lane order), per-token fp16 scale and zero.
-struct KiviVTile {
-  static constexpr int PLANES = 0, SKETCH = 2 * kTile * 16, NORM = SKETCH, GAMMA = NORM + kTile * 2;
-  static constexpr int BYTES = GAMMA + kTile * 2;
-  static bool matches(const SideLayout& L) {
-    return L.off_planes == PLANES && L.off_norm == NORM && L.off_gamma == GAMMA && L.tile_bytes == BYTES && L.bits == 2 &&
-           !L.qjl;
-  }
-};
-constexpr int kKiviStats = 2 * kHeadDim * 2;  // a key group's fp16 scales and zeros
 
 // KV: the KIVI instance (2-bit unsigned codes b0 + 2 b1 instead of Walsh planes; per-group query
 // digits; per-token value scale and zero; no rotation).

@@ -122,13 +122,17 @@ struct DecodeParams {
   int cache_after_wait;   // fused step: the cache is written by this kernel's predecessor (wait first)
   int use_tc;             // decode on the tcgen05 kernel (one CTA per sequence, kv-head and split)
   // mixed-precision window: bf16 K and V of the sink and recent tokens, [B][Hkv][win_slots][d] each;
-  // lens above counts the coded history only, tot_lens every token; wpart [B][Hq][part_stride] gets
-  // the window's softmax state, which the reduce merges with the splits' (null: no window)
+  // lens above counts the coded history only, tot_lens every token; wpart [B][Hq][win_parts]
+  // [part_stride] gets the softmax states of the window's parts of 64 slots, which the reduce merges
+  // with the splits' (null: no window)
   const uint16_t* wk;
   const uint16_t* wv;
   int win_sink, win_recent, win_slots;
   const int* tot_lens;
   float* wpart;
+  int win_parts;
+  int win_fused;           // the mma.sync split kernel runs the window parts in CTAs past its splits'
+
   int win_kivi;            // KIVI caches: window = the incomplete last key group; outputs not rotated
   const char* kstats;      // KIVI caches: [B][Hkv][groups][2][d] fp16 key scales, zeros
   int groups_per_seq;
@@ -167,7 +171,7 @@ cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t 
 bool mma_decode_supported(const DecodeParams& p);
 // Resident CTAs per SM of the tensor-core decode kernel for a chunk of `chunk` tokens (shared
 // memory and registers), as the split plan counts them.
-int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk);
+int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk, bool kivi = false);
 // True when the tensor-core decode kernel handles this query group and code combination (the
 // cache then stores its keys in kOrderOctet).
 bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl);
@@ -185,6 +189,8 @@ int tc_chunk_max(int group);     // largest chunk (tokens) of one CTA
 cudaError_t launch_decode_lm_tc(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp);
 // The tcgen05 kernel's KIVI instance (chunks of whole 128-token key groups).
 cudaError_t launch_decode_kivi_tc(const DecodeParams& p, cudaStream_t s);
+// KIVI instance of the mma.sync split kernel (chunks of whole 128-token key groups).
+cudaError_t launch_decode_kivi_mma(const DecodeParams& p, cudaStream_t s);
 cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s);
 cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s);
 bool mla_mma_supported(const MlaParams& p);
@@ -220,7 +226,8 @@ struct kvq_cache {
   uint16_t* d_win = nullptr;// window caches: bf16 K then V window, [batch][kv-heads][sink + recent][d] each
   std::vector<int> hlens;   // host mirror of d_hlens
   bool kivi = false;        // KIVI codes (no rotation); the window is the incomplete last key group
-  bool kivi_tc = false;     // KIVI decode on the tcgen05 kernel (else the CUDA-core kernel)
+  bool kivi_tc = false;     // KIVI decode on the tcgen05 kernel
+  bool kivi_cuda = false;   // KIVI decode on the CUDA-core kernel (neither: the mma.sync kernel)
   char* d_kstats = nullptr; // KIVI: [batch][kv-heads][groups][2][d] fp16 key scales and zeros
   int groups_per_seq = 0;
   char* dev = nullptr;

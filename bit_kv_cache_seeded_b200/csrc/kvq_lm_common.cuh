@@ -73,5 +73,18 @@ struct TileLayout {
   }
 };
 
+// KIVI value tile: two code planes (byte-lane order), per-token fp16 scale (norm slot) and zero
+// (gamma slot). KIVI key tiles are TileLayout<2, false> (their norm slot unused).
+struct KiviVTile {
+  static constexpr int PLANES = 0, SKETCH = 2 * kTile * 16, NORM = SKETCH, GAMMA = NORM + kTile * 2;
+  static constexpr int BYTES = GAMMA + kTile * 2;
+  static bool matches(const SideLayout& L) {
+    return L.off_planes == PLANES && L.off_norm == NORM && L.off_gamma == GAMMA && L.tile_bytes == BYTES && L.bits == 2 &&
+           !L.qjl;
+  }
+};
+constexpr int kKiviStats = 2 * kHeadDim * 2;  // a key group's fp16 scales and zeros
+constexpr int kKiviGroup = 128;               // tokens per KIVI key group
+
 }  // namespace lmc
 }  // namespace kvq

@@ -96,13 +96,15 @@ def key_stats(cache, arena, pair, g):
     return st[:128], st[128:]
 
 
-@pytest.mark.parametrize("kernel", ["tc", "cuda"])
-@pytest.mark.parametrize("name,lens", [("llama8b", [1000, 128, 127, 0]), ("llama70b", [700, 300]), ("tiny", [1024])])
+@pytest.mark.parametrize("kernel", ["mma", "tc", "cuda"])
+@pytest.mark.parametrize("name,lens", [("llama8b", [1000, 128, 127, 0]), ("llama70b", [700, 300]), ("tiny", [1024]),
+                                       ("llama8b", [4000, 2500, 129])])
 def test_kivi_prefill(name, lens, kernel, monkeypatch):
-    """Both KIVI decode kernels: the tcgen05 instance (default) and the CUDA-core one
-    (KVQ_DECODE_KERNEL=cuda)."""
-    if kernel == "cuda":
-        monkeypatch.setenv("KVQ_DECODE_KERNEL", "cuda")
+    """The three KIVI decode kernels: the mma.sync instance (default), the tcgen05 one
+    (KVQ_DECODE_KERNEL=tc) and the CUDA-core one (KVQ_DECODE_KERNEL=cuda); the longest case spans
+    several splits per sequence."""
+    if kernel != "mma":
+        monkeypatch.setenv("KVQ_DECODE_KERNEL", kernel)
     w = kivi_workload(name, len(lens))
     data = generate(w, DEV, seqs=range(len(lens)), ctx=max(lens))
     cache = kvq.KvqCache(kvq.cfg_for_workload(w), len(lens), max(lens) + 128)
