@@ -60,6 +60,7 @@ constexpr int kSmemPerSm = 233472;                   // shared memory per SM (22
 constexpr int kSmemReserved = 1024 + 128;            // per CTA: the runtime's reserve + static arrays
 constexpr int kPdStride = 96;                        // weight-digit row stride (bytes): 64 tokens + pad
 constexpr int kNormBlock = 256;                      // staged value norms / gammas of two cache tiles
+constexpr int kKeyChains = 2;                        // independent key accumulators (coordinate blocks m % 2)
 
 // A int8, B uint8 (the value-phase weight digits are non-negative bytes).
 __device__ __forceinline__ void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -600,13 +601,13 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
       const int s0 = (tl % kTile) + g, s1 = s0 + 8;
       const int o0 = (tl % kTile) / 8;
       const uint32_t mg = 0x01010101u << g;
-      int acc[2][KNT][4], accz[2][KNT][4];  // independent chains: coordinate block parity m & 1
+      int acc[kKeyChains][KNT][4], accz[kKeyChains][KNT][4];  // independent chains: m % kKeyChains
 #pragma unroll
       for (int m = 0; m < 4; ++m)
 #pragma unroll
         for (int nt = 0; nt < KNT; ++nt)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) { if (m < 2) { acc[m][nt][c] = 0; accz[m][nt][c] = 0; } }
+          for (int c = 0; c < 4; ++c) { if (m < kKeyChains) { acc[m][nt][c] = 0; accz[m][nt][c] = 0; } }
       // this thread's words of octet o: 8t + 2m + h, m = 0..3, h = 0..1 (32 contiguous bytes)
       const unsigned char* kp = ktile + KL::PLANES + o0 * 128 + t * 32;
 #pragma unroll
@@ -644,8 +645,8 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
             const uint32_t a0 = xa0 & mg, a1 = xb0 & mg, a2 = xa1 & mg, a3 = xb1 & mg;
 #pragma unroll
             for (int nt = 0; nt < KNT; ++nt) {
-              if (sk) mma_s8(accz[m & 1][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
-              else mma_s8(acc[m & 1][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+              if (sk) mma_s8(accz[m % kKeyChains][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
+              else mma_s8(acc[m % kKeyChains][nt], a0, a1, a2, a3, qb[P][m][nt][0], qb[P][m][nt][1]);
             }
           }
         }
@@ -664,8 +665,13 @@ decode_lm_mma(const __grid_constant__ DecodeParams p) {
         int c[4], cz[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          c[e] = acc[0][nt][e] + acc[1][nt][e];
-          cz[e] = accz[0][nt][e] + accz[1][nt][e];
+          c[e] = acc[0][nt][e];
+          cz[e] = accz[0][nt][e];
+#pragma unroll
+          for (int ch = 1; ch < kKeyChains; ++ch) {
+            c[e] += acc[ch][nt][e];
+            cz[e] += accz[ch][nt][e];
+          }
         }
         // hi * 256 + lo: exact in int32 up to 2 Walsh planes (|hi| < 2^22), else in fp32
         const float c01 = KB <= 2 ? (float)(c[0] * 256 + c[1]) : fmaf((float)c[0], 256.f, (float)c[1]);
