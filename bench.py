@@ -103,9 +103,32 @@ def window_len(w, L):
 # packed streams, from ncu captures (full size, or a smaller context scaled to the full launch by the
 # tokens processed). A record only counts while the kernel's sources are the ones captured (their
 # SHA-256 below); after any change the bench reports null until a new capture.
-TRAFFIC = {}
-TRAFFIC_SOURCES = ("bit_kv_cache_seeded_b200/csrc/kvq_decode_mma.cu", "bit_kv_cache_seeded_b200/csrc/kvq_async.cuh",
-                   "bit_kv_cache_seeded_b200/csrc/kvq_internal.h", "bit_kv_cache_seeded_b200/csrc/kvq_mla_umma.cu")
+TRAFFIC = {
+    "llama70b": {"dram_bytes": 2039889920, "captured": "ctx 8192, scaled x4 by the tokens processed",
+        "lsu_global_sectors_per_request": 7.17,
+        "sources_sha256": "ec782ae4be4b7bfc911497174a1e0b3bd51ec715daa3b05f8ca87898cb2dc724"},
+    "llama8b": {"dram_bytes": 113211392, "captured": "full size",
+        "lsu_global_sectors_per_request": 6.73,
+        "sources_sha256": "ec782ae4be4b7bfc911497174a1e0b3bd51ec715daa3b05f8ca87898cb2dc724"},
+    "onebit": {"dram_bytes": 1258420224, "captured": "ctx 4096, scaled x4 by the tokens processed",
+        "lsu_global_sectors_per_request": 5.83,
+        "sources_sha256": "ec782ae4be4b7bfc911497174a1e0b3bd51ec715daa3b05f8ca87898cb2dc724"},
+    "mla_fp4": {"dram_bytes": 443340288, "captured": "ctx 524288, scaled x2 by the tokens processed",
+        "lsu_global_sectors_per_request": 19.23,
+        "sources_sha256": "ec782ae4be4b7bfc911497174a1e0b3bd51ec715daa3b05f8ca87898cb2dc724"},
+    "llama8b_kivi": {"dram_bytes": 79322368, "captured": "full size",
+        "lsu_global_sectors_per_request": 1.73,
+        "sources_sha256": "ec782ae4be4b7bfc911497174a1e0b3bd51ec715daa3b05f8ca87898cb2dc724"},
+    "llama8b_window": {"dram_bytes": 129805056, "captured": "full size",
+        "lsu_global_sectors_per_request": 5.57,
+        "sources_sha256": "ec782ae4be4b7bfc911497174a1e0b3bd51ec715daa3b05f8ca87898cb2dc724"},
+    "llama8b_paged": {"dram_bytes": 112907264, "captured": "full size",
+        "lsu_global_sectors_per_request": 6.67,
+        "sources_sha256": "ec782ae4be4b7bfc911497174a1e0b3bd51ec715daa3b05f8ca87898cb2dc724"},
+}
+TRAFFIC_SOURCES = tuple("bit_kv_cache_seeded_b200/csrc/" + f for f in (
+    "kvq_decode_mma.cu", "kvq_async.cuh", "kvq_internal.h", "kvq_lm_common.cuh", "kvq_tiles.cuh", "kvq_window.cuh",
+    "kvq_quantize_lm.cuh", "kvq_mla_umma.cu", "kvq_tcgen05.cuh"))
 
 
 def kernel_sources_sha():
@@ -539,7 +562,9 @@ def measure(kvq, w, args, world, dev):
                          kernel=KERNEL_NAMES[w.name],
                          bytes_per_launch=bytes_kernel, ms_per_launch=kern_ms[1],
                          load_efficiency=dict(load_eff, dram_over_algorithmic=None if tr is None else
-                                              tr["dram_bytes"] / bytes_kernel)),
+                                              tr["dram_bytes"] / bytes_kernel,
+                                              lsu_global_sectors_per_request=None if tr is None else
+                                              tr["lsu_global_sectors_per_request"])),
         "decode_call": {"ms": call_ms, "bytes": bytes_step, "gbs": achieved_call,
                         "kernels_ms": {"prep": kern_ms[0], "split": kern_ms[1], "reduce": kern_ms[2]}},
         "e2e": {"value": e2e_value, "unit": "KV tokens/s", "h2d_bytes_per_step": h2d,

@@ -25,9 +25,9 @@ def _lib():
     kvq.load()
 
 
-def kivi_workload(name, batch):
+def kivi_workload(name, batch, **over):
     w = WORKLOADS[name]
-    return w.with_(batch=batch, k_mode="kivi", v_mode="kivi", k_bits=2, v_bits=2, qjl_dim=0)
+    return w.with_(batch=batch, k_mode="kivi", v_mode="kivi", k_bits=2, v_bits=2, qjl_dim=0, **over)
 
 
 def f64(t):
@@ -111,6 +111,18 @@ def test_kivi_prefill(name, lens, kernel, monkeypatch):
     for b, T in enumerate(lens):
         if T:
             cache.quantize(data["k"][b:b + 1, :, :T].contiguous(), data["v"][b:b + 1, :, :T].contiguous(), seq_ids=[b])
+    check(w, cache, data, lens)
+    cache.close()
+
+
+def test_kivi_query_group_2():
+    """The KIVI instance for query groups of 2 (16 query heads over 8 kv-heads)."""
+    lens = [640, 200]
+    w = kivi_workload("llama8b", len(lens), n_q_heads=16)
+    data = generate(w, DEV, seqs=range(len(lens)), ctx=max(lens))
+    cache = kvq.KvqCache(kvq.cfg_for_workload(w), len(lens), max(lens) + 128)
+    for b, T in enumerate(lens):
+        cache.quantize(data["k"][b:b + 1, :, :T].contiguous(), data["v"][b:b + 1, :, :T].contiguous(), seq_ids=[b])
     check(w, cache, data, lens)
     cache.close()
 
