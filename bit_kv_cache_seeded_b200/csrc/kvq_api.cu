@@ -271,10 +271,11 @@ int decode_max_units(const kvq_cache* c) {
 }
 
 // The LM decode kernel a cache uses: the mma.sync kernel (measured faster), or the tcgen05 kernel
-// when the environment variable KVQ_DECODE_KERNEL is "tc" at cache creation.
+// when the environment variable KVQ_DECODE_KERNEL is "tc" (lockstep) or "ws" (warp-specialised) at
+// cache creation.
 bool choose_tc(const kvq_cfg& cfg, const SideLayout& k, const SideLayout& v) {
   const char* e = std::getenv("KVQ_DECODE_KERNEL");
-  if (!e || std::strcmp(e, "tc") != 0) return false;
+  if (!e || (std::strcmp(e, "tc") != 0 && std::strcmp(e, "ws") != 0)) return false;
   return k.order == kOrderOctet && tc_modes_supported(cfg.n_q_heads / cfg.n_kv_heads, k.bits, k.qjl, v.bits, v.qjl);
 }
 
@@ -418,6 +419,7 @@ kvq_status cache_init(kvq_cache** out, const kvq_cfg* cfg, int32_t batch, int32_
   }
   c->signs_stride = cfg->rot_per_head ? kHeadDim : 0;
   c->tc = !P.fp4_mode && !P.kivi && choose_tc(*cfg, P.k, P.v);
+  c->ws = c->tc && std::strcmp(std::getenv("KVQ_DECODE_KERNEL"), "ws") == 0;
   {
     const char* e = std::getenv("KVQ_DECODE_KERNEL");
     // KIVI decode: the mma.sync kernel, or (KVQ_DECODE_KERNEL at cache creation) "tc" the tcgen05
@@ -735,7 +737,7 @@ kvq_status decode_impl(const kvq_cache* c, const void* q, kvq_dtype dtype, float
   p.err = c->d_status;
   p.wait_limit = wait_limit;
   p.debug_unset_wait = debug_unset_wait;
-  p.use_tc = c->tc ? 1 : 0;
+  p.use_tc = c->tc ? (c->ws ? 2 : 1) : 0;
   if (has_window(c)) {
     const size_t pairs_kv = (size_t)c->batch * c->cfg.n_kv_heads;
     p.wk = c->d_win;

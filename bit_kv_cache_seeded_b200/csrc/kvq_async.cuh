@@ -28,6 +28,10 @@ __device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
 }
+// One arrival (count 1) on the barrier, releasing this thread's earlier shared-memory accesses.
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
 // Orders this thread's earlier generic-proxy shared-memory accesses (after a barrier, those of
 // the whole CTA) before later bulk copies into the same buffer.
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
@@ -54,6 +58,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
     asm volatile(
         "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2, %3;\n selp.u32 %0, 1, 0, q;\n}\n"
         : "=r"(done) : "r"(bar), "r"(parity), "r"(100000u) : "memory");
+    if (done) return true;
+    if (clock64() - t0 > limit) return false;
+  }
+}
+
+// The same wait without a suspend-time hint: each try_wait returns after the hardware's own short
+// limit, so a thread that waits on a neighbour in a pipeline resumes as soon as the phase completes.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(done) : "r"(bar), "r"(parity) : "memory");
     if (done) return true;
     if (clock64() - t0 > limit) return false;
   }

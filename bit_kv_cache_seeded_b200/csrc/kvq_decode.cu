@@ -410,7 +410,10 @@ cudaError_t dispatch_modes(const DecodeParams& p, dim3 grid, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_decode_lm(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp) {
-  if (p.use_tc) return tc_decode_supported(p) ? launch_decode_lm_tc(p, s, ev_mid, qp) : cudaErrorNotSupported;
+  if (p.use_tc) {
+    if (!tc_decode_supported(p)) return cudaErrorNotSupported;
+    return p.use_tc == 2 ? launch_decode_lm_ws(p, s, ev_mid, qp) : launch_decode_lm_tc(p, s, ev_mid, qp);
+  }
   if (mma_decode_supported(p)) return launch_decode_lm_mma(p, s, ev_mid, qp);
   if (qp) return cudaErrorNotSupported;
   if (ev_mid && cudaEventRecord(ev_mid, s) != cudaSuccess) return cudaErrorUnknown;

@@ -120,7 +120,8 @@ struct DecodeParams {
   long long wait_limit;   // SM clock cycles a kernel waits for staged data before giving up
   int debug_unset_wait;   // test entry: also wait once on a barrier nothing completes
   int cache_after_wait;   // fused step: the cache is written by this kernel's predecessor (wait first)
-  int use_tc;             // decode on the tcgen05 kernel (one CTA per sequence, kv-head and split)
+  int use_tc;             // decode on a tcgen05 kernel (one CTA per sequence, kv-head and split):
+                          // 1 the lockstep kernel, 2 the warp-specialised one
   // mixed-precision window: bf16 K and V of the sink and recent tokens, [B][Hkv][win_slots][d] each;
   // lens above counts the coded history only, tot_lens every token; wpart [B][Hq][win_parts]
   // [part_stride] gets the softmax states of the window's parts of 64 slots, which the reduce merges
@@ -187,6 +188,8 @@ bool tc_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl)
 bool tc_decode_supported(const DecodeParams& p);
 int tc_chunk_max(int group);     // largest chunk (tokens) of one CTA
 cudaError_t launch_decode_lm_tc(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp);
+// Warp-specialised tcgen05 kernel (kvq_decode_ws.cu): same modes, chunks and prep area as the tcgen05 kernel.
+cudaError_t launch_decode_lm_ws(const DecodeParams& p, cudaStream_t s, cudaEvent_t ev_mid, const QuantizeParams* qp);
 // The tcgen05 kernel's KIVI instance (chunks of whole 128-token key groups).
 cudaError_t launch_decode_kivi_tc(const DecodeParams& p, cudaStream_t s);
 // KIVI instance of the mma.sync split kernel (chunks of whole 128-token key groups).
@@ -218,7 +221,8 @@ struct kvq_cache {
   int batch = 0, capacity = 0, tiles_per_seq = 0, sms = 148;
   int signs_stride = 0;     // 0, or kHeadDim when every kv-head has its own rotation diagonal
   int device = -1;          // the CUDA device whose memory holds the arena (current at init)
-  bool tc = false;          // LM decode runs on the tcgen05 kernel (else mma.sync / CUDA cores)
+  bool tc = false;          // LM decode runs on a tcgen05 kernel (else mma.sync / CUDA cores)
+  bool ws = false;          // ... the warp-specialised one
   int sink = 0, recent = 0; // mixed-precision window (0, 0: none)
   const int* table = nullptr;  // paged caches: caller's device block table [batch][pages_per_seq]
   int pages_per_seq = 0, n_pages = 0;

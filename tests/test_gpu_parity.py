@@ -522,24 +522,28 @@ def test_tile_quantize_equals_token_by_token(name):
 
 # ---------------------------------------------------------------- the two LM decode kernels
 
+@pytest.mark.parametrize("kernel", ["tc", "ws"])
 @pytest.mark.parametrize("name,lens", [("llama8b", [700, 65]), ("llama70b", [1000, 129]), ("onebit", [300, 1])])
-def test_tcgen05_kernel_parity(name, lens, monkeypatch):
-    """The tcgen05 decode kernel (chosen with KVQ_DECODE_KERNEL=tc at cache creation) against the
-    oracle, as the mma.sync kernel is by default."""
-    monkeypatch.setenv("KVQ_DECODE_KERNEL", "tc")
+def test_tcgen05_kernel_parity(name, lens, kernel, monkeypatch):
+    """The tcgen05 decode kernels (chosen with KVQ_DECODE_KERNEL=tc, the lockstep one, or =ws, the
+    warp-specialised one, at cache creation) against the oracle, as the mma.sync kernel is by
+    default."""
+    monkeypatch.setenv("KVQ_DECODE_KERNEL", kernel)
     run_small(name, len(lens), lens, seed_appends=2)
 
 
+@pytest.mark.parametrize("kernel", ["tc", "ws"])
 @pytest.mark.parametrize("name", ["llama8b", "llama70b", "onebit"])
-def test_tcgen05_and_mma_sync_kernels_agree(name, monkeypatch):
-    """Both LM decode kernels on the same cache contents: outputs within the attention tolerance of
-    each other, over contexts that span several iterations with a ragged tail."""
+def test_tcgen05_and_mma_sync_kernels_agree(name, kernel, monkeypatch):
+    """A tcgen05 kernel and the mma.sync kernel on the same cache contents: outputs within the
+    attention tolerance of each other, over contexts that span several iterations with a ragged
+    tail."""
     w = WORKLOADS[name].with_(batch=3)
     lens = [1500, 700, 64]
     data = generate(w, DEV, seqs=range(3), ctx=max(lens))
     monkeypatch.delenv("KVQ_DECODE_KERNEL", raising=False)
     c_mma = new_cache(w, 3, 1536)[0]
-    monkeypatch.setenv("KVQ_DECODE_KERNEL", "tc")
+    monkeypatch.setenv("KVQ_DECODE_KERNEL", kernel)
     c_tc = new_cache(w, 3, 1536)[0]
     for c in (c_mma, c_tc):
         for b, L in enumerate(lens):
