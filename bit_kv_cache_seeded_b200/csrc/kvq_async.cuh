@@ -12,6 +12,11 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
 }
+// Arrives once on the mbarrier when every cp.async this thread issued before has completed (the
+// barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
@@ -75,6 +80,18 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, lo
     if (done) return true;
     if (clock64() - t0 > limit) return false;
   }
+}
+
+// The same wait polling with the non-blocking test (and a short sleep between tests), for warps
+// that wait on a neighbour in a pipeline: a blocking try_wait would hold the barrier unit while
+// other warps of the CTA need it.
+__device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (clock64() - t0 > limit) return false;
+    __nanosleep(20);
+  }
+  return true;
 }
 
 // Programmatic dependent launch (sm_90+). A kernel launched with programmatic stream

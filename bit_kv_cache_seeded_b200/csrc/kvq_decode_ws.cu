@@ -9,9 +9,11 @@
 // instead of every warp taking every step between CTA barriers, each warp has one role and the
 // roles hand work to each other through mbarriers, so expansion, tensor-core products and
 // epilogues of neighbouring iterations overlap.
-//   * warp 12 (one thread): the bulk copies of the cache tiles into four shared-memory stages, each
-//     as soon as the stage's previous contents have been consumed;
-//   * warp 13 (one thread): the tcgen05.mma issue of every iteration, committing to the barriers of
+//   * warps 12-14: the bulk copies of the cache tiles into six shared-memory stages, fill f by warp
+//     12 + f % 3, each as soon as the stage's previous contents have been consumed (the lanes issue
+//     pieces of a fill at once; one copying warp alone held a CTA to about one fill per memory
+//     latency);
+//   * warp 15 (one thread): the tcgen05.mma issue of every iteration, committing to the barriers of
 //     whoever waits;
 //   * warps 0-7, expansion: key bits (pass 1) and value bits (pass 2) of the iteration's 128 tokens
 //     expanded into one of two tensor-memory A buffers; warp w reaches lanes 32 (w % 4) .. + 31 and
@@ -43,12 +45,14 @@ namespace {
 using namespace lmc;
 
 constexpr int kTokW = 128;                          // tokens per iteration (four cache tiles)
-constexpr int kStagesW = 6;                         // bulk-copy stages
+constexpr int kMaxStagesW = 12;                     // bulk-copy stages: as many as shared memory holds
+constexpr int kSmemW = 227 * 1024;                  // dynamic shared memory of one CTA (at most)
 constexpr int kNBV = 4;                             // weight-digit (B_v) buffers
 constexpr int kExpW = 8;                            // expansion warps 0 .. 7
 constexpr int kEpiW = 4;                            // epilogue warps 8 .. 11
-constexpr int kProdW = kExpW + kEpiW;               // warp 12: bulk copies
-constexpr int kIssW = kProdW + 1;                   // warp 13: MMA issue
+constexpr int kProdW = kExpW + kEpiW;               // warps 12 .. 14: bulk copies
+constexpr int kNProd = 3;
+constexpr int kIssW = kProdW + kNProd;              // warp 15: MMA issue (16 warps: 128 registers)
 constexpr int kThreadsW = (kIssW + 1) * 32;
 constexpr uint32_t kTmemColsW = 512;
 constexpr int kKNW = 16;                            // key-phase N: 8 heads x 2 digits
@@ -85,6 +89,11 @@ struct WsCfg {
   static constexpr int BK = KP * kKNW * 128;                  // query digits, [KP][16 rows][128 K]
   static constexpr int BV = VN * kTokW;                       // one weight-digit buffer (kNBV of them)
   static constexpr int TPT = G;                               // tokens per weight task (128 tasks)
+  static constexpr int CHUNK = G > 4 ? 4096 : 8192;           // largest chunk (the split plan's bound)
+  static constexpr int LGS = 4 * G * ((CHUNK + kTokW - 1) / kTokW * kTokW + 8);
+  static constexpr int FIXED = BK + kNBV * BV + LGS + 4 * (8 * G + 8 + 3 * kTokW + 3 * G) + 1024;
+  static constexpr int NS0 = (kSmemW - FIXED) / STAGE;
+  static constexpr int NS = NS0 > kMaxStagesW ? kMaxStagesW : NS0;  // stages
 };
 
 __host__ __device__ inline int ws_logit_stride(int chunk) { return (chunk + kTokW - 1) / kTokW * kTokW + 8; }
@@ -92,7 +101,7 @@ __host__ __device__ inline int ws_logit_stride(int chunk) { return (chunk + kTok
 // Dynamic shared memory: stages | B_k | kNBV x B_v | logits [G][stride] | head constants | reductions.
 template <class C>
 size_t ws_smem_bytes(int G, int chunk) {
-  return (size_t)kStagesW * C::STAGE + C::BK + kNBV * C::BV +
+  return (size_t)C::NS * C::STAGE + C::BK + kNBV * C::BV +
          sizeof(float) * ((size_t)G * ws_logit_stride(chunk) + 4 * G + 4 * G + 8 + 3 * kTokW + 3 * G);
 }
 
@@ -112,13 +121,15 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
   using KL = typename C::KL;
   using VL = typename C::VL;
   constexpr int KP = C::KP, VP = C::VP, VWP = C::VWP, NK0 = C::NK0, TPT = C::TPT, NA = C::NA, DKB = C::DKB;
+  constexpr int kStagesW = C::NS;
+  static_assert(kStagesW >= 4, "stages");
   constexpr int vtb = VL::BYTES;
   extern __shared__ __align__(1024) unsigned char smem[];
   // barriers: stage full / consumed, A buffer full / free, key accumulator full / free, weight
   // digits full / free, value products done, one nothing completes (test entry). A ring of R uses
   // slot u % R and completes phase u / R of its barriers.
   enum {
-    FULL = 0, EMPTY = FULL + kStagesW, AF = EMPTY + kStagesW, AE = AF + 8, DKF = AE + 8, DKE = DKF + 4,
+    FULL = 0, EMPTY = FULL + kMaxStagesW, AF = EMPTY + kMaxStagesW, AE = AF + 8, DKF = AE + 8, DKE = DKF + 4,
     BVF = DKE + 4, BVE = BVF + kNBV, DVD = BVE + kNBV, UNSET = DVD + 1, NBAR = UNSET + 1
   };
   __shared__ __align__(8) uint64_t bars[NBAR];
@@ -210,43 +221,51 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
     }
   };
 
-  if (warp == kProdW) {
-    // ======================= bulk copies (one thread)
-    if (lane == 0) {
-      // Fill f < n_iter: the K tiles of pass-1 iteration f (each at stride KT) and their value norms;
-      // fill n_iter + i: the V tiles of pass-2 iteration i. Tiles past the chunk's last token pair
-      // are not copied (their rows are masked or weighted zero).
-      auto issue = [&](int f) {
-        const int st = f % kStagesW;
-        const uint32_t fb = bar(FULL + st);
-        unsigned char* dst = stages + st * C::STAGE;
-        const int it = f < n_iter ? f : f - n_iter;
-        const int t0 = t_begin + it * kTokW;
-        const int tile0 = (unsigned)t0 / kTile;
-        const int ntiles = 2 * min(2, (t_end - t0 + 2 * kTile - 1) / (2 * kTile));
+  if (warp >= kProdW && warp < kProdW + kNProd) {
+    // ======================= bulk copies (one warp)
+    // A bulk copy instruction occupies its issuing thread for a time that grows with its size, so
+    // the copies of a fill are cut into pieces issued by different lanes at once: K fills, 4 pieces
+    // of each tile (lanes 0-15) and the tiles' value norms (lanes 16-19); V fills, 8 pieces of each
+    // tile pair (lanes 0-15). Fill f < n_iter: the K tiles of pass-1 iteration f (each at stride KT);
+    // fill n_iter + i: the V tiles of pass-2 iteration i. Tiles past the chunk's last token pair are
+    // not copied (their rows are masked or weighted zero).
+    constexpr int kPcK = 4, kPcV = 8;
+    static_assert(KL::BYTES % (16 * kPcK) == 0 && (2 * vtb) % (16 * kPcV) == 0, "16-byte pieces");
+    constexpr uint32_t pbk = KL::BYTES / kPcK, pbv = 2 * vtb / kPcV;
+    for (int f = warp - kProdW; f < n_fill; f += kNProd) {
+      const int st = f % kStagesW;
+      const uint32_t fb = bar(FULL + st);
+      unsigned char* dst = stages + st * C::STAGE;
+      const int it = f < n_iter ? f : f - n_iter;
+      const int t0 = t_begin + it * kTokW;
+      const int tile0 = (unsigned)t0 / kTile;
+      const int ntiles = 2 * min(2, (t_end - t0 + 2 * kTile - 1) / (2 * kTile));
+      constexpr uint32_t nb = VQ ? 128u : 64u;  // value norms (+ gammas, contiguous) per tile
+      if (lane == 0) {
+        if (f >= kStagesW) wait(EMPTY + st, ((unsigned)(f / kStagesW) - 1u) & 1u);
         fence_proxy_async();  // the stage's previous contents were read by the generic proxy
-        if (f < n_iter) {
-          constexpr uint32_t nb = VQ ? 128u : 64u;  // value norms (+ gammas, contiguous) per tile
-          mbar_arrive_expect_tx(fb, (uint32_t)ntiles * (KL::BYTES + nb));
-          for (int tt = 0; tt < ntiles; ++tt) {
-            const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk,
-                                            tile0 + tt, p.err);
-            bulk_g2s(smem_addr(dst + tt * C::KT), kreg + (size_t)ti * KL::BYTES, KL::BYTES, fb);
-            bulk_g2s(smem_addr(dst + C::KNORM + tt * 128), vreg + (size_t)ti * vtb + VL::NORM, nb, fb);
-          }
-        } else {
-          mbar_arrive_expect_tx(fb, (uint32_t)ntiles * vtb);
-          for (int j = 0; j < ntiles / 2; ++j) {
-            const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk,
-                                            tile0 + 2 * j, p.err);
-            bulk_g2s(smem_addr(dst + 2 * j * vtb), vreg + (size_t)ti * vtb, 2u * vtb, fb);
-          }
-        }
-      };
-      for (int f = 0; f < n_fill; ++f) {
-        if (f >= kStagesW) wait(EMPTY + f % kStagesW, ((unsigned)(f / kStagesW) - 1u) & 1u);
-        issue(f);
+        mbar_arrive_expect_tx(fb, f < n_iter ? (uint32_t)ntiles * (KL::BYTES + nb) : (uint32_t)ntiles * vtb);
       }
+      __syncwarp();
+      if (f < n_iter) {
+        const int tt = lane < 16 ? lane / kPcK : lane - 16, pc = lane % kPcK;
+        if (tt < ntiles && lane < 20) {
+          const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk,
+                                          tile0 + tt, p.err);
+          if (lane < 16)
+            bulk_g2s(smem_addr(dst + tt * C::KT + pc * pbk), kreg + (size_t)ti * KL::BYTES + pc * pbk, pbk, fb);
+          else
+            bulk_g2s(smem_addr(dst + C::KNORM + tt * 128), vreg + (size_t)ti * vtb + VL::NORM, nb, fb);
+        }
+      } else {
+        const int j = lane / kPcV, pc = lane % kPcV;
+        if (lane < 16 && j < ntiles / 2) {
+          const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk,
+                                          tile0 + 2 * j, p.err);
+          bulk_g2s(smem_addr(dst + 2 * j * vtb + pc * pbv), vreg + (size_t)ti * vtb + pc * pbv, pbv, fb);
+        }
+      }
+      __syncwarp();
     }
   } else if (warp == kIssW) {
     // ======================= MMA issue (one thread)
@@ -307,31 +326,36 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
     };
     // Planes of half hf: plane P for P = hf, hf + 2, ..; with 3-bit codes half 0 takes planes 0, 1
     // (and the sketch) and half 1 plane 2 and the parity plane b0 ^ b1 ^ b2 from the same loads.
+    // All of a half's loads are issued before its first store (a tensor-memory store is a barrier
+    // to the compiler, so loads after it would wait for it).
     auto expand = [&](auto load, int nwalsh, int bits, bool sketch, uint32_t mask, uint32_t col0) {
-      uint32_t r[32];
+      uint32_t ra[32], rb[32];
       if (bits == 3) {
         if (hf == 0) {
-          load(0, r); put(r, mask, col0 + 0 * 32);
-          load(1, r); put(r, mask, col0 + 1 * 32);
-          if (sketch) { load(-1, r); put(r, mask, col0 + nwalsh * 32); }
+          load(0, ra);
+          load(1, rb);
+          put(ra, mask, col0 + 0 * 32);
+          put(rb, mask, col0 + 1 * 32);
+          if (sketch) {
+            load(-1, ra);
+            put(ra, mask, col0 + nwalsh * 32);
+          }
         } else {
-          uint32_t t1[32];
-          load(2, r);
-          load(0, t1);
+          uint32_t rc[32];
+          load(2, ra);
+          load(0, rb);
+          load(1, rc);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) t1[c] ^= r[c];
-          put(r, mask, col0 + 2 * 32);
-          load(1, r);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) r[c] ^= t1[c];
-          put(r, mask, col0 + 3 * 32);
+          for (int c = 0; c < 32; ++c) rc[c] ^= rb[c] ^ ra[c];
+          put(ra, mask, col0 + 2 * 32);
+          put(rc, mask, col0 + 3 * 32);
         }
       } else {
-        const int np = nwalsh + (sketch ? 1 : 0);
-        for (int P = hf; P < np; P += 2) {
-          load(P < nwalsh ? P : -1, r);
-          put(r, mask, col0 + P * 32);
-        }
+        const int np = nwalsh + (sketch ? 1 : 0);  // at most 3: planes hf and hf + 2
+        if (hf < np) load(hf < nwalsh ? hf : -1, ra);
+        if (hf + 2 < np) load(hf + 2 < nwalsh ? hf + 2 : -1, rb);
+        if (hf < np) put(ra, mask, col0 + hf * 32);
+        if (hf + 2 < np) put(rb, mask, col0 + (hf + 2) * 32);
       }
     };
     for (int i = 0; i < n_iter; ++i) {
@@ -349,13 +373,12 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
         }
       };
       expand(load, C::KWP, KB, KQ, 0x01010101u << jbit, C::COL_A + ab * C::APL * 32);
+      __syncwarp();  // every lane's loads of the stage have been consumed by its stores
+      if (lane == 0) mbar_arrive(bar(EMPTY + st));
       tc::wait_st();
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(AF + ab));
-        mbar_arrive(bar(EMPTY + st));
-      }
+      if (lane == 0) mbar_arrive(bar(AF + ab));
     }
     // pass 2: row 32 qtr + lane = byte lane 4 qtr + lane / 8, bit lane % 8 (coordinate 32 qtr + lane)
     const int vlane = 4 * qtr + (lane >> 3);
@@ -377,13 +400,12 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
       };
       // tiles past the chunk's data were not copied: their tokens have zero weights (0 x anything)
       expand(load, VWP, VB, VQ, 0x01010101u << jbit, C::COL_A + ab * C::APL * 32);
+      __syncwarp();  // every lane's loads of the stage have been consumed by its stores
+      if (lane == 0) mbar_arrive(bar(EMPTY + st));
       tc::wait_st();
       tc::fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(AF + ab));
-        mbar_arrive(bar(EMPTY + st));
-      }
+      if (lane == 0) mbar_arrive(bar(AF + ab));
     }
   } else {
     // ======================= epilogues (warps 8 .. 11, lane quarters 0 .. 3)
@@ -399,6 +421,17 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
     for (int i = 0; i < n_iter; ++i) {
       const int db = i % DKB, st = i % kStagesW;
       wait(FULL + st, ((unsigned)i / kStagesW) & 1u);
+      // the stage's norms of this thread's token (key norm, residual norm, value norm and gamma),
+      // then the stage is released: its refill does not wait for this iteration's products
+      const unsigned char* kt = stages + st * C::STAGE;
+      const int tok = i * kTokW + tt * kTile + slot;  // chunk-relative
+      const bool valid = t_begin + tok < t_end;
+      const float nk = half_at(kt + tt * C::KT + KL::NORM + slot * 2);
+      const float gk = KQ ? half_at(kt + tt * C::KT + KL::GAMMA + slot * 2) : 0.f;
+      const float wn = half_at(kt + C::KNORM + tt * 128 + slot * 2) * kInvSqrtD;
+      const float wg = VQ ? half_at(kt + C::KNORM + tt * 128 + 64 + slot * 2) : 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(EMPTY + st));
       wait(DKF + db, ((unsigned)i / DKB) & 1u);
       tc::fence_after();
       uint32_t dm[16], dz[16];
@@ -408,11 +441,6 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
       tc::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(DKE + db));
-      const unsigned char* kt = stages + st * C::STAGE;
-      const int tok = i * kTokW + tt * kTile + slot;  // chunk-relative
-      const bool valid = t_begin + tok < t_end;
-      const float nk = half_at(kt + tt * C::KT + KL::NORM + slot * 2);
-      const float gk = KQ ? half_at(kt + tt * C::KT + KL::GAMMA + slot * 2) : 0.f;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const int c0 = (int)dm[2 * h], c1 = (int)dm[2 * h + 1];
@@ -428,13 +456,9 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
         mrow[h] = fmaxf(mrow[h], lg);
       }
       if (valid) {  // the largest value weight of each kind (staged norms: [tile][64 B | 64 B gammas])
-        const unsigned char* nb = kt + C::KNORM + tt * 128 + slot * 2;
-        const float w = half_at(nb) * kInvSqrtD;
-        wmax = fmaxf(wmax, w);
-        if (VQ) wmaxz = fmaxf(wmaxz, w * (half_at(nb + 64) * vkappa));
+        wmax = fmaxf(wmax, wn);
+        if (VQ) wmaxz = fmaxf(wmaxz, wn * (wg * vkappa));
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(EMPTY + st));
     }
     // chunk maxima per head and the weight scales, over the four epilogue warps
     float* hm = red;           // [4][G]
@@ -475,23 +499,32 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
     for (int i = 0; i < n_iter; ++i) {
       const int g = n_iter + i, st = g % kStagesW, bb = i % kNBV;
       wait(FULL + st, ((unsigned)g / kStagesW) & 1u);
-      if (i >= kNBV) wait(BVE + bb, ((unsigned)i / kNBV - 1u) & 1u);
+      // the value norms (and gammas) of the task's tokens, then the stage is released
       const unsigned char* vt = stages + st * C::STAGE;
+      float nrm[TPT], gzv[TPT];
+#pragma unroll
+      for (int e = 0; e < TPT; ++e) {
+        const int T = task_T + e;
+        const bool ok = t_begin + i * kTokW + T < t_end;
+        const unsigned char* vtile = vt + (T / kTile) * vtb;
+        nrm[e] = ok ? half_at(vtile + VL::NORM + (T % kTile) * 2) : 0.f;
+        gzv[e] = (VQ && ok) ? half_at(vtile + VL::GAMMA + (T % kTile) * 2) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(EMPTY + st));
+      if (i >= kNBV) wait(BVE + bb, ((unsigned)i / kNBV - 1u) & 1u);
       uint32_t bc[TPT], bz[TPT];
       float psum = 0.f;
 #pragma unroll
       for (int e = 0; e < TPT; ++e) {
         const int T = task_T + e;
         const bool ok = t_begin + i * kTokW + T < t_end;
-        const unsigned char* vtile = vt + (T / kTile) * vtb;
         const float pe = ok ? ex2(lgs[task_h * lgst + i * kTokW + T] - task_m) : 0.f;
         psum += pe;
-        const float nrm = ok ? half_at(vtile + VL::NORM + (T % kTile) * 2) : 0.f;
-        bc[e] = __float_as_uint(fmaf(pe, nrm * (kInvSqrtD * wsc), kRoundBias));
+        bc[e] = __float_as_uint(fmaf(pe, nrm[e] * (kInvSqrtD * wsc), kRoundBias));
         task_wc += bc[e] - 0x4B000000u;
         if (VQ) {
-          const float gz = ok ? half_at(vtile + VL::GAMMA + (T % kTile) * 2) : 0.f;
-          bz[e] = __float_as_uint(fmaf(pe, nrm * gz * (kInvSqrtD * wscz * vkappa), kRoundBias));
+          bz[e] = __float_as_uint(fmaf(pe, nrm[e] * gzv[e] * (kInvSqrtD * wscz * vkappa), kRoundBias));
           task_wz += bz[e] - 0x4B000000u;
         }
       }
@@ -522,10 +555,7 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
       }
       fence_proxy_async();  // the digits are read by the tensor cores
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(BVF + bb));
-        mbar_arrive(bar(EMPTY + st));
-      }
+      if (lane == 0) mbar_arrive(bar(BVF + bb));
     }
     grid_dep_launch();  // the split reduce may be scheduled; it waits for this grid to finish
     // ---- finish: value accumulators, per-head sums, this thread's coordinate row
