@@ -9,21 +9,22 @@
 // instead of every warp taking every step between CTA barriers, each warp has one role and the
 // roles hand work to each other through mbarriers, so expansion, tensor-core products and
 // epilogues of neighbouring iterations overlap.
-//   * warps 12-14: the bulk copies of the cache tiles into six shared-memory stages, fill f by warp
-//     12 + f % 3, each as soon as the stage's previous contents have been consumed (the lanes issue
-//     pieces of a fill at once; one copying warp alone held a CTA to about one fill per memory
-//     latency);
-//   * warp 15 (one thread): the tcgen05.mma issue of every iteration, committing to the barriers of
-//     whoever waits;
+//   * warps 12-13: the bulk copies of the cache tiles into the shared-memory stages, fill f by warp
+//     12 + f % 2, each as soon as the stage's previous contents have been consumed. A copy
+//     instruction holds its thread for about 140 ns whatever its size (1-16 KB), so a fill is as few
+//     copies as the layout allows: its tiles in one copy (one per page of a paged cache), plus one
+//     small copy per tile for the value norms that pass 1 needs;
+//   * warps 14-15 (one thread each): the tcgen05.mma issue, pass 1 by alternate iterations and
+//     pass 2 by alternate planes (one instruction takes an issuing thread about 50 cycles, and
+//     threads issue in parallel), committing to the barriers of whoever waits;
 //   * warps 0-7, expansion: key bits (pass 1) and value bits (pass 2) of the iteration's 128 tokens
-//     expanded into one of two tensor-memory A buffers; warp w reaches lanes 32 (w % 4) .. + 31 and
+//     expanded into one of the tensor-memory A buffers; warp w reaches lanes 32 (w % 4) .. + 31 and
 //     takes half of the planes (w / 4);
 //   * warps 8-11, epilogue: pass 1 reads each iteration's logit accumulators and writes the chunk's
 //     logits; pass 2 turns logits and value norms into the weight digits (the B operand) of each
 //     iteration; at the end they read the value accumulators and write the partials.
-// Every key tile of an iteration is staged at a stride that is an odd multiple of 16 bytes modulo
-// 128, and a warp's 32 token rows are one octet of each of the four tiles, so the eight 16-byte
-// loads a thread makes per plane hit four different bank groups. Every wait is bounded; after one
+// A warp's 32 token rows are one octet of each of the iteration's four key tiles, which are staged
+// contiguously as they lie in the cache. Every wait is bounded; after one
 // gives up (bit 0 of the cache's status word) the CTA's later waits return at once, and the kernel
 // still waits, bounded, for its own copies and products before it frees its tensor memory.
 #include <algorithm>
@@ -50,10 +51,11 @@ constexpr int kSmemW = 227 * 1024;                  // dynamic shared memory of 
 constexpr int kNBV = 4;                             // weight-digit (B_v) buffers
 constexpr int kExpW = 8;                            // expansion warps 0 .. 7
 constexpr int kEpiW = 4;                            // epilogue warps 8 .. 11
-constexpr int kProdW = kExpW + kEpiW;               // warps 12 .. 14: bulk copies
-constexpr int kNProd = 3;
-constexpr int kIssW = kProdW + kNProd;              // warp 15: MMA issue (16 warps: 128 registers)
-constexpr int kThreadsW = (kIssW + 1) * 32;
+constexpr int kProdW = kExpW + kEpiW;               // warps 12, 13: bulk copies
+constexpr int kNProd = 2;
+constexpr int kIssW = kProdW + kNProd;              // warps 14, 15: MMA issue (16 warps: 128 registers)
+constexpr int kNIss = 2;
+constexpr int kThreadsW = (kIssW + kNIss) * 32;
 constexpr uint32_t kTmemColsW = 512;
 constexpr int kKNW = 16;                            // key-phase N: 8 heads x 2 digits
 constexpr int kEpiBar = 1;                          // named barrier of the 128 epilogue threads
@@ -81,7 +83,7 @@ struct WsCfg {
   static constexpr bool FITS = NA >= 2;
   using KL = TileLayout<KB, KQ>;
   using VL = TileLayout<VB, VQ>;
-  static constexpr int KT = (KL::BYTES + 31) / 32 * 32 + 16;  // staged key tile stride: 16 mod 32
+  static constexpr int KT = KL::BYTES;                        // staged key tile stride
   static constexpr int KNORM = 4 * KT;                        // value norms (+ gammas) of the four tiles
   static constexpr int KSTAGE = KNORM + 4 * 128;
   static constexpr int VSTAGE = 4 * VL::BYTES;
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
     }
     for (int i = 0; i < NA; ++i) {
       mbar_init(bar(AF + i), kExpW);
-      mbar_init(bar(AE + i), 1);
+      mbar_init(bar(AE + i), kNIss);
     }
     for (int i = 0; i < DKB; ++i) {
       mbar_init(bar(DKF + i), 1);
@@ -169,9 +171,9 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
     }
     for (int i = 0; i < kNBV; ++i) {
       mbar_init(bar(BVF + i), kEpiW);
-      mbar_init(bar(BVE + i), 1);
+      mbar_init(bar(BVE + i), kNIss);
     }
-    mbar_init(bar(DVD), 1);
+    mbar_init(bar(DVD), kNIss);
     mbar_init(bar(UNSET), 1);
     mbar_init_fence();
     s_fail = 0;
@@ -222,16 +224,10 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
   };
 
   if (warp >= kProdW && warp < kProdW + kNProd) {
-    // ======================= bulk copies (one warp)
-    // A bulk copy instruction occupies its issuing thread for a time that grows with its size, so
-    // the copies of a fill are cut into pieces issued by different lanes at once: K fills, 4 pieces
-    // of each tile (lanes 0-15) and the tiles' value norms (lanes 16-19); V fills, 8 pieces of each
-    // tile pair (lanes 0-15). Fill f < n_iter: the K tiles of pass-1 iteration f (each at stride KT);
-    // fill n_iter + i: the V tiles of pass-2 iteration i. Tiles past the chunk's last token pair are
-    // not copied (their rows are masked or weighted zero).
-    constexpr int kPcK = 4, kPcV = 8;
-    static_assert(KL::BYTES % (16 * kPcK) == 0 && (2 * vtb) % (16 * kPcV) == 0, "16-byte pieces");
-    constexpr uint32_t pbk = KL::BYTES / kPcK, pbv = 2 * vtb / kPcV;
+    // ======================= bulk copies (one warp per fill)
+    // Fill f < n_iter: the K tiles of pass-1 iteration f (lane 0: one copy; paged, lanes 0-1: one per
+    // page) and their value norms (lanes 16-19); fill n_iter + i: the V tiles of pass-2 iteration i.
+    // Tiles past the chunk's last token pair are not copied (their rows are masked or weighted zero).
     for (int f = warp - kProdW; f < n_fill; f += kNProd) {
       const int st = f % kStagesW;
       const uint32_t fb = bar(FULL + st);
@@ -248,32 +244,46 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
       }
       __syncwarp();
       if (f < n_iter) {
-        const int tt = lane < 16 ? lane / kPcK : lane - 16, pc = lane % kPcK;
-        if (tt < ntiles && lane < 20) {
+        if (!p.table) {
+          if (lane == 0 && ntiles > 0) {
+            const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk, tile0, p.err);
+            bulk_g2s(smem_addr(dst), kreg + (size_t)ti * KL::BYTES, (uint32_t)ntiles * KL::BYTES, fb);
+          }
+        } else if (lane < ntiles / 2) {
           const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk,
-                                          tile0 + tt, p.err);
-          if (lane < 16)
-            bulk_g2s(smem_addr(dst + tt * C::KT + pc * pbk), kreg + (size_t)ti * KL::BYTES + pc * pbk, pbk, fb);
-          else
-            bulk_g2s(smem_addr(dst + C::KNORM + tt * 128), vreg + (size_t)ti * vtb + VL::NORM, nb, fb);
+                                          tile0 + 2 * lane, p.err);
+          bulk_g2s(smem_addr(dst + 2 * lane * KL::BYTES), kreg + (size_t)ti * KL::BYTES, 2u * KL::BYTES, fb);
+        }
+        if (lane >= 16 && lane - 16 < ntiles) {
+          const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk,
+                                          tile0 + lane - 16, p.err);
+          bulk_g2s(smem_addr(dst + C::KNORM + (lane - 16) * 128), vreg + (size_t)ti * vtb + VL::NORM, nb, fb);
         }
       } else {
-        const int j = lane / kPcV, pc = lane % kPcV;
-        if (lane < 16 && j < ntiles / 2) {
+        if (!p.table) {
+          if (lane == 0 && ntiles > 0) {
+            const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk, tile0, p.err);
+            bulk_g2s(smem_addr(dst), vreg + (size_t)ti * vtb, (uint32_t)ntiles * vtb, fb);
+          }
+        } else if (lane < ntiles / 2) {
           const long ti = tile_index_read(p.table, p.pages_per_seq, p.n_pages, p.tiles_per_seq, p.Hkv, b, hk,
-                                          tile0 + 2 * j, p.err);
-          bulk_g2s(smem_addr(dst + 2 * j * vtb + pc * pbv), vreg + (size_t)ti * vtb + pc * pbv, pbv, fb);
+                                          tile0 + 2 * lane, p.err);
+          bulk_g2s(smem_addr(dst + 2 * lane * vtb), vreg + (size_t)ti * vtb, 2u * vtb, fb);
         }
       }
       __syncwarp();
     }
-  } else if (warp == kIssW) {
-    // ======================= MMA issue (one thread)
+  } else if (warp >= kIssW) {
+    // ======================= MMA issue (lane 0 of each issuing warp)
+    // A thread's tcgen05.mma instructions issue about one per 50 cycles, so two threads share them:
+    // pass 1 by iteration (each iteration's logits have their own accumulator), pass 2 by plane
+    // (each plane has its own value accumulator); a buffer is free once both have committed to it.
+    const int j = warp - kIssW;
     if (lane == 0) {
       constexpr uint32_t kIdK = tc::idesc_i8(0, 1, 128, kKNW);  // u8 key bits x s8 query digits
       constexpr uint32_t kIdV = tc::idesc_i8(0, 0, 128, NK0);   // u8 value bits x u8 weight digits
       const uint32_t bk0 = smem_addr(bk);
-      for (int i = 0; i < n_iter; ++i) {
+      for (int i = j; i < n_iter; i += kNIss) {
         const int ab = i % NA, db = i % DKB;
         wait(AF + ab, ((unsigned)i / NA) & 1u);
         if (i >= DKB) wait(DKE + db, ((unsigned)i / DKB - 1u) & 1u);
@@ -289,7 +299,8 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
                            tc::smem_desc(bk0 + P * (kKNW * 128) + 2 * kk * 128, 128, 8 * 128), kIdK,
                            (sk ? kk > 0 : (P > 0 || kk > 0)) ? 1u : 0u);
         }
-        tc::commit(bar(AE + ab));
+#pragma unroll
+        for (int c = 0; c < kNIss; ++c) tc::commit(bar(AE + ab));
         tc::commit(bar(DKF + db));
       }
       for (int i = 0; i < n_iter; ++i) {
@@ -301,6 +312,7 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
         const uint32_t bv0 = smem_addr(bv + bb * C::BV);
 #pragma unroll
         for (int P = 0; P < VP; ++P) {
+          if (P % kNIss != j) continue;
           const int kind = (VQ && P == VP - 1) ? 1 : 0;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -624,7 +636,7 @@ __global__ void __launch_bounds__(kThreadsW, 1) decode_lm_ws(const __grid_consta
   if (warp == kProdW && lane == 0 && s_fail)
     for (int f = max(0, n_fill - kStagesW); f < n_fill; ++f)
       mbar_wait(bar(FULL + f % kStagesW), ((unsigned)f / kStagesW) & 1u, p.wait_limit);
-  if (warp == kIssW && lane == 0 && s_fail) mbar_wait(bar(DVD), 0u, p.wait_limit);
+  if (warp >= kIssW && lane == 0 && s_fail) mbar_wait(bar(DVD), 0u, p.wait_limit);
   tc::fence_before();
   __syncthreads();
   if (warp == 0) {
