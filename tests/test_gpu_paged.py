@@ -32,8 +32,15 @@ def contiguous_info(info, side, ntiles):
     return i
 
 
+@pytest.mark.parametrize("kernel", ["mma", "tc", "ws"])
 @pytest.mark.parametrize("name,lens", [("llama8b", [900, 64, 1]), ("llama70b", [700, 130]), ("onebit", [333, 64])])
-def test_shuffled_pages_equal_contiguous(name, lens):
+def test_shuffled_pages_equal_contiguous(name, lens, kernel, monkeypatch):
+    """On each LM decode kernel (mma.sync by default, tcgen05 with KVQ_DECODE_KERNEL=tc or ws), whose
+    fills find a paged cache's tiles through the block table."""
+    if kernel == "mma":
+        monkeypatch.delenv("KVQ_DECODE_KERNEL", raising=False)
+    else:
+        monkeypatch.setenv("KVQ_DECODE_KERNEL", kernel)
     w = WORKLOADS[name].with_(batch=len(lens))
     pps = (max(lens) + 63) // 64 + 1
     n_pages = len(lens) * pps + 3

@@ -138,13 +138,15 @@ def test_window_decode_step_equals_append_then_decode():
     ("tiny", {}, 8, 40, [300], "mma"),                                   # query group 1
     ("llama8b", {"n_q_heads": 16}, 16, 48, [400, 33], "mma"),           # query group 2
     ("llama8b", {}, 512, 512, [1500, 1024, 600], "mma"),                # the largest window: 16 parts
-    ("llama8b", {}, 64, 256, [900, 200], "tc"),                         # window kernel beside the tcgen05 kernel
+    ("llama8b", {}, 64, 256, [900, 200], "tc"),                         # window kernel beside the tcgen05 kernels
+    ("llama8b", {}, 64, 256, [900, 200], "ws"),
     ("llama8b", {"k_bits": 1, "v_mode": "lm", "v_bits": 1}, 32, 64, [600, 50], "mma"),  # beside the CUDA-core kernel
 ])
 def test_window_decode_paths(name, over, sink, recent, lens, kernel, monkeypatch):
     """The window parts on every decode path: as extra CTAs of the mma.sync split kernel (query
-    groups 1, 2, 4; 16 parts), and as their own kernel beside the tcgen05 split kernel and beside
-    the CUDA-core kernel (a code combination without a tensor-core instance)."""
+    groups 1, 2, 4; 16 parts), and as their own kernel beside the tcgen05 split kernels (lockstep
+    and warp-specialised) and beside the CUDA-core kernel (a code combination without a tensor-core
+    instance)."""
     if kernel != "mma":
         monkeypatch.setenv("KVQ_DECODE_KERNEL", kernel)
     w = WORKLOADS[name].with_(batch=len(lens), sink_tokens=sink, recent_tokens=recent, **over)
