@@ -566,6 +566,12 @@ kvq_status quantize_window(kvq_cache* c, const void* K, const void* V, kvq_dtype
     ph.win_src = 1;
     ph.n_new = max_cnt;
     ph.lens = c->d_hlens;
+    // a prefill (every sequence at the same length inside the sink, the same history count) codes
+    // its history straight from the input rows after the sink, in whole tiles
+    ph.win_input_only = 1;
+    ph.src_row0 = c->sink;
+    for (int i = 0; i < cnt; ++i)
+      if (p.total0[i] != p.total0[0] || p.total0[i] > c->sink || p.cnt[i] != max_cnt) ph.win_input_only = 0;
     if (launch_quantize_lm(ph, 2, s) != cudaSuccess) return KVQ_ERR_CUDA;
     for (int i = 0; i < cnt; ++i) c->hlens[p.seq[i]] = h1[i];
   }

@@ -83,6 +83,10 @@ struct QuantizeParams {
   // when it is below total0[s] (the length before the call), else from input row
   // (that position - total0[s]) of the call's src_rows rows. Window writes use total0 the same way.
   int win_src;
+  // History appends whose tokens all come from the input (every sequence of the launch had the same
+  // length, at most win_sink, before the call, and takes n_new = cnt[s] tokens): the tile kernel may
+  // code them, history position pos[s] + t from input row src_row0 - total0[s] + t.
+  int win_input_only, src_row0;
   const uint16_t* ring[2];  // bf16 window of K and V: [n_seq][heads][win_slots][d]
   int win_sink, win_recent, win_slots, src_rows;
   int win_kivi;             // KIVI caches: the window is the incomplete last key group (T % 128 tokens)

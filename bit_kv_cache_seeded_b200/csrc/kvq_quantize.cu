@@ -114,7 +114,7 @@ int grid_for(long work_items, int per_block) {
 }  // namespace
 
 cudaError_t launch_quantize_lm(const QuantizeParams& p, int n_sides, cudaStream_t s) {
-  if (n_sides == 2 && !p.skip_rotation && !p.win_src && p.n_new >= kTileQuantizeMinTokens) {
+  if (n_sides == 2 && !p.skip_rotation && (!p.win_src || p.win_input_only) && p.n_new >= kTileQuantizeMinTokens) {
     // appends of many tokens per sequence: whole tiles per block, 16-byte stores, S^T staged once
     const bool sketch = p.side[0].qjl || p.side[1].qjl;
     const long tiles = (long)p.n_seq * p.heads * qtile::max_tiles(p.n_new);

@@ -94,7 +94,10 @@ __device__ void quantize_tiles(const QuantizeParams& p, int side, float* st_s, S
 #pragma unroll 1
     for (int slot = warp; slot < kTile; slot += kWarps) {
       if (slot < lo || slot >= hi) continue;
-      const size_t base = (((size_t)s * p.heads + h) * p.n_new + (t0 + slot - pos0)) * kHeadDim;
+      // input rows of this (sequence, head): the call's n_new, or for window history the call's
+      // src_rows, of which the history starts at row src_row0 - total0[s]
+      const int rows = p.win_src ? p.src_rows : p.n_new, row0 = p.win_src ? p.src_row0 - p.total0[s] : 0;
+      const size_t base = (((size_t)s * p.heads + h) * rows + (row0 + t0 + slot - pos0)) * kHeadDim;
       float u[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) u[q] = qlm::load_elem(p.src[side], base + 32 * q + lane, p.bf16);
