@@ -16,15 +16,20 @@
 //      ahead) and dequantises it to f16, with the RoPE key, into the free one of two shared-memory
 //      buffers in the canonical no-swizzle "core matrix" layout (8 rows x 16 B blocks) that both
 //      MMAs read; this overlaps S of the current tile on the tensor cores;
-//   2. thread 0 issues S = Q K^T into tensor memory and commits to an mbarrier (for the next tile
-//      right after the current tile's O^T product);
-//   3. lanes 0..15 of warps 0..3 (the rows of S for an M=64 MMA) load their head's 64 logits,
+//   2. S = Q K^T goes into tensor memory as two accumulators over halves of K (the latent's first
+//      256 channels; the rest and the RoPE part), issued by lane 0 of warps 5 and 6, each committing
+//      to the S barrier; one thread issues a tcgen05.mma only about every 50 cycles, so the 52
+//      products of a tile are spread over four threads (O^T below on warps 4 and 7) that do no
+//      softmax;
+//   3. lanes 0..15 of warps 0..3 (the rows of S for an M=64 MMA) load and add their head's 64 logits,
 //      update a lazily rescaled running maximum (rescale only when it grows by more than 8 in
 //      log2 units), write P = 2^(l - m) (<= 256) as f16 in core-matrix layout;
 //   4. if a head's maximum moved, every thread rescales that head's column of O^T in tensor
 //      memory (load, multiply, store);
-//   5. thread 0 issues O^T += latent^T P^T and commits; the next iteration waits for it before
-//      it overwrites that latent buffer, P or O.
+//   5. lane 0 of warps 4 and 7 issue O^T += latent^T P^T (two M-blocks each) and commit; warps 5 and
+//      6 issue S of the next tile only after that (a named barrier of warps 4..7), so the tensor pipe
+//      runs O^T first and the next iteration, which waits for O^T before it overwrites that latent
+//      buffer, P or O, starts dequantising while S runs.
 // Every mbarrier wait is bounded (the cache status word records a wait that gave up). Partials
 // (m, l, o[512]) per (sequence, head, split) go to the workspace in the format of the other
 // MLA kernels; the same reduce kernel finishes.
@@ -44,8 +49,10 @@ constexpr int kLatU = 512, kRopeU = 64, kDqU = kLatU + kRopeU;
 constexpr int kHeadsU = 64;
 constexpr int kCore = 128;              // bytes of one core matrix (8 rows x 16 B)
 constexpr float kLazyRescale = 8.f;     // rescale O only when the running max grows by more than this
-constexpr uint32_t kTmemCols = 512;     // allocation: O^T in columns 0..255, S in 256..319
-constexpr uint32_t kColO = 0, kColS = 256;
+constexpr uint32_t kTmemCols = 512;     // allocation: O^T in columns 0..255, S in 256..319 and 320..383
+constexpr uint32_t kColO = 0, kColS = 256, kColS2 = 320;
+constexpr int kWarpO = 4, kWarpO2 = 7, kWarpS = 5;  // O^T: lane 0 of warps 4, 7; S: of warps 5, 6
+constexpr int kIssueBar = 2;                         // named barrier of warps 4..7: S after O^T
 
 // Shared-memory layout (bytes). Q: [8 head groups][72 dim chunks] core matrices; LAT (x2): [8 token
 // groups][64 dim chunks]; ROPE (x2): [8 token groups][8 dim chunks]; P: [8 head groups][8 token
@@ -168,8 +175,8 @@ __device__ __forceinline__ void dequant_tile(const TileRegs& r, unsigned char* l
 
 __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_constant__ MlaParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t bar_s;  // S = Q K^T done (all earlier MMAs too)
-  __shared__ __align__(8) uint64_t bar_o;  // O^T += latent^T P^T done (all earlier MMAs too)
+  __shared__ __align__(8) uint64_t bar_s;  // S = Q K^T done, both halves (their issuers' earlier MMAs too)
+  __shared__ __align__(8) uint64_t bar_o;  // O^T += latent^T P^T done, both halves (earlier MMAs too)
   __shared__ uint32_t s_tmem;              // tensor-memory base address
   __shared__ float s_alpha[kHeadsU];       // per-head O rescale factor of this iteration
   __shared__ float s_hsc[kHeadsU];         // per-head power-of-two query scale
@@ -188,8 +195,8 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
   auto tile_count = [&](int it) { return min(kTokU, t_end - (t_begin + it * kTokU)); };
 
   if (tid == 0) {
-    mbar_init(smem_addr(&bar_s), 1);
-    mbar_init(smem_addr(&bar_o), 1);
+    mbar_init(smem_addr(&bar_s), 2);
+    mbar_init(smem_addr(&bar_o), 2);
     mbar_init_fence();
     s_fail = 0;
   }
@@ -253,22 +260,30 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
   constexpr uint32_t kIdSr = idesc_f16(1, 0, 0, 64, kTokU);      // bf16 (RoPE part)
   constexpr uint32_t kIdO = idesc_f16(0, 1, 0, 128, kHeadsU);    // A (latent^T) MN-major
   const uint32_t aQ = smem_addr(sQ), aP = smem_addr(smem + kOffP);
-  auto issue_s = [&](int buf) {  // S = Q K^T over latent/RoPE buffer `buf`
+  // S = Q K^T over latent/RoPE buffer `buf`: half 0 takes latent K steps 0..15 into columns kColS,
+  // half 1 steps 16..31 and the RoPE part into kColS2 (the softmax adds the two)
+  auto issue_s = [&](int buf, int half) {
     const uint32_t aLat = smem_addr(smem + kOffLat + buf * kSizeLat), aRope = smem_addr(smem + kOffRope + buf * kSizeRope);
+    const uint32_t d = tmem + (half ? kColS2 : kColS);
 #pragma unroll 4
-    for (int kk = 0; kk < kLatU / 16; ++kk)
-      umma_f16(tmem + kColS, smem_desc(aQ + kk * 2 * kCore, kCore, (kDqU / 8) * kCore),
-               smem_desc(aLat + kk * 2 * kCore, kCore, (kLatU / 8) * kCore), kIdS, kk > 0);
+    for (int k = 0; k < kLatU / 32; ++k) {
+      const int kk = half * (kLatU / 32) + k;
+      umma_f16(d, smem_desc(aQ + kk * 2 * kCore, kCore, (kDqU / 8) * kCore),
+               smem_desc(aLat + kk * 2 * kCore, kCore, (kLatU / 8) * kCore), kIdS, k > 0);
+    }
+    if (half) {
 #pragma unroll
-    for (int kk = 0; kk < kRopeU / 16; ++kk)
-      umma_f16(tmem + kColS, smem_desc(aQ + (kLatU / 8 + 2 * kk) * kCore, kCore, (kDqU / 8) * kCore),
-               smem_desc(aRope + kk * 2 * kCore, kCore, (kRopeU / 8) * kCore), kIdSr, 1u);
+      for (int kk = 0; kk < kRopeU / 16; ++kk)
+        umma_f16(d, smem_desc(aQ + (kLatU / 8 + 2 * kk) * kCore, kCore, (kDqU / 8) * kCore),
+                 smem_desc(aRope + kk * 2 * kCore, kCore, (kRopeU / 8) * kCore), kIdSr, 1u);
+    }
     umma_commit(smem_addr(&bar_s));
   };
-  auto issue_o = [&](int buf, bool first) {  // O^T += latent^T P^T over buffer `buf`
+  // O^T += latent^T P^T over buffer `buf`, M-blocks (latent dims / 128) 2 half .. 2 half + 1
+  auto issue_o = [&](int buf, bool first, int half) {
     const uint32_t aLat = smem_addr(smem + kOffLat + buf * kSizeLat);
 #pragma unroll
-    for (int mt4 = 0; mt4 < kLatU / 128; ++mt4)
+    for (int mt4 = 2 * half; mt4 < 2 * half + 2; ++mt4)
 #pragma unroll
       for (int kk = 0; kk < kTokU / 16; ++kk)
         umma_f16(tmem + kColO + mt4 * kHeadsU,
@@ -276,9 +291,10 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
                  smem_desc(aP + kk * 2 * kCore, kCore, (kTokU / 8) * kCore), kIdO, (!first || kk > 0) ? 1u : 0u);
     umma_commit(smem_addr(&bar_o));
   };
-  if (tid == 0 && n_iter > 0) {
+  const bool s_issuer = lane == 0 && (warp == kWarpS || warp == kWarpS + 1);
+  if (s_issuer && n_iter > 0) {
     tc_fence_after();
-    issue_s(0);
+    issue_s(0, warp - kWarpS);
   }
 
   for (int it = 0; it < n_iter; ++it) {
@@ -300,9 +316,17 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
     // ---- softmax rows: lanes 0..15 of warps 0..3 hold head 16 warp + lane
     uint32_t sv0[32], sv1[32];
     if (warp < 4) {
+      uint32_t sx[32];
       tmem_ld32(tmem_warp + kColS, sv0);
       tmem_ld32(tmem_warp + kColS + 32, sv1);
+      tmem_ld32(tmem_warp + kColS2, sx);
       tmem_wait_ld();
+#pragma unroll
+      for (int t = 0; t < 32; ++t) sv0[t] = __float_as_uint(__uint_as_float(sv0[t]) + __uint_as_float(sx[t]));
+      tmem_ld32(tmem_warp + kColS2 + 32, sx);
+      tmem_wait_ld();
+#pragma unroll
+      for (int t = 0; t < 32; ++t) sv1[t] = __float_as_uint(__uint_as_float(sv1[t]) + __uint_as_float(sx[t]));
     }
     int moved = 0;
     if (head_lane) {
@@ -358,11 +382,20 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
     tc_fence_before();
     __syncthreads();
 
-    // ---- O^T += latent^T P^T for this tile, then S for the next one
-    if (tid == 0) {
-      tc_fence_after();
-      issue_o(buf, it == 0);
-      if (it + 1 < n_iter) issue_s(buf ^ 1);
+    // ---- O^T += latent^T P^T for this tile, then (other threads) S for the next one
+    if (warp == kWarpO || warp == kWarpO2) {
+      if (lane == 0) {
+        tc_fence_after();
+        issue_o(buf, it == 0, warp == kWarpO2);
+      }
+      __syncwarp();
+      asm volatile("bar.arrive %0, %1;\n" ::"n"(kIssueBar), "n"(128) : "memory");
+    } else if (warp == kWarpS || warp == kWarpS + 1) {
+      asm volatile("bar.sync %0, %1;\n" ::"n"(kIssueBar), "n"(128) : "memory");
+      if (lane == 0 && it + 1 < n_iter) {
+        tc_fence_after();
+        issue_s(buf ^ 1, warp - kWarpS);
+      }
     }
   }
 
@@ -390,7 +423,10 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
   }
 
   // ---- teardown: after a wait that gave up, wait once more (bounded) for the last MMAs
-  if (tid == 0 && s_fail && n_iter > 0) mbar_wait(smem_addr(&bar_o), (uint32_t)(n_iter - 1) & 1u, p.wait_limit);
+  if (tid == 0 && s_fail && n_iter > 0) {
+    mbar_wait(smem_addr(&bar_o), (uint32_t)(n_iter - 1) & 1u, p.wait_limit);
+    mbar_wait(smem_addr(&bar_s), (uint32_t)(n_iter - 1) & 1u, p.wait_limit);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
