@@ -331,13 +331,14 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
     int moved = 0;
     if (head_lane) {
       float x[kTokU];
-      float mt = -INFINITY;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
 #pragma unroll
       for (int t = 0; t < kTokU; ++t) {
         const float sv = __uint_as_float(t < 32 ? sv0[t] : sv1[t - 32]);
         x[t] = t < count ? sv * lsc : -INFINITY;
-        mt = fmaxf(mt, x[t]);
+        m4[t & 3] = fmaxf(m4[t & 3], x[t]);
       }
+      const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       float alpha = 1.f;
       if (mt > m_used + kLazyRescale) {  // also the first tile (m_used = -inf)
         alpha = m_used == -INFINITY ? 0.f : ex2f(m_used - mt);
@@ -346,7 +347,7 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
         moved = 1;
       }
       s_alpha[my_h] = alpha;
-      float ls = 0.f;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int tc = 0; tc < kTokU / 8; ++tc) {
         uint32_t h2[4];
@@ -354,13 +355,13 @@ __global__ void __launch_bounds__(kThreadsU, 1) decode_mla_umma(const __grid_con
         for (int e = 0; e < 4; ++e) {
           const float p0 = ex2f(x[8 * tc + 2 * e] - m_used);  // 2^-inf = +0
           const float p1 = ex2f(x[8 * tc + 2 * e + 1] - m_used);
-          ls += p0 + p1;
+          ls4[e] += p0 + p1;
           const __half2 hp = __floats2half2_rn(p0, p1);
           h2[e] = *reinterpret_cast<const uint32_t*>(&hp);
         }
         *reinterpret_cast<uint4*>(smem + kOffP + core_off(my_h, 8 * tc, kTokU / 8)) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
       }
-      l_run += ls;
+      l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
     }
     const int any_moved = __syncthreads_or(moved);
 
