@@ -97,6 +97,28 @@ def test_window_prefill(name, sink, recent, lens):
     cache.close()
 
 
+@pytest.mark.parametrize("first", [[10, 10], [10, 20], [32, 32]])
+def test_window_batched_prefill_after_a_short_start(first):
+    """A batched append after each sequence already holds a few tokens inside the sink: with equal
+    lengths the history is coded from the input rows after the sink (whole tiles), with unequal
+    lengths token by token; both against the oracle."""
+    w = WORKLOADS["llama8b"].with_(batch=2, sink_tokens=32, recent_tokens=64)
+    n_more = 700
+    T = [first[0] + n_more, first[1] + n_more]
+    data = generate(w, DEV, seqs=range(2), ctx=max(T))
+    cache = kvq.KvqCache(kvq.cfg_for_workload(w), 2, max(T) + 64)
+    for b in range(2):
+        cache.quantize(data["k"][b:b + 1, :, :first[b]].contiguous(), data["v"][b:b + 1, :, :first[b]].contiguous(),
+                       seq_ids=[b])
+    k_more = torch.stack([data["k"][b, :, first[b]:first[b] + n_more] for b in range(2)]).contiguous()
+    v_more = torch.stack([data["v"][b, :, first[b]:first[b] + n_more] for b in range(2)]).contiguous()
+    cache.quantize(k_more, v_more)
+    stats = {}
+    check(w, cache, data, T, data["q"], stats)
+    check_flip_rates(stats, "window batched prefill")
+    cache.close()
+
+
 def test_window_appends_move_tokens_through_the_ring():
     """Token-by-token appends (each evicting one ring token into the history), then appends of 40
     and of 150 tokens (more than the window holds: some go straight to the history)."""
