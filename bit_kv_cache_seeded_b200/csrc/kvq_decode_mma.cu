@@ -55,7 +55,6 @@ constexpr int kWarpsM = 4;
 constexpr int kThreadsM = kWarpsM * 32;
 constexpr int kCtaTok = 64;
 constexpr int kStagesM = 4;                          // bulk-copy stages (tile pairs in flight)
-constexpr int kMinBlocksM = 4;                       // resident CTAs per SM the registers are sized for
 constexpr int kSmemPerSm = 233472;                   // shared memory per SM (228 KB)
 constexpr int kSmemReserved = 1024 + 128;            // per CTA: the runtime's reserve + static arrays
 constexpr int kPdStride = 96;                        // weight-digit row stride (bytes): 64 tokens + pad
@@ -1096,9 +1095,47 @@ bool mma_modes_supported(int group, int k_bits, int k_qjl, int v_bits, int v_qjl
   return false;
 }
 
+// Resident CTAs per SM of one instance as its registers and threads allow (shared memory aside),
+// from the runtime's occupancy calculator, once per instance.
+template <int G, int KB, bool KQ, int VB, bool VQ, bool KV>
+int mma_reg_slots() {
+  static int slots = 0;
+  if (slots == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_lm_mma<G, KB, KQ, VB, VQ, KV>,
+                                                      MmaCfg<G, KB, KQ, VB, VQ>::NT, 0) != cudaSuccess || n < 1)
+      n = 16 / MmaCfg<G, KB, KQ, VB, VQ>::NW;  // the launch bounds' guarantee
+    slots = n;
+  }
+  return slots;
+}
+
+template <int G>
+int mma_reg_slots_modes(const SideLayout& k, const SideLayout& v, bool kivi) {
+  if (kivi) return mma_reg_slots<G, 2, false, 2, false, true>();
+#define KVQ_SLOTS_CASE(KB, KQ, VB, VQ) \
+  if (k.bits == KB && k.qjl == KQ && v.bits == VB && v.qjl == VQ) return mma_reg_slots<G, KB, KQ, VB, VQ, false>();
+  KVQ_SLOTS_CASE(2, true, 2, true)
+  KVQ_SLOTS_CASE(3, true, 3, false)
+  KVQ_SLOTS_CASE(1, false, 1, false)
+  KVQ_SLOTS_CASE(2, true, 2, false)
+  KVQ_SLOTS_CASE(3, true, 3, true)
+  KVQ_SLOTS_CASE(2, false, 2, false)
+  KVQ_SLOTS_CASE(3, false, 3, false)
+#undef KVQ_SLOTS_CASE
+  return 16 / Warps<G>::N;
+}
+
 int lm_mma_slots_per_sm(int group, const SideLayout& k, const SideLayout& v, int chunk, bool kivi) {
   const size_t per = mma_smem_bytes(group, k, v, chunk, kivi) + kSmemReserved;
-  const int by_regs = group > 4 ? kMinBlocksM / 2 : kMinBlocksM;  // 8-warp CTAs: half as many
+  int by_regs = 16 / Warps<8>::N;
+  switch (group) {
+    case 1: by_regs = mma_reg_slots_modes<1>(k, v, kivi); break;
+    case 2: by_regs = mma_reg_slots_modes<2>(k, v, kivi); break;
+    case 4: by_regs = mma_reg_slots_modes<4>(k, v, kivi); break;
+    case 8: by_regs = mma_reg_slots_modes<8>(k, v, kivi); break;
+    default: break;
+  }
   return std::max(1, std::min(by_regs, (int)(kSmemPerSm / per)));
 }
 

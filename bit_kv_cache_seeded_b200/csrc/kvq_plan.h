@@ -4,8 +4,9 @@
 // A split covers a whole number of 64-token units (two cache tiles), at most `max_units` of them.
 // plan_splits picks the split count that minimises waves x (units per CTA + a fixed per-CTA
 // overhead of 4 units), a wave holding slots_per_sm(units per CTA) resident CTAs on each of `sms`
-// SMs. max_splits bounds the split count for every length up to the capacity: the workspace is
-// sized from it once, so no call may plan more splits than it returns.
+// SMs; chunks may be as small as half the largest (smaller chunks need less shared memory for their
+// logits, so more CTAs can be resident). max_splits bounds the split count for every length up to
+// the capacity: the workspace is sized from it once, so no call may plan more splits than it returns.
 #pragma once
 
 #include <algorithm>
@@ -15,9 +16,11 @@ namespace kvq {
 constexpr int kPlanUnitTokens = 64;  // tokens of one split unit
 constexpr int kPlanUnitTiles = 2;    // cache tiles of one split unit
 
+inline int min_plan_units(int max_units) { return std::max(1, max_units / 2); }
+
 inline int max_splits(int pairs, int sms, int tiles, int max_units, int waves_bound) {
   const int units = std::max(1, tiles / kPlanUnitTiles);
-  const int need = (units + max_units - 1) / max_units;
+  const int need = (units + min_plan_units(max_units) - 1) / min_plan_units(max_units);
   const int bound = std::max(1, (waves_bound * sms + pairs - 1) / pairs);
   return std::max(need, std::min(bound, units));
 }
