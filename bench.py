@@ -104,27 +104,27 @@ def window_len(w, L):
 # tokens processed). A record only counts while the kernel's sources are the ones captured (their
 # SHA-256 below); after any change the bench reports null until a new capture.
 TRAFFIC = {
-    "llama70b": {"dram_bytes": 2039719936, "captured": "ctx 8192, scaled x4 by the tokens processed",
+    "llama70b": {"dram_bytes": 2039258112, "captured": "ctx 8192, scaled x4 by the tokens processed",
         "lsu_global_sectors_per_request": 7.17,
-        "sources_sha256": "12b81f64b763ee0fdef29347a8dccfef81f76f0bc3e34c9f19a6929524257b0e"},
-    "llama8b": {"dram_bytes": 113218304, "captured": "full size",
+        "sources_sha256": "dea02c0843e6721dbcef2a62c5c8e5d49bdfabf21868936614c2c7adb4ab0fe5"},
+    "llama8b": {"dram_bytes": 112607232, "captured": "full size",
         "lsu_global_sectors_per_request": 6.73,
-        "sources_sha256": "12b81f64b763ee0fdef29347a8dccfef81f76f0bc3e34c9f19a6929524257b0e"},
-    "onebit": {"dram_bytes": 1253391360, "captured": "ctx 4096, scaled x4 by the tokens processed",
+        "sources_sha256": "dea02c0843e6721dbcef2a62c5c8e5d49bdfabf21868936614c2c7adb4ab0fe5"},
+    "onebit": {"dram_bytes": 1261775872, "captured": "ctx 4096, scaled x4 by the tokens processed",
         "lsu_global_sectors_per_request": 5.83,
-        "sources_sha256": "12b81f64b763ee0fdef29347a8dccfef81f76f0bc3e34c9f19a6929524257b0e"},
-    "mla_fp4": {"dram_bytes": 443811328, "captured": "ctx 524288, scaled x2 by the tokens processed",
+        "sources_sha256": "dea02c0843e6721dbcef2a62c5c8e5d49bdfabf21868936614c2c7adb4ab0fe5"},
+    "mla_fp4": {"dram_bytes": 444171776, "captured": "ctx 524288, scaled x2 by the tokens processed",
         "lsu_global_sectors_per_request": 19.23,
-        "sources_sha256": "12b81f64b763ee0fdef29347a8dccfef81f76f0bc3e34c9f19a6929524257b0e"},
-    "llama8b_kivi": {"dram_bytes": 79204096, "captured": "full size",
-        "lsu_global_sectors_per_request": 1.73,
-        "sources_sha256": "12b81f64b763ee0fdef29347a8dccfef81f76f0bc3e34c9f19a6929524257b0e"},
-    "llama8b_window": {"dram_bytes": 129705984, "captured": "full size",
+        "sources_sha256": "dea02c0843e6721dbcef2a62c5c8e5d49bdfabf21868936614c2c7adb4ab0fe5"},
+    "llama8b_kivi": {"dram_bytes": 79039488, "captured": "full size",
+        "lsu_global_sectors_per_request": 1.77,
+        "sources_sha256": "dea02c0843e6721dbcef2a62c5c8e5d49bdfabf21868936614c2c7adb4ab0fe5"},
+    "llama8b_window": {"dram_bytes": 130097920, "captured": "full size",
         "lsu_global_sectors_per_request": 5.57,
-        "sources_sha256": "12b81f64b763ee0fdef29347a8dccfef81f76f0bc3e34c9f19a6929524257b0e"},
-    "llama8b_paged": {"dram_bytes": 112803328, "captured": "full size",
+        "sources_sha256": "dea02c0843e6721dbcef2a62c5c8e5d49bdfabf21868936614c2c7adb4ab0fe5"},
+    "llama8b_paged": {"dram_bytes": 112652544, "captured": "full size",
         "lsu_global_sectors_per_request": 6.67,
-        "sources_sha256": "12b81f64b763ee0fdef29347a8dccfef81f76f0bc3e34c9f19a6929524257b0e"},
+        "sources_sha256": "dea02c0843e6721dbcef2a62c5c8e5d49bdfabf21868936614c2c7adb4ab0fe5"},
 }
 TRAFFIC_SOURCES = tuple("bit_kv_cache_seeded_b200/csrc/" + f for f in (
     "kvq_decode_mma.cu", "kvq_async.cuh", "kvq_internal.h", "kvq_lm_common.cuh", "kvq_tiles.cuh", "kvq_window.cuh",
