@@ -25,6 +25,13 @@ static int slots_smem(int units) {
   const int n = 233472 / per;
   return n < 1 ? 1 : (n > 4 ? 4 : n);
 }
+// shaped like the 1-bit instance's: registers allow 7 CTAs per SM, shared memory (the chunk's
+// logits) fewer for long chunks
+static int slots_onebit(int units) {
+  const int per = 5120 + 16 * (units * 64 + 8) + 2048 + 1152;
+  const int n = 233472 / per;
+  return n < 1 ? 1 : (n > 7 ? 7 : n);
+}
 
 template <class F>
 int check(const F& slots, const char* name) {
@@ -53,11 +60,15 @@ int check(const F& slots, const char* name) {
 }
 
 int main() {
-  if (check(slots_const1, "1") || check(slots_const4, "4") || check(slots_smem, "smem")) return 1;
+  if (check(slots_const1, "1") || check(slots_const4, "4") || check(slots_smem, "smem") || check(slots_onebit, "onebit"))
+    return 1;
   // the 8B-shaped decode step: 16 x 8 rows, 8192 + 1 tokens, four CTAs per SM, 35-unit chunks
   int splits = 0, chunk = 0;
   plan_splits(128, 148, slots_const4, 35, 16, 8193, &splits, &chunk);
   printf("llama8b %d %d\n", splits, chunk);
+  // the 1-bit layer's shape: 256 x 8 rows, 16384 + 1 tokens; shorter chunks let 7 CTAs share an SM
+  plan_splits(2048, 148, slots_onebit, 35, 16, 16385, &splits, &chunk);
+  printf("onebit %d %d\n", splits, chunk);
   return 0;
 }
 """
@@ -75,4 +86,7 @@ def test_split_plan_invariants(tmp_path):
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=600)
     assert out.returncode == 0, out.stdout + out.stderr
     # 129 units over 4 splits of 33: 512 CTAs, one wave of four per SM
-    assert out.stdout.split()[-3:] == ["llama8b", "4", "2112"], out.stdout
+    assert out.stdout.split()[-6:-3] == ["llama8b", "4", "2112"], out.stdout
+    # 257 units over 11 splits of 24 (1536 tokens), 7 CTAs per SM, rather than 8 splits of the
+    # largest chunk (5 per SM)
+    assert out.stdout.split()[-3:] == ["onebit", "11", "1536"], out.stdout
