@@ -138,19 +138,60 @@ decode_mla_simple(const __grid_constant__ MlaParams p) {
   }
 }
 
-__global__ void __launch_bounds__(kLat) reduce_mla(const __grid_constant__ MlaParams p) {
-  const int row = blockIdx.x, c = threadIdx.x;
+// Merge of a row's split partials (log-sum-exp): block (row, quarter) takes latent channels
+// 128 quarter .. + 127. The splits' maximum and their weights 2^(m_s - M) are formed once per block
+// (threads over splits, a fixed reduction order) and staged in shared memory, kRedChunk splits at a
+// time; thread (group g, channel) then sums its channel over the splits s = g mod 4 (reading them
+// coalesced, several loads in flight) and the four groups' sums are added in a fixed order.
+constexpr int kRedChannels = 128, kRedGroups = 4, kRedThreads = kRedChannels * kRedGroups, kRedChunk = 512;
+
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float x = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, x) : v + x;
+  }
+  __syncthreads();  // sh may still be read from the previous reduction
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  float r = sh[0];
+#pragma unroll
+  for (int w = 1; w < kRedThreads / 32; ++w) r = is_max ? fmaxf(r, sh[w]) : r + sh[w];
+  return r;
+}
+
+__global__ void __launch_bounds__(kRedThreads) reduce_mla(const __grid_constant__ MlaParams p) {
+  __shared__ float s_w[kRedChunk];
+  __shared__ float s_red[kRedThreads / 32];
+  __shared__ float s_o[kRedGroups][kRedChannels];
+  const int row = blockIdx.x / (kLat / kRedChannels), tid = threadIdx.x;
+  const int grp = tid / kRedChannels, c = (blockIdx.x % (kLat / kRedChannels)) * kRedChannels + tid % kRedChannels;
   const int stride = 2 + kLat;
   const float* part = p.part + (size_t)row * p.splits * stride;
-  float M = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) M = fmaxf(M, part[(size_t)s * stride]);
-  float L = 0.f, o = 0.f;
-  for (int s = 0; s < p.splits; ++s) {
-    const float* ps = part + (size_t)s * stride;
-    const float w = exp2_diff(ps[0], M);
-    L += w * ps[1];
-    o += w * ps[2 + c];
+  float m = -INFINITY;
+  for (int sp = tid; sp < p.splits; sp += kRedThreads) m = fmaxf(m, part[(size_t)sp * stride]);
+  const float M = block_reduce(m, true, s_red);
+  float l = 0.f, o = 0.f;
+  for (int s0 = 0; s0 < p.splits; s0 += kRedChunk) {
+    const int n = min(kRedChunk, p.splits - s0);
+    __syncthreads();  // the previous chunk's weights have been used
+    for (int i = tid; i < n; i += kRedThreads) {
+      const float* ps = part + (size_t)(s0 + i) * stride;
+      const float w = exp2_diff(ps[0], M);
+      s_w[i] = w;
+      l += w * ps[1];
+    }
+    __syncthreads();
+    const float* pc = part + (size_t)s0 * stride + 2 + c;
+#pragma unroll 8
+    for (int i = grp; i < n; i += kRedGroups) o = fmaf(s_w[i], pc[(size_t)i * stride], o);
   }
+  const float L = block_reduce(l, false, s_red);
+  s_o[grp][tid % kRedChannels] = o;
+  __syncthreads();
+  if (grp != 0) return;
+  o = (s_o[0][tid] + s_o[1][tid]) + (s_o[2][tid] + s_o[3][tid]);
   if (p.pout) {  // merged softmax state: running maximum (log2 units), sum of weights, unnormalised o
     float* st = p.pout + (size_t)row * stride;
     st[2 + c] = o;
@@ -192,7 +233,7 @@ cudaError_t launch_decode_mla(const MlaParams& p, cudaStream_t s) {
 }
 
 cudaError_t launch_reduce_mla(const MlaParams& p, cudaStream_t s) {
-  reduce_mla<<<p.B * p.Hq, kLat, 0, s>>>(p);
+  reduce_mla<<<p.B * p.Hq * (kLat / kRedChannels), kRedThreads, 0, s>>>(p);
   return launched();
 }
 
