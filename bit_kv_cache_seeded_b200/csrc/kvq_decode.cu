@@ -250,8 +250,8 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
 }
 
 // One block per (sequence, kv-head), 128 threads per query head of the group. Merge: thread
-// (h, i) merges head h's split partials at coordinate i (the loads of 4 splits issued together,
-// one memory latency per 4 splits). Value sketch fold-back, o_r += S^T acc_z, with S staged in
+// (h, i) merges head h's split partials at coordinate i (the loads of 8 splits issued together,
+// one memory latency per 8 splits). Value sketch fold-back, o_r += S^T acc_z, with S staged in
 // shared memory by cp.async while the partials are merged: thread (q, i) sums the rows j of
 // quarter q (of G) for all G heads at once, so each staged S element is read once; the G partial
 // sums of a head meet in shared memory. Warp h then undoes the rotation of head h
@@ -259,7 +259,7 @@ decode_lm_simple(const __grid_constant__ DecodeParams p) {
 template <int G>
 __global__ void __launch_bounds__(G * kHeadDim)
 reduce_lm(const __grid_constant__ DecodeParams p, int vq) {
-  constexpr int kSplitBatch = 4;
+  constexpr int kSplitBatch = 8;
   constexpr int kRows = kHeadDim / G;                 // sketch rows per thread in the fold-back
   extern __shared__ __align__(16) float rs[];
   float* S_s = rs;                                   // [m][d] when vq
