@@ -242,6 +242,13 @@ def test_fp4_small_ragged():
     fp4_check(0, batch=3, lens=[1000, 0, 33])
 
 
+def test_fp4_few_tiles_per_cta():
+    """A context whose split plan gives every CTA a few 64-token tiles, the last one ragged: the
+    tcgen05 kernel's first, middle and last iterations (S of the next tile issued after O^T of
+    the current one) on every CTA."""
+    fp4_check(0, batch=1, lens=[3 * 147 * 64 + 33])
+
+
 def test_fp4_sixteen_heads_ragged():
     """16 query heads decode on the mma.sync kernel (the tcgen05 kernel is for 64 heads)."""
     fp4_check(0, batch=2, lens=[700, 65], n_q_heads=16)
